@@ -1,0 +1,194 @@
+"""Float64 CPU oracle for the selective state-space scan.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py``'s CPU-baseline / reference leg may import this package.  The
+product path (``selective_state_space_28_b200``) never imports it, and the two
+share no code: the oracle is plain C (``ssm_oracle.c``) in float64, written as
+the pages' token loop, loaded here with ctypes.
+
+Every function takes numpy arrays (any float dtype; they are widened to
+float64) and returns float64 numpy arrays.  Sources, per function, are in
+``ssm_oracle.h`` / ``ssm_oracle.c``:
+
+* ``m1_scan``    -- "Mamba" (nnterp guide): the per-channel recurrence, the
+  values table; "Falcon-Mamba": the weightless norms on B, C and the step.
+* ``m2_scan``    -- "Mamba-2" (nnterp encyclopedia): one scalar decay per head
+  and token, an N x P state per head, key side first.
+* ``m1_step`` / ``m2_step`` -- the decode step: update the state, then read.
+* ``m1_quadratic`` / ``m2_quadratic`` -- "Mamba-2", "The hidden attention":
+  the O(L^2) masked form, evaluated by brute force.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+SOFTPLUS = 1
+RMS_BC = 2
+RMS_DT = 4
+
+_lib = None
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.c_int64
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        for name, argtypes in {
+            "orc_m1_scan": [_I64] * 5 + [ctypes.c_uint32, ctypes.c_double] + [_D] * 12 + [ctypes.c_int],
+            "orc_m2_scan": [_I64] * 6 + [ctypes.c_uint32] + [_D] * 12 + [ctypes.c_int],
+            "orc_m1_step": [_I64] * 4 + [ctypes.c_uint32, ctypes.c_double] + [_D] * 10,
+            "orc_m2_step": [_I64] * 5 + [ctypes.c_uint32] + [_D] * 10,
+            "orc_m2_quadratic": [_I64] * 6 + [_D] * 9,
+            "orc_m1_quadratic": [_I64] * 5 + [_D] * 9,
+        }.items():
+            fn = getattr(lib, name)
+            fn.argtypes = argtypes
+            fn.restype = ctypes.c_int
+        lib.orc_softplus.argtypes = [ctypes.c_double]
+        lib.orc_softplus.restype = ctypes.c_double
+        lib.orc_silu.argtypes = [ctypes.c_double]
+        lib.orc_silu.restype = ctypes.c_double
+        lib.orc_rms_rows.argtypes = [_I64, _I64, ctypes.c_double, _D, _D]
+        lib.orc_rms_rows.restype = None
+        _lib = lib
+    return _lib
+
+
+def _f64(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # a torch tensor: widen on the host
+        a = a.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _p(a):
+    return a.ctypes.data_as(_D) if a is not None else None
+
+
+def default_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def m1_scan(x, dt, B, C, A, D=None, z=None, dt_bias=None, h0=None, *,
+            flags=SOFTPLUS, rms_eps=1e-6, want_states=False, nthreads=None):
+    """Mamba-1 scan.  x, dt, z: [b, L, C]; B, C: [b, L, G, N]; A: [C, N].
+
+    Returns (y [b,L,C], h_last [b,C,N], states [b,L,C,N] or None)."""
+    x, dt, z, B, C, A, D, dt_bias, h0 = map(_f64, (x, dt, z, B, C, A, D, dt_bias, h0))
+    b, L, Cn = x.shape
+    G, N = B.shape[2], B.shape[3]
+    y = np.empty_like(x)
+    h_last = np.empty((b, Cn, N))
+    states = np.empty((b, L, Cn, N)) if want_states else None
+    rc = _load().orc_m1_scan(b, L, Cn, N, G, flags, rms_eps, _p(x), _p(dt), _p(z),
+                             _p(B), _p(C), _p(A), _p(D), _p(dt_bias), _p(h0),
+                             _p(y), _p(h_last), _p(states),
+                             nthreads or default_threads())
+    if rc:
+        raise ValueError("orc_m1_scan failed: %d" % rc)
+    return y, h_last, states
+
+
+def m2_scan(x, dt, B, C, A, D=None, z=None, dt_bias=None, h0=None, *,
+            flags=SOFTPLUS, want_states=False, nthreads=None):
+    """Mamba-2 scan.  x, z: [b, L, H, P]; dt: [b, L, H]; B, C: [b, L, G, N].
+
+    Returns (y [b,L,H,P], h_last [b,H,N,P], states [b,L,H,N,P] or None)."""
+    x, dt, z, B, C, A, D, dt_bias, h0 = map(_f64, (x, dt, z, B, C, A, D, dt_bias, h0))
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    y = np.empty_like(x)
+    h_last = np.empty((b, H, N, P))
+    states = np.empty((b, L, H, N, P)) if want_states else None
+    rc = _load().orc_m2_scan(b, L, H, P, N, G, flags, _p(x), _p(dt), _p(z), _p(B),
+                             _p(C), _p(A), _p(D), _p(dt_bias), _p(h0), _p(y),
+                             _p(h_last), _p(states), nthreads or default_threads())
+    if rc:
+        raise ValueError("orc_m2_scan failed: %d" % rc)
+    return y, h_last, states
+
+
+def m1_step(state, x, dt, B, C, A, D=None, z=None, dt_bias=None, *,
+            flags=SOFTPLUS, rms_eps=1e-6):
+    """One Mamba-1 decode token.  state: [b, C, N]; x, dt, z: [b, C];
+    B, C: [b, G, N].  Returns (new_state, y)."""
+    st = _f64(state).copy()
+    x, dt, z, B, C, A, D, dt_bias = map(_f64, (x, dt, z, B, C, A, D, dt_bias))
+    b, Cn = x.shape
+    G, N = B.shape[1], B.shape[2]
+    y = np.empty_like(x)
+    rc = _load().orc_m1_step(b, Cn, N, G, flags, rms_eps, _p(x), _p(dt), _p(z), _p(B),
+                             _p(C), _p(A), _p(D), _p(dt_bias), _p(st), _p(y))
+    if rc:
+        raise ValueError("orc_m1_step failed: %d" % rc)
+    return st, y
+
+
+def m2_step(state, x, dt, B, C, A, D=None, z=None, dt_bias=None, *, flags=SOFTPLUS):
+    """One Mamba-2 decode token.  state: [b, H, N, P]; x, z: [b, H, P];
+    dt: [b, H]; B, C: [b, G, N].  Returns (new_state, y)."""
+    st = _f64(state).copy()
+    x, dt, z, B, C, A, D, dt_bias = map(_f64, (x, dt, z, B, C, A, D, dt_bias))
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    y = np.empty_like(x)
+    rc = _load().orc_m2_step(b, H, P, N, G, flags, _p(x), _p(dt), _p(z), _p(B),
+                             _p(C), _p(A), _p(D), _p(dt_bias), _p(st), _p(y))
+    if rc:
+        raise ValueError("orc_m2_step failed: %d" % rc)
+    return st, y
+
+
+def m2_quadratic(x, betas, B, C, A, D=None, z=None, h0=None):
+    """Brute-force hidden-attention form (Mamba-2 layout); betas = the step
+    after bias and softplus, [b, L, H]."""
+    x, betas, z, B, C, A, D, h0 = map(_f64, (x, betas, z, B, C, A, D, h0))
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    y = np.empty_like(x)
+    rc = _load().orc_m2_quadratic(b, L, H, P, N, G, _p(x), _p(betas), _p(z), _p(B),
+                                  _p(C), _p(A), _p(D), _p(h0), _p(y))
+    if rc:
+        raise ValueError("orc_m2_quadratic failed: %d" % rc)
+    return y
+
+
+def m1_quadratic(x, betas, B, C, A, D=None, z=None, h0=None):
+    """Brute-force hidden-attention form (Mamba-1 layout); betas: [b, L, C]."""
+    x, betas, z, B, C, A, D, h0 = map(_f64, (x, betas, z, B, C, A, D, h0))
+    b, L, Cn = x.shape
+    G, N = B.shape[2], B.shape[3]
+    y = np.empty_like(x)
+    rc = _load().orc_m1_quadratic(b, L, Cn, N, G, _p(x), _p(betas), _p(z), _p(B),
+                                  _p(C), _p(A), _p(D), _p(h0), _p(y))
+    if rc:
+        raise ValueError("orc_m1_quadratic failed: %d" % rc)
+    return y
+
+
+def softplus(v):
+    lib = _load()
+    return np.vectorize(lib.orc_softplus, otypes=[np.float64])(np.asarray(v, np.float64))
+
+
+def silu(v):
+    lib = _load()
+    return np.vectorize(lib.orc_silu, otypes=[np.float64])(np.asarray(v, np.float64))
+
+
+def rms_rows(v, eps):
+    v = _f64(v)
+    out = np.empty_like(v)
+    n = v.shape[-1]
+    _load().orc_rms_rows(v.size // n, n, eps, _p(v), _p(out))
+    return out

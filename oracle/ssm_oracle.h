@@ -1,0 +1,102 @@
+/*
+ * ssm_oracle.h -- float64 CPU oracle for the selective state-space scan.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this code: only the tests, the smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code, header, table or constant with
+ * the CUDA library.
+ *
+ * Every array is a dense, row-major float64 array.  Optional inputs may be
+ * NULL (D, dt_bias, h0 -> zeros; z -> no gate); optional outputs may be NULL.
+ *
+ * Sources (page title, section):
+ *   - "Mamba" (nnterp guide, architectures/mamba): intro paragraph (the
+ *     per-channel recurrence), "The values" table (layouts, betas =
+ *     softplus(dt + dt_bias), y = C.h + D*x before the gate), "The state"
+ *     (state after every token, decode step updates first then reads).
+ *   - "Mamba" (tokentrails lineage), "Code" and steps 3-4.
+ *   - "Mamba-2" (nnterp encyclopedia), "The mixer's values", "The hidden
+ *     attention", "The state", "A zero step skips a token exactly".
+ *   - "Falcon-Mamba" (nnterp encyclopedia), "Where the norms sit".
+ */
+#ifndef SSM_ORACLE_H
+#define SSM_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ORC_SOFTPLUS 1u  /* dt <- softplus(dt + dt_bias)                     */
+#define ORC_RMS_BC   2u  /* B, C <- weightless RMS norm over the state axis   */
+#define ORC_RMS_DT   4u  /* dt_raw <- weightless RMS norm over the channels   */
+
+/* Mamba-1 selective scan.  x, dt, z, y: [b, L, C]; B, Cm: [b, L, G, N];
+ * A: [C, N]; D, dt_bias: [C]; h0, h_last: [b, C, N]; states: [b, L, C, N].
+ * Channel c reads group c / (C / G).  Work is split over nthreads threads. */
+int orc_m1_scan(int64_t batch, int64_t seqlen, int64_t channels, int64_t state,
+                int64_t groups, uint32_t flags, double rms_eps,
+                const double *x, const double *dt, const double *z,
+                const double *B, const double *Cm, const double *A,
+                const double *D, const double *dt_bias, const double *h0,
+                double *y, double *h_last, double *states, int nthreads);
+
+/* Mamba-2 (SSD) scan, written as the token recurrence.  x, z, y: [b, L, H, P];
+ * dt: [b, L, H]; B, Cm: [b, L, G, N]; A, D, dt_bias: [H];
+ * h0, h_last: [b, H, N, P] (key side first); states: [b, L, H, N, P].
+ * Head h reads group h / (H / G).  Only ORC_SOFTPLUS is meaningful. */
+int orc_m2_scan(int64_t batch, int64_t seqlen, int64_t heads, int64_t head_dim,
+                int64_t state, int64_t groups, uint32_t flags,
+                const double *x, const double *dt, const double *z,
+                const double *B, const double *Cm, const double *A,
+                const double *D, const double *dt_bias, const double *h0,
+                double *y, double *h_last, double *states, int nthreads);
+
+/* One decode token, Mamba-1: state [b, C, N] is updated in place, then read.
+ * x, dt, z, y: [b, C]; B, Cm: [b, G, N]. */
+int orc_m1_step(int64_t batch, int64_t channels, int64_t state, int64_t groups,
+                uint32_t flags, double rms_eps,
+                const double *x, const double *dt, const double *z,
+                const double *B, const double *Cm, const double *A,
+                const double *D, const double *dt_bias,
+                double *state_io, double *y);
+
+/* One decode token, Mamba-2: state [b, H, N, P] updated in place, then read.
+ * x, z, y: [b, H, P]; dt: [b, H]; B, Cm: [b, G, N]. */
+int orc_m2_step(int64_t batch, int64_t heads, int64_t head_dim, int64_t state,
+                int64_t groups, uint32_t flags,
+                const double *x, const double *dt, const double *z,
+                const double *B, const double *Cm, const double *A,
+                const double *D, const double *dt_bias,
+                double *state_io, double *y);
+
+/* Brute-force quadratic ("hidden attention") form, Mamba-2 layout, O(L^3):
+ *   y_t = sum_{s<=t} (C_t . B_s) * exp(sum_{r=s+1..t} dt_r A) * dt_s * x_s
+ *         + C_t . (exp(sum_{r<=t} dt_r A) h0) + D x_t,   then the gate.
+ * dt here is the step AFTER bias and softplus (the pages' "betas"). */
+int orc_m2_quadratic(int64_t batch, int64_t seqlen, int64_t heads,
+                     int64_t head_dim, int64_t state, int64_t groups,
+                     const double *x, const double *betas, const double *z,
+                     const double *B, const double *Cm, const double *A,
+                     const double *D, const double *h0, double *y);
+
+/* The same quadratic form for Mamba-1 (per channel c and state n, A[c, n]).
+ * betas: [b, L, C], the step after bias/softplus; B, Cm already normed. */
+int orc_m1_quadratic(int64_t batch, int64_t seqlen, int64_t channels,
+                     int64_t state, int64_t groups,
+                     const double *x, const double *betas, const double *z,
+                     const double *B, const double *Cm, const double *A,
+                     const double *D, const double *h0, double *y);
+
+/* Elementwise helpers exposed for the pins. */
+double orc_softplus(double v);
+double orc_silu(double v);
+/* Weightless RMS norm of rows of length n: out = v / sqrt(mean(v^2) + eps). */
+void orc_rms_rows(int64_t rows, int64_t n, double eps, const double *in,
+                  double *out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

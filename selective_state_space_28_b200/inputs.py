@@ -1,0 +1,192 @@
+"""Seeded synthetic inputs for the scan workloads.
+
+This module only draws numbers; it holds none of the scan's arithmetic.  The
+same draws feed the CUDA library and the float64 oracle, so both read
+identical values: every tensor is rounded to its I/O dtype here, on the host,
+before anyone reads it.
+
+Recipe (the pages print no dataset; these follow the shapes of the models
+the pages describe):
+
+* ``A = -exp(A_log)`` with ``A_log[c, n] = log(n + 1)`` for Mamba-1 (the
+  S4D-real initialisation, "Mamba" tokentrails "Code": ``A = -exp(A_log)``),
+  and ``A_h = -exp(U[log 1, log 16])`` per head for Mamba-2.
+* ``dt_bias = softplus^-1(dt0)``, ``dt0 = exp(U[log 1e-3, log 0.1])`` per
+  channel / head (1e-3 is the configs' ``time_step_min``).
+* ``D = 1``; ``x, z, dt_raw, B, C ~ N(0, 1)``; decode states ``~ N(0, 0.1^2)``.
+* Draw order: A, dt_bias, D, x, z, dt_raw, B, C, then the state.
+"""
+import math
+from dataclasses import dataclass, field
+from typing import Optional
+
+import torch
+
+SOFTPLUS = 1
+RMS_BC = 2
+RMS_DT = 4
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One named scan workload.  ``kind`` is "m1", "ssd" or "decode"."""
+    name: str
+    kind: str
+    batch: int
+    seqlen: int = 1
+    channels: int = 0          # Mamba-1 inner width
+    heads: int = 0             # Mamba-2 heads
+    head_dim: int = 0
+    state: int = 16
+    groups: int = 1
+    chunk: int = 256
+    io: str = "bf16"
+    gate: bool = True
+    flags: int = SOFTPLUS
+    rms_eps: float = 1e-6
+    want_states: bool = False
+    layers: int = 1            # decode stacks: one call per layer
+    m1_layers: int = 0         # decode stacks: Mamba-1 layers after the Mamba-2 ones
+    m1_channels: int = 0
+    m1_state: int = 16
+    seed: int = 0
+    extra: dict = field(default_factory=dict)
+
+
+WORKLOADS = {
+    # Mamba-1 toy scan, float32 I/O, with the per-token states.
+    "m1_toy_b1_l64_c32_n4_f32": Workload(
+        "m1_toy_b1_l64_c32_n4_f32", "m1", batch=1, seqlen=64, channels=32,
+        state=4, io="f32", gate=True, want_states=True, seed=0),
+    # One Mamba-130m-shaped mixer scan (inner width 1536, state 16).
+    "m1_130m_b8_l2048_c1536_n16_bf16": Workload(
+        "m1_130m_b8_l2048_c1536_n16_bf16", "m1", batch=8, seqlen=2048,
+        channels=1536, state=16, io="bf16", gate=True, seed=1),
+    # Falcon-Mamba-7B width (8192) with the weightless norms, long sequence.
+    "m1_falcon_rms_b4_l8192_c8192_n16_bf16": Workload(
+        "m1_falcon_rms_b4_l8192_c8192_n16_bf16", "m1", batch=4, seqlen=8192,
+        channels=8192, state=16, io="bf16", gate=True,
+        flags=SOFTPLUS | RMS_BC | RMS_DT, seed=2),
+    # Mamba-2 2.7B-shaped SSD chunk scan (80 heads x 64, state 128, chunk 256).
+    "ssd_2p7b_b4_l4096_h80_p64_n128_bf16": Workload(
+        "ssd_2p7b_b4_l4096_h80_p64_n128_bf16", "ssd", batch=4, seqlen=4096,
+        heads=80, head_dim=64, state=128, chunk=256, io="bf16", gate=False,
+        seed=3),
+    # Decode across a Mamba-2 2.7B stack (64 layers) plus a Mamba-130m stack
+    # (24 layers of 1536 x 16), batch 256, one token per layer.
+    "decode_2p7b_stack_b256": Workload(
+        "decode_2p7b_stack_b256", "decode", batch=256, heads=80, head_dim=64,
+        state=128, io="bf16", gate=False, layers=64, m1_layers=24,
+        m1_channels=1536, m1_state=16, seed=4),
+}
+
+
+def _dtype(io):
+    return {"bf16": torch.bfloat16, "f32": torch.float32}[io]
+
+
+def _gen(seed, device):
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _randn(shape, g, dtype, device, std=1.0):
+    t = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
+    if std != 1.0:
+        t.mul_(std)
+    return t.to(dtype)
+
+
+def _dt_bias(n, g, device):
+    # dt0 = exp(U[log 1e-3, log 1e-1]); bias = dt0 + log(-expm1(-dt0)) is the
+    # inverse of softplus at dt0.
+    u = torch.rand(n, generator=g, dtype=torch.float64, device=device)
+    dt0 = torch.exp(u * (math.log(0.1) - math.log(1e-3)) + math.log(1e-3))
+    return (dt0 + torch.log(-torch.expm1(-dt0))).to(torch.float32)
+
+
+def m1_inputs(batch, seqlen, channels, state, groups=1, io="bf16", gate=True,
+              seed=0, h0=False, device="cpu"):
+    """Inputs of one Mamba-1 scan: dict of tensors on ``device``."""
+    g = _gen(seed, device)
+    dt_ = _dtype(io)
+    A_log = torch.log(torch.arange(1, state + 1, dtype=torch.float32, device=device))
+    A = (-torch.exp(A_log)).unsqueeze(0).expand(channels, state).contiguous()
+    out = {"A": A, "dt_bias": _dt_bias(channels, g, device),
+           "D": torch.ones(channels, dtype=torch.float32, device=device)}
+    out["x"] = _randn((batch, seqlen, channels), g, dt_, device)
+    out["z"] = _randn((batch, seqlen, channels), g, dt_, device) if gate else None
+    out["dt"] = _randn((batch, seqlen, channels), g, dt_, device)
+    out["B"] = _randn((batch, seqlen, groups, state), g, dt_, device)
+    out["C"] = _randn((batch, seqlen, groups, state), g, dt_, device)
+    out["h0"] = (_randn((batch, channels, state), g, torch.float32, device, 0.1)
+                 if h0 else None)
+    return out
+
+
+def ssd_inputs(batch, seqlen, heads, head_dim, state, groups=1, io="bf16",
+               gate=False, seed=0, h0=False, device="cpu"):
+    """Inputs of one Mamba-2 SSD scan: dict of tensors on ``device``."""
+    g = _gen(seed, device)
+    dt_ = _dtype(io)
+    u = torch.rand(heads, generator=g, dtype=torch.float64, device=device)
+    A = (-torch.exp(u * math.log(16.0))).to(torch.float32)
+    out = {"A": A, "dt_bias": _dt_bias(heads, g, device),
+           "D": torch.ones(heads, dtype=torch.float32, device=device)}
+    out["x"] = _randn((batch, seqlen, heads, head_dim), g, dt_, device)
+    out["z"] = _randn((batch, seqlen, heads, head_dim), g, dt_, device) if gate else None
+    out["dt"] = _randn((batch, seqlen, heads), g, dt_, device)
+    out["B"] = _randn((batch, seqlen, groups, state), g, dt_, device)
+    out["C"] = _randn((batch, seqlen, groups, state), g, dt_, device)
+    out["h0"] = (_randn((batch, heads, state, head_dim), g, torch.float32, device, 0.1)
+                 if h0 else None)
+    return out
+
+
+def m2_step_inputs(batch, heads, head_dim, state, groups=1, io="bf16", gate=False,
+                   seed=0, device="cpu"):
+    """One Mamba-2 decode token plus its cached state ~ N(0, 0.1^2)."""
+    g = _gen(seed, device)
+    dt_ = _dtype(io)
+    u = torch.rand(heads, generator=g, dtype=torch.float64, device=device)
+    A = (-torch.exp(u * math.log(16.0))).to(torch.float32)
+    out = {"A": A, "dt_bias": _dt_bias(heads, g, device),
+           "D": torch.ones(heads, dtype=torch.float32, device=device)}
+    out["x"] = _randn((batch, heads, head_dim), g, dt_, device)
+    out["z"] = _randn((batch, heads, head_dim), g, dt_, device) if gate else None
+    out["dt"] = _randn((batch, heads), g, dt_, device)
+    out["B"] = _randn((batch, groups, state), g, dt_, device)
+    out["C"] = _randn((batch, groups, state), g, dt_, device)
+    out["state"] = _randn((batch, heads, state, head_dim), g, torch.float32, device, 0.1)
+    return out
+
+
+def m1_step_inputs(batch, channels, state, groups=1, io="bf16", gate=True, seed=0,
+                   device="cpu"):
+    """One Mamba-1 decode token plus its cached state ~ N(0, 0.1^2)."""
+    g = _gen(seed, device)
+    dt_ = _dtype(io)
+    A_log = torch.log(torch.arange(1, state + 1, dtype=torch.float32, device=device))
+    A = (-torch.exp(A_log)).unsqueeze(0).expand(channels, state).contiguous()
+    out = {"A": A, "dt_bias": _dt_bias(channels, g, device),
+           "D": torch.ones(channels, dtype=torch.float32, device=device)}
+    out["x"] = _randn((batch, channels), g, dt_, device)
+    out["z"] = _randn((batch, channels), g, dt_, device) if gate else None
+    out["dt"] = _randn((batch, channels), g, dt_, device)
+    out["B"] = _randn((batch, groups, state), g, dt_, device)
+    out["C"] = _randn((batch, groups, state), g, dt_, device)
+    out["state"] = _randn((batch, channels, state), g, torch.float32, device, 0.1)
+    return out
+
+
+def workload_inputs(w: Workload, device="cpu", seed: Optional[int] = None):
+    """Inputs of a scan workload (Mamba-1 or SSD)."""
+    s = w.seed if seed is None else seed
+    if w.kind == "m1":
+        return m1_inputs(w.batch, w.seqlen, w.channels, w.state, w.groups, w.io,
+                         w.gate, s, device=device)
+    if w.kind == "ssd":
+        return ssd_inputs(w.batch, w.seqlen, w.heads, w.head_dim, w.state, w.groups,
+                          w.io, w.gate, s, device=device)
+    raise ValueError("no scan inputs for kind %r" % w.kind)

@@ -1,0 +1,364 @@
+"""Pins of the float64 oracle to facts that do not come from the oracle itself.
+
+Each test fixes one part of the oracle against a closed form, a library
+routine, a brute-force sum, an invariant the pages state, or a number the
+pages print.  tests/test_oracle_mutants.py checks that plausible mistakes in
+the oracle's source fail at least one of these pins.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng
+
+
+def _m1_rand(b, L, C, N, G=1, seed=0, h0=True, z=True):
+    r = rng(seed)
+    d = dict(x=r.standard_normal((b, L, C)), dt=r.standard_normal((b, L, C)),
+             B=r.standard_normal((b, L, G, N)), C=r.standard_normal((b, L, G, N)),
+             A=-np.exp(r.uniform(-1, 1.5, (C, N))), D=r.standard_normal(C),
+             dt_bias=r.uniform(-4, -1, C))
+    d["z"] = r.standard_normal((b, L, C)) if z else None
+    d["h0"] = r.standard_normal((b, C, N)) if h0 else None
+    return d
+
+
+def _m2_rand(b, L, H, P, N, G=1, seed=0, h0=True, z=True):
+    r = rng(seed)
+    d = dict(x=r.standard_normal((b, L, H, P)), dt=r.standard_normal((b, L, H)),
+             B=r.standard_normal((b, L, G, N)), C=r.standard_normal((b, L, G, N)),
+             A=-np.exp(r.uniform(0, 2.7, H)), D=r.standard_normal(H),
+             dt_bias=r.uniform(-4, -1, H))
+    d["z"] = r.standard_normal((b, L, H, P)) if z else None
+    d["h0"] = r.standard_normal((b, H, N, P)) if h0 else None
+    return d
+
+
+# ------------------------------------------------------- elementwise pieces
+
+def test_softplus_matches_library():
+    v = np.concatenate([np.linspace(-60, 60, 2401), [-1e300, 0.0, 1e-12, -1e-12, 700.0]])
+    got = oracle.softplus(v)
+    ref = np.logaddexp(0.0, v)                      # numpy: log(exp(0) + exp(v))
+    np.testing.assert_allclose(got, ref, rtol=1e-15, atol=0)
+    ref_t = F.softplus(torch.tensor(v), beta=1.0, threshold=1e9).numpy()
+    np.testing.assert_allclose(got[:-1], ref_t[:-1], rtol=1e-14, atol=1e-300)
+    assert oracle.softplus(np.array([-np.inf]))[0] == 0.0   # a zero step stays zero
+
+
+def test_silu_matches_library():
+    v = np.linspace(-40, 40, 1601)
+    np.testing.assert_allclose(oracle.silu(v), F.silu(torch.tensor(v)).numpy(),
+                               rtol=1e-14, atol=1e-300)
+
+
+def test_rms_matches_library():
+    v = rng(1).standard_normal((37, 16)) * 3.0
+    for eps in (1e-6, 1e-5, 0.5):
+        ref = F.rms_norm(torch.tensor(v), (16,), eps=eps).numpy()
+        np.testing.assert_allclose(oracle.rms_rows(v, eps), ref, rtol=1e-13, atol=1e-15)
+
+
+# --------------------------------------------------------------- closed forms
+
+def test_m1_zero_decay_is_cumulative_sum():
+    """A = 0: nothing decays, so h_t = sum_{s<=t} dt_s B_s x_s (a running sum)."""
+    d = _m1_rand(2, 23, 5, 3, seed=2, h0=False, z=False)
+    d["A"] = np.zeros_like(d["A"])
+    y, h_last, states = oracle.m1_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"],
+                                       flags=0, want_states=True)
+    w = d["dt"][..., None] * d["x"][..., None] * d["B"][:, :, 0, None, :]  # [b,L,C,N]
+    h = np.cumsum(w, axis=1)
+    np.testing.assert_allclose(states, h, rtol=1e-12, atol=1e-12)
+    y_ref = np.einsum("bln,blcn->blc", d["C"][:, :, 0, :], h) + d["D"] * d["x"]
+    np.testing.assert_allclose(y, y_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(h_last, h[:, -1], rtol=1e-12, atol=1e-12)
+
+
+def test_m1_zero_step_is_skip_connection():
+    """dt = 0: no write and no decay ("Mamba-2", a zero step skips a token
+    exactly); y reduces to the gated skip D*x*silu(z) and the state is h0."""
+    d = _m1_rand(2, 17, 6, 4, seed=3)
+    zero = np.zeros_like(d["dt"])
+    y, h_last, states = oracle.m1_scan(d["x"], zero, d["B"], d["C"], d["A"], d["D"],
+                                       z=d["z"], h0=d["h0"], flags=0, want_states=True)
+    assert np.array_equal(h_last, d["h0"])
+    assert np.array_equal(states, np.broadcast_to(d["h0"][:, None], states.shape))
+    ch0 = np.einsum("bln,bcn->blc", d["C"][:, :, 0, :], d["h0"])
+    sig = 1.0 / (1.0 + np.exp(-d["z"]))
+    np.testing.assert_allclose(y, (ch0 + d["D"] * d["x"]) * d["z"] * sig, rtol=1e-13, atol=1e-13)
+
+
+def test_m1_single_state_geometric_series():
+    """N = 1 with constant inputs: h_t = a^t h0 + beta (1 - a^t) / (1 - a)."""
+    L, a_log, dt, Bv, Cv, xv, h0 = 40, -0.7, 0.3, 1.7, -0.4, 0.9, 2.5
+    ones = np.ones((1, L, 1))
+    y, h_last, states = oracle.m1_scan(xv * ones, dt * ones, Bv * ones[..., None],
+                                       Cv * ones[..., None], np.array([[a_log]]),
+                                       np.zeros(1), h0=np.array([[[h0]]]), flags=0,
+                                       want_states=True)
+    a, beta = math.exp(dt * a_log), dt * Bv * xv
+    t = np.arange(1, L + 1)
+    h = a ** t * h0 + beta * (1 - a ** t) / (1 - a)
+    np.testing.assert_allclose(states[0, :, 0, 0], h, rtol=1e-13)
+    np.testing.assert_allclose(y[0, :, 0], Cv * h, rtol=1e-13)
+
+
+def test_m1_time_invariant_is_a_convolution():
+    """Same step, B and C at every token (the S4 case of "Mamba", tokentrails,
+    step 3): y = K * x with K_k = sum_n C_n exp(dt A_n)^k dt B_n, plus D x."""
+    r = rng(5)
+    L, N = 50, 4
+    x = r.standard_normal((1, L, 1))
+    dt, A = 0.21, -np.exp(r.uniform(-1, 1, (1, N)))
+    Bv, Cv, D = r.standard_normal(N), r.standard_normal(N), 0.37
+    y, _, _ = oracle.m1_scan(x, np.full((1, L, 1), dt), np.tile(Bv, (1, L, 1, 1)),
+                             np.tile(Cv, (1, L, 1, 1)), A, np.array([D]), flags=0)
+    k = np.arange(L)
+    K = (Cv[None, :] * np.exp(dt * A[0])[None, :] ** k[:, None] * dt * Bv[None, :]).sum(1)
+    y_ref = np.convolve(x[0, :, 0], K)[:L] + D * x[0, :, 0]
+    np.testing.assert_allclose(y[0, :, 0], y_ref, rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------- brute force
+
+@pytest.mark.parametrize("G", [1, 2])
+def test_m2_scan_equals_hidden_attention(G):
+    """"Mamba-2", "The hidden attention": the scan equals the causal masked
+    form sum_s (C_t.B_s) exp(decays_{s+1..t}) betas_s x_s + D x_t (brute force)."""
+    d = _m2_rand(2, 19, 4, 3, 5, G=G, seed=6)
+    y, _, _ = oracle.m2_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                             dt_bias=d["dt_bias"], h0=d["h0"])
+    betas = oracle.softplus(d["dt"] + d["dt_bias"])
+    y_q = oracle.m2_quadratic(d["x"], betas, d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                              h0=d["h0"])
+    np.testing.assert_allclose(y, y_q, rtol=1e-11, atol=1e-11)
+
+
+@pytest.mark.parametrize("G", [1, 3])
+def test_m1_scan_equals_hidden_attention(G):
+    d = _m1_rand(2, 14, 6, 4, G=G, seed=7)
+    y, _, _ = oracle.m1_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                             dt_bias=d["dt_bias"], h0=d["h0"])
+    betas = oracle.softplus(d["dt"] + d["dt_bias"])
+    y_q = oracle.m1_quadratic(d["x"], betas, d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                              h0=d["h0"])
+    np.testing.assert_allclose(y, y_q, rtol=1e-11, atol=1e-11)
+
+
+def test_hidden_attention_by_einsum():
+    """The masked form rebuilt with torch einsum on cumulative decays, as the
+    "Mamba-2" page's own check does, agrees with the brute-force sum."""
+    d = _m2_rand(1, 12, 3, 4, 6, G=1, seed=8, h0=False, z=False)
+    betas = oracle.softplus(d["dt"] + d["dt_bias"])[0]            # [L, H]
+    decays = betas * d["A"]
+    cum = torch.tensor(decays).cumsum(0)
+    causal = torch.ones(12, 12, dtype=torch.bool).tril()[..., None]
+    kept = (cum[:, None] - cum[None, :]).masked_fill(~causal, -torch.inf).exp()
+    Cm = torch.tensor(d["C"][0]).repeat_interleave(3, 1)
+    Bm = torch.tensor(d["B"][0]).repeat_interleave(3, 1)
+    alpha = torch.einsum("thn,shn->tsh", Cm, Bm) * kept * torch.tensor(betas)
+    y_e = torch.einsum("tsh,shd->thd", alpha, torch.tensor(d["x"][0])) \
+        + torch.tensor(d["D"])[:, None] * torch.tensor(d["x"][0])
+    y_q = oracle.m2_quadratic(d["x"], betas[None], d["B"], d["C"], d["A"], d["D"])
+    np.testing.assert_allclose(y_q[0], y_e.numpy(), rtol=1e-11, atol=1e-11)
+
+
+# ------------------------------------------------------------------ invariants
+
+def test_split_and_carry_equals_full_scan():
+    """Carrying state_output into the next call's state_input continues the
+    scan exactly ("Mamba-2", "The state"; "Mamba", decode hand-off)."""
+    d = _m1_rand(2, 31, 5, 4, seed=9)
+    full = oracle.m1_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                          dt_bias=d["dt_bias"], h0=d["h0"], want_states=True)
+    for k in (1, 13, 30):
+        sl = lambda a, s: None if a is None else a[:, s]
+        a = oracle.m1_scan(*(sl(d[n], slice(0, k)) for n in ("x", "dt", "B", "C")),
+                           d["A"], d["D"], z=sl(d["z"], slice(0, k)), dt_bias=d["dt_bias"],
+                           h0=d["h0"])
+        b = oracle.m1_scan(*(sl(d[n], slice(k, None)) for n in ("x", "dt", "B", "C")),
+                           d["A"], d["D"], z=sl(d["z"], slice(k, None)),
+                           dt_bias=d["dt_bias"], h0=a[1])
+        assert np.array_equal(np.concatenate([a[0], b[0]], 1), full[0])
+        assert np.array_equal(b[1], full[1])
+    d2 = _m2_rand(1, 20, 2, 3, 4, seed=10)
+    f2 = oracle.m2_scan(d2["x"], d2["dt"], d2["B"], d2["C"], d2["A"], d2["D"], z=d2["z"],
+                        dt_bias=d2["dt_bias"], h0=d2["h0"])
+    a = oracle.m2_scan(d2["x"][:, :7], d2["dt"][:, :7], d2["B"][:, :7], d2["C"][:, :7],
+                       d2["A"], d2["D"], z=d2["z"][:, :7], dt_bias=d2["dt_bias"], h0=d2["h0"])
+    b = oracle.m2_scan(d2["x"][:, 7:], d2["dt"][:, 7:], d2["B"][:, 7:], d2["C"][:, 7:],
+                       d2["A"], d2["D"], z=d2["z"][:, 7:], dt_bias=d2["dt_bias"], h0=a[1])
+    assert np.array_equal(np.concatenate([a[0], b[0]], 1), f2[0])
+    assert np.array_equal(b[1], f2[1])
+
+
+def test_last_state_equals_state_output():
+    """states[:, -1] == state_output, bit for bit ("Mamba-2", "The state")."""
+    d = _m1_rand(2, 9, 3, 4, seed=11)
+    _, h_last, states = oracle.m1_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"],
+                                       dt_bias=d["dt_bias"], h0=d["h0"], want_states=True)
+    assert np.array_equal(states[:, -1], h_last)
+    d2 = _m2_rand(2, 9, 2, 3, 4, seed=12)
+    _, h2, s2 = oracle.m2_scan(d2["x"], d2["dt"], d2["B"], d2["C"], d2["A"], d2["D"],
+                               dt_bias=d2["dt_bias"], h0=d2["h0"], want_states=True)
+    assert np.array_equal(s2[:, -1], h2)
+
+
+def test_zero_step_token_keeps_state_bitwise():
+    """A zero step at token 3 leaves states[:, 3] == states[:, 2] exactly
+    ("Mamba-2", "A zero step skips a token exactly"); dt_raw = -inf gives a
+    softplus step of exactly 0."""
+    d = _m2_rand(1, 8, 3, 4, 5, seed=13)
+    d["dt"][:, 3] = -np.inf
+    _, _, s = oracle.m2_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"],
+                             dt_bias=d["dt_bias"], h0=d["h0"], want_states=True)
+    assert np.array_equal(s[:, 3], s[:, 2])
+    m = _m1_rand(1, 8, 3, 4, seed=14)
+    m["dt"][:, 3] = -np.inf
+    _, _, s1 = oracle.m1_scan(m["x"], m["dt"], m["B"], m["C"], m["A"], m["D"],
+                              dt_bias=m["dt_bias"], h0=m["h0"], want_states=True)
+    assert np.array_equal(s1[:, 3], s1[:, 2])
+
+
+def test_mamba2_is_mamba1_with_shared_decay():
+    """A Mamba-2 head of P channels is P Mamba-1 channels whose A[c, :] are
+    all A_h and whose step is the head's: the two recurrences coincide."""
+    H, P, N = 3, 4, 5
+    d = _m2_rand(2, 11, H, P, N, seed=15)
+    y2, h2, _ = oracle.m2_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                               dt_bias=d["dt_bias"], h0=d["h0"])
+    b, L = 2, 11
+    rep = lambda v: np.repeat(v, P, axis=-1)
+    y1, h1, _ = oracle.m1_scan(d["x"].reshape(b, L, H * P), rep(d["dt"]), d["B"], d["C"],
+                               np.repeat(d["A"], P)[:, None] * np.ones((1, N)),
+                               rep(d["D"]), z=d["z"].reshape(b, L, H * P),
+                               dt_bias=rep(d["dt_bias"]),
+                               h0=d["h0"].transpose(0, 1, 3, 2).reshape(b, H * P, N))
+    np.testing.assert_allclose(y1.reshape(y2.shape), y2, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(h1.reshape(b, H, P, N).transpose(0, 1, 3, 2), h2,
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_step_is_scan_of_one_token():
+    """The decode step equals the scan of one token from the cached state, with
+    y read after the update ("Mamba", "Read order on a decode step")."""
+    d = _m1_rand(3, 1, 7, 4, G=1, seed=16)
+    y, h_last, _ = oracle.m1_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"],
+                                  z=d["z"], dt_bias=d["dt_bias"], h0=d["h0"])
+    st, ys = oracle.m1_step(d["h0"], d["x"][:, 0], d["dt"][:, 0], d["B"][:, 0], d["C"][:, 0],
+                            d["A"], d["D"], z=d["z"][:, 0], dt_bias=d["dt_bias"])
+    assert np.array_equal(st, h_last) and np.array_equal(ys, y[:, 0])
+    e = _m2_rand(2, 1, 3, 4, 5, seed=17)
+    y2, h2, _ = oracle.m2_scan(e["x"], e["dt"], e["B"], e["C"], e["A"], e["D"], z=e["z"],
+                               dt_bias=e["dt_bias"], h0=e["h0"])
+    st2, ys2 = oracle.m2_step(e["h0"], e["x"][:, 0], e["dt"][:, 0], e["B"][:, 0],
+                              e["C"][:, 0], e["A"], e["D"], z=e["z"][:, 0],
+                              dt_bias=e["dt_bias"])
+    assert np.array_equal(st2, h2) and np.array_equal(ys2, y2[:, 0])
+
+
+def test_norm_flags_act_on_the_stated_axes():
+    """"Falcon-Mamba", "Where the norms sit": B and C are RMS-normed over the
+    state axis, the step input over its last axis (the channels), before the
+    bias and softplus.  Pre-norming with torch's rms_norm gives the same scan."""
+    d = _m1_rand(2, 10, 6, 4, seed=18)
+    eps = 1e-6
+    y, h, _ = oracle.m1_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                             dt_bias=d["dt_bias"], h0=d["h0"],
+                             flags=oracle.SOFTPLUS | oracle.RMS_BC | oracle.RMS_DT,
+                             rms_eps=eps)
+    rn = lambda v, n: F.rms_norm(torch.tensor(v), (n,), eps=eps).numpy()
+    y2, h2, _ = oracle.m1_scan(d["x"], rn(d["dt"], 6), rn(d["B"], 4), rn(d["C"], 4),
+                               d["A"], d["D"], z=d["z"], dt_bias=d["dt_bias"], h0=d["h0"],
+                               flags=oracle.SOFTPLUS)
+    np.testing.assert_allclose(y, y2, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(h, h2, rtol=1e-13, atol=1e-13)
+    st, ys = oracle.m1_step(d["h0"], d["x"][:, 0], d["dt"][:, 0], d["B"][:, 0], d["C"][:, 0],
+                            d["A"], d["D"], z=d["z"][:, 0], dt_bias=d["dt_bias"],
+                            flags=oracle.SOFTPLUS | oracle.RMS_BC | oracle.RMS_DT,
+                            rms_eps=eps)
+    y1, h1, _ = oracle.m1_scan(d["x"][:, :1], d["dt"][:, :1], d["B"][:, :1], d["C"][:, :1],
+                               d["A"], d["D"], z=d["z"][:, :1], dt_bias=d["dt_bias"],
+                               h0=d["h0"],
+                               flags=oracle.SOFTPLUS | oracle.RMS_BC | oracle.RMS_DT,
+                               rms_eps=eps)
+    np.testing.assert_allclose(st, h1, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(ys, y1[:, 0], rtol=1e-13, atol=1e-13)
+
+
+def test_extreme_rates_stay_finite():
+    """The pages quote A down to -36316 and up to -4e-4 ("Mamba-2", "The
+    mixer's values"); large steps then drive the decay to 0, tiny ones to 1."""
+    d = _m1_rand(1, 30, 4, 4, seed=19)
+    d["A"][0] = -36316.0
+    d["A"][1] = -4e-4
+    d["dt"][0, ::3] = 30.0
+    d["dt"][0, 1::3] = -30.0
+    y, h, _ = oracle.m1_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                             dt_bias=d["dt_bias"], h0=d["h0"])
+    assert np.isfinite(y).all() and np.isfinite(h).all()
+    # channel 0 forgets everything on a step of ~30: its state is the last write
+    betas = oracle.softplus(d["dt"][0, -1, 0] + d["dt_bias"][0])
+    np.testing.assert_allclose(h[0, 0], betas * d["B"][0, -1, 0] * d["x"][0, -1, 0],
+                               rtol=1e-12, atol=1e-300)
+
+
+# ------------------------------------------------------ printed page values
+
+def _golden():
+    with open(os.path.join(GOLDEN, "page_shapes.json")) as f:
+        return json.load(f)
+
+
+def test_page_shapes():
+    """The oracle's outputs carry the layouts the pages print for a 10-token
+    prompt on mamba-130m and for mamba2-130m's state."""
+    g = _golden()
+    t = g["mamba1_trace"]
+    d = _m1_rand(t["batch"], t["seqlen"], t["channels"], t["state"], seed=20)
+    y, h, s = oracle.m1_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                             dt_bias=d["dt_bias"], want_states=True)
+    assert list(d["B"].shape) == t["B"] and list(d["C"].shape) == t["C"]
+    assert list(d["x"].shape) == t["x"] and list(d["dt"].shape) == t["dt"]
+    assert list(y.shape) == t["y"] and list(h.shape) == t["state_output"]
+    assert list(s.shape) == g["mamba1_states"]["states"]
+    st, ys = oracle.m1_step(h, d["x"][:, 0], d["dt"][:, 0], d["B"][:, 0], d["C"][:, 0],
+                            d["A"], d["D"], z=d["z"][:, 0], dt_bias=d["dt_bias"])
+    assert list(st.shape) == g["mamba1_decode"]["state_input"]
+    assert list(ys[:, None].shape) == g["mamba1_decode"]["y"]
+    m = g["mamba2_130m"]
+    e = _m2_rand(1, 3, m["heads"], m["head_dim"], m["state"], seed=21)
+    _, h2, _ = oracle.m2_scan(e["x"], e["dt"], e["B"], e["C"], e["A"], e["D"])
+    assert list(h2.shape[1:]) == m["state_output_tail"]
+
+
+def test_page_state_sizes():
+    """The state the scan hands on has the size the pages print: 1.3 MiB for
+    Mamba-130m (crossing GPT-2's 36 KiB/token cache near 38 tokens) and 82 MiB
+    for Mamba-2 2.7B, both in bf16 and counting the width-4 convolution's
+    three carried tokens."""
+    g = _golden()
+    m = g["mamba130m_memory"]
+    ssm = m["layers"] * m["channels"] * m["state"] * m["bytes_per_value"]
+    conv = m["layers"] * m["channels"] * (m["conv_width"] - 1) * m["bytes_per_value"]
+    mib = (ssm + conv) / 2 ** 20
+    assert round(mib, 1) == m["state_mib_printed"]
+    kv = m["gpt2_layers"] * 2 * m["gpt2_d_model"] * m["bytes_per_value"]
+    assert kv / 1024 == m["gpt2_kib_per_token"]
+    assert round((ssm + conv) / kv) == m["crossover_tokens"]
+    q = g["mamba2_2p7b_memory"]
+    d_inner = q["expand"] * q["d_model"]
+    assert d_inner == q["heads"] * q["head_dim"]
+    ssm2 = q["layers"] * q["heads"] * q["state"] * q["head_dim"] * q["bytes_per_value"]
+    conv2 = q["layers"] * (d_inner + 2 * q["groups"] * q["state"]) * (q["conv_width"] - 1) \
+        * q["bytes_per_value"]
+    assert round((ssm2 + conv2) / 2 ** 20) == q["state_mib_printed"]
