@@ -1,0 +1,523 @@
+#!/usr/bin/env python
+"""Benchmark of the selective state-space scan on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  The headline workload is one Mamba-130m-shaped
+mixer scan (ssm_scan_fwd: batch 8, seq 2048, 1536 channels, state 16, bf16
+I/O, fp32 state, silu(z) gate); a step is one call over one batch.  ``value``
+is algorithmic GB/s over all ranks (inputs read once, outputs written once),
+timed with CUDA events over exactly K steps with inputs rotated over enough
+buffer sets to exceed L2.  Beside it, under ``workloads``, the same
+measurement for the Mamba-2 2.7B-shaped SSD chunk scan (tokens/s and tensor
+FLOP rate), the 2.7B decode stack (64 + 24 layer steps, GB/s) and the
+Falcon-width scan with its RMS norms (GB/s).
+
+With N > 1 (launched by torchrun) every rank runs its own independent batch
+(weak scaling, no collective on the data path); time is the max over ranks.
+
+``--impl reference`` times the float64 CPU oracle on the host cores instead,
+on bounded samples of the same workload (one batch row per step).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HEADLINE = "m1_130m_b8_l2048_c1536_n16_bf16"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true",
+                    help="measure only the headline workload")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+# ------------------------------------------------------------------ bytes/flops
+
+def _esz(io):
+    return 2 if io == "bf16" else 4
+
+
+def m1_bytes(w):
+    e = _esz(w.io)
+    tc = w.batch * w.seqlen * w.channels
+    n = (3 + (1 if w.gate else 0)) * tc * e            # x, dt, y (+ z)
+    n += 2 * w.batch * w.seqlen * w.groups * w.state * e  # B, C
+    n += w.channels * w.state * 4 + 2 * w.channels * 4    # A, D, dt_bias
+    n += w.batch * w.channels * w.state * 4               # h_last
+    return n
+
+
+def ssd_bytes(w):
+    e = _esz(w.io)
+    n = 2 * w.batch * w.seqlen * w.heads * w.head_dim * e  # x, y
+    if w.gate:
+        n += w.batch * w.seqlen * w.heads * w.head_dim * e
+    n += w.batch * w.seqlen * w.heads * e                  # dt
+    n += 2 * w.batch * w.seqlen * w.groups * w.state * e   # B, C
+    n += w.batch * w.heads * w.state * w.head_dim * 4      # h_last
+    n += 3 * w.heads * 4
+    return n
+
+
+def ssd_flops(w):
+    """Algorithmic FLOPs of the chunked form with chunk Q, causal half counted:
+    C.B^T per (chunk, group) 2Q^2N; masked product per (chunk, head) Q(Q+1)P;
+    chunk state and state-to-output 2QNP each."""
+    Q = w.chunk
+    nch = w.batch * ((w.seqlen + Q - 1) // Q)
+    cb = nch * w.groups * 2 * Q * Q * w.state
+    per_head = Q * (Q + 1) * w.head_dim + 2 * (2 * Q * w.state * w.head_dim)
+    return cb + nch * w.heads * per_head
+
+
+def decode_bytes(w):
+    e = _esz(w.io)
+    m2 = 2 * w.batch * w.heads * w.state * w.head_dim * 4 \
+        + 2 * w.batch * w.heads * w.head_dim * e + w.batch * w.heads * e \
+        + 2 * w.batch * w.groups * w.state * e + 3 * w.heads * 4
+    m1 = 2 * w.batch * w.m1_channels * w.m1_state * 4 + 4 * w.batch * w.m1_channels * e \
+        + 2 * w.batch * w.groups * w.m1_state * e + (w.m1_state + 2) * w.m1_channels * 4
+    return m2 * w.layers + m1 * w.m1_layers, m2, m1
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler(threading.Thread):
+    """Samples SM clock and throttle reasons with NVML every 50 ms."""
+
+    def __init__(self, index):
+        super().__init__(daemon=True)
+        self.index = index
+        self.samples = []
+        self.stop_ev = threading.Event()
+        self.ok = False
+        self.max_mhz = None
+
+    def run(self):
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            h = N.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+            self.ok = True
+            while not self.stop_ev.is_set():
+                mhz = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+                reasons = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+                util = N.nvmlDeviceGetUtilizationRates(h).gpu
+                self.samples.append((mhz, reasons, util))
+                time.sleep(0.05)
+        except Exception as exc:  # NVML missing: report no clocks
+            self.err = repr(exc)
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "note": "nvml unavailable"}
+        names = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+                 0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+                 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+                 0x100: "display_clock_setting"}
+        loaded = [s for s in self.samples if s[2] > 0] or self.samples
+        rs = set()
+        for _, r, _ in loaded:
+            for bit, n in names.items():
+                if r & bit and n != "gpu_idle":
+                    rs.add(n)
+        return {"sm_mhz": statistics.median(s[0] for s in loaded), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(rs), "samples": len(loaded)}
+
+
+# ------------------------------------------------------------------ helpers
+
+def traffic_for(kernel_key):
+    """dram read+write bytes per launch from the committed ncu summary, or None
+    if the kernel's source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel_key)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != d["source_sha256"]:
+            return None
+    return d["bytes_per_launch"]
+
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, v, device):
+        if not self.pg:
+            return v
+        import torch
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+def timed(step, K, W, dist, device):
+    """W untimed steps, then exactly K steps between two events, with a barrier
+    and a device synchronize on both sides.  Returns max-over-ranks ms."""
+    import torch
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize(device)
+    dist.barrier()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(K):
+        step(W + i)
+    e.record()
+    torch.cuda.synchronize(device)
+    dist.barrier()
+    return dist.max(s.elapsed_time(e), device)
+
+
+def per_launch_ms(step, n, device):
+    """Average device time of one step measured by an event pair around each."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for i, (a, b) in enumerate(evs):
+        a.record()
+        step(i)
+        b.record()
+    torch.cuda.synchronize(device)
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def n_sets(bytes_per_set):
+    return max(2, -(-3 * L2_BYTES // max(1, bytes_per_set)))
+
+
+# ------------------------------------------------------------------ ours
+
+def bench_m1(w, K, W, dist, device, pk, seed_base):
+    import torch
+    from selective_state_space_28_b200 import inputs as I
+    from selective_state_space_28_b200 import ops
+    nb = m1_bytes(w)
+    sets = []
+    for r in range(n_sets(nb)):
+        d = I.workload_inputs(w, device=device, seed=seed_base + 1000 * r)
+        d["y"] = torch.empty_like(d["x"])
+        d["h_last"] = torch.empty((w.batch, w.channels, w.state), device=device)
+        sets.append(d)
+
+    def step(i):
+        d = sets[i % len(sets)]
+        ops.ssm_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                         dt_bias=d["dt_bias"], flags=w.flags, rms_eps=w.rms_eps,
+                         y=d["y"], h_last=d["h_last"])
+    ms = timed(step, K, W, dist, device) / K
+    launch_ms = per_launch_ms(step, max(5, min(K, 20)), device)
+    launches = 2 if (w.flags & I.RMS_DT) else 1
+    return {"ms_per_step": ms, "bytes": nb, "launch_ms": launch_ms, "sets": len(sets),
+            "launches_per_step": launches}
+
+
+def bench_ssd(w, K, W, dist, device, pk, seed_base):
+    import torch
+    from selective_state_space_28_b200 import inputs as I
+    from selective_state_space_28_b200 import ops
+    nb = ssd_bytes(w)
+    sets = []
+    for r in range(n_sets(nb)):
+        d = I.workload_inputs(w, device=device, seed=seed_base + 1000 * r)
+        d["y"] = torch.empty_like(d["x"])
+        d["h_last"] = torch.empty((w.batch, w.heads, w.state, w.head_dim), device=device)
+        sets.append(d)
+    ws = ops.ssd_workspace_bytes(batch=w.batch, seqlen=w.seqlen, heads=w.heads,
+                                 head_dim=w.head_dim, state=w.state, groups=w.groups,
+                                 chunk=w.chunk, io=1 if w.io == "bf16" else 0, flags=w.flags)
+    wsb = torch.empty(max(ws, 1), dtype=torch.uint8, device=device)
+
+    def step(i):
+        d = sets[i % len(sets)]
+        ops.ssd_chunk_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                               dt_bias=d["dt_bias"], chunk=w.chunk, flags=w.flags,
+                               y=d["y"], h_last=d["h_last"], workspace=wsb)
+    ms = timed(step, K, W, dist, device) / K
+    launch_ms = per_launch_ms(step, max(3, min(K, 10)), device)
+    return {"ms_per_step": ms, "bytes": nb, "flops": ssd_flops(w), "launch_ms": launch_ms,
+            "tokens": w.batch * w.seqlen, "sets": len(sets), "launches_per_step": 1}
+
+
+def bench_decode(w, K, W, dist, device, pk, seed_base):
+    import torch
+    from selective_state_space_28_b200 import inputs as I
+    from selective_state_space_28_b200 import ops
+    total, m2b, m1b = decode_bytes(w)
+    m2_layers, m1_layers = [], []
+    for l in range(w.layers):
+        m2_layers.append(I.m2_step_inputs(w.batch, w.heads, w.head_dim, w.state, w.groups,
+                                          w.io, w.gate, seed=seed_base + l, device=device))
+        m2_layers[-1]["y"] = torch.empty_like(m2_layers[-1]["x"])
+    for l in range(w.m1_layers):
+        m1_layers.append(I.m1_step_inputs(w.batch, w.m1_channels, w.m1_state, w.groups,
+                                          w.io, True, seed=seed_base + 500 + l, device=device))
+        m1_layers[-1]["y"] = torch.empty_like(m1_layers[-1]["x"])
+
+    def one(d):
+        ops.ssm_scan_step(d["state"], d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"],
+                          z=d["z"], dt_bias=d["dt_bias"], y=d["y"])
+
+    def step(i):
+        for d in m2_layers:
+            one(d)
+        for d in m1_layers:
+            one(d)
+    ms = timed(step, K, W, dist, device) / K
+    m2_ms = per_launch_ms(lambda i: one(m2_layers[i % len(m2_layers)]), 16, device)
+    return {"ms_per_step": ms, "bytes": total, "launch_ms": m2_ms, "launch_bytes": m2b,
+            "launches_per_step": w.layers + w.m1_layers}
+
+
+def e2e_m1(w, device, n_steps=5):
+    """The same metric through the public API with pinned HOST buffers: each
+    step copies its inputs host->device, scans, and reads y and h_last back."""
+    import torch
+    from selective_state_space_28_b200 import inputs as I
+    from selective_state_space_28_b200 import ops
+    d = I.workload_inputs(w, device="cpu")
+    d = {k: (v.pin_memory() if v is not None else None) for k, v in d.items()}
+    h2d = sum(v.numel() * v.element_size() for v in d.values() if v is not None)
+    d2h = d["x"].numel() * d["x"].element_size() + w.batch * w.channels * w.state * 4
+
+    def step():
+        y, h, _ = ops.ssm_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"],
+                                   z=d["z"], dt_bias=d["dt_bias"], flags=w.flags,
+                                   rms_eps=w.rms_eps)
+        return y, h
+    step()
+    torch.cuda.synchronize(device)
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(n_steps):
+        step()
+    e.record()
+    torch.cuda.synchronize(device)
+    ms = s.elapsed_time(e) / n_steps
+    return {"ms": ms, "h2d": h2d, "d2h": d2h}
+
+
+def cpu_baseline_m1(w, rows=1):
+    """The oracle, as it stands, on a bounded sample: `rows` batch rows of the
+    workload, all channels and tokens, on every host core it may use."""
+    import oracle
+    from selective_state_space_28_b200 import inputs as I
+    d = I.workload_inputs(w, device="cpu")
+    sub = {k: (v[:rows] if (v is not None and k in ("x", "dt", "z", "B", "C")) else v)
+           for k, v in d.items()}
+    threads = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.m1_scan(sub["x"], sub["dt"], sub["B"], sub["C"], sub["A"], sub["D"], z=sub["z"],
+                   dt_bias=sub["dt_bias"], flags=w.flags, rms_eps=w.rms_eps, nthreads=threads)
+    sec = time.perf_counter() - t0
+    frac = rows / w.batch
+    gbs = m1_bytes(w) * frac / sec / 1e9
+    return {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": "%d of %d batch rows of %s (all %d tokens x %d channels x state %d), "
+                      "float64 C token loop, %.2f s" % (rows, w.batch, w.name, w.seqlen,
+                                                        w.channels, w.state, sec)}
+
+
+def run_ours(args):
+    import torch
+    from selective_state_space_28_b200 import build as B
+    from selective_state_space_28_b200 import inputs as I
+    B.build()
+    dist = Dist()
+    torch.cuda.set_device(dist.local)
+    device = torch.device("cuda", dist.local)
+    dist.init("nccl")
+    pk = peaks()
+    K, W = args.steps, args.warmup
+    sampler = ClockSampler(dist.local)
+    sampler.start()
+    time.sleep(0.2)
+
+    w = I.WORKLOADS[HEADLINE]
+    r = bench_m1(w, K, W, dist, device, pk, seed_base=w.seed + 7919 * dist.rank)
+    sampler.stop_ev.set()
+    sampler.join(timeout=2)
+    clocks = sampler.summary()
+    hbm = pk["hbm_gbs"]
+    value = r["bytes"] * dist.world / (r["ms_per_step"] * 1e-3) / 1e9
+    achieved = r["bytes"] / (r["launch_ms"] * 1e-3) / 1e9
+    out = {
+        "metric": "Mamba-1 selective scan algorithmic HBM throughput (GB/s); "
+                  "SSD chunk-scan tokens/s under workloads",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": dist.world, "steps": K,
+        "warmup": W, "ms_per_step": round(r["ms_per_step"], 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) inputs, S4D-real A, softplus^-1 dt_bias)",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen,
+                   "channels": w.channels, "state": w.state, "groups": w.groups,
+                   "io_dtype": w.io, "state_dtype": "f32", "gate": w.gate,
+                   "l2": "inputs rotated over %d buffer sets (%.0f MB each) > L2"
+                         % (r["sets"], r["bytes"] / 1e6),
+                   "parallelism": "dp%d (independent batches per GPU)" % dist.world},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm,
+                     "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                     "traffic": traffic_for("m1_scan_130m"),
+                     "peak_source": "%s hbm_gbs (copy)" % pk["_source"],
+                     "kernel": "m1_scan_kernel"},
+        "clocks": clocks,
+        "gpu_launches": r["launches_per_step"] * K,
+    }
+    if not args.no_e2e:
+        e = e2e_m1(w, device)
+        out["e2e"] = {"value": round(r["bytes"] / (e["ms"] * 1e-3) / 1e9, 3), "unit": "GB/s",
+                      "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                      "ms_per_step": round(e["ms"], 3)}
+    if not args.no_extra:
+        wl = {}
+        ws = I.WORKLOADS["ssd_2p7b_b4_l4096_h80_p64_n128_bf16"]
+        Ke = max(3, min(K, 20))
+        s = bench_ssd(ws, Ke, max(3, W), dist, device, pk, ws.seed + 7919 * dist.rank)
+        tf = s["flops"] / (s["launch_ms"] * 1e-3) / 1e12
+        wl[ws.name] = {
+            "value": round(s["tokens"] * dist.world / (s["ms_per_step"] * 1e-3), 1),
+            "unit": "tokens/s", "ms_per_step": round(s["ms_per_step"], 4),
+            "gbs": round(s["bytes"] / (s["ms_per_step"] * 1e-3) / 1e9, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2),
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(tf / pk["bf16_tflops"], 4),
+                         "traffic": traffic_for("ssd_2p7b"),
+                         "flops_per_launch": s["flops"], "bytes_per_launch": s["bytes"],
+                         "hbm_frac": round(s["bytes"] / (s["launch_ms"] * 1e-3) / 1e9 / hbm, 4)}}
+        wd = I.WORKLOADS["decode_2p7b_stack_b256"]
+        dd = bench_decode(wd, max(3, min(K, 5)), 3, dist, device, pk, wd.seed + 7919 * dist.rank)
+        ach = dd["launch_bytes"] / (dd["launch_ms"] * 1e-3) / 1e9
+        wl[wd.name] = {
+            "value": round(dd["bytes"] * dist.world / (dd["ms_per_step"] * 1e-3) / 1e9, 2),
+            "unit": "GB/s", "ms_per_step": round(dd["ms_per_step"], 4),
+            "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
+                         "frac": round(ach / hbm, 4), "traffic": traffic_for("m2_step_2p7b"),
+                         "kernel": "mamba-2 layer step"}}
+        del dd
+        torch.cuda.empty_cache()
+        wf = I.WORKLOADS["m1_falcon_rms_b4_l8192_c8192_n16_bf16"]
+        f = bench_m1(wf, max(3, min(K, 10)), 3, dist, device, pk, wf.seed + 7919 * dist.rank)
+        ach = f["bytes"] / (f["launch_ms"] * 1e-3) / 1e9
+        wl[wf.name] = {
+            "value": round(f["bytes"] * dist.world / (f["ms_per_step"] * 1e-3) / 1e9, 2),
+            "unit": "GB/s", "ms_per_step": round(f["ms_per_step"], 4),
+            "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
+                         "frac": round(ach / hbm, 4), "traffic": traffic_for("m1_scan_falcon"),
+                         "note": "algorithmic bytes exclude the step-norm pre-pass re-read"}}
+        out["workloads"] = wl
+        out["gpu_launches"] += (s["launches_per_step"] * Ke)
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_m1(w)
+    dist.close()
+    if dist.rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------------ reference
+
+def run_reference(args):
+    dist = Dist()
+    if dist.rank != 0:
+        return
+    from selective_state_space_28_b200 import inputs as I
+    import oracle
+    w = I.WORKLOADS[HEADLINE]
+    d = I.workload_inputs(w, device="cpu")
+    threads = oracle.default_threads()
+    rows = 1
+
+    def step(i):
+        r = i % w.batch
+        sub = {k: (v[r:r + rows] if (v is not None and k in ("x", "dt", "z", "B", "C")) else v)
+               for k, v in d.items()}
+        oracle.m1_scan(sub["x"], sub["dt"], sub["B"], sub["C"], sub["A"], sub["D"], z=sub["z"],
+                       dt_bias=sub["dt_bias"], flags=w.flags, rms_eps=w.rms_eps,
+                       nthreads=threads)
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    sec = (time.perf_counter() - t0) / args.steps
+    nb = m1_bytes(w) * rows / w.batch
+    value = nb / sec / 1e9
+    sample = ("one of %d batch rows of %s per step (all %d tokens x %d channels x state %d), "
+              "float64 C token loop" % (w.batch, w.name, w.seqlen, w.channels, w.state))
+    out = {"impl": "reference", "metric": "Mamba-1 selective scan algorithmic HBM throughput "
+           "(GB/s); SSD chunk-scan tokens/s under workloads", "value": round(value, 4),
+           "unit": "GB/s", "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen,
+                      "channels": w.channels, "state": w.state, "io_dtype": w.io,
+                      "sample_rows_per_step": rows},
+           "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)

@@ -1,0 +1,204 @@
+/*
+ * ssm.h -- C ABI of libssm: the selective state-space scan on NVIDIA B200
+ * (sm_100a).
+ *
+ * Three operations, each a plain C call on plain pointers and sizes:
+ *
+ *   ssm_scan_fwd        Mamba-1 selective scan over a prompt.
+ *   ssd_chunk_scan_fwd  Mamba-2 (SSD) scan over a prompt, chunked.
+ *   ssm_scan_step       one decode token against a cached state.
+ *
+ * Conventions for every call
+ * --------------------------
+ * - Pointers are DEVICE pointers (cudaMalloc'd or otherwise device-visible),
+ *   owned by the caller.  The library allocates nothing, keeps no state
+ *   between calls, and is reentrant.  Work is queued on `stream` (a
+ *   cudaStream_t passed as void*; NULL = the legacy default stream) and the
+ *   call returns without synchronising; results are ordered on `stream`.
+ * - Layouts are dense, row-major and tokens-first, as the pages' values are
+ *   ("Mamba" nnterp guide, "The values" table: x is [batch, seq, channels],
+ *   state is [batch, channels, state_dim]; "Mamba-2": the state is
+ *   [batch, heads, key_dim, value_dim], key side first).
+ * - `io` selects the element type of x, dt, z, B, C and y (SSM_F32 or
+ *   SSM_BF16).  A, D, dt_bias and every state are float32, and all
+ *   arithmetic is float32.
+ * - Arguments are validated on the host before anything is launched.  On an
+ *   error the call returns a status and launches nothing.  Launch failures
+ *   return SSM_ERR_CUDA.  There is no CPU fallback.
+ * - Aliasing: inputs and outputs must not overlap, except that h_last may
+ *   equal h0 (the state hand-off), and the decode step updates its state in
+ *   place.
+ */
+#ifndef SSM_H
+#define SSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SSM_ABI_VERSION 1
+
+typedef enum ssm_status {
+  SSM_OK = 0,
+  SSM_ERR_NULL = 1,        /* a required pointer is NULL                      */
+  SSM_ERR_SHAPE = 2,       /* a size is <= 0, or groups does not divide       */
+  SSM_ERR_DTYPE = 3,       /* io is not SSM_F32 / SSM_BF16                    */
+  SSM_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned                */
+  SSM_ERR_UNSUPPORTED = 5, /* a valid combination this build has no kernel for */
+  SSM_ERR_WORKSPACE = 6,   /* workspace missing or smaller than required      */
+  SSM_ERR_CUDA = 7,        /* a CUDA launch or runtime call failed            */
+  SSM_ERR_TIMEOUT = 8      /* reserved: a bounded device wait ran out         */
+} ssm_status_t;
+
+typedef enum ssm_dtype { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
+
+/* flags */
+#define SSM_DT_SOFTPLUS 1u /* step = softplus(dt + dt_bias); else dt + dt_bias  */
+#define SSM_RMSNORM_BC 2u  /* B, C <- v / sqrt(mean_N(v^2) + rms_eps) (no gain) */
+#define SSM_RMSNORM_DT 4u  /* dt <- dt / sqrt(mean_C(dt^2) + rms_eps), before
+                              the bias (Mamba-1 scan only)                      */
+
+/* ------------------------------------------------------------------------
+ * ssm_scan_fwd -- Mamba-1 selective scan.
+ *
+ * Defined by: "Mamba" (nnterp guide, architectures/mamba), intro and "The
+ * values" table; "Mamba" (tokentrails lineage), "Code"; "Falcon-Mamba"
+ * (nnterp encyclopedia), "Where the norms sit" for the two RMS flags.
+ * For every batch b, channel c (group g = c / (channels / groups)) and token t:
+ *
+ *   d     = dt[b,t,c]  (* RMS factor of dt[b,t,:] if SSM_RMSNORM_DT)
+ *   d     = softplus(d + dt_bias[c])  (or d + dt_bias[c] without SSM_DT_SOFTPLUS)
+ *   h[n]  = exp(d * A[c,n]) * h[n] + d * B[b,t,g,n] * x[b,t,c]   (n < state)
+ *   y     = sum_n C[b,t,g,n] * h[n] + D[c] * x[b,t,c]
+ *   y    *= silu(z[b,t,c])             if z != NULL
+ *
+ * with h starting from h0[b,c,:] (zeros if h0 == NULL).  y_t reads the state
+ * after token t's write.
+ *
+ *   x, dt, z, y : [batch, seqlen, channels]   io type; z may be NULL (no gate)
+ *   B, C        : [batch, seqlen, groups, state]  io type
+ *   A           : [channels, state]  float32 (pass -exp(A_log))
+ *   D, dt_bias  : [channels]         float32, may be NULL (= 0)
+ *   h0          : [batch, channels, state] float32 or NULL (= zeros)
+ *   h_last      : [batch, channels, state] float32 or NULL; may equal h0
+ *   states      : [batch, seqlen, channels, state] float32 or NULL: the state
+ *                 after every token (states[:, -1] == h_last bit for bit)
+ *   workspace   : needed only with SSM_RMSNORM_DT; size from
+ *                 ssm_scan_workspace().  Device memory, caller-owned.
+ *
+ * Supported: state in {4, 8, 16, 32, 64}; groups must divide channels, and
+ * with groups > 1 channels/groups must be a multiple of 32.
+ * ---------------------------------------------------------------------- */
+typedef struct ssm_scan_args {
+  int64_t batch, seqlen, channels, state, groups;
+  int32_t io;        /* ssm_dtype_t */
+  uint32_t flags;
+  float rms_eps;
+  const void *x, *dt, *z, *B, *C;
+  const float *A, *D, *dt_bias, *h0;
+  void *y;
+  float *h_last, *states;
+  void *workspace;
+  size_t workspace_bytes;
+} ssm_scan_args_t;
+
+/* Bytes of device workspace ssm_scan_fwd needs for these arguments (0 unless
+ * SSM_RMSNORM_DT).  Validates sizes, dtype and flags as ssm_scan_fwd does;
+ * the tensor pointers are not looked at. */
+ssm_status_t ssm_scan_workspace(const ssm_scan_args_t *args, size_t *bytes);
+ssm_status_t ssm_scan_fwd(const ssm_scan_args_t *args, void *stream);
+
+/* ------------------------------------------------------------------------
+ * ssd_chunk_scan_fwd -- Mamba-2 (SSD) scan.
+ *
+ * Defined by: "Mamba-2" (nnterp encyclopedia), "The mixer's values" (one
+ * scalar decay per head and token; B and C shared by the heads of a group),
+ * "The hidden attention" (the causal masked form the chunked algorithm
+ * evaluates), "The state" (key side first).  For batch b, head h (group
+ * g = h / (heads / groups)), token t:
+ *
+ *   d      = softplus(dt[b,t,h] + dt_bias[h])   (flag SSM_DT_SOFTPLUS)
+ *   S      = exp(d * A[h]) * S + d * outer(B[b,t,g,:], x[b,t,h,:])   (N x P)
+ *   y[p]   = sum_n C[b,t,g,n] * S[n,p] + D[h] * x[b,t,h,p];  *= silu(z) if z
+ *
+ * evaluated chunk by chunk (`chunk` tokens): within a chunk as the masked
+ * product y_t = sum_{s<=t} (C_t . B_s) exp(cum_t - cum_s) d_s x_s, across
+ * chunks through the carried N x P state.  The result does not depend on
+ * `chunk` beyond rounding.
+ *
+ *   x, z, y  : [batch, seqlen, heads, head_dim]  io type; z may be NULL
+ *   dt       : [batch, seqlen, heads]            io type
+ *   B, C     : [batch, seqlen, groups, state]    io type
+ *   A        : [heads] float32; D, dt_bias: [heads] float32 or NULL (= 0)
+ *   h0       : [batch, heads, state, head_dim] float32 or NULL (= zeros)
+ *   h_last   : [batch, heads, state, head_dim] float32 or NULL; may equal h0
+ *   states   : [batch, seqlen, heads, state, head_dim] float32 or NULL
+ *   workspace: device memory of ssd_chunk_scan_workspace() bytes, or NULL if
+ *              that is 0.
+ *
+ * Only SSM_DT_SOFTPLUS is accepted in flags.
+ * ---------------------------------------------------------------------- */
+typedef struct ssd_scan_args {
+  int64_t batch, seqlen, heads, head_dim, state, groups, chunk;
+  int32_t io;
+  uint32_t flags;
+  const void *x, *z, *dt, *B, *C;
+  const float *A, *D, *dt_bias, *h0;
+  void *y;
+  float *h_last, *states;
+  void *workspace;
+  size_t workspace_bytes;
+} ssd_scan_args_t;
+
+/* Bytes of device workspace ssd_chunk_scan_fwd needs (sizes, dtype and flags
+ * are validated; the tensor pointers are not looked at). */
+ssm_status_t ssd_chunk_scan_workspace(const ssd_scan_args_t *args, size_t *bytes);
+ssm_status_t ssd_chunk_scan_fwd(const ssd_scan_args_t *args, void *stream);
+
+/* ------------------------------------------------------------------------
+ * ssm_scan_step -- one decode token per sequence, state updated in place.
+ *
+ * Defined by: "Mamba" (nnterp guide), "The state" and the "Read order on a
+ * decode step" warning: the decode kernel updates the state first and reads
+ * y from the updated state; the state is handed from one step's output to
+ * the next step's input.  "Mamba-2", "The state", for the N x P form.
+ *
+ * SSM_STEP_MAMBA1: units = channels, head_dim = 1.
+ *   x, dt, z, y: [batch, channels]; B, C: [batch, groups, state];
+ *   A: [channels, state]; D, dt_bias: [channels]; state: [batch, channels, state]
+ * SSM_STEP_MAMBA2: units = heads.
+ *   x, z, y: [batch, heads, head_dim]; dt: [batch, heads];
+ *   B, C: [batch, groups, state]; A, D, dt_bias: [heads];
+ *   state: [batch, heads, state, head_dim] (key side first)
+ *
+ * The arithmetic is one token of ssm_scan_fwd / ssd_chunk_scan_fwd.  flags:
+ * SSM_DT_SOFTPLUS, and for Mamba-1 also SSM_RMSNORM_BC.
+ * ---------------------------------------------------------------------- */
+typedef enum ssm_step_kind { SSM_STEP_MAMBA1 = 1, SSM_STEP_MAMBA2 = 2 } ssm_step_kind_t;
+
+typedef struct ssm_step_args {
+  int32_t kind; /* ssm_step_kind_t */
+  int32_t io;
+  uint32_t flags;
+  float rms_eps;
+  int64_t batch, units, head_dim, state, groups;
+  const void *x, *dt, *z, *B, *C;
+  const float *A, *D, *dt_bias;
+  float *state_io;
+  void *y;
+} ssm_step_args_t;
+
+ssm_status_t ssm_scan_step(const ssm_step_args_t *args, void *stream);
+
+/* A short English description of a status; never NULL. */
+const char *ssm_status_string(ssm_status_t status);
+/* SSM_ABI_VERSION of the library. */
+int ssm_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSM_H */

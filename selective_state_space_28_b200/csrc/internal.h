@@ -1,0 +1,55 @@
+// internal.h -- launcher interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssm {
+
+// Mamba-1 scan, device pointers as in ssm_scan_args_t.
+struct M1Params {
+  int64_t batch, L, C, N, G;
+  uint32_t flags;
+  float eps;
+  int io;  // 0 = f32, 1 = bf16
+  const void *x, *dt, *z, *B, *Cm;
+  const float *A, *D, *dt_bias, *h0;
+  void *y;
+  float *h_last, *states;
+  float *rstd;  // [batch * L] RMS factors of dt rows, or nullptr
+};
+
+// Mamba-2 token recurrence (the decode step, and the SSD path for shapes the
+// chunked tensor-core kernel does not cover).
+struct M2Params {
+  int64_t batch, L, H, P, N, G;
+  uint32_t flags;
+  int io;
+  const void *x, *z, *dt, *B, *Cm;
+  const float *A, *D, *dt_bias;
+  const float *h0;  // initial state or nullptr (the step passes its state)
+  void *y;
+  float *h_last, *states;
+};
+
+struct M1StepParams {
+  int64_t batch, C, N, G;
+  uint32_t flags;
+  float eps;
+  int io;
+  const void *x, *dt, *z, *B, *Cm;
+  const float *A, *D, *dt_bias;
+  float *state;
+  void *y;
+};
+
+// Each returns cudaSuccess, cudaErrorNotSupported for a shape without a
+// kernel (checked before any launch), or the launch error.
+cudaError_t launch_m1_scan(const M1Params &p, cudaStream_t s);
+bool m1_scan_supported(int64_t N, int64_t C, int64_t G);
+cudaError_t launch_m2_recurrent(const M2Params &p, cudaStream_t s);
+bool m2_recurrent_supported(int64_t N, int64_t P);
+cudaError_t launch_m1_step(const M1StepParams &p, cudaStream_t s);
+bool m1_step_supported(int64_t N);
+
+}  // namespace ssm

@@ -1,0 +1,256 @@
+// ssm_api.cu -- the exported C ABI (include/ssm.h): argument validation on
+// the host, then dispatch to the kernels.  Nothing is launched when a check
+// fails, and nothing here allocates memory.
+#include <stdint.h>
+#include <string.h>
+
+#include "internal.h"
+#include "ssm.h"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Every non-NULL pointer must be 16-byte aligned.
+template <typename... Ps>
+bool all_aligned(Ps... ps) {
+  const void *arr[] = {static_cast<const void *>(ps)...};
+  for (const void *p : arr)
+    if (p && !aligned16(p)) return false;
+  return true;
+}
+
+ssm_status_t from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return SSM_OK;
+  if (e == cudaErrorNotSupported) return SSM_ERR_UNSUPPORTED;
+  return SSM_ERR_CUDA;
+}
+
+// seqlen == 0: the state passes through unchanged (h_last = h0, or zeros).
+ssm_status_t pass_state(const float *h0, float *h_last, size_t bytes, cudaStream_t s) {
+  if (!h_last || bytes == 0) return SSM_OK;
+  cudaError_t e = cudaSuccess;
+  if (!h0) e = cudaMemsetAsync(h_last, 0, bytes, s);
+  else if (h0 != h_last) e = cudaMemcpyAsync(h_last, h0, bytes, cudaMemcpyDeviceToDevice, s);
+  return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+// shapes_only: the workspace query validates sizes and flags, not pointers.
+ssm_status_t check_scan(const ssm_scan_args_t *a, size_t *ws, bool shapes_only = false) {
+  if (!a) return SSM_ERR_NULL;
+  if (a->io != SSM_F32 && a->io != SSM_BF16) return SSM_ERR_DTYPE;
+  if (a->batch < 0 || a->seqlen < 0 || a->channels <= 0 || a->state <= 0 ||
+      a->groups <= 0 || a->channels % a->groups)
+    return SSM_ERR_SHAPE;
+  if (a->flags & ~(SSM_DT_SOFTPLUS | SSM_RMSNORM_BC | SSM_RMSNORM_DT))
+    return SSM_ERR_UNSUPPORTED;
+  if ((a->flags & (SSM_RMSNORM_BC | SSM_RMSNORM_DT)) && !(a->rms_eps >= 0.f))
+    return SSM_ERR_SHAPE;
+  if (!shapes_only && a->batch > 0 && a->seqlen > 0 &&
+      (!a->x || !a->dt || !a->B || !a->C || !a->A || !a->y))
+    return SSM_ERR_NULL;
+  if (!shapes_only &&
+      !all_aligned(a->x, a->dt, a->z, a->B, a->C, a->A, a->D, a->dt_bias, a->h0, a->y,
+                   a->h_last, a->states, a->workspace))
+    return SSM_ERR_ALIGN;
+  if (!ssm::m1_scan_supported(a->state, a->channels, a->groups) || a->batch > 65535)
+    return SSM_ERR_UNSUPPORTED;
+  *ws = (a->flags & SSM_RMSNORM_DT) ? (size_t)(a->batch * a->seqlen) * sizeof(float) : 0;
+  return SSM_OK;
+}
+
+ssm_status_t check_ssd(const ssd_scan_args_t *a, size_t *ws, bool shapes_only = false) {
+  if (!a) return SSM_ERR_NULL;
+  if (a->io != SSM_F32 && a->io != SSM_BF16) return SSM_ERR_DTYPE;
+  if (a->batch < 0 || a->seqlen < 0 || a->heads <= 0 || a->head_dim <= 0 ||
+      a->state <= 0 || a->groups <= 0 || a->chunk <= 0 || a->heads % a->groups)
+    return SSM_ERR_SHAPE;
+  if (a->flags & ~SSM_DT_SOFTPLUS) return SSM_ERR_UNSUPPORTED;
+  if (!shapes_only && a->batch > 0 && a->seqlen > 0 &&
+      (!a->x || !a->dt || !a->B || !a->C || !a->A || !a->y))
+    return SSM_ERR_NULL;
+  if (!shapes_only &&
+      !all_aligned(a->x, a->z, a->dt, a->B, a->C, a->A, a->D, a->dt_bias, a->h0, a->y,
+                   a->h_last, a->states, a->workspace))
+    return SSM_ERR_ALIGN;
+  if (!ssm::m2_recurrent_supported(a->state, a->head_dim) || a->batch > 65535)
+    return SSM_ERR_UNSUPPORTED;
+  *ws = 0;
+  return SSM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssm_abi_version(void) { return SSM_ABI_VERSION; }
+
+const char *ssm_status_string(ssm_status_t s) {
+  switch (s) {
+    case SSM_OK: return "ok";
+    case SSM_ERR_NULL: return "a required pointer is NULL";
+    case SSM_ERR_SHAPE: return "invalid size or shape";
+    case SSM_ERR_DTYPE: return "unsupported io dtype";
+    case SSM_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case SSM_ERR_UNSUPPORTED: return "combination not supported by this build";
+    case SSM_ERR_WORKSPACE: return "workspace missing or too small";
+    case SSM_ERR_CUDA: return "CUDA error";
+    case SSM_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+ssm_status_t ssm_scan_workspace(const ssm_scan_args_t *a, size_t *bytes) {
+  if (!bytes) return SSM_ERR_NULL;
+  size_t ws = 0;
+  ssm_status_t st = check_scan(a, &ws, true);
+  if (st == SSM_OK) *bytes = ws;
+  return st;
+}
+
+ssm_status_t ssm_scan_fwd(const ssm_scan_args_t *a, void *stream) {
+  size_t ws = 0;
+  ssm_status_t st = check_scan(a, &ws);
+  if (st != SSM_OK) return st;
+  if (ws && (!a->workspace || a->workspace_bytes < ws)) return SSM_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (a->batch == 0) return SSM_OK;
+  if (a->seqlen == 0)
+    return pass_state(a->h0, a->h_last,
+                      (size_t)(a->batch * a->channels * a->state) * sizeof(float), s);
+  ssm::M1Params p;
+  p.batch = a->batch;
+  p.L = a->seqlen;
+  p.C = a->channels;
+  p.N = a->state;
+  p.G = a->groups;
+  p.flags = a->flags;
+  p.eps = a->rms_eps;
+  p.io = a->io;
+  p.x = a->x;
+  p.dt = a->dt;
+  p.z = a->z;
+  p.B = a->B;
+  p.Cm = a->C;
+  p.A = a->A;
+  p.D = a->D;
+  p.dt_bias = a->dt_bias;
+  p.h0 = a->h0;
+  p.y = a->y;
+  p.h_last = a->h_last;
+  p.states = a->states;
+  p.rstd = (a->flags & SSM_RMSNORM_DT) ? static_cast<float *>(a->workspace) : nullptr;
+  return from_cuda(ssm::launch_m1_scan(p, s));
+}
+
+ssm_status_t ssd_chunk_scan_workspace(const ssd_scan_args_t *a, size_t *bytes) {
+  if (!bytes) return SSM_ERR_NULL;
+  size_t ws = 0;
+  ssm_status_t st = check_ssd(a, &ws, true);
+  if (st == SSM_OK) *bytes = ws;
+  return st;
+}
+
+ssm_status_t ssd_chunk_scan_fwd(const ssd_scan_args_t *a, void *stream) {
+  size_t ws = 0;
+  ssm_status_t st = check_ssd(a, &ws);
+  if (st != SSM_OK) return st;
+  if (ws && (!a->workspace || a->workspace_bytes < ws)) return SSM_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (a->batch == 0) return SSM_OK;
+  if (a->seqlen == 0)
+    return pass_state(a->h0, a->h_last,
+                      (size_t)(a->batch * a->heads * a->state * a->head_dim) * sizeof(float),
+                      s);
+  ssm::M2Params p;
+  p.batch = a->batch;
+  p.L = a->seqlen;
+  p.H = a->heads;
+  p.P = a->head_dim;
+  p.N = a->state;
+  p.G = a->groups;
+  p.flags = a->flags;
+  p.io = a->io;
+  p.x = a->x;
+  p.z = a->z;
+  p.dt = a->dt;
+  p.B = a->B;
+  p.Cm = a->C;
+  p.A = a->A;
+  p.D = a->D;
+  p.dt_bias = a->dt_bias;
+  p.h0 = a->h0;
+  p.y = a->y;
+  p.h_last = a->h_last;
+  p.states = a->states;
+  return from_cuda(ssm::launch_m2_recurrent(p, s));
+}
+
+ssm_status_t ssm_scan_step(const ssm_step_args_t *a, void *stream) {
+  if (!a) return SSM_ERR_NULL;
+  if (a->io != SSM_F32 && a->io != SSM_BF16) return SSM_ERR_DTYPE;
+  if (a->kind != SSM_STEP_MAMBA1 && a->kind != SSM_STEP_MAMBA2) return SSM_ERR_UNSUPPORTED;
+  if (a->batch < 0 || a->units <= 0 || a->head_dim <= 0 || a->state <= 0 ||
+      a->groups <= 0 || a->units % a->groups)
+    return SSM_ERR_SHAPE;
+  if (a->kind == SSM_STEP_MAMBA1 && a->head_dim != 1) return SSM_ERR_SHAPE;
+  const uint32_t allowed =
+      a->kind == SSM_STEP_MAMBA1 ? (SSM_DT_SOFTPLUS | SSM_RMSNORM_BC) : SSM_DT_SOFTPLUS;
+  if (a->flags & ~allowed) return SSM_ERR_UNSUPPORTED;
+  if ((a->flags & SSM_RMSNORM_BC) && !(a->rms_eps >= 0.f)) return SSM_ERR_SHAPE;
+  if (a->batch > 0 && (!a->x || !a->dt || !a->B || !a->C || !a->A || !a->state_io || !a->y))
+    return SSM_ERR_NULL;
+  if (!all_aligned(a->x, a->dt, a->z, a->B, a->C, a->A, a->D, a->dt_bias, a->state_io, a->y))
+    return SSM_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (a->kind == SSM_STEP_MAMBA1) {
+    if (!ssm::m1_step_supported(a->state)) return SSM_ERR_UNSUPPORTED;
+    if (a->batch == 0) return SSM_OK;
+    ssm::M1StepParams p;
+    p.batch = a->batch;
+    p.C = a->units;
+    p.N = a->state;
+    p.G = a->groups;
+    p.flags = a->flags;
+    p.eps = a->rms_eps;
+    p.io = a->io;
+    p.x = a->x;
+    p.dt = a->dt;
+    p.z = a->z;
+    p.B = a->B;
+    p.Cm = a->C;
+    p.A = a->A;
+    p.D = a->D;
+    p.dt_bias = a->dt_bias;
+    p.state = a->state_io;
+    p.y = a->y;
+    return from_cuda(ssm::launch_m1_step(p, s));
+  }
+  if (!ssm::m2_recurrent_supported(a->state, a->head_dim) || a->batch > 65535)
+    return SSM_ERR_UNSUPPORTED;
+  if (a->batch == 0) return SSM_OK;
+  ssm::M2Params p;
+  p.batch = a->batch;
+  p.L = 1;
+  p.H = a->units;
+  p.P = a->head_dim;
+  p.N = a->state;
+  p.G = a->groups;
+  p.flags = a->flags;
+  p.io = a->io;
+  p.x = a->x;
+  p.z = a->z;
+  p.dt = a->dt;
+  p.B = a->B;
+  p.Cm = a->C;
+  p.A = a->A;
+  p.D = a->D;
+  p.dt_bias = a->dt_bias;
+  p.h0 = a->state_io;
+  p.y = a->y;
+  p.h_last = a->state_io;
+  p.states = nullptr;
+  return from_cuda(ssm::launch_m2_recurrent(p, s));
+}
+
+}  // extern "C"

@@ -1,0 +1,180 @@
+"""Python binding of libssm: the three C-ABI calls, same names, torch tensors in.
+
+Argument marshalling only: shapes are read off the tensors, outputs and the
+workspace are allocated with torch (device memory), and the call is queued
+on the current torch stream.  Every step of the scan runs in the library's
+CUDA kernels; if ``libssm.so`` is missing these functions raise.
+
+Host tensors are accepted too: they are copied to the GPU on the current
+stream, the call runs there, the outputs are copied back into host tensors
+(pinned when the inputs were pinned) and the stream is synchronised before
+returning.  This is the end-to-end path a caller with host buffers uses.
+"""
+import ctypes
+
+import torch
+
+from . import _lib as L
+
+SOFTPLUS = L.SSM_DT_SOFTPLUS
+RMS_BC = L.SSM_RMSNORM_BC
+RMS_DT = L.SSM_RMSNORM_DT
+
+_IO = {torch.float32: L.SSM_F32, torch.bfloat16: L.SSM_BF16}
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream, device):
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+class _Staging:
+    """Moves host inputs to the device and device outputs back, on one stream."""
+
+    def __init__(self, tensors):
+        firsts = [t for t in tensors if t is not None]
+        self.host = firsts[0].device.type == "cpu"
+        self.pinned = self.host and firsts[0].is_pinned()
+        self.device = torch.device("cuda", torch.cuda.current_device()) if self.host \
+            else firsts[0].device
+
+    def dev(self, t):
+        if t is None:
+            return None
+        if self.host:
+            return t.contiguous().to(self.device, non_blocking=self.pinned)
+        return t.contiguous()
+
+    def back(self, outs):
+        if not self.host:
+            return outs
+        res = []
+        for t in outs:
+            if t is None:
+                res.append(None)
+                continue
+            h = torch.empty(t.shape, dtype=t.dtype, pin_memory=self.pinned)
+            h.copy_(t, non_blocking=self.pinned)
+            res.append(h)
+        torch.cuda.current_stream(self.device).synchronize()
+        return tuple(res)
+
+
+def _io_of(x):
+    if x.dtype not in _IO:
+        raise TypeError("io dtype must be float32 or bfloat16, got %s" % x.dtype)
+    return _IO[x.dtype]
+
+
+def ssm_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
+                 flags=SOFTPLUS, rms_eps=1e-6, want_states=False, y=None, h_last=None,
+                 stream=None):
+    """Mamba-1 selective scan (include/ssm.h, ssm_scan_fwd).
+
+    x, dt, z: [b, L, C]; B, C: [b, L, G, N]; A: [C, N] f32; D, dt_bias: [C] f32;
+    h0: [b, C, N] f32.  Returns (y [b, L, C], h_last [b, C, N] f32,
+    states [b, L, C, N] f32 or None)."""
+    sg = _Staging([x, dt, A, B, C, D, z, dt_bias, h0])
+    x, dt, A, B, C, D, z, dt_bias, h0 = map(sg.dev, (x, dt, A, B, C, D, z, dt_bias, h0))
+    b, Lq, Cn = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if y is None:
+        y = torch.empty_like(x)
+    if h_last is None:
+        h_last = torch.empty((b, Cn, N), dtype=torch.float32, device=x.device)
+    states = (torch.empty((b, Lq, Cn, N), dtype=torch.float32, device=x.device)
+              if want_states else None)
+    a = L.ScanArgs(batch=b, seqlen=Lq, channels=Cn, state=N, groups=G, io=_io_of(x),
+                   flags=flags, rms_eps=rms_eps, x=_ptr(x), dt=_ptr(dt), z=_ptr(z),
+                   B=_ptr(B), C=_ptr(C), A=_ptr(A), D=_ptr(D), dt_bias=_ptr(dt_bias),
+                   h0=_ptr(h0), y=_ptr(y), h_last=_ptr(h_last), states=_ptr(states))
+    lib = L.lib()
+    nbytes = ctypes.c_size_t(0)
+    L.check(lib.ssm_scan_workspace(ctypes.byref(a), ctypes.byref(nbytes)), "ssm_scan_workspace")
+    ws = None
+    if nbytes.value:
+        ws = torch.empty(nbytes.value, dtype=torch.uint8, device=x.device)
+        a.workspace, a.workspace_bytes = ws.data_ptr(), nbytes.value
+    L.check(lib.ssm_scan_fwd(ctypes.byref(a), _stream(stream, x.device)), "ssm_scan_fwd")
+    return sg.back((y, h_last, states))
+
+
+def ssd_workspace_bytes(**shape):
+    a = L.SsdArgs(**shape)
+    n = ctypes.c_size_t(0)
+    L.check(L.lib().ssd_chunk_scan_workspace(ctypes.byref(a), ctypes.byref(n)),
+            "ssd_chunk_scan_workspace")
+    return n.value
+
+
+def ssd_chunk_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
+                       chunk=256, flags=SOFTPLUS, want_states=False, y=None, h_last=None,
+                       workspace=None, stream=None):
+    """Mamba-2 SSD scan (include/ssm.h, ssd_chunk_scan_fwd).
+
+    x, z: [b, L, H, P]; dt: [b, L, H]; B, C: [b, L, G, N]; A, D, dt_bias: [H] f32;
+    h0: [b, H, N, P] f32.  Returns (y, h_last [b, H, N, P], states or None)."""
+    sg = _Staging([x, dt, A, B, C, D, z, dt_bias, h0])
+    x, dt, A, B, C, D, z, dt_bias, h0 = map(sg.dev, (x, dt, A, B, C, D, z, dt_bias, h0))
+    b, Lq, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if y is None:
+        y = torch.empty_like(x)
+    if h_last is None:
+        h_last = torch.empty((b, H, N, P), dtype=torch.float32, device=x.device)
+    states = (torch.empty((b, Lq, H, N, P), dtype=torch.float32, device=x.device)
+              if want_states else None)
+    a = L.SsdArgs(batch=b, seqlen=Lq, heads=H, head_dim=P, state=N, groups=G, chunk=chunk,
+                  io=_io_of(x), flags=flags, x=_ptr(x), z=_ptr(z), dt=_ptr(dt), B=_ptr(B),
+                  C=_ptr(C), A=_ptr(A), D=_ptr(D), dt_bias=_ptr(dt_bias), h0=_ptr(h0),
+                  y=_ptr(y), h_last=_ptr(h_last), states=_ptr(states))
+    lib = L.lib()
+    nbytes = ctypes.c_size_t(0)
+    L.check(lib.ssd_chunk_scan_workspace(ctypes.byref(a), ctypes.byref(nbytes)),
+            "ssd_chunk_scan_workspace")
+    if nbytes.value:
+        if workspace is None or workspace.numel() * workspace.element_size() < nbytes.value:
+            workspace = torch.empty(nbytes.value, dtype=torch.uint8, device=x.device)
+        a.workspace, a.workspace_bytes = workspace.data_ptr(), nbytes.value
+    L.check(lib.ssd_chunk_scan_fwd(ctypes.byref(a), _stream(stream, x.device)),
+            "ssd_chunk_scan_fwd")
+    return sg.back((y, h_last, states))
+
+
+def ssm_scan_step(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, *, flags=SOFTPLUS,
+                  rms_eps=1e-6, y=None, stream=None):
+    """One decode token (include/ssm.h, ssm_scan_step); ``state`` is updated in place.
+
+    Mamba-1: state [b, C, N], x/dt/z [b, C], B/C [b, G, N], A [C, N].
+    Mamba-2: state [b, H, N, P], x/z [b, H, P], dt [b, H], B/C [b, G, N], A [H].
+    Returns y (and, for host tensors, the updated state copied back)."""
+    if state.dim() == 3:
+        kind, (b, U, N), P = L.SSM_STEP_MAMBA1, state.shape, 1
+    elif state.dim() == 4:
+        kind, (b, U, N, P) = L.SSM_STEP_MAMBA2, state.shape
+    else:
+        raise ValueError("state must be [b, C, N] or [b, H, N, P]")
+    sg = _Staging([state, x, dt, A, B, C, D, z, dt_bias])
+    host_state = state
+    state = state if not sg.host else state.contiguous().to(sg.device, non_blocking=sg.pinned)
+    if not state.is_contiguous():
+        raise ValueError("state must be contiguous (it is updated in place)")
+    x, dt, A, B, C, D, z, dt_bias = map(sg.dev, (x, dt, A, B, C, D, z, dt_bias))
+    G = B.shape[1]
+    if y is None:
+        y = torch.empty_like(x)
+    a = L.StepArgs(kind=kind, io=_io_of(x), flags=flags, rms_eps=rms_eps, batch=b, units=U,
+                   head_dim=P, state=N, groups=G, x=_ptr(x), dt=_ptr(dt), z=_ptr(z),
+                   B=_ptr(B), C=_ptr(C), A=_ptr(A), D=_ptr(D), dt_bias=_ptr(dt_bias),
+                   state_io=_ptr(state), y=_ptr(y))
+    L.check(L.lib().ssm_scan_step(ctypes.byref(a), _stream(stream, x.device)), "ssm_scan_step")
+    if sg.host:
+        y_h, st_h = sg.back((y, state))
+        host_state.copy_(st_h)
+        return y_h
+    return y

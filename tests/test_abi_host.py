@@ -1,0 +1,145 @@
+"""Host-only checks of the C ABI: the library loads, exports every function
+include/ssm.h declares, and rejects bad arguments with the documented status
+before launching anything.  No call here reaches a kernel, so these run
+without a GPU; fake device addresses are never dereferenced."""
+import ctypes
+import subprocess
+
+import pytest
+
+from selective_state_space_28_b200 import _lib as L
+from selective_state_space_28_b200 import build as B
+
+OK, NULL, SHAPE, DTYPE, ALIGN, UNSUP, WS = 0, 1, 2, 3, 4, 5, 6
+P = 0x7f0000001000  # a 16-byte-aligned fake device address
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = L.header_functions()
+    assert {"ssm_scan_fwd", "ssm_scan_workspace", "ssd_chunk_scan_fwd",
+            "ssd_chunk_scan_workspace", "ssm_scan_step", "ssm_status_string",
+            "ssm_abi_version"} <= set(names)
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], check=True,
+                         capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert getattr(lib, n) is not None
+
+
+def test_no_runtime_symbols_leak(lib):
+    """The static CUDA runtime stays private to the library."""
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], check=True,
+                         capture_output=True, text=True).stdout
+    assert not [l for l in out.splitlines() if " cuda" in l and " T " in l]
+
+
+def test_version_and_strings(lib):
+    assert lib.ssm_abi_version() == 1
+    for s in range(9):
+        assert lib.ssm_status_string(s)
+    assert lib.ssm_status_string(99) == b"unknown status"
+
+
+def _scan(**kw):
+    d = dict(batch=2, seqlen=8, channels=64, state=16, groups=1, io=1, flags=1,
+             rms_eps=1e-6, x=P, dt=P, z=None, B=P, C=P, A=P, D=None, dt_bias=None,
+             h0=None, y=P, h_last=None, states=None)
+    d.update(kw)
+    return L.ScanArgs(**d)
+
+
+def _call_scan(lib, a):
+    return lib.ssm_scan_fwd(ctypes.byref(a), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), NULL), (dict(dt=None), NULL), (dict(B=None), NULL), (dict(A=None), NULL),
+    (dict(y=None), NULL), (dict(io=7), DTYPE), (dict(channels=0), SHAPE),
+    (dict(state=0), SHAPE), (dict(batch=-1), SHAPE), (dict(groups=3), SHAPE),
+    (dict(groups=0), SHAPE), (dict(x=P + 2), ALIGN), (dict(h_last=P + 8), ALIGN),
+    (dict(state=12), UNSUP), (dict(state=128), UNSUP), (dict(flags=8), UNSUP),
+    (dict(groups=2, channels=48), UNSUP), (dict(batch=70000), UNSUP),
+    (dict(flags=5), WS), (dict(flags=3, rms_eps=-1.0), SHAPE),
+])
+def test_scan_rejects(lib, kw, status):
+    assert _call_scan(lib, _scan(**kw)) == status
+
+
+def test_scan_null_args(lib):
+    assert lib.ssm_scan_fwd(None, None) == NULL
+    n = ctypes.c_size_t(0)
+    assert lib.ssm_scan_workspace(None, ctypes.byref(n)) == NULL
+    assert lib.ssm_scan_workspace(ctypes.byref(_scan()), None) == NULL
+
+
+def test_scan_workspace_sizes(lib):
+    n = ctypes.c_size_t(123)
+    assert lib.ssm_scan_workspace(ctypes.byref(_scan()), ctypes.byref(n)) == OK
+    assert n.value == 0
+    assert lib.ssm_scan_workspace(ctypes.byref(_scan(flags=5)), ctypes.byref(n)) == OK
+    assert n.value == 2 * 8 * 4
+    a = _scan(flags=5, workspace=P, workspace_bytes=63)
+    assert _call_scan(lib, a) == WS
+
+
+def test_scan_empty_batch_is_a_no_op(lib):
+    # batch 0: nothing to do, nothing launched, even with NULL tensors
+    assert _call_scan(lib, _scan(batch=0, x=None, dt=None, B=None, C=None, A=None,
+                                 y=None)) == OK
+
+
+def _ssd(**kw):
+    d = dict(batch=1, seqlen=64, heads=4, head_dim=64, state=128, groups=1, chunk=256,
+             io=1, flags=1, x=P, z=None, dt=P, B=P, C=P, A=P, D=None, dt_bias=None,
+             h0=None, y=P, h_last=None, states=None)
+    d.update(kw)
+    return L.SsdArgs(**d)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), NULL), (dict(C=None), NULL), (dict(io=2), DTYPE), (dict(heads=0), SHAPE),
+    (dict(groups=3), SHAPE), (dict(chunk=0), SHAPE), (dict(head_dim=6), UNSUP),
+    (dict(flags=2), UNSUP), (dict(B=P + 4), ALIGN), (dict(batch=70000), UNSUP),
+])
+def test_ssd_rejects(lib, kw, status):
+    assert lib.ssd_chunk_scan_fwd(ctypes.byref(_ssd(**kw)), None) == status
+
+
+def _step(**kw):
+    d = dict(kind=2, io=1, flags=1, rms_eps=1e-6, batch=4, units=8, head_dim=64, state=128,
+             groups=1, x=P, dt=P, z=None, B=P, C=P, A=P, D=None, dt_bias=None, state_io=P,
+             y=P)
+    d.update(kw)
+    return L.StepArgs(**d)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(state_io=None), NULL), (dict(y=None), NULL), (dict(kind=3), UNSUP),
+    (dict(io=5), DTYPE), (dict(units=0), SHAPE), (dict(kind=1, head_dim=2), SHAPE),
+    (dict(kind=1, head_dim=1, state=12), UNSUP), (dict(flags=4), UNSUP),
+    (dict(kind=2, flags=2), UNSUP), (dict(x=P + 1), ALIGN), (dict(groups=3), SHAPE),
+])
+def test_step_rejects(lib, kw, status):
+    assert lib.ssm_scan_step(ctypes.byref(_step(**kw)), None) == status
+
+
+def test_step_empty_batch_is_a_no_op(lib):
+    assert lib.ssm_scan_step(ctypes.byref(_step(batch=0, x=None, dt=None, B=None, C=None,
+                                                A=None, state_io=None, y=None)), None) == OK
+
+
+def test_workspace_queries_need_no_pointers(lib):
+    n = ctypes.c_size_t(7)
+    a = _scan(x=None, dt=None, B=None, C=None, A=None, y=None, flags=5)
+    assert lib.ssm_scan_workspace(ctypes.byref(a), ctypes.byref(n)) == OK
+    assert n.value == 2 * 8 * 4
+    s = _ssd(x=None, dt=None, B=None, C=None, A=None, y=None)
+    assert lib.ssd_chunk_scan_workspace(ctypes.byref(s), ctypes.byref(n)) == OK
