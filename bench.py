@@ -227,16 +227,19 @@ def timed(step, K, W, dist, device):
 
 
 def per_launch_ms(step, n, device):
-    """Average device time of one step measured by an event pair around each."""
+    """Average device time of one step: n steps queued back to back between
+    one event pair (the host enqueues faster than the GPU drains them)."""
     import torch
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(n)]
-    for i, (a, b) in enumerate(evs):
-        a.record()
-        step(i)
-        b.record()
+    step(0)
     torch.cuda.synchronize(device)
-    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(n):
+        step(i)
+    b.record()
+    torch.cuda.synchronize(device)
+    return a.elapsed_time(b) / n
 
 
 def n_sets(bytes_per_set):
@@ -263,7 +266,7 @@ def bench_m1(w, K, W, dist, device, pk, seed_base):
                          dt_bias=d["dt_bias"], flags=w.flags, rms_eps=w.rms_eps,
                          y=d["y"], h_last=d["h_last"])
     ms = timed(step, K, W, dist, device) / K
-    launch_ms = per_launch_ms(step, max(5, min(K, 20)), device)
+    launch_ms = per_launch_ms(step, max(10, K), device)
     launches = 2 if (w.flags & I.RMS_DT) else 1
     return {"ms_per_step": ms, "bytes": nb, "launch_ms": launch_ms, "sets": len(sets),
             "launches_per_step": launches}
@@ -291,7 +294,7 @@ def bench_ssd(w, K, W, dist, device, pk, seed_base):
                                dt_bias=d["dt_bias"], chunk=w.chunk, flags=w.flags,
                                y=d["y"], h_last=d["h_last"], workspace=wsb)
     ms = timed(step, K, W, dist, device) / K
-    launch_ms = per_launch_ms(step, max(3, min(K, 10)), device)
+    launch_ms = per_launch_ms(step, max(5, K), device)
     return {"ms_per_step": ms, "bytes": nb, "flops": ssd_flops(w), "launch_ms": launch_ms,
             "tokens": w.batch * w.seqlen, "sets": len(sets), "launches_per_step": 1}
 
@@ -321,7 +324,8 @@ def bench_decode(w, K, W, dist, device, pk, seed_base):
         for d in m1_layers:
             one(d)
     ms = timed(step, K, W, dist, device) / K
-    m2_ms = per_launch_ms(lambda i: one(m2_layers[i % len(m2_layers)]), 16, device)
+    m2_ms = per_launch_ms(lambda i: one(m2_layers[i % len(m2_layers)]), 2 * len(m2_layers),
+                          device)
     return {"ms_per_step": ms, "bytes": total, "launch_ms": m2_ms, "launch_bytes": m2b,
             "launches_per_step": w.layers + w.m1_layers}
 
@@ -355,24 +359,26 @@ def e2e_m1(w, device, n_steps=5):
     return {"ms": ms, "h2d": h2d, "d2h": d2h}
 
 
-def cpu_baseline_m1(w, rows=1):
-    """The oracle, as it stands, on a bounded sample: `rows` batch rows of the
-    workload, all channels and tokens, on every host core it may use."""
+def cpu_baseline_m1(w, min_seconds=10.0):
+    """The oracle, as it stands, on a bounded sample of the workload: whole
+    passes over all batch rows, repeated until about `min_seconds` of CPU
+    time, on every host core the process may use."""
     import oracle
     from selective_state_space_28_b200 import inputs as I
     d = I.workload_inputs(w, device="cpu")
-    sub = {k: (v[:rows] if (v is not None and k in ("x", "dt", "z", "B", "C")) else v)
-           for k, v in d.items()}
     threads = oracle.default_threads()
-    t0 = time.perf_counter()
-    oracle.m1_scan(sub["x"], sub["dt"], sub["B"], sub["C"], sub["A"], sub["D"], z=sub["z"],
-                   dt_bias=sub["dt_bias"], flags=w.flags, rms_eps=w.rms_eps, nthreads=threads)
-    sec = time.perf_counter() - t0
-    frac = rows / w.batch
-    gbs = m1_bytes(w) * frac / sec / 1e9
+    passes, sec = 0, 0.0
+    while sec < min_seconds and passes < 50:
+        t0 = time.perf_counter()
+        oracle.m1_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                       dt_bias=d["dt_bias"], flags=w.flags, rms_eps=w.rms_eps,
+                       nthreads=threads)
+        sec += time.perf_counter() - t0
+        passes += 1
+    gbs = m1_bytes(w) * passes / sec / 1e9
     return {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": "%d of %d batch rows of %s (all %d tokens x %d channels x state %d), "
-                      "float64 C token loop, %.2f s" % (rows, w.batch, w.name, w.seqlen,
+            "sample": "%d full pass(es) of %s (batch %d x %d tokens x %d channels x state %d), "
+                      "float64 C token loop, %.1f s" % (passes, w.name, w.batch, w.seqlen,
                                                         w.channels, w.state, sec)}
 
 

@@ -17,6 +17,9 @@ struct M1Params {
   void *y;
   float *h_last, *states;
   float *rstd;  // [batch * L] RMS factors of dt rows, or nullptr
+  int swx;      // states per lane (of 4) whose decay uses the FMA-pipe exp2
+  int pipelined;  // use the TMA-pipelined kernel where the shape allows
+  int *status;  // device word set non-zero if a bounded wait ran out, or nullptr
 };
 
 // Mamba-2 token recurrence (the decode step, and the SSD path for shapes the
@@ -47,9 +50,15 @@ struct M1StepParams {
 // kernel (checked before any launch), or the launch error.
 cudaError_t launch_m1_scan(const M1Params &p, cudaStream_t s);
 bool m1_scan_supported(int64_t N, int64_t C, int64_t G);
+bool m1_scan_tma_supported(const M1Params &p);
+cudaError_t launch_m1_scan_tma(const M1Params &p, cudaStream_t s);
 cudaError_t launch_m2_recurrent(const M2Params &p, cudaStream_t s);
 bool m2_recurrent_supported(int64_t N, int64_t P);
 cudaError_t launch_m1_step(const M1StepParams &p, cudaStream_t s);
 bool m1_step_supported(int64_t N);
+// Tensor-core SSD (bf16 I/O, state 128, head dim 64, no per-token states).
+// `status` is a device word the kernel sets non-zero if a bounded wait ran out.
+bool ssd_tc_supported(const M2Params &p);
+cudaError_t launch_ssd_tc(const M2Params &p, int *status, cudaStream_t s);
 
 }  // namespace ssm

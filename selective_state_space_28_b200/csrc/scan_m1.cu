@@ -1,4 +1,6 @@
-// scan_m1.cu -- Mamba-1 selective scan (kernel a).
+// scan_m1.cu -- Mamba-1 selective scan (kernel a): the generic form, used for
+// shapes the pipelined form (scan_m1_tma.cu) cannot tile, and the pre-pass
+// for the step-input RMS norm.
 //
 // Computes, per batch b, channel c and token t ("Mamba", nnterp guide, intro
 // and "The values"; "Mamba", tokentrails, "Code"):
@@ -184,6 +186,7 @@ cudaError_t launch_t(const M1Params &p, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  if (p.pipelined && m1_scan_tma_supported(p)) return launch_m1_scan_tma(p, s);
   switch (p.N) {
     case 4: return launch_n<4, T>(p, s);
     case 8: return launch_n<8, T>(p, s);

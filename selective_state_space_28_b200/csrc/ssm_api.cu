@@ -2,6 +2,7 @@
 // the host, then dispatch to the kernels.  Nothing is launched when a check
 // fails, and nothing here allocates memory.
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "internal.h"
@@ -18,6 +19,29 @@ bool all_aligned(Ps... ps) {
   for (const void *p : arr)
     if (p && !aligned16(p)) return false;
   return true;
+}
+
+// How many of the 4 states per lane take their decay from the FMA-pipe
+// exponential instead of the SFU (0, 1 or 2); SSM_M1_EXP_SPLIT overrides the
+// default for tuning.
+int m1_exp_split() {
+  static int v = -1;
+  if (v < 0) {
+    const char *e = getenv("SSM_M1_EXP_SPLIT");
+    v = (e && e[0] >= '0' && e[0] <= '2') ? e[0] - '0' : 1;
+  }
+  return v;
+}
+
+// The TMA-pipelined Mamba-1 kernel is opt-in (SSM_M1_PIPELINED=1) until it
+// has been validated on hardware.
+int m1_pipelined() {
+  static int v = -1;
+  if (v < 0) {
+    const char *e = getenv("SSM_M1_PIPELINED");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v;
 }
 
 ssm_status_t from_cuda(cudaError_t e) {
@@ -59,6 +83,34 @@ ssm_status_t check_scan(const ssm_scan_args_t *a, size_t *ws, bool shapes_only =
   return SSM_OK;
 }
 
+// The tensor-core SSD path keeps a device status word in the workspace.
+constexpr size_t kSsdStatusBytes = 256;
+
+ssm::M2Params ssd_params(const ssd_scan_args_t *a) {
+  ssm::M2Params p;
+  p.batch = a->batch;
+  p.L = a->seqlen;
+  p.H = a->heads;
+  p.P = a->head_dim;
+  p.N = a->state;
+  p.G = a->groups;
+  p.flags = a->flags;
+  p.io = a->io;
+  p.x = a->x;
+  p.z = a->z;
+  p.dt = a->dt;
+  p.B = a->B;
+  p.Cm = a->C;
+  p.A = a->A;
+  p.D = a->D;
+  p.dt_bias = a->dt_bias;
+  p.h0 = a->h0;
+  p.y = a->y;
+  p.h_last = a->h_last;
+  p.states = a->states;
+  return p;
+}
+
 ssm_status_t check_ssd(const ssd_scan_args_t *a, size_t *ws, bool shapes_only = false) {
   if (!a) return SSM_ERR_NULL;
   if (a->io != SSM_F32 && a->io != SSM_BF16) return SSM_ERR_DTYPE;
@@ -75,7 +127,7 @@ ssm_status_t check_ssd(const ssd_scan_args_t *a, size_t *ws, bool shapes_only = 
     return SSM_ERR_ALIGN;
   if (!ssm::m2_recurrent_supported(a->state, a->head_dim) || a->batch > 65535)
     return SSM_ERR_UNSUPPORTED;
-  *ws = 0;
+  *ws = ssm::ssd_tc_supported(ssd_params(a)) ? kSsdStatusBytes : 0;
   return SSM_OK;
 }
 
@@ -140,6 +192,9 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_args_t *a, void *stream) {
   p.h_last = a->h_last;
   p.states = a->states;
   p.rstd = (a->flags & SSM_RMSNORM_DT) ? static_cast<float *>(a->workspace) : nullptr;
+  p.swx = m1_exp_split();
+  p.pipelined = m1_pipelined();
+  p.status = nullptr;
   return from_cuda(ssm::launch_m1_scan(p, s));
 }
 
@@ -162,27 +217,12 @@ ssm_status_t ssd_chunk_scan_fwd(const ssd_scan_args_t *a, void *stream) {
     return pass_state(a->h0, a->h_last,
                       (size_t)(a->batch * a->heads * a->state * a->head_dim) * sizeof(float),
                       s);
-  ssm::M2Params p;
-  p.batch = a->batch;
-  p.L = a->seqlen;
-  p.H = a->heads;
-  p.P = a->head_dim;
-  p.N = a->state;
-  p.G = a->groups;
-  p.flags = a->flags;
-  p.io = a->io;
-  p.x = a->x;
-  p.z = a->z;
-  p.dt = a->dt;
-  p.B = a->B;
-  p.Cm = a->C;
-  p.A = a->A;
-  p.D = a->D;
-  p.dt_bias = a->dt_bias;
-  p.h0 = a->h0;
-  p.y = a->y;
-  p.h_last = a->h_last;
-  p.states = a->states;
+  const ssm::M2Params p = ssd_params(a);
+  if (ssm::ssd_tc_supported(p)) {
+    int *status = static_cast<int *>(a->workspace);
+    if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return SSM_ERR_CUDA;
+    return from_cuda(ssm::launch_ssd_tc(p, status, s));
+  }
   return from_cuda(ssm::launch_m2_recurrent(p, s));
 }
 

@@ -108,3 +108,16 @@ def test_2p7b_full_size_sampled(cuda_ok):
     hsel = torch.tensor(hs).cuda()
     assert_close_normwise(y[rows][:, :, hsel], ref[0], REL[torch.bfloat16], "y")
     assert_close_normwise(h[rows][:, hsel], ref[1], REL[torch.bfloat16], "h_last")
+
+
+def test_ssd_status_word_clear(cuda_ok):
+    """The tensor-core path reports bounded-wait timeouts in the first word of
+    its workspace; a normal call leaves it zero."""
+    ops = _ops()
+    d = I.ssd_inputs(2, 300, 3, 64, 128, io="bf16", seed=9, h0=True)
+    dv = {k: (v.cuda() if v is not None else None) for k, v in d.items()}
+    ws = torch.full((256,), 7, dtype=torch.uint8, device="cuda")
+    ops.ssd_chunk_scan_fwd(dv["x"], dv["dt"], dv["A"], dv["B"], dv["C"], D=dv["D"],
+                           dt_bias=dv["dt_bias"], h0=dv["h0"], workspace=ws)
+    torch.cuda.synchronize()
+    assert ws[:4].view(torch.int32).item() == 0
