@@ -111,6 +111,29 @@ typedef struct ssm_scan_args {
 ssm_status_t ssm_scan_workspace(const ssm_scan_args_t *args, size_t *bytes);
 ssm_status_t ssm_scan_fwd(const ssm_scan_args_t *args, void *stream);
 
+/* ssm_scan_fwd_static -- ssm_scan_fwd without a caller-provided workspace.
+ *
+ * The pages have no counterpart: this is a deployment variant.  Some callers
+ * cannot allocate device memory where they run the scan -- an engine's
+ * enqueue callback that may only use memory reserved up front, a decode loop
+ * with a latency budget that must not meet an allocator that can
+ * synchronise the device, a process whose device memory another component
+ * has reserved.  With SSM_RMSNORM_DT, ssm_scan_fwd needs a workspace of
+ * batch * seqlen floats; this entry point uses a fixed array in the
+ * library's own device memory instead (static, 1 MiB per GPU, held until the
+ * process exits), so the caller passes only inputs and outputs.
+ *
+ * Arguments, layouts, results and errors are those of ssm_scan_fwd;
+ * args->workspace is ignored.  Limit: with SSM_RMSNORM_DT, batch * seqlen
+ * must not exceed 262144; larger problems return SSM_ERR_WORKSPACE before
+ * anything touches the device.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  All calls share the
+ * array, which keeps the last call's contents (nothing in it needs to start
+ * at zero); calls that overlap on the GPU -- on different streams, or from
+ * several threads -- race on it and must be serialised by the caller. */
+ssm_status_t ssm_scan_fwd_static(const ssm_scan_args_t *args, void *stream);
+
 /* ------------------------------------------------------------------------
  * ssd_chunk_scan_fwd -- Mamba-2 (SSD) scan.
  *
