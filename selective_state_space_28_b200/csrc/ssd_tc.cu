@@ -15,12 +15,17 @@
 // 256-token masked form, up to rounding.
 //
 // One CTA (4 warps, 128 threads) owns one (batch, head) and walks the tiles in
-// order.  Per tile, TMA brings C and B ([128 x 128] bf16, two 64-column slabs,
-// 128-byte swizzle) and x ([128 x 64]) into a double-buffered stage; four
-// tcgen05 MMAs (bf16 in, fp32 accumulate in TMEM) do the contractions:
+// order; two CTAs share an SM (256 TMEM columns and ~100 KB of shared memory
+// each), so one's tensor-core work overlaps the other's elementwise work.
+// Per tile, TMA brings C and B ([128 x 128] bf16, two 64-column slabs,
+// 128-byte swizzle) and x ([128 x 64]); the next tile's C is fetched as soon
+// as this tile's MMAs on C finish, B and x as soon as the state MMA
+// finishes.  Four tcgen05 MMAs (bf16 in, fp32 accumulate in TMEM) do the
+// contractions:
 //   S   = C B^T                 [128 x 128]   A, B K-major from shared memory
 //   Yd  = (S o mask) x          [128 x 64]    A = masked S, bf16, from TMEM
-//   Sc  = B^T (w o x)           [128 x 64]    A = B read MN-major, B = scaled x
+//   Sc  = B^T (w o x)           [128 x 64]    A = B read MN-major, B = x scaled
+//                                             in place once the output is out
 //   Yo  = C h_prev              [128 x 64]    B = bf16 copy of the carried state
 // The mask exp(cum_i - cum_j) d_j is applied elementwise only on the four
 // 32 x 32 diagonal blocks; below them it factors as
@@ -46,21 +51,22 @@ constexpr int kN = 128;   // state size
 constexpr int kP = 64;    // head dim
 constexpr long long kWaitLimit = 2000000000ll;  // cycles (about a second)
 
-// TMEM columns
-constexpr uint32_t kColS = 0, kColM = 128, kColYd = 192, kColYo = 256, kColSc = 320;
+// TMEM columns (256 per CTA, so two CTAs share an SM): the masked S is
+// written over S as it is read, and the tile's state contribution reuses the
+// half of S that is dead by then.
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0, kColM = 0, kColSc = 64, kColYd = 128, kColYo = 192;
 
 struct __align__(1024) SsdSmem {
-  uint8_t C[2][2][kQ * 128];  // [stage][slab]: 128 tokens x 64 state values
-  uint8_t B[2][2][kQ * 128];
-  uint8_t X[2][kQ * 128];     // [stage]: 128 tokens x 64 head values
-  uint8_t Xw[kQ * 128];       // w o x
-  uint8_t Hb[kN * 128];       // bf16 copy of the carried state, rows n
+  uint8_t C[2][kQ * 128];  // [slab]: 128 tokens x 64 state values, 128-byte swizzle
+  uint8_t B[2][kQ * 128];
+  uint8_t X[kQ * 128];     // 128 tokens x 64 head values; later w o x in place
+  uint8_t Hb[kN * 128];    // bf16 copy of the carried state, rows n
   float cum[kQ];
   float dd[kQ];
   float vd[kQ];
   float wsum[4];
-  uint64_t full[2];
-  uint64_t bar_s, bar_so, bar_y;
+  uint64_t full_c, full_bx, bar_s, bar_y, bar_sc;
   uint32_t taddr;
 };
 
@@ -93,7 +99,7 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
                     pack_bf16x2(f[6], f[7]));
 }
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128, 2)
     ssd_tc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mB,
                   const __grid_constant__ CUtensorMap mC, const SsdTcParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -112,18 +118,18 @@ __global__ void __launch_bounds__(128, 1)
   const bool softplus_on = p.flags & 1u;
 
   if (tid == 0) {
-    mbar_init(&s.full[0], 1);
-    mbar_init(&s.full[1], 1);
+    mbar_init(&s.full_c, 1);
+    mbar_init(&s.full_bx, 1);
     mbar_init(&s.bar_s, 1);
-    mbar_init(&s.bar_so, 1);
     mbar_init(&s.bar_y, 1);
+    mbar_init(&s.bar_sc, 1);
     fence_mbar_init();
     tma_prefetch_desc(&mX);
     tma_prefetch_desc(&mB);
     tma_prefetch_desc(&mC);
   }
   if (warp == 0) {
-    tmem_alloc(&s.taddr, 512);
+    tmem_alloc(&s.taddr, kTmemCols);
     tmem_relinquish();
   }
 
@@ -150,37 +156,43 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const uint32_t tb = s.taddr;
 
-  auto issue_loads = [&](int c, int st) {
-    const int t0 = c * kQ;
-    mbar_expect_tx(&s.full[st], 4 * kQ * 128 + kQ * 128);
-    tma_load_3d(s.C[st][0], &mC, &s.full[st], g * kN, t0, (int)b);
-    tma_load_3d(s.C[st][1], &mC, &s.full[st], g * kN + 64, t0, (int)b);
-    tma_load_3d(s.B[st][0], &mB, &s.full[st], g * kN, t0, (int)b);
-    tma_load_3d(s.B[st][1], &mB, &s.full[st], g * kN + 64, t0, (int)b);
-    tma_load_4d(s.X[st], &mX, &s.full[st], 0, (int)hd, t0, (int)b);
+  auto load_c = [&](int c) {
+    mbar_expect_tx(&s.full_c, 2 * kQ * 128);
+    tma_load_3d(s.C[0], &mC, &s.full_c, g * kN, c * kQ, (int)b);
+    tma_load_3d(s.C[1], &mC, &s.full_c, g * kN + 64, c * kQ, (int)b);
+  };
+  auto load_bx = [&](int c) {
+    mbar_expect_tx(&s.full_bx, 3 * kQ * 128);
+    tma_load_3d(s.B[0], &mB, &s.full_bx, g * kN, c * kQ, (int)b);
+    tma_load_3d(s.B[1], &mB, &s.full_bx, g * kN + 64, c * kQ, (int)b);
+    tma_load_4d(s.X, &mX, &s.full_bx, 0, (int)hd, c * kQ, (int)b);
   };
   if (tid == 0) {
-    issue_loads(0, 0);
-    if (nch > 1) issue_loads(1, 1);
+    load_c(0);
+    load_bx(0);
   }
 
   const uint32_t id_S = idesc_bf16_f32(128, 128, false, false);
   const uint32_t id_Y = idesc_bf16_f32(128, 64, false, true);
   const uint32_t id_Sc = idesc_bf16_f32(128, 64, true, true);
 
+  // Raw step of this thread's token, one tile ahead.
+  float dt_next = 0.f;
+  if (tid < L) dt_next = ld(p.dt + (b * L + tid) * H + hd);
+
   bool aborted = false;
   for (int c = 0; c < nch; ++c) {
-    const int st = c & 1;
-    const uint32_t par = c & 1, par_full = (c >> 1) & 1;
+    const uint32_t par = c & 1;
     const int64_t t0 = (int64_t)c * kQ;
     const int valid = (int)(L - t0 < kQ ? L - t0 : kQ);
 
     // ---- step, log2-decay and its inclusive sum over the tile (thread = token)
     float d = 0.f;
     if (tid < valid) {
-      d = ld(p.dt + (b * L + t0 + tid) * H + hd) + bias;
+      d = dt_next + bias;
       if (softplus_on) d = softplus(d);
     }
+    if (t0 + kQ + tid < L) dt_next = ld(p.dt + (b * L + t0 + kQ + tid) * H + hd);
     float cs = d * A2;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -205,46 +217,39 @@ __global__ void __launch_bounds__(128, 1)
     const float w_i = ex2(total - cs) * d;     // weight of token i in the tile's state
     const float a_c = ex2(total);              // decay across the whole tile
 
-    if (!wait_all(&s.full[st], par_full, p.status, 1)) { aborted = true; break; }
-
-    // ---- x scaled by w (row i = token i), the B operand of the state MMA
-#pragma unroll
-    for (int cc = 0; cc < 8; ++cc) {
-      float f[8];
-      unpack8(*reinterpret_cast<const uint4 *>(s.X[st] + sw128(tid, cc)), f);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) f[k] *= w_i;
-      *reinterpret_cast<uint4 *>(s.Xw + sw128(tid, cc)) = pack8(f);
+    // ---- S = C B^T and Yo = C h_prev
+    {
+      const bool ok_c = mbar_wait(&s.full_c, par, kWaitLimit);
+      const bool ok_bx = mbar_wait(&s.full_bx, par, kWaitLimit);
+      if (__syncthreads_or(!(ok_c && ok_bx))) {
+        if (tid == 0 && p.status) atomicExch(p.status, 1);
+        aborted = true;
+        break;
+      }
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t c0 = smem_u32(s.C[st][0]), b0 = smem_u32(s.B[st][0]);
-      const uint32_t xw = smem_u32(s.Xw), hb = smem_u32(s.Hb);
+      const uint32_t c0 = smem_u32(s.C[0]), b0 = smem_u32(s.B[0]), hb = smem_u32(s.Hb);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {  // S = C B^T
+      for (int k = 0; k < 8; ++k) {
         const uint32_t ko = (k >> 2) * (kQ * 128) + (k & 3) * 32;
         mma_ss(tb + kColS, smem_desc(c0 + ko, 16, 1024, kSwizzle128B),
                smem_desc(b0 + ko, 16, 1024, kSwizzle128B), id_S, k > 0);
       }
-      mma_commit(&s.bar_s);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {  // Sc = B^T (w o x);  Yo = C h_prev
+      for (int k = 0; k < 8; ++k) {
         const uint32_t ko = (k >> 2) * (kQ * 128) + (k & 3) * 32;
-        mma_ss(tb + kColSc, smem_desc(b0 + k * 2048, kQ * 128, 1024, kSwizzle128B),
-               smem_desc(xw + k * 2048, kQ * 128, 1024, kSwizzle128B), id_Sc, k > 0);
         mma_ss(tb + kColYo, smem_desc(c0 + ko, 16, 1024, kSwizzle128B),
                smem_desc(hb + k * 2048, kN * 128, 1024, kSwizzle128B), id_Y, k > 0);
       }
-      mma_commit(&s.bar_so);
+      mma_commit(&s.bar_s);
     }
-
-    // ---- masked S -> bf16 A operand in TMEM
     if (!wait_all(&s.bar_s, par, p.status, 2)) { aborted = true; break; }
     tc_fence_after();
+    // C is free: fetch the next tile's C under the rest of this tile.
+    if (tid == 0 && c + 1 < nch) load_c(c + 1);
+
+    // ---- masked S -> bf16 A operand in TMEM, written over S as S is read
     {
       const float cum_i = cs;
 #pragma unroll
@@ -286,36 +291,17 @@ __global__ void __launch_bounds__(128, 1)
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t x0 = smem_u32(s.X[st]);
+      const uint32_t x0 = smem_u32(s.X);
 #pragma unroll
       for (int k = 0; k < 8; ++k)  // Yd = M x
         mma_ts(tb + kColYd, tb + kColM + 8 * k,
                smem_desc(x0 + k * 2048, kQ * 128, 1024, kSwizzle128B), id_Y, k > 0);
       mma_commit(&s.bar_y);
     }
-
-    // ---- carried state: h = a h + Sc  (thread n = row n)
-    if (!wait_all(&s.bar_so, par, p.status, 3)) { aborted = true; break; }
+    if (!wait_all(&s.bar_y, par, p.status, 3)) { aborted = true; break; }
     tc_fence_after();
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint32_t r[16];
-      tmem_ld16(tb + lane_base + kColSc + 16 * q, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int k = 0; k < 16; ++k) h[16 * q + k] = fmaf(a_c, h[16 * q + k], __uint_as_float(r[k]));
-    }
-#pragma unroll
-    for (int cc = 0; cc < 8; ++cc) {
-      float f[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) f[k] = h[8 * cc + k];
-      *reinterpret_cast<uint4 *>(s.Hb + sw128(tid, cc)) = pack8(f);
-    }
 
-    // ---- output: y = Yd + e_i Yo + D x, gate, store (thread i = token i)
-    if (!wait_all(&s.bar_y, par, p.status, 4)) { aborted = true; break; }
-    tc_fence_after();
+    // ---- output y = Yd + e_i Yo + D x (thread i = token i), then w o x in place
     {
       const int64_t row = (b * L + t0 + tid) * H + hd;
 #pragma unroll
@@ -324,9 +310,11 @@ __global__ void __launch_bounds__(128, 1)
         tmem_ld16(tb + lane_base + kColYd + 16 * q, yd);
         tmem_ld16(tb + lane_base + kColYo + 16 * q, yo);
         tmem_ld_wait();
+        uint4 *xp0 = reinterpret_cast<uint4 *>(s.X + sw128(tid, 2 * q));
+        uint4 *xp1 = reinterpret_cast<uint4 *>(s.X + sw128(tid, 2 * q + 1));
         float x0[8], x1[8], o[16];
-        unpack8(*reinterpret_cast<const uint4 *>(s.X[st] + sw128(tid, 2 * q)), x0);
-        unpack8(*reinterpret_cast<const uint4 *>(s.X[st] + sw128(tid, 2 * q + 1)), x1);
+        unpack8(*xp0, x0);
+        unpack8(*xp1, x1);
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
           const float xv = k < 8 ? x0[k] : x1[k - 8];
@@ -354,15 +342,51 @@ __global__ void __launch_bounds__(128, 1)
           yp[0] = pack8(a);
           yp[1] = pack8(bb);
         }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          x0[k] *= w_i;
+          x1[k] *= w_i;
+        }
+        *xp0 = pack8(x0);
+        *xp1 = pack8(x1);
       }
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && c + 2 < nch) {
+    if (tid == 0) {
       tc_fence_after();
-      issue_loads(c + 2, st);
+      const uint32_t b0 = smem_u32(s.B[0]), xw = smem_u32(s.X);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)  // Sc = B^T (w o x)
+        mma_ss(tb + kColSc, smem_desc(b0 + k * 2048, kQ * 128, 1024, kSwizzle128B),
+               smem_desc(xw + k * 2048, kQ * 128, 1024, kSwizzle128B), id_Sc, k > 0);
+      mma_commit(&s.bar_sc);
     }
+    if (!wait_all(&s.bar_sc, par, p.status, 4)) { aborted = true; break; }
+    tc_fence_after();
+    // B and x are free: fetch the next tile's.
+    if (tid == 0 && c + 1 < nch) load_bx(c + 1);
+
+    // ---- carried state: h = a h + Sc  (thread n = row n)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t r[16];
+      tmem_ld16(tb + lane_base + kColSc + 16 * q, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int k = 0; k < 16; ++k) h[16 * q + k] = fmaf(a_c, h[16 * q + k], __uint_as_float(r[k]));
+    }
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+      float f[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) f[k] = h[8 * cc + k];
+      *reinterpret_cast<uint4 *>(s.Hb + sw128(tid, cc)) = pack8(f);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
   }
 
   if (!aborted && p.h_last) {
@@ -374,7 +398,7 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tb, 512);
+  if (warp == 0) tmem_dealloc(tb, kTmemCols);
 }
 
 bool encode(CUtensorMap *m, const void *ptr, int rank, const uint64_t *dims,
