@@ -46,6 +46,8 @@ def parse():
                     help="measure only the headline workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["m1", "ssd", "decode", "decode_layer", "falcon"],
+                    help="run just one workload's timed loop (for profiling); prints its timing")
     return ap.parse_args()
 
 
@@ -382,6 +384,27 @@ def cpu_baseline_m1(w, min_seconds=10.0):
                                                         w.channels, w.state, sec)}
 
 
+def run_only(args):
+    """One workload's warm-up and timed loop, nothing else (used under ncu)."""
+    import torch
+    from selective_state_space_28_b200 import build as B
+    from selective_state_space_28_b200 import inputs as I
+    B.build()
+    dist = Dist()
+    torch.cuda.set_device(dist.local)
+    device = torch.device("cuda", dist.local)
+    pk = peaks()
+    name = {"m1": HEADLINE, "ssd": "ssd_2p7b_b4_l4096_h80_p64_n128_bf16",
+            "decode": "decode_2p7b_stack_b256", "decode_layer": "decode_2p7b_layer_b256",
+            "falcon": "m1_falcon_rms_b4_l8192_c8192_n16_bf16"}[args.only]
+    w = I.WORKLOADS[name]
+    fn = {"m1": bench_m1, "falcon": bench_m1, "ssd": bench_ssd, "decode": bench_decode,
+          "decode_layer": bench_decode}[args.only]
+    r = fn(w, args.steps, args.warmup, dist, device, pk, w.seed)
+    print(json.dumps({"only": name, "ms_per_step": r["ms_per_step"],
+                      "launch_ms": r["launch_ms"]}), flush=True)
+
+
 def run_ours(args):
     import torch
     from selective_state_space_28_b200 import build as B
@@ -525,5 +548,7 @@ if __name__ == "__main__":
     a = parse()
     if a.impl == "reference":
         run_reference(a)
+    elif a.only:
+        run_only(a)
     else:
         run_ours(a)

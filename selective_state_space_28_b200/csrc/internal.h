@@ -17,8 +17,8 @@ struct M1Params {
   void *y;
   float *h_last, *states;
   float *rstd;  // [batch * L] RMS factors of dt rows, or nullptr
-  int swx;      // states per lane (of 4) whose decay uses the FMA-pipe exp2
   int pipelined;  // use the TMA-pipelined kernel where the shape allows
+  int variant;    // pipelined-kernel variant (tuning)
   int *status;  // device word set non-zero if a bounded wait ran out, or nullptr
 };
 

@@ -146,15 +146,34 @@ struct alignas(128) M1Smem {
   uint64_t full[kNS];
 };
 
-template <int N, typename T, int CT, bool HAS_Z, int SWX>
-__global__ void __launch_bounds__(CT *(N / 4))
+// softplus(v) = log(1 + e^v), float32, from the SFU's ex2/lg2: for e^v < 1/32
+// a 4-term series of log1p (relative error below 2e-7), above it lg2(1 + e^v)
+// (the rounding of 1 + e^v then costs at most 2 ulp relative); v > 20 gives v.
+__device__ __forceinline__ float softplus_sfu(float v) {
+  const float u = ex2(v * kLog2e);
+  float lg;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(1.f + u));
+  const float series = u * fmaf(u, fmaf(u, fmaf(u, -0.25f, 0.33333334f), -0.5f), 1.f);
+  const float r = u < 0.03125f ? series : lg * 0.6931471806f;
+  return v > 20.f ? v : r;
+}
+
+// SPL states per lane (2 or 4), G = N / SPL lanes per channel.  SWX of a
+// lane's SPL decays use the FMA-pipe exp2.  STATES: also store every token's
+// state.
+// PK: packed f32x2 state arithmetic (else scalar); UT: token groups per loop
+// iteration (2 lets one group's shuffle reduction overlap the next group's
+// arithmetic).
+template <int N, typename T, int CT, bool HAS_Z, int SWX, int SPL, bool STATES, bool PK, int UT>
+__global__ void __launch_bounds__(CT *(N / SPL))
     m1_scan_tma_kernel(const __grid_constant__ CUtensorMap mx,
                        const __grid_constant__ CUtensorMap mdt,
                        const __grid_constant__ CUtensorMap mz,
                        const __grid_constant__ CUtensorMap mB,
                        const __grid_constant__ CUtensorMap mC, const M1Params p) {
-  constexpr int G = N / 4;  // lanes per channel
+  constexpr int G = N / SPL;  // lanes per channel
   constexpr int NT = CT * G;
+  constexpr int NP = SPL / 2;  // state pairs per lane
   constexpr bool kBF16 = sizeof(T) == 2;
   using S = M1Smem<N, T, CT>;
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -191,20 +210,25 @@ __global__ void __launch_bounds__(CT *(N / 4))
   if (tid == 0)
     for (int i = 0; i < kNS && i < nst; ++i) issue(i);
 
-  float h[4], A2[4], lim[4];
+  float h[SPL], A2[SPL], lim[SPL];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    h[j] = (cvalid && p.h0) ? p.h0[(b * C + c) * N + 4 * q + j] : 0.f;
-    A2[j] = cvalid ? p.A[c * N + 4 * q + j] * kLog2e : 0.f;
+  for (int j = 0; j < SPL; ++j) {
+    h[j] = (cvalid && p.h0) ? p.h0[(b * C + c) * N + SPL * q + j] : 0.f;
+    A2[j] = cvalid ? p.A[c * N + SPL * q + j] * kLog2e : 0.f;
     lim[j] = A2[j] < 0.f ? -127.f / A2[j] : 3.0e38f;
   }
   // The FMA-pipe exponential assumes decays (d >= 0, A < 0); a warp where any
   // of its states could grow uses the SFU for all of them.
   bool sw_ok = softplus_on;
 #pragma unroll
-  for (int j = 4 - SWX; j < 4; ++j) sw_ok = sw_ok && (A2[j] < 0.f || !cvalid);
+  for (int j = SPL - SWX; j < SPL; ++j) sw_ok = sw_ok && (A2[j] < 0.f || !cvalid);
   sw_ok = __all_sync(0xffffffffu, sw_ok);
   const float Dc = (cvalid && p.D) ? p.D[c] : 0.f;
+  // Prologue mapping: this thread always handles column pc of the tile.
+  constexpr int TPR = NT / CT;
+  const int pc = tid % CT, pt0 = tid / CT;
+  const bool pvalid = c0 + pc < C;
+  const float bias_pc = (pvalid && p.dt_bias) ? p.dt_bias[c0 + pc] : 0.f;
 
   for (int sg = 0; sg < nst; ++sg) {
     const int buf = sg % kNS;
@@ -216,17 +240,17 @@ __global__ void __launch_bounds__(CT *(N / 4))
       return;
     }
     // ---- prologue, once per (token, channel) and per (token, B/C row)
-    for (int e = tid; e < kTL * CT; e += NT) {
-      const int t = e / CT, cc = e % CT;
+#pragma unroll 4
+    for (int t = pt0; t < kTL; t += TPR) {
       float dv = 0.f, xv = 0.f;
-      if (t < tn && c0 + cc < C) {
-        xv = ld(&s.x[buf][t][cc]);
-        dv = ld(&s.dt[buf][t][cc]);
+      if (t < tn && pvalid) {
+        xv = ld(&s.x[buf][t][pc]);
+        dv = ld(&s.dt[buf][t][pc]);
         if (p.rstd) dv *= p.rstd[b * L + t0 + t];
-        if (p.dt_bias) dv += p.dt_bias[c0 + cc];
-        if (softplus_on) dv = softplus(dv);
+        dv += bias_pc;
+        if (softplus_on) dv = softplus_sfu(dv);
       }
-      s.ddx[t][cc] = make_float2(dv, dv * xv);
+      s.ddx[t][pc] = make_float2(dv, dv * xv);
     }
     for (int e = tid; e < kTL * 2; e += NT) {
       const int t = e >> 1, which = e & 1;
@@ -246,51 +270,90 @@ __global__ void __launch_bounds__(CT *(N / 4))
     }
     __syncthreads();
 
-    // ---- recurrence, G tokens at a time
+    // ---- recurrence, G tokens at a time, UT groups per iteration
 #pragma unroll 1
-    for (int tg = 0; tg < kTL; tg += G) {
-      float part[G];
+    for (int tg0 = 0; tg0 < kTL; tg0 += G * UT) {
 #pragma unroll
-      for (int u = 0; u < G; ++u) {
-        const int t = tg + u;
-        const float2 ddx = s.ddx[t][cl];
-        const float4 b4 = *reinterpret_cast<const float4 *>(&s.bc[t][0][4 * q]);
-        const float4 c4 = *reinterpret_cast<const float4 *>(&s.bc[t][1][4 * q]);
-        const float d = ddx.x;
-        float a[4];
-        if (SWX == 0 || !sw_ok) {
-          const f2 x01 = mul2(mk2(d, d), mk2(A2[0], A2[1]));
-          const f2 x23 = mul2(mk2(d, d), mk2(A2[2], A2[3]));
-          a[0] = ex2(x01.x); a[1] = ex2(x01.y); a[2] = ex2(x23.x); a[3] = ex2(x23.y);
-        } else if (SWX == 1) {
-          const f2 x01 = mul2(mk2(d, d), mk2(A2[0], A2[1]));
-          a[0] = ex2(x01.x); a[1] = ex2(x01.y); a[2] = ex2(d * A2[2]);
-          a[3] = exp2_fma1(d, A2[3], lim[3]);
-        } else {
-          const f2 x01 = mul2(mk2(d, d), mk2(A2[0], A2[1]));
-          a[0] = ex2(x01.x); a[1] = ex2(x01.y);
-          const f2 a23 = exp2_fma2(d, mk2(A2[2], A2[3]), mk2(lim[2], lim[3]));
-          a[2] = a23.x; a[3] = a23.y;
+      for (int ug = 0; ug < UT; ++ug) {
+        const int tg = tg0 + ug * G;
+        float part[G];
+#pragma unroll
+        for (int u = 0; u < G; ++u) {
+          const int t = tg + u;
+          const float2 ddx = s.ddx[t][cl];
+          const float d = ddx.x, dx = ddx.y;
+          float bv[SPL], cv[SPL], a[SPL];
+          if constexpr (SPL == 4) {
+            const float4 b4 = *reinterpret_cast<const float4 *>(&s.bc[t][0][4 * q]);
+            const float4 c4 = *reinterpret_cast<const float4 *>(&s.bc[t][1][4 * q]);
+            bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
+            cv[0] = c4.x; cv[1] = c4.y; cv[2] = c4.z; cv[3] = c4.w;
+          } else {
+            const float2 b2 = *reinterpret_cast<const float2 *>(&s.bc[t][0][2 * q]);
+            const float2 c2 = *reinterpret_cast<const float2 *>(&s.bc[t][1][2 * q]);
+            bv[0] = b2.x; bv[1] = b2.y;
+            cv[0] = c2.x; cv[1] = c2.y;
+          }
+          if constexpr (PK) {
+#pragma unroll
+            for (int pr = 0; pr < NP; ++pr) {
+              const bool fma_pair = (SWX == 2 && SPL == 4 && pr == 1) && sw_ok;
+              const bool fma_last = (SWX == 1 && pr == NP - 1) && sw_ok;
+              if (fma_pair) {
+                const f2 e = exp2_fma2(d, mk2(A2[2], A2[3]), mk2(lim[2], lim[3]));
+                a[2] = e.x; a[3] = e.y;
+              } else {
+                const f2 xx = mul2(mk2(d, d), mk2(A2[2 * pr], A2[2 * pr + 1]));
+                a[2 * pr] = ex2(xx.x);
+                a[2 * pr + 1] =
+                    fma_last ? exp2_fma1(d, A2[2 * pr + 1], lim[2 * pr + 1]) : ex2(xx.y);
+              }
+            }
+            const f2 dx2 = mk2(dx, dx);
+            f2 yacc = mk2(0.f, 0.f);
+#pragma unroll
+            for (int pr = 0; pr < NP; ++pr) {
+              const f2 hn = fma2(mk2(a[2 * pr], a[2 * pr + 1]), mk2(h[2 * pr], h[2 * pr + 1]),
+                                 mul2(dx2, mk2(bv[2 * pr], bv[2 * pr + 1])));
+              h[2 * pr] = hn.x;
+              h[2 * pr + 1] = hn.y;
+              yacc = fma2(mk2(cv[2 * pr], cv[2 * pr + 1]), hn, yacc);
+            }
+            part[u] = yacc.x + yacc.y;
+          } else {
+#pragma unroll
+            for (int j = 0; j < SPL; ++j) {
+              const bool fma_j = (j >= SPL - SWX) && sw_ok;
+              a[j] = fma_j ? exp2_fma1(d, A2[j], lim[j]) : ex2(d * A2[j]);
+            }
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < SPL; ++j) {
+              h[j] = fmaf(a[j], h[j], dx * bv[j]);
+              acc = fmaf(cv[j], h[j], acc);
+            }
+            part[u] = acc;
+          }
+          if constexpr (STATES) {
+            if (cvalid && t < tn) {
+              float *sp = p.states + ((b * L + t0 + t) * C + c) * N + SPL * q;
+              if constexpr (SPL == 4)
+                *reinterpret_cast<float4 *>(sp) = make_float4(h[0], h[1], h[2], h[3]);
+              else
+                *reinterpret_cast<float2 *>(sp) = make_float2(h[0], h[1]);
+            }
+          }
         }
-        const f2 dx2 = mk2(ddx.y, ddx.y);
-        f2 h01 = fma2(mk2(a[0], a[1]), mk2(h[0], h[1]), mul2(dx2, mk2(b4.x, b4.y)));
-        f2 h23 = fma2(mk2(a[2], a[3]), mk2(h[2], h[3]), mul2(dx2, mk2(b4.z, b4.w)));
-        h[0] = h01.x; h[1] = h01.y; h[2] = h23.x; h[3] = h23.y;
-        const f2 y2 = fma2(mk2(c4.z, c4.w), h23, mul2(mk2(c4.x, c4.y), h01));
-        part[u] = y2.x + y2.y;
-        if (p.states != nullptr && cvalid && t < tn)
-          *reinterpret_cast<float4 *>(p.states + ((b * L + t0 + t) * C + c) * N + 4 * q) =
-              make_float4(h[0], h[1], h[2], h[3]);
-      }
-      const float yq = transpose_reduce<G>(part, q);
-      const int tt = tg + q;  // this lane's token
-      if (tt < tn && cvalid) {
-        float yv = yq + Dc * ld(&s.x[buf][tt][cl]);
-        if (HAS_Z) {
-          const float zv = ld(&s.z[buf][tt][cl]);
-          yv *= kBF16 ? silu_fast(zv) : silu(zv);
+        const float yq = transpose_reduce<G>(part, q);
+        const int tt = tg + q;  // this lane's token
+        if (tt < tn && cvalid) {
+          float yv = yq + Dc * ld(&s.x[buf][tt][cl]);
+          if (HAS_Z) {
+            const float zv = ld(&s.z[buf][tt][cl]);
+            yv *= kBF16 ? silu_fast(zv) : silu(zv);
+          }
+          st(&s.y[tt][cl], yv);
         }
-        st(&s.y[tt][cl], yv);
       }
     }
     __syncthreads();
@@ -312,9 +375,13 @@ __global__ void __launch_bounds__(CT *(N / 4))
       }
     }
   }
-  if (p.h_last && cvalid)
-    *reinterpret_cast<float4 *>(p.h_last + (b * C + c) * N + 4 * q) =
-        make_float4(h[0], h[1], h[2], h[3]);
+  if (p.h_last && cvalid) {
+    float *hp = p.h_last + (b * C + c) * N + SPL * q;
+    if constexpr (SPL == 4)
+      *reinterpret_cast<float4 *>(hp) = make_float4(h[0], h[1], h[2], h[3]);
+    else
+      *reinterpret_cast<float2 *>(hp) = make_float2(h[0], h[1]);
+  }
 }
 
 template <typename T>
@@ -322,7 +389,8 @@ CUtensorMapDataType tmap_type() {
   return sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
 }
 
-template <int N, typename T, int CT, bool HZ, int SWX>
+template <int N, typename T, int CT, bool HZ, int SWX, int SPL, bool ST, bool PK = true,
+          int UT = 1>
 cudaError_t launch_tma(const M1Params &p, cudaStream_t s) {
   CUtensorMap mx, mdt, mz, mB, mC;
   const uint64_t es = sizeof(T);
@@ -347,34 +415,45 @@ cudaError_t launch_tma(const M1Params &p, cudaStream_t s) {
         !encode_tiled(&mC, tmap_type<T>(), 3, p.Cm, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
-  auto k = m1_scan_tma_kernel<N, T, CT, HZ, SWX>;
+  auto k = m1_scan_tma_kernel<N, T, CT, HZ, SWX, SPL, ST, PK, UT>;
   const size_t smem = sizeof(M1Smem<N, T, CT>) + 128;
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid((unsigned)((p.C + CT - 1) / CT), (unsigned)p.batch);
-  k<<<grid, CT * (N / 4), smem, s>>>(mx, mdt, mz, mB, mC, p);
+  k<<<grid, CT * (N / SPL), smem, s>>>(mx, mdt, mz, mB, mC, p);
   return cudaGetLastError();
 }
 
-template <int N, typename T, int CT>
-cudaError_t launch_z(const M1Params &p, cudaStream_t s) {
-  const int swx = p.swx;
-  if (p.z) {
-    if (swx == 1) return launch_tma<N, T, CT, true, 1>(p, s);
-    if (swx == 2) return launch_tma<N, T, CT, true, 2>(p, s);
-    return launch_tma<N, T, CT, true, 0>(p, s);
+// Variant choice: per-token states (tests only) take one fixed form; the
+// others follow p.variant (states per lane, packed math, unrolling, and 8 =
+// one decay per lane on the FMA-pipe exp2).
+template <int N, typename T, bool HZ>
+cudaError_t launch_v(const M1Params &p, cudaStream_t s) {
+  if (p.states) return launch_tma<N, T, 16, HZ, 0, 4, true>(p, s);
+  // variant = 4 * (packed) + 2 * (two groups per iteration) + (2 states per lane)
+  switch (p.variant) {
+    case 0: return launch_tma<N, T, 16, HZ, 0, 4, false, false, 1>(p, s);
+    case 1: return launch_tma<N, T, 16, HZ, 0, 2, false, false, 1>(p, s);
+    case 2: return launch_tma<N, T, 16, HZ, 0, 4, false, false, 2>(p, s);
+    case 3: return launch_tma<N, T, 16, HZ, 0, 2, false, false, 2>(p, s);
+    case 4: return launch_tma<N, T, 16, HZ, 0, 4, false, true, 1>(p, s);
+    case 5: return launch_tma<N, T, 16, HZ, 0, 2, false, true, 1>(p, s);
+    case 6: return launch_tma<N, T, 16, HZ, 0, 4, false, true, 2>(p, s);
+    case 7: return launch_tma<N, T, 16, HZ, 0, 2, false, true, 2>(p, s);
+    case 8: return launch_tma<N, T, 16, HZ, 1, 4, false, true, 1>(p, s);
   }
-  if (swx == 1) return launch_tma<N, T, CT, false, 1>(p, s);
-  if (swx == 2) return launch_tma<N, T, CT, false, 2>(p, s);
-  return launch_tma<N, T, CT, false, 0>(p, s);
+  return launch_tma<N, T, 16, HZ, 0, 2, false, true, 1>(p, s);
 }
 
 template <typename T>
 cudaError_t launch_tma_t(const M1Params &p, cudaStream_t s) {
+  const bool hz = p.z != nullptr;
   switch (p.N) {
-    case 8: return launch_z<8, T, 16>(p, s);
-    case 16: return launch_z<16, T, 16>(p, s);
-    case 32: return launch_z<32, T, 16>(p, s);
+    case 8: return hz ? launch_tma<8, T, 16, true, 0, 4, false>(p, s)
+                      : launch_tma<8, T, 16, false, 0, 4, false>(p, s);
+    case 16: return hz ? launch_v<16, T, true>(p, s) : launch_v<16, T, false>(p, s);
+    case 32: return hz ? launch_tma<32, T, 16, true, 0, 4, false>(p, s)
+                       : launch_tma<32, T, 16, false, 0, 4, false>(p, s);
   }
   return cudaErrorNotSupported;
 }
@@ -382,8 +461,10 @@ cudaError_t launch_tma_t(const M1Params &p, cudaStream_t s) {
 }  // namespace
 
 // The pipelined kernel needs 16-byte rows for TMA (a 16-channel tile and the
-// B/C rows), a channel tile inside one group, and N in {8, 16, 32}.
+// B/C rows), a channel tile inside one group, and N in {8, 16, 32}; per-token
+// states only with N = 16.
 bool m1_scan_tma_supported(const M1Params &p) {
+  if (p.states && p.N != 16) return false;
   const int64_t es = p.io == 1 ? 2 : 4;
   if (p.N != 8 && p.N != 16 && p.N != 32) return false;
   if ((p.N * es) % 16 || (p.C * es) % 16 || (p.G * p.N * es) % 16) return false;

@@ -21,25 +21,24 @@ bool all_aligned(Ps... ps) {
   return true;
 }
 
-// How many of the 4 states per lane take their decay from the FMA-pipe
-// exponential instead of the SFU (0, 1 or 2); SSM_M1_EXP_SPLIT overrides the
-// default for tuning.
-int m1_exp_split() {
+// Variant of the pipelined Mamba-1 kernel (0..8, see scan_m1_tma.cu);
+// SSM_M1_VARIANT overrides the default for tuning.
+int m1_variant() {
   static int v = -1;
   if (v < 0) {
-    const char *e = getenv("SSM_M1_EXP_SPLIT");
-    v = (e && e[0] >= '0' && e[0] <= '2') ? e[0] - '0' : 1;
+    const char *e = getenv("SSM_M1_VARIANT");
+    v = (e && e[0] >= '0' && e[0] <= '8') ? e[0] - '0' : 5;
   }
   return v;
 }
 
-// The TMA-pipelined Mamba-1 kernel is opt-in (SSM_M1_PIPELINED=1) until it
-// has been validated on hardware.
+// The TMA-pipelined Mamba-1 kernel is used wherever the shape allows;
+// SSM_M1_PIPELINED=0 forces the generic kernel (for comparisons).
 int m1_pipelined() {
   static int v = -1;
   if (v < 0) {
     const char *e = getenv("SSM_M1_PIPELINED");
-    v = (e && e[0] == '1') ? 1 : 0;
+    v = (e && e[0] == '0') ? 0 : 1;
   }
   return v;
 }
@@ -192,8 +191,8 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_args_t *a, void *stream) {
   p.h_last = a->h_last;
   p.states = a->states;
   p.rstd = (a->flags & SSM_RMSNORM_DT) ? static_cast<float *>(a->workspace) : nullptr;
-  p.swx = m1_exp_split();
   p.pipelined = m1_pipelined();
+  p.variant = m1_variant();
   p.status = nullptr;
   return from_cuda(ssm::launch_m1_scan(p, s));
 }

@@ -23,6 +23,10 @@
 namespace ssm {
 namespace {
 
+// Row of the k-th state row a lane of the P = 64 step kernel owns: blocks of
+// 8 consecutive rows, the next block 128 rows further on.
+__device__ __forceinline__ int rowof(int n0, int k) { return n0 + (k & 7) + 128 * (k >> 3); }
+
 template <typename T, bool HAS_Z, int K, int TT>
 __global__ void __launch_bounds__(256) m2_recurrent_kernel(const M2Params p) {
   extern __shared__ __align__(16) float smem[];
@@ -173,6 +177,89 @@ cudaError_t launch_m2_t(const M2Params &p, int K, int RS, cudaStream_t s) {
   return cudaErrorNotSupported;
 }
 
+// ------------------------------------------------- Mamba-2 step, P = 64
+
+// One decode token for one (batch, head) per CTA of 256 threads, head dim 64,
+// state N = 16 * K.  Lane l of warp w owns the four value columns 4(l%16)..+3
+// of the K rows n = 16 w + 8 (l / 16) + k: each float4 load/store of a warp
+// covers two 256-byte row segments.  The token's inputs are read straight
+// from global memory (B and C rows as one 16-byte load per lane), so the only
+// barrier is the one that combines the eight warps' partial C^T h.
+template <typename T, bool HAS_Z, int K>
+__global__ void __launch_bounds__(256, 3) m2_step_kernel(const M2Params p) {
+  constexpr int kP = 64;
+  constexpr int N = 16 * K;
+  __shared__ float4 ys[8][16];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int pq = lane & 15, half = lane >> 4;
+  const int64_t hd = blockIdx.x, b = blockIdx.y;
+  const int64_t H = p.H, G = p.G;
+  const int64_t g = hd / (H / G);
+  const int n0 = 16 * warp + 8 * half;  // rows rowof(n0, k), k < K
+  float *state = const_cast<float *>(p.h0) + (b * H + hd) * (int64_t)N * kP;
+
+  // State first: every load in flight before any arithmetic.
+  float4 S[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k)
+    S[k] = ld_stream4(reinterpret_cast<const float4 *>(state + (int64_t)(rowof(n0, k)) * kP + 4 * pq));
+
+  const T *Bp = static_cast<const T *>(p.B) + (b * G + g) * N;
+  const T *Cp = static_cast<const T *>(p.Cm) + (b * G + g) * N;
+  float bn[K], cn[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    bn[k] = ld(Bp + rowof(n0, k));
+    cn[k] = ld(Cp + rowof(n0, k));
+  }
+  const T *xp = static_cast<const T *>(p.x) + (b * H + hd) * kP + 4 * pq;
+  const float4 xq = make_float4(ld(xp), ld(xp + 1), ld(xp + 2), ld(xp + 3));
+  float d = ld(static_cast<const T *>(p.dt) + b * H + hd) + (p.dt_bias ? p.dt_bias[hd] : 0.f);
+  if (p.flags & 1u) d = softplus(d);
+  const float a = ex2(d * (p.A[hd] * kLog2e));
+
+  float4 yp = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const float w = d * bn[k];
+    S[k].x = a * S[k].x + w * xq.x;
+    S[k].y = a * S[k].y + w * xq.y;
+    S[k].z = a * S[k].z + w * xq.z;
+    S[k].w = a * S[k].w + w * xq.w;
+    yp.x += cn[k] * S[k].x;
+    yp.y += cn[k] * S[k].y;
+    yp.z += cn[k] * S[k].z;
+    yp.w += cn[k] * S[k].w;
+  }
+#pragma unroll
+  for (int k = 0; k < K; ++k)
+    st_stream4(reinterpret_cast<float4 *>(state + (int64_t)(rowof(n0, k)) * kP + 4 * pq), S[k]);
+  yp.x += __shfl_xor_sync(0xffffffffu, yp.x, 16);
+  yp.y += __shfl_xor_sync(0xffffffffu, yp.y, 16);
+  yp.z += __shfl_xor_sync(0xffffffffu, yp.z, 16);
+  yp.w += __shfl_xor_sync(0xffffffffu, yp.w, 16);
+  if (half == 0) ys[warp][pq] = yp;
+  __syncthreads();
+  if (tid < 16) {
+    float4 acc = ys[0][tid];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) {
+      const float4 v = ys[w][tid];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    const float Dh = p.D ? p.D[hd] : 0.f;
+    const T *xr = static_cast<const T *>(p.x) + (b * H + hd) * kP + 4 * tid;
+    float o[4] = {acc.x + Dh * ld(xr), acc.y + Dh * ld(xr + 1), acc.z + Dh * ld(xr + 2),
+                  acc.w + Dh * ld(xr + 3)};
+    T *yo = static_cast<T *>(p.y) + (b * H + hd) * kP + 4 * tid;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (HAS_Z) o[j] *= silu(ld(static_cast<const T *>(p.z) + (b * H + hd) * kP + 4 * tid + j));
+      st(yo + j, o[j]);
+    }
+  }
+}
+
 // ------------------------------------------------------------ Mamba-1 step
 
 template <int N, typename T, bool HAS_Z>
@@ -271,6 +358,20 @@ cudaError_t launch_m2_recurrent(const M2Params &p, cudaStream_t s) {
   int K, RS;
   if (!m2_shape(p.N, p.P, &K, &RS)) return cudaErrorNotSupported;
   if (p.batch == 0 || p.L == 0) return cudaSuccess;
+  // The decode step (one token, state updated in place) with head dim 64 and
+  // state 128 has its own kernel.
+  if (p.L == 1 && p.P == 64 && p.N == 128 && p.states == nullptr && p.h0 != nullptr &&
+      p.h0 == p.h_last) {
+    dim3 grid((unsigned)p.H, (unsigned)p.batch);
+    const bool hz = p.z != nullptr;
+    if (p.io == 1)
+      hz ? m2_step_kernel<__nv_bfloat16, true, 8><<<grid, 256, 0, s>>>(p)
+         : m2_step_kernel<__nv_bfloat16, false, 8><<<grid, 256, 0, s>>>(p);
+    else
+      hz ? m2_step_kernel<float, true, 8><<<grid, 256, 0, s>>>(p)
+         : m2_step_kernel<float, false, 8><<<grid, 256, 0, s>>>(p);
+    return cudaGetLastError();
+  }
   const bool hz = p.z != nullptr;
   if (p.io == 1)
     return hz ? launch_m2_t<__nv_bfloat16, true>(p, K, RS, s)

@@ -78,6 +78,11 @@ WORKLOADS = {
         "decode_2p7b_stack_b256", "decode", batch=256, heads=80, head_dim=64,
         state=128, io="bf16", gate=False, layers=64, m1_layers=24,
         m1_channels=1536, m1_state=16, seed=4),
+    # One layer of each decode stack (a small case of the same kernels).
+    "decode_2p7b_layer_b256": Workload(
+        "decode_2p7b_layer_b256", "decode", batch=256, heads=80, head_dim=64,
+        state=128, io="bf16", gate=False, layers=1, m1_layers=1,
+        m1_channels=1536, m1_state=16, seed=4),
 }
 
 
