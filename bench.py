@@ -36,7 +36,7 @@ L2_BYTES = 126 * 2 ** 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
@@ -48,7 +48,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["m1", "ssd", "decode", "decode_layer", "falcon"],
                     help="run just one workload's timed loop (for profiling); prints its timing")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def peaks():
@@ -207,6 +207,18 @@ class Dist:
     def close(self):
         if self.pg:
             self.pg.destroy_process_group()
+
+
+def rank_seed(seed, rank):
+    """Seed of one rank's batch: every rank scans its own independent batch of
+    the same shape (weak scaling, nothing exchanged on the data path)."""
+    return seed + 7919 * rank
+
+
+def job_value(units_per_rank, world, ms_per_step):
+    """Whole-job throughput: the units every rank processed in one step, over
+    the slowest rank's step time (ms), per second."""
+    return units_per_rank * world / (ms_per_step * 1e-3)
 
 
 def timed(step, K, W, dist, device):
@@ -421,12 +433,13 @@ def run_ours(args):
     time.sleep(0.2)
 
     w = I.WORKLOADS[HEADLINE]
-    r = bench_m1(w, K, W, dist, device, pk, seed_base=w.seed + 7919 * dist.rank)
+    generic = os.environ.get("SSM_M1_PIPELINED", "1") == "0"
+    r = bench_m1(w, K, W, dist, device, pk, seed_base=rank_seed(w.seed, dist.rank))
     sampler.stop_ev.set()
     sampler.join(timeout=2)
     clocks = sampler.summary()
     hbm = pk["hbm_gbs"]
-    value = r["bytes"] * dist.world / (r["ms_per_step"] * 1e-3) / 1e9
+    value = job_value(r["bytes"], dist.world, r["ms_per_step"]) / 1e9
     achieved = r["bytes"] / (r["launch_ms"] * 1e-3) / 1e9
     out = {
         "metric": "Mamba-1 selective scan algorithmic HBM throughput (GB/s); "
@@ -443,9 +456,9 @@ def run_ours(args):
                    "parallelism": "dp%d (independent batches per GPU)" % dist.world},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm,
                      "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                     "traffic": traffic_for("m1_scan_130m"),
+                     "traffic": traffic_for("m1_scan_130m" if generic else "m1_scan_tma_130m"),
                      "peak_source": "%s hbm_gbs (copy)" % pk["_source"],
-                     "kernel": "m1_scan_kernel"},
+                     "kernel": "m1_scan_kernel" if generic else "m1_scan_tma_kernel"},
         "clocks": clocks,
         "gpu_launches": r["launches_per_step"] * K,
     }
@@ -458,10 +471,10 @@ def run_ours(args):
         wl = {}
         ws = I.WORKLOADS["ssd_2p7b_b4_l4096_h80_p64_n128_bf16"]
         Ke = max(3, min(K, 20))
-        s = bench_ssd(ws, Ke, max(3, W), dist, device, pk, ws.seed + 7919 * dist.rank)
+        s = bench_ssd(ws, Ke, max(3, W), dist, device, pk, rank_seed(ws.seed, dist.rank))
         tf = s["flops"] / (s["launch_ms"] * 1e-3) / 1e12
         wl[ws.name] = {
-            "value": round(s["tokens"] * dist.world / (s["ms_per_step"] * 1e-3), 1),
+            "value": round(job_value(s["tokens"], dist.world, s["ms_per_step"]), 1),
             "unit": "tokens/s", "ms_per_step": round(s["ms_per_step"], 4),
             "gbs": round(s["bytes"] / (s["ms_per_step"] * 1e-3) / 1e9, 1),
             "roofline": {"bound": "tensor", "achieved": round(tf, 2),
@@ -471,10 +484,10 @@ def run_ours(args):
                          "flops_per_launch": s["flops"], "bytes_per_launch": s["bytes"],
                          "hbm_frac": round(s["bytes"] / (s["launch_ms"] * 1e-3) / 1e9 / hbm, 4)}}
         wd = I.WORKLOADS["decode_2p7b_stack_b256"]
-        dd = bench_decode(wd, max(3, min(K, 5)), 3, dist, device, pk, wd.seed + 7919 * dist.rank)
+        dd = bench_decode(wd, max(3, min(K, 5)), 3, dist, device, pk, rank_seed(wd.seed, dist.rank))
         ach = dd["launch_bytes"] / (dd["launch_ms"] * 1e-3) / 1e9
         wl[wd.name] = {
-            "value": round(dd["bytes"] * dist.world / (dd["ms_per_step"] * 1e-3) / 1e9, 2),
+            "value": round(job_value(dd["bytes"], dist.world, dd["ms_per_step"]) / 1e9, 2),
             "unit": "GB/s", "ms_per_step": round(dd["ms_per_step"], 4),
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(ach / hbm, 4), "traffic": traffic_for("m2_step_2p7b"),
@@ -482,10 +495,10 @@ def run_ours(args):
         del dd
         torch.cuda.empty_cache()
         wf = I.WORKLOADS["m1_falcon_rms_b4_l8192_c8192_n16_bf16"]
-        f = bench_m1(wf, max(3, min(K, 10)), 3, dist, device, pk, wf.seed + 7919 * dist.rank)
+        f = bench_m1(wf, max(3, min(K, 10)), 3, dist, device, pk, rank_seed(wf.seed, dist.rank))
         ach = f["bytes"] / (f["launch_ms"] * 1e-3) / 1e9
         wl[wf.name] = {
-            "value": round(f["bytes"] * dist.world / (f["ms_per_step"] * 1e-3) / 1e9, 2),
+            "value": round(job_value(f["bytes"], dist.world, f["ms_per_step"]) / 1e9, 2),
             "unit": "GB/s", "ms_per_step": round(f["ms_per_step"], 4),
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(ach / hbm, 4), "traffic": traffic_for("m1_scan_falcon"),

@@ -59,6 +59,61 @@ __device__ __forceinline__ float silu(float z) {
   return z / (1.f + ex2(-z * kLog2e));
 }
 
+// silu(z) = z * sigmoid(z) = z * (1 + tanh(z / 2)) / 2, with the SFU's
+// tanh.approx.f32 (one SFU operation instead of ex2 and a reciprocal).  Its
+// absolute error is a few 2^-11 of z: enough for bfloat16 outputs.
+__device__ __forceinline__ float silu_tanh(float z) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+  return z * fmaf(0.5f, t, 0.5f);
+}
+
+// ------------------------------------------------------------ packed f32x2
+
+struct f2 {
+  float x, y;
+};
+__device__ __forceinline__ f2 mk2(float a, float b) { return {a, b}; }
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// softplus(v) = log(1 + e^v), float32, from the SFU's ex2/lg2: for e^v < 1/32
+// a 4-term series of log1p (relative error below 2e-7), above it lg2(1 + e^v)
+// (the rounding of 1 + e^v then costs at most 2 ulp relative); v > 20 gives v.
+__device__ __forceinline__ float softplus_sfu(float v) {
+  const float u = ex2(v * kLog2e);
+  float lg;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(1.f + u));
+  const float series = u * fmaf(u, fmaf(u, fmaf(u, -0.25f, 0.33333334f), -0.5f), 1.f);
+  const float r = u < 0.03125f ? series : lg * 0.6931471806f;
+  return v > 20.f ? v : r;
+}
+
 // --------------------------------------------------------- cache hints
 
 // Streaming 16-byte load/store (no reuse expected: evict-first).

@@ -46,40 +46,6 @@ constexpr float kMagic = 12583039.0f;
 constexpr float kP1 = 6.931468844e-01f, kP2 = 2.402223796e-01f, kP3 = 5.550893024e-02f,
                 kP4 = 9.671698324e-03f, kP5 = 1.321867225e-03f;
 
-// ------------------------------------------------------------ packed f32x2
-
-struct f2 {
-  float x, y;
-};
-__device__ __forceinline__ f2 mk2(float a, float b) { return {a, b}; }
-__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
-  f2 d;
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return d;
-}
-__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
-  f2 d;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
-__device__ __forceinline__ f2 add2(f2 a, f2 b) {
-  f2 d;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
-
 // 2^(d*A2) for two states on the FMA pipe, for d >= 0 and A2 < 0 (a decay):
 // d is first clamped to lim = -127 / A2 so that the exponent never drops below
 // -127, where the result is exactly 0.
@@ -127,12 +93,6 @@ __device__ __forceinline__ float transpose_reduce(float (&p)[G], int q) {
   return p[0];
 }
 
-__device__ __forceinline__ float silu_fast(float z) {  // z * sigmoid(z) via tanh
-  float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
-  return z * fmaf(0.5f, t, 0.5f);
-}
-
 template <int N, typename T, int CT>
 struct alignas(128) M1Smem {
   T x[kNS][kTL][CT];
@@ -145,18 +105,6 @@ struct alignas(128) M1Smem {
   T y[kTL][CT];
   uint64_t full[kNS];
 };
-
-// softplus(v) = log(1 + e^v), float32, from the SFU's ex2/lg2: for e^v < 1/32
-// a 4-term series of log1p (relative error below 2e-7), above it lg2(1 + e^v)
-// (the rounding of 1 + e^v then costs at most 2 ulp relative); v > 20 gives v.
-__device__ __forceinline__ float softplus_sfu(float v) {
-  const float u = ex2(v * kLog2e);
-  float lg;
-  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(1.f + u));
-  const float series = u * fmaf(u, fmaf(u, fmaf(u, -0.25f, 0.33333334f), -0.5f), 1.f);
-  const float r = u < 0.03125f ? series : lg * 0.6931471806f;
-  return v > 20.f ? v : r;
-}
 
 // SPL states per lane (2 or 4), G = N / SPL lanes per channel.  SWX of a
 // lane's SPL decays use the FMA-pipe exp2.  STATES: also store every token's
@@ -257,9 +205,23 @@ __global__ void __launch_bounds__(CT *(N / SPL))
       const T *src = which ? s.C[buf][t] : s.B[buf][t];
       float v[N];
       float ss = 0.f;
+      if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int n = 0; n < N; n += 8) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(src + n);
+          v[n] = bf16lo(w.x); v[n + 1] = bf16hi(w.x); v[n + 2] = bf16lo(w.y); v[n + 3] = bf16hi(w.y);
+          v[n + 4] = bf16lo(w.z); v[n + 5] = bf16hi(w.z); v[n + 6] = bf16lo(w.w); v[n + 7] = bf16hi(w.w);
+        }
+      } else {
+#pragma unroll
+        for (int n = 0; n < N; n += 4) {
+          const float4 w = *reinterpret_cast<const float4 *>(src + n);
+          v[n] = w.x; v[n + 1] = w.y; v[n + 2] = w.z; v[n + 3] = w.w;
+        }
+      }
 #pragma unroll
       for (int n = 0; n < N; ++n) {
-        v[n] = t < tn ? ld(src + n) : 0.f;
+        if (t >= tn) v[n] = 0.f;
         ss += v[n] * v[n];
       }
       const float r = rms_bc ? rsqrtf(ss / N + p.eps) : 1.f;
@@ -283,11 +245,14 @@ __global__ void __launch_bounds__(CT *(N / SPL))
           const float2 ddx = s.ddx[t][cl];
           const float d = ddx.x, dx = ddx.y;
           float bv[SPL], cv[SPL], a[SPL];
-          if constexpr (SPL == 4) {
-            const float4 b4 = *reinterpret_cast<const float4 *>(&s.bc[t][0][4 * q]);
-            const float4 c4 = *reinterpret_cast<const float4 *>(&s.bc[t][1][4 * q]);
-            bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
-            cv[0] = c4.x; cv[1] = c4.y; cv[2] = c4.z; cv[3] = c4.w;
+          if constexpr (SPL >= 4) {
+#pragma unroll
+            for (int v = 0; v < SPL / 4; ++v) {
+              const float4 b4 = *reinterpret_cast<const float4 *>(&s.bc[t][0][SPL * q + 4 * v]);
+              const float4 c4 = *reinterpret_cast<const float4 *>(&s.bc[t][1][SPL * q + 4 * v]);
+              bv[4 * v] = b4.x; bv[4 * v + 1] = b4.y; bv[4 * v + 2] = b4.z; bv[4 * v + 3] = b4.w;
+              cv[4 * v] = c4.x; cv[4 * v + 1] = c4.y; cv[4 * v + 2] = c4.z; cv[4 * v + 3] = c4.w;
+            }
           } else {
             const float2 b2 = *reinterpret_cast<const float2 *>(&s.bc[t][0][2 * q]);
             const float2 c2 = *reinterpret_cast<const float2 *>(&s.bc[t][1][2 * q]);
@@ -337,10 +302,9 @@ __global__ void __launch_bounds__(CT *(N / SPL))
           if constexpr (STATES) {
             if (cvalid && t < tn) {
               float *sp = p.states + ((b * L + t0 + t) * C + c) * N + SPL * q;
-              if constexpr (SPL == 4)
-                *reinterpret_cast<float4 *>(sp) = make_float4(h[0], h[1], h[2], h[3]);
-              else
-                *reinterpret_cast<float2 *>(sp) = make_float2(h[0], h[1]);
+#pragma unroll
+              for (int j = 0; j < SPL; j += 2)
+                *reinterpret_cast<float2 *>(sp + j) = make_float2(h[j], h[j + 1]);
             }
           }
         }
@@ -350,7 +314,7 @@ __global__ void __launch_bounds__(CT *(N / SPL))
           float yv = yq + Dc * ld(&s.x[buf][tt][cl]);
           if (HAS_Z) {
             const float zv = ld(&s.z[buf][tt][cl]);
-            yv *= kBF16 ? silu_fast(zv) : silu(zv);
+            yv *= kBF16 ? silu_tanh(zv) : silu(zv);
           }
           st(&s.y[tt][cl], yv);
         }
@@ -377,10 +341,8 @@ __global__ void __launch_bounds__(CT *(N / SPL))
   }
   if (p.h_last && cvalid) {
     float *hp = p.h_last + (b * C + c) * N + SPL * q;
-    if constexpr (SPL == 4)
-      *reinterpret_cast<float4 *>(hp) = make_float4(h[0], h[1], h[2], h[3]);
-    else
-      *reinterpret_cast<float2 *>(hp) = make_float2(h[0], h[1]);
+#pragma unroll
+    for (int j = 0; j < SPL; j += 2) *reinterpret_cast<float2 *>(hp + j) = make_float2(h[j], h[j + 1]);
   }
 }
 
@@ -441,6 +403,11 @@ cudaError_t launch_v(const M1Params &p, cudaStream_t s) {
     case 6: return launch_tma<N, T, 16, HZ, 0, 4, false, true, 2>(p, s);
     case 7: return launch_tma<N, T, 16, HZ, 0, 2, false, true, 2>(p, s);
     case 8: return launch_tma<N, T, 16, HZ, 1, 4, false, true, 1>(p, s);
+    case 9: return launch_tma<N, T, 16, HZ, 0, 8, false, true, 1>(p, s);
+    case 10:  // 32-channel tiles: a tile must not straddle two B/C groups
+      if (p.G == 1 || (p.C / p.G) % 32 == 0) return launch_tma<N, T, 32, HZ, 0, 16, false, true, 1>(p, s);
+      return launch_tma<N, T, 16, HZ, 0, 8, false, true, 1>(p, s);
+    case 11: return launch_tma<N, T, 16, HZ, 0, 8, false, false, 1>(p, s);
   }
   return launch_tma<N, T, 16, HZ, 0, 2, false, true, 1>(p, s);
 }

@@ -15,31 +15,38 @@
 // 256-token masked form, up to rounding.
 //
 // One CTA per (batch, head), warp-specialised, tiles pipelined:
-//   warp 8      TMA producer: C, B ([128 x 128] bf16, two 64-column slabs) and
+//   warp 12     TMA producer: C, B ([128 x 128] bf16, two 64-column slabs) and
 //               x ([128 x 64]), 128-byte swizzle, double-buffered stages.
-//   warp 9      MMA issuer (tcgen05, bf16 in, fp32 accumulators in TMEM):
-//                 S  = C B^T            A, B K-major          (two buffers)
-//                 Yd = (S o mask) x     A = masked S from TMEM, B MN-major
-//                 Sc = B^T (w o x)      A = B read MN-major, B = scaled x
-//                 Yo = C h_prev         B = bf16 copy of the carried state
-//               issued per tile in the order Sc(c), S(c+1), Yo(c), Yd(c).
+//   warp 13     MMA issuer (tcgen05, bf16 in, fp32 accumulators in TMEM):
+//                 S  = C B^T                 A, B K-major     (two buffers)
+//                 Sc = B^T (w o x)           A = B read MN-major (two buffers)
+//                 Y  = M x + (e o C) h_prev  A = M and e o C from TMEM, both
+//                                            held in S's columns (two buffers)
+//               issued per tile in the order Sc(c), S(c+1), Y(c).
 //   warps 4-7   mask group, thread = token: the tile's step, cumulative decay
 //               and weights, w o x, then the mask applied to S as it is read
-//               from TMEM, written back as the bf16 A operand.  The mask
-//               exp(cum_i - cum_j) d_j is elementwise only on the four 32 x 32
-//               diagonal blocks; below them it is a row factor times a column
-//               factor, both <= 1 for a decaying state.
+//               from TMEM (D on its diagonal, so Y holds D x), and the row-
+//               scaled C, e_i C_i with e_i = exp(cum_i), both written back as
+//               the bf16 A operand of Y.  The mask exp(cum_i - cum_j) d_j is
+//               elementwise on the four 32 x 32 diagonal blocks; below them it
+//               is a row factor times a column factor, both <= 1 for a
+//               decaying state.
 //   warps 0-3   state group: thread n keeps row n of the float32 state in
-//               registers, h = exp(cum_last) h + Sc, writes its bf16 copy for
-//               the next tile's Yo; then, thread = token, the output
-//               y = Yd + exp(cum_i) Yo + D x (* silu(z)).
-// The carried-state chain per tile is only the state group's update; the
-// contractions of the next tile run under it.
+//               registers, h = exp(cum_last) h + Sc, and writes its bf16 copy
+//               for Y of the next tile (two buffers).
+//   warps 8-11  output group, thread = token: y = Y (* silu(z)), with z
+//               fetched one tile ahead.
+// With Y, Sc and the bf16 state double-buffered, the only chain carried from
+// tile to tile is the state group's update; every other role has a tile of
+// slack, and the contractions of the next tile run under this tile's
+// elementwise work.
 //
-// Every wait is bounded.  A group votes on its waits (bar.red.or) so its
-// threads always take the same branch; a wait that runs out sets the device
-// status word and a shared abort flag, every role leaves its loop, and the
-// CTA frees its TMEM and returns.
+// Every wait is bounded.  The mask group votes on its waits (bar.red.or) so
+// its threads always take the same branch; the state and output groups sync
+// only within a warp and arrive once per warp.  A wait that runs out sets the
+// device status word and a shared abort flag, every role leaves its loop, the
+// MMA issuer and the producer wait (bounded) for their operations in flight,
+// and the CTA frees its TMEM and returns.
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -53,29 +60,31 @@ using namespace sm100;
 constexpr int kQ = 128;   // tokens per tile
 constexpr int kN = 128;   // state size
 constexpr int kP = 64;    // head dim
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr long long kWaitLimit = 2000000000ll;  // cycles (about a second)
 
+// TMEM columns: S[2] (fp32 S; then masked S in the first 64 columns and e o C
+// in the next 64, as packed bf16), Sc[2], Y[2].
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColSc = 256, kColYd = 320, kColYo = 384;
+constexpr uint32_t kColS = 0, kColSc = 256, kColY = 384;
 
 struct __align__(1024) SsdSmem {
   uint8_t C[2][2][kQ * 128];  // [stage][slab]
   uint8_t B[2][2][kQ * 128];
   uint8_t X[2][kQ * 128];     // [stage]
-  uint8_t Xw[2][kQ * 128];    // [tile parity]: w o x
-  uint8_t Hb[kN * 128];       // bf16 copy of the carried state, rows n
-  float cum[2][kQ];           // [tile parity]
-  float dd[2][kQ];
-  float vd[2][kQ];
-  float e[2][kQ];
-  float a[2];
+  uint8_t Xw[kQ * 128];       // w o x of the tile whose Sc is next
+  uint8_t Hb[2][kN * 128];    // bf16 copy of the carried state, rows n
+  float cum[kQ];
+  float dd[kQ];
+  float vd[kQ];
+  float a[4];                 // exp(cum_last) per tile, ring of four
   float wsum[4];
-  // Per-tile signals come in pairs indexed by tile parity, so a waiter would
-  // have to fall two tiles behind to miss a phase; the stage dependencies
-  // bound every role's lead to one tile.
-  uint64_t full[2], empty[2], sdone[2];
-  uint64_t scdone[2], yodone[2], yddone[2], xready[2], mready[2], stdone[2], yfree[2];
+  // Per-tile signals come in pairs indexed by tile parity (xready in fours);
+  // the dependencies between roles bound every waiter's lag to less than one
+  // lap of its ring, so no waiter can miss a phase.
+  uint64_t full[2], empty[2], sdone[2], scdone[2], mready[2], stdone[2], yready[2], yfree[2];
+  uint64_t xready[4];
+  uint64_t fin;
   uint32_t taddr;
   int abort;
 };
@@ -90,16 +99,7 @@ struct SsdTcParams {
   int *status;
 };
 
-__device__ __forceinline__ void unpack8(uint4 v, float (&f)[8]) {
-  f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
-  f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
-}
-__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
-  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                    pack_bf16x2(f[6], f[7]));
-}
-
-// Named barrier for one 128-thread group (ids 1 and 2; 0 is __syncthreads).
+// Named barrier for the mask group (id 1; 0 is __syncthreads).
 __device__ __forceinline__ void group_sync(int id) {
   asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
 }
@@ -119,6 +119,27 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// a * b on two packed bfloat16 pairs, round to nearest even.
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// 16-byte global load / store that bypass L1 allocation (streamed once).
+__device__ __forceinline__ uint4 ld_cs_u4(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.cs.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+__device__ __forceinline__ void st_cs_u4(void *p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 __device__ __forceinline__ bool aborted(const SsdSmem &s) {
   return *(volatile const int *)&s.abort != 0;
 }
@@ -135,12 +156,20 @@ __device__ __forceinline__ bool wait1(SsdSmem &s, uint64_t *bar, uint32_t parity
   set_abort(s, status, code);
   return false;
 }
-// A 128-thread group's wait: every thread waits (bounded), then the group votes.
-__device__ __forceinline__ bool waitg(SsdSmem &s, int gid, uint64_t *bar, uint32_t parity,
-                                      int *status, int code) {
+// The mask group's wait: every thread waits (bounded), then the group votes.
+__device__ __forceinline__ bool waitg(SsdSmem &s, uint64_t *bar, uint32_t parity, int *status,
+                                      int code) {
   bool ok = !aborted(s) && mbar_wait(bar, parity, kWaitLimit);
-  const bool fail = group_any(gid, !ok);
+  const bool fail = group_any(1, !ok);
   if (fail && (threadIdx.x & 127) == 0) set_abort(s, status, code);
+  return !fail;
+}
+// A warp's wait: every lane waits (bounded), then the warp votes.
+__device__ __forceinline__ bool waitw(SsdSmem &s, uint64_t *bar, uint32_t parity, int *status,
+                                      int code) {
+  bool ok = !aborted(s) && mbar_wait(bar, parity, kWaitLimit);
+  const bool fail = __any_sync(0xffffffffu, !ok);
+  if (fail && (threadIdx.x & 31) == 0) set_abort(s, status, code);
   return !fail;
 }
 
@@ -156,43 +185,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t L = p.L, H = p.H;
   const int g = (int)(hd / (H / p.G));
   const int nch = (int)((L + kQ - 1) / kQ);
+  // TMEM lane quarter of this warp (warp i may only touch lanes 32 (i % 4) ..)
+  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], 2);   // the tile's last MMA commit + the output group
+      mbar_init(&s.empty[i], 1);
       mbar_init(&s.sdone[i], 1);
       mbar_init(&s.scdone[i], 1);
-      mbar_init(&s.yodone[i], 1);
-      mbar_init(&s.yddone[i], 1);
-      mbar_init(&s.xready[i], 1);
       mbar_init(&s.mready[i], 1);
-      mbar_init(&s.stdone[i], 1);
-      mbar_init(&s.yfree[i], 1);
+      mbar_init(&s.stdone[i], 4);  // one arrival per state-group warp
+      mbar_init(&s.yready[i], 1);
+      mbar_init(&s.yfree[i], 4);   // one arrival per output-group warp
     }
+    for (int i = 0; i < 4; ++i) mbar_init(&s.xready[i], 1);
+    mbar_init(&s.fin, 1);
     s.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(&s.taddr, kTmemCols);
     tmem_relinquish();
   }
 
-  // State group: row n of the carried state in float32 registers.
-  float h[kP];
+  // The bf16 copy of the initial state, for Y(0), goes to Hb[1] (tile c
+  // reads Hb[(c + 1) & 1]).
   if (warp < 4) {
     const float *src = p.h0 ? p.h0 + ((b * H + hd) * kN + tid) * kP : nullptr;
 #pragma unroll
-    for (int q = 0; q < kP; q += 4) {
-      float4 v = src ? *reinterpret_cast<const float4 *>(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-      h[q] = v.x; h[q + 1] = v.y; h[q + 2] = v.z; h[q + 3] = v.w;
-    }
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float f[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) f[k] = h[8 * c + k];
-      *reinterpret_cast<uint4 *>(s.Hb + sw128(tid, c)) = pack8(f);
+    for (int cc = 0; cc < 8; ++cc) {
+      float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+      if (src) {
+        v0 = *reinterpret_cast<const float4 *>(src + 8 * cc);
+        v1 = *reinterpret_cast<const float4 *>(src + 8 * cc + 4);
+      }
+      *reinterpret_cast<uint4 *>(s.Hb[1] + sw128(tid, cc)) =
+          make_uint4(pack_bf16x2(v0.x, v0.y), pack_bf16x2(v0.z, v0.w), pack_bf16x2(v1.x, v1.y),
+                     pack_bf16x2(v1.z, v1.w));
     }
     fence_async_smem();
   }
@@ -201,12 +231,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tb = s.taddr;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&mX);
       tma_prefetch_desc(&mB);
       tma_prefetch_desc(&mC);
+      int issued = 0;
       for (int c = 0; c < nch; ++c) {
         const int st = c & 1;
         if (c >= 2 && !wait1(s, &s.empty[st], ((c >> 1) + 1) & 1, p.status, 1)) break;
@@ -216,10 +247,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(s.B[st][0], &mB, &s.full[st], g * kN, c * kQ, (int)b);
         tma_load_3d(s.B[st][1], &mB, &s.full[st], g * kN + 64, c * kQ, (int)b);
         tma_load_4d(s.X[st], &mX, &s.full[st], 0, (int)hd, c * kQ, (int)b);
+        issued = c + 1;
       }
+      // Leave no copy in flight: the last two tiles issued have landed (a
+      // phase already completed passes at once).
+      for (int c = issued - 2; c < issued; ++c)
+        if (c >= 0) mbar_wait(&s.full[c & 1], (c >> 1) & 1, kWaitLimit);
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id_S = idesc_bf16_f32(128, 128, false, false);
@@ -228,86 +264,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto mma_S = [&](int c) {  // S(c) = C B^T into S[c & 1]
         const int st = c & 1;
         const uint32_t c0 = smem_u32(s.C[st][0]), b0 = smem_u32(s.B[st][0]);
-        const uint32_t dcol = st ? kColS1 : kColS0;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t ko = (k >> 2) * (kQ * 128) + (k & 3) * 32;
-          mma_ss(tb + dcol, smem_desc(c0 + ko, 16, 1024, kSwizzle128B),
+          mma_ss(tb + kColS + 128 * st, smem_desc(c0 + ko, 16, 1024, kSwizzle128B),
                  smem_desc(b0 + ko, 16, 1024, kSwizzle128B), id_S, k > 0);
         }
         mma_commit(&s.sdone[st]);
       };
-      bool ok = wait1(s, &s.full[0], 0, p.status, 2);
+      bool ok = nch > 0 && wait1(s, &s.full[0], 0, p.status, 2);
       if (ok) mma_S(0);
       for (int c = 0; ok && c < nch; ++c) {
-        const int st = c & 1, pv = (c + 1) & 1;  // pv: parity slot of tile c-1
-        const uint32_t ph = (c >> 1) & 1, php = ((c - 1) >> 1) & 1;
-        // Sc(c) = B^T (w o x): needs w o x, and the state group done with Sc(c-1)
-        if (!wait1(s, &s.xready[st], ph, p.status, 3)) break;
-        if (c > 0 && !wait1(s, &s.stdone[pv], php, p.status, 4)) break;
+        const int k = c & 1;
+        const uint32_t ph = (c >> 1) & 1;
+        // Sc(c) = B^T (w o x): needs w o x of tile c
+        if (!wait1(s, &s.xready[c & 3], (c >> 2) & 1, p.status, 3)) break;
         tc_fence_after();
         {
-          const uint32_t b0 = smem_u32(s.B[st][0]), xw = smem_u32(s.Xw[st]);
+          const uint32_t b0 = smem_u32(s.B[k][0]), xw = smem_u32(s.Xw);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mma_ss(tb + kColSc, smem_desc(b0 + k * 2048, kQ * 128, 1024, kSwizzle128B),
-                   smem_desc(xw + k * 2048, kQ * 128, 1024, kSwizzle128B), id_Sc, k > 0);
-          mma_commit(&s.scdone[st]);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tb + kColSc + 64 * k, smem_desc(b0 + kk * 2048, kQ * 128, 1024, kSwizzle128B),
+                   smem_desc(xw + kk * 2048, kQ * 128, 1024, kSwizzle128B), id_Sc, kk > 0);
+          mma_commit(&s.scdone[k]);
         }
         // S(c+1), as soon as its tile has landed
         if (c + 1 < nch) {
-          if (!wait1(s, &s.full[(c + 1) & 1], ((c + 1) >> 1) & 1, p.status, 5)) break;
+          if (!wait1(s, &s.full[(c + 1) & 1], ((c + 1) >> 1) & 1, p.status, 4)) break;
           mma_S(c + 1);
         }
-        // Yo(c) = C h_prev: needs the output group done with Yo/Yd of c-1
-        if (c > 0 && !wait1(s, &s.yfree[pv], php, p.status, 6)) break;
+        // Y(c) = M x + (e o C) h_prev: needs the mask group's operands, the
+        // state of tile c-1 in Hb, and Y[k] read out by the output group
+        if (!wait1(s, &s.mready[k], ph, p.status, 5)) break;
+        if (c >= 1 && !wait1(s, &s.stdone[k ^ 1], ((c - 1) >> 1) & 1, p.status, 6)) break;
+        if (c >= 2 && !wait1(s, &s.yfree[k], ((c - 2) >> 1) & 1, p.status, 7)) break;
         tc_fence_after();
         {
-          const uint32_t c0 = smem_u32(s.C[st][0]), hb = smem_u32(s.Hb);
+          const uint32_t x0 = smem_u32(s.X[k]), hb = smem_u32(s.Hb[k ^ 1]);
+          const uint32_t acol = kColS + 128 * k, dcol = kColY + 64 * k;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint32_t ko = (k >> 2) * (kQ * 128) + (k & 3) * 32;
-            mma_ss(tb + kColYo, smem_desc(c0 + ko, 16, 1024, kSwizzle128B),
-                   smem_desc(hb + k * 2048, kN * 128, 1024, kSwizzle128B), id_Y, k > 0);
-          }
-          mma_commit(&s.yodone[st]);
-        }
-        // Yd(c) = M x: needs the masked S
-        if (!wait1(s, &s.mready[st], ph, p.status, 7)) break;
-        tc_fence_after();
-        {
-          const uint32_t x0 = smem_u32(s.X[st]);
-          const uint32_t mcol = st ? kColS1 : kColS0;
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tb + dcol, tb + acol + 8 * kk,
+                   smem_desc(x0 + kk * 2048, kQ * 128, 1024, kSwizzle128B), id_Y, kk > 0);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mma_ts(tb + kColYd, tb + mcol + 8 * k,
-                   smem_desc(x0 + k * 2048, kQ * 128, 1024, kSwizzle128B), id_Y, k > 0);
-          mma_commit(&s.yddone[st]);
-          mma_commit(&s.empty[st]);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tb + dcol, tb + acol + 64 + 8 * kk,
+                   smem_desc(hb + kk * 2048, kN * 128, 1024, kSwizzle128B), id_Y, true);
+          mma_commit(&s.yready[k]);
+          mma_commit(&s.empty[k]);
         }
       }
+      // Leave no MMA in flight before TMEM is freed.
+      mma_commit(&s.fin);
+      mbar_wait(&s.fin, 0, kWaitLimit);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ mask group
     const int i = tid - 128;  // token of the tile; TMEM lane i
     const int mw = warp - 4;
-    const uint32_t lane_base = (uint32_t)(32 * mw) << 16;
     const float A2 = p.A[hd] * kLog2e;
     const float bias = p.dt_bias ? p.dt_bias[hd] : 0.f;
+    const float Dh = p.D ? p.D[hd] : 0.f;
     const bool softplus_on = p.flags & 1u;
     float dt_next = i < L ? ld(p.dt + (b * L + i) * H + hd) : 0.f;
     for (int c = 0; c < nch; ++c) {
-      const int st = c & 1, k = c & 1;
+      const int k = c & 1;
       const int64_t t0 = (int64_t)c * kQ;
       const int valid = (int)(L - t0 < kQ ? L - t0 : kQ);
-      if (!waitg(s, 1, &s.full[st], (c >> 1) & 1, p.status, 8)) break;
-      // step, log2-decay and its inclusive sum over the tile
+      // step, log2-decay and its inclusive sum over the tile (needs only dt,
+      // so it runs while the tile's TMA is in flight)
       float d = 0.f;
       if (i < valid) {
         d = dt_next + bias;
-        if (softplus_on) d = softplus(d);
+        if (softplus_on) d = softplus_sfu(d);
       }
       if (t0 + kQ + i < L) dt_next = ld(p.dt + (b * L + t0 + kQ + i) * H + hd);
       float cs = d * A2;
@@ -325,171 +356,217 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (w < mw) cs += v;
         total += v;
       }
-      s.cum[k][i] = cs;
-      s.dd[k][i] = d;
-      s.e[k][i] = ex2(cs);
-      if (i == 0) s.a[k] = ex2(total);
+      s.cum[i] = cs;
+      s.dd[i] = d;
+      if (i == 0) s.a[c & 3] = ex2(total);
       group_sync(1);
-      s.vd[k][i] = ex2(s.cum[k][mw * 32 + 31] - cs) * d;
+      s.vd[i] = ex2(s.cum[mw * 32 + 31] - cs) * d;
+      const float e_i = ex2(cs);
       const float w_i = ex2(total - cs) * d;
-      // w o x (row i), the B operand of Sc
+      // w o x (row i), the B operand of Sc(c): x of tile c has landed and
+      // Sc(c-1) is done with the buffer
+      if (!waitg(s, &s.full[k], (c >> 1) & 1, p.status, 8)) break;
+      if (c >= 1 && !waitg(s, &s.scdone[k ^ 1], ((c - 1) >> 1) & 1, p.status, 9)) break;
+      {
+        const uint32_t w2 = pack_bf16x2(w_i, w_i);
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        float f[8];
-        unpack8(*reinterpret_cast<const uint4 *>(s.X[st] + sw128(i, cc)), f);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) f[q] *= w_i;
-        *reinterpret_cast<uint4 *>(s.Xw[k] + sw128(i, cc)) = pack8(f);
+        for (int cc = 0; cc < 8; ++cc) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(s.X[k] + sw128(i, cc));
+          *reinterpret_cast<uint4 *>(s.Xw + sw128(i, cc)) =
+              make_uint4(bmul2(v.x, w2), bmul2(v.y, w2), bmul2(v.z, w2), bmul2(v.w, w2));
+        }
       }
       fence_async_smem();
       group_sync(1);
-      if (i == 0) mbar_arrive(&s.xready[k]);
-      // masked S -> bf16 A operand, written over S as S is read
-      if (!waitg(s, 1, &s.sdone[k], (c >> 1) & 1, p.status, 9)) break;
+      if (i == 0) mbar_arrive(&s.xready[c & 3]);
+      // masked S -> bf16, written over S's first 64 columns as S is read,
+      // 32 columns at a time
+      if (!waitg(s, &s.sdone[k], (c >> 1) & 1, p.status, 10)) break;
       tc_fence_after();
-      {
-        const uint32_t col = k ? kColS1 : kColS0;
-        const float *cum = s.cum[k];
-#pragma unroll
-        for (int J = 0; J < 4; ++J) {
-          uint32_t m[16];
-          if (J > mw) {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) m[q] = 0u;
-          } else {
-            uint32_t r0[16], r1[16];
-            tmem_ld16(tb + lane_base + col + 32 * J, r0);
-            tmem_ld16(tb + lane_base + col + 32 * J + 16, r1);
-            tmem_ld_wait();
-            float f[32];
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              f[q] = __uint_as_float(r0[q]);
-              f[16 + q] = __uint_as_float(r1[q]);
-            }
-            if (J < mw) {
-              const float u = ex2(cs - cum[32 * J + 31]);
-              const float *vd = s.vd[k] + 32 * J;
-#pragma unroll
-              for (int q = 0; q < 32; ++q) f[q] *= u * vd[q];
-            } else {
-              const float *dd = s.dd[k] + 32 * J;
-#pragma unroll
-              for (int q = 0; q < 32; ++q) {
-                const int j = 32 * J + q;
-                f[q] = (j <= i) ? f[q] * ex2(cs - cum[j]) * dd[q] : 0.f;
-              }
-            }
-#pragma unroll
-            for (int q = 0; q < 16; ++q) m[q] = pack_bf16x2(f[2 * q], f[2 * q + 1]);
-          }
-          tmem_st16(tb + lane_base + col + 16 * J, m);
+      const uint32_t col = kColS + 128 * k;
+#pragma unroll 1
+      for (int J = 0; J < 4; ++J) {
+        uint32_t r[32];
+        uint32_t m[16];
+        if (J <= mw) {
+          tmem_ld16(tb + lane_base + col + 32 * J, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+          tmem_ld16(tb + lane_base + col + 32 * J + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+          tmem_ld_wait();
         }
-        tmem_st_wait();
+        if (J > mw) {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) m[q] = 0u;
+        } else if (J < mw) {
+          // below the diagonal: S_ij * exp2(cum_i - cum_r) * vd_j, r the
+          // block's last token; both factors <= 1
+          const float u = ex2(cs - s.cum[32 * J + 31]);
+          const float4 *vd4 = reinterpret_cast<const float4 *>(s.vd + 32 * J);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 v = vd4[q];
+            const f2 a = mul2(mul2(mk2(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])),
+                                   mk2(v.x, v.y)),
+                              mk2(u, u));
+            const f2 bq = mul2(mul2(mk2(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])),
+                                    mk2(v.z, v.w)),
+                               mk2(u, u));
+            m[2 * q] = pack_bf16x2(a.x, a.y);
+            m[2 * q + 1] = pack_bf16x2(bq.x, bq.y);
+          }
+        } else {
+          // diagonal block: S_ij * exp2(cum_i - cum_j) * d_j for j <= i, + D at j = i
+          const float4 *c4 = reinterpret_cast<const float4 *>(s.cum + 32 * J);
+          const float4 *d4 = reinterpret_cast<const float4 *>(s.dd + 32 * J);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 cj = c4[q], dj = d4[q];
+            const float cjs[4] = {cj.x, cj.y, cj.z, cj.w}, djs[4] = {dj.x, dj.y, dj.z, dj.w};
+            float f[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = 32 * J + 4 * q + e;
+              const float sv = __uint_as_float(r[4 * q + e]);
+              f[e] = (j <= i) ? sv * (ex2(cs - cjs[e]) * djs[e]) + (j == i ? Dh : 0.f) : 0.f;
+            }
+            m[2 * q] = pack_bf16x2(f[0], f[1]);
+            m[2 * q + 1] = pack_bf16x2(f[2], f[3]);
+          }
+        }
+        tmem_st16(tb + lane_base + col + 16 * J, m);
       }
+      // e_i C_i -> bf16, into columns 64..127 (S there has been read)
+      {
+        const uint32_t e2 = pack_bf16x2(e_i, e_i);
+#pragma unroll
+        for (int hs = 0; hs < 2; ++hs) {
+#pragma unroll
+          for (int c4 = 0; c4 < 2; ++c4) {
+            uint32_t m[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 v = *reinterpret_cast<const uint4 *>(s.C[k][hs] + sw128(i, 4 * c4 + q));
+              m[4 * q] = bmul2(v.x, e2);
+              m[4 * q + 1] = bmul2(v.y, e2);
+              m[4 * q + 2] = bmul2(v.z, e2);
+              m[4 * q + 3] = bmul2(v.w, e2);
+            }
+            tmem_st16(tb + lane_base + col + 64 + 32 * hs + 16 * c4, m);
+          }
+        }
+      }
+      tmem_st_wait();
       tc_fence_before();
       group_sync(1);
       if (i == 0) mbar_arrive(&s.mready[k]);
     }
-  } else {
+  } else if (warp < 4) {
     // ------------------------------------------------------------ state group
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    const float Dh = p.D ? p.D[hd] : 0.f;
-    for (int c = 0; c < nch; ++c) {
-      const int st = c & 1, k = c & 1;
-      const uint32_t ph = (c >> 1) & 1;
-      const int64_t t0 = (int64_t)c * kQ;
-      const int valid = (int)(L - t0 < kQ ? L - t0 : kQ);
-      // h = a h + Sc (thread = row n); a and e come from the mask group
-      if (!waitg(s, 2, &s.xready[k], ph, p.status, 10)) break;
-      if (!waitg(s, 2, &s.scdone[k], ph, p.status, 11)) break;
-      tc_fence_after();
-      const float a_c = s.a[k];
+    const int n = tid;
+    float h[kP];
+    {
+      const float *src = p.h0 ? p.h0 + ((b * H + hd) * kN + n) * kP : nullptr;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t r[16];
-        tmem_ld16(tb + lane_base + kColSc + 16 * q, r);
+      for (int q = 0; q < kP; q += 4) {
+        const float4 v = src ? *reinterpret_cast<const float4 *>(src + q)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        h[q] = v.x; h[q + 1] = v.y; h[q + 2] = v.z; h[q + 3] = v.w;
+      }
+    }
+    for (int c = 0; c < nch; ++c) {
+      const int k = c & 1;
+      // h = a h + Sc (thread = row n); a comes from the mask group, whose
+      // xready arrival orders its write before this read
+      if (!waitw(s, &s.xready[c & 3], (c >> 2) & 1, p.status, 11)) break;
+      if (!waitw(s, &s.scdone[k], (c >> 1) & 1, p.status, 12)) break;
+      tc_fence_after();
+      const float a_c = s.a[c & 3];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[32];
+        tmem_ld16(tb + lane_base + kColSc + 64 * k + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+        tmem_ld16(tb + lane_base + kColSc + 64 * k + 32 * hh + 16,
+                  *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) h[16 * q + j] = fmaf(a_c, h[16 * q + j], __uint_as_float(r[j]));
-      }
-      // the bf16 copy for Yo(c+1), once Yo(c) has read the old one
-      if (!waitg(s, 2, &s.yodone[k], ph, p.status, 12)) break;
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        float f[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) f[j] = h[8 * cc + j];
-        *reinterpret_cast<uint4 *>(s.Hb + sw128(tid, cc)) = pack8(f);
-      }
-      fence_async_smem();
-      tc_fence_before();
-      group_sync(2);
-      if (tid == 0) mbar_arrive(&s.stdone[k]);
-      // output y = Yd + e_i Yo + D x (thread = token i)
-      if (!waitg(s, 2, &s.yddone[k], ph, p.status, 13)) break;
-      tc_fence_after();
-      {
-        const int i = tid;
-        const float e_i = s.e[k][i];
-        const int64_t row = (b * L + t0 + i) * H + hd;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t yd[16], yo[16];
-          tmem_ld16(tb + lane_base + kColYd + 16 * q, yd);
-          tmem_ld16(tb + lane_base + kColYo + 16 * q, yo);
-          tmem_ld_wait();
-          float x0[8], x1[8], o[16];
-          unpack8(*reinterpret_cast<const uint4 *>(s.X[st] + sw128(i, 2 * q)), x0);
-          unpack8(*reinterpret_cast<const uint4 *>(s.X[st] + sw128(i, 2 * q + 1)), x1);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float xv = j < 8 ? x0[j] : x1[j - 8];
-            o[j] = fmaf(e_i, __uint_as_float(yo[j]), __uint_as_float(yd[j])) + Dh * xv;
-          }
-          if (i < valid) {
-            if (p.z) {
-              const uint4 *zp = reinterpret_cast<const uint4 *>(p.z + row * kP + 16 * q);
-              float z0[8], z1[8];
-              unpack8(zp[0], z0);
-              unpack8(zp[1], z1);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                o[j] *= silu(z0[j]);
-                o[8 + j] *= silu(z1[j]);
-              }
-            }
-            float lo[8], hi[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              lo[j] = o[j];
-              hi[j] = o[8 + j];
-            }
-            uint4 *yp = reinterpret_cast<uint4 *>(p.y + row * kP + 16 * q);
-            yp[0] = pack8(lo);
-            yp[1] = pack8(hi);
-          }
+        for (int j = 0; j < 32; j += 2) {
+          const f2 hn = fma2(mk2(a_c, a_c), mk2(h[32 * hh + j], h[32 * hh + j + 1]),
+                             mk2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])));
+          h[32 * hh + j] = hn.x;
+          h[32 * hh + j + 1] = hn.y;
         }
       }
       tc_fence_before();
-      group_sync(2);
-      if (tid == 0) {
-        mbar_arrive(&s.yfree[k]);
-        mbar_arrive(&s.empty[st]);
+      // bf16 copy for Y(c+1); its previous contents (tile c-2) were read by
+      // Y(c-1), which completed before Sc(c) (one issuer, in order)
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc)
+        *reinterpret_cast<uint4 *>(s.Hb[k] + sw128(n, cc)) =
+            make_uint4(pack_bf16x2(h[8 * cc], h[8 * cc + 1]), pack_bf16x2(h[8 * cc + 2], h[8 * cc + 3]),
+                       pack_bf16x2(h[8 * cc + 4], h[8 * cc + 5]),
+                       pack_bf16x2(h[8 * cc + 6], h[8 * cc + 7]));
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.stdone[k]);
+    }
+    if (!aborted(s) && p.h_last) {
+      float *dst = p.h_last + ((b * H + hd) * kN + n) * kP;
+#pragma unroll
+      for (int q = 0; q < kP; q += 4)
+        *reinterpret_cast<float4 *>(dst + q) = make_float4(h[q], h[q + 1], h[q + 2], h[q + 3]);
+    }
+  } else {
+    // ------------------------------------------------------------ output group
+    const int i = tid - 256;  // token of the tile; TMEM lane i
+    uint4 zr[8];
+    auto load_z = [&](int c) {
+      const int64_t t = (int64_t)c * kQ + i;
+      if (p.z && c < nch && t < L) {
+        const __nv_bfloat16 *zp = p.z + ((b * L + t) * H + hd) * kP;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) zr[q] = ld_cs_u4(zp + 8 * q);
       }
+    };
+    load_z(0);
+    for (int c = 0; c < nch; ++c) {
+      const int k = c & 1;
+      const int64_t t = (int64_t)c * kQ + i;
+      if (!waitw(s, &s.yready[k], (c >> 1) & 1, p.status, 13)) break;
+      tc_fence_after();
+      uint32_t v[64];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        tmem_ld16(tb + lane_base + kColY + 64 * k + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * q]));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.yfree[k]);
+      if (t < L) {
+        __nv_bfloat16 *yp = p.y + ((b * L + t) * H + hd) * kP;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float o[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) o[j] = __uint_as_float(v[8 * q + j]);
+          if (p.z) {
+            const uint32_t zw[4] = {zr[q].x, zr[q].y, zr[q].z, zr[q].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              o[2 * j] *= silu_tanh(bf16lo(zw[j]));
+              o[2 * j + 1] *= silu_tanh(bf16hi(zw[j]));
+            }
+          }
+          st_cs_u4(yp + 8 * q, make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                          pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7])));
+        }
+      }
+      load_z(c + 1);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp < 4 && !aborted(s) && p.h_last) {
-    float *dst = p.h_last + ((b * H + hd) * kN + tid) * kP;
-#pragma unroll
-    for (int q = 0; q < kP; q += 4)
-      *reinterpret_cast<float4 *>(dst + q) = make_float4(h[q], h[q + 1], h[q + 2], h[q + 3]);
-  }
-  if (warp == 9) tmem_dealloc(tb, kTmemCols);
+  if (warp == 13) tmem_dealloc(tb, kTmemCols);
 }
 
 bool encode(CUtensorMap *m, const void *ptr, int rank, const uint64_t *dims,
