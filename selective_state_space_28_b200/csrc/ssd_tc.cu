@@ -23,8 +23,10 @@
 //                 Y  = M x + (e o C) h_prev  A = M and e o C from TMEM, both
 //                                            held in S's columns (two buffers)
 //               issued per tile in the order Sc(c), S(c+1), Y(c).
-//   warps 4-7   mask group, thread = token: the tile's step, cumulative decay
-//               and weights, w o x, then the mask applied to S as it is read
+//   warps 4-7   mask group, thread = token (each warp also recomputes the
+//               whole tile's cumulative decay, so the warps run unsynchronised):
+//               the tile's step, cumulative decay and weights, w o x, then
+//               the mask applied to S as it is read
 //               from TMEM (D on its diagonal, so Y holds D x), and the row-
 //               scaled C, e_i C_i with e_i = exp(cum_i), both written back as
 //               the bf16 A operand of Y.  The mask exp(cum_i - cum_j) d_j is
@@ -41,9 +43,9 @@
 // slack, and the contractions of the next tile run under this tile's
 // elementwise work.
 //
-// Every wait is bounded.  The mask group votes on its waits (bar.red.or) so
-// its threads always take the same branch; the state and output groups sync
-// only within a warp and arrive once per warp.  A wait that runs out sets the
+// Every wait is bounded and every warp votes on its waits, so its lanes
+// always take the same branch; warps of a group never wait for each other,
+// they arrive once per warp on four-count barriers.  A wait that runs out sets the
 // device status word and a shared abort flag, every role leaves its loop, the
 // MMA issuer and the producer wait (bounded) for their operations in flight,
 // and the CTA frees its TMEM and returns.
@@ -74,17 +76,15 @@ struct __align__(1024) SsdSmem {
   uint8_t X[2][kQ * 128];     // [stage]
   uint8_t Xw[kQ * 128];       // w o x of the tile whose Sc is next
   uint8_t Hb[2][kN * 128];    // bf16 copy of the carried state, rows n
-  float cum[kQ];
-  float dd[kQ];
-  float vd[kQ];
+  float cumw[4][kQ];          // per mask-group warp: cumulative log2-decay,
+  float ddw[4][kQ];           //   step d_j,
+  float vdw[4][kQ];           //   column factor of the off-diagonal mask
   float a[4];                 // exp(cum_last) per tile, ring of four
-  float wsum[4];
   // Per-tile signals come in pairs indexed by tile parity (xready in fours);
   // the dependencies between roles bound every waiter's lag to less than one
   // lap of its ring, so no waiter can miss a phase.
   uint64_t full[2], empty[2], sdone[2], scdone[2], mready[2], stdone[2], yready[2], yfree[2];
   uint64_t xready[4];
-  uint64_t fin;
   uint32_t taddr;
   int abort;
 };
@@ -99,24 +99,17 @@ struct SsdTcParams {
   int *status;
 };
 
-// Named barrier for the mask group (id 1; 0 is __syncthreads).
-__device__ __forceinline__ void group_sync(int id) {
-  asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
-}
-// Group barrier that also ORs a predicate over the group.
-__device__ __forceinline__ bool group_any(int id, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(id)
-      : "memory");
-  return r != 0;
-}
-
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// One lane of the (fully active) warp is elected; the others get false.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 // a * b on two packed bfloat16 pairs, round to nearest even.
@@ -156,18 +149,12 @@ __device__ __forceinline__ bool wait1(SsdSmem &s, uint64_t *bar, uint32_t parity
   set_abort(s, status, code);
   return false;
 }
-// The mask group's wait: every thread waits (bounded), then the group votes.
-__device__ __forceinline__ bool waitg(SsdSmem &s, uint64_t *bar, uint32_t parity, int *status,
-                                      int code) {
-  bool ok = !aborted(s) && mbar_wait(bar, parity, kWaitLimit);
-  const bool fail = group_any(1, !ok);
-  if (fail && (threadIdx.x & 127) == 0) set_abort(s, status, code);
-  return !fail;
-}
-// A warp's wait: every lane waits (bounded), then the warp votes.
+// A warp's wait: every lane polls (bounded), then the warp votes, so its
+// lanes always take the same branch.  (Polling from lane 0 alone, with the
+// verdict broadcast, measured slower.)
 __device__ __forceinline__ bool waitw(SsdSmem &s, uint64_t *bar, uint32_t parity, int *status,
                                       int code) {
-  bool ok = !aborted(s) && mbar_wait(bar, parity, kWaitLimit);
+  const bool ok = !aborted(s) && mbar_wait(bar, parity, kWaitLimit);
   const bool fail = __any_sync(0xffffffffu, !ok);
   if (fail && (threadIdx.x & 31) == 0) set_abort(s, status, code);
   return !fail;
@@ -194,13 +181,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.empty[i], 1);
       mbar_init(&s.sdone[i], 1);
       mbar_init(&s.scdone[i], 1);
-      mbar_init(&s.mready[i], 1);
+      mbar_init(&s.mready[i], 4);  // one arrival per mask-group warp
       mbar_init(&s.stdone[i], 4);  // one arrival per state-group warp
       mbar_init(&s.yready[i], 1);
       mbar_init(&s.yfree[i], 4);   // one arrival per output-group warp
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&s.xready[i], 1);
-    mbar_init(&s.fin, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&s.xready[i], 4);
     s.abort = 0;
     fence_mbar_init();
   }
@@ -257,116 +243,161 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t id_S = idesc_bf16_f32(128, 128, false, false);
-      const uint32_t id_Y = idesc_bf16_f32(128, 64, false, true);
-      const uint32_t id_Sc = idesc_bf16_f32(128, 64, true, true);
-      auto mma_S = [&](int c) {  // S(c) = C B^T into S[c & 1]
-        const int st = c & 1;
-        const uint32_t c0 = smem_u32(s.C[st][0]), b0 = smem_u32(s.B[st][0]);
-        tc_fence_after();
+    // The whole warp runs the loop (waits, descriptors: warp-uniform); one
+    // elected lane issues the tcgen05 operations.
+    const bool leader = elect_one();
+    const uint32_t id_S = idesc_bf16_f32(128, 128, false, false);
+    const uint32_t id_Y = idesc_bf16_f32(128, 64, false, true);
+    const uint32_t id_Sc = idesc_bf16_f32(128, 64, true, true);
+    // K-major C / B for S (16-byte K steps inside a slab, slabs 16 KB apart),
+    // MN-major B / x / w o x / state copy (2 KB per 16-row K step).
+    const uint64_t dCk[2] = {smem_desc(smem_u32(s.C[0][0]), 16, 1024, kSwizzle128B),
+                             smem_desc(smem_u32(s.C[1][0]), 16, 1024, kSwizzle128B)};
+    const uint64_t dBk[2] = {smem_desc(smem_u32(s.B[0][0]), 16, 1024, kSwizzle128B),
+                             smem_desc(smem_u32(s.B[1][0]), 16, 1024, kSwizzle128B)};
+    const uint64_t dBm[2] = {smem_desc(smem_u32(s.B[0][0]), kQ * 128, 1024, kSwizzle128B),
+                             smem_desc(smem_u32(s.B[1][0]), kQ * 128, 1024, kSwizzle128B)};
+    const uint64_t dX[2] = {smem_desc(smem_u32(s.X[0]), kQ * 128, 1024, kSwizzle128B),
+                            smem_desc(smem_u32(s.X[1]), kQ * 128, 1024, kSwizzle128B)};
+    const uint64_t dXw = smem_desc(smem_u32(s.Xw), kQ * 128, 1024, kSwizzle128B);
+    const uint64_t dH[2] = {smem_desc(smem_u32(s.Hb[0]), kN * 128, 1024, kSwizzle128B),
+                            smem_desc(smem_u32(s.Hb[1]), kN * 128, 1024, kSwizzle128B)};
+    // (descriptor start addresses are in 16-byte units in the low 14 bits;
+    // every operand lies below 232448 bytes, so adding an offset never
+    // carries out of the field)
+    uint64_t *last_bar = nullptr;  // barrier and phase parity of the last commit
+    uint32_t last_par = 0;
+    auto mma_S = [&](int c) {  // S(c) = C B^T into S[c & 1]
+      const int st = c & 1;
+      tc_fence_after();
+      if (leader) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t ko = (k >> 2) * (kQ * 128) + (k & 3) * 32;
-          mma_ss(tb + kColS + 128 * st, smem_desc(c0 + ko, 16, 1024, kSwizzle128B),
-                 smem_desc(b0 + ko, 16, 1024, kSwizzle128B), id_S, k > 0);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ko = ((kk >> 2) * (kQ * 128) + (kk & 3) * 32) >> 4;
+          mma_ss(tb + kColS + 128 * st, dCk[st] + ko, dBk[st] + ko, id_S, kk > 0);
         }
         mma_commit(&s.sdone[st]);
-      };
-      bool ok = nch > 0 && wait1(s, &s.full[0], 0, p.status, 2);
-      if (ok) mma_S(0);
-      for (int c = 0; ok && c < nch; ++c) {
-        const int k = c & 1;
-        const uint32_t ph = (c >> 1) & 1;
-        // Sc(c) = B^T (w o x): needs w o x of tile c
-        if (!wait1(s, &s.xready[c & 3], (c >> 2) & 1, p.status, 3)) break;
-        tc_fence_after();
-        {
-          const uint32_t b0 = smem_u32(s.B[k][0]), xw = smem_u32(s.Xw);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tb + kColSc + 64 * k, smem_desc(b0 + kk * 2048, kQ * 128, 1024, kSwizzle128B),
-                   smem_desc(xw + kk * 2048, kQ * 128, 1024, kSwizzle128B), id_Sc, kk > 0);
-          mma_commit(&s.scdone[k]);
-        }
-        // S(c+1), as soon as its tile has landed
-        if (c + 1 < nch) {
-          if (!wait1(s, &s.full[(c + 1) & 1], ((c + 1) >> 1) & 1, p.status, 4)) break;
-          mma_S(c + 1);
-        }
-        // Y(c) = M x + (e o C) h_prev: needs the mask group's operands, the
-        // state of tile c-1 in Hb, and Y[k] read out by the output group
-        if (!wait1(s, &s.mready[k], ph, p.status, 5)) break;
-        if (c >= 1 && !wait1(s, &s.stdone[k ^ 1], ((c - 1) >> 1) & 1, p.status, 6)) break;
-        if (c >= 2 && !wait1(s, &s.yfree[k], ((c - 2) >> 1) & 1, p.status, 7)) break;
-        tc_fence_after();
-        {
-          const uint32_t x0 = smem_u32(s.X[k]), hb = smem_u32(s.Hb[k ^ 1]);
-          const uint32_t acol = kColS + 128 * k, dcol = kColY + 64 * k;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tb + dcol, tb + acol + 8 * kk,
-                   smem_desc(x0 + kk * 2048, kQ * 128, 1024, kSwizzle128B), id_Y, kk > 0);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tb + dcol, tb + acol + 64 + 8 * kk,
-                   smem_desc(hb + kk * 2048, kN * 128, 1024, kSwizzle128B), id_Y, true);
-          mma_commit(&s.yready[k]);
-          mma_commit(&s.empty[k]);
-        }
       }
-      // Leave no MMA in flight before TMEM is freed.
-      mma_commit(&s.fin);
-      mbar_wait(&s.fin, 0, kWaitLimit);
+      __syncwarp();
+      last_bar = &s.sdone[st];
+      last_par = (c >> 1) & 1;
+    };
+    bool ok = nch > 0 && waitw(s, &s.full[0], 0, p.status, 2);
+    if (ok) mma_S(0);
+    for (int c = 0; ok && c < nch; ++c) {
+      const int k = c & 1;
+      const uint32_t ph = (c >> 1) & 1;
+      // Sc(c) = B^T (w o x): needs w o x of tile c
+      if (!waitw(s, &s.xready[c & 3], (c >> 2) & 1, p.status, 3)) break;
+      tc_fence_after();
+      if (leader) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tb + kColSc + 64 * k, dBm[k] + kk * 128, dXw + kk * 128, id_Sc, kk > 0);
+        mma_commit(&s.scdone[k]);
+      }
+      __syncwarp();
+      last_bar = &s.scdone[k];
+      last_par = ph;
+      // S(c+1), as soon as its tile has landed
+      if (c + 1 < nch) {
+        if (!waitw(s, &s.full[k ^ 1], ((c + 1) >> 1) & 1, p.status, 4)) break;
+        mma_S(c + 1);
+      }
+      // Y(c) = M x + (e o C) h_prev: needs the mask group's operands, the
+      // state of tile c-1 in Hb, and Y[k] read out by the output group
+      if (!waitw(s, &s.mready[k], ph, p.status, 5)) break;
+      if (c >= 1 && !waitw(s, &s.stdone[k ^ 1], ((c - 1) >> 1) & 1, p.status, 6)) break;
+      if (c >= 2 && !waitw(s, &s.yfree[k], ((c - 2) >> 1) & 1, p.status, 7)) break;
+      tc_fence_after();
+      if (leader) {
+        const uint32_t acol = tb + kColS + 128 * k, dcol = tb + kColY + 64 * k;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(dcol, acol + 8 * kk, dX[k] + kk * 128, id_Y, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(dcol, acol + 64 + 8 * kk, dH[k ^ 1] + kk * 128, id_Y, true);
+        mma_commit(&s.yready[k]);
+        mma_commit(&s.empty[k]);
+      }
+      __syncwarp();
+      last_bar = &s.empty[k];
+      last_par = ph;
     }
+    // Leave no MMA in flight before TMEM is freed: wait (bounded) for the
+    // barrier of the last commit issued, which tracks every earlier MMA.
+    if (lane == 0 && last_bar) mbar_wait(last_bar, last_par, kWaitLimit);
     __syncwarp();
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ mask group
-    const int i = tid - 128;  // token of the tile; TMEM lane i
+    // Each warp works on its own 32 rows and keeps its own copy of the
+    // tile's per-token factors, so the four warps never wait for each other;
+    // they meet only in the four-count xready and mready barriers.
     const int mw = warp - 4;
+    const int i = 32 * mw + lane;  // token of the tile; TMEM lane i
     const float A2 = p.A[hd] * kLog2e;
     const float bias = p.dt_bias ? p.dt_bias[hd] : 0.f;
     const float Dh = p.D ? p.D[hd] : 0.f;
     const bool softplus_on = p.flags & 1u;
-    float dt_next = i < L ? ld(p.dt + (b * L + i) * H + hd) : 0.f;
+    float *cumw = s.cumw[mw], *ddw = s.ddw[mw], *vdw = s.vdw[mw];
+    // lane l handles tokens 4l .. 4l+3 of the tile in the prologue; their dt
+    // is fetched a tile ahead and kept as raw bfloat16 bits until used
+    const uint16_t *dtb = reinterpret_cast<const uint16_t *>(p.dt);
+    uint32_t dtraw[4];
+    auto fetch_dt = [&](int c) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int64_t t = (int64_t)c * kQ + 4 * lane + q;
+        dtraw[q] = t < L ? (uint32_t)dtb[(b * L + t) * H + hd] : 0u;
+      }
+    };
+    fetch_dt(0);
     for (int c = 0; c < nch; ++c) {
       const int k = c & 1;
       const int64_t t0 = (int64_t)c * kQ;
       const int valid = (int)(L - t0 < kQ ? L - t0 : kQ);
-      // step, log2-decay and its inclusive sum over the tile (needs only dt,
-      // so it runs while the tile's TMA is in flight)
-      float d = 0.f;
-      if (i < valid) {
-        d = dt_next + bias;
-        if (softplus_on) d = softplus_sfu(d);
+      // step, log2-decay and inclusive sums over the whole tile (needs only
+      // dt, so it runs while the tile's TMA is in flight)
+      float d4[4], p4[4];
+      float run = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float d = 0.f;
+        if (4 * lane + q < valid) {
+          d = __uint_as_float(dtraw[q] << 16) + bias;
+          if (softplus_on) d = softplus_sfu(d);
+        }
+        d4[q] = d;
+        run += d * A2;
+        p4[q] = run;
       }
-      if (t0 + kQ + i < L) dt_next = ld(p.dt + (b * L + t0 + kQ + i) * H + hd);
-      float cs = d * A2;
+      float incl = run;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
-        const float v = __shfl_up_sync(0xffffffffu, cs, off);
-        if (lane >= off) cs += v;
+        const float v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
       }
-      if (lane == 31) s.wsum[mw] = cs;
-      group_sync(1);
-      float total = 0.f;
+      const float total = __shfl_sync(0xffffffffu, incl, 31);
+      const float excl = incl - run;
+      // cum at the last token of each 32-token block (lanes 7, 15, 23, 31)
+      const float blk_end = __shfl_sync(0xffffffffu, incl, (lane & ~7) | 7);
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float v = s.wsum[w];
-        if (w < mw) cs += v;
-        total += v;
+      for (int q = 0; q < 4; ++q) {
+        const float cq = excl + p4[q];
+        cumw[4 * lane + q] = cq;
+        ddw[4 * lane + q] = d4[q];
+        vdw[4 * lane + q] = ex2(blk_end - cq) * d4[q];
       }
-      s.cum[i] = cs;
-      s.dd[i] = d;
-      if (i == 0) s.a[c & 3] = ex2(total);
-      group_sync(1);
-      s.vd[i] = ex2(s.cum[mw * 32 + 31] - cs) * d;
+      if (mw == 0 && lane == 0) s.a[c & 3] = ex2(total);
+      __syncwarp();
+      const float cs = cumw[i];
       const float e_i = ex2(cs);
-      const float w_i = ex2(total - cs) * d;
-      // w o x (row i), the B operand of Sc(c): x of tile c has landed and
-      // Sc(c-1) is done with the buffer
-      if (!waitg(s, &s.full[k], (c >> 1) & 1, p.status, 8)) break;
-      if (c >= 1 && !waitg(s, &s.scdone[k ^ 1], ((c - 1) >> 1) & 1, p.status, 9)) break;
+      const float w_i = ex2(total - cs) * ddw[i];
+      // w o x (rows of this warp), the B operand of Sc(c): x of tile c has
+      // landed and Sc(c-1) is done with the buffer
+      if (!waitw(s, &s.full[k], (c >> 1) & 1, p.status, 8)) break;
+      if (c >= 1 && !waitw(s, &s.scdone[k ^ 1], ((c - 1) >> 1) & 1, p.status, 9)) break;
       {
         const uint32_t w2 = pack_bf16x2(w_i, w_i);
 #pragma unroll
@@ -377,11 +408,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       fence_async_smem();
-      group_sync(1);
-      if (i == 0) mbar_arrive(&s.xready[c & 3]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.xready[c & 3]);
+      // next tile's dt, issued after the proxy fence so the fence never
+      // waits for it; it has the rest of this tile to arrive
+      if (c + 1 < nch) fetch_dt(c + 1);
       // masked S -> bf16, written over S's first 64 columns as S is read,
       // 32 columns at a time
-      if (!waitg(s, &s.sdone[k], (c >> 1) & 1, p.status, 10)) break;
+      if (!waitw(s, &s.sdone[k], (c >> 1) & 1, p.status, 10)) break;
       tc_fence_after();
       const uint32_t col = kColS + 128 * k;
 #pragma unroll 1
@@ -399,8 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (J < mw) {
           // below the diagonal: S_ij * exp2(cum_i - cum_r) * vd_j, r the
           // block's last token; both factors <= 1
-          const float u = ex2(cs - s.cum[32 * J + 31]);
-          const float4 *vd4 = reinterpret_cast<const float4 *>(s.vd + 32 * J);
+          const float u = ex2(cs - cumw[32 * J + 31]);
+          const float4 *vd4 = reinterpret_cast<const float4 *>(vdw + 32 * J);
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const float4 v = vd4[q];
@@ -415,11 +449,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           // diagonal block: S_ij * exp2(cum_i - cum_j) * d_j for j <= i, + D at j = i
-          const float4 *c4 = reinterpret_cast<const float4 *>(s.cum + 32 * J);
-          const float4 *d4 = reinterpret_cast<const float4 *>(s.dd + 32 * J);
+          const float4 *c4 = reinterpret_cast<const float4 *>(cumw + 32 * J);
+          const float4 *d4p = reinterpret_cast<const float4 *>(ddw + 32 * J);
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const float4 cj = c4[q], dj = d4[q];
+            const float4 cj = c4[q], dj = d4p[q];
             const float cjs[4] = {cj.x, cj.y, cj.z, cj.w}, djs[4] = {dj.x, dj.y, dj.z, dj.w};
             float f[4];
 #pragma unroll
@@ -456,8 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      group_sync(1);
-      if (i == 0) mbar_arrive(&s.mready[k]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.mready[k]);
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ state group
