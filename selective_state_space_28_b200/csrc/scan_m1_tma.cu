@@ -393,6 +393,7 @@ template <int N, typename T, bool HZ>
 cudaError_t launch_v(const M1Params &p, cudaStream_t s) {
   if (p.states) return launch_tma<N, T, 16, HZ, 0, 4, true>(p, s);
   // variant = 4 * (packed) + 2 * (two groups per iteration) + (2 states per lane)
+  const bool ok32 = p.G == 1 || (p.C / p.G) % 32 == 0;
   switch (p.variant) {
     case 0: return launch_tma<N, T, 16, HZ, 0, 4, false, false, 1>(p, s);
     case 1: return launch_tma<N, T, 16, HZ, 0, 2, false, false, 1>(p, s);
@@ -403,11 +404,20 @@ cudaError_t launch_v(const M1Params &p, cudaStream_t s) {
     case 6: return launch_tma<N, T, 16, HZ, 0, 4, false, true, 2>(p, s);
     case 7: return launch_tma<N, T, 16, HZ, 0, 2, false, true, 2>(p, s);
     case 8: return launch_tma<N, T, 16, HZ, 1, 4, false, true, 1>(p, s);
-    case 9: return launch_tma<N, T, 16, HZ, 0, 8, false, true, 1>(p, s);
-    case 10:  // 32-channel tiles: a tile must not straddle two B/C groups
-      if (p.G == 1 || (p.C / p.G) % 32 == 0) return launch_tma<N, T, 32, HZ, 0, 16, false, true, 1>(p, s);
-      return launch_tma<N, T, 16, HZ, 0, 8, false, true, 1>(p, s);
-    case 11: return launch_tma<N, T, 16, HZ, 0, 8, false, false, 1>(p, s);
+    // 9..12: 32-channel tiles (a tile must not straddle two B/C groups,
+    // else the default form runs)
+    case 9:
+      if (ok32) return launch_tma<N, T, 32, HZ, 0, 4, false, true, 1>(p, s);
+      break;
+    case 10:
+      if (ok32) return launch_tma<N, T, 32, HZ, 0, 8, false, true, 1>(p, s);
+      break;
+    case 11:
+      if (ok32) return launch_tma<N, T, 32, HZ, 0, 2, false, true, 1>(p, s);
+      break;
+    case 12:
+      if (ok32) return launch_tma<N, T, 32, HZ, 1, 4, false, true, 1>(p, s);
+      break;
   }
   return launch_tma<N, T, 16, HZ, 0, 2, false, true, 1>(p, s);
 }
