@@ -23,10 +23,11 @@
 //                 Y  = M x + (e o C) h_prev  A = M and e o C from TMEM, both
 //                                            held in S's columns (two buffers)
 //               issued per tile in the order Sc(c), S(c+1), Y(c).
-//   warps 4-7   mask group, thread = token (each warp also recomputes the
-//               whole tile's cumulative decay, so the warps run unsynchronised):
-//               the tile's step, cumulative decay and weights, w o x, then
-//               the mask applied to S as it is read
+//   warps 4-7 and 14-17   mask group, thread = token, two warps per TMEM
+//               lane quarter each taking half of every row's work (each warp
+//               also recomputes the whole tile's cumulative decay, so the
+//               warps run unsynchronised): the tile's step, cumulative decay
+//               and weights, w o x, then the mask applied to S as it is read
 //               from TMEM (D on its diagonal, so Y holds D x), and the row-
 //               scaled C, e_i C_i with e_i = exp(cum_i), both written back as
 //               the bf16 A operand of Y.  The mask exp(cum_i - cum_j) d_j is
@@ -62,7 +63,7 @@ using namespace sm100;
 constexpr int kQ = 128;   // tokens per tile
 constexpr int kN = 128;   // state size
 constexpr int kP = 64;    // head dim
-constexpr int kThreads = 448;
+constexpr int kThreads = 576;  // 18 warps
 constexpr long long kWaitLimit = 2000000000ll;  // cycles (about a second)
 
 // TMEM columns: S[2] (fp32 S; then masked S in the first 64 columns and e o C
@@ -76,9 +77,9 @@ struct __align__(1024) SsdSmem {
   uint8_t X[2][kQ * 128];     // [stage]
   uint8_t Xw[kQ * 128];       // w o x of the tile whose Sc is next
   uint8_t Hb[2][kN * 128];    // bf16 copy of the carried state, rows n
-  float cumw[4][kQ];          // per mask-group warp: cumulative log2-decay,
-  float ddw[4][kQ];           //   step d_j,
-  float vdw[4][kQ];           //   column factor of the off-diagonal mask
+  float cumw[8][kQ];          // per mask-group warp: cumulative log2-decay,
+  float ddw[8][kQ];           //   step d_j,
+  float vdw[8][kQ];           //   column factor of the off-diagonal mask
   float a[4];                 // exp(cum_last) per tile, ring of four
   // Per-tile signals come in pairs indexed by tile parity (xready in fours);
   // the dependencies between roles bound every waiter's lag to less than one
@@ -88,6 +89,19 @@ struct __align__(1024) SsdSmem {
   uint32_t taddr;
   int abort;
 };
+
+// Packed-bf16 TMEM columns (within an S buffer) of Y's A operand.  The mask
+// for tokens 32 J + 16 h .. + 16 (K step 2 J + h of M x), written by the
+// mask warp of half h, sits inside the S columns that warp itself read
+// (its halves of fp32 blocks 0 and 1); e o C for states 16 kk .. + 16 (K
+// step kk of (e o C) h_prev) sits inside the S columns the warp of half
+// kk / 4 read in blocks 2 and 3.
+__host__ __device__ constexpr uint32_t mask_col(int J, int h) {
+  return 32u * (uint32_t)(J >> 1) + 16u * (uint32_t)h + 8u * (uint32_t)(J & 1);
+}
+__host__ __device__ constexpr uint32_t ec_col(int kk) {
+  return 64u + 16u * (uint32_t)(kk >> 2) + 32u * (uint32_t)((kk >> 1) & 1) + 8u * (uint32_t)(kk & 1);
+}
 
 struct SsdTcParams {
   int64_t batch, L, H, G;
@@ -154,7 +168,9 @@ __device__ __forceinline__ bool wait1(SsdSmem &s, uint64_t *bar, uint32_t parity
 // verdict broadcast, measured slower.)
 __device__ __forceinline__ bool waitw(SsdSmem &s, uint64_t *bar, uint32_t parity, int *status,
                                       int code) {
-  const bool ok = !aborted(s) && mbar_wait(bar, parity, kWaitLimit);
+  // (no abort-flag read on this path: a role that gave up stops arriving,
+  // and every wait on it runs out by itself)
+  const bool ok = mbar_wait(bar, parity, kWaitLimit);
   const bool fail = __any_sync(0xffffffffu, !ok);
   if (fail && (threadIdx.x & 31) == 0) set_abort(s, status, code);
   return !fail;
@@ -181,12 +197,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.empty[i], 1);
       mbar_init(&s.sdone[i], 1);
       mbar_init(&s.scdone[i], 1);
-      mbar_init(&s.mready[i], 4);  // one arrival per mask-group warp
+      mbar_init(&s.mready[i], 8);  // one arrival per mask-group warp
       mbar_init(&s.stdone[i], 4);  // one arrival per state-group warp
       mbar_init(&s.yready[i], 1);
       mbar_init(&s.yfree[i], 4);   // one arrival per output-group warp
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&s.xready[i], 4);
+    for (int i = 0; i < 4; ++i) mbar_init(&s.xready[i], 8);
     s.abort = 0;
     fence_mbar_init();
   }
@@ -314,10 +330,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t acol = tb + kColS + 128 * k, dcol = tb + kColY + 64 * k;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(dcol, acol + 8 * kk, dX[k] + kk * 128, id_Y, kk > 0);
+          mma_ts(dcol, acol + mask_col(kk >> 1, kk & 1), dX[k] + kk * 128, id_Y, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(dcol, acol + 64 + 8 * kk, dH[k ^ 1] + kk * 128, id_Y, true);
+          mma_ts(dcol, acol + ec_col(kk), dH[k ^ 1] + kk * 128, id_Y, true);
         mma_commit(&s.yready[k]);
         mma_commit(&s.empty[k]);
       }
@@ -329,18 +345,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     // barrier of the last commit issued, which tracks every earlier MMA.
     if (lane == 0 && last_bar) mbar_wait(last_bar, last_par, kWaitLimit);
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
+  } else if ((warp >= 4 && warp < 8) || warp >= 14) {
     // ------------------------------------------------------------ mask group
-    // Each warp works on its own 32 rows and keeps its own copy of the
-    // tile's per-token factors, so the four warps never wait for each other;
-    // they meet only in the four-count xready and mready barriers.
-    const int mw = warp - 4;
-    const int i = 32 * mw + lane;  // token of the tile; TMEM lane i
+    // Two warps per TMEM lane quarter (warps 4-7 and 14-17): each takes 32
+    // rows and, of every row, half the work (16 of each 32-column block of
+    // the mask, one 64-state slab of e o C, half of w o x).  Each warp keeps
+    // its own copy of the tile's per-token factors, so the eight warps never
+    // wait for each other; they meet only in the eight-count xready and
+    // mready barriers.
+    const int half = warp >= 14 ? 1 : 0;
+    const int mw = warp & 3;           // lane quarter = row block
+    const int mg = 4 * half + mw;      // this warp's factor copy
+    const int i = 32 * mw + lane;      // token of the tile; TMEM lane i
     const float A2 = p.A[hd] * kLog2e;
     const float bias = p.dt_bias ? p.dt_bias[hd] : 0.f;
     const float Dh = p.D ? p.D[hd] : 0.f;
     const bool softplus_on = p.flags & 1u;
-    float *cumw = s.cumw[mw], *ddw = s.ddw[mw], *vdw = s.vdw[mw];
+    float *cumw = s.cumw[mg], *ddw = s.ddw[mg], *vdw = s.vdw[mg];
     // lane l handles tokens 4l .. 4l+3 of the tile in the prologue; their dt
     // is fetched a tile ahead and kept as raw bfloat16 bits until used
     const uint16_t *dtb = reinterpret_cast<const uint16_t *>(p.dt);
@@ -389,19 +410,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         ddw[4 * lane + q] = d4[q];
         vdw[4 * lane + q] = ex2(blk_end - cq) * d4[q];
       }
-      if (mw == 0 && lane == 0) s.a[c & 3] = ex2(total);
+      if (mg == 0 && lane == 0) s.a[c & 3] = ex2(total);
       __syncwarp();
       const float cs = cumw[i];
       const float e_i = ex2(cs);
       const float w_i = ex2(total - cs) * ddw[i];
-      // w o x (rows of this warp), the B operand of Sc(c): x of tile c has
-      // landed and Sc(c-1) is done with the buffer
+      // w o x (this warp's rows, half the columns), the B operand of Sc(c):
+      // x of tile c has landed and Sc(c-1) is done with the buffer
       if (!waitw(s, &s.full[k], (c >> 1) & 1, p.status, 8)) break;
       if (c >= 1 && !waitw(s, &s.scdone[k ^ 1], ((c - 1) >> 1) & 1, p.status, 9)) break;
       {
         const uint32_t w2 = pack_bf16x2(w_i, w_i);
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int cc = 4 * half + c4;
           const uint4 v = *reinterpret_cast<const uint4 *>(s.X[k] + sw128(i, cc));
           *reinterpret_cast<uint4 *>(s.Xw + sw128(i, cc)) =
               make_uint4(bmul2(v.x, w2), bmul2(v.y, w2), bmul2(v.z, w2), bmul2(v.w, w2));
@@ -413,30 +435,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       // next tile's dt, issued after the proxy fence so the fence never
       // waits for it; it has the rest of this tile to arrive
       if (c + 1 < nch) fetch_dt(c + 1);
-      // masked S -> bf16, written over S's first 64 columns as S is read,
-      // 32 columns at a time
+      // masked S -> bf16.  Of each 32-column block J this warp takes the 16
+      // columns from 32 J + 16 half.  Its packed results go only where this
+      // warp itself has already read S (its own halves of blocks 0 and 1),
+      // so the pair never overwrites what the other still has to read:
+      // block J -> packed columns mask_col(J, half) .. + 8, and the MMA
+      // walks its K steps through the same map.
       if (!waitw(s, &s.sdone[k], (c >> 1) & 1, p.status, 10)) break;
       tc_fence_after();
       const uint32_t col = kColS + 128 * k;
 #pragma unroll 1
       for (int J = 0; J < 4; ++J) {
-        uint32_t r[32];
-        uint32_t m[16];
+        const int j0 = 32 * J + 16 * half;
+        uint32_t r[16];
+        uint32_t m[8];
         if (J <= mw) {
-          tmem_ld16(tb + lane_base + col + 32 * J, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-          tmem_ld16(tb + lane_base + col + 32 * J + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+          tmem_ld16(tb + lane_base + col + j0, r);
           tmem_ld_wait();
         }
         if (J > mw) {
 #pragma unroll
-          for (int q = 0; q < 16; ++q) m[q] = 0u;
+          for (int q = 0; q < 8; ++q) m[q] = 0u;
         } else if (J < mw) {
           // below the diagonal: S_ij * exp2(cum_i - cum_r) * vd_j, r the
           // block's last token; both factors <= 1
           const float u = ex2(cs - cumw[32 * J + 31]);
-          const float4 *vd4 = reinterpret_cast<const float4 *>(vdw + 32 * J);
+          const float4 *vd4 = reinterpret_cast<const float4 *>(vdw + j0);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
+          for (int q = 0; q < 4; ++q) {
             const float4 v = vd4[q];
             const f2 a = mul2(mul2(mk2(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])),
                                    mk2(v.x, v.y)),
@@ -449,16 +475,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           // diagonal block: S_ij * exp2(cum_i - cum_j) * d_j for j <= i, + D at j = i
-          const float4 *c4 = reinterpret_cast<const float4 *>(cumw + 32 * J);
-          const float4 *d4p = reinterpret_cast<const float4 *>(ddw + 32 * J);
+          const float4 *c4 = reinterpret_cast<const float4 *>(cumw + j0);
+          const float4 *d4p = reinterpret_cast<const float4 *>(ddw + j0);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
+          for (int q = 0; q < 4; ++q) {
             const float4 cj = c4[q], dj = d4p[q];
             const float cjs[4] = {cj.x, cj.y, cj.z, cj.w}, djs[4] = {dj.x, dj.y, dj.z, dj.w};
             float f[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int j = 32 * J + 4 * q + e;
+              const int j = j0 + 4 * q + e;
               const float sv = __uint_as_float(r[4 * q + e]);
               f[e] = (j <= i) ? sv * (ex2(cs - cjs[e]) * djs[e]) + (j == i ? Dh : 0.f) : 0.f;
             }
@@ -466,26 +492,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             m[2 * q + 1] = pack_bf16x2(f[2], f[3]);
           }
         }
-        tmem_st16(tb + lane_base + col + 16 * J, m);
+        tmem_st8(tb + lane_base + col + mask_col(J, half), m);
       }
-      // e_i C_i -> bf16, into columns 64..127 (S there has been read)
+      // e_i C_i -> bf16 for the states of slab `half`: 32 packed columns,
+      // again only where this warp read S (its halves of blocks 2 and 3:
+      // ec_col(2 c4 + kq) for K step kq of the slab); a warp that skipped
+      // those blocks writes columns nobody reads S from.
       {
         const uint32_t e2 = pack_bf16x2(e_i, e_i);
 #pragma unroll
-        for (int hs = 0; hs < 2; ++hs) {
+        for (int c4 = 0; c4 < 2; ++c4) {
+          uint32_t m[16];
 #pragma unroll
-          for (int c4 = 0; c4 < 2; ++c4) {
-            uint32_t m[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 v = *reinterpret_cast<const uint4 *>(s.C[k][hs] + sw128(i, 4 * c4 + q));
-              m[4 * q] = bmul2(v.x, e2);
-              m[4 * q + 1] = bmul2(v.y, e2);
-              m[4 * q + 2] = bmul2(v.z, e2);
-              m[4 * q + 3] = bmul2(v.w, e2);
-            }
-            tmem_st16(tb + lane_base + col + 64 + 32 * hs + 16 * c4, m);
+          for (int q = 0; q < 4; ++q) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(s.C[k][half] + sw128(i, 4 * c4 + q));
+            m[4 * q] = bmul2(v.x, e2);
+            m[4 * q + 1] = bmul2(v.y, e2);
+            m[4 * q + 2] = bmul2(v.z, e2);
+            m[4 * q + 3] = bmul2(v.w, e2);
           }
+          tmem_st16(tb + lane_base + col + ec_col(4 * half + 2 * c4), m);
         }
       }
       tmem_st_wait();
@@ -515,18 +541,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float a_c = s.a[c & 3];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t r[32];
-        tmem_ld16(tb + lane_base + kColSc + 64 * k + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-        tmem_ld16(tb + lane_base + kColSc + 64 * k + 32 * hh + 16,
-                  *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+      for (int hh = 0; hh < 4; ++hh) {
+        uint32_t r[16];
+        tmem_ld16(tb + lane_base + kColSc + 64 * k + 16 * hh, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const f2 hn = fma2(mk2(a_c, a_c), mk2(h[32 * hh + j], h[32 * hh + j + 1]),
+        for (int j = 0; j < 16; j += 2) {
+          const f2 hn = fma2(mk2(a_c, a_c), mk2(h[16 * hh + j], h[16 * hh + j + 1]),
                              mk2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])));
-          h[32 * hh + j] = hn.x;
-          h[32 * hh + j + 1] = hn.y;
+          h[16 * hh + j] = hn.x;
+          h[16 * hh + j + 1] = hn.y;
         }
       }
       tc_fence_before();
@@ -566,31 +590,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t t = (int64_t)c * kQ + i;
       if (!waitw(s, &s.yready[k], (c >> 1) & 1, p.status, 13)) break;
       tc_fence_after();
-      uint32_t v[64];
+      __nv_bfloat16 *yp = p.y + ((b * L + t) * H + hd) * kP;
+      // two halves of 32 columns; Y[k] is released after the second load
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        tmem_ld16(tb + lane_base + kColY + 64 * k + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * q]));
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.yfree[k]);
-      if (t < L) {
-        __nv_bfloat16 *yp = p.y + ((b * L + t) * H + hd) * kP;
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t v[32];
+        tmem_ld16(tb + lane_base + kColY + 64 * k + 32 * hh, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+        tmem_ld16(tb + lane_base + kColY + 64 * k + 32 * hh + 16,
+                  *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+        tmem_ld_wait();
+        if (hh == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.yfree[k]);
+        }
+        if (t < L) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float o[8];
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int q = 4 * hh + q4;
+            float o[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) o[j] = __uint_as_float(v[8 * q + j]);
-          if (p.z) {
-            const uint32_t zw[4] = {zr[q].x, zr[q].y, zr[q].z, zr[q].w};
+            for (int j = 0; j < 8; ++j) o[j] = __uint_as_float(v[8 * q4 + j]);
+            if (p.z) {
+              const uint32_t zw[4] = {zr[q].x, zr[q].y, zr[q].z, zr[q].w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              o[2 * j] *= silu_tanh(bf16lo(zw[j]));
-              o[2 * j + 1] *= silu_tanh(bf16hi(zw[j]));
+              for (int j = 0; j < 4; ++j) {
+                o[2 * j] *= silu_tanh(bf16lo(zw[j]));
+                o[2 * j + 1] *= silu_tanh(bf16hi(zw[j]));
+              }
             }
+            st_cs_u4(yp + 8 * q, make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                            pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7])));
           }
-          st_cs_u4(yp + 8 * q, make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
-                                          pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7])));
         }
       }
       load_z(c + 1);
