@@ -418,6 +418,8 @@ cudaError_t launch_v(const M1Params &p, cudaStream_t s) {
     case 12:
       if (ok32) return launch_tma<N, T, 32, HZ, 1, 4, false, true, 1>(p, s);
       break;
+    case 13: return launch_tma<N, T, 16, HZ, 1, 2, false, true, 1>(p, s);
+    case 14: return launch_tma<N, T, 16, HZ, 1, 2, false, true, 2>(p, s);
   }
   return launch_tma<N, T, 16, HZ, 0, 2, false, true, 1>(p, s);
 }

@@ -21,14 +21,14 @@ bool all_aligned(Ps... ps) {
   return true;
 }
 
-// Variant of the pipelined Mamba-1 kernel (0..12, see scan_m1_tma.cu);
+// Variant of the pipelined Mamba-1 kernel (0..14, see scan_m1_tma.cu);
 // SSM_M1_VARIANT overrides the default for tuning.
 int m1_variant() {
   static int v = -1;
   if (v < 0) {
     const char *e = getenv("SSM_M1_VARIANT");
     v = e ? atoi(e) : 5;
-    if (v < 0 || v > 12) v = 5;
+    if (v < 0 || v > 14) v = 5;
   }
   return v;
 }
