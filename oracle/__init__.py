@@ -46,6 +46,7 @@ def _load():
             "orc_m2_step": [_I64] * 5 + [ctypes.c_uint32] + [_D] * 10,
             "orc_m2_quadratic": [_I64] * 6 + [_D] * 9,
             "orc_m1_quadratic": [_I64] * 5 + [_D] * 9,
+            "orc_conv1d": [_I64] * 4 + [_D] * 4 + [ctypes.c_int] + [_D] * 2,
         }.items():
             fn = getattr(lib, name)
             fn.argtypes = argtypes
@@ -174,6 +175,25 @@ def m1_quadratic(x, betas, B, C, A, D=None, z=None, h0=None):
     if rc:
         raise ValueError("orc_m1_quadratic failed: %d" % rc)
     return y
+
+
+def conv1d(x, w, bias=None, state=None, act=True):
+    """Causal depthwise convolution over tokens, then silu when act (the
+    mixers' conv1d: module tree, kernel W, padding W - 1, groups = channels;
+    "Mamba-2" "The mixer's values", "Mamba" tokentrails "Code").
+    x [b, L, C]; w [C, W]; bias [C]; state [b, C, W - 1] (inputs before the
+    sequence, oldest first) or None for zeros.  Returns (u [b, L, C],
+    state_out [b, C, W - 1])."""
+    x, w, bias, state = _f64(x), _f64(w), _f64(bias), _f64(state)
+    b, L, C = x.shape
+    W = w.shape[1]
+    u = np.zeros((b, L, C))
+    so = np.zeros((b, C, max(W - 1, 0)))
+    rc = _load().orc_conv1d(b, L, C, W, _p(x), _p(w), _p(bias), _p(state), int(bool(act)),
+                            _p(u), _p(so) if W > 1 else None)
+    if rc:
+        raise ValueError("orc_conv1d: bad arguments")
+    return u, so
 
 
 def softplus(v):

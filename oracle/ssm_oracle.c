@@ -420,3 +420,37 @@ int orc_m1_quadratic(int64_t batch, int64_t seqlen, int64_t channels,
     }
   return 0;
 }
+
+/* Causal depthwise convolution ("Mamba-2", module tree and "The mixer's
+ * values"; "Mamba", tokentrails, "Code"): the module's Conv1d with padding
+ * W - 1 on both ends and the output cut to the first L positions is, per
+ * channel, a weighted sum of the current input and the W - 1 before it,
+ * weight k multiplying the input W - 1 - k tokens back; inputs before the
+ * sequence start come from state_in (zero without one). */
+static double conv_in(const double *x, const double *state_in, int64_t b, int64_t L, int64_t Cc,
+                      int64_t W, int64_t c, int64_t tau) {
+  if (tau >= 0) return x[(b * L + tau) * Cc + c];
+  if (!state_in) return 0.0;
+  return state_in[(b * Cc + c) * (W - 1) + (W - 1) + tau];
+}
+
+int orc_conv1d(int64_t batch, int64_t seqlen, int64_t channels, int64_t width,
+               const double *x, const double *w, const double *bias,
+               const double *state_in, int act, double *u, double *state_out) {
+  const int64_t L = seqlen, Cc = channels, W = width;
+  if (batch < 0 || L < 0 || Cc <= 0 || W <= 0 || !w) return 1;
+  for (int64_t b = 0; b < batch; ++b)
+    for (int64_t c = 0; c < Cc; ++c) {
+      for (int64_t t = 0; t < L; ++t) {
+        double acc = bias ? bias[c] : 0.0;
+        for (int64_t k = 0; k < W; ++k)
+          acc += w[c * W + k] * conv_in(x, state_in, b, L, Cc, W, c, t - (W - 1) + k);
+        u[(b * L + t) * Cc + c] = act ? orc_silu(acc) : acc;
+      }
+      if (state_out)
+        for (int64_t j = 0; j < W - 1; ++j)
+          state_out[(b * Cc + c) * (W - 1) + j] =
+              conv_in(x, state_in, b, L, Cc, W, c, L - (W - 1) + j);
+    }
+  return 0;
+}

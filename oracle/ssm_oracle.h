@@ -18,6 +18,11 @@
  *   - "Mamba-2" (nnterp encyclopedia), "The mixer's values", "The hidden
  *     attention", "The state", "A zero step skips a token exactly".
  *   - "Falcon-Mamba" (nnterp encyclopedia), "Where the norms sit".
+ *   - The mixers' causal convolution: "Mamba-2" (nnterp encyclopedia), the
+ *     module tree (Conv1d, kernel 4, padding 3, groups = channels) and "The
+ *     mixer's values" (x, B, C = silu(conv1d(xBC)), causal, width 4);
+ *     "Mamba" (tokentrails lineage), "Code" (x = silu(causal_conv1d(x)),
+ *     depthwise, width 4).
  */
 #ifndef SSM_ORACLE_H
 #define SSM_ORACLE_H
@@ -88,6 +93,19 @@ int orc_m1_quadratic(int64_t batch, int64_t seqlen, int64_t channels,
                      const double *x, const double *betas, const double *z,
                      const double *B, const double *Cm, const double *A,
                      const double *D, const double *h0, double *y);
+
+/* Causal depthwise convolution over tokens, then silu when act != 0: the
+ * module tree's Conv1d(channels, channels, kernel W, padding W - 1,
+ * groups = channels) with its output cut to the input length, so
+ *   u[t, c] = bias[c] + sum_{k<W} w[c, k] * x[t - (W - 1) + k, c].
+ * x, u: [b, L, Cc]; w: [Cc, W]; bias: [Cc] or NULL (zero); state_in:
+ * [b, Cc, W - 1], the inputs of the W - 1 tokens before t = 0, oldest first,
+ * or NULL (zeros: a sequence start); state_out: [b, Cc, W - 1] or NULL, the
+ * last W - 1 inputs (state_in's entries when L < W - 1), so that a sequence
+ * cut in two and run with state_out -> state_in gives the same u. */
+int orc_conv1d(int64_t batch, int64_t seqlen, int64_t channels, int64_t width,
+               const double *x, const double *w, const double *bias,
+               const double *state_in, int act, double *u, double *state_out);
 
 /* Elementwise helpers exposed for the pins. */
 double orc_softplus(double v);

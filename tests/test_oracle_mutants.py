@@ -66,6 +66,20 @@ MUTANTS = {
         "        y[(b * heads + hd) * P + q] = yv;\n      }\n"
         "      for (int64_t n = 0; n < N; ++n)\n        for (int64_t q = 0; q < P; ++q)\n"
         "          S[n * P + q] = a * S[n * P + q] + d * Bg[n] * xh[q];"),
+    "conv_weight_reversed": ("acc += w[c * W + k] * conv_in(x, state_in, b, L, Cc, W, c, t - (W - 1) + k);",
+                             "acc += w[c * W + (W - 1 - k)] * conv_in(x, state_in, b, L, Cc, W, c, t - (W - 1) + k);"),
+    "conv_not_causal": ("acc += w[c * W + k] * conv_in(x, state_in, b, L, Cc, W, c, t - (W - 1) + k);",
+                        "acc += w[c * W + k] * conv_in(x, state_in, b, L, Cc, W, c, t - (W - 2) + k);"),
+    "conv_state_newest_first": ("return state_in[(b * Cc + c) * (W - 1) + (W - 1) + tau];",
+                                "return state_in[(b * Cc + c) * (W - 1) - 1 - tau];"),
+    "conv_silu_before_bias": ("        double acc = bias ? bias[c] : 0.0;\n        for (int64_t k = 0; k < W; ++k)\n"
+                              "          acc += w[c * W + k] * conv_in(x, state_in, b, L, Cc, W, c, t - (W - 1) + k);\n"
+                              "        u[(b * L + t) * Cc + c] = act ? orc_silu(acc) : acc;",
+                              "        double acc = 0.0;\n        for (int64_t k = 0; k < W; ++k)\n"
+                              "          acc += w[c * W + k] * conv_in(x, state_in, b, L, Cc, W, c, t - (W - 1) + k);\n"
+                              "        u[(b * L + t) * Cc + c] = (act ? orc_silu(acc) : acc) + (bias ? bias[c] : 0.0);"),
+    "conv_state_out_off_by_one": ("conv_in(x, state_in, b, L, Cc, W, c, L - (W - 1) + j);",
+                                  "conv_in(x, state_in, b, L, Cc, W, c, L - W + j);"),
 }
 
 
@@ -104,7 +118,7 @@ def test_mutant_is_caught(key):
         mlib = ctypes.CDLL(_build_mutant(src.replace(old, new), tmp, key))
         for name in ("orc_m1_scan", "orc_m2_scan", "orc_m1_step", "orc_m2_step",
                      "orc_m2_quadratic", "orc_m1_quadratic", "orc_softplus", "orc_silu",
-                     "orc_rms_rows"):
+                     "orc_rms_rows", "orc_conv1d"):
             getattr(mlib, name).argtypes = getattr(real, name).argtypes
             getattr(mlib, name).restype = getattr(real, name).restype
         caught = None

@@ -362,3 +362,95 @@ def test_page_state_sizes():
     conv2 = q["layers"] * (d_inner + 2 * q["groups"] * q["state"]) * (q["conv_width"] - 1) \
         * q["bytes_per_value"]
     assert round((ssm2 + conv2) / 2 ** 20) == q["state_mib_printed"]
+
+
+# ---------------------------------------------------------------- conv1d
+# The mixers' causal depthwise convolution ("Mamba-2" module tree: Conv1d,
+# kernel 4, padding 3, groups = channels; "The mixer's values" and "Mamba"
+# tokentrails "Code": silu(conv1d(.)), causal, width 4).
+
+def test_conv1d_matches_library_convolution():
+    # Per channel, a causal convolution is the first L terms of the full
+    # convolution with the kernel reversed (weight k multiplies the input
+    # W - 1 - k tokens back): numpy's convolve is an independent routine.
+    r = rng(40)
+    x, w, bias = r.standard_normal((2, 37, 6)), r.standard_normal((6, 4)), r.standard_normal(6)
+    u, _ = oracle.conv1d(x, w, bias, act=False)
+    for b in range(2):
+        for c in range(6):
+            ref = np.convolve(x[b, :, c], w[c, ::-1])[:37] + bias[c]
+            np.testing.assert_allclose(u[b, :, c], ref, rtol=0, atol=1e-12)
+
+
+def test_conv1d_matches_torch_module_layout():
+    # The module tree's layer itself: Conv1d(C, C, 4, padding=3, groups=C) on
+    # [b, C, L], output cut to the first L positions.
+    r = rng(41)
+    x, w, bias = r.standard_normal((2, 19, 5)), r.standard_normal((5, 4)), r.standard_normal(5)
+    u, _ = oracle.conv1d(x, w, bias, act=True)
+    xt = torch.tensor(x).transpose(1, 2)
+    ref = F.conv1d(xt, torch.tensor(w).unsqueeze(1), torch.tensor(bias), padding=3, groups=5)
+    ref = F.silu(ref[..., :19]).transpose(1, 2).numpy()
+    np.testing.assert_allclose(u, ref, rtol=0, atol=1e-12)
+
+
+def test_conv1d_impulse_response_orientation():
+    # One nonzero input at t0: the output at t0 + j is the weight that
+    # multiplies an input j tokens back, w[W - 1 - j]; nothing before t0.
+    w = np.array([[0.1, 0.2, 0.3, 0.4]])
+    x = np.zeros((1, 12, 1))
+    x[0, 5, 0] = 1.0
+    u, _ = oracle.conv1d(x, w, act=False)
+    assert np.all(u[0, :5, 0] == 0.0)
+    assert list(u[0, 5:9, 0]) == [0.4, 0.3, 0.2, 0.1]
+    assert np.all(u[0, 9:, 0] == 0.0)
+
+
+def test_conv1d_constant_input_from_a_cold_start():
+    # Constant input c with no history: the first W - 1 outputs see only the
+    # tokens since the start (partial sums of the newest weights), the rest
+    # the full sum.
+    w = np.array([[1.0, 2.0, 4.0, 8.0]])
+    x = np.full((1, 6, 1), 3.0)
+    u, st = oracle.conv1d(x, w, bias=np.array([0.5]), act=False)
+    assert list(u[0, :, 0]) == [0.5 + 24.0, 0.5 + 36.0, 0.5 + 42.0, 0.5 + 45.0, 45.5, 45.5]
+    assert list(st[0, 0]) == [3.0, 3.0, 3.0]
+
+
+def test_conv1d_split_and_carry_equals_full():
+    # The conv state carries the last W - 1 inputs: a sequence cut anywhere
+    # (also before W - 1 tokens) gives the same outputs, bit for bit.
+    r = rng(42)
+    x, w, bias = r.standard_normal((2, 23, 7)), r.standard_normal((7, 4)), r.standard_normal(7)
+    st0 = r.standard_normal((2, 7, 3))
+    u, st = oracle.conv1d(x, w, bias, state=st0)
+    for cut in (1, 2, 3, 10, 22):
+        u1, s1 = oracle.conv1d(x[:, :cut], w, bias, state=st0)
+        u2, s2 = oracle.conv1d(x[:, cut:], w, bias, state=s1)
+        assert np.array_equal(np.concatenate([u1, u2], axis=1), u)
+        assert np.array_equal(s2, st)
+
+
+def test_conv1d_state_is_the_history():
+    # Running one token at a time from a state equals running the whole
+    # sequence: the decode form of the same convolution.
+    r = rng(43)
+    x, w = r.standard_normal((1, 9, 3)), r.standard_normal((3, 4))
+    st = r.standard_normal((1, 3, 3))
+    u_full, st_full = oracle.conv1d(x, w, state=st)
+    s = st
+    for t in range(9):
+        u1, s = oracle.conv1d(x[:, t:t + 1], w, state=s)
+        assert np.array_equal(u1[:, 0], u_full[:, t])
+    assert np.array_equal(s, st_full)
+    # and the state is literally the last three inputs
+    assert np.array_equal(st_full[0], x[0, -3:].T)
+
+
+def test_conv1d_width_one_is_elementwise():
+    r = rng(44)
+    x, w, bias = r.standard_normal((2, 5, 4)), r.standard_normal((4, 1)), r.standard_normal(4)
+    u, st = oracle.conv1d(x, w, bias, act=True)
+    v = x * w[:, 0] + bias
+    np.testing.assert_allclose(u, v / (1 + np.exp(-v)), rtol=1e-15, atol=0)
+    assert st.shape == (2, 4, 0)
