@@ -46,7 +46,7 @@ def parse(argv=None):
                     help="measure only the headline workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["m1", "ssd", "decode", "decode_layer", "falcon"],
+    ap.add_argument("--only", choices=["m1", "ssd", "decode", "decode_layer", "falcon", "conv"],
                     help="run just one workload's timed loop (for profiling); prints its timing")
     return ap.parse_args(argv)
 
@@ -100,6 +100,17 @@ def ssd_flops(w):
     cb = nch * w.groups * 2 * Q * Q * w.state
     per_head = Q * (Q + 1) * w.head_dim + 2 * (2 * Q * w.state * w.head_dim)
     return cb + nch * w.heads * per_head
+
+
+def conv_bytes(w):
+    """x read and u written once in the I/O type, the float32 weights and
+    bias, and the carried conv state read and written."""
+    e = _esz(w.io)
+    W = w.extra.get("width", 4)
+    n = 2 * w.batch * w.seqlen * w.channels * e + (W + 1) * w.channels * 4
+    if w.extra.get("state", False):
+        n += 2 * w.batch * w.channels * (W - 1) * 4
+    return n
 
 
 def decode_bytes(w):
@@ -286,6 +297,29 @@ def bench_m1(w, K, W, dist, device, pk, seed_base):
             "launches_per_step": launches}
 
 
+def bench_conv(w, K, W, dist, device, pk, seed_base):
+    import torch
+    from selective_state_space_28_b200 import inputs as I
+    from selective_state_space_28_b200 import ops
+    nb = conv_bytes(w)
+    sets = []
+    for r in range(n_sets(nb)):
+        d = I.workload_inputs(w, device=device, seed=seed_base + 1000 * r)
+        d["u"] = torch.empty_like(d["x"])
+        d["state_out"] = torch.empty((w.batch, w.channels, w.extra.get("width", 4) - 1),
+                                     device=device)
+        sets.append(d)
+
+    def step(i):
+        d = sets[i % len(sets)]
+        ops.ssm_conv1d_fwd(d["x"], d["w"], d["bias"], d["state"], silu=True, u=d["u"],
+                           state_out=d["state_out"])
+    ms = timed(step, K, W, dist, device) / K
+    launch_ms = per_launch_ms(step, max(10, K), device)
+    return {"ms_per_step": ms, "bytes": nb, "launch_ms": launch_ms, "sets": len(sets),
+            "launches_per_step": 1}
+
+
 def bench_ssd(w, K, W, dist, device, pk, seed_base):
     import torch
     from selective_state_space_28_b200 import inputs as I
@@ -408,10 +442,11 @@ def run_only(args):
     pk = peaks()
     name = {"m1": HEADLINE, "ssd": "ssd_2p7b_b4_l4096_h80_p64_n128_bf16",
             "decode": "decode_2p7b_stack_b256", "decode_layer": "decode_2p7b_layer_b256",
-            "falcon": "m1_falcon_rms_b4_l8192_c8192_n16_bf16"}[args.only]
+            "falcon": "m1_falcon_rms_b4_l8192_c8192_n16_bf16",
+            "conv": "conv_2p7b_b4_l4096_c5376_bf16"}[args.only]
     w = I.WORKLOADS[name]
     fn = {"m1": bench_m1, "falcon": bench_m1, "ssd": bench_ssd, "decode": bench_decode,
-          "decode_layer": bench_decode}[args.only]
+          "decode_layer": bench_decode, "conv": bench_conv}[args.only]
     r = fn(w, args.steps, args.warmup, dist, device, pk, w.seed)
     print(json.dumps({"only": name, "ms_per_step": r["ms_per_step"],
                       "launch_ms": r["launch_ms"]}), flush=True)
@@ -476,6 +511,7 @@ def run_ours(args):
         wl[ws.name] = {
             "value": round(job_value(s["tokens"], dist.world, s["ms_per_step"]), 1),
             "unit": "tokens/s", "ms_per_step": round(s["ms_per_step"], 4),
+            "gpu_launches": s["launches_per_step"] * Ke,
             "gbs": round(s["bytes"] / (s["ms_per_step"] * 1e-3) / 1e9, 1),
             "roofline": {"bound": "tensor", "achieved": round(tf, 2),
                          "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
@@ -503,8 +539,17 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(ach / hbm, 4), "traffic": traffic_for("m1_scan_falcon"),
                          "note": "algorithmic bytes exclude the step-norm pre-pass re-read"}}
+        wc = I.WORKLOADS["conv_2p7b_b4_l4096_c5376_bf16"]
+        cv = bench_conv(wc, max(3, min(K, 20)), max(3, W), dist, device, pk,
+                        rank_seed(wc.seed, dist.rank))
+        ach = cv["bytes"] / (cv["launch_ms"] * 1e-3) / 1e9
+        wl[wc.name] = {
+            "value": round(job_value(cv["bytes"], dist.world, cv["ms_per_step"]) / 1e9, 2),
+            "unit": "GB/s", "ms_per_step": round(cv["ms_per_step"], 4),
+            "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
+                         "frac": round(ach / hbm, 4), "traffic": traffic_for("conv_2p7b"),
+                         "kernel": "conv1d_vec_kernel"}}
         out["workloads"] = wl
-        out["gpu_launches"] += (s["launches_per_step"] * Ke)
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline_m1(w)
     dist.close()

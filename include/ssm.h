@@ -7,6 +7,8 @@
  *   ssm_scan_fwd        Mamba-1 selective scan over a prompt.
  *   ssd_chunk_scan_fwd  Mamba-2 (SSD) scan over a prompt, chunked.
  *   ssm_scan_step       one decode token against a cached state.
+ *   ssm_conv1d_fwd      the mixers' causal depthwise convolution (+ silu),
+ *                       over a prompt or, in place, one decode token.
  *
  * Conventions for every call
  * --------------------------
@@ -215,6 +217,47 @@ typedef struct ssm_step_args {
 } ssm_step_args_t;
 
 ssm_status_t ssm_scan_step(const ssm_step_args_t *args, void *stream);
+
+/* ------------------------------------------------------------------------
+ * ssm_conv1d_fwd -- the mixers' causal depthwise convolution, then silu.
+ *
+ * Defined by: "Mamba-2" (nnterp encyclopedia), the module tree
+ * (Conv1d(channels, channels, kernel_size 4, padding 3, groups = channels))
+ * and "The mixer's values" (x, B, C = silu(conv1d(xBC)), causal, width 4);
+ * "Mamba" (tokentrails lineage), "Code" (x = silu(causal_conv1d(x)),
+ * depthwise, width 4).  The layer's output is cut to the input length, so
+ *
+ *   u[t, c] = act(bias[c] + sum_{k < width} w[c, k] * x[t - (width - 1) + k, c])
+ *
+ * with act = silu when flags has SSM_CONV_SILU, else the identity.
+ *   x, u: [batch, seqlen, channels] (io); w: [channels, width] float32;
+ *   bias: [channels] float32 or NULL (zero);
+ *   state_in: [batch, channels, width - 1] float32 or NULL (zeros, a
+ *     sequence start): the inputs of the width - 1 tokens before t = 0,
+ *     oldest first;
+ *   state_out: [batch, channels, width - 1] float32 or NULL: the last
+ *     width - 1 inputs (state_in's entries where seqlen < width - 1), so a
+ *     sequence cut in two and run with state_out -> state_in gives the same
+ *     u.
+ * width 1..4 (else SSM_ERR_UNSUPPORTED).  state_out may equal state_in:
+ * with seqlen 1 that is the decode form (state updated in place); no other
+ * overlap is allowed, and x and u must not overlap.  seqlen 0 copies (or
+ * zeroes) the state.  bf16 outputs use silu = z (1 + tanh(z / 2)) / 2 with
+ * the hardware tanh; float32 uses z / (1 + exp(-z)).
+ * ---------------------------------------------------------------------- */
+#define SSM_CONV_SILU 1u
+
+typedef struct ssm_conv_args {
+  int64_t batch, seqlen, channels, width;
+  int32_t io;
+  uint32_t flags;
+  const void *x;
+  const float *w, *bias, *state_in;
+  void *u;
+  float *state_out;
+} ssm_conv_args_t;
+
+ssm_status_t ssm_conv1d_fwd(const ssm_conv_args_t *args, void *stream);
 
 /* A short English description of a status; never NULL. */
 const char *ssm_status_string(ssm_status_t status);

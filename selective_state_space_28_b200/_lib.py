@@ -19,6 +19,8 @@ STATUS = {0: "SSM_OK", 1: "SSM_ERR_NULL", 2: "SSM_ERR_SHAPE", 3: "SSM_ERR_DTYPE"
           4: "SSM_ERR_ALIGN", 5: "SSM_ERR_UNSUPPORTED", 6: "SSM_ERR_WORKSPACE",
           7: "SSM_ERR_CUDA", 8: "SSM_ERR_TIMEOUT"}
 
+SSM_CONV_SILU = 1
+
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
 
@@ -53,6 +55,13 @@ class StepArgs(ctypes.Structure):
                 ("state_io", _vp), ("y", _vp)]
 
 
+class ConvArgs(ctypes.Structure):
+    _fields_ = [("batch", _i64), ("seqlen", _i64), ("channels", _i64), ("width", _i64),
+                ("io", ctypes.c_int32), ("flags", ctypes.c_uint32),
+                ("x", _vp), ("w", _vp), ("bias", _vp), ("state_in", _vp),
+                ("u", _vp), ("state_out", _vp)]
+
+
 def header_functions(path=HEADER):
     """Names of the functions include/ssm.h declares."""
     with open(path) as f:
@@ -79,8 +88,9 @@ def lib():
         L.ssd_chunk_scan_workspace.argtypes = [ctypes.POINTER(SsdArgs),
                                                ctypes.POINTER(ctypes.c_size_t)]
         L.ssm_scan_step.argtypes = [ctypes.POINTER(StepArgs), _vp]
+        L.ssm_conv1d_fwd.argtypes = [ctypes.POINTER(ConvArgs), _vp]
         for fn in (L.ssm_scan_fwd, L.ssm_scan_workspace, L.ssd_chunk_scan_fwd,
-                   L.ssd_chunk_scan_workspace, L.ssm_scan_step):
+                   L.ssd_chunk_scan_workspace, L.ssm_scan_step, L.ssm_conv1d_fwd):
             fn.restype = ctypes.c_int
         L.ssm_status_string.argtypes = [ctypes.c_int]
         L.ssm_status_string.restype = ctypes.c_char_p

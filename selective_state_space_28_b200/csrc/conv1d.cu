@@ -1,0 +1,227 @@
+// conv1d.cu -- causal depthwise convolution over tokens, then silu: the
+// mixers' conv1d ("Mamba-2", nnterp encyclopedia: the module tree's
+// Conv1d(channels, channels, kernel 4, padding 3, groups = channels) and "The
+// mixer's values", x, B, C = silu(conv1d(xBC)); "Mamba", tokentrails, "Code":
+// x = silu(causal_conv1d(x)), depthwise, width 4):
+//
+//   u[t, c] = silu(bias[c] + sum_{k<W} w[c, k] * x[t - (W - 1) + k, c]),
+//
+// inputs before t = 0 taken from the conv state (the W - 1 inputs before the
+// sequence, oldest first; zeros without one); the state after the call is the
+// last W - 1 inputs.  With seqlen 1 and the state updated in place this is the
+// decode form of the same convolution.
+//
+// HBM-streaming layout: a thread owns V = 4 consecutive channels (an 8-byte
+// (bf16) or 16-byte (f32) vector of the tokens-first rows) over a run of kRun tokens, keeps the W - 1
+// previous inputs in registers, and reads each input once (plus a W - 1 token
+// halo at the start of its run, mostly from L2) and writes each output once,
+// with streaming (evict-first) vector loads and stores, kAhead tokens'
+// loads in flight; a warp covers 32 consecutive vectors of a row, so every
+// access is coalesced.
+#include "common.cuh"
+#include "internal.h"
+
+namespace ssm {
+namespace {
+
+constexpr int kRun = 64;    // tokens per thread (when the state is not updated in place)
+constexpr int kAhead = 4;  // loads in flight per thread
+
+// Streaming (evict-first) vector loads and stores through the compiler's
+// intrinsics, so that loads of later tokens can be issued ahead of earlier
+// stores.
+template <typename T> struct Vec;
+template <> struct Vec<__nv_bfloat16> {
+  static constexpr int V = 4;
+  using Raw = uint2;
+  static __device__ __forceinline__ Raw load(const __nv_bfloat16 *p) {
+    return __ldcs(reinterpret_cast<const uint2 *>(p));
+  }
+  static __device__ __forceinline__ void widen(const Raw &w, float (&f)[4]) {
+    f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&f)[4]) {
+    __stcs(reinterpret_cast<uint2 *>(p), make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3])));
+  }
+};
+template <> struct Vec<float> {
+  static constexpr int V = 4;
+  using Raw = float4;
+  static __device__ __forceinline__ Raw load(const float *p) {
+    return __ldcs(reinterpret_cast<const float4 *>(p));
+  }
+  static __device__ __forceinline__ void widen(const Raw &v, float (&f)[4]) {
+    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+  }
+  static __device__ __forceinline__ void store(float *p, const float (&f)[4]) {
+    __stcs(reinterpret_cast<float4 *>(p), make_float4(f[0], f[1], f[2], f[3]));
+  }
+};
+
+template <typename T> __device__ __forceinline__ float act(float v, bool on) {
+  if (!on) return v;
+  return sizeof(T) == 2 ? silu_tanh(v) : silu(v);
+}
+
+// Vector form: channels % V == 0.  Thread =
+// (batch row, vector of V channels, run of kRun tokens).
+template <typename T, int W>
+__global__ void __launch_bounds__(128)
+    conv1d_vec_kernel(ConvParams p) {
+  constexpr int V = Vec<T>::V;
+  const int64_t nvec = p.Cc / V;
+  const int64_t gv = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gv >= nvec * p.batch) return;
+  const int64_t b = gv / nvec, c0 = (gv % nvec) * V;
+  const int64_t L = p.L, Cc = p.Cc;
+  const int64_t t0 = (int64_t)blockIdx.y * p.run;
+  if (t0 >= L) return;
+  const int64_t t1 = t0 + p.run < L ? t0 + p.run : L;
+  const T *x = static_cast<const T *>(p.x);
+  T *u = static_cast<T *>(p.u);
+
+  float w[V][W], bias[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+#pragma unroll
+    for (int k = 0; k < W; ++k) w[v][k] = p.w[(c0 + v) * W + k];
+    bias[v] = p.bias ? p.bias[c0 + v] : 0.f;
+  }
+  // hist[j][v]: input j + 1 tokens before the current one (j < W - 1)
+  float hist[W > 1 ? W - 1 : 1][V];
+#pragma unroll
+  for (int j = 0; j < W - 1; ++j) {
+    const int64_t tau = t0 - 1 - j;
+    if (tau >= 0) {
+      Vec<T>::widen(Vec<T>::load(x + (b * L + tau) * Cc + c0), hist[j]);
+    } else {
+#pragma unroll
+      for (int v = 0; v < V; ++v)
+        hist[j][v] = p.state_in ? p.state_in[((b * Cc) + c0 + v) * (W - 1) + (W - 1) + tau] : 0.f;
+    }
+  }
+  // kAhead tokens' loads are issued before any of them is used
+  for (int64_t tb = t0; tb < t1; tb += kAhead) {
+    typename Vec<T>::Raw raw[kAhead];
+#pragma unroll
+    for (int a = 0; a < kAhead; ++a)
+      if (tb + a < t1) raw[a] = Vec<T>::load(x + (b * L + tb + a) * Cc + c0);
+#pragma unroll
+    for (int a = 0; a < kAhead; ++a) {
+      if (tb + a >= t1) break;
+      float xv[V], o[V];
+      Vec<T>::widen(raw[a], xv);
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        float acc = fmaf(w[v][W - 1], xv[v], bias[v]);
+#pragma unroll
+        for (int j = 0; j < W - 1; ++j) acc = fmaf(w[v][W - 2 - j], hist[j][v], acc);
+        o[v] = act<T>(acc, p.silu);
+      }
+      Vec<T>::store(u + (b * L + tb + a) * Cc + c0, o);
+#pragma unroll
+      for (int j = W - 2; j > 0; --j)
+#pragma unroll
+        for (int v = 0; v < V; ++v) hist[j][v] = hist[j - 1][v];
+      if (W > 1) {
+#pragma unroll
+        for (int v = 0; v < V; ++v) hist[0][v] = xv[v];
+      }
+    }
+  }
+  // The run that ends the sequence leaves the state: the last W - 1 inputs,
+  // oldest first (from before the sequence when it is shorter than that).
+  if (p.state_out && t1 == L) {
+#pragma unroll
+    for (int j = 0; j < W - 1; ++j)
+#pragma unroll
+      for (int v = 0; v < V; ++v)
+        p.state_out[((b * Cc) + c0 + v) * (W - 1) + (W - 2 - j)] = hist[j][v];
+  }
+}
+
+// Scalar form, for any channel count: thread = (batch row, channel, run).
+template <typename T, int W>
+__global__ void __launch_bounds__(128)
+    conv1d_scalar_kernel(ConvParams p) {
+  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= p.Cc * p.batch) return;
+  const int64_t b = g / p.Cc, c = g % p.Cc;
+  const int64_t L = p.L, Cc = p.Cc;
+  const int64_t t0 = (int64_t)blockIdx.y * p.run;
+  if (t0 >= L) return;
+  const int64_t t1 = t0 + p.run < L ? t0 + p.run : L;
+  const T *x = static_cast<const T *>(p.x);
+  T *u = static_cast<T *>(p.u);
+  float w[W];
+#pragma unroll
+  for (int k = 0; k < W; ++k) w[k] = p.w[c * W + k];
+  const float bias = p.bias ? p.bias[c] : 0.f;
+  float hist[W > 1 ? W - 1 : 1];
+#pragma unroll
+  for (int j = 0; j < W - 1; ++j) {
+    const int64_t tau = t0 - 1 - j;
+    hist[j] = tau >= 0 ? ld(x + (b * L + tau) * Cc + c)
+                       : (p.state_in ? p.state_in[(b * Cc + c) * (W - 1) + (W - 1) + tau] : 0.f);
+  }
+  for (int64_t t = t0; t < t1; ++t) {
+    const float xv = ld(x + (b * L + t) * Cc + c);
+    float acc = fmaf(w[W - 1], xv, bias);
+#pragma unroll
+    for (int j = 0; j < W - 1; ++j) acc = fmaf(w[W - 2 - j], hist[j], acc);
+    st(u + (b * L + t) * Cc + c, act<T>(acc, p.silu));
+#pragma unroll
+    for (int j = W - 2; j > 0; --j) hist[j] = hist[j - 1];
+    if (W > 1) hist[0] = xv;
+  }
+  if (p.state_out && t1 == L) {
+#pragma unroll
+    for (int j = 0; j < W - 1; ++j) p.state_out[(b * Cc + c) * (W - 1) + (W - 2 - j)] = hist[j];
+  }
+}
+
+template <typename T, int W>
+cudaError_t launch_w(const ConvParams &p, cudaStream_t s) {
+  constexpr int V = Vec<T>::V;
+  const bool vec = (p.Cc % V) == 0;  // rows then hold whole vectors (bases are 16-byte aligned)
+  const int64_t runs = (p.L + p.run - 1) / p.run;
+  const int64_t units = vec ? p.batch * (p.Cc / V) : p.batch * p.Cc;
+  dim3 grid((unsigned)((units + 127) / 128), (unsigned)runs);
+  if (vec)
+    conv1d_vec_kernel<T, W><<<grid, 128, 0, s>>>(p);
+  else
+    conv1d_scalar_kernel<T, W><<<grid, 128, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_t(const ConvParams &p, cudaStream_t s) {
+  switch (p.W) {
+    case 1: return launch_w<T, 1>(p, s);
+    case 2: return launch_w<T, 2>(p, s);
+    case 3: return launch_w<T, 3>(p, s);
+    case 4: return launch_w<T, 4>(p, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+// Tokens per thread: kRun, or the whole sequence when the state is updated
+// in place (the run that reads the incoming state must be the one that
+// writes the new state).
+int64_t conv1d_run_length(int64_t L, bool state_in_place) {
+  return state_in_place ? (L > 0 ? L : 1) : kRun;
+}
+
+bool conv1d_supported(const ConvParams &p) {
+  const int64_t run = p.run > 0 ? p.run : 1;
+  return p.W >= 1 && p.W <= kConvMaxWidth && (p.L + run - 1) / run <= 65535 &&
+         (p.batch * p.Cc + 127) / 128 < (1ll << 31);
+}
+
+cudaError_t launch_conv1d(const ConvParams &p, cudaStream_t s) {
+  return p.io == 1 ? launch_t<__nv_bfloat16>(p, s) : launch_t<float>(p, s);
+}
+
+}  // namespace ssm

@@ -46,6 +46,20 @@ struct M1StepParams {
   void *y;
 };
 
+// Causal depthwise convolution over tokens (then silu when `silu`).
+constexpr int kConvMaxWidth = 4;
+struct ConvParams {
+  int64_t batch, L, Cc;
+  int W;
+  int io;
+  bool silu;
+  int64_t run;  // tokens per thread (conv1d_run_length)
+  const void *x;
+  const float *w, *bias, *state_in;
+  void *u;
+  float *state_out;
+};
+
 // Each returns cudaSuccess, cudaErrorNotSupported for a shape without a
 // kernel (checked before any launch), or the launch error.
 cudaError_t launch_m1_scan(const M1Params &p, cudaStream_t s);
@@ -59,6 +73,9 @@ bool m1_step_supported(int64_t N);
 // Tensor-core SSD (bf16 I/O, state 128, head dim 64, no per-token states).
 // `status` is a device word the kernel sets non-zero if a bounded wait ran out.
 bool ssd_tc_supported(const M2Params &p);
+int64_t conv1d_run_length(int64_t L, bool state_in_place);
+bool conv1d_supported(const ConvParams &p);
+cudaError_t launch_conv1d(const ConvParams &p, cudaStream_t s);
 cudaError_t launch_ssd_tc(const M2Params &p, int *status, cudaStream_t s);
 
 }  // namespace ssm

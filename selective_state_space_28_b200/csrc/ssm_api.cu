@@ -293,4 +293,46 @@ ssm_status_t ssm_scan_step(const ssm_step_args_t *a, void *stream) {
   return from_cuda(ssm::launch_m2_recurrent(p, s));
 }
 
+ssm_status_t ssm_conv1d_fwd(const ssm_conv_args_t *a, void *stream) {
+  if (!a) return SSM_ERR_NULL;
+  if (a->io != SSM_F32 && a->io != SSM_BF16) return SSM_ERR_DTYPE;
+  if (a->batch < 0 || a->seqlen < 0 || a->channels <= 0 || a->width <= 0) return SSM_ERR_SHAPE;
+  if (a->width > ssm::kConvMaxWidth || (a->flags & ~SSM_CONV_SILU)) return SSM_ERR_UNSUPPORTED;
+  if (!a->w) return SSM_ERR_NULL;
+  const bool work = a->batch > 0 && a->seqlen > 0;
+  if (work && (!a->x || !a->u)) return SSM_ERR_NULL;
+  if (!all_aligned(a->x, a->u, a->w, a->bias, a->state_in, a->state_out)) return SSM_ERR_ALIGN;
+  const size_t esz = a->io == SSM_BF16 ? 2 : 4;
+  const size_t xbytes = (size_t)a->batch * a->seqlen * a->channels * esz;
+  const size_t sbytes = (size_t)a->batch * a->channels * (a->width - 1) * sizeof(float);
+  // x and u must not overlap; the state may be updated in place, nothing else
+  auto overlap = [](const void *p, const void *q, size_t n) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(p), b0 = reinterpret_cast<uintptr_t>(q);
+    return n > 0 && a0 < b0 + n && b0 < a0 + n;
+  };
+  if (work && overlap(a->x, a->u, xbytes)) return SSM_ERR_SHAPE;
+  const bool in_place = a->state_in && a->state_out == a->state_in;
+  if (a->state_in && a->state_out && !in_place && overlap(a->state_in, a->state_out, sbytes))
+    return SSM_ERR_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (a->batch == 0) return SSM_OK;
+  if (a->seqlen == 0) return pass_state(a->state_in, a->state_out, sbytes, s);
+  ssm::ConvParams p;
+  p.batch = a->batch;
+  p.L = a->seqlen;
+  p.Cc = a->channels;
+  p.W = (int)a->width;
+  p.io = a->io;
+  p.silu = (a->flags & SSM_CONV_SILU) != 0;
+  p.run = ssm::conv1d_run_length(a->seqlen, in_place);
+  p.x = a->x;
+  p.w = a->w;
+  p.bias = a->bias;
+  p.state_in = a->state_in;
+  p.u = a->u;
+  p.state_out = a->width > 1 ? a->state_out : nullptr;
+  if (!ssm::conv1d_supported(p)) return SSM_ERR_UNSUPPORTED;
+  return from_cuda(ssm::launch_conv1d(p, s));
+}
+
 }  // extern "C"

@@ -15,6 +15,11 @@ the pages describe):
   channel / head (1e-3 is the configs' ``time_step_min``).
 * ``D = 1``; ``x, z, dt_raw, B, C ~ N(0, 1)``; decode states ``~ N(0, 0.1^2)``.
 * Draw order: A, dt_bias, D, x, z, dt_raw, B, C, then the state.
+* Convolution (the mixers' conv1d): ``x ~ N(0, 1)``; weight and bias
+  ``U(-1/sqrt(W), 1/sqrt(W))``, the layer's default initialisation for a
+  depthwise kernel of width W (fan-in W); conv state ``~ N(0, 1)`` (it holds
+  past inputs).  Draw order: w, bias, x, state.  The Mamba-2 2.7B channel
+  count is d_inner + 2 G N = 5120 + 256 (the module tree's Conv1d over xBC).
 """
 import math
 from dataclasses import dataclass, field
@@ -29,7 +34,7 @@ RMS_DT = 4
 
 @dataclass(frozen=True)
 class Workload:
-    """One named scan workload.  ``kind`` is "m1", "ssd" or "decode"."""
+    """One named scan workload.  ``kind`` is "m1", "ssd", "decode" or "conv"."""
     name: str
     kind: str
     batch: int
@@ -83,6 +88,11 @@ WORKLOADS = {
         "decode_2p7b_layer_b256", "decode", batch=256, heads=80, head_dim=64,
         state=128, io="bf16", gate=False, layers=1, m1_layers=1,
         m1_channels=1536, m1_state=16, seed=4),
+    # The Mamba-2 2.7B mixer's causal convolution over xBC (d_inner 5120 plus
+    # B and C, 2 x 128) for the SSD workload's prompt, with a carried state.
+    "conv_2p7b_b4_l4096_c5376_bf16": Workload(
+        "conv_2p7b_b4_l4096_c5376_bf16", "conv", batch=4, seqlen=4096, channels=5376,
+        io="bf16", seed=5, extra={"width": 4, "state": True}),
 }
 
 
@@ -185,6 +195,21 @@ def m1_step_inputs(batch, channels, state, groups=1, io="bf16", gate=True, seed=
     return out
 
 
+def conv_inputs(batch, seqlen, channels, width=4, io="bf16", seed=0, state=False,
+                device="cpu"):
+    """Inputs of one causal convolution: dict of tensors on ``device``."""
+    g = _gen(seed, device)
+    bound = 1.0 / math.sqrt(width)
+    out = {"w": (torch.rand((channels, width), generator=g, dtype=torch.float32, device=device)
+                 * 2 - 1) * bound,
+           "bias": (torch.rand(channels, generator=g, dtype=torch.float32, device=device)
+                    * 2 - 1) * bound}
+    out["x"] = _randn((batch, seqlen, channels), g, _dtype(io), device)
+    out["state"] = (_randn((batch, channels, width - 1), g, torch.float32, device)
+                    if state else None)
+    return out
+
+
 def workload_inputs(w: Workload, device="cpu", seed: Optional[int] = None):
     """Inputs of a scan workload (Mamba-1 or SSD)."""
     s = w.seed if seed is None else seed
@@ -194,4 +219,7 @@ def workload_inputs(w: Workload, device="cpu", seed: Optional[int] = None):
     if w.kind == "ssd":
         return ssd_inputs(w.batch, w.seqlen, w.heads, w.head_dim, w.state, w.groups,
                           w.io, w.gate, s, device=device)
+    if w.kind == "conv":
+        return conv_inputs(w.batch, w.seqlen, w.channels, w.extra.get("width", 4), w.io, s,
+                           state=w.extra.get("state", False), device=device)
     raise ValueError("no scan inputs for kind %r" % w.kind)

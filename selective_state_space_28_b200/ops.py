@@ -1,4 +1,4 @@
-"""Python binding of libssm: the three C-ABI calls, same names, torch tensors in.
+"""Python binding of libssm: the C-ABI calls, same names, torch tensors in.
 
 Argument marshalling only: shapes are read off the tensors, outputs and the
 workspace are allocated with torch (device memory), and the call is queued
@@ -178,3 +178,42 @@ def ssm_scan_step(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, *, flags=
         host_state.copy_(st_h)
         return y_h
     return y
+
+
+def ssm_conv1d_fwd(x, w, bias=None, state=None, *, silu=True, u=None, state_out=None,
+                   in_place=False, stream=None):
+    """The mixers' causal depthwise convolution, then silu (include/ssm.h,
+    ssm_conv1d_fwd).
+
+    x: [b, L, C] (float32 or bfloat16); w: [C, W] float32 (W <= 4); bias: [C]
+    float32; state: [b, C, W - 1] float32, the inputs before the sequence
+    (oldest first) or None for a sequence start.  Returns (u, state_out):
+    u [b, L, C] in x's dtype and the last W - 1 inputs.  With in_place=True
+    the state tensor itself is updated (the decode form, one token)."""
+    sg = _Staging([x, w, bias, state])
+    host_state = state
+    x, w, bias = map(sg.dev, (x, w, bias))
+    if state is not None:
+        state = sg.dev(state)
+    b, Lq, C = x.shape
+    W = w.shape[1]
+    if u is None:
+        u = torch.empty_like(x)
+    if in_place:
+        if state is None:
+            raise ValueError("in_place needs a state tensor")
+        state_out = state
+    elif state_out is None:
+        state_out = torch.empty((b, C, max(W - 1, 0)), dtype=torch.float32, device=x.device)
+    a = L.ConvArgs(batch=b, seqlen=Lq, channels=C, width=W, io=_io_of(x),
+                   flags=L.SSM_CONV_SILU if silu else 0, x=_ptr(x), w=_ptr(w),
+                   bias=_ptr(bias), state_in=_ptr(state), u=_ptr(u),
+                   state_out=_ptr(state_out) if W > 1 else None)
+    L.check(L.lib().ssm_conv1d_fwd(ctypes.byref(a), _stream(stream, x.device)),
+            "ssm_conv1d_fwd")
+    if sg.host:
+        u_h, so_h = sg.back((u, state_out))
+        if in_place:
+            host_state.copy_(so_h)
+        return u_h, so_h
+    return u, state_out

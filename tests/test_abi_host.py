@@ -24,7 +24,7 @@ def test_exports_every_declared_symbol(lib):
     names = L.header_functions()
     assert {"ssm_scan_fwd", "ssm_scan_workspace", "ssd_chunk_scan_fwd",
             "ssd_chunk_scan_workspace", "ssm_scan_step", "ssm_status_string",
-            "ssm_abi_version"} <= set(names)
+            "ssm_abi_version", "ssm_conv1d_fwd", "ssm_scan_fwd_static"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], check=True,
                          capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
@@ -143,3 +143,29 @@ def test_workspace_queries_need_no_pointers(lib):
     assert n.value == 2 * 8 * 4
     s = _ssd(x=None, dt=None, B=None, C=None, A=None, y=None)
     assert lib.ssd_chunk_scan_workspace(ctypes.byref(s), ctypes.byref(n)) == OK
+
+
+def _conv(**kw):
+    d = dict(batch=2, seqlen=8, channels=64, width=4, io=1, flags=1, x=P, w=P + 0x10000,
+             bias=None, state_in=None, u=P + 0x20000, state_out=None)
+    d.update(kw)
+    return L.ConvArgs(**d)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(width=0), SHAPE), (dict(width=5), UNSUP), (dict(channels=0), SHAPE),
+    (dict(batch=-1), SHAPE), (dict(seqlen=-1), SHAPE), (dict(io=7), DTYPE),
+    (dict(flags=2), UNSUP), (dict(w=None), NULL), (dict(x=None), NULL), (dict(u=None), NULL),
+    (dict(x=P + 4), ALIGN), (dict(state_in=P + 0x30004), ALIGN),
+    # x and u overlap (the call's x is 2*8*64*2 bytes)
+    (dict(u=P + 0x100), SHAPE),
+    # partially overlapping states (equal pointers are the in-place form)
+    (dict(state_in=P + 0x30000, state_out=P + 0x30010), SHAPE),
+])
+def test_conv_rejects(lib, kw, status):
+    assert lib.ssm_conv1d_fwd(ctypes.byref(_conv(**kw)), None) == status
+
+
+def test_conv_empty_batch_is_a_no_op(lib):
+    # batch 0: nothing to read or write, no pointer is looked at
+    assert lib.ssm_conv1d_fwd(ctypes.byref(_conv(batch=0, x=None, u=None)), None) == OK
