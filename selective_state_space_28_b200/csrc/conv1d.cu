@@ -25,7 +25,7 @@ namespace ssm {
 namespace {
 
 constexpr int kRun = 64;    // tokens per thread (when the state is not updated in place)
-constexpr int kAhead = 4;  // loads in flight per thread
+constexpr int kAhead = 8;  // loads in flight per thread
 
 // Streaming (evict-first) vector loads and stores through the compiler's
 // intrinsics, so that loads of later tokens can be issued ahead of earlier
