@@ -47,6 +47,7 @@ def _load():
             "orc_m2_quadratic": [_I64] * 6 + [_D] * 9,
             "orc_m1_quadratic": [_I64] * 5 + [_D] * 9,
             "orc_conv1d": [_I64] * 4 + [_D] * 4 + [ctypes.c_int] + [_D] * 2,
+            "orc_gated_rmsnorm": [_I64] * 2 + [ctypes.c_double] + [_D] * 4,
         }.items():
             fn = getattr(lib, name)
             fn.argtypes = argtypes
@@ -194,6 +195,21 @@ def conv1d(x, w, bias=None, state=None, act=True):
     if rc:
         raise ValueError("orc_conv1d: bad arguments")
     return u, so
+
+
+def gated_rmsnorm(y, z=None, weight=None, eps=1e-5):
+    """The Mamba-2 mixer's gated norm over the last axis (the mixer's whole
+    width): y * silu(z), then RMS-normalised, then times weight ("Mamba-2",
+    "The mixer's values" and the paragraph on the block's norms).
+    y, z: [..., width]; weight: [width].  Returns float64 of y's shape."""
+    y, z, weight = _f64(y), _f64(z), _f64(weight)
+    width = y.shape[-1]
+    rows = int(np.prod(y.shape[:-1])) if y.ndim > 1 else 1
+    out = np.zeros_like(y)
+    rc = _load().orc_gated_rmsnorm(rows, width, float(eps), _p(y), _p(z), _p(weight), _p(out))
+    if rc:
+        raise ValueError("orc_gated_rmsnorm: bad arguments")
+    return out
 
 
 def softplus(v):

@@ -454,3 +454,24 @@ int orc_conv1d(int64_t batch, int64_t seqlen, int64_t channels, int64_t width,
     }
   return 0;
 }
+
+/* Gated RMS norm ("Mamba-2", "The mixer's values" and the paragraph on the
+ * block's norms): the gate first, y * silu(z), then one RMS norm over the
+ * whole row -- the mixer's full width, not per group -- then the weight. */
+int orc_gated_rmsnorm(int64_t rows, int64_t width, double eps, const double *y,
+                      const double *z, const double *weight, double *out) {
+  if (rows < 0 || width <= 0 || !y || !out) return 1;
+  for (int64_t r = 0; r < rows; ++r) {
+    const double *yr = y + r * width;
+    double *o = out + r * width;
+    double ss = 0.0;
+    for (int64_t i = 0; i < width; ++i) {
+      const double g = z ? yr[i] * orc_silu(z[r * width + i]) : yr[i];
+      o[i] = g;
+      ss += g * g;
+    }
+    const double inv = 1.0 / sqrt(ss / (double)width + eps);
+    for (int64_t i = 0; i < width; ++i) o[i] = o[i] * inv * (weight ? weight[i] : 1.0);
+  }
+  return 0;
+}

@@ -23,6 +23,10 @@
  *     mixer's values" (x, B, C = silu(conv1d(xBC)), causal, width 4);
  *     "Mamba" (tokentrails lineage), "Code" (x = silu(causal_conv1d(x)),
  *     depthwise, width 4).
+ *   - The Mamba-2 mixer's gated norm: "Mamba-2" (nnterp encyclopedia), "The
+ *     mixer's values" (out_proj(norm(y * silu(z)))) and the paragraph on the
+ *     block's norms (the gated norm multiplies y by silu(z), then normalizes
+ *     over the mixer's whole width, whatever n_groups is).
  */
 #ifndef SSM_ORACLE_H
 #define SSM_ORACLE_H
@@ -106,6 +110,13 @@ int orc_m1_quadratic(int64_t batch, int64_t seqlen, int64_t channels,
 int orc_conv1d(int64_t batch, int64_t seqlen, int64_t channels, int64_t width,
                const double *x, const double *w, const double *bias,
                const double *state_in, int act, double *u, double *state_out);
+
+/* The Mamba-2 mixer's gated RMS norm over each row of `width` values (a
+ * token's whole mixer width, heads x head_dim): g = y * silu(z) (g = y when
+ * z is NULL), out = g / sqrt(mean(g^2) + eps) * weight (weight NULL = 1).
+ * y, z, out: [rows, width]; weight: [width]. */
+int orc_gated_rmsnorm(int64_t rows, int64_t width, double eps, const double *y,
+                      const double *z, const double *weight, double *out);
 
 /* Elementwise helpers exposed for the pins. */
 double orc_softplus(double v);

@@ -80,6 +80,14 @@ MUTANTS = {
                               "        u[(b * L + t) * Cc + c] = (act ? orc_silu(acc) : acc) + (bias ? bias[c] : 0.0);"),
     "conv_state_out_off_by_one": ("conv_in(x, state_in, b, L, Cc, W, c, L - (W - 1) + j);",
                                   "conv_in(x, state_in, b, L, Cc, W, c, L - W + j);"),
+    "gated_norm_gate_after": ("      const double g = z ? yr[i] * orc_silu(z[r * width + i]) : yr[i];\n      o[i] = g;\n      ss += g * g;",
+                              "      const double g = yr[i];\n      o[i] = z ? g * orc_silu(z[r * width + i]) : g;\n      ss += g * g;"),
+    "gated_norm_per_half": ("const double inv = 1.0 / sqrt(ss / (double)width + eps);\n    for (int64_t i = 0; i < width; ++i) o[i] = o[i] * inv * (weight ? weight[i] : 1.0);",
+                            "double s1 = 0.0;\n    for (int64_t i = 0; i < width / 2; ++i) s1 += o[i] * o[i];\n"
+                            "    for (int64_t i = 0; i < width; ++i) o[i] = o[i] * (1.0 / sqrt((i < width / 2 ? s1 : ss - s1) / (double)(width / 2) + eps)) * (weight ? weight[i] : 1.0);"),
+    "gated_norm_no_weight": ("o[i] = o[i] * inv * (weight ? weight[i] : 1.0);", "o[i] = o[i] * inv;"),
+    "gated_norm_eps_outside": ("const double inv = 1.0 / sqrt(ss / (double)width + eps);",
+                               "const double inv = 1.0 / (sqrt(ss / (double)width) + eps);"),
 }
 
 
@@ -118,7 +126,7 @@ def test_mutant_is_caught(key):
         mlib = ctypes.CDLL(_build_mutant(src.replace(old, new), tmp, key))
         for name in ("orc_m1_scan", "orc_m2_scan", "orc_m1_step", "orc_m2_step",
                      "orc_m2_quadratic", "orc_m1_quadratic", "orc_softplus", "orc_silu",
-                     "orc_rms_rows", "orc_conv1d"):
+                     "orc_rms_rows", "orc_conv1d", "orc_gated_rmsnorm"):
             getattr(mlib, name).argtypes = getattr(real, name).argtypes
             getattr(mlib, name).restype = getattr(real, name).restype
         caught = None

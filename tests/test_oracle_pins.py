@@ -454,3 +454,45 @@ def test_conv1d_width_one_is_elementwise():
     v = x * w[:, 0] + bias
     np.testing.assert_allclose(u, v / (1 + np.exp(-v)), rtol=1e-15, atol=0)
     assert st.shape == (2, 4, 0)
+
+
+# ------------------------------------------------------------ gated norm
+# "Mamba-2": out_proj(norm(y * silu(z))); the gated norm multiplies y by
+# silu(z), then normalizes over the mixer's whole width, whatever n_groups is.
+
+def test_gated_norm_matches_library():
+    r = rng(50)
+    y, z, wt = r.standard_normal((3, 5, 96)), r.standard_normal((3, 5, 96)), r.standard_normal(96)
+    out = oracle.gated_rmsnorm(y, z, wt, eps=1e-5)
+    g = torch.tensor(y) * F.silu(torch.tensor(z))
+    ref = F.rms_norm(g, (96,), torch.tensor(wt), eps=1e-5).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_gated_norm_spans_the_whole_width():
+    # Normalizing per group (here per half of the width) gives a different
+    # answer: the norm's statistic is the whole row's.
+    r = rng(51)
+    y = r.standard_normal((4, 64))
+    y[:, 32:] *= 10.0
+    out = oracle.gated_rmsnorm(y, eps=0.0)
+    np.testing.assert_allclose(np.mean(out ** 2, axis=-1), 1.0, rtol=1e-12)
+    halves = np.concatenate([oracle.gated_rmsnorm(y[:, :32], eps=0.0),
+                             oracle.gated_rmsnorm(y[:, 32:], eps=0.0)], axis=-1)
+    assert np.max(np.abs(halves - out)) > 0.1
+
+
+def test_gated_norm_gate_before_norm_and_scale_invariance():
+    r = rng(52)
+    y, z = r.standard_normal((2, 40)), r.standard_normal((2, 40))
+    out = oracle.gated_rmsnorm(y, z, eps=0.0)
+    # the gate acts before the norm: out is g / rms(g), g = y * silu(z)
+    g = y * z / (1 + np.exp(-z))
+    np.testing.assert_allclose(out, g / np.sqrt(np.mean(g ** 2, axis=-1, keepdims=True)),
+                               rtol=1e-13)
+    # and without eps the result does not depend on the scale of y
+    np.testing.assert_allclose(oracle.gated_rmsnorm(7.5 * y, z, eps=0.0), out, rtol=1e-13)
+    # no gate: a plain RMS norm
+    np.testing.assert_allclose(oracle.gated_rmsnorm(y, None, eps=1e-3),
+                               y / np.sqrt(np.mean(y ** 2, axis=-1, keepdims=True) + 1e-3),
+                               rtol=1e-13)
