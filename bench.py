@@ -46,7 +46,8 @@ def parse(argv=None):
                     help="measure only the headline workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["m1", "ssd", "decode", "decode_layer", "falcon", "conv"],
+    ap.add_argument("--only", choices=["m1", "ssd", "decode", "decode_layer", "falcon", "conv",
+                                       "gnorm"],
                     help="run just one workload's timed loop (for profiling); prints its timing")
     return ap.parse_args(argv)
 
@@ -111,6 +112,13 @@ def conv_bytes(w):
     if w.extra.get("state", False):
         n += 2 * w.batch * w.channels * (W - 1) * 4
     return n
+
+
+def gnorm_bytes(w):
+    """y and z read and out written once in the I/O type, and the weight."""
+    e = _esz(w.io)
+    rows = w.batch * w.seqlen
+    return (3 if w.gate else 2) * rows * w.channels * e + w.channels * 4
 
 
 def decode_bytes(w):
@@ -320,6 +328,26 @@ def bench_conv(w, K, W, dist, device, pk, seed_base):
             "launches_per_step": 1}
 
 
+def bench_gnorm(w, K, W, dist, device, pk, seed_base):
+    import torch
+    from selective_state_space_28_b200 import inputs as I
+    from selective_state_space_28_b200 import ops
+    nb = gnorm_bytes(w)
+    sets = []
+    for r in range(n_sets(nb)):
+        d = I.workload_inputs(w, device=device, seed=seed_base + 1000 * r)
+        d["out"] = torch.empty_like(d["y"])
+        sets.append(d)
+
+    def step(i):
+        d = sets[i % len(sets)]
+        ops.ssm_gated_rmsnorm_fwd(d["y"], d["z"], d["weight"], w.rms_eps, out=d["out"])
+    ms = timed(step, K, W, dist, device) / K
+    launch_ms = per_launch_ms(step, max(10, K), device)
+    return {"ms_per_step": ms, "bytes": nb, "launch_ms": launch_ms, "sets": len(sets),
+            "launches_per_step": 1}
+
+
 def bench_ssd(w, K, W, dist, device, pk, seed_base):
     import torch
     from selective_state_space_28_b200 import inputs as I
@@ -443,10 +471,11 @@ def run_only(args):
     name = {"m1": HEADLINE, "ssd": "ssd_2p7b_b4_l4096_h80_p64_n128_bf16",
             "decode": "decode_2p7b_stack_b256", "decode_layer": "decode_2p7b_layer_b256",
             "falcon": "m1_falcon_rms_b4_l8192_c8192_n16_bf16",
-            "conv": "conv_2p7b_b4_l4096_c5376_bf16"}[args.only]
+            "conv": "conv_2p7b_b4_l4096_c5376_bf16",
+            "gnorm": "gnorm_2p7b_b4_l4096_w5120_bf16"}[args.only]
     w = I.WORKLOADS[name]
     fn = {"m1": bench_m1, "falcon": bench_m1, "ssd": bench_ssd, "decode": bench_decode,
-          "decode_layer": bench_decode, "conv": bench_conv}[args.only]
+          "decode_layer": bench_decode, "conv": bench_conv, "gnorm": bench_gnorm}[args.only]
     r = fn(w, args.steps, args.warmup, dist, device, pk, w.seed)
     print(json.dumps({"only": name, "ms_per_step": r["ms_per_step"],
                       "launch_ms": r["launch_ms"]}), flush=True)
@@ -549,6 +578,16 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(ach / hbm, 4), "traffic": traffic_for("conv_2p7b"),
                          "kernel": "conv1d_vec_kernel"}}
+        wg = I.WORKLOADS["gnorm_2p7b_b4_l4096_w5120_bf16"]
+        gn = bench_gnorm(wg, max(3, min(K, 20)), max(3, W), dist, device, pk,
+                         rank_seed(wg.seed, dist.rank))
+        ach = gn["bytes"] / (gn["launch_ms"] * 1e-3) / 1e9
+        wl[wg.name] = {
+            "value": round(job_value(gn["bytes"], dist.world, gn["ms_per_step"]) / 1e9, 2),
+            "unit": "GB/s", "ms_per_step": round(gn["ms_per_step"], 4),
+            "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
+                         "frac": round(ach / hbm, 4), "traffic": traffic_for("gnorm_2p7b"),
+                         "kernel": "gated_norm_kernel"}}
         out["workloads"] = wl
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline_m1(w)

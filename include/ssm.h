@@ -9,6 +9,7 @@
  *   ssm_scan_step       one decode token against a cached state.
  *   ssm_conv1d_fwd      the mixers' causal depthwise convolution (+ silu),
  *                       over a prompt or, in place, one decode token.
+ *   ssm_gated_rmsnorm_fwd  the Mamba-2 mixer's gated RMS norm after the SSD.
  *
  * Conventions for every call
  * --------------------------
@@ -258,6 +259,35 @@ typedef struct ssm_conv_args {
 } ssm_conv_args_t;
 
 ssm_status_t ssm_conv1d_fwd(const ssm_conv_args_t *args, void *stream);
+
+/* ------------------------------------------------------------------------
+ * ssm_gated_rmsnorm_fwd -- the Mamba-2 mixer's gated norm, after the SSD.
+ *
+ * Defined by: "Mamba-2" (nnterp encyclopedia), "The mixer's values"
+ * (return out_proj(norm(y * silu(z)))) and the paragraph on the block's
+ * norms: the gated norm multiplies y by silu(z) and then normalizes over the
+ * mixer's whole width, whatever n_groups is.  Per row (one token's
+ * heads x head_dim values):
+ *
+ *   g = y * silu(z)   (g = y when z is NULL)
+ *   out = g / sqrt(mean(g^2) + eps) * weight   (weight NULL = ones)
+ *
+ *   y, z, out: [rows, width] (io); weight: [width] float32.
+ * rows = batch * seqlen tokens, width 1..49152.  out may equal y (in place);
+ * no other overlap.  flags must be 0.  bf16 uses silu = z (1 + tanh(z/2)) / 2
+ * with the hardware tanh; float32 uses z / (1 + exp(-z)).
+ * ---------------------------------------------------------------------- */
+typedef struct ssm_gated_norm_args {
+  int64_t rows, width;
+  int32_t io;
+  uint32_t flags;
+  float eps;
+  const void *y, *z;
+  const float *weight;
+  void *out;
+} ssm_gated_norm_args_t;
+
+ssm_status_t ssm_gated_rmsnorm_fwd(const ssm_gated_norm_args_t *args, void *stream);
 
 /* A short English description of a status; never NULL. */
 const char *ssm_status_string(ssm_status_t status);

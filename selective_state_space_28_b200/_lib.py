@@ -62,6 +62,12 @@ class ConvArgs(ctypes.Structure):
                 ("u", _vp), ("state_out", _vp)]
 
 
+class GatedNormArgs(ctypes.Structure):
+    _fields_ = [("rows", _i64), ("width", _i64), ("io", ctypes.c_int32),
+                ("flags", ctypes.c_uint32), ("eps", ctypes.c_float),
+                ("y", _vp), ("z", _vp), ("weight", _vp), ("out", _vp)]
+
+
 def header_functions(path=HEADER):
     """Names of the functions include/ssm.h declares."""
     with open(path) as f:
@@ -89,8 +95,10 @@ def lib():
                                                ctypes.POINTER(ctypes.c_size_t)]
         L.ssm_scan_step.argtypes = [ctypes.POINTER(StepArgs), _vp]
         L.ssm_conv1d_fwd.argtypes = [ctypes.POINTER(ConvArgs), _vp]
+        L.ssm_gated_rmsnorm_fwd.argtypes = [ctypes.POINTER(GatedNormArgs), _vp]
         for fn in (L.ssm_scan_fwd, L.ssm_scan_workspace, L.ssd_chunk_scan_fwd,
-                   L.ssd_chunk_scan_workspace, L.ssm_scan_step, L.ssm_conv1d_fwd):
+                   L.ssd_chunk_scan_workspace, L.ssm_scan_step, L.ssm_conv1d_fwd,
+                   L.ssm_gated_rmsnorm_fwd):
             fn.restype = ctypes.c_int
         L.ssm_status_string.argtypes = [ctypes.c_int]
         L.ssm_status_string.restype = ctypes.c_char_p

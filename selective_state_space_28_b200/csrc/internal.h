@@ -60,6 +60,17 @@ struct ConvParams {
   float *state_out;
 };
 
+// The Mamba-2 mixer's gated RMS norm over rows of `width` values.
+constexpr int64_t kGatedNormMaxWidth = 49152;  // the row lives in shared memory
+struct GatedNormParams {
+  int64_t rows, width;
+  int io;
+  float eps;
+  const void *y, *z;
+  const float *weight;
+  void *out;
+};
+
 // Each returns cudaSuccess, cudaErrorNotSupported for a shape without a
 // kernel (checked before any launch), or the launch error.
 cudaError_t launch_m1_scan(const M1Params &p, cudaStream_t s);
@@ -75,6 +86,8 @@ bool m1_step_supported(int64_t N);
 bool ssd_tc_supported(const M2Params &p);
 int64_t conv1d_run_length(int64_t L, bool state_in_place);
 bool conv1d_supported(const ConvParams &p);
+bool gated_norm_supported(const GatedNormParams &p);
+cudaError_t launch_gated_norm(const GatedNormParams &p, cudaStream_t s);
 cudaError_t launch_conv1d(const ConvParams &p, cudaStream_t s);
 cudaError_t launch_ssd_tc(const M2Params &p, int *status, cudaStream_t s);
 

@@ -335,4 +335,33 @@ ssm_status_t ssm_conv1d_fwd(const ssm_conv_args_t *a, void *stream) {
   return from_cuda(ssm::launch_conv1d(p, s));
 }
 
+ssm_status_t ssm_gated_rmsnorm_fwd(const ssm_gated_norm_args_t *a, void *stream) {
+  if (!a) return SSM_ERR_NULL;
+  if (a->io != SSM_F32 && a->io != SSM_BF16) return SSM_ERR_DTYPE;
+  if (a->rows < 0 || a->width <= 0 || !(a->eps >= 0.f) || a->eps > 3.0e38f) return SSM_ERR_SHAPE;
+  if (a->flags) return SSM_ERR_UNSUPPORTED;
+  if (a->rows > 0 && (!a->y || !a->out)) return SSM_ERR_NULL;
+  if (!all_aligned(a->y, a->z, a->weight, a->out)) return SSM_ERR_ALIGN;
+  const size_t bytes = (size_t)a->rows * a->width * (a->io == SSM_BF16 ? 2 : 4);
+  auto overlap = [](const void *p, const void *q, size_t n) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(p), b0 = reinterpret_cast<uintptr_t>(q);
+    return p && q && n > 0 && a0 < b0 + n && b0 < a0 + n;
+  };
+  // out may be y itself; nothing else may overlap it
+  if (a->out != a->y && overlap(a->out, a->y, bytes)) return SSM_ERR_SHAPE;
+  if (overlap(a->out, a->z, bytes)) return SSM_ERR_SHAPE;
+  ssm::GatedNormParams p;
+  p.rows = a->rows;
+  p.width = a->width;
+  p.io = a->io;
+  p.eps = a->eps;
+  p.y = a->y;
+  p.z = a->z;
+  p.weight = a->weight;
+  p.out = a->out;
+  if (!ssm::gated_norm_supported(p)) return SSM_ERR_UNSUPPORTED;
+  if (a->rows == 0) return SSM_OK;
+  return from_cuda(ssm::launch_gated_norm(p, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

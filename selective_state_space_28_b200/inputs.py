@@ -20,6 +20,10 @@ the pages describe):
   depthwise kernel of width W (fan-in W); conv state ``~ N(0, 1)`` (it holds
   past inputs).  Draw order: w, bias, x, state.  The Mamba-2 2.7B channel
   count is d_inner + 2 G N = 5120 + 256 (the module tree's Conv1d over xBC).
+* Gated norm: ``y, z ~ N(0, 1)`` (the SSD's output and the gate), weight
+  ``1 + 0.1 N(0, 1)`` (the norm's ones initialisation, perturbed so that the
+  weight is exercised); eps 1e-5 (the Mamba-2 configs' layer-norm epsilon).
+  Draw order: weight, y, z.
 """
 import math
 from dataclasses import dataclass, field
@@ -34,7 +38,7 @@ RMS_DT = 4
 
 @dataclass(frozen=True)
 class Workload:
-    """One named scan workload.  ``kind`` is "m1", "ssd", "decode" or "conv"."""
+    """One named scan workload.  ``kind`` is "m1", "ssd", "decode", "conv" or "gnorm"."""
     name: str
     kind: str
     batch: int
@@ -93,6 +97,11 @@ WORKLOADS = {
     "conv_2p7b_b4_l4096_c5376_bf16": Workload(
         "conv_2p7b_b4_l4096_c5376_bf16", "conv", batch=4, seqlen=4096, channels=5376,
         io="bf16", seed=5, extra={"width": 4, "state": True}),
+    # The Mamba-2 2.7B mixer's gated norm after the SSD workload: one row of
+    # heads x head_dim = 5120 values per token.
+    "gnorm_2p7b_b4_l4096_w5120_bf16": Workload(
+        "gnorm_2p7b_b4_l4096_w5120_bf16", "gnorm", batch=4, seqlen=4096, channels=5120,
+        io="bf16", gate=True, rms_eps=1e-5, seed=6),
 }
 
 
@@ -210,6 +219,17 @@ def conv_inputs(batch, seqlen, channels, width=4, io="bf16", seed=0, state=False
     return out
 
 
+def gnorm_inputs(batch, seqlen, width, io="bf16", seed=0, gate=True, weight=True,
+                 device="cpu"):
+    """Inputs of one gated norm: y, z [b, L, width], weight [width]."""
+    g = _gen(seed, device)
+    out = {"weight": (1.0 + 0.1 * torch.randn(width, generator=g, dtype=torch.float32,
+                                              device=device)) if weight else None}
+    out["y"] = _randn((batch, seqlen, width), g, _dtype(io), device)
+    out["z"] = _randn((batch, seqlen, width), g, _dtype(io), device) if gate else None
+    return out
+
+
 def workload_inputs(w: Workload, device="cpu", seed: Optional[int] = None):
     """Inputs of a scan workload (Mamba-1 or SSD)."""
     s = w.seed if seed is None else seed
@@ -219,6 +239,8 @@ def workload_inputs(w: Workload, device="cpu", seed: Optional[int] = None):
     if w.kind == "ssd":
         return ssd_inputs(w.batch, w.seqlen, w.heads, w.head_dim, w.state, w.groups,
                           w.io, w.gate, s, device=device)
+    if w.kind == "gnorm":
+        return gnorm_inputs(w.batch, w.seqlen, w.channels, w.io, s, gate=w.gate, device=device)
     if w.kind == "conv":
         return conv_inputs(w.batch, w.seqlen, w.channels, w.extra.get("width", 4), w.io, s,
                            state=w.extra.get("state", False), device=device)

@@ -217,3 +217,23 @@ def ssm_conv1d_fwd(x, w, bias=None, state=None, *, silu=True, u=None, state_out=
             host_state.copy_(so_h)
         return u_h, so_h
     return u, state_out
+
+
+def ssm_gated_rmsnorm_fwd(y, z=None, weight=None, eps=1e-5, *, out=None, stream=None):
+    """The Mamba-2 mixer's gated norm (include/ssm.h, ssm_gated_rmsnorm_fwd):
+    y * silu(z), RMS-normalised over the last axis (the mixer's whole width,
+    heads x head_dim), times weight.  y, z: [..., width] (float32 or
+    bfloat16); weight: [width] float32.  out may be y (in place)."""
+    sg = _Staging([y, z, weight])
+    y, z, weight = map(sg.dev, (y, z, weight))
+    width = y.shape[-1]
+    rows = y.numel() // width if width else 0
+    if out is None:
+        out = torch.empty_like(y)
+    a = L.GatedNormArgs(rows=rows, width=width, io=_io_of(y), flags=0, eps=eps, y=_ptr(y),
+                        z=_ptr(z), weight=_ptr(weight), out=_ptr(out))
+    L.check(L.lib().ssm_gated_rmsnorm_fwd(ctypes.byref(a), _stream(stream, y.device)),
+            "ssm_gated_rmsnorm_fwd")
+    if sg.host:
+        return sg.back((out,))[0]
+    return out

@@ -24,7 +24,8 @@ def test_exports_every_declared_symbol(lib):
     names = L.header_functions()
     assert {"ssm_scan_fwd", "ssm_scan_workspace", "ssd_chunk_scan_fwd",
             "ssd_chunk_scan_workspace", "ssm_scan_step", "ssm_status_string",
-            "ssm_abi_version", "ssm_conv1d_fwd", "ssm_scan_fwd_static"} <= set(names)
+            "ssm_abi_version", "ssm_conv1d_fwd", "ssm_scan_fwd_static",
+            "ssm_gated_rmsnorm_fwd"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], check=True,
                          capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
@@ -169,3 +170,24 @@ def test_conv_rejects(lib, kw, status):
 def test_conv_empty_batch_is_a_no_op(lib):
     # batch 0: nothing to read or write, no pointer is looked at
     assert lib.ssm_conv1d_fwd(ctypes.byref(_conv(batch=0, x=None, u=None)), None) == OK
+
+
+def _gnorm(**kw):
+    d = dict(rows=8, width=256, io=1, flags=0, eps=1e-5, y=P, z=None, weight=None,
+             out=P + 0x10000)
+    d.update(kw)
+    return L.GatedNormArgs(**d)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(width=0), SHAPE), (dict(rows=-1), SHAPE), (dict(eps=-1.0), SHAPE),
+    (dict(eps=float("nan")), SHAPE), (dict(io=5), DTYPE), (dict(flags=1), UNSUP),
+    (dict(width=49153, out=P + 0x10000000), UNSUP), (dict(y=None), NULL), (dict(out=None), NULL),
+    (dict(y=P + 8), ALIGN), (dict(out=P + 0x100), SHAPE), (dict(z=P + 0x10000), SHAPE),
+])
+def test_gnorm_rejects(lib, kw, status):
+    assert lib.ssm_gated_rmsnorm_fwd(ctypes.byref(_gnorm(**kw)), None) == status
+
+
+def test_gnorm_empty_is_a_no_op(lib):
+    assert lib.ssm_gated_rmsnorm_fwd(ctypes.byref(_gnorm(rows=0, y=None, out=None)), None) == OK
