@@ -42,6 +42,8 @@ def _load():
         for name, argtypes in {
             "orc_m1_scan": [_I64] * 5 + [ctypes.c_uint32, ctypes.c_double] + [_D] * 12 + [ctypes.c_int],
             "orc_m2_scan": [_I64] * 6 + [ctypes.c_uint32] + [_D] * 12 + [ctypes.c_int],
+            "orc_m1_scan_write": [_I64] * 5 + [ctypes.c_uint32, ctypes.c_double] + [_D] * 9
+                                 + [_I64, _D] + [_D] * 3 + [ctypes.c_int],
             "orc_m1_step": [_I64] * 4 + [ctypes.c_uint32, ctypes.c_double] + [_D] * 10,
             "orc_m2_step": [_I64] * 5 + [ctypes.c_uint32] + [_D] * 10,
             "orc_m2_quadratic": [_I64] * 6 + [_D] * 9,
@@ -98,6 +100,28 @@ def m1_scan(x, dt, B, C, A, D=None, z=None, dt_bias=None, h0=None, *,
                              nthreads or default_threads())
     if rc:
         raise ValueError("orc_m1_scan failed: %d" % rc)
+    return y, h_last, states
+
+
+def m1_scan_write(x, dt, B, C, A, D=None, z=None, dt_bias=None, h0=None, *, t, state,
+                  flags=SOFTPLUS, rms_eps=1e-6, want_states=False, nthreads=None):
+    """Mamba-1 scan with the state written at token t ("Mamba", nnterp guide,
+    "The state"): after token t's update the state is replaced by ``state``
+    [b, C, N]; y_t reads it and tokens t+1.. continue from it.
+    Returns (y, h_last, states or None) as m1_scan."""
+    x, dt, z, B, C, A, D, dt_bias, h0, state = map(
+        _f64, (x, dt, z, B, C, A, D, dt_bias, h0, state))
+    b, L, Cn = x.shape
+    G, N = B.shape[2], B.shape[3]
+    y = np.empty_like(x)
+    h_last = np.empty((b, Cn, N))
+    states = np.empty((b, L, Cn, N)) if want_states else None
+    rc = _load().orc_m1_scan_write(b, L, Cn, N, G, flags, rms_eps, _p(x), _p(dt), _p(z),
+                                   _p(B), _p(C), _p(A), _p(D), _p(dt_bias), _p(h0),
+                                   int(t), _p(state), _p(y), _p(h_last), _p(states),
+                                   nthreads or default_threads())
+    if rc:
+        raise ValueError("orc_m1_scan_write failed: %d" % rc)
     return y, h_last, states
 
 

@@ -96,6 +96,8 @@ typedef struct {
   const double *dt_scale; /* [b, L] RMS factor of dt_raw, or NULL */
   const double *bc_norm;  /* [b, L, G, 2, N]: normed B then C, or NULL */
   double *y, *h_last, *states;
+  int64_t t_write;            /* token whose state is replaced, or -1       */
+  const double *state_write;  /* [b, C, N]: the state written at t_write     */
 } m1_ctx;
 
 /* One (batch, channel) pair: the token loop of the recurrence
@@ -131,6 +133,16 @@ static void m1_unit(void *p, int64_t u) {
       h[n] = exp(d * k->A[c * N + n]) * h[n] + d * Bt[n] * xv;
       acc += Ct[n] * h[n];
     }
+    if (k->state_write && t == k->t_write) {
+      /* A state written at token t replaces h_t: y_t reads the written
+       * state, and later tokens continue from it ("Mamba", nnterp guide,
+       * "The state": a write at token t changes token t's own output). */
+      acc = 0.0;
+      for (int64_t n = 0; n < N; ++n) {
+        h[n] = k->state_write[(b * Cn + c) * N + n];
+        acc += Ct[n] * h[n];
+      }
+    }
     double yv = acc + Dc * xv;
     if (k->z) yv *= orc_silu(k->z[i]);
     k->y[i] = yv;
@@ -140,15 +152,16 @@ static void m1_unit(void *p, int64_t u) {
   if (k->h_last) memcpy(k->h_last + (b * Cn + c) * N, h, sizeof(double) * N);
 }
 
-int orc_m1_scan(int64_t batch, int64_t seqlen, int64_t channels, int64_t state,
-                int64_t groups, uint32_t flags, double rms_eps,
-                const double *x, const double *dt, const double *z,
-                const double *B, const double *Cm, const double *A,
-                const double *D, const double *dt_bias, const double *h0,
-                double *y, double *h_last, double *states, int nthreads) {
+static int m1_scan_impl(int64_t batch, int64_t seqlen, int64_t channels, int64_t state,
+                        int64_t groups, uint32_t flags, double rms_eps,
+                        const double *x, const double *dt, const double *z,
+                        const double *B, const double *Cm, const double *A,
+                        const double *D, const double *dt_bias, const double *h0,
+                        double *y, double *h_last, double *states, int nthreads,
+                        int64_t t_write, const double *state_write) {
   if (state > 1024 || groups < 1 || channels % groups) return -1;
   m1_ctx k = {batch, seqlen, channels, state, groups, flags, x, dt, z, B, Cm,
-              A, D, dt_bias, h0, NULL, NULL, y, h_last, states};
+              A, D, dt_bias, h0, NULL, NULL, y, h_last, states, t_write, state_write};
   double *dt_scale = NULL, *bc_norm = NULL;
   if (flags & ORC_RMS_DT) {
     /* One factor per (b, t): 1 / sqrt(mean over channels of dt_raw^2 + eps). */
@@ -180,6 +193,28 @@ int orc_m1_scan(int64_t batch, int64_t seqlen, int64_t channels, int64_t state,
   free(dt_scale);
   free(bc_norm);
   return rc;
+}
+
+int orc_m1_scan(int64_t batch, int64_t seqlen, int64_t channels, int64_t state,
+                int64_t groups, uint32_t flags, double rms_eps,
+                const double *x, const double *dt, const double *z,
+                const double *B, const double *Cm, const double *A,
+                const double *D, const double *dt_bias, const double *h0,
+                double *y, double *h_last, double *states, int nthreads) {
+  return m1_scan_impl(batch, seqlen, channels, state, groups, flags, rms_eps, x, dt, z, B, Cm,
+                      A, D, dt_bias, h0, y, h_last, states, nthreads, -1, NULL);
+}
+
+int orc_m1_scan_write(int64_t batch, int64_t seqlen, int64_t channels, int64_t state,
+                      int64_t groups, uint32_t flags, double rms_eps,
+                      const double *x, const double *dt, const double *z,
+                      const double *B, const double *Cm, const double *A,
+                      const double *D, const double *dt_bias, const double *h0,
+                      int64_t t_write, const double *state_write,
+                      double *y, double *h_last, double *states, int nthreads) {
+  if (t_write < 0 || t_write >= seqlen || !state_write) return -1;
+  return m1_scan_impl(batch, seqlen, channels, state, groups, flags, rms_eps, x, dt, z, B, Cm,
+                      A, D, dt_bias, h0, y, h_last, states, nthreads, t_write, state_write);
 }
 
 /* ------------------------------------------------------------- Mamba-2 */

@@ -51,6 +51,18 @@ int orc_m1_scan(int64_t batch, int64_t seqlen, int64_t channels, int64_t state,
                 const double *D, const double *dt_bias, const double *h0,
                 double *y, double *h_last, double *states, int nthreads);
 
+/* orc_m1_scan with a state written at token t_write ("Mamba", nnterp guide,
+ * "The state": writing the state at token t replaces h_t, so y_t reads the
+ * written state and tokens t+1.. continue from it).  state_write: [b, C, N];
+ * 0 <= t_write < seqlen. */
+int orc_m1_scan_write(int64_t batch, int64_t seqlen, int64_t channels, int64_t state,
+                      int64_t groups, uint32_t flags, double rms_eps,
+                      const double *x, const double *dt, const double *z,
+                      const double *B, const double *Cm, const double *A,
+                      const double *D, const double *dt_bias, const double *h0,
+                      int64_t t_write, const double *state_write,
+                      double *y, double *h_last, double *states, int nthreads);
+
 /* Mamba-2 (SSD) scan, written as the token recurrence.  x, z, y: [b, L, H, P];
  * dt: [b, L, H]; B, Cm: [b, L, G, N]; A, D, dt_bias: [H];
  * h0, h_last: [b, H, N, P] (key side first); states: [b, L, H, N, P].

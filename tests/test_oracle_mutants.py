@@ -88,6 +88,9 @@ MUTANTS = {
     "gated_norm_no_weight": ("o[i] = o[i] * inv * (weight ? weight[i] : 1.0);", "o[i] = o[i] * inv;"),
     "gated_norm_eps_outside": ("const double inv = 1.0 / sqrt(ss / (double)width + eps);",
                                "const double inv = 1.0 / (sqrt(ss / (double)width) + eps);"),
+    "state_write_keeps_old_readout": ("      acc = 0.0;\n      for (int64_t n = 0; n < N; ++n) {\n        h[n] = k->state_write[(b * Cn + c) * N + n];\n        acc += Ct[n] * h[n];\n      }",
+                                      "      for (int64_t n = 0; n < N; ++n) {\n        h[n] = k->state_write[(b * Cn + c) * N + n];\n      }"),
+    "state_write_one_token_late": ("if (k->state_write && t == k->t_write) {", "if (k->state_write && t == k->t_write + 1) {"),
 }
 
 
@@ -126,7 +129,7 @@ def test_mutant_is_caught(key):
         mlib = ctypes.CDLL(_build_mutant(src.replace(old, new), tmp, key))
         for name in ("orc_m1_scan", "orc_m2_scan", "orc_m1_step", "orc_m2_step",
                      "orc_m2_quadratic", "orc_m1_quadratic", "orc_softplus", "orc_silu",
-                     "orc_rms_rows", "orc_conv1d", "orc_gated_rmsnorm"):
+                     "orc_rms_rows", "orc_conv1d", "orc_gated_rmsnorm", "orc_m1_scan_write"):
             getattr(mlib, name).argtypes = getattr(real, name).argtypes
             getattr(mlib, name).restype = getattr(real, name).restype
         caught = None

@@ -496,3 +496,44 @@ def test_gated_norm_gate_before_norm_and_scale_invariance():
     np.testing.assert_allclose(oracle.gated_rmsnorm(y, None, eps=1e-3),
                                y / np.sqrt(np.mean(y ** 2, axis=-1, keepdims=True) + 1e-3),
                                rtol=1e-13)
+
+
+# ------------------------------------------------------- state write at t
+# "Mamba" (nnterp guide), "The state": writing the state at token t replaces
+# h_t; y_t reads the written state and later tokens continue from it.
+
+def test_state_write_of_the_same_state_changes_nothing():
+    d = _m1_rand(2, 11, 6, 4, seed=60)
+    y, h, st = oracle.m1_scan(**d, want_states=True)
+    for t in (0, 4, 10):
+        y2, h2, st2 = oracle.m1_scan_write(**d, t=t, state=st[:, t], want_states=True)
+        assert np.array_equal(y2, y) and np.array_equal(h2, h) and np.array_equal(st2, st)
+
+
+def test_state_write_zero_restarts_the_scan():
+    # writing zeros at t: y_t = D x_t (gated) exactly, and the tokens after t
+    # are a fresh scan from a zero state, bit for bit
+    d = _m1_rand(2, 12, 5, 3, seed=61)
+    t = 5
+    y, h, st = oracle.m1_scan_write(**d, t=t, state=np.zeros((2, 5, 3)), want_states=True)
+    z = d["z"][:, t]
+    np.testing.assert_array_equal(y[:, t], d["D"] * d["x"][:, t] * (z / (1 + np.exp(-z))))
+    assert np.all(st[:, t] == 0.0)
+    tail = {k: (v[:, t + 1:] if k in ("x", "dt", "z", "B", "C") else v) for k, v in d.items()}
+    tail["h0"] = None
+    y_t, h_t, _ = oracle.m1_scan(**tail)
+    assert np.array_equal(y[:, t + 1:], y_t) and np.array_equal(h, h_t)
+    # and the tokens before t are untouched
+    y_full, _, _ = oracle.m1_scan(**d)
+    assert np.array_equal(y[:, :t], y_full[:, :t])
+
+
+def test_state_write_at_the_last_token_is_the_last_state():
+    d = _m1_rand(1, 7, 4, 2, seed=62)
+    s = rng(63).standard_normal((1, 4, 2))
+    y, h, _ = oracle.m1_scan_write(**d, t=6, state=s)
+    assert np.array_equal(h, s)
+    # y_6 = C_6 . s + D x_6, gated
+    c6, x6, z6 = d["C"][0, 6, 0], d["x"][0, 6], d["z"][0, 6]
+    ref = (s[0] @ c6 + d["D"] * x6) * (z6 / (1 + np.exp(-z6)))
+    np.testing.assert_allclose(y[0, 6], ref, rtol=1e-14)
