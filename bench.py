@@ -281,20 +281,30 @@ def n_sets(bytes_per_set):
 
 # ------------------------------------------------------------------ ours
 
-def bench_m1(w, K, W, dist, device, pk, seed_base):
+def bench_m1(w, K, W, dist, device, pk, seed_base, write_at=None):
+    """The Mamba-1 scan; with write_at = t, the same scan with the state
+    written at token t (ssm_scan_fwd_write; the written state adds its bytes)."""
     import torch
     from selective_state_space_28_b200 import inputs as I
     from selective_state_space_28_b200 import ops
-    nb = m1_bytes(w)
+    nb = m1_bytes(w) + (w.batch * w.channels * w.state * 4 if write_at is not None else 0)
     sets = []
     for r in range(n_sets(nb)):
         d = I.workload_inputs(w, device=device, seed=seed_base + 1000 * r)
         d["y"] = torch.empty_like(d["x"])
         d["h_last"] = torch.empty((w.batch, w.channels, w.state), device=device)
+        if write_at is not None:
+            d["s_write"] = torch.zeros((w.batch, w.channels, w.state), device=device)
         sets.append(d)
 
     def step(i):
         d = sets[i % len(sets)]
+        if write_at is not None:
+            ops.ssm_scan_fwd_write(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                                   dt_bias=d["dt_bias"], flags=w.flags, rms_eps=w.rms_eps,
+                                   y=d["y"], h_last=d["h_last"], t=write_at,
+                                   state=d["s_write"])
+            return
         ops.ssm_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
                          dt_bias=d["dt_bias"], flags=w.flags, rms_eps=w.rms_eps,
                          y=d["y"], h_last=d["h_last"])
@@ -578,6 +588,15 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(ach / hbm, 4), "traffic": traffic_for("conv_2p7b"),
                          "kernel": "conv1d_vec_kernel"}}
+        sw = bench_m1(w, max(3, min(K, 10)), 3, dist, device, pk, rank_seed(w.seed, dist.rank),
+                      write_at=w.seqlen // 2)
+        ach = sw["bytes"] / (sw["launch_ms"] * 1e-3) / 1e9
+        wl[w.name + "_state_write_t%d" % (w.seqlen // 2)] = {
+            "value": round(job_value(sw["bytes"], dist.world, sw["ms_per_step"]) / 1e9, 2),
+            "unit": "GB/s", "ms_per_step": round(sw["ms_per_step"], 4),
+            "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
+                         "frac": round(ach / hbm, 4), "traffic": None,
+                         "kernel": "m1_scan_kernel (per-token form, carries the write)"}}
         wg = I.WORKLOADS["gnorm_2p7b_b4_l4096_w5120_bf16"]
         gn = bench_gnorm(wg, max(3, min(K, 20)), max(3, W), dist, device, pk,
                          rank_seed(wg.seed, dist.rank))

@@ -4,7 +4,8 @@
  *
  * Three operations, each a plain C call on plain pointers and sizes:
  *
- *   ssm_scan_fwd        Mamba-1 selective scan over a prompt.
+ *   ssm_scan_fwd        Mamba-1 selective scan over a prompt
+ *                       (ssm_scan_fwd_write: with a state written at one token).
  *   ssd_chunk_scan_fwd  Mamba-2 (SSD) scan over a prompt, chunked.
  *   ssm_scan_step       one decode token against a cached state.
  *   ssm_conv1d_fwd      the mixers' causal depthwise convolution (+ silu),
@@ -136,6 +137,19 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_args_t *args, void *stream);
  * at zero); calls that overlap on the GPU -- on different streams, or from
  * several threads -- race on it and must be serialised by the caller. */
 ssm_status_t ssm_scan_fwd_static(const ssm_scan_args_t *args, void *stream);
+
+/* ssm_scan_fwd_write -- ssm_scan_fwd with the state written at one token.
+ *
+ * Defined by: "Mamba" (nnterp guide), "The state": writing the state at
+ * token t replaces h_t -- y_t reads the written state (a write at token t
+ * changes token t's own output) and tokens t+1.. continue from it.
+ * state_write: [batch, channels, state] float32, 0 <= t_write < seqlen.
+ * Everything else as ssm_scan_fwd (same workspace query); the per-token
+ * float32 kernel carries the write, so this form runs slower than
+ * ssm_scan_fwd.  (The Mamba-2 page marks the same write unavailable for the
+ * chunked scan: there is no SSD counterpart.) */
+ssm_status_t ssm_scan_fwd_write(const ssm_scan_args_t *args, int64_t t_write,
+                                const float *state_write, void *stream);
 
 /* ------------------------------------------------------------------------
  * ssd_chunk_scan_fwd -- Mamba-2 (SSD) scan.

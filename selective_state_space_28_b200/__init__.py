@@ -12,7 +12,7 @@ Import the binding lazily so that the input generators (``.inputs``) can be
 used without a GPU.
 """
 
-__all__ = ["ssm_scan_fwd", "ssd_chunk_scan_fwd", "ssm_scan_step", "ssm_conv1d_fwd",
+__all__ = ["ssm_scan_fwd", "ssm_scan_fwd_write", "ssd_chunk_scan_fwd", "ssm_scan_step", "ssm_conv1d_fwd",
            "ssm_gated_rmsnorm_fwd", "SOFTPLUS", "RMS_BC", "RMS_DT"]
 
 

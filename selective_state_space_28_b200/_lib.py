@@ -96,9 +96,10 @@ def lib():
         L.ssm_scan_step.argtypes = [ctypes.POINTER(StepArgs), _vp]
         L.ssm_conv1d_fwd.argtypes = [ctypes.POINTER(ConvArgs), _vp]
         L.ssm_gated_rmsnorm_fwd.argtypes = [ctypes.POINTER(GatedNormArgs), _vp]
+        L.ssm_scan_fwd_write.argtypes = [ctypes.POINTER(ScanArgs), _i64, _vp, _vp]
         for fn in (L.ssm_scan_fwd, L.ssm_scan_workspace, L.ssd_chunk_scan_fwd,
                    L.ssd_chunk_scan_workspace, L.ssm_scan_step, L.ssm_conv1d_fwd,
-                   L.ssm_gated_rmsnorm_fwd):
+                   L.ssm_gated_rmsnorm_fwd, L.ssm_scan_fwd_write):
             fn.restype = ctypes.c_int
         L.ssm_status_string.argtypes = [ctypes.c_int]
         L.ssm_status_string.restype = ctypes.c_char_p

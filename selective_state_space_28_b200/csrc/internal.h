@@ -20,6 +20,8 @@ struct M1Params {
   int pipelined;  // use the TMA-pipelined kernel where the shape allows
   int variant;    // pipelined-kernel variant (tuning)
   int *status;  // device word set non-zero if a bounded wait ran out, or nullptr
+  int64_t t_write = -1;                 // token whose state is replaced (generic kernel)
+  const float *state_write = nullptr;   // [batch, C, N] state written at t_write
 };
 
 // Mamba-2 token recurrence (the decode step, and the SSD path for shapes the

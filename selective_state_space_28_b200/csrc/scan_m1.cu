@@ -119,6 +119,13 @@ __global__ void __launch_bounds__(kCT *(N / 4))
       h[1] = ex2(d * Al[1]) * h[1] + dx * b4.y;
       h[2] = ex2(d * Al[2]) * h[2] + dx * b4.z;
       h[3] = ex2(d * Al[3]) * h[3] + dx * b4.w;
+      if (p.state_write && t0 + t == p.t_write && cvalid) {
+        // a state written at this token replaces h_t: y_t reads it and the
+        // tokens after continue from it ("Mamba", nnterp guide, "The state")
+        const float4 w4 =
+            *reinterpret_cast<const float4 *>(p.state_write + (b * C + c) * N + 4 * q);
+        h[0] = w4.x; h[1] = w4.y; h[2] = w4.z; h[3] = w4.w;
+      }
       float acc = c4.x * h[0] + c4.y * h[1] + c4.z * h[2] + c4.w * h[3];
 #pragma unroll
       for (int off = LPC / 2; off > 0; off >>= 1)
@@ -186,7 +193,7 @@ cudaError_t launch_t(const M1Params &p, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (p.pipelined && m1_scan_tma_supported(p)) return launch_m1_scan_tma(p, s);
+  if (p.pipelined && !p.state_write && m1_scan_tma_supported(p)) return launch_m1_scan_tma(p, s);
   switch (p.N) {
     case 4: return launch_n<4, T>(p, s);
     case 8: return launch_n<8, T>(p, s);

@@ -195,6 +195,49 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_args_t *a, void *stream) {
   p.pipelined = m1_pipelined();
   p.variant = m1_variant();
   p.status = nullptr;
+  p.t_write = -1;
+  p.state_write = nullptr;
+  return from_cuda(ssm::launch_m1_scan(p, s));
+}
+
+ssm_status_t ssm_scan_fwd_write(const ssm_scan_args_t *a, int64_t t_write,
+                                const float *state_write, void *stream) {
+  size_t ws = 0;
+  ssm_status_t st = check_scan(a, &ws);
+  if (st != SSM_OK) return st;
+  if (a->batch > 0 && !state_write) return SSM_ERR_NULL;
+  if (!all_aligned(state_write)) return SSM_ERR_ALIGN;
+  if (t_write < 0 || t_write >= a->seqlen) return SSM_ERR_SHAPE;
+  if (ws && (!a->workspace || a->workspace_bytes < ws)) return SSM_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (a->batch == 0) return SSM_OK;
+  ssm::M1Params p;
+  p.batch = a->batch;
+  p.L = a->seqlen;
+  p.C = a->channels;
+  p.N = a->state;
+  p.G = a->groups;
+  p.flags = a->flags;
+  p.eps = a->rms_eps;
+  p.io = a->io;
+  p.x = a->x;
+  p.dt = a->dt;
+  p.z = a->z;
+  p.B = a->B;
+  p.Cm = a->C;
+  p.A = a->A;
+  p.D = a->D;
+  p.dt_bias = a->dt_bias;
+  p.h0 = a->h0;
+  p.y = a->y;
+  p.h_last = a->h_last;
+  p.states = a->states;
+  p.rstd = (a->flags & SSM_RMSNORM_DT) ? static_cast<float *>(a->workspace) : nullptr;
+  p.pipelined = 0;  // the generic kernel carries the write
+  p.variant = 0;
+  p.status = nullptr;
+  p.t_write = t_write;
+  p.state_write = state_write;
   return from_cuda(ssm::launch_m1_scan(p, s));
 }
 

@@ -73,7 +73,7 @@ def _io_of(x):
 
 def ssm_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
                  flags=SOFTPLUS, rms_eps=1e-6, want_states=False, y=None, h_last=None,
-                 stream=None):
+                 stream=None, _write=None):
     """Mamba-1 selective scan (include/ssm.h, ssm_scan_fwd).
 
     x, dt, z: [b, L, C]; B, C: [b, L, G, N]; A: [C, N] f32; D, dt_bias: [C] f32;
@@ -81,6 +81,8 @@ def ssm_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
     states [b, L, C, N] f32 or None)."""
     sg = _Staging([x, dt, A, B, C, D, z, dt_bias, h0])
     x, dt, A, B, C, D, z, dt_bias, h0 = map(sg.dev, (x, dt, A, B, C, D, z, dt_bias, h0))
+    if _write is not None:
+        _write = (_write[0], sg.dev(_write[1]))
     b, Lq, Cn = x.shape
     G, N = B.shape[2], B.shape[3]
     if y is None:
@@ -100,8 +102,26 @@ def ssm_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
     if nbytes.value:
         ws = torch.empty(nbytes.value, dtype=torch.uint8, device=x.device)
         a.workspace, a.workspace_bytes = ws.data_ptr(), nbytes.value
-    L.check(lib.ssm_scan_fwd(ctypes.byref(a), _stream(stream, x.device)), "ssm_scan_fwd")
+    if _write is None:
+        L.check(lib.ssm_scan_fwd(ctypes.byref(a), _stream(stream, x.device)), "ssm_scan_fwd")
+    else:
+        L.check(lib.ssm_scan_fwd_write(ctypes.byref(a), int(_write[0]), _ptr(_write[1]),
+                                       _stream(stream, x.device)), "ssm_scan_fwd_write")
     return sg.back((y, h_last, states))
+
+
+def ssm_scan_fwd_write(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, t, state,
+                       flags=SOFTPLUS, rms_eps=1e-6, want_states=False, y=None, h_last=None,
+                       stream=None):
+    """Mamba-1 scan with the state written at token t (include/ssm.h,
+    ssm_scan_fwd_write): h_t is replaced by ``state`` [b, C, N] float32, y_t
+    reads it and tokens t+1.. continue from it.  Arguments and results as
+    ssm_scan_fwd."""
+    if state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    return ssm_scan_fwd(x, dt, A, B, C, D, z, dt_bias, h0, flags=flags, rms_eps=rms_eps,
+                        want_states=want_states, y=y, h_last=h_last, stream=stream,
+                        _write=(t, state))
 
 
 def ssd_workspace_bytes(**shape):

@@ -25,7 +25,7 @@ def test_exports_every_declared_symbol(lib):
     assert {"ssm_scan_fwd", "ssm_scan_workspace", "ssd_chunk_scan_fwd",
             "ssd_chunk_scan_workspace", "ssm_scan_step", "ssm_status_string",
             "ssm_abi_version", "ssm_conv1d_fwd", "ssm_scan_fwd_static",
-            "ssm_gated_rmsnorm_fwd"} <= set(names)
+            "ssm_gated_rmsnorm_fwd", "ssm_scan_fwd_write"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], check=True,
                          capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
@@ -191,3 +191,10 @@ def test_gnorm_rejects(lib, kw, status):
 
 def test_gnorm_empty_is_a_no_op(lib):
     assert lib.ssm_gated_rmsnorm_fwd(ctypes.byref(_gnorm(rows=0, y=None, out=None)), None) == OK
+
+
+@pytest.mark.parametrize("t,state,status", [
+    (-1, P + 0x40000, SHAPE), (8, P + 0x40000, SHAPE), (0, None, NULL), (0, P + 0x40004, ALIGN),
+])
+def test_scan_write_rejects(lib, t, state, status):
+    assert lib.ssm_scan_fwd_write(ctypes.byref(_scan()), t, state, None) == status

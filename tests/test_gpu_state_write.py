@@ -1,0 +1,75 @@
+"""GPU parity of the Mamba-1 scan with the state written at one token
+(ssm_scan_fwd_write, through the C ABI) against the float64 oracle."""
+import pytest
+import torch
+
+import oracle
+from selective_state_space_28_b200 import inputs as I
+from tests.parity import REL, assert_close_normwise
+
+pytestmark = pytest.mark.gpu
+
+
+def _ops():
+    from selective_state_space_28_b200 import ops
+    return ops
+
+
+def _dev(d):
+    return {k: (v.cuda() if v is not None else None) for k, v in d.items()}
+
+
+def _args(d):
+    return (d["x"], d["dt"], d["A"], d["B"], d["C"])
+
+
+def _kw(d):
+    return dict(D=d["D"], z=d["z"], dt_bias=d["dt_bias"], h0=d["h0"])
+
+
+@pytest.mark.parametrize("t", [0, 31, 32, 70, 99])
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_state_write_matches_oracle(cuda_ok, t, io):
+    d = I.m1_inputs(2, 100, 64, 16, io=io, seed=t, h0=True)
+    s = torch.randn((2, 64, 16), generator=torch.Generator().manual_seed(t)) * 0.5
+    y, h, _ = _ops().ssm_scan_fwd_write(*_args(_dev(d)), **_kw(_dev(d)), t=t, state=s.cuda())
+    yr, hr, _ = oracle.m1_scan_write(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                                     dt_bias=d["dt_bias"], h0=d["h0"], t=t, state=s)
+    rel = REL[torch.float32 if io == "f32" else torch.bfloat16]
+    assert_close_normwise(y.float().cpu(), yr, rel, "y")
+    assert_close_normwise(h.cpu(), hr, rel, "h_last")
+
+
+def test_state_write_with_norms_and_states(cuda_ok):
+    d = I.m1_inputs(2, 50, 32, 16, io="f32", seed=3, h0=True)
+    s = torch.zeros((2, 32, 16))
+    flags = I.SOFTPLUS | I.RMS_BC | I.RMS_DT
+    y, h, st = _ops().ssm_scan_fwd_write(*_args(_dev(d)), **_kw(_dev(d)), t=20, state=s.cuda(),
+                                         flags=flags, want_states=True)
+    yr, hr, sr = oracle.m1_scan_write(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"],
+                                      z=d["z"], dt_bias=d["dt_bias"], h0=d["h0"], t=20,
+                                      state=s, flags=flags, want_states=True)
+    assert_close_normwise(y.cpu(), yr, REL[torch.float32], "y")
+    assert_close_normwise(st.cpu(), sr, REL[torch.float32], "states")
+    assert torch.count_nonzero(st[:, 20]) == 0
+
+
+def test_state_write_of_the_scans_own_state_is_the_scan(cuda_ok):
+    # writing back the state the scan had at t reproduces the plain scan on
+    # the same (per-token) kernel: every other token's arithmetic is unchanged
+    d = _dev(I.m1_inputs(1, 80, 32, 16, io="bf16", seed=4, h0=True))
+    ops = _ops()
+    y, h, st = ops.ssm_scan_fwd_write(*_args(d), **_kw(d), t=79, state=torch.zeros(
+        (1, 32, 16), device="cuda"), want_states=True)
+    y2, h2, _ = ops.ssm_scan_fwd_write(*_args(d), **_kw(d), t=40, state=st[:, 40].contiguous())
+    assert torch.equal(y2[:, :79], y[:, :79])
+
+
+def test_state_write_rejects_bad_token(cuda_ok):
+    d = _dev(I.m1_inputs(1, 10, 32, 16, io="f32", seed=5))
+    ops = _ops()
+    from selective_state_space_28_b200._lib import SsmError
+    for t in (-1, 10):
+        with pytest.raises(SsmError):
+            ops.ssm_scan_fwd_write(*_args(d), **_kw(d), t=t,
+                                   state=torch.zeros((1, 32, 16), device="cuda"))
