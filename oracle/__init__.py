@@ -50,6 +50,7 @@ def _load():
             "orc_m1_quadratic": [_I64] * 5 + [_D] * 9,
             "orc_conv1d": [_I64] * 4 + [_D] * 4 + [ctypes.c_int] + [_D] * 2,
             "orc_gated_rmsnorm": [_I64] * 2 + [ctypes.c_double] + [_D] * 4,
+            "orc_m2_attention": [_I64] * 5 + [ctypes.c_uint32] + [_D] * 6,
         }.items():
             fn = getattr(lib, name)
             fn.argtypes = argtypes
@@ -234,6 +235,22 @@ def gated_rmsnorm(y, z=None, weight=None, eps=1e-5):
     if rc:
         raise ValueError("orc_gated_rmsnorm: bad arguments")
     return out
+
+
+def m2_attention(dt, B, C, A, dt_bias=None, *, flags=SOFTPLUS, heads=None):
+    """The hidden attention of the Mamba-2 map ("Mamba-2", "The hidden
+    attention"): alpha [b, H, L, L] (query t, key s), causal, with
+    y_t = sum_s alpha[t, s] x_s + D x_t from a zero state.
+    dt [b, L, H]; B, C [b, L, G, N]; A, dt_bias [H]."""
+    dt, B, C, A, dt_bias = map(_f64, (dt, B, C, A, dt_bias))
+    b, L, H = dt.shape
+    G, N = B.shape[2], B.shape[3]
+    alpha = np.zeros((b, H, L, L))
+    rc = _load().orc_m2_attention(b, L, H, N, G, flags, _p(dt), _p(B), _p(C), _p(A),
+                                  _p(dt_bias), _p(alpha))
+    if rc:
+        raise ValueError("orc_m2_attention: bad arguments")
+    return alpha
 
 
 def softplus(v):

@@ -510,3 +510,39 @@ int orc_gated_rmsnorm(int64_t rows, int64_t width, double eps, const double *y,
   }
   return 0;
 }
+
+/* The hidden attention ("Mamba-2", "The hidden attention"), by its
+ * definition: the decay between key s and query t is the sum of the decays
+ * of tokens s+1 .. t, summed term by term. */
+int orc_m2_attention(int64_t batch, int64_t seqlen, int64_t heads, int64_t state,
+                     int64_t groups, uint32_t flags, const double *dt, const double *B,
+                     const double *Cm, const double *A, const double *dt_bias, double *alpha) {
+  const int64_t L = seqlen, H = heads, N = state, G = groups;
+  if (batch < 0 || L < 0 || H <= 0 || N <= 0 || G <= 0 || H % G || !alpha) return 1;
+  double *beta = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+  if (!beta) return 2;
+  for (int64_t b = 0; b < batch; ++b)
+    for (int64_t h = 0; h < H; ++h) {
+      const int64_t g = h / (H / G);
+      for (int64_t t = 0; t < L; ++t) {
+        double d = dt[(b * L + t) * H + h] + (dt_bias ? dt_bias[h] : 0.0);
+        if (flags & ORC_SOFTPLUS) d = orc_softplus(d);
+        beta[t] = d;
+      }
+      for (int64_t t = 0; t < L; ++t)
+        for (int64_t s2 = 0; s2 < L; ++s2) {
+          double v = 0.0;
+          if (s2 <= t) {
+            double cb = 0.0;
+            for (int64_t n = 0; n < N; ++n)
+              cb += Cm[((b * L + t) * G + g) * N + n] * B[((b * L + s2) * G + g) * N + n];
+            double dsum = 0.0;
+            for (int64_t r = s2 + 1; r <= t; ++r) dsum += beta[r] * A[h];
+            v = cb * exp(dsum) * beta[s2];
+          }
+          alpha[((b * H + h) * L + t) * L + s2] = v;
+        }
+    }
+  free(beta);
+  return 0;
+}

@@ -130,6 +130,17 @@ int orc_conv1d(int64_t batch, int64_t seqlen, int64_t channels, int64_t width,
 int orc_gated_rmsnorm(int64_t rows, int64_t width, double eps, const double *y,
                       const double *z, const double *weight, double *out);
 
+/* The hidden attention of the Mamba-2 (SSD) map ("Mamba-2", nnterp
+ * encyclopedia, "The hidden attention"): per head, the causal [seq, seq]
+ * matrix with y_t = sum_s alpha[t, s] x_s + D x_t (zero initial state),
+ *   alpha[t, s] = (C_t . B_s) * exp(decays_{s+1} + ... + decays_t) * betas_s
+ * for s <= t and 0 above the diagonal, with betas = softplus(dt + dt_bias)
+ * (when ORC_SOFTPLUS) and decays = betas * A_h.  dt: [b, L, H]; B, Cm:
+ * [b, L, G, N]; A, dt_bias: [H]; alpha: [b, H, L, L] (query t, key s). */
+int orc_m2_attention(int64_t batch, int64_t seqlen, int64_t heads, int64_t state,
+                     int64_t groups, uint32_t flags, const double *dt, const double *B,
+                     const double *Cm, const double *A, const double *dt_bias, double *alpha);
+
 /* Elementwise helpers exposed for the pins. */
 double orc_softplus(double v);
 double orc_silu(double v);

@@ -91,6 +91,10 @@ MUTANTS = {
     "state_write_keeps_old_readout": ("      acc = 0.0;\n      for (int64_t n = 0; n < N; ++n) {\n        h[n] = k->state_write[(b * Cn + c) * N + n];\n        acc += Ct[n] * h[n];\n      }",
                                       "      for (int64_t n = 0; n < N; ++n) {\n        h[n] = k->state_write[(b * Cn + c) * N + n];\n      }"),
     "state_write_one_token_late": ("if (k->state_write && t == k->t_write) {", "if (k->state_write && t == k->t_write + 1) {"),
+    "attention_decay_includes_key": ("for (int64_t r = s2 + 1; r <= t; ++r) dsum += beta[r] * A[h];",
+                                     "for (int64_t r = s2; r <= t; ++r) dsum += beta[r] * A[h];"),
+    "attention_beta_of_query": ("v = cb * exp(dsum) * beta[s2];", "v = cb * exp(dsum) * beta[t];"),
+    "attention_not_causal": ("if (s2 <= t) {", "if (1) {"),
 }
 
 
@@ -129,7 +133,8 @@ def test_mutant_is_caught(key):
         mlib = ctypes.CDLL(_build_mutant(src.replace(old, new), tmp, key))
         for name in ("orc_m1_scan", "orc_m2_scan", "orc_m1_step", "orc_m2_step",
                      "orc_m2_quadratic", "orc_m1_quadratic", "orc_softplus", "orc_silu",
-                     "orc_rms_rows", "orc_conv1d", "orc_gated_rmsnorm", "orc_m1_scan_write"):
+                     "orc_rms_rows", "orc_conv1d", "orc_gated_rmsnorm", "orc_m1_scan_write",
+                     "orc_m2_attention"):
             getattr(mlib, name).argtypes = getattr(real, name).argtypes
             getattr(mlib, name).restype = getattr(real, name).restype
         caught = None

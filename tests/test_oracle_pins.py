@@ -537,3 +537,54 @@ def test_state_write_at_the_last_token_is_the_last_state():
     c6, x6, z6 = d["C"][0, 6, 0], d["x"][0, 6], d["z"][0, 6]
     ref = (s[0] @ c6 + d["D"] * x6) * (z6 / (1 + np.exp(-z6)))
     np.testing.assert_allclose(y[0, 6], ref, rtol=1e-14)
+
+
+# ------------------------------------------------------ hidden attention
+# "Mamba-2", "The hidden attention": alpha[t, s] = (C_t . B_s) *
+# exp(decays_{s+1} + ... + decays_t) * betas_s, causal, one [seq, seq]
+# matrix per head; y_t = sum_s alpha[t, s] x_s + D x_t.
+
+def test_attention_rebuilds_the_scan(G=1):
+    d = _m2_rand(2, 23, 4, 3, 5, G=G, seed=70, h0=False, z=False)
+    al = oracle.m2_attention(d["dt"], d["B"], d["C"], d["A"], d["dt_bias"])
+    y, _, _ = oracle.m2_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"],
+                             dt_bias=d["dt_bias"])
+    y_att = np.einsum("bhts,bshp->bthp", al, d["x"]) + d["D"][None, None, :, None] * d["x"]
+    np.testing.assert_allclose(y_att, y, rtol=1e-10, atol=1e-12)
+
+
+def test_attention_matches_the_pages_recipe():
+    # the page's own rebuild: cum = decays.cumsum(0), kept = exp(cum_t - cum_s)
+    # below the diagonal, alpha = einsum(C, B) * kept * betas
+    d = _m2_rand(1, 17, 3, 2, 4, G=1, seed=71, h0=False, z=False)
+    al = oracle.m2_attention(d["dt"], d["B"], d["C"], d["A"], d["dt_bias"])
+    beta = F.softplus(torch.tensor(d["dt"][0] + d["dt_bias"]))          # [seq, heads]
+    decay = beta * torch.tensor(d["A"])
+    cum = decay.cumsum(0)
+    causal = torch.ones(17, 17, dtype=torch.bool).tril()[..., None]
+    kept = (cum[:, None] - cum[None, :]).masked_fill(~causal, -torch.inf).exp()
+    Cg = torch.tensor(d["C"][0]).repeat_interleave(3, 1)
+    Bg = torch.tensor(d["B"][0]).repeat_interleave(3, 1)
+    ref = torch.einsum("thn,shn->tsh", Cg, Bg) * kept * beta           # [t, s, h]
+    np.testing.assert_allclose(al[0], ref.permute(2, 0, 1).numpy(), rtol=1e-10, atol=1e-13)
+
+
+def test_attention_is_causal_with_a_plain_diagonal():
+    d = _m2_rand(1, 9, 2, 2, 3, G=2, seed=72, h0=False, z=False)
+    al = oracle.m2_attention(d["dt"], d["B"], d["C"], d["A"], d["dt_bias"])
+    assert np.all(np.triu(al[0, 0], 1) == 0.0) and np.all(np.triu(al[0, 1], 1) == 0.0)
+    # no decay between a token and itself: alpha[t, t] = (C_t . B_t) betas_t
+    beta = np.logaddexp(0.0, d["dt"][0] + d["dt_bias"])
+    for h in range(2):
+        for t in range(9):
+            cb = d["C"][0, t, h] @ d["B"][0, t, h]
+            assert al[0, h, t, t] == pytest.approx(cb * beta[t, h], rel=1e-13, abs=0)
+
+
+def test_attention_without_decay_is_masked_cb():
+    d = _m2_rand(1, 8, 2, 2, 4, G=1, seed=73, h0=False, z=False)
+    al = oracle.m2_attention(d["dt"], d["B"], d["C"], np.zeros(2), d["dt_bias"], flags=0)
+    beta = d["dt"][0] + d["dt_bias"]                                   # no softplus
+    cb = d["C"][0, :, 0] @ d["B"][0, :, 0].T
+    for h in range(2):
+        np.testing.assert_allclose(al[0, h], np.tril(cb * beta[None, :, h]), rtol=1e-14)
