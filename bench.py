@@ -47,7 +47,7 @@ def parse(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["m1", "ssd", "decode", "decode_layer", "falcon", "conv",
-                                       "gnorm"],
+                                       "gnorm", "attn"],
                     help="run just one workload's timed loop (for profiling); prints its timing")
     return ap.parse_args(argv)
 
@@ -119,6 +119,14 @@ def gnorm_bytes(w):
     e = _esz(w.io)
     rows = w.batch * w.seqlen
     return (3 if w.gate else 2) * rows * w.channels * e + w.channels * 4
+
+
+def attn_bytes(w):
+    """alpha [b, H, L, L] float32 written once (every entry), plus dt, B, C
+    and the per-head parameters read."""
+    e = _esz(w.io)
+    return (4 * w.batch * w.heads * w.seqlen * w.seqlen + w.batch * w.seqlen * w.heads * e
+            + 2 * w.batch * w.seqlen * w.groups * w.state * e + 2 * w.heads * 4)
 
 
 def decode_bytes(w):
@@ -358,6 +366,26 @@ def bench_gnorm(w, K, W, dist, device, pk, seed_base):
             "launches_per_step": 1}
 
 
+def bench_attn(w, K, W, dist, device, pk, seed_base):
+    import torch
+    from selective_state_space_28_b200 import inputs as I
+    from selective_state_space_28_b200 import ops
+    nb = attn_bytes(w)
+    sets = []
+    for r in range(n_sets(nb)):
+        d = I.workload_inputs(w, device=device, seed=seed_base + 1000 * r)
+        d["alpha"] = torch.empty((w.batch, w.heads, w.seqlen, w.seqlen), device=device)
+        sets.append(d)
+
+    def step(i):
+        d = sets[i % len(sets)]
+        ops.ssd_attention_fwd(d["dt"], d["A"], d["B"], d["C"], d["dt_bias"], alpha=d["alpha"])
+    ms = timed(step, K, W, dist, device) / K
+    launch_ms = per_launch_ms(step, max(10, K), device)
+    return {"ms_per_step": ms, "bytes": nb, "launch_ms": launch_ms, "sets": len(sets),
+            "launches_per_step": 2}
+
+
 def bench_ssd(w, K, W, dist, device, pk, seed_base):
     import torch
     from selective_state_space_28_b200 import inputs as I
@@ -482,10 +510,12 @@ def run_only(args):
             "decode": "decode_2p7b_stack_b256", "decode_layer": "decode_2p7b_layer_b256",
             "falcon": "m1_falcon_rms_b4_l8192_c8192_n16_bf16",
             "conv": "conv_2p7b_b4_l4096_c5376_bf16",
-            "gnorm": "gnorm_2p7b_b4_l4096_w5120_bf16"}[args.only]
+            "gnorm": "gnorm_2p7b_b4_l4096_w5120_bf16",
+            "attn": "attn_2p7b_b1_l1024_h80_n128_bf16"}[args.only]
     w = I.WORKLOADS[name]
     fn = {"m1": bench_m1, "falcon": bench_m1, "ssd": bench_ssd, "decode": bench_decode,
-          "decode_layer": bench_decode, "conv": bench_conv, "gnorm": bench_gnorm}[args.only]
+          "decode_layer": bench_decode, "conv": bench_conv, "gnorm": bench_gnorm,
+          "attn": bench_attn}[args.only]
     r = fn(w, args.steps, args.warmup, dist, device, pk, w.seed)
     print(json.dumps({"only": name, "ms_per_step": r["ms_per_step"],
                       "launch_ms": r["launch_ms"]}), flush=True)
@@ -607,6 +637,16 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(ach / hbm, 4), "traffic": traffic_for("gnorm_2p7b"),
                          "kernel": "gated_norm_kernel"}}
+        wa = I.WORKLOADS["attn_2p7b_b1_l1024_h80_n128_bf16"]
+        at = bench_attn(wa, max(3, min(K, 20)), max(3, W), dist, device, pk,
+                        rank_seed(wa.seed, dist.rank))
+        ach = at["bytes"] / (at["launch_ms"] * 1e-3) / 1e9
+        wl[wa.name] = {
+            "value": round(job_value(at["bytes"], dist.world, at["ms_per_step"]) / 1e9, 2),
+            "unit": "GB/s", "ms_per_step": round(at["ms_per_step"], 4),
+            "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
+                         "frac": round(ach / hbm, 4), "traffic": traffic_for("attn_2p7b"),
+                         "kernel": "attn_kernel (+ attn_prep_kernel)"}}
         out["workloads"] = wl
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline_m1(w)

@@ -11,6 +11,7 @@
  *   ssm_conv1d_fwd      the mixers' causal depthwise convolution (+ silu),
  *                       over a prompt or, in place, one decode token.
  *   ssm_gated_rmsnorm_fwd  the Mamba-2 mixer's gated RMS norm after the SSD.
+ *   ssd_attention_fwd   the SSD map's hidden attention matrix, per head.
  *
  * Conventions for every call
  * --------------------------
@@ -302,6 +303,41 @@ typedef struct ssm_gated_norm_args {
 } ssm_gated_norm_args_t;
 
 ssm_status_t ssm_gated_rmsnorm_fwd(const ssm_gated_norm_args_t *args, void *stream);
+
+/* ------------------------------------------------------------------------
+ * ssd_attention_fwd -- the hidden attention of the Mamba-2 (SSD) map.
+ *
+ * Defined by: "Mamba-2" (nnterp encyclopedia), "The hidden attention": per
+ * head the scan is a causal linear map over tokens, y_t = sum_s
+ * alpha[t, s] x_s + D x_t (zero initial state), with
+ *
+ *   alpha[t, s] = (C_t . B_s) * exp(decays_{s+1} + ... + decays_t) * betas_s
+ *
+ * for s <= t and 0 above the diagonal; betas = softplus(dt + dt_bias) when
+ * flags has SSM_DT_SOFTPLUS (else dt + dt_bias), decays = betas * A_h, and
+ * head h reads group h / (heads / groups).
+ *   dt: [batch, seqlen, heads] (io); B, C: [batch, seqlen, groups, state]
+ *   (io); A, dt_bias: [heads] float32 (dt_bias may be NULL);
+ *   alpha: [batch, heads, seqlen, seqlen] float32 (query t, key s), every
+ *   entry written.
+ * state 1..256.  The workspace (ssd_attention_workspace) holds the steps and
+ * the running decay sums (float64).  The decay factor is exact for A <= 0
+ * (a decaying state); it is taken as a product of two factors below the
+ * diagonal 32 x 32 blocks, each <= 1 in that case.
+ * ---------------------------------------------------------------------- */
+typedef struct ssd_attention_args {
+  int64_t batch, seqlen, heads, state, groups;
+  int32_t io;
+  uint32_t flags;
+  const void *dt, *B, *C;
+  const float *A, *dt_bias;
+  float *alpha;
+  void *workspace;
+  size_t workspace_bytes;
+} ssd_attention_args_t;
+
+ssm_status_t ssd_attention_workspace(const ssd_attention_args_t *args, size_t *bytes);
+ssm_status_t ssd_attention_fwd(const ssd_attention_args_t *args, void *stream);
 
 /* A short English description of a status; never NULL. */
 const char *ssm_status_string(ssm_status_t status);

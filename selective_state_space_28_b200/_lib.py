@@ -68,6 +68,13 @@ class GatedNormArgs(ctypes.Structure):
                 ("y", _vp), ("z", _vp), ("weight", _vp), ("out", _vp)]
 
 
+class AttnArgs(ctypes.Structure):
+    _fields_ = [("batch", _i64), ("seqlen", _i64), ("heads", _i64), ("state", _i64),
+                ("groups", _i64), ("io", ctypes.c_int32), ("flags", ctypes.c_uint32),
+                ("dt", _vp), ("B", _vp), ("C", _vp), ("A", _vp), ("dt_bias", _vp),
+                ("alpha", _vp), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
 def header_functions(path=HEADER):
     """Names of the functions include/ssm.h declares."""
     with open(path) as f:
@@ -97,9 +104,13 @@ def lib():
         L.ssm_conv1d_fwd.argtypes = [ctypes.POINTER(ConvArgs), _vp]
         L.ssm_gated_rmsnorm_fwd.argtypes = [ctypes.POINTER(GatedNormArgs), _vp]
         L.ssm_scan_fwd_write.argtypes = [ctypes.POINTER(ScanArgs), _i64, _vp, _vp]
+        L.ssd_attention_fwd.argtypes = [ctypes.POINTER(AttnArgs), _vp]
+        L.ssd_attention_workspace.argtypes = [ctypes.POINTER(AttnArgs),
+                                              ctypes.POINTER(ctypes.c_size_t)]
         for fn in (L.ssm_scan_fwd, L.ssm_scan_workspace, L.ssd_chunk_scan_fwd,
                    L.ssd_chunk_scan_workspace, L.ssm_scan_step, L.ssm_conv1d_fwd,
-                   L.ssm_gated_rmsnorm_fwd, L.ssm_scan_fwd_write):
+                   L.ssm_gated_rmsnorm_fwd, L.ssm_scan_fwd_write, L.ssd_attention_fwd,
+                   L.ssd_attention_workspace):
             fn.restype = ctypes.c_int
         L.ssm_status_string.argtypes = [ctypes.c_int]
         L.ssm_status_string.restype = ctypes.c_char_p

@@ -1,0 +1,321 @@
+// attention.cu -- the hidden attention of the Mamba-2 (SSD) map ("Mamba-2",
+// nnterp encyclopedia, "The hidden attention"): per head the causal
+// [seq, seq] matrix
+//
+//   alpha[t, s] = (C_t . B_s) * exp(decays_{s+1} + ... + decays_t) * betas_s
+//
+// for s <= t (zero above the diagonal), with betas = softplus(dt + dt_bias)
+// and decays = betas * A_h, so that y_t = sum_s alpha[t, s] x_s + D x_t from
+// a zero state.
+//
+// Writing b * H * L^2 float32 values dominates; C . B^T does not depend on the
+// head, so one pass computes each 128 x 128 tile of it on or below the
+// diagonal once per (batch, group) into the workspace (where it stays in L2),
+// and the mask pass -- one CTA per (query tile, key tile, four heads of the
+// group) -- reads its share of the tile once and applies each head's decay
+// mask to it.  The decay between s and t is taken as the
+// difference of a running sum kept in float64 (a pre-pass), so that long
+// sequences lose no precision to the cancellation.  Below the diagonal 32 x 32
+// blocks the factor exp(cum_t - cum_s) is split at the last key r of s's
+// 32-token block into exp(cum_t - cum_r) * exp(cum_r - cum_s), both <= 1 for
+// a decaying state; on the diagonal blocks it is taken element by element.
+#include "common.cuh"
+#include "internal.h"
+
+namespace ssm {
+namespace {
+
+constexpr int kTile = 128;   // query and key tokens per tile
+constexpr int kK = 32;       // state columns per shared-memory chunk of C and B
+constexpr int kPitch = 132;  // floats per row of the k-major chunks (16-byte rows)
+constexpr int kHeadsPerCta = 4;
+
+// Pre-pass: per (batch, head) the step betas_t and the running sum of the
+// log2-decays, cum_t = sum_{r <= t} betas_r A_h log2(e), in float64.  One
+// block per (batch, head), kPrep tokens per round: each thread loads one
+// token, and a block-wide scan (warp shuffles, then the warps' totals)
+// gives the running sums.
+constexpr int kPrep = 1024;
+template <typename T>
+__global__ void __launch_bounds__(kPrep) attn_prep_kernel(AttnParams p) {
+  __shared__ double wsum[kPrep / 32];
+  const int64_t unit = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t b = unit / p.H, h = unit % p.H;
+  const T *dt = static_cast<const T *>(p.dt);
+  const double A2 = (double)p.A[h] * 1.4426950408889634;
+  const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+  double carry = 0.0;
+  for (int64_t t0 = 0; t0 < p.L; t0 += kPrep) {
+    const int64_t t = t0 + tid;
+    float d = 0.f;
+    if (t < p.L) {
+      d = ld(dt + (b * p.L + t) * p.H + h) + bias;
+      if (p.flags & 1u) d = softplus(d);
+    }
+    double v = (double)d * A2;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const double u = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += u;
+    }
+    if (lane == 31) wsum[warp] = v;
+    __syncthreads();
+    double before = carry, total = carry;
+    for (int w = 0; w < kPrep / 32; ++w) {
+      const double x = wsum[w];
+      if (w < warp) before += x;
+      total += x;
+    }
+    if (t < p.L) {
+      p.beta[unit * p.L + t] = d;
+      p.cum[unit * p.L + t] = before + v;
+    }
+    carry = total;
+    __syncthreads();  // wsum is rewritten next round
+  }
+}
+
+// Tile index of query tile qt, key tile kt <= qt in the packed lower
+// triangle of tiles.
+__device__ __forceinline__ int64_t lower_index(int64_t qt, int64_t kt) {
+  return qt * (qt + 1) / 2 + kt;
+}
+
+// C . B^T for every tile on or below the diagonal, once per (batch, group):
+// sixteen CTAs per tile, one per 32 x 32 block, each staging its 32 query and
+// 32 key rows of C and B over the whole state axis in one load (for state up
+// to 128; longer states take more passes).  256 threads: thread (ty, tx)
+// owns row ty and columns 4 tx .. 4 tx + 3 of the block.  The tile goes to
+// the workspace (float32, rows of 128), where it stays in L2 for the mask
+// pass.
+constexpr int kBlk = 32;
+constexpr int kKc = 128;     // state columns per pass
+constexpr int kBPitch = 36;  // floats per row of the k-major staging (16-byte rows)
+template <typename T>
+__global__ void __launch_bounds__(256) attn_cb_kernel(AttnParams p) {
+  __shared__ __align__(16) float Cs[kKc][kBPitch];  // [k][query]
+  __shared__ __align__(16) float Bs[kKc][kBPitch];  // [k][key]
+  const int tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
+  const int64_t L = p.L;
+  // blockIdx.x enumerates (packed lower triangle of tiles) x (16 blocks)
+  const int64_t li = blockIdx.x >> 4;
+  const int blk = blockIdx.x & 15, br = blk >> 2, bc = blk & 3;
+  int64_t qt = (int64_t)((sqrt(8.0 * (double)li + 1.0) - 1.0) / 2.0);
+  while (qt * (qt + 1) / 2 > li) --qt;
+  while ((qt + 1) * (qt + 2) / 2 <= li) ++qt;
+  const int64_t kt = li - qt * (qt + 1) / 2;
+  const int64_t t0 = qt * kTile + br * kBlk, s0 = kt * kTile + bc * kBlk;
+  const int64_t g = blockIdx.y, b = blockIdx.z;
+  const T *Cg = static_cast<const T *>(p.Cm);
+  const T *Bg = static_cast<const T *>(p.B);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int64_t k0 = 0; k0 < p.N; k0 += kKc) {
+    for (int e = tid; e < kBlk * kKc; e += 256) {
+      const int r = e / kKc, k = e % kKc;
+      const int64_t tq = t0 + r, tk = s0 + r;
+      const bool kin = k0 + k < p.N;
+      Cs[k][r] = (tq < L && kin) ? ld(Cg + ((b * L + tq) * p.G + g) * p.N + k0 + k) : 0.f;
+      Bs[k][r] = (tk < L && kin) ? ld(Bg + ((b * L + tk) * p.G + g) * p.N + k0 + k) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < kKc; ++k) {
+      const float a = Cs[k][ty];
+      const float4 c4 = *reinterpret_cast<const float4 *>(&Bs[k][4 * tx]);
+      acc[0] = fmaf(a, c4.x, acc[0]);
+      acc[1] = fmaf(a, c4.y, acc[1]);
+      acc[2] = fmaf(a, c4.z, acc[2]);
+      acc[3] = fmaf(a, c4.w, acc[3]);
+    }
+    __syncthreads();
+  }
+  float *tile = p.cb + ((b * p.G + g) * p.ntri + li) * (int64_t)(kTile * kTile);
+  *reinterpret_cast<float4 *>(tile + (br * kBlk + ty) * kTile + bc * kBlk + 4 * tx) =
+      make_float4(acc[0], acc[1], acc[2], acc[3]);
+}
+
+// The mask pass: one CTA per (query tile, key tile, run of heads of one
+// group), 256 threads with the same element ownership as the C . B^T pass.
+// A tile above the diagonal is zeros; otherwise the thread reads its 64
+// values of C . B^T (from L2) once and, per head, scales them by the decay
+// factors and streams the rows out.
+__global__ void __launch_bounds__(256) attn_mask_kernel(AttnParams p) {
+  __shared__ __align__(16) float colf[kHeadsPerCta][kTile];  // per key: exp2(cum_r - cum_s) beta_s
+  __shared__ __align__(16) float betas[kHeadsPerCta][kTile];
+  __shared__ __align__(16) float rowf[kHeadsPerCta][kTile][4];  // per query, key block
+  __shared__ double cq[kHeadsPerCta][kTile], ck[kHeadsPerCta][kTile];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int64_t L = p.L, H = p.H;
+  const int64_t ntile = (L + kTile - 1) / kTile;
+  const int64_t qt = blockIdx.x / ntile, kt = blockIdx.x % ntile;
+  const int64_t t0 = qt * kTile, s0 = kt * kTile;
+  const int64_t b = blockIdx.z;
+  const int64_t h0 = (int64_t)blockIdx.y * p.heads_per_cta;
+  const int nh = (int)(H - h0 < p.heads_per_cta ? H - h0 : p.heads_per_cta);
+  const int64_t g = h0 / (H / p.G);
+
+  // row i of this thread's 8 x 8 block of head h's tile
+  auto store_row = [&](int64_t h, int i, const float (&v)[8]) {
+    const int64_t t = t0 + 8 * ty + i;
+    if (t >= L) return;
+    float *row = p.alpha + ((b * H + h) * L + t) * L + s0;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int c = 64 * half + 4 * tx;
+      if (s0 + c + 4 <= L && (L & 3) == 0) {
+        st_stream4(reinterpret_cast<float4 *>(row + c),
+                   make_float4(v[4 * half], v[4 * half + 1], v[4 * half + 2], v[4 * half + 3]));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (s0 + c + j < L) row[c + j] = v[4 * half + j];
+      }
+    }
+  };
+
+  if (kt > qt) {  // above the diagonal: zeros
+    const float zero[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int hh = 0; hh < nh; ++hh)
+      for (int i = 0; i < 8; ++i) store_row(h0 + hh, i, zero);
+    return;
+  }
+  // every head's factors first (threads 0..127: one key each; 128..255: one
+  // query each), read straight from the running sums; one barrier
+  for (int hh = 0; hh < nh; ++hh) {
+    const int64_t base = (b * H + h0 + hh) * L;
+    if (tid < kTile) {
+      const int64_t tk = s0 + tid;
+      const int rk = (tid | 31) < (int)(L - s0) ? (tid | 31) : (int)(L - s0 - 1);
+      const double ckt = tk < L ? p.cum[base + tk] : 0.0;
+      const float bt = tk < L ? p.beta[base + tk] : 0.f;
+      colf[hh][tid] = ex2((float)(p.cum[base + s0 + rk] - ckt)) * bt;
+      ck[hh][tid] = ckt;
+      betas[hh][tid] = bt;
+    } else {
+      const int q = tid - kTile;
+      const int64_t tq = t0 + q;
+      const double cqt = tq < L ? p.cum[base + tq] : 0.0;
+      cq[hh][q] = cqt;
+#pragma unroll
+      for (int J = 0; J < 4; ++J) {
+        const int rk = (32 * J + 31) < (int)(L - s0) ? 32 * J + 31 : (int)(L - s0 - 1);
+        rowf[hh][q][J] = ex2((float)(cqt - p.cum[base + s0 + rk]));
+      }
+    }
+  }
+  float acc[8][8];
+  {
+    const float *tile =
+        p.cb + ((b * p.G + g) * p.ntri + lower_index(qt, kt)) * (int64_t)(kTile * kTile);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float *row = tile + (8 * ty + i) * kTile;
+      const float4 u0 = *reinterpret_cast<const float4 *>(row + 4 * tx);
+      const float4 u1 = *reinterpret_cast<const float4 *>(row + 64 + 4 * tx);
+      acc[i][0] = u0.x; acc[i][1] = u0.y; acc[i][2] = u0.z; acc[i][3] = u0.w;
+      acc[i][4] = u1.x; acc[i][5] = u1.y; acc[i][6] = u1.z; acc[i][7] = u1.w;
+    }
+  }
+  __syncthreads();
+
+  const bool diag = qt == kt;
+  for (int hh = 0; hh < nh; ++hh) {
+    const int64_t h = h0 + hh;
+    if (!diag) {
+      // below the diagonal tile: every factor is rowf * colf (one key block
+      // per column half of this thread)
+      const float4 c0 = *reinterpret_cast<const float4 *>(&colf[hh][4 * tx]);
+      const float4 c1 = *reinterpret_cast<const float4 *>(&colf[hh][64 + 4 * tx]);
+      const float cf[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      const int J0 = tx >> 3, J1 = 2 + (tx >> 3);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int qi = 8 * ty + i;
+        const float r0 = rowf[hh][qi][J0], r1 = rowf[hh][qi][J1];
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = acc[i][j] * (r0 * cf[j]);
+#pragma unroll
+        for (int j = 4; j < 8; ++j) v[j] = acc[i][j] * (r1 * cf[j]);
+        store_row(h, i, v);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int qi = 8 * ty + i;
+        const int64_t tq = t0 + qi;
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int kj = (j < 4 ? 4 * tx : 60 + 4 * tx) + j;  // 4 tx + j, or 64 + 4 tx + (j - 4)
+          const int64_t tk = s0 + kj;
+          float f;
+          if (tk > tq) {
+            f = 0.f;
+          } else if ((tq >> 5) > (tk >> 5)) {
+            f = rowf[hh][qi][kj >> 5] * colf[hh][kj];  // below the diagonal 32 x 32 blocks
+          } else {
+            f = ex2((float)(cq[hh][qi] - ck[hh][kj])) * betas[hh][kj];  // on a diagonal block
+          }
+          v[j] = acc[i][j] * f;
+        }
+        store_row(h, i, v);
+      }
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_t(const AttnParams &p, cudaStream_t s) {
+  const int64_t units = p.batch * p.H;
+  attn_prep_kernel<T><<<(unsigned)units, kPrep, 0, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_cb_kernel<T><<<dim3((unsigned)(16 * p.ntri), (unsigned)p.G, (unsigned)p.batch), 256, 0, s>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t ntile = (p.L + kTile - 1) / kTile;
+  dim3 grid((unsigned)(ntile * ntile), (unsigned)((p.H + p.heads_per_cta - 1) / p.heads_per_cta),
+            (unsigned)p.batch);
+  attn_mask_kernel<<<grid, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Heads per CTA: the largest divisor of heads-per-group not above four, so
+// that a CTA's heads share one C . B^T.
+int attn_heads_per_cta(int64_t H, int64_t G) {
+  const int64_t hpg = H / G;
+  for (int k = kHeadsPerCta; k > 1; --k)
+    if (hpg % k == 0) return k;
+  return 1;
+}
+
+bool attention_supported(const AttnParams &p) {
+  const int64_t ntile = (p.L + kTile - 1) / kTile;
+  return p.N >= 1 && p.N <= 256 && ntile * ntile < (1ll << 31) &&
+         16 * (ntile * (ntile + 1) / 2) < (1ll << 31) && p.batch <= 65535 &&
+         p.G <= 65535 && (p.H + p.heads_per_cta - 1) / p.heads_per_cta <= 65535;
+}
+
+// The steps and running sums (float64) per (batch, head, token), then C . B^T
+// of every tile on or below the diagonal per (batch, group).
+size_t attention_workspace_bytes(int64_t batch, int64_t H, int64_t G, int64_t L) {
+  const int64_t ntile = (L + kTile - 1) / kTile;
+  const int64_t ntri = ntile * (ntile + 1) / 2;
+  return (((size_t)(batch * H * L) * (sizeof(double) + sizeof(float)) + 15) & ~(size_t)15) +
+         (size_t)(batch * G * ntri) * kTile * kTile * sizeof(float);
+}
+
+int64_t attention_lower_tiles(int64_t L) {
+  const int64_t ntile = (L + kTile - 1) / kTile;
+  return ntile * (ntile + 1) / 2;
+}
+
+cudaError_t launch_attention(const AttnParams &p, cudaStream_t s) {
+  return p.io == 1 ? launch_t<__nv_bfloat16>(p, s) : launch_t<float>(p, s);
+}
+
+}  // namespace ssm

@@ -73,6 +73,21 @@ struct GatedNormParams {
   void *out;
 };
 
+// The hidden attention of the SSD map, exported as [b, H, L, L] float32.
+struct AttnParams {
+  int64_t batch, L, H, N, G;
+  uint32_t flags;
+  int io;
+  int heads_per_cta;
+  const void *dt, *B, *Cm;
+  const float *A, *dt_bias;
+  float *alpha;
+  float *beta;   // workspace: [b, H, L] steps
+  double *cum;   // workspace: [b, H, L] running log2-decay sums
+  float *cb;     // workspace: [b, G, ntri, 128, 128] C . B^T of the lower tiles
+  int64_t ntri;  // tiles on or below the diagonal
+};
+
 // Each returns cudaSuccess, cudaErrorNotSupported for a shape without a
 // kernel (checked before any launch), or the launch error.
 cudaError_t launch_m1_scan(const M1Params &p, cudaStream_t s);
@@ -89,6 +104,11 @@ bool ssd_tc_supported(const M2Params &p);
 int64_t conv1d_run_length(int64_t L, bool state_in_place);
 bool conv1d_supported(const ConvParams &p);
 bool gated_norm_supported(const GatedNormParams &p);
+int attn_heads_per_cta(int64_t H, int64_t G);
+bool attention_supported(const AttnParams &p);
+size_t attention_workspace_bytes(int64_t batch, int64_t H, int64_t G, int64_t L);
+int64_t attention_lower_tiles(int64_t L);
+cudaError_t launch_attention(const AttnParams &p, cudaStream_t s);
 cudaError_t launch_gated_norm(const GatedNormParams &p, cudaStream_t s);
 cudaError_t launch_conv1d(const ConvParams &p, cudaStream_t s);
 cudaError_t launch_ssd_tc(const M2Params &p, int *status, cudaStream_t s);

@@ -407,4 +407,70 @@ ssm_status_t ssm_gated_rmsnorm_fwd(const ssm_gated_norm_args_t *a, void *stream)
   return from_cuda(ssm::launch_gated_norm(p, static_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+ssm_status_t check_attn(const ssd_attention_args_t *a, size_t *ws, bool shapes_only) {
+  if (!a) return SSM_ERR_NULL;
+  if (a->io != SSM_F32 && a->io != SSM_BF16) return SSM_ERR_DTYPE;
+  if (a->batch < 0 || a->seqlen < 0 || a->heads <= 0 || a->state <= 0 || a->groups <= 0 ||
+      a->heads % a->groups)
+    return SSM_ERR_SHAPE;
+  if (a->flags & ~SSM_DT_SOFTPLUS) return SSM_ERR_UNSUPPORTED;
+  const bool work = a->batch > 0 && a->seqlen > 0;
+  if (!shapes_only && work && (!a->dt || !a->B || !a->C || !a->A || !a->alpha))
+    return SSM_ERR_NULL;
+  if (!shapes_only && !all_aligned(a->dt, a->B, a->C, a->A, a->dt_bias, a->alpha, a->workspace))
+    return SSM_ERR_ALIGN;
+  ssm::AttnParams p;
+  p.batch = a->batch;
+  p.L = a->seqlen;
+  p.H = a->heads;
+  p.N = a->state;
+  p.G = a->groups;
+  p.heads_per_cta = ssm::attn_heads_per_cta(a->heads, a->groups);
+  if (!ssm::attention_supported(p)) return SSM_ERR_UNSUPPORTED;
+  *ws = ssm::attention_workspace_bytes(a->batch, a->heads, a->groups, a->seqlen);
+  return SSM_OK;
+}
+}  // namespace
+
+ssm_status_t ssd_attention_workspace(const ssd_attention_args_t *a, size_t *bytes) {
+  if (!bytes) return SSM_ERR_NULL;
+  size_t ws = 0;
+  ssm_status_t st = check_attn(a, &ws, true);
+  if (st != SSM_OK) return st;
+  *bytes = ws;
+  return SSM_OK;
+}
+
+ssm_status_t ssd_attention_fwd(const ssd_attention_args_t *a, void *stream) {
+  size_t ws = 0;
+  ssm_status_t st = check_attn(a, &ws, false);
+  if (st != SSM_OK) return st;
+  if (a->batch == 0 || a->seqlen == 0) return SSM_OK;
+  if (!a->workspace || a->workspace_bytes < ws) return SSM_ERR_WORKSPACE;
+  ssm::AttnParams p;
+  p.batch = a->batch;
+  p.L = a->seqlen;
+  p.H = a->heads;
+  p.N = a->state;
+  p.G = a->groups;
+  p.flags = a->flags;
+  p.io = a->io;
+  p.heads_per_cta = ssm::attn_heads_per_cta(a->heads, a->groups);
+  p.dt = a->dt;
+  p.B = a->B;
+  p.Cm = a->C;
+  p.A = a->A;
+  p.dt_bias = a->dt_bias;
+  p.alpha = a->alpha;
+  const size_t nbh = (size_t)(a->batch * a->heads * a->seqlen);
+  p.cum = static_cast<double *>(a->workspace);
+  p.beta = reinterpret_cast<float *>(static_cast<char *>(a->workspace) + nbh * sizeof(double));
+  // C . B^T tiles after the steps, on a 16-byte boundary
+  p.cb = reinterpret_cast<float *>(static_cast<char *>(a->workspace) +
+                                   ((nbh * (sizeof(double) + sizeof(float)) + 15) & ~(size_t)15));
+  p.ntri = ssm::attention_lower_tiles(a->seqlen);
+  return from_cuda(ssm::launch_attention(p, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -38,7 +38,8 @@ RMS_DT = 4
 
 @dataclass(frozen=True)
 class Workload:
-    """One named scan workload.  ``kind`` is "m1", "ssd", "decode", "conv" or "gnorm"."""
+    """One named scan workload.  ``kind`` is "m1", "ssd", "decode", "conv", "gnorm"
+    or "attn" (the SSD map's hidden attention; its inputs are the SSD's)."""
     name: str
     kind: str
     batch: int
@@ -102,6 +103,11 @@ WORKLOADS = {
     "gnorm_2p7b_b4_l4096_w5120_bf16": Workload(
         "gnorm_2p7b_b4_l4096_w5120_bf16", "gnorm", batch=4, seqlen=4096, channels=5120,
         io="bf16", gate=True, rms_eps=1e-5, seed=6),
+    # The hidden attention of the Mamba-2 2.7B map for one 1024-token prompt:
+    # 80 heads x 1024 x 1024 float32 (the interpretability workload).
+    "attn_2p7b_b1_l1024_h80_n128_bf16": Workload(
+        "attn_2p7b_b1_l1024_h80_n128_bf16", "attn", batch=1, seqlen=1024, heads=80,
+        head_dim=64, state=128, io="bf16", gate=False, seed=7),
 }
 
 
@@ -236,7 +242,7 @@ def workload_inputs(w: Workload, device="cpu", seed: Optional[int] = None):
     if w.kind == "m1":
         return m1_inputs(w.batch, w.seqlen, w.channels, w.state, w.groups, w.io,
                          w.gate, s, device=device)
-    if w.kind == "ssd":
+    if w.kind in ("ssd", "attn"):
         return ssd_inputs(w.batch, w.seqlen, w.heads, w.head_dim, w.state, w.groups,
                           w.io, w.gate, s, device=device)
     if w.kind == "gnorm":

@@ -257,3 +257,33 @@ def ssm_gated_rmsnorm_fwd(y, z=None, weight=None, eps=1e-5, *, out=None, stream=
     if sg.host:
         return sg.back((out,))[0]
     return out
+
+
+def ssd_attention_fwd(dt, A, B, C, dt_bias=None, *, flags=SOFTPLUS, alpha=None,
+                      workspace=None, stream=None):
+    """The hidden attention of the SSD map (include/ssm.h, ssd_attention_fwd):
+    alpha [b, H, L, L] float32 (query t, key s), causal, with
+    y_t = sum_s alpha[t, s] x_s + D x_t from a zero state.
+    dt [b, L, H] and B, C [b, L, G, N] (float32 or bfloat16); A, dt_bias [H]."""
+    sg = _Staging([dt, A, B, C, dt_bias])
+    dt, A, B, C, dt_bias = map(sg.dev, (dt, A, B, C, dt_bias))
+    b, Lq, H = dt.shape
+    G, N = B.shape[2], B.shape[3]
+    if alpha is None:
+        alpha = torch.empty((b, H, Lq, Lq), dtype=torch.float32, device=dt.device)
+    a = L.AttnArgs(batch=b, seqlen=Lq, heads=H, state=N, groups=G, io=_io_of(dt), flags=flags,
+                   dt=_ptr(dt), B=_ptr(B), C=_ptr(C), A=_ptr(A), dt_bias=_ptr(dt_bias),
+                   alpha=_ptr(alpha))
+    lib = L.lib()
+    nbytes = ctypes.c_size_t(0)
+    L.check(lib.ssd_attention_workspace(ctypes.byref(a), ctypes.byref(nbytes)),
+            "ssd_attention_workspace")
+    if nbytes.value:
+        if workspace is None or workspace.numel() * workspace.element_size() < nbytes.value:
+            workspace = torch.empty(nbytes.value, dtype=torch.uint8, device=dt.device)
+        a.workspace, a.workspace_bytes = workspace.data_ptr(), nbytes.value
+    L.check(lib.ssd_attention_fwd(ctypes.byref(a), _stream(stream, dt.device)),
+            "ssd_attention_fwd")
+    if sg.host:
+        return sg.back((alpha,))[0]
+    return alpha

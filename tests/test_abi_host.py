@@ -25,7 +25,8 @@ def test_exports_every_declared_symbol(lib):
     assert {"ssm_scan_fwd", "ssm_scan_workspace", "ssd_chunk_scan_fwd",
             "ssd_chunk_scan_workspace", "ssm_scan_step", "ssm_status_string",
             "ssm_abi_version", "ssm_conv1d_fwd", "ssm_scan_fwd_static",
-            "ssm_gated_rmsnorm_fwd", "ssm_scan_fwd_write"} <= set(names)
+            "ssm_gated_rmsnorm_fwd", "ssm_scan_fwd_write", "ssd_attention_fwd",
+            "ssd_attention_workspace"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], check=True,
                          capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
@@ -198,3 +199,30 @@ def test_gnorm_empty_is_a_no_op(lib):
 ])
 def test_scan_write_rejects(lib, t, state, status):
     assert lib.ssm_scan_fwd_write(ctypes.byref(_scan()), t, state, None) == status
+
+
+def _attn(**kw):
+    d = dict(batch=1, seqlen=16, heads=4, state=64, groups=1, io=1, flags=1, dt=P, B=P, C=P,
+             A=P, dt_bias=None, alpha=P + 0x100000, workspace=P + 0x200000,
+             workspace_bytes=1 << 20)
+    d.update(kw)
+    return L.AttnArgs(**d)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(heads=0), SHAPE), (dict(groups=3), SHAPE), (dict(state=0), SHAPE),
+    (dict(state=257), UNSUP), (dict(io=2), DTYPE), (dict(flags=2), UNSUP),
+    (dict(alpha=None), NULL), (dict(dt=None), NULL), (dict(alpha=P + 0x100004), ALIGN),
+    (dict(workspace=None), WS), (dict(workspace_bytes=16), WS),
+])
+def test_attention_rejects(lib, kw, status):
+    assert lib.ssd_attention_fwd(ctypes.byref(_attn(**kw)), None) == status
+
+
+def test_attention_workspace_size(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.ssd_attention_workspace(ctypes.byref(_attn(batch=2, seqlen=100, heads=8,
+                                                          dt=None, B=None)), ctypes.byref(n)) == OK
+    # steps and float64 running sums per (batch, head, token), then one
+    # 128 x 128 float32 C . B^T tile per (batch, group) for the single tile
+    assert n.value == 2 * 8 * 100 * 12 + 2 * 1 * 128 * 128 * 4
