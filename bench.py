@@ -626,7 +626,7 @@ def run_ours(args):
             "unit": "GB/s", "ms_per_step": round(sw["ms_per_step"], 4),
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(ach / hbm, 4), "traffic": None,
-                         "kernel": "m1_scan_kernel (per-token form, carries the write)"}}
+                         "kernel": "m1_scan_tma_kernel (write form)"}}
         wg = I.WORKLOADS["gnorm_2p7b_b4_l4096_w5120_bf16"]
         gn = bench_gnorm(wg, max(3, min(K, 20)), max(3, W), dist, device, pk,
                          rank_seed(wg.seed, dist.rank))

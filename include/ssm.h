@@ -145,10 +145,9 @@ ssm_status_t ssm_scan_fwd_static(const ssm_scan_args_t *args, void *stream);
  * token t replaces h_t -- y_t reads the written state (a write at token t
  * changes token t's own output) and tokens t+1.. continue from it.
  * state_write: [batch, channels, state] float32, 0 <= t_write < seqlen.
- * Everything else as ssm_scan_fwd (same workspace query); the per-token
- * float32 kernel carries the write, so this form runs slower than
- * ssm_scan_fwd.  (The Mamba-2 page marks the same write unavailable for the
- * chunked scan: there is no SSD counterpart.) */
+ * Everything else as ssm_scan_fwd (same workspace query).  (The Mamba-2
+ * page marks the same write unavailable for the chunked scan: there is no
+ * SSD counterpart.) */
 ssm_status_t ssm_scan_fwd_write(const ssm_scan_args_t *args, int64_t t_write,
                                 const float *state_write, void *stream);
 

@@ -31,6 +31,8 @@
 #include "sm100.cuh"
 #include "tma.h"
 
+#include <type_traits>
+
 namespace ssm {
 namespace {
 
@@ -112,7 +114,8 @@ struct alignas(128) M1Smem {
 // PK: packed f32x2 state arithmetic (else scalar); UT: token groups per loop
 // iteration (2 lets one group's shuffle reduction overlap the next group's
 // arithmetic).
-template <int N, typename T, int CT, bool HAS_Z, int SWX, int SPL, bool STATES, bool PK, int UT>
+template <int N, typename T, int CT, bool HAS_Z, int SWX, int SPL, bool STATES, bool PK, int UT,
+          bool WR = false>
 __global__ void __launch_bounds__(CT *(N / SPL))
     m1_scan_tma_kernel(const __grid_constant__ CUtensorMap mx,
                        const __grid_constant__ CUtensorMap mdt,
@@ -123,6 +126,7 @@ __global__ void __launch_bounds__(CT *(N / SPL))
   constexpr int NT = CT * G;
   constexpr int NP = SPL / 2;  // state pairs per lane
   constexpr bool kBF16 = sizeof(T) == 2;
+  static_assert(!WR || PK, "the state write is carried by the packed form only");
   using S = M1Smem<N, T, CT>;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   S &s = *reinterpret_cast<S *>(smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u));
@@ -232,92 +236,124 @@ __global__ void __launch_bounds__(CT *(N / SPL))
     }
     __syncthreads();
 
-    // ---- recurrence, G tokens at a time, UT groups per iteration
+    // ---- recurrence, G tokens at a time, UT groups per iteration.  With a
+    // state write, only the group holding the written token takes the form
+    // that lets y read the written state; the others run the plain body.
+    const int tw = (WR && p.t_write >= t0 && p.t_write < t0 + tn) ? (int)(p.t_write - t0) : -1;
 #pragma unroll 1
     for (int tg0 = 0; tg0 < kTL; tg0 += G * UT) {
+      auto group = [&](auto wr) {
 #pragma unroll
-      for (int ug = 0; ug < UT; ++ug) {
-        const int tg = tg0 + ug * G;
-        float part[G];
+        for (int ug = 0; ug < UT; ++ug) {
+          const int tg = tg0 + ug * G;
+          float part[G];
 #pragma unroll
-        for (int u = 0; u < G; ++u) {
-          const int t = tg + u;
-          const float2 ddx = s.ddx[t][cl];
-          const float d = ddx.x, dx = ddx.y;
-          float bv[SPL], cv[SPL], a[SPL];
-          if constexpr (SPL >= 4) {
+          for (int u = 0; u < G; ++u) {
+            const int t = tg + u;
+            const float2 ddx = s.ddx[t][cl];
+            const float d = ddx.x, dx = ddx.y;
+            float bv[SPL], cv[SPL], a[SPL];
+            if constexpr (SPL >= 4) {
 #pragma unroll
-            for (int v = 0; v < SPL / 4; ++v) {
-              const float4 b4 = *reinterpret_cast<const float4 *>(&s.bc[t][0][SPL * q + 4 * v]);
-              const float4 c4 = *reinterpret_cast<const float4 *>(&s.bc[t][1][SPL * q + 4 * v]);
-              bv[4 * v] = b4.x; bv[4 * v + 1] = b4.y; bv[4 * v + 2] = b4.z; bv[4 * v + 3] = b4.w;
-              cv[4 * v] = c4.x; cv[4 * v + 1] = c4.y; cv[4 * v + 2] = c4.z; cv[4 * v + 3] = c4.w;
+              for (int v = 0; v < SPL / 4; ++v) {
+                const float4 b4 = *reinterpret_cast<const float4 *>(&s.bc[t][0][SPL * q + 4 * v]);
+                const float4 c4 = *reinterpret_cast<const float4 *>(&s.bc[t][1][SPL * q + 4 * v]);
+                bv[4 * v] = b4.x; bv[4 * v + 1] = b4.y; bv[4 * v + 2] = b4.z; bv[4 * v + 3] = b4.w;
+                cv[4 * v] = c4.x; cv[4 * v + 1] = c4.y; cv[4 * v + 2] = c4.z; cv[4 * v + 3] = c4.w;
+              }
+            } else {
+              const float2 b2 = *reinterpret_cast<const float2 *>(&s.bc[t][0][2 * q]);
+              const float2 c2 = *reinterpret_cast<const float2 *>(&s.bc[t][1][2 * q]);
+              bv[0] = b2.x; bv[1] = b2.y;
+              cv[0] = c2.x; cv[1] = c2.y;
             }
-          } else {
-            const float2 b2 = *reinterpret_cast<const float2 *>(&s.bc[t][0][2 * q]);
-            const float2 c2 = *reinterpret_cast<const float2 *>(&s.bc[t][1][2 * q]);
-            bv[0] = b2.x; bv[1] = b2.y;
-            cv[0] = c2.x; cv[1] = c2.y;
-          }
-          if constexpr (PK) {
+            if constexpr (PK) {
 #pragma unroll
-            for (int pr = 0; pr < NP; ++pr) {
-              const bool fma_pair = (SWX == 2 && SPL == 4 && pr == 1) && sw_ok;
-              const bool fma_last = (SWX == 1 && pr == NP - 1) && sw_ok;
-              if (fma_pair) {
-                const f2 e = exp2_fma2(d, mk2(A2[2], A2[3]), mk2(lim[2], lim[3]));
-                a[2] = e.x; a[3] = e.y;
+              for (int pr = 0; pr < NP; ++pr) {
+                const bool fma_pair = (SWX == 2 && SPL == 4 && pr == 1) && sw_ok;
+                const bool fma_last = (SWX == 1 && pr == NP - 1) && sw_ok;
+                if (fma_pair) {
+                  const f2 e = exp2_fma2(d, mk2(A2[2], A2[3]), mk2(lim[2], lim[3]));
+                  a[2] = e.x; a[3] = e.y;
+                } else {
+                  const f2 xx = mul2(mk2(d, d), mk2(A2[2 * pr], A2[2 * pr + 1]));
+                  a[2 * pr] = ex2(xx.x);
+                  a[2 * pr + 1] =
+                      fma_last ? exp2_fma1(d, A2[2 * pr + 1], lim[2 * pr + 1]) : ex2(xx.y);
+                }
+              }
+              const f2 dx2 = mk2(dx, dx);
+              f2 yacc = mk2(0.f, 0.f);
+              if constexpr (decltype(wr)::value) {
+                // a state written at this token replaces h_t before y_t reads
+                // it ("Mamba", nnterp guide, "The state")
+#pragma unroll
+                for (int pr = 0; pr < NP; ++pr) {
+                  const f2 hn = fma2(mk2(a[2 * pr], a[2 * pr + 1]), mk2(h[2 * pr], h[2 * pr + 1]),
+                                     mul2(dx2, mk2(bv[2 * pr], bv[2 * pr + 1])));
+                  h[2 * pr] = hn.x;
+                  h[2 * pr + 1] = hn.y;
+                }
+                if (t == tw && cvalid) {
+#pragma unroll
+                  for (int j = 0; j < SPL; ++j) h[j] = p.state_write[(b * C + c) * N + SPL * q + j];
+                }
+#pragma unroll
+                for (int pr = 0; pr < NP; ++pr)
+                  yacc = fma2(mk2(cv[2 * pr], cv[2 * pr + 1]), mk2(h[2 * pr], h[2 * pr + 1]), yacc);
               } else {
-                const f2 xx = mul2(mk2(d, d), mk2(A2[2 * pr], A2[2 * pr + 1]));
-                a[2 * pr] = ex2(xx.x);
-                a[2 * pr + 1] =
-                    fma_last ? exp2_fma1(d, A2[2 * pr + 1], lim[2 * pr + 1]) : ex2(xx.y);
+#pragma unroll
+                for (int pr = 0; pr < NP; ++pr) {
+                  const f2 hn = fma2(mk2(a[2 * pr], a[2 * pr + 1]), mk2(h[2 * pr], h[2 * pr + 1]),
+                                     mul2(dx2, mk2(bv[2 * pr], bv[2 * pr + 1])));
+                  h[2 * pr] = hn.x;
+                  h[2 * pr + 1] = hn.y;
+                  yacc = fma2(mk2(cv[2 * pr], cv[2 * pr + 1]), hn, yacc);
+                }
+              }
+              part[u] = yacc.x + yacc.y;
+            } else {
+#pragma unroll
+              for (int j = 0; j < SPL; ++j) {
+                const bool fma_j = (j >= SPL - SWX) && sw_ok;
+                a[j] = fma_j ? exp2_fma1(d, A2[j], lim[j]) : ex2(d * A2[j]);
+              }
+              float acc = 0.f;
+#pragma unroll
+              for (int j = 0; j < SPL; ++j) {
+                h[j] = fmaf(a[j], h[j], dx * bv[j]);
+                acc = fmaf(cv[j], h[j], acc);
+              }
+              part[u] = acc;
+            }
+            if constexpr (STATES) {
+              if (cvalid && t < tn) {
+                float *sp = p.states + ((b * L + t0 + t) * C + c) * N + SPL * q;
+#pragma unroll
+                for (int j = 0; j < SPL; j += 2)
+                  *reinterpret_cast<float2 *>(sp + j) = make_float2(h[j], h[j + 1]);
               }
             }
-            const f2 dx2 = mk2(dx, dx);
-            f2 yacc = mk2(0.f, 0.f);
-#pragma unroll
-            for (int pr = 0; pr < NP; ++pr) {
-              const f2 hn = fma2(mk2(a[2 * pr], a[2 * pr + 1]), mk2(h[2 * pr], h[2 * pr + 1]),
-                                 mul2(dx2, mk2(bv[2 * pr], bv[2 * pr + 1])));
-              h[2 * pr] = hn.x;
-              h[2 * pr + 1] = hn.y;
-              yacc = fma2(mk2(cv[2 * pr], cv[2 * pr + 1]), hn, yacc);
-            }
-            part[u] = yacc.x + yacc.y;
-          } else {
-#pragma unroll
-            for (int j = 0; j < SPL; ++j) {
-              const bool fma_j = (j >= SPL - SWX) && sw_ok;
-              a[j] = fma_j ? exp2_fma1(d, A2[j], lim[j]) : ex2(d * A2[j]);
-            }
-            float acc = 0.f;
-#pragma unroll
-            for (int j = 0; j < SPL; ++j) {
-              h[j] = fmaf(a[j], h[j], dx * bv[j]);
-              acc = fmaf(cv[j], h[j], acc);
-            }
-            part[u] = acc;
           }
-          if constexpr (STATES) {
-            if (cvalid && t < tn) {
-              float *sp = p.states + ((b * L + t0 + t) * C + c) * N + SPL * q;
-#pragma unroll
-              for (int j = 0; j < SPL; j += 2)
-                *reinterpret_cast<float2 *>(sp + j) = make_float2(h[j], h[j + 1]);
+          const float yq = transpose_reduce<G>(part, q);
+          const int tt = tg + q;  // this lane's token
+          if (tt < tn && cvalid) {
+            float yv = yq + Dc * ld(&s.x[buf][tt][cl]);
+            if (HAS_Z) {
+              const float zv = ld(&s.z[buf][tt][cl]);
+              yv *= kBF16 ? silu_tanh(zv) : silu(zv);
             }
+            st(&s.y[tt][cl], yv);
           }
         }
-        const float yq = transpose_reduce<G>(part, q);
-        const int tt = tg + q;  // this lane's token
-        if (tt < tn && cvalid) {
-          float yv = yq + Dc * ld(&s.x[buf][tt][cl]);
-          if (HAS_Z) {
-            const float zv = ld(&s.z[buf][tt][cl]);
-            yv *= kBF16 ? silu_tanh(zv) : silu(zv);
-          }
-          st(&s.y[tt][cl], yv);
-        }
+      };
+      if constexpr (WR) {
+        if (tw >= tg0 && tw < tg0 + G * UT)
+          group(std::true_type{});
+        else
+          group(std::false_type{});
+      } else {
+        group(std::false_type{});
       }
     }
     __syncthreads();
@@ -352,7 +388,7 @@ CUtensorMapDataType tmap_type() {
 }
 
 template <int N, typename T, int CT, bool HZ, int SWX, int SPL, bool ST, bool PK = true,
-          int UT = 1>
+          int UT = 1, bool WR = false>
 cudaError_t launch_tma(const M1Params &p, cudaStream_t s) {
   CUtensorMap mx, mdt, mz, mB, mC;
   const uint64_t es = sizeof(T);
@@ -377,7 +413,7 @@ cudaError_t launch_tma(const M1Params &p, cudaStream_t s) {
         !encode_tiled(&mC, tmap_type<T>(), 3, p.Cm, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
-  auto k = m1_scan_tma_kernel<N, T, CT, HZ, SWX, SPL, ST, PK, UT>;
+  auto k = m1_scan_tma_kernel<N, T, CT, HZ, SWX, SPL, ST, PK, UT, WR>;
   const size_t smem = sizeof(M1Smem<N, T, CT>) + 128;
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -392,6 +428,8 @@ cudaError_t launch_tma(const M1Params &p, cudaStream_t s) {
 template <int N, typename T, bool HZ>
 cudaError_t launch_v(const M1Params &p, cudaStream_t s) {
   if (p.states) return launch_tma<N, T, 16, HZ, 0, 4, true>(p, s);
+  // a state written at one token: the default lane split, with the write
+  if (p.state_write) return launch_tma<N, T, 16, HZ, 0, 2, false, true, 1, true>(p, s);
   // variant = 4 * (packed) + 2 * (two groups per iteration) + (2 states per lane)
   const bool ok32 = p.G == 1 || (p.C / p.G) % 32 == 0;
   switch (p.variant) {

@@ -233,8 +233,8 @@ ssm_status_t ssm_scan_fwd_write(const ssm_scan_args_t *a, int64_t t_write,
   p.h_last = a->h_last;
   p.states = a->states;
   p.rstd = (a->flags & SSM_RMSNORM_DT) ? static_cast<float *>(a->workspace) : nullptr;
-  p.pipelined = 0;  // the generic kernel carries the write
-  p.variant = 0;
+  p.pipelined = m1_pipelined();  // the pipelined kernel carries it where it can (N = 16)
+  p.variant = m1_variant();
   p.status = nullptr;
   p.t_write = t_write;
   p.state_write = state_write;

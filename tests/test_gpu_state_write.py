@@ -55,14 +55,28 @@ def test_state_write_with_norms_and_states(cuda_ok):
 
 
 def test_state_write_of_the_scans_own_state_is_the_scan(cuda_ok):
-    # writing back the state the scan had at t reproduces the plain scan on
-    # the same (per-token) kernel: every other token's arithmetic is unchanged
-    d = _dev(I.m1_inputs(1, 80, 32, 16, io="bf16", seed=4, h0=True))
+    # writing back the state the scan itself had at t reproduces the plain
+    # scan bit for bit: the state at t comes from a scan of tokens 0..t on the
+    # same kernel, and the write form does the same arithmetic per token
+    d = _dev(I.m1_inputs(2, 150, 64, 16, io="bf16", seed=4, h0=True))
     ops = _ops()
-    y, h, st = ops.ssm_scan_fwd_write(*_args(d), **_kw(d), t=79, state=torch.zeros(
-        (1, 32, 16), device="cuda"), want_states=True)
-    y2, h2, _ = ops.ssm_scan_fwd_write(*_args(d), **_kw(d), t=40, state=st[:, 40].contiguous())
-    assert torch.equal(y2[:, :79], y[:, :79])
+    y, h, _ = ops.ssm_scan_fwd(*_args(d), **_kw(d))
+    t = 70
+    head = {k: (v[:, :t + 1].contiguous() if k in ("x", "dt", "z", "B", "C") else v)
+            for k, v in d.items()}
+    _, h_t, _ = ops.ssm_scan_fwd(*_args(head), **_kw(head))
+    y2, h2, _ = ops.ssm_scan_fwd_write(*_args(d), **_kw(d), t=t, state=h_t)
+    assert torch.equal(y2, y) and torch.equal(h2, h)
+
+
+def test_state_write_per_token_kernel_with_states(cuda_ok):
+    # with per-token states the per-token kernel carries the write; its
+    # states at t are the written state and later ones continue from it
+    d = _dev(I.m1_inputs(1, 80, 32, 16, io="f32", seed=6, h0=True))
+    s = torch.randn((1, 32, 16), device="cuda")
+    y, h, st = _ops().ssm_scan_fwd_write(*_args(d), **_kw(d), t=33, state=s, want_states=True)
+    assert torch.equal(st[:, 33], s)
+    assert torch.equal(st[:, -1], h)
 
 
 def test_state_write_rejects_bad_token(cuda_ok):
