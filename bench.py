@@ -607,6 +607,7 @@ def run_ours(args):
             "unit": "GB/s", "ms_per_step": round(f["ms_per_step"], 4),
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(ach / hbm, 4), "traffic": traffic_for("m1_scan_falcon"),
+                         "kernel": "m1_scan_tma_kernel (+ dt_rms_kernel)",
                          "note": "algorithmic bytes exclude the step-norm pre-pass re-read"}}
         wc = I.WORKLOADS["conv_2p7b_b4_l4096_c5376_bf16"]
         cv = bench_conv(wc, max(3, min(K, 20)), max(3, W), dist, device, pk,
@@ -646,7 +647,7 @@ def run_ours(args):
             "unit": "GB/s", "ms_per_step": round(at["ms_per_step"], 4),
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(ach / hbm, 4), "traffic": traffic_for("attn_2p7b"),
-                         "kernel": "attn_kernel (+ attn_prep_kernel)"}}
+                         "kernel": "attn_mask_kernel (+ attn_prep_kernel, attn_cb_kernel)"}}
         out["workloads"] = wl
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline_m1(w)
