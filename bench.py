@@ -80,6 +80,20 @@ def m1_bytes(w):
     return n
 
 
+def m1_sfu_roofline(w, launch_ms, clocks):
+    """The unit that binds the Mamba-1 scan: the special-function unit.  Per
+    (token, channel) it evaluates N decays exp(d A), the softplus (ex2, lg2)
+    and, with a gate, one tanh; its nominal rate is 16 results per clock per
+    SM, 148 SMs, at the SM clock sampled under load."""
+    ops = w.batch * w.seqlen * w.channels * (w.state + 2 + (1 if w.gate else 0))
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+    peak = 148 * 16 * mhz * 1e6
+    ach = ops / (launch_ms * 1e-3)
+    return {"ops_per_launch": ops, "achieved_gops": round(ach / 1e9, 1),
+            "peak_gops": round(peak / 1e9, 1), "frac": round(ach / peak, 4),
+            "peak_source": "nominal 16/clk/SM x 148 SMs x sampled SM clock"}
+
+
 def ssd_bytes(w):
     e = _esz(w.io)
     n = 2 * w.batch * w.seqlen * w.heads * w.head_dim * e  # x, y
@@ -562,7 +576,8 @@ def run_ours(args):
                      "unit": "GB/s", "frac": round(achieved / hbm, 4),
                      "traffic": traffic_for("m1_scan_130m" if generic else "m1_scan_tma_130m"),
                      "peak_source": "%s hbm_gbs (copy)" % pk["_source"],
-                     "kernel": "m1_scan_kernel" if generic else "m1_scan_tma_kernel"},
+                     "kernel": "m1_scan_kernel" if generic else "m1_scan_tma_kernel",
+                     "sfu": m1_sfu_roofline(w, r["launch_ms"], clocks)},
         "clocks": clocks,
         "gpu_launches": r["launches_per_step"] * K,
     }

@@ -12,24 +12,23 @@
 // decode form of the same convolution.
 //
 // HBM-streaming layout: a thread owns V = 4 consecutive channels (an 8-byte
-// (bf16) or 16-byte (f32) vector of the tokens-first rows) over a run of kRun tokens, keeps the W - 1
-// previous inputs in registers, and reads each input once (plus a W - 1 token
-// halo at the start of its run, mostly from L2) and writes each output once,
-// with streaming (evict-first) vector loads and stores, kAhead tokens'
-// loads in flight; a warp covers 32 consecutive vectors of a row, so every
-// access is coalesced.
+// (bf16) or 16-byte (f32) vector of the tokens-first rows) over a run of kRun
+// tokens, keeps the W - 1 previous inputs in registers, and reads each input
+// once (plus a W - 1 token halo at the start of its run, mostly from L2) and
+// writes each output once; a warp covers 32 consecutive vectors of a row, so
+// every access is coalesced.  The inputs reach the thread through its own
+// shared-memory slots, copied asynchronously several batches ahead, so that
+// enough bytes are in flight per SM without holding them in registers.
 #include "common.cuh"
 #include "internal.h"
 
 namespace ssm {
 namespace {
 
-constexpr int kRun = 64;    // tokens per thread (when the state is not updated in place)
-constexpr int kAhead = 8;  // loads in flight per thread
+constexpr int kRun = 128;  // tokens per thread (when the state is not updated in place)
 
 // Streaming (evict-first) vector loads and stores through the compiler's
-// intrinsics, so that loads of later tokens can be issued ahead of earlier
-// stores.
+// intrinsics (the halo loads and the output stores).
 template <typename T> struct Vec;
 template <> struct Vec<__nv_bfloat16> {
   static constexpr int V = 4;
@@ -64,11 +63,39 @@ template <typename T> __device__ __forceinline__ float act(float v, bool on) {
 }
 
 // Vector form: channels % V == 0.  Thread =
-// (batch row, vector of V channels, run of kRun tokens).
+// (batch row, vector of V channels, run of kRun tokens).  A thread's next
+// kTok-token batches are copied into its own shared-memory slots with
+// cp.async, kStages - 1 batches ahead: the copies in flight hold no
+// registers, and each thread waits only for its own copies (no barrier).
+// Four stages of 8 tokens measured best for bf16 (24 tokens, 192 bytes in
+// flight per thread); float32 vectors, twice the size, keep three.
+constexpr int kTok = 8;
+constexpr int kStages = 4;
+
+template <int BYTES>
+__device__ __forceinline__ void cp_async(void *dst, const void *src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  if constexpr (BYTES == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(d), "l"(src), "n"(BYTES)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 template <typename T, int W>
 __global__ void __launch_bounds__(128)
     conv1d_vec_kernel(ConvParams p) {
   constexpr int V = Vec<T>::V;
+  using Raw = typename Vec<T>::Raw;
+  constexpr int NS = sizeof(Raw) == 16 ? 3 : kStages;
+  constexpr int NT = sizeof(Raw) == 16 ? 8 : kTok;
+  __shared__ Raw stage[NS][NT][128];
   const int64_t nvec = p.Cc / V;
   const int64_t gv = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (gv >= nvec * p.batch) return;
@@ -79,6 +106,22 @@ __global__ void __launch_bounds__(128)
   const int64_t t1 = t0 + p.run < L ? t0 + p.run : L;
   const T *x = static_cast<const T *>(p.x);
   T *u = static_cast<T *>(p.u);
+  const int tid = threadIdx.x;
+  const int nb = (int)((t1 - t0 + NT - 1) / NT);  // batches in this run
+
+  const T *px = x + (b * L + t0) * Cc + c0;  // next row to copy
+  int64_t tc = t0;                            // its token
+  auto issue = [&](int slot) {
+#pragma unroll
+    for (int a = 0; a < NT; ++a) {
+      if (tc < t1) cp_async<sizeof(Raw)>(&stage[slot][a][tid], px);
+      px += Cc;
+      ++tc;
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int s = 0; s < NS - 1; ++s) issue(s);
 
   float w[V][W], bias[V];
 #pragma unroll
@@ -100,17 +143,17 @@ __global__ void __launch_bounds__(128)
         hist[j][v] = p.state_in ? p.state_in[((b * Cc) + c0 + v) * (W - 1) + (W - 1) + tau] : 0.f;
     }
   }
-  // kAhead tokens' loads are issued before any of them is used
-  for (int64_t tb = t0; tb < t1; tb += kAhead) {
-    typename Vec<T>::Raw raw[kAhead];
+  T *pu = u + (b * L + t0) * Cc + c0;
+  for (int i = 0; i < nb; ++i) {
+    issue((i + NS - 1) % NS);  // the slot batch i - 1 used (an empty group past the end)
+    cp_async_wait<NS - 1>();   // batch i has landed
+    const int slot = i % NS;
+    const int na = (int)(t1 - (t0 + (int64_t)i * NT) < NT ? t1 - (t0 + (int64_t)i * NT) : NT);
 #pragma unroll
-    for (int a = 0; a < kAhead; ++a)
-      if (tb + a < t1) raw[a] = Vec<T>::load(x + (b * L + tb + a) * Cc + c0);
-#pragma unroll
-    for (int a = 0; a < kAhead; ++a) {
-      if (tb + a >= t1) break;
+    for (int a = 0; a < NT; ++a) {
+      if (a >= na) break;
       float xv[V], o[V];
-      Vec<T>::widen(raw[a], xv);
+      Vec<T>::widen(stage[slot][a][tid], xv);
 #pragma unroll
       for (int v = 0; v < V; ++v) {
         float acc = fmaf(w[v][W - 1], xv[v], bias[v]);
@@ -118,7 +161,8 @@ __global__ void __launch_bounds__(128)
         for (int j = 0; j < W - 1; ++j) acc = fmaf(w[v][W - 2 - j], hist[j][v], acc);
         o[v] = act<T>(acc, p.silu);
       }
-      Vec<T>::store(u + (b * L + tb + a) * Cc + c0, o);
+      Vec<T>::store(pu, o);
+      pu += Cc;
 #pragma unroll
       for (int j = W - 2; j > 0; --j)
 #pragma unroll
@@ -129,6 +173,7 @@ __global__ void __launch_bounds__(128)
       }
     }
   }
+  cp_async_wait<0>();
   // The run that ends the sequence leaves the state: the last W - 1 inputs,
   // oldest first (from before the sequence when it is shorter than that).
   if (p.state_out && t1 == L) {
@@ -187,8 +232,14 @@ cudaError_t launch_w(const ConvParams &p, cudaStream_t s) {
   const int64_t runs = (p.L + p.run - 1) / p.run;
   const int64_t units = vec ? p.batch * (p.Cc / V) : p.batch * p.Cc;
   dim3 grid((unsigned)((units + 127) / 128), (unsigned)runs);
-  if (vec)
+  if (vec) {
+    // the slots (24-32 KB per CTA) need the shared-memory carve-out for
+    // several CTAs per SM
+    static const cudaError_t carve = cudaFuncSetAttribute(
+        conv1d_vec_kernel<T, W>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    (void)carve;
     conv1d_vec_kernel<T, W><<<grid, 128, 0, s>>>(p);
+  }
   else
     conv1d_scalar_kernel<T, W><<<grid, 128, 0, s>>>(p);
   return cudaGetLastError();

@@ -79,6 +79,28 @@ def test_state_write_per_token_kernel_with_states(cuda_ok):
     assert torch.equal(st[:, -1], h)
 
 
+def test_state_write_130m_full_size_sampled(cuda_ok):
+    """The state write at full Mamba-130m size (b8 L2048 C1536 N16, bf16), at
+    token 1024, in the launch configuration the benchmark times; the oracle
+    checks a sample of channels of two batch rows (channels are independent)."""
+    w = I.WORKLOADS["m1_130m_b8_l2048_c1536_n16_bf16"]
+    d = I.workload_inputs(w)
+    s = torch.randn((w.batch, w.channels, w.state),
+                    generator=torch.Generator().manual_seed(1024)) * 0.5
+    dd = _dev(d)
+    y, h, _ = _ops().ssm_scan_fwd_write(*_args(dd), D=dd["D"], z=dd["z"],
+                                        dt_bias=dd["dt_bias"], t=1024, state=s.cuda())
+    rows, cols = [0, 7], list(range(0, 64)) + list(range(1472, 1536))
+    sel = torch.tensor(cols)
+    sub = {k: d[k][rows][:, :, sel] for k in ("x", "dt", "z")}
+    yr, hr, _ = oracle.m1_scan_write(sub["x"], sub["dt"], d["B"][rows], d["C"][rows],
+                                     d["A"][sel], d["D"][sel], z=sub["z"],
+                                     dt_bias=d["dt_bias"][sel], t=1024,
+                                     state=s[rows][:, sel])
+    assert_close_normwise(y[rows][:, :, sel.cuda()].float().cpu(), yr, REL[torch.bfloat16], "y")
+    assert_close_normwise(h[rows][:, sel.cuda()].cpu(), hr, REL[torch.bfloat16], "h_last")
+
+
 def test_state_write_rejects_bad_token(cuda_ok):
     d = _dev(I.m1_inputs(1, 10, 32, 16, io="f32", seed=5))
     ops = _ops()
