@@ -81,10 +81,10 @@ def m1_bytes(w):
 
 
 def m1_sfu_roofline(w, launch_ms, clocks):
-    """The unit that binds the Mamba-1 scan: the special-function unit.  Per
-    (token, channel) it evaluates N decays exp(d A), the softplus (ex2, lg2)
-    and, with a gate, one tanh; its nominal rate is 16 results per clock per
-    SM, 148 SMs, at the SM clock sampled under load."""
+    """The Mamba-1 scan's arithmetic floor on the special-function unit.
+    Per (token, channel) it evaluates N decays exp(d A), the softplus (ex2,
+    lg2) and, with a gate, one tanh; the unit's nominal rate is 16 results
+    per clock per SM, 148 SMs, at the SM clock sampled under load."""
     ops = w.batch * w.seqlen * w.channels * (w.state + 2 + (1 if w.gate else 0))
     mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
     peak = 148 * 16 * mhz * 1e6
