@@ -423,8 +423,11 @@ def bench_ssd(w, K, W, dist, device, pk, seed_base):
                                y=d["y"], h_last=d["h_last"], workspace=wsb)
     ms = timed(step, K, W, dist, device) / K
     launch_ms = per_launch_ms(step, max(5, K), device)
+    # a workspace beyond the status word means the last wave is cut into
+    # sequence segments: two SSD launches and the carry between them
+    launches = 3 if ws > 256 else 1
     return {"ms_per_step": ms, "bytes": nb, "flops": ssd_flops(w), "launch_ms": launch_ms,
-            "tokens": w.batch * w.seqlen, "sets": len(sets), "launches_per_step": 1}
+            "tokens": w.batch * w.seqlen, "sets": len(sets), "launches_per_step": launches}
 
 
 def bench_decode(w, K, W, dist, device, pk, seed_base):

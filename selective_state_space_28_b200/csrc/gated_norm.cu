@@ -8,11 +8,13 @@
 // the mean taken over a token's whole row (heads x head_dim).  The statistic
 // needs every head of the token, so it is a pass of its own after the SSD.
 //
-// One CTA per row: the first pass reads y and z with 16-byte streaming loads,
-// keeps g in shared memory and accumulates its sum of squares; a block
-// reduction gives the row's scale; the second pass writes out.  Every input
-// is read once and every output written once.  out may be y itself (the whole
-// row is read before any of it is written).
+// One CTA per row: the first pass reads y and z with 16-byte streaming loads
+// (for rows up to 8192 bf16 / 4096 float32 values, all of a thread's loads
+// are issued before any is used, so enough bytes are in flight), keeps g in
+// shared memory and accumulates its sum of squares; a block reduction gives
+// the row's scale; the second pass writes out.  Every input is read once and
+// every output written once.  out may be y itself (the whole row is read
+// before any of it is written).
 #include "common.cuh"
 #include "internal.h"
 
@@ -63,6 +65,29 @@ __device__ __forceinline__ float block_sum(float v, float *red) {
   return t;
 }
 
+// Raw 16-byte vectors, widened after all of a thread's loads are issued.
+template <typename T> struct NRaw;
+template <> struct NRaw<__nv_bfloat16> {
+  using R = uint4;
+  static __device__ __forceinline__ R load(const __nv_bfloat16 *p) {
+    return __ldcs(reinterpret_cast<const uint4 *>(p));
+  }
+  static __device__ __forceinline__ void widen(const R &w, float (&f)[8]) {
+    f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+    f[4] = bf16lo(w.z); f[5] = bf16hi(w.z); f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
+  }
+};
+template <> struct NRaw<float> {
+  using R = float4;
+  static __device__ __forceinline__ R load(const float *p) {
+    return __ldcs(reinterpret_cast<const float4 *>(p));
+  }
+  static __device__ __forceinline__ void widen(const R &v, float (&f)[4]) {
+    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+  }
+};
+constexpr int kMaxVec = 4;  // vectors per thread held in flight at once
+
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads) gated_norm_kernel(GatedNormParams p) {
   extern __shared__ float4 g4[];  // [width]: this row's gated values
@@ -75,21 +100,49 @@ __global__ void __launch_bounds__(kThreads) gated_norm_kernel(GatedNormParams p)
   float ss = 0.f;
   if constexpr (VEC) {
     constexpr int V = NVec<T>::V;
-    for (int64_t i = (int64_t)threadIdx.x * V; i < W; i += (int64_t)kThreads * V) {
-      float yv[V], zv[V];
-      NVec<T>::load(y + i, yv);
-      if (z) NVec<T>::load(z + i, zv);
-      float gv[V];
+    if (W <= (int64_t)kThreads * V * kMaxVec) {
+      // every load of the thread issued before any is used
+      typename NRaw<T>::R ry[kMaxVec], rz[kMaxVec];
 #pragma unroll
-      for (int v = 0; v < V; ++v) {
-        gv[v] = z ? yv[v] * gate<T>(zv[v]) : yv[v];
-        ss = fmaf(gv[v], gv[v], ss);
+      for (int k = 0; k < kMaxVec; ++k) {
+        const int64_t i = ((int64_t)k * kThreads + threadIdx.x) * V;
+        if (i < W) {
+          ry[k] = NRaw<T>::load(y + i);
+          if (z) rz[k] = NRaw<T>::load(z + i);
+        }
       }
-      // 16-byte shared stores: a thread's V values are contiguous, so scalar
-      // stores would put lanes 32 / V apart on the same bank
 #pragma unroll
-      for (int v = 0; v < V; v += 4)
-        *reinterpret_cast<float4 *>(&g[i + v]) = make_float4(gv[v], gv[v + 1], gv[v + 2], gv[v + 3]);
+      for (int k = 0; k < kMaxVec; ++k) {
+        const int64_t i = ((int64_t)k * kThreads + threadIdx.x) * V;
+        if (i < W) {
+          float yv[V], zv[V], gv[V];
+          NRaw<T>::widen(ry[k], yv);
+          if (z) NRaw<T>::widen(rz[k], zv);
+#pragma unroll
+          for (int v = 0; v < V; ++v) {
+            gv[v] = z ? yv[v] * gate<T>(zv[v]) : yv[v];
+            ss = fmaf(gv[v], gv[v], ss);
+          }
+#pragma unroll
+          for (int v = 0; v < V; v += 4)
+            *reinterpret_cast<float4 *>(&g[i + v]) = make_float4(gv[v], gv[v + 1], gv[v + 2], gv[v + 3]);
+        }
+      }
+    } else {
+      for (int64_t i = (int64_t)threadIdx.x * V; i < W; i += (int64_t)kThreads * V) {
+        float yv[V], zv[V];
+        NVec<T>::load(y + i, yv);
+        if (z) NVec<T>::load(z + i, zv);
+        float gv[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+          gv[v] = z ? yv[v] * gate<T>(zv[v]) : yv[v];
+          ss = fmaf(gv[v], gv[v], ss);
+        }
+#pragma unroll
+        for (int v = 0; v < V; v += 4)
+          *reinterpret_cast<float4 *>(&g[i + v]) = make_float4(gv[v], gv[v + 1], gv[v + 2], gv[v + 3]);
+      }
     }
   } else {
     for (int64_t i = threadIdx.x; i < W; i += kThreads) {

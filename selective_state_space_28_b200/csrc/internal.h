@@ -101,6 +101,15 @@ bool m1_step_supported(int64_t N);
 // Tensor-core SSD (bf16 I/O, state 128, head dim 64, no per-token states).
 // `status` is a device word the kernel sets non-zero if a bounded wait ran out.
 bool ssd_tc_supported(const M2Params &p);
+// How the tensor-core SSD cuts the (batch, head) units of a partial last wave
+// into sequence segments (nseg == 1: no cut), and the workspace that takes.
+struct SsdSplit {
+  int64_t ntail = 0;
+  int nseg = 1;
+};
+SsdSplit ssd_tc_split(int64_t batch, int64_t H, int64_t L, int sms);
+size_t ssd_tc_split_bytes(const SsdSplit &r);
+int device_sm_count();  // the current device's SMs (148 when it cannot be read)
 int64_t conv1d_run_length(int64_t L, bool state_in_place);
 bool conv1d_supported(const ConvParams &p);
 bool gated_norm_supported(const GatedNormParams &p);
@@ -111,6 +120,7 @@ int64_t attention_lower_tiles(int64_t L);
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t s);
 cudaError_t launch_gated_norm(const GatedNormParams &p, cudaStream_t s);
 cudaError_t launch_conv1d(const ConvParams &p, cudaStream_t s);
-cudaError_t launch_ssd_tc(const M2Params &p, int *status, cudaStream_t s);
+cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split, void *seg_ws,
+                          cudaStream_t s);
 
 }  // namespace ssm

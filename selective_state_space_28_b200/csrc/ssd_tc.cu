@@ -55,6 +55,8 @@
 #include "sm100.cuh"
 #include "tma.h"
 
+#include <algorithm>
+
 namespace ssm {
 namespace {
 
@@ -111,6 +113,15 @@ struct SsdTcParams {
   __nv_bfloat16 *y;
   float *h_last;
   int *status;
+  // Work of a 1-D grid: blocks [0, nfull) run the whole (batch, head) units
+  // 0 .. nfull - 1 (unit = b H + h); the others run segments seg_lo .. nseg - 1
+  // of the tail units tail0 .. tail0 + ntail - 1, segment s covering tiles
+  // [s nch / nseg, (s + 1) nch / nseg) of the sequence.
+  int64_t nfull, tail0, ntail;
+  int nseg, seg_lo;
+  float *seg_hend;       // [ntail][nseg][N][P]: end state from the segment's own start state
+  float *seg_decay;      // [ntail][nseg]: product of the segment's tile decays
+  const float *seg_hin;  // [ntail][nseg][N][P]: the state entering each segment
 };
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
@@ -184,10 +195,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   SsdSmem &s = *reinterpret_cast<SsdSmem *>(base);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t hd = blockIdx.x, b = blockIdx.y;
   const int64_t L = p.L, H = p.H;
+  // This CTA's unit, its tiles [cb, cb + nch), where its start state comes
+  // from and where its end state goes.  With seg_lo == 0 (the first pass over
+  // the tail) a segment other than the first starts from zeros, writes no y
+  // and leaves its end state and decay product for the carry; with seg_lo > 0
+  // it starts from the carried state and writes y (and the last one h_last).
+  const int nch_all = (int)((L + kQ - 1) / kQ);
+  int64_t unit;
+  int cb = 0, ce = nch_all;
+  const float *h0u;
+  float *hlu, *decu = nullptr;
+  bool write_y = true;
+  if ((int64_t)blockIdx.x < p.nfull) {
+    unit = blockIdx.x;
+    h0u = p.h0 ? p.h0 + unit * kN * kP : nullptr;
+    hlu = p.h_last ? p.h_last + unit * kN * kP : nullptr;
+  } else {
+    const int per = p.nseg - p.seg_lo;
+    const int64_t r = (int64_t)blockIdx.x - p.nfull;
+    const int64_t tu = r / per;
+    const int sg = p.seg_lo + (int)(r % per);
+    const int64_t slot = tu * p.nseg + sg;
+    unit = p.tail0 + tu;
+    cb = (int)((int64_t)sg * nch_all / p.nseg);
+    ce = (int)((int64_t)(sg + 1) * nch_all / p.nseg);
+    if (p.seg_lo == 0) {
+      h0u = (sg == 0 && p.h0) ? p.h0 + unit * kN * kP : nullptr;
+      hlu = p.seg_hend + slot * kN * kP;
+      decu = p.seg_decay + slot;
+      write_y = sg == 0;
+    } else {
+      h0u = p.seg_hin + slot * kN * kP;
+      hlu = (sg == p.nseg - 1 && p.h_last) ? p.h_last + unit * kN * kP : nullptr;
+    }
+  }
+  const int64_t hd = unit % H, b = unit / H;
   const int g = (int)(hd / (H / p.G));
-  const int nch = (int)((L + kQ - 1) / kQ);
+  const int nch = ce - cb;
   // TMEM lane quarter of this warp (warp i may only touch lanes 32 (i % 4) ..)
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
 
@@ -214,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The bf16 copy of the initial state, for Y(0), goes to Hb[1] (tile c
   // reads Hb[(c + 1) & 1]).
   if (warp < 4) {
-    const float *src = p.h0 ? p.h0 + ((b * H + hd) * kN + tid) * kP : nullptr;
+    const float *src = h0u ? h0u + tid * kP : nullptr;
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc) {
       float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
@@ -244,11 +289,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = c & 1;
         if (c >= 2 && !wait1(s, &s.empty[st], ((c >> 1) + 1) & 1, p.status, 1)) break;
         mbar_expect_tx(&s.full[st], 5 * kQ * 128);
-        tma_load_3d(s.C[st][0], &mC, &s.full[st], g * kN, c * kQ, (int)b);
-        tma_load_3d(s.C[st][1], &mC, &s.full[st], g * kN + 64, c * kQ, (int)b);
-        tma_load_3d(s.B[st][0], &mB, &s.full[st], g * kN, c * kQ, (int)b);
-        tma_load_3d(s.B[st][1], &mB, &s.full[st], g * kN + 64, c * kQ, (int)b);
-        tma_load_4d(s.X[st], &mX, &s.full[st], 0, (int)hd, c * kQ, (int)b);
+        const int tq = (cb + c) * kQ;
+        tma_load_3d(s.C[st][0], &mC, &s.full[st], g * kN, tq, (int)b);
+        tma_load_3d(s.C[st][1], &mC, &s.full[st], g * kN + 64, tq, (int)b);
+        tma_load_3d(s.B[st][0], &mB, &s.full[st], g * kN, tq, (int)b);
+        tma_load_3d(s.B[st][1], &mB, &s.full[st], g * kN + 64, tq, (int)b);
+        tma_load_4d(s.X[st], &mX, &s.full[st], 0, (int)hd, tq, (int)b);
         issued = c + 1;
       }
       // Leave no copy in flight: the last two tiles issued have landed (a
@@ -369,14 +415,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto fetch_dt = [&](int c) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int64_t t = (int64_t)c * kQ + 4 * lane + q;
+        const int64_t t = (int64_t)(cb + c) * kQ + 4 * lane + q;
         dtraw[q] = t < L ? (uint32_t)dtb[(b * L + t) * H + hd] : 0u;
       }
     };
     fetch_dt(0);
     for (int c = 0; c < nch; ++c) {
       const int k = c & 1;
-      const int64_t t0 = (int64_t)c * kQ;
+      const int64_t t0 = (int64_t)(cb + c) * kQ;
       const int valid = (int)(L - t0 < kQ ? L - t0 : kQ);
       // step, log2-decay and inclusive sums over the whole tile (needs only
       // dt, so it runs while the tile's TMA is in flight)
@@ -524,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n = tid;
     float h[kP];
     {
-      const float *src = p.h0 ? p.h0 + ((b * H + hd) * kN + n) * kP : nullptr;
+      const float *src = h0u ? h0u + n * kP : nullptr;
 #pragma unroll
       for (int q = 0; q < kP; q += 4) {
         const float4 v = src ? *reinterpret_cast<const float4 *>(src + q)
@@ -532,6 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         h[q] = v.x; h[q + 1] = v.y; h[q + 2] = v.z; h[q + 3] = v.w;
       }
     }
+    float dprod = 1.f;  // the segment's decay product (the carry's factor)
     for (int c = 0; c < nch; ++c) {
       const int k = c & 1;
       // h = a h + Sc (thread = row n); a comes from the mask group, whose
@@ -540,6 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!waitw(s, &s.scdone[k], (c >> 1) & 1, p.status, 12)) break;
       tc_fence_after();
       const float a_c = s.a[c & 3];
+      dprod *= a_c;
 #pragma unroll
       for (int hh = 0; hh < 4; ++hh) {
         uint32_t r[16];
@@ -566,19 +614,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.stdone[k]);
     }
-    if (!aborted(s) && p.h_last) {
-      float *dst = p.h_last + ((b * H + hd) * kN + n) * kP;
+    if (!aborted(s) && hlu) {
+      float *dst = hlu + n * kP;
 #pragma unroll
       for (int q = 0; q < kP; q += 4)
         *reinterpret_cast<float4 *>(dst + q) = make_float4(h[q], h[q + 1], h[q + 2], h[q + 3]);
     }
+    if (!aborted(s) && decu && n == 0) *decu = dprod;
   } else {
     // ------------------------------------------------------------ output group
     const int i = tid - 256;  // token of the tile; TMEM lane i
     uint4 zr[8];
     auto load_z = [&](int c) {
-      const int64_t t = (int64_t)c * kQ + i;
-      if (p.z && c < nch && t < L) {
+      const int64_t t = (int64_t)(cb + c) * kQ + i;
+      if (write_y && p.z && c < nch && t < L) {
         const __nv_bfloat16 *zp = p.z + ((b * L + t) * H + hd) * kP;
 #pragma unroll
         for (int q = 0; q < 8; ++q) zr[q] = ld_cs_u4(zp + 8 * q);
@@ -587,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     load_z(0);
     for (int c = 0; c < nch; ++c) {
       const int k = c & 1;
-      const int64_t t = (int64_t)c * kQ + i;
+      const int64_t t = (int64_t)(cb + c) * kQ + i;
       if (!waitw(s, &s.yready[k], (c >> 1) & 1, p.status, 13)) break;
       tc_fence_after();
       __nv_bfloat16 *yp = p.y + ((b * L + t) * H + hd) * kP;
@@ -604,7 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&s.yfree[k]);
         }
-        if (t < L) {
+        if (write_y && t < L) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             const int q = 4 * hh + q4;
@@ -634,6 +683,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 13) tmem_dealloc(tb, kTmemCols);
 }
 
+// The state entering each segment of a tail unit: segment 0 started from the
+// unit's own start state, so its end state is exact; the state is linear in
+// the start state, so segment s's exact end is its end from zeros plus its
+// decay product times the state that entered it.  Block = tail unit.
+__global__ void __launch_bounds__(256)
+    ssd_seg_carry_kernel(const float *hend, const float *decay, float *hin, int nseg) {
+  constexpr int kNP = kN * kP;
+  const int64_t tu = blockIdx.x;
+  const float *he = hend + tu * nseg * kNP;
+  const float *dc = decay + tu * nseg;
+  float *hi = hin + tu * nseg * kNP;
+  for (int e = threadIdx.x * 4; e < kNP; e += 256 * 4) {
+    float4 h = *reinterpret_cast<const float4 *>(he + e);
+    for (int sg = 1; sg < nseg; ++sg) {
+      *reinterpret_cast<float4 *>(hi + (int64_t)sg * kNP + e) = h;
+      if (sg + 1 < nseg) {
+        const float4 l = *reinterpret_cast<const float4 *>(he + (int64_t)sg * kNP + e);
+        const float d = dc[sg];
+        h = make_float4(fmaf(d, h.x, l.x), fmaf(d, h.y, l.y), fmaf(d, h.z, l.z), fmaf(d, h.w, l.w));
+      }
+    }
+  }
+}
+
 bool encode(CUtensorMap *m, const void *ptr, int rank, const uint64_t *dims,
             const uint64_t *strides, const uint32_t *box) {
   return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, ptr, dims, strides, box,
@@ -644,12 +717,37 @@ bool encode(CUtensorMap *m, const void *ptr, int rank, const uint64_t *dims,
 
 bool ssd_tc_supported(const M2Params &p) {
   return p.io == 1 && p.N == kN && p.P == kP && p.states == nullptr && p.H <= 65535 &&
-         p.L < (1ll << 31) && p.batch <= 65535;
+         p.L < (1ll << 31) && p.batch <= 65535 && p.batch * p.H < (1ll << 31);
+}
+
+// One CTA per (batch, head) unit fills `sms` SMs a wave at a time; when the
+// last wave is partial, its units are cut into segments that together fill
+// one wave.  A cut pays for itself only with three segments or more (the
+// segments run twice, once from zeros and once from the carried state), and
+// a segment keeps at least four tiles.
+SsdSplit ssd_tc_split(int64_t batch, int64_t H, int64_t L, int sms) {
+  SsdSplit r;
+  const int64_t units = batch * H, nch = (L + kQ - 1) / kQ;
+  if (sms <= 0 || units <= 0) return r;
+  const int64_t tail = units % sms;  // units of the partial wave (all, below one wave)
+  if (tail == 0) return r;
+  const int64_t nseg = std::min<int64_t>(sms / tail, nch / 4);
+  if (nseg < 3) return r;
+  r.ntail = tail;
+  r.nseg = (int)nseg;
+  return r;
+}
+
+size_t ssd_tc_split_bytes(const SsdSplit &r) {
+  if (r.nseg <= 1) return 0;
+  const size_t slots = (size_t)r.ntail * (size_t)r.nseg;
+  return slots * (2 * (size_t)kN * kP + 4) * sizeof(float);
 }
 
 size_t ssd_tc_smem_bytes() { return sizeof(SsdSmem) + 1024; }
 
-cudaError_t launch_ssd_tc(const M2Params &p, int *status, cudaStream_t stream) {
+cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split, void *seg_ws,
+                          cudaStream_t stream) {
   const int64_t GN = p.G * kN;
   CUtensorMap mX, mB, mC;
   {
@@ -681,6 +779,14 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, cudaStream_t stream) {
   q.y = static_cast<__nv_bfloat16 *>(p.y);
   q.h_last = p.h_last;
   q.status = status;
+  q.nfull = p.batch * p.H;
+  q.tail0 = 0;
+  q.ntail = 0;
+  q.nseg = 1;
+  q.seg_lo = 0;
+  q.seg_hend = nullptr;
+  q.seg_decay = nullptr;
+  q.seg_hin = nullptr;
   const size_t smem = ssd_tc_smem_bytes();
   static bool attr_set = false;
   if (!attr_set) {
@@ -689,8 +795,34 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid((unsigned)p.H, (unsigned)p.batch);
-  ssd_tc_kernel<<<grid, kThreads, smem, stream>>>(mX, mB, mC, q);
+  if (split.nseg <= 1) {
+    ssd_tc_kernel<<<(unsigned)q.nfull, kThreads, smem, stream>>>(mX, mB, mC, q);
+    return cudaGetLastError();
+  }
+  // Tail cut into segments: (1) every segment of the tail units from its own
+  // start (the unit's start state for the first, zeros for the others),
+  // (2) the carry, (3) the whole units and segments 1.. from the carried state.
+  const int64_t units = q.nfull, slots = split.ntail * split.nseg;
+  float *hend = static_cast<float *>(seg_ws);
+  float *hin = hend + slots * kN * kP;
+  float *dec = hin + slots * kN * kP;
+  q.nfull = 0;
+  q.tail0 = units - split.ntail;
+  q.ntail = split.ntail;
+  q.nseg = split.nseg;
+  q.seg_hend = hend;
+  q.seg_decay = dec;
+  q.seg_hin = hin;
+  ssd_tc_kernel<<<(unsigned)slots, kThreads, smem, stream>>>(mX, mB, mC, q);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  ssd_seg_carry_kernel<<<(unsigned)split.ntail, 256, 0, stream>>>(hend, dec, hin, split.nseg);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  q.nfull = units - split.ntail;
+  q.seg_lo = 1;
+  ssd_tc_kernel<<<(unsigned)(q.nfull + split.ntail * (split.nseg - 1)), kThreads, smem, stream>>>(
+      mX, mB, mC, q);
   return cudaGetLastError();
 }
 

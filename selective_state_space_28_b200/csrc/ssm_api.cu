@@ -44,6 +44,22 @@ int m1_pipelined() {
   return v;
 }
 
+}  // namespace
+
+namespace ssm {
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();  // (no device here: size for a B200)
+    return 148;
+  }
+  return n;
+}
+}  // namespace ssm
+
+namespace {
+
 ssm_status_t from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return SSM_OK;
   if (e == cudaErrorNotSupported) return SSM_ERR_UNSUPPORTED;
@@ -83,7 +99,9 @@ ssm_status_t check_scan(const ssm_scan_args_t *a, size_t *ws, bool shapes_only =
   return SSM_OK;
 }
 
-// The tensor-core SSD path keeps a device status word in the workspace.
+// The tensor-core SSD path keeps a device status word at the start of the
+// workspace, then (when the last wave's units are cut into segments) the
+// segments' end states, carried states and decay products.
 constexpr size_t kSsdStatusBytes = 256;
 
 ssm::M2Params ssd_params(const ssd_scan_args_t *a) {
@@ -127,7 +145,10 @@ ssm_status_t check_ssd(const ssd_scan_args_t *a, size_t *ws, bool shapes_only = 
     return SSM_ERR_ALIGN;
   if (!ssm::m2_recurrent_supported(a->state, a->head_dim) || a->batch > 65535)
     return SSM_ERR_UNSUPPORTED;
-  *ws = ssm::ssd_tc_supported(ssd_params(a)) ? kSsdStatusBytes : 0;
+  *ws = ssm::ssd_tc_supported(ssd_params(a))
+            ? kSsdStatusBytes + ssm::ssd_tc_split_bytes(ssm::ssd_tc_split(
+                                    a->batch, a->heads, a->seqlen, ssm::device_sm_count()))
+            : 0;
   return SSM_OK;
 }
 
@@ -264,7 +285,10 @@ ssm_status_t ssd_chunk_scan_fwd(const ssd_scan_args_t *a, void *stream) {
   if (ssm::ssd_tc_supported(p)) {
     int *status = static_cast<int *>(a->workspace);
     if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return SSM_ERR_CUDA;
-    return from_cuda(ssm::launch_ssd_tc(p, status, s));
+    const ssm::SsdSplit split =
+        ssm::ssd_tc_split(a->batch, a->heads, a->seqlen, ssm::device_sm_count());
+    return from_cuda(ssm::launch_ssd_tc(p, status, split,
+                                        static_cast<char *>(a->workspace) + kSsdStatusBytes, s));
   }
   return from_cuda(ssm::launch_m2_recurrent(p, s));
 }

@@ -147,6 +147,28 @@ def test_workspace_queries_need_no_pointers(lib):
     assert lib.ssd_chunk_scan_workspace(ctypes.byref(s), ctypes.byref(n)) == OK
 
 
+@pytest.mark.parametrize("batch,heads,seqlen,segs", [
+    (4, 80, 4096, (24, 6)),   # 320 units: a 24-unit last wave cut six ways
+    (1, 4, 4096, (4, 8)),     # below one wave: 37 ways, capped at 32 tiles / 4
+    (1, 150, 1536, (2, 3)),   # 148 whole units, a 2-unit tail cut three ways
+    (2, 74, 4096, None),      # 148 units: whole waves, no cut
+    (1, 60, 4096, None),      # 148 // 60 = 2 segments: not worth a cut
+    (1, 4, 1300, None),       # 11 tiles: fewer than three 4-tile segments
+    (1, 8, 128, None),        # one tile
+])
+def test_ssd_workspace_follows_the_wave_cut(lib, batch, heads, seqlen, segs):
+    """With no device the SSD sizes its workspace for 148 SMs: the status word,
+    then per tail segment an end state, a carried state and a decay (float32).
+    A partial last wave of `tail` units is cut into min(148 // tail, tiles // 4)
+    segments when that is three or more."""
+    n = ctypes.c_size_t(0)
+    s = _ssd(batch=batch, heads=heads, seqlen=seqlen, x=None, dt=None, B=None, C=None, A=None,
+             y=None)
+    assert lib.ssd_chunk_scan_workspace(ctypes.byref(s), ctypes.byref(n)) == OK
+    extra = 0 if segs is None else segs[0] * segs[1] * (2 * 128 * 64 + 4) * 4
+    assert n.value == 256 + extra
+
+
 def _conv(**kw):
     d = dict(batch=2, seqlen=8, channels=64, width=4, io=1, flags=1, x=P, w=P + 0x10000,
              bias=None, state_in=None, u=P + 0x20000, state_out=None)

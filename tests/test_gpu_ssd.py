@@ -97,7 +97,7 @@ def test_2p7b_full_size_sampled(cuda_ok):
     w = I.WORKLOADS["ssd_2p7b_b4_l4096_h80_p64_n128_bf16"]
     d = I.workload_inputs(w)
     y, h, _ = _run(d, chunk=w.chunk)
-    rows, hs = [0, 3], [0, 40, 79]
+    rows, hs = [0, 3], [0, 40, 60, 79]  # (3, 60) and (3, 79) are in the cut last wave
     sub = dict(d)
     sub["x"] = d["x"][rows][:, :, hs]
     sub["dt"] = d["dt"][rows][:, :, hs]
@@ -108,6 +108,37 @@ def test_2p7b_full_size_sampled(cuda_ok):
     hsel = torch.tensor(hs).cuda()
     assert_close_normwise(y[rows][:, :, hsel], ref[0], REL[torch.bfloat16], "y")
     assert_close_normwise(h[rows][:, hsel], ref[1], REL[torch.bfloat16], "h_last")
+
+
+@pytest.mark.parametrize("b,H,L,h0,gate", [
+    (1, 4, 4096, True, True),      # every unit cut into 8 segments
+    (2, 3, 1700, False, False),    # ragged last tile, zero start state, 3 segments
+    (1, 150, 1536, True, False),   # 148 whole units and a 2-unit tail in 3 segments
+])
+def test_ssd_sequence_segments(cuda_ok, b, H, L, h0, gate):
+    """Units of a partial last wave run as sequence segments, the state
+    carried from segment to segment (shapes chosen so that 148 SMs cut them)."""
+    d = I.ssd_inputs(b, L, H, 64, 128, io="bf16", gate=gate, seed=L + H, h0=h0)
+    got, ref = _run(d), _oracle(d)
+    assert_close_normwise(got[0], ref[0], REL[torch.bfloat16], "y")
+    assert_close_normwise(got[1], ref[1], REL[torch.bfloat16], "h_last")
+
+
+def test_ssd_segments_match_whole_units(cuda_ok):
+    """The same heads computed in a cut last wave and in whole waves agree
+    to rounding (h_last, y)."""
+    d = I.ssd_inputs(1, 2048, 150, 64, 128, io="bf16", seed=21, h0=True)
+    full = _run(d)                                   # heads 148, 149 cut
+    sub = dict(d)
+    for k in ("x", "dt"):
+        sub[k] = d[k][:, :, 2:].contiguous()
+    for k in ("A", "D", "dt_bias"):
+        sub[k] = d[k][2:].contiguous()
+    sub["h0"] = d["h0"][:, 2:].contiguous()
+    part = _run(sub)                                 # 148 heads: whole units
+    assert_close_normwise(full[1][:, -2:], part[1][:, -2:].cpu(), REL[torch.bfloat16], "h_last")
+    assert_close_normwise(full[0][:, :, -2:], part[0][:, :, -2:].float().cpu(),
+                          REL[torch.bfloat16], "y")
 
 
 def test_ssd_status_word_clear(cuda_ok):
