@@ -44,6 +44,13 @@
 // slack, and the contractions of the next tile run under this tile's
 // elementwise work.
 //
+// A CTA runs either a whole (batch, head) unit or a segment of its tiles:
+// when the last wave of units is partial, the host cuts those units into
+// sequence segments (first every segment from its own start, then
+// ssd_seg_carry_kernel chains the end states -- the state is linear in the
+// start state, with one scalar decay per tile -- then the segments again
+// from the carried states beside the whole units).
+//
 // Every wait is bounded and every warp votes on its waits, so its lanes
 // always take the same branch; warps of a group never wait for each other,
 // they arrive once per warp on four-count barriers.  A wait that runs out sets the
@@ -686,23 +693,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 // The state entering each segment of a tail unit: segment 0 started from the
 // unit's own start state, so its end state is exact; the state is linear in
 // the start state, so segment s's exact end is its end from zeros plus its
-// decay product times the state that entered it.  Block = tail unit.
-__global__ void __launch_bounds__(256)
+// decay product times the state that entered it.  Block = (tail unit, 1024
+// of its N x P values); a thread carries four of them through the segments.
+constexpr int kCarrySlice = 1024;
+__global__ void __launch_bounds__(kCarrySlice / 4)
     ssd_seg_carry_kernel(const float *hend, const float *decay, float *hin, int nseg) {
   constexpr int kNP = kN * kP;
   const int64_t tu = blockIdx.x;
-  const float *he = hend + tu * nseg * kNP;
+  const int e = blockIdx.y * kCarrySlice + threadIdx.x * 4;
+  const float *he = hend + tu * nseg * kNP + e;
   const float *dc = decay + tu * nseg;
-  float *hi = hin + tu * nseg * kNP;
-  for (int e = threadIdx.x * 4; e < kNP; e += 256 * 4) {
-    float4 h = *reinterpret_cast<const float4 *>(he + e);
-    for (int sg = 1; sg < nseg; ++sg) {
-      *reinterpret_cast<float4 *>(hi + (int64_t)sg * kNP + e) = h;
-      if (sg + 1 < nseg) {
-        const float4 l = *reinterpret_cast<const float4 *>(he + (int64_t)sg * kNP + e);
-        const float d = dc[sg];
-        h = make_float4(fmaf(d, h.x, l.x), fmaf(d, h.y, l.y), fmaf(d, h.z, l.z), fmaf(d, h.w, l.w));
-      }
+  float *hi = hin + tu * nseg * kNP + e;
+  float4 h = *reinterpret_cast<const float4 *>(he);
+#pragma unroll 4
+  for (int sg = 1; sg < nseg; ++sg) {
+    *reinterpret_cast<float4 *>(hi + (int64_t)sg * kNP) = h;
+    if (sg + 1 < nseg) {
+      const float4 l = *reinterpret_cast<const float4 *>(he + (int64_t)sg * kNP);
+      const float d = dc[sg];
+      h = make_float4(fmaf(d, h.x, l.x), fmaf(d, h.y, l.y), fmaf(d, h.z, l.z), fmaf(d, h.w, l.w));
     }
   }
 }
@@ -816,7 +825,8 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
   ssd_tc_kernel<<<(unsigned)slots, kThreads, smem, stream>>>(mX, mB, mC, q);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  ssd_seg_carry_kernel<<<(unsigned)split.ntail, 256, 0, stream>>>(hend, dec, hin, split.nseg);
+  ssd_seg_carry_kernel<<<dim3((unsigned)split.ntail, kN * kP / kCarrySlice), kCarrySlice / 4, 0,
+                         stream>>>(hend, dec, hin, split.nseg);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   q.nfull = units - split.ntail;
