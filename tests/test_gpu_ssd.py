@@ -124,6 +124,22 @@ def test_ssd_sequence_segments(cuda_ok, b, H, L, h0, gate):
     assert_close_normwise(got[1], ref[1], REL[torch.bfloat16], "h_last")
 
 
+def test_ssd_segments_in_place_state_and_groups(cuda_ok):
+    """A cut call with h_last aliasing h0 (the ABI allows it: the first pass
+    reads the start states before any segment writes an end state) and two
+    B/C groups."""
+    d = I.ssd_inputs(1, 2048, 8, 64, 128, groups=2, io="bf16", gate=True, seed=33, h0=True)
+    ref = _oracle(d)
+    dv = {k: (v.cuda() if v is not None else None) for k, v in d.items()}
+    state = dv["h0"].clone()
+    y, h, _ = _ops().ssd_chunk_scan_fwd(dv["x"], dv["dt"], dv["A"], dv["B"], dv["C"], D=dv["D"],
+                                        z=dv["z"], dt_bias=dv["dt_bias"], h0=state, h_last=state)
+    torch.cuda.synchronize()
+    assert h.data_ptr() == state.data_ptr()
+    assert_close_normwise(y, ref[0], REL[torch.bfloat16], "y")
+    assert_close_normwise(state, ref[1], REL[torch.bfloat16], "h_last")
+
+
 def test_ssd_segments_match_whole_units(cuda_ok):
     """The same heads computed in a cut last wave and in whole waves agree
     to rounding (h_last, y)."""
