@@ -181,26 +181,52 @@ __global__ void __launch_bounds__(256) attn_mask_kernel(AttnParams p) {
     return;
   }
   // every head's factors first (threads 0..127: one key each; 128..255: one
-  // query each), read straight from the running sums; one barrier
-  for (int hh = 0; hh < nh; ++hh) {
-    const int64_t base = (b * H + h0 + hh) * L;
-    if (tid < kTile) {
-      const int64_t tk = s0 + tid;
-      const int rk = (tid | 31) < (int)(L - s0) ? (tid | 31) : (int)(L - s0 - 1);
-      const double ckt = tk < L ? p.cum[base + tk] : 0.0;
-      const float bt = tk < L ? p.beta[base + tk] : 0.f;
-      colf[hh][tid] = ex2((float)(p.cum[base + s0 + rk] - ckt)) * bt;
-      ck[hh][tid] = ckt;
-      betas[hh][tid] = bt;
-    } else {
-      const int q = tid - kTile;
-      const int64_t tq = t0 + q;
-      const double cqt = tq < L ? p.cum[base + tq] : 0.0;
-      cq[hh][q] = cqt;
+  // query each), read straight from the running sums -- all of a thread's
+  // loads issued before any is used; one barrier
+  if (tid < kTile) {
+    const int64_t tk = s0 + tid;
+    const int rk = (tid | 31) < (int)(L - s0) ? (tid | 31) : (int)(L - s0 - 1);
+    double ckt[kHeadsPerCta], crk[kHeadsPerCta];
+    float bt[kHeadsPerCta];
 #pragma unroll
-      for (int J = 0; J < 4; ++J) {
-        const int rk = (32 * J + 31) < (int)(L - s0) ? 32 * J + 31 : (int)(L - s0 - 1);
-        rowf[hh][q][J] = ex2((float)(cqt - p.cum[base + s0 + rk]));
+    for (int hh = 0; hh < kHeadsPerCta; ++hh) {
+      if (hh < nh) {
+        const int64_t base = (b * H + h0 + hh) * L;
+        ckt[hh] = tk < L ? p.cum[base + tk] : 0.0;
+        bt[hh] = tk < L ? p.beta[base + tk] : 0.f;
+        crk[hh] = p.cum[base + s0 + rk];
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < kHeadsPerCta; ++hh) {
+      if (hh < nh) {
+        colf[hh][tid] = ex2((float)(crk[hh] - ckt[hh])) * bt[hh];
+        ck[hh][tid] = ckt[hh];
+        betas[hh][tid] = bt[hh];
+      }
+    }
+  } else {
+    const int q = tid - kTile;
+    const int64_t tq = t0 + q;
+    double cqt[kHeadsPerCta], crk[kHeadsPerCta][4];
+#pragma unroll
+    for (int hh = 0; hh < kHeadsPerCta; ++hh) {
+      if (hh < nh) {
+        const int64_t base = (b * H + h0 + hh) * L;
+        cqt[hh] = tq < L ? p.cum[base + tq] : 0.0;
+#pragma unroll
+        for (int J = 0; J < 4; ++J) {
+          const int rk = (32 * J + 31) < (int)(L - s0) ? 32 * J + 31 : (int)(L - s0 - 1);
+          crk[hh][J] = p.cum[base + s0 + rk];
+        }
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < kHeadsPerCta; ++hh) {
+      if (hh < nh) {
+        cq[hh][q] = cqt[hh];
+#pragma unroll
+        for (int J = 0; J < 4; ++J) rowf[hh][q][J] = ex2((float)(cqt[hh] - crk[hh][J]));
       }
     }
   }
