@@ -10,7 +10,8 @@
 //
 // Writing b * H * L^2 float32 values dominates; C . B^T does not depend on the
 // head, so one pass computes each 128 x 128 tile of it on or below the
-// diagonal once per (batch, group) into the workspace (where it stays in L2),
+// diagonal once per (batch, group) into the workspace (where it stays in L2;
+// on the tensor cores for bf16 inputs with state 128, else on the CUDA cores),
 // and the mask pass -- one CTA per (query tile, key tile, four heads of the
 // group) -- reads its share of the tile once and applies each head's decay
 // mask to it.  The decay between s and t is taken as the
@@ -21,13 +22,17 @@
 // a decaying state; on the diagonal blocks it is taken element by element.
 #include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
+#include "tma.h"
+
+#include <type_traits>
 
 namespace ssm {
 namespace {
 
+using namespace sm100;
+
 constexpr int kTile = 128;   // query and key tokens per tile
-constexpr int kK = 32;       // state columns per shared-memory chunk of C and B
-constexpr int kPitch = 132;  // floats per row of the k-major chunks (16-byte rows)
 constexpr int kHeadsPerCta = 4;
 
 // Pre-pass: per (batch, head) the step betas_t and the running sum of the
@@ -133,6 +138,99 @@ __global__ void __launch_bounds__(256) attn_cb_kernel(AttnParams p) {
   float *tile = p.cb + ((b * p.G + g) * p.ntri + li) * (int64_t)(kTile * kTile);
   *reinterpret_cast<float4 *>(tile + (br * kBlk + ty) * kTile + bc * kBlk + 4 * tx) =
       make_float4(acc[0], acc[1], acc[2], acc[3]);
+}
+
+// The same tile on the tensor cores (bf16 inputs, state 128): one CTA of 128
+// threads per (lower tile, group, batch).  The TMA brings the tile's 128 query
+// rows of C and 128 key rows of B as two 64-state slabs each (128-byte
+// swizzle; rows past the sequence end arrive as zeros); one thread issues the
+// eight K = 16 steps of the 128 x 128 x 128 product into 128 TMEM columns
+// (row t in lane t, key s in column s); each warp then reads its quarter of
+// the lanes and writes those rows to the workspace.  Both waits are bounded;
+// a wait that runs out leaves NaN rows in the tile, so the failure shows in
+// alpha, and the CTA still frees its TMEM.
+struct __align__(1024) CbSmem {
+  uint8_t C[2][kTile * 128];  // [slab]: 128 rows x 64 bf16
+  uint8_t B[2][kTile * 128];
+  uint64_t full, done;
+  uint32_t taddr;
+};
+constexpr long long kCbWaitLimit = 2000000000ll;  // cycles (about a second)
+
+__global__ void __launch_bounds__(128)
+    attn_cb_tc_kernel(const __grid_constant__ CUtensorMap mB,
+                      const __grid_constant__ CUtensorMap mC, AttnParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  CbSmem &s = *reinterpret_cast<CbSmem *>(smem_raw +
+                                          ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t li = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  int64_t qt = (int64_t)((sqrt(8.0 * (double)li + 1.0) - 1.0) / 2.0);
+  while (qt * (qt + 1) / 2 > li) --qt;
+  while ((qt + 1) * (qt + 2) / 2 <= li) ++qt;
+  const int64_t kt = li - qt * (qt + 1) / 2;
+
+  if (tid == 0) {
+    mbar_init(&s.full, 1);
+    mbar_init(&s.done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&s.taddr, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = s.taddr;
+
+  if (tid == 0) {
+    const int gx = (int)(g * 128);
+    mbar_expect_tx(&s.full, 4 * kTile * 128);
+    tma_load_3d(s.C[0], &mC, &s.full, gx, (int)(qt * kTile), (int)b);
+    tma_load_3d(s.C[1], &mC, &s.full, gx + 64, (int)(qt * kTile), (int)b);
+    tma_load_3d(s.B[0], &mB, &s.full, gx, (int)(kt * kTile), (int)b);
+    tma_load_3d(s.B[1], &mB, &s.full, gx + 64, (int)(kt * kTile), (int)b);
+    if (mbar_wait(&s.full, 0, kCbWaitLimit)) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16_f32(128, 128, false, false);
+      const uint64_t dC = smem_desc(smem_u32(s.C[0]), 16, 1024, kSwizzle128B);
+      const uint64_t dB = smem_desc(smem_u32(s.B[0]), 16, 1024, kSwizzle128B);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        // K step kk: slab kk / 4, 32 bytes per step inside the slab
+        const uint32_t ko = ((kk >> 2) * (kTile * 128) + (kk & 3) * 32) >> 4;
+        mma_ss(tb, dC + ko, dB + ko, id, kk > 0);
+      }
+      mma_commit(&s.done);
+    }
+  }
+  const bool got = mbar_wait(&s.done, 0, kCbWaitLimit);
+  const bool all = __all_sync(0xffffffffu, got);
+  tc_fence_after();
+  float *row = p.cb + ((b * p.G + g) * p.ntri + li) * (int64_t)(kTile * kTile) +
+               (int64_t)(32 * warp + lane) * kTile;
+  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+#pragma unroll 1
+  for (int c = 0; c < kTile; c += 16) {
+    uint32_t r[16];
+    if (all) {
+      tmem_ld16(tb + lane_base + (uint32_t)c, r);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) r[j] = 0x7fc00000u;  // NaN
+    }
+#pragma unroll
+    for (int j = 0; j < 16; j += 4)
+      *reinterpret_cast<float4 *>(row + c + j) =
+          make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                      __uint_as_float(r[j + 3]));
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tb, 128);
 }
 
 // The mask pass: one CTA per (query tile, key tile, run of heads of one
@@ -298,7 +396,28 @@ cudaError_t launch_t(const AttnParams &p, cudaStream_t s) {
   attn_prep_kernel<T><<<(unsigned)units, kPrep, 0, s>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_cb_kernel<T><<<dim3((unsigned)(16 * p.ntri), (unsigned)p.G, (unsigned)p.batch), 256, 0, s>>>(p);
+  if (std::is_same<T, __nv_bfloat16>::value && p.N == 128) {
+    // tensor-core C . B^T: B and C as [batch, L, G * 128] bf16, 64 x 128 boxes
+    const uint64_t GN = (uint64_t)(p.G * 128);
+    uint64_t dims[3] = {GN, (uint64_t)p.L, (uint64_t)p.batch};
+    uint64_t strides[2] = {GN * 2, (uint64_t)p.L * GN * 2};
+    uint32_t box[3] = {64, (uint32_t)kTile, 1};
+    CUtensorMap mB, mC;
+    if (!encode_tiled(&mB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.B, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tiled(&mC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.Cm, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    const size_t smem = sizeof(CbSmem) + 1024;
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        attn_cb_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (attr != cudaSuccess) return attr;
+    attn_cb_tc_kernel<<<dim3((unsigned)p.ntri, (unsigned)p.G, (unsigned)p.batch), 128, smem, s>>>(
+        mB, mC, p);
+  } else {
+    attn_cb_kernel<T><<<dim3((unsigned)(16 * p.ntri), (unsigned)p.G, (unsigned)p.batch), 256, 0,
+                        s>>>(p);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t ntile = (p.L + kTile - 1) / kTile;

@@ -44,6 +44,17 @@ def test_attention_groups_and_states(cuda_ok, N, G, H):
     assert_close_normwise(al, ref, REL[torch.float32], "alpha")
 
 
+@pytest.mark.parametrize("L,G", [(1, 1), (129, 1), (300, 2)])
+def test_attention_tensor_core_tiles(cuda_ok, L, G):
+    # bf16 inputs with state 128 take the tensor-core C . B^T: one tile, a
+    # ragged second tile (rows past the end arrive as zeros), two groups
+    d = I.ssd_inputs(1, L, 4, 16, 128, groups=G, io="bf16", seed=L + G)
+    al = _run(d)
+    ref = oracle.m2_attention(d["dt"], d["B"], d["C"], d["A"], d["dt_bias"])
+    assert_close_normwise(al, ref, REL[torch.float32], "alpha")
+    assert torch.count_nonzero(torch.triu(al, 1)) == 0
+
+
 def test_attention_without_softplus(cuda_ok):
     d = I.ssd_inputs(1, 90, 2, 16, 32, io="f32", seed=3)
     d["dt"] = d["dt"].abs() * 0.1   # a positive step without softplus, and no bias
