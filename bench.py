@@ -665,7 +665,7 @@ def run_ours(args):
             "unit": "GB/s", "ms_per_step": round(at["ms_per_step"], 4),
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(ach / hbm, 4), "traffic": traffic_for("attn_2p7b"),
-                         "kernel": "attn_mask_kernel (+ attn_prep_kernel, attn_cb_kernel)"}}
+                         "kernel": "attn_mask_kernel (+ attn_prep_kernel, attn_cb_tc_kernel)"}}
         out["workloads"] = wl
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline_m1(w)
