@@ -194,7 +194,14 @@ typedef struct ssd_scan_args {
 } ssd_scan_args_t;
 
 /* Bytes of device workspace ssd_chunk_scan_fwd needs (sizes, dtype and flags
- * are validated; the tensor pointers are not looked at). */
+ * are validated; the tensor pointers are not looked at).  On the tensor-core
+ * path (bf16, state 128, head_dim 64, no per-token states) it holds a status
+ * word and, when batch x heads leaves the last wave of the current device's
+ * SMs partial, the float32 end states, carried states and decay products of
+ * the sequence segments that wave is cut into; the size therefore depends on
+ * the device current at the query (148 SMs are assumed when none can be
+ * read), and a call with less workspace than its own device needs returns
+ * SSM_ERR_WORKSPACE. */
 ssm_status_t ssd_chunk_scan_workspace(const ssd_scan_args_t *args, size_t *bytes);
 ssm_status_t ssd_chunk_scan_fwd(const ssd_scan_args_t *args, void *stream);
 
