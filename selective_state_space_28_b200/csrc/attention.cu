@@ -409,7 +409,8 @@ cudaError_t launch_t(const AttnParams &p, cudaStream_t s) {
                       CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
     const size_t smem = sizeof(CbSmem) + 1024;
-    static const cudaError_t attr = cudaFuncSetAttribute(
+    // (set on every call: the attribute belongs to the current device)
+    const cudaError_t attr = cudaFuncSetAttribute(
         attn_cb_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (attr != cudaSuccess) return attr;
     attn_cb_tc_kernel<<<dim3((unsigned)p.ntri, (unsigned)p.G, (unsigned)p.batch), 128, smem, s>>>(

@@ -234,10 +234,10 @@ cudaError_t launch_w(const ConvParams &p, cudaStream_t s) {
   dim3 grid((unsigned)((units + 127) / 128), (unsigned)runs);
   if (vec) {
     // the slots (24-32 KB per CTA) need the shared-memory carve-out for
-    // several CTAs per SM
-    static const cudaError_t carve = cudaFuncSetAttribute(
-        conv1d_vec_kernel<T, W>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    (void)carve;
+    // several CTAs per SM (a preference of the current device: set per call)
+    if (cudaFuncSetAttribute(conv1d_vec_kernel<T, W>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+      cudaGetLastError();  // a preference only: never fail the call on it
     conv1d_vec_kernel<T, W><<<grid, 128, 0, s>>>(p);
   }
   else

@@ -797,12 +797,11 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
   q.seg_decay = nullptr;
   q.seg_hin = nullptr;
   const size_t smem = ssd_tc_smem_bytes();
-  static bool attr_set = false;
-  if (!attr_set) {
+  // (set on every call: the attribute belongs to the current device)
+  {
     cudaError_t e = cudaFuncSetAttribute(ssd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   if (split.nseg <= 1) {
     ssd_tc_kernel<<<(unsigned)q.nfull, kThreads, smem, stream>>>(mX, mB, mC, q);
