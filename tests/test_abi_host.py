@@ -248,3 +248,22 @@ def test_attention_workspace_size(lib):
     # steps and float64 running sums per (batch, head, token), then one
     # 128 x 128 float32 C . B^T tile per (batch, group) for the single tile
     assert n.value == 2 * 8 * 100 * 12 + 2 * 1 * 128 * 128 * 4
+
+
+def test_empty_calls_launch_nothing(lib):
+    """An empty batch (or, where the state needs no pass-through, an empty
+    sequence) returns OK before any device call: these run without a GPU."""
+    a = _ssd(batch=0, io=0, x=None, dt=None, B=None, C=None, A=None, y=None)
+    assert lib.ssd_chunk_scan_fwd(ctypes.byref(a), None) == OK
+    # the tensor-core shapes still want their (status-word) workspace
+    a = _ssd(batch=0, x=None, dt=None, B=None, C=None, A=None, y=None)
+    assert lib.ssd_chunk_scan_fwd(ctypes.byref(a), None) == WS
+    a = _ssd(batch=0, x=None, dt=None, B=None, C=None, A=None, y=None, workspace=P,
+             workspace_bytes=256)
+    assert lib.ssd_chunk_scan_fwd(ctypes.byref(a), None) == OK
+    s = _scan(batch=0, x=None, dt=None, B=None, C=None, A=None, y=None)
+    assert lib.ssm_scan_fwd_write(ctypes.byref(s), 0, ctypes.c_void_p(P), None) == OK
+    for kw in (dict(batch=0), dict(seqlen=0)):
+        t = _attn(dt=None, B=None, C=None, A=None, alpha=None, workspace=None,
+                  workspace_bytes=0, **kw)
+        assert lib.ssd_attention_fwd(ctypes.byref(t), None) == OK
