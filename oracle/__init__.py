@@ -269,3 +269,79 @@ def rms_rows(v, eps):
     n = v.shape[-1]
     _load().orc_rms_rows(v.size // n, n, eps, _p(v), _p(out))
     return out
+
+
+# ------------------------------------------------------------------ the block
+# "Falcon-Mamba" and "Mamba-2" (nnterp encyclopedia), "The block, in order":
+# out = x + mixer(norm(x)), the add in float32 (residual_in_fp32); the mixer's
+# output (attention_output) is in the load dtype and is all the block adds
+# ("The contribution is the whole block").  The blocks below are wrappers for
+# the oracle's residual-identity checks: seeded random weights, the oracle's
+# own scan as the mixer's core, library matmuls for the projections.
+
+def _round_to(a, load_dtype):
+    """Round float64 values to the load dtype, returned as float32."""
+    if load_dtype == "float32":
+        return np.asarray(a, dtype=np.float32)
+    if load_dtype == "bfloat16":
+        import torch
+        return torch.tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16).float().numpy()
+    raise ValueError("load dtype %r" % load_dtype)
+
+
+def _rmsnorm_gain(h, w, eps):
+    return h / np.sqrt(np.mean(h * h, axis=-1, keepdims=True) + eps) * w
+
+
+def falcon_mamba_block(h, W, *, rms_eps=1e-6, norm_eps=1e-5, load_dtype="float32"):
+    """One Falcon-Mamba block ("Falcon-Mamba", "The block, in order" and
+    "Where the norms sit"): norm, in_proj to (u, z), silu(conv1d(u)), x_proj to
+    the low-rank step and B, C, the three weightless RMS norms, dt_proj, the
+    scan with D*u and the silu(z) gate, out_proj; then the residual add.
+
+    h: [b, L, d_model]; W: dict of weights (norm, in_proj, conv_w, conv_b,
+    x_proj, dt_proj_w, dt_proj_b, A, D, out_proj).  Returns (layer_output
+    float32, attention_output in the load dtype, widened to float32)."""
+    h64 = _f64(h)
+    R, N = W["dt_proj_w"].shape[1], W["A"].shape[1]
+    hn = _rmsnorm_gain(h64, W["norm"], norm_eps)
+    uz = hn @ W["in_proj"].T
+    di = uz.shape[-1] // 2
+    u, z = uz[..., :di], uz[..., di:]
+    u, _ = conv1d(u, W["conv_w"], W["conv_b"], act=True)
+    dbc = u @ W["x_proj"].T
+    low = rms_rows(dbc[..., :R], rms_eps)
+    Bn = rms_rows(dbc[..., R:R + N], rms_eps)
+    Cn = rms_rows(dbc[..., R + N:], rms_eps)
+    dt = low @ W["dt_proj_w"].T
+    y, _, _ = m1_scan(u, dt, Bn[:, :, None, :], Cn[:, :, None, :], W["A"], W["D"], z=z,
+                      dt_bias=W["dt_proj_b"])
+    attn = _round_to(y @ W["out_proj"].T, load_dtype)
+    out = np.asarray(h, dtype=np.float32) + attn       # the add, in float32
+    return out, attn
+
+
+def mamba2_block(h, W, *, heads, groups=1, norm_eps=1e-5, load_dtype="float32"):
+    """One Mamba-2 block ("Mamba-2", "The block, in order"): norm, in_proj to
+    (z, xBC, dt), silu(conv1d(xBC)) split into x, B, C, the SSD with D*x, the
+    gated norm over the mixer's width, out_proj; then the residual add.
+
+    h: [b, L, d_model]; W: dict (norm, in_proj, conv_w, conv_b, A, D,
+    dt_bias, gnorm, out_proj).  Returns (layer_output float32,
+    attention_output in the load dtype, widened to float32)."""
+    h64 = _f64(h)
+    b, L, _ = h64.shape
+    di = W["out_proj"].shape[1]
+    N = (W["conv_w"].shape[0] - di) // (2 * groups)
+    hn = _rmsnorm_gain(h64, W["norm"], norm_eps)
+    proj = hn @ W["in_proj"].T
+    z, xbc, dt = proj[..., :di], proj[..., di:2 * di + 2 * groups * N], proj[..., -heads:]
+    xbc, _ = conv1d(xbc, W["conv_w"], W["conv_b"], act=True)
+    x = xbc[..., :di].reshape(b, L, heads, di // heads)
+    Bm = xbc[..., di:di + groups * N].reshape(b, L, groups, N)
+    Cm = xbc[..., di + groups * N:].reshape(b, L, groups, N)
+    y, _, _ = m2_scan(x, dt, Bm, Cm, W["A"], W["D"], dt_bias=W["dt_bias"])
+    g = gated_rmsnorm(y.reshape(b, L, di), z, W["gnorm"], eps=norm_eps)
+    attn = _round_to(g @ W["out_proj"].T, load_dtype)
+    out = np.asarray(h, dtype=np.float32) + attn       # the add, in float32
+    return out, attn

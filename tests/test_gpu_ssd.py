@@ -1,5 +1,6 @@
 """GPU parity of the Mamba-2 SSD scan (ssd_chunk_scan_fwd, through the C ABI)
 against the float64 oracle's token loop."""
+import numpy as np
 import pytest
 import torch
 
@@ -168,3 +169,96 @@ def test_ssd_status_word_clear(cuda_ok):
                            dt_bias=dv["dt_bias"], h0=dv["h0"], workspace=ws)
     torch.cuda.synchronize()
     assert ws[:4].view(torch.int32).item() == 0
+
+
+# ------------------------------------------------ the tensor-core path's edges
+# The shapes below (bf16 I/O, state 128, head_dim 64, no per-token states) run
+# the tcgen05 kernel; each test first checks, through the workspace size, that
+# the call takes that path.  Values from the "Mamba-2" page: a zero step skips
+# a token exactly ("A zero step skips a token exactly"), and the checkpoints'
+# A_h span -exp(A_log) from about -36316 to -4e-4 ("The mixer's values").
+
+def _assert_tensor_core_path(d):
+    import ctypes
+    from selective_state_space_28_b200 import _lib as L
+    b, Lq, H, P = d["x"].shape
+    G, N = d["B"].shape[2], d["B"].shape[3]
+    a = L.SsdArgs(batch=b, seqlen=Lq, heads=H, head_dim=P, state=N, groups=G, chunk=256,
+                  io=L.SSM_BF16, flags=L.SSM_DT_SOFTPLUS)
+    n = ctypes.c_size_t(0)
+    L.check(L.lib().ssd_chunk_scan_workspace(ctypes.byref(a), ctypes.byref(n)), "ws")
+    assert n.value > 0, "not the tensor-core path"
+
+
+def _check(d, what=""):
+    _assert_tensor_core_path(d)
+    got, ref = _run(d), _oracle(d)
+    assert_close_normwise(got[0], ref[0], REL[torch.bfloat16], what + " y")
+    assert_close_normwise(got[1], ref[1], REL[torch.bfloat16], what + " h_last")
+    return got, ref
+
+
+@pytest.mark.parametrize("gate", [False, True])
+def test_ssd_tc_zero_steps_at_tile_edges(cuda_ok, gate):
+    """dt_raw = -inf gives a zero step: the token adds nothing and decays
+    nothing.  Zero steps at the first token, on both sides of 128-token tile
+    and 256-token chunk boundaries, in runs, and at the last token."""
+    d = I.ssd_inputs(2, 600, 4, 64, 128, io="bf16", gate=gate, seed=41, h0=True)
+    for t in (0, 1, 127, 128, 129, 255, 256, 300, 301, 302, 383, 384, 599):
+        d["dt"][:, t] = -float("inf")
+    d["dt"][1, 400:520, 2] = -float("inf")  # a whole tile of one head skipped
+    _check(d, "zero steps")
+
+
+def test_ssd_tc_all_zero_steps_keep_the_state(cuda_ok):
+    """Every step zero: y = C_t . h0 + D x_t and h_last = h0 (to rounding of
+    the bf16 operands the tensor cores read)."""
+    d = I.ssd_inputs(1, 300, 3, 64, 128, io="bf16", seed=42, h0=True)
+    d["dt"][:] = -float("inf")
+    got, ref = _check(d, "all zero")
+    np.testing.assert_array_equal(ref[1], d["h0"].double().numpy())
+
+
+@pytest.mark.parametrize("L", [300, 1536])
+def test_ssd_tc_extreme_rates(cuda_ok, L):
+    """Per-head A_h at the pages' extremes (-36316 and -4e-4) beside ordinary
+    ones, and steps driven to +-25 on scattered tokens: a state wiped out in
+    one token, a state that barely decays over the whole prompt, and tokens
+    that add almost nothing."""
+    d = I.ssd_inputs(1, L, 6, 64, 128, io="bf16", gate=True, seed=43 + L, h0=True)
+    d["A"] = torch.tensor([-36316.0, -4e-4, -1.0, -16.0, -36316.0, -4e-4])
+    g = torch.Generator().manual_seed(L)
+    pick = torch.rand(d["dt"].shape, generator=g)
+    d["dt"][pick < 0.05] = 25.0
+    d["dt"][pick > 0.95] = -25.0
+    _check(d, "extreme rates")
+
+
+def test_ssd_tc_split_and_carry_through_h0(cuda_ok):
+    """A prompt cut at a token that is not a tile boundary and continued
+    from h_last through h0 agrees with the whole prompt and the oracle."""
+    d = I.ssd_inputs(2, 700, 4, 64, 128, io="bf16", gate=True, seed=44, h0=True)
+    _assert_tensor_core_path(d)
+    k = 333
+    cut = ("x", "dt", "z", "B", "C")
+    first = {n: (v[:, :k].contiguous() if v is not None and n in cut else v)
+             for n, v in d.items()}
+    rest = {n: (v[:, k:].contiguous() if v is not None and n in cut else v)
+            for n, v in d.items()}
+    a = _run(first)
+    b = _run(rest, h0=a[1])
+    ref = _oracle(d)
+    assert_close_normwise(torch.cat([a[0], b[0]], 1), ref[0], REL[torch.bfloat16], "y")
+    assert_close_normwise(b[1], ref[1], REL[torch.bfloat16], "h_last")
+
+
+def test_ssd_tc_cut_wave_with_extreme_values(cuda_ok):
+    """A shape whose last wave is cut into sequence segments (one batch row,
+    four heads, 4096 tokens), with zero steps on segment boundaries and the
+    extreme A_h: the carried state and the decay products stay exact enough."""
+    d = I.ssd_inputs(1, 4096, 4, 64, 128, io="bf16", gate=False, seed=45, h0=True)
+    d["A"] = torch.tensor([-36316.0, -4e-4, -2.0, -4e-4])
+    for t in range(0, 4096, 512):
+        d["dt"][:, t] = -float("inf")
+    d["dt"][0, 1000:1100, 1] = 25.0
+    _check(d, "cut wave")

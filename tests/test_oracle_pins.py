@@ -154,22 +154,29 @@ def test_m1_scan_equals_hidden_attention(G):
     np.testing.assert_allclose(y, y_q, rtol=1e-11, atol=1e-11)
 
 
-def test_hidden_attention_by_einsum():
-    """The masked form rebuilt with torch einsum on cumulative decays, as the
-    "Mamba-2" page's own check does, agrees with the brute-force sum."""
-    d = _m2_rand(1, 12, 3, 4, 6, G=1, seed=8, h0=False, z=False)
+def test_hidden_attention_by_running_products():
+    """The masked form rebuilt another way: per head, the transfer matrix
+    T[t, s] = prod_{s<r<=t} exp(betas_r A_h) built one row at a time from
+    the row above (T[t, :t] = a_t T[t-1, :t], T[t, t] = 1), then
+    y = ((C B^T) * T * betas) x + D x as numpy matrix products.  It agrees
+    with the brute-force sum, which sums exponents instead of multiplying
+    factors."""
+    H, Lq, P, N = 3, 12, 4, 6
+    d = _m2_rand(1, Lq, H, P, N, G=1, seed=8, h0=False, z=False)
     betas = oracle.softplus(d["dt"] + d["dt_bias"])[0]            # [L, H]
-    decays = betas * d["A"]
-    cum = torch.tensor(decays).cumsum(0)
-    causal = torch.ones(12, 12, dtype=torch.bool).tril()[..., None]
-    kept = (cum[:, None] - cum[None, :]).masked_fill(~causal, -torch.inf).exp()
-    Cm = torch.tensor(d["C"][0]).repeat_interleave(3, 1)
-    Bm = torch.tensor(d["B"][0]).repeat_interleave(3, 1)
-    alpha = torch.einsum("thn,shn->tsh", Cm, Bm) * kept * torch.tensor(betas)
-    y_e = torch.einsum("tsh,shd->thd", alpha, torch.tensor(d["x"][0])) \
-        + torch.tensor(d["D"])[:, None] * torch.tensor(d["x"][0])
+    y_t = np.zeros((Lq, H, P))
+    for h in range(H):
+        a = np.exp(betas[:, h] * d["A"][h])
+        T = np.zeros((Lq, Lq))
+        for t in range(Lq):
+            if t:
+                T[t, :t] = a[t] * T[t - 1, :t]
+            T[t, t] = 1.0
+        cb = d["C"][0, :, 0, :] @ d["B"][0, :, 0, :].T               # [t, s]
+        M = cb * T * betas[None, :, h]
+        y_t[:, h, :] = M @ d["x"][0, :, h, :] + d["D"][h] * d["x"][0, :, h, :]
     y_q = oracle.m2_quadratic(d["x"], betas[None], d["B"], d["C"], d["A"], d["D"])
-    np.testing.assert_allclose(y_q[0], y_e.numpy(), rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(y_q[0], y_t, rtol=1e-11, atol=1e-11)
 
 
 # ------------------------------------------------------------------ invariants
@@ -553,20 +560,20 @@ def test_attention_rebuilds_the_scan(G=1):
     np.testing.assert_allclose(y_att, y, rtol=1e-10, atol=1e-12)
 
 
-def test_attention_matches_the_pages_recipe():
-    # the page's own rebuild: cum = decays.cumsum(0), kept = exp(cum_t - cum_s)
-    # below the diagonal, alpha = einsum(C, B) * kept * betas
-    d = _m2_rand(1, 17, 3, 2, 4, G=1, seed=71, h0=False, z=False)
+def test_attention_columns_are_impulse_responses():
+    """Column s of a head's attention matrix is that head's response to a
+    unit input at token s: the oracle scan with one value channel, x = 1 at
+    token s and 0 elsewhere, zero start state and no skip term, returns
+    y_t = alpha[t, s] for every t."""
+    b, Lq, H, N, G = 1, 11, 4, 5, 2
+    d = _m2_rand(b, Lq, H, 1, N, G=G, seed=71, h0=False, z=False)
     al = oracle.m2_attention(d["dt"], d["B"], d["C"], d["A"], d["dt_bias"])
-    beta = F.softplus(torch.tensor(d["dt"][0] + d["dt_bias"]))          # [seq, heads]
-    decay = beta * torch.tensor(d["A"])
-    cum = decay.cumsum(0)
-    causal = torch.ones(17, 17, dtype=torch.bool).tril()[..., None]
-    kept = (cum[:, None] - cum[None, :]).masked_fill(~causal, -torch.inf).exp()
-    Cg = torch.tensor(d["C"][0]).repeat_interleave(3, 1)
-    Bg = torch.tensor(d["B"][0]).repeat_interleave(3, 1)
-    ref = torch.einsum("thn,shn->tsh", Cg, Bg) * kept * beta           # [t, s, h]
-    np.testing.assert_allclose(al[0], ref.permute(2, 0, 1).numpy(), rtol=1e-10, atol=1e-13)
+    for s in range(Lq):
+        x = np.zeros((b, Lq, H, 1))
+        x[:, s] = 1.0
+        y, _, _ = oracle.m2_scan(x, d["dt"], d["B"], d["C"], d["A"], np.zeros(H),
+                                 dt_bias=d["dt_bias"])
+        np.testing.assert_allclose(al[0, :, :, s], y[0, :, :, 0].T, rtol=1e-12, atol=1e-15)
 
 
 def test_attention_is_causal_with_a_plain_diagonal():
@@ -588,3 +595,77 @@ def test_attention_without_decay_is_masked_cb():
     cb = d["C"][0, :, 0] @ d["B"][0, :, 0].T
     for h in range(2):
         np.testing.assert_allclose(al[0, h], np.tril(cb * beta[None, :, h]), rtol=1e-14)
+
+
+# ------------------------------------------------------------------ the block
+# "Falcon-Mamba" / "Mamba-2" (nnterp encyclopedia), "The block, in order" and
+# "The contribution is the whole block": out = x + mixer(norm(x)), the add in
+# float32, the mixer's output in the load dtype.
+
+def _falcon_weights(seed, dm=8, di=16, N=4, R=3):
+    r = rng(seed)
+    return dict(norm=1 + 0.1 * r.standard_normal(dm),
+                in_proj=r.standard_normal((2 * di, dm)) / 3,
+                conv_w=r.uniform(-0.5, 0.5, (di, 4)), conv_b=r.uniform(-0.5, 0.5, di),
+                x_proj=r.standard_normal((R + 2 * N, di)) / 4,
+                dt_proj_w=r.standard_normal((di, R)) / 2, dt_proj_b=r.uniform(-4, -1, di),
+                A=-np.exp(r.uniform(-1, 1.5, (di, N))), D=r.standard_normal(di),
+                out_proj=r.standard_normal((dm, di)) / 4)
+
+
+def _mamba2_weights(seed, dm=8, H=4, P=4, N=4, G=2):
+    r = rng(seed)
+    di = H * P
+    conv = di + 2 * G * N
+    return dict(norm=1 + 0.1 * r.standard_normal(dm),
+                in_proj=r.standard_normal((di + conv + H, dm)) / 3,
+                conv_w=r.uniform(-0.5, 0.5, (conv, 4)), conv_b=r.uniform(-0.5, 0.5, conv),
+                A=-np.exp(r.uniform(0, 2.7, H)), D=r.standard_normal(H),
+                dt_bias=r.uniform(-4, -1, H), gnorm=1 + 0.1 * r.standard_normal(di),
+                out_proj=r.standard_normal((dm, di)) / 4)
+
+
+def _block(kind, h, W, **kw):
+    if kind == "falcon":
+        return oracle.falcon_mamba_block(h, W, **kw)
+    return oracle.mamba2_block(h, W, heads=4, groups=2, **kw)
+
+
+@pytest.mark.parametrize("kind", ["falcon", "mamba2"])
+@pytest.mark.parametrize("load", ["float32", "bfloat16"])
+def test_block_output_is_input_plus_mixer_output_in_float32(kind, load):
+    """layer_input + attention_output == layer_output, bit for bit, with the
+    add done in float32 on the mixer output rounded to the load dtype."""
+    W = _falcon_weights(80) if kind == "falcon" else _mamba2_weights(81)
+    h = rng(82).standard_normal((2, 9, 8)) * 3
+    out, attn = _block(kind, h, W, load_dtype=load)
+    assert out.dtype == np.float32
+    direct = np.add(h.astype(np.float32), attn.astype(np.float32), dtype=np.float32)
+    np.testing.assert_array_equal(out, direct)
+    if load == "bfloat16":  # attention_output really is in the load dtype
+        bits = attn.astype(np.float32).view(np.uint32)
+        assert np.all(bits & 0xFFFF == 0)
+
+
+@pytest.mark.parametrize("kind", ["falcon", "mamba2"])
+def test_block_without_the_mixer_output_is_the_identity(kind):
+    """Ablating attention_output (out_proj = 0) ablates the block: the stream
+    passes through unchanged."""
+    W = _falcon_weights(83) if kind == "falcon" else _mamba2_weights(84)
+    W["out_proj"] = np.zeros_like(W["out_proj"])
+    h = rng(85).standard_normal((1, 7, 8))
+    out, attn = _block(kind, h, W)
+    assert not attn.any()
+    np.testing.assert_array_equal(out, h.astype(np.float32))
+
+
+@pytest.mark.parametrize("kind", ["falcon", "mamba2"])
+def test_block_contribution_reads_only_the_normed_input(kind):
+    """The mixer sees norm(x), so scaling the stream by c > 0 leaves the
+    mixer's output unchanged (the norm's eps taken to ~0) while the output
+    moves by exactly the residual: out(c x) - c x == out(x) - x."""
+    W = _falcon_weights(86) if kind == "falcon" else _mamba2_weights(87)
+    h = rng(88).standard_normal((1, 10, 8))
+    _, a1 = _block(kind, h, W, norm_eps=1e-300)
+    _, a3 = _block(kind, 3.0 * h, W, norm_eps=1e-300)
+    np.testing.assert_allclose(a3, a1, rtol=1e-6, atol=1e-7)
