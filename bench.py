@@ -317,6 +317,7 @@ def bench_m1(w, K, W, dist, device, pk, seed_base, write_at=None):
         d["h_last"] = torch.empty((w.batch, w.channels, w.state), device=device)
         if write_at is not None:
             d["s_write"] = torch.zeros((w.batch, w.channels, w.state), device=device)
+        d["ws"] = torch.zeros(m1_workspace_bytes(w), dtype=torch.uint8, device=device)
         sets.append(d)
 
     def step(i):
@@ -329,12 +330,42 @@ def bench_m1(w, K, W, dist, device, pk, seed_base, write_at=None):
             return
         ops.ssm_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
                          dt_bias=d["dt_bias"], flags=w.flags, rms_eps=w.rms_eps,
-                         y=d["y"], h_last=d["h_last"])
+                         y=d["y"], h_last=d["h_last"], workspace=d["ws"])
     ms = timed(step, K, W, dist, device) / K
     launch_ms = per_launch_ms(step, max(10, K), device)
-    launches = 2 if (w.flags & I.RMS_DT) else 1
+    ops._check_status(sets[0]["ws"], torch.cuda.current_stream(device).cuda_stream, "bench")
+    nseg = m1_segments(w) if write_at is None else 1
+    launches = (2 if (w.flags & I.RMS_DT) else 1) + (2 if nseg > 1 else 0)
     return {"ms_per_step": ms, "bytes": nb, "launch_ms": launch_ms, "sets": len(sets),
-            "launches_per_step": launches}
+            "launches_per_step": launches, "segments": nseg}
+
+
+def m1_workspace_bytes(w):
+    """ssm_scan_workspace for the workload, on the current device."""
+    import ctypes
+    from selective_state_space_28_b200 import _lib as L
+    a = L.ScanArgs(batch=w.batch, seqlen=w.seqlen, channels=w.channels, state=w.state,
+                   groups=w.groups, io=L.SSM_BF16 if w.io == "bf16" else L.SSM_F32,
+                   flags=w.flags, rms_eps=w.rms_eps)
+    n = ctypes.c_size_t(0)
+    L.check(L.lib().ssm_scan_workspace(ctypes.byref(a), ctypes.byref(n)), "ssm_scan_workspace")
+    return n.value
+
+
+def m1_segments(w):
+    """Sequence segments the scan cuts the workload into: read back from the
+    workspace size (status word, step-norm factors, then the segments'
+    (S - 1) end states, (S - 1) step sums and S entering states)."""
+    r256 = lambda v: (v + 255) // 256 * 256
+    base = 256 + (r256(w.batch * w.seqlen * 4) if w.flags & 4 else 0)
+    extra = m1_workspace_bytes(w) - base
+    if extra <= 0:
+        return 1
+    bcn, bc = w.batch * w.channels * w.state * 4, w.batch * w.channels * 4
+    for S in range(2, 65):
+        if r256(bcn * (S - 1)) + r256(bc * (S - 1)) + r256(bcn * S) == extra:
+            return S
+    return -1
 
 
 def bench_conv(w, K, W, dist, device, pk, seed_base):
@@ -554,7 +585,6 @@ def run_ours(args):
     time.sleep(0.2)
 
     w = I.WORKLOADS[HEADLINE]
-    generic = os.environ.get("SSM_M1_PIPELINED", "1") == "0"
     r = bench_m1(w, K, W, dist, device, pk, seed_base=rank_seed(w.seed, dist.rank))
     sampler.stop_ev.set()
     sampler.join(timeout=2)
@@ -577,9 +607,9 @@ def run_ours(args):
                    "parallelism": "dp%d (independent batches per GPU)" % dist.world},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": hbm,
                      "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                     "traffic": traffic_for("m1_scan_130m" if generic else "m1_scan_tma_130m"),
+                     "traffic": traffic_for("m1_scan_tma_130m"),
                      "peak_source": "%s hbm_gbs (copy)" % pk["_source"],
-                     "kernel": "m1_scan_kernel" if generic else "m1_scan_tma_kernel",
+                     "kernel": "m1_scan_tma_kernel",
                      "sfu": m1_sfu_roofline(w, r["launch_ms"], clocks)},
         "clocks": clocks,
         "gpu_launches": r["launches_per_step"] * K,

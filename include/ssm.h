@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define SSM_ABI_VERSION 1
+#define SSM_ABI_VERSION 2
 
 typedef enum ssm_status {
   SSM_OK = 0,
@@ -55,7 +55,8 @@ typedef enum ssm_status {
   SSM_ERR_UNSUPPORTED = 5, /* a valid combination this build has no kernel for */
   SSM_ERR_WORKSPACE = 6,   /* workspace missing or smaller than required      */
   SSM_ERR_CUDA = 7,        /* a CUDA launch or runtime call failed            */
-  SSM_ERR_TIMEOUT = 8      /* reserved: a bounded device wait ran out         */
+  SSM_ERR_TIMEOUT = 8      /* a bounded device wait ran out (see
+                              ssm_workspace_status)                           */
 } ssm_status_t;
 
 typedef enum ssm_dtype { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
@@ -91,8 +92,19 @@ typedef enum ssm_dtype { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
  *   h_last      : [batch, channels, state] float32 or NULL; may equal h0
  *   states      : [batch, seqlen, channels, state] float32 or NULL: the state
  *                 after every token (states[:, -1] == h_last bit for bit)
- *   workspace   : needed only with SSM_RMSNORM_DT; size from
- *                 ssm_scan_workspace().  Device memory, caller-owned.
+ *   workspace   : device memory of ssm_scan_workspace() bytes (at least 256),
+ *                 caller-owned.  Word 0 (int32) is the call's status word:
+ *                 the call zeroes it, and a kernel whose bounded wait for its
+ *                 own copies runs out (about a second: a fault elsewhere on the
+ *                 device) sets it non-zero and leaves y and h_last
+ *                 incomplete; ssm_workspace_status() reads it.  The rest
+ *                 holds the step-input RMS factors (SSM_RMSNORM_DT) and, when
+ *                 batch x channels is too small to fill the device's SMs,
+ *                 the states of the sequence segments the scan is cut into
+ *                 (their end states, the sums of their steps and the carried
+ *                 states); its size therefore depends on the device current at
+ *                 the query, and a call with less than its own device needs
+ *                 returns SSM_ERR_WORKSPACE.
  *
  * Supported: state in {4, 8, 16, 32, 64}; groups must divide channels, and
  * with groups > 1 channels/groups must be a multiple of 32.
@@ -110,9 +122,9 @@ typedef struct ssm_scan_args {
   size_t workspace_bytes;
 } ssm_scan_args_t;
 
-/* Bytes of device workspace ssm_scan_fwd needs for these arguments (0 unless
- * SSM_RMSNORM_DT).  Validates sizes, dtype and flags as ssm_scan_fwd does;
- * the tensor pointers are not looked at. */
+/* Bytes of device workspace ssm_scan_fwd needs for these arguments.
+ * Validates sizes, dtype and flags as ssm_scan_fwd does; the tensor pointers
+ * are not looked at. */
 ssm_status_t ssm_scan_workspace(const ssm_scan_args_t *args, size_t *bytes);
 ssm_status_t ssm_scan_fwd(const ssm_scan_args_t *args, void *stream);
 
@@ -123,20 +135,25 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_args_t *args, void *stream);
  * enqueue callback that may only use memory reserved up front, a decode loop
  * with a latency budget that must not meet an allocator that can
  * synchronise the device, a process whose device memory another component
- * has reserved.  With SSM_RMSNORM_DT, ssm_scan_fwd needs a workspace of
- * batch * seqlen floats; this entry point uses a fixed array in the
- * library's own device memory instead (static, 1 MiB per GPU, held until the
- * process exits), so the caller passes only inputs and outputs.
+ * has reserved.  ssm_scan_fwd needs a caller workspace (a status word, the
+ * step-input RMS factors with SSM_RMSNORM_DT, and sequence segments' states
+ * when it cuts a long sequence); this entry point uses a fixed array in the
+ * library's own device memory instead (static, 256 bytes + 1 MiB per GPU,
+ * held until the process exits) and never cuts the sequence, so the caller
+ * passes only inputs and outputs.
  *
  * Arguments, layouts, results and errors are those of ssm_scan_fwd;
- * args->workspace is ignored.  Limit: with SSM_RMSNORM_DT, batch * seqlen
- * must not exceed 262144; larger problems return SSM_ERR_WORKSPACE before
- * anything touches the device.  The first call on each device looks up the
+ * args->workspace is ignored.  Every host-side check runs before anything
+ * touches the device.  Limit: with SSM_RMSNORM_DT, batch * seqlen must not
+ * exceed 262144; larger problems return SSM_ERR_WORKSPACE.  The first call
+ * on each device (and after the device's context is recreated) looks up the
  * array's device address (cudaGetSymbolAddress) with that device current;
  * make that first call before any stream capture.  All calls share the
- * array, which keeps the last call's contents (nothing in it needs to start
- * at zero); calls that overlap on the GPU -- on different streams, or from
- * several threads -- race on it and must be serialised by the caller. */
+ * array, which keeps the last call's contents: each call clears the status
+ * word it uses, and the RMS factors need no clearing (every one the scan
+ * reads is written first).  Calls that overlap on the GPU -- on different
+ * streams, or from several threads -- race on it and must be serialised by
+ * the caller.  ssm_workspace_status(NULL, stream) reads its status word. */
 ssm_status_t ssm_scan_fwd_static(const ssm_scan_args_t *args, void *stream);
 
 /* ssm_scan_fwd_write -- ssm_scan_fwd with the state written at one token.
@@ -150,6 +167,17 @@ ssm_status_t ssm_scan_fwd_static(const ssm_scan_args_t *args, void *stream);
  * SSD counterpart.) */
 ssm_status_t ssm_scan_fwd_write(const ssm_scan_args_t *args, int64_t t_write,
                                 const float *state_write, void *stream);
+
+/* ssm_workspace_status -- did the call that used this workspace finish?
+ *
+ * Synchronises `stream`, reads word 0 of `workspace` (a workspace of
+ * ssm_scan_fwd, ssm_scan_fwd_write or ssd_chunk_scan_fwd, after a call queued
+ * on `stream`) and returns SSM_OK, or SSM_ERR_TIMEOUT when one of that call's
+ * bounded device waits ran out (its outputs are then incomplete).
+ * workspace == NULL reads the status word of ssm_scan_fwd_static's static
+ * scratch on the current device.  SSM_ERR_CUDA if the copy or the
+ * synchronisation fails. */
+ssm_status_t ssm_workspace_status(const void *workspace, void *stream);
 
 /* ------------------------------------------------------------------------
  * ssd_chunk_scan_fwd -- Mamba-2 (SSD) scan.
@@ -177,7 +205,10 @@ ssm_status_t ssm_scan_fwd_write(const ssm_scan_args_t *args, int64_t t_write,
  *   h_last   : [batch, heads, state, head_dim] float32 or NULL; may equal h0
  *   states   : [batch, seqlen, heads, state, head_dim] float32 or NULL
  *   workspace: device memory of ssd_chunk_scan_workspace() bytes, or NULL if
- *              that is 0.
+ *              that is 0.  When non-zero, word 0 (int32) is the call's
+ *              status word, as for ssm_scan_fwd: zeroed by the call, set
+ *              non-zero when a bounded device wait runs out (y and h_last
+ *              then incomplete); read it with ssm_workspace_status().
  *
  * Only SSM_DT_SOFTPLUS is accepted in flags.
  * ---------------------------------------------------------------------- */

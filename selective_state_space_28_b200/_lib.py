@@ -107,7 +107,10 @@ def lib():
         L.ssd_attention_fwd.argtypes = [ctypes.POINTER(AttnArgs), _vp]
         L.ssd_attention_workspace.argtypes = [ctypes.POINTER(AttnArgs),
                                               ctypes.POINTER(ctypes.c_size_t)]
-        for fn in (L.ssm_scan_fwd, L.ssm_scan_workspace, L.ssd_chunk_scan_fwd,
+        L.ssm_scan_fwd_static.argtypes = [ctypes.POINTER(ScanArgs), _vp]
+        L.ssm_workspace_status.argtypes = [_vp, _vp]
+        for fn in (L.ssm_scan_fwd_static, L.ssm_workspace_status,
+                   L.ssm_scan_fwd, L.ssm_scan_workspace, L.ssd_chunk_scan_fwd,
                    L.ssd_chunk_scan_workspace, L.ssm_scan_step, L.ssm_conv1d_fwd,
                    L.ssm_gated_rmsnorm_fwd, L.ssm_scan_fwd_write, L.ssd_attention_fwd,
                    L.ssd_attention_workspace):

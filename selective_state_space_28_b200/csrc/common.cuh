@@ -114,6 +114,36 @@ __device__ __forceinline__ float softplus_sfu(float v) {
   return v > 20.f ? v : r;
 }
 
+// ------------------------------------------------- exp2 on the FMA pipe
+// 2^x on the FMA pipe instead of the SFU, for decays (x = d * A2 with d >= 0
+// and A2 < 0): Cody-Waite reduction 2^x = 2^j 2^f with j = round(x) and
+// f = x - j in [-1/2, 1/2], a degree-5 polynomial for 2^f (coefficients and
+// their weighted least-squares fit on Chebyshev nodes in gen_exp2_poly.py;
+// max relative error 1.9e-7 in float32; exactly 1 at f = 0), 2^j applied
+// through the exponent field.  d is first clamped to lim = -127 / A2 so that
+// the exponent never drops below -127, where the result is exactly 0.
+
+// 1.5 * 2^23 + 127: adding it rounds x to an integer j held in the low
+// mantissa bits, biased by 127 so that (bits << 23) is the float 2^j.
+constexpr float kMagic = 12583039.0f;
+constexpr float kP1 = 6.931468844e-01f, kP2 = 2.402223796e-01f, kP3 = 5.550893024e-02f,
+                kP4 = 9.671698324e-03f, kP5 = 1.321867225e-03f;
+
+__device__ __forceinline__ f2 exp2_fma2(float d, f2 A2, f2 lim) {
+  const f2 dc = mk2(fminf(d, lim.x), fminf(d, lim.y));
+  const f2 t = fma2(dc, A2, mk2(kMagic, kMagic));      // j + magic
+  const f2 r = add2(t, mk2(-kMagic, -kMagic));          // j
+  const f2 f = fma2(dc, A2, mk2(-r.x, -r.y));           // x - j in [-1/2, 1/2]
+  f2 p = fma2(mk2(kP5, kP5), f, mk2(kP4, kP4));
+  p = fma2(p, f, mk2(kP3, kP3));
+  p = fma2(p, f, mk2(kP2, kP2));
+  p = fma2(p, f, mk2(kP1, kP1));
+  p = fma2(p, f, mk2(1.f, 1.f));                        // ~ 2^f, exactly 1 at f = 0
+  const f2 s = mk2(__uint_as_float(__float_as_uint(t.x) << 23),
+                   __uint_as_float(__float_as_uint(t.y) << 23));  // 2^j
+  return mul2(p, s);
+}
+
 // --------------------------------------------------------- cache hints
 
 // Streaming 16-byte load/store (no reuse expected: evict-first).

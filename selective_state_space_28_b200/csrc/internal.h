@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "ssm.h"
+
 namespace ssm {
 
 // Mamba-1 scan, device pointers as in ssm_scan_args_t.
@@ -16,13 +18,27 @@ struct M1Params {
   const float *A, *D, *dt_bias, *h0;
   void *y;
   float *h_last, *states;
-  float *rstd;  // [batch * L] RMS factors of dt rows, or nullptr
-  int pipelined;  // use the TMA-pipelined kernel where the shape allows
-  int variant;    // pipelined-kernel variant (tuning)
-  int *status;  // device word set non-zero if a bounded wait ran out, or nullptr
-  int64_t t_write = -1;                 // token whose state is replaced (generic kernel)
+  float *rstd = nullptr;  // [batch * L] RMS factors of dt rows, or nullptr
+  int *status = nullptr;  // device word set non-zero if a bounded wait ran out
+  int64_t t_write = -1;                 // token whose state is replaced
   const float *state_write = nullptr;   // [batch, C, N] state written at t_write
+  // sequence segments of the pipelined kernel (nseg 1: the whole sequence)
+  int nseg = 1;
+  int64_t seg_len = 0;
+  float *seg_end = nullptr;   // [nseg - 1, batch, C, N] end states from zero / h0
+  float *seg_dsum = nullptr;  // [nseg - 1, batch, C] sums of the segments' steps
+  float *seg_ent = nullptr;   // [nseg, batch, C, N] states entering each segment
 };
+
+// How the pipelined Mamba-1 kernel cuts the sequence (nseg 1: no cut).
+struct M1Split {
+  int nseg = 1;
+  int64_t seg_len = 0;
+};
+M1Split m1_scan_split(int64_t batch, int64_t C, int64_t L, int64_t N, int sms);
+size_t m1_scan_split_bytes(const M1Split &r, int64_t batch, int64_t C, int64_t N);
+void m1_scan_split_carve(const M1Split &r, int64_t batch, int64_t C, int64_t N, void *ws,
+                         M1Params &p);
 
 // Mamba-2 token recurrence (the decode step, and the SSD path for shapes the
 // chunked tensor-core kernel does not cover).
@@ -122,5 +138,17 @@ cudaError_t launch_gated_norm(const GatedNormParams &p, cudaStream_t s);
 cudaError_t launch_conv1d(const ConvParams &p, cudaStream_t s);
 cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split, void *seg_ws,
                           cudaStream_t s);
+
+// The Mamba-1 scan behind ssm_scan_fwd, ssm_scan_fwd_write (t_write >= 0)
+// and ssm_scan_fwd_static (allow_cut false: the sequence is never cut into
+// segments, so the workspace is the status word and the dt-norm factors).
+ssm_status_t scan_run(const ssm_scan_args_t *a, int64_t t_write, const float *state_write,
+                      void *stream, bool allow_cut);
+// Every host-side check of ssm_scan_fwd (pointers included), touching no
+// device: SSM_OK or the error status.
+ssm_status_t scan_validate(const ssm_scan_args_t *a);
+// Device address of the allocation-free entry point's static scratch on the
+// current device (its first word is that entry point's status word).
+cudaError_t static_scratch_address(void **out);
 
 }  // namespace ssm

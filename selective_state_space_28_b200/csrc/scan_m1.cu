@@ -193,9 +193,9 @@ cudaError_t launch_t(const M1Params &p, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  // the pipelined kernel carries a state write for N = 16 without per-token states
-  const bool tma_write_ok = !p.state_write || (p.N == 16 && !p.states);
-  if (p.pipelined && tma_write_ok && m1_scan_tma_supported(p)) return launch_m1_scan_tma(p, s);
+  // the pipelined kernel wherever the shape allows; a state write together
+  // with per-token states takes the generic kernel
+  if (!(p.state_write && p.states) && m1_scan_tma_supported(p)) return launch_m1_scan_tma(p, s);
   switch (p.N) {
     case 4: return launch_n<4, T>(p, s);
     case 8: return launch_n<8, T>(p, s);

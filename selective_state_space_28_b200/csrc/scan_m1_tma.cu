@@ -2,36 +2,51 @@
 //
 // Same arithmetic as scan_m1.cu ("Mamba", nnterp guide, intro and "The
 // values"; "Mamba", tokentrails, "Code"; "Falcon-Mamba", "Where the norms
-// sit"), organised for throughput on sm_100a:
+// sit"):
+//   d = softplus(dt * rstd + dt_bias[c]);  h[n] = exp(d A[c,n]) h[n] + d B[n] x
+//   y = C . h + D[c] x;  y *= silu(z)
+// organised for throughput on sm_100a.
 //
-// * One CTA owns one batch row and CT channels for the whole sequence (the
-//   recurrence never leaves the CTA).  Each channel's N states sit in
-//   G = N/4 lanes, 4 float32 states per lane, in registers.
-// * The sequence is walked in stages of 32 tokens.  TMA brings the stage's
-//   x, dt, z ([32 x CT]) and B, C ([32 x N]) tiles into a double buffer, so
-//   the loads of stage s+1 run under the arithmetic of stage s.
-// * Prologue, once per element: d = softplus(dt * rstd + dt_bias) and d*x
-//   (float2 per (token, channel)); B and C widened to float32 (and RMS-normed
-//   per token when asked).
-// * Recurrence: per token each lane updates its 4 states with packed f32x2
-//   multiply/FMA and forms its partial C.h.  Every G tokens the G lanes of a
-//   channel exchange partials in log2(G) shuffle rounds so that lane q ends
-//   with the complete C.h of token q of the group (a transposing
-//   reduction: G-1 shuffles per lane per G tokens) and applies the skip
-//   term, the gate and the bf16 rounding for that one token.
-// * exp(d A) costs one SFU ex2 per state; the SFU issues 16 per SM per
-//   clock, a quarter of what the other work needs, so SWX of the 4 states
-//   of a lane take a second exponential on the FMA pipe instead: Cody-Waite
-//   reduction 2^x = 2^j 2^f with j = round(x), and a degree-5 polynomial
-//   for 2^f on [-1/2, 1/2] (coefficients and their fit in
-//   gen_exp2_poly.py; max relative error 1.9e-7 in float32), 2^j applied
-//   through the exponent field.
+// Work split.  A CTA owns one batch row, 32 channels and one segment of the
+// sequence.  Each channel's N states sit in G = N/4 lanes of one warp, four
+// float32 states per lane, in registers; a warp holds 32/G channels.  The
+// segment is walked in stages of 32 tokens that TMA brings into a ring of NS
+// stage buffers (x, dt, z as [32 tokens x 32 channels], B and C as
+// [32 tokens x N]).
+//
+// Per stage, every warp (no CTA-wide barrier anywhere in the loop):
+//   1. waits for the stage's bytes (mbarrier `full`);
+//   2. widens (and, with SSM_RMSNORM_BC, RMS-normalises) its share of the
+//      stage's B and C rows into float32, then arrives on `conv`;
+//   3. computes d and d*x for its own channels, one token per lane;
+//   4. waits on `conv` (every warp's B/C share), then runs the recurrence:
+//      per token each lane updates its four states with packed f32x2
+//      arithmetic and forms its partial C.h; every G tokens the G lanes of a
+//      channel trade partials in log2(G) shuffle rounds so that lane q ends
+//      with token q's complete C.h (a transposing reduction), and applies the
+//      skip term, the gate and the rounding for that token;
+//   5. arrives on `empty`; the issuing thread refills a stage's buffer once
+//      every warp has released it.
+//
+// Sequence segments (the carry across chunks).  When batch x channels gives
+// too few warps to fill the SMs, the sequence is cut into S segments and run
+// in three launches: (1) segments 0..S-2 scanned from their own start (h0 for
+// the first, zeros for the others) without any readout, leaving their end
+// states and the sum of their steps; (2) a carry kernel that chains them: the
+// state entering segment k+1 is P_k * (state entering k) + E_k with
+// P_k[n] = exp(A[c,n] * sum of the segment's steps), evaluated as an
+// inclusive warp-shuffle scan over the (P, E) pairs, which compose
+// associatively; (3) every segment rescanned from its entering state with the
+// readout.  Rescanning from the carried state computes exactly
+// h_t = (local state from zero)_t + (prod of decays)_t * carry, the fix-up,
+// without storing the local states.
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 #include "tma.h"
 
-#include <type_traits>
+#include <algorithm>
+#include <cmath>
 
 namespace ssm {
 namespace {
@@ -39,43 +54,39 @@ namespace {
 using namespace sm100;
 
 constexpr int kTL = 32;  // tokens per stage
-constexpr int kNS = 2;   // stages in flight
-constexpr long long kWaitLimit = 2000000000ll;
+constexpr int kCT = 32;  // channels per CTA
+constexpr long long kWaitLimit = 2000000000ll;  // clock cycles (about one second)
 
-// 1.5 * 2^23 + 127: adding it rounds x to an integer j held in the low
-// mantissa bits, biased by 127 so that (bits << 23) is the float 2^j.
-constexpr float kMagic = 12583039.0f;
-constexpr float kP1 = 6.931468844e-01f, kP2 = 2.402223796e-01f, kP3 = 5.550893024e-02f,
-                kP4 = 9.671698324e-03f, kP5 = 1.321867225e-03f;
+enum { kModeFull = 0, kModeStateOnly = 1 };
 
-// 2^(d*A2) for two states on the FMA pipe, for d >= 0 and A2 < 0 (a decay):
-// d is first clamped to lim = -127 / A2 so that the exponent never drops below
-// -127, where the result is exactly 0.
-__device__ __forceinline__ f2 exp2_fma2(float d, f2 A2, f2 lim) {
-  const f2 dc = mk2(fminf(d, lim.x), fminf(d, lim.y));
-  const f2 t = fma2(dc, A2, mk2(kMagic, kMagic));      // j + magic
-  const f2 r = add2(t, mk2(-kMagic, -kMagic));          // j
-  const f2 f = fma2(dc, A2, mk2(-r.x, -r.y));           // x - j in [-1/2, 1/2]
-  f2 p = fma2(mk2(kP5, kP5), f, mk2(kP4, kP4));
-  p = fma2(p, f, mk2(kP3, kP3));
-  p = fma2(p, f, mk2(kP2, kP2));
-  p = fma2(p, f, mk2(kP1, kP1));
-  p = fma2(p, f, mk2(1.f, 1.f));                        // ~ 2^f, exactly 1 at f = 0
-  const f2 s = mk2(__uint_as_float(__float_as_uint(t.x) << 23),
-                   __uint_as_float(__float_as_uint(t.y) << 23));  // 2^j
-  return mul2(p, s);
-}
-__device__ __forceinline__ float exp2_fma1(float d, float A2, float lim) {
-  const float dc = fminf(d, lim);
-  const float t = fmaf(dc, A2, kMagic);
-  const float r = t - kMagic;
-  const float f = fmaf(dc, A2, -r);
-  float p = fmaf(kP5, f, kP4);
-  p = fmaf(p, f, kP3);
-  p = fmaf(p, f, kP2);
-  p = fmaf(p, f, kP1);
-  p = fmaf(p, f, 1.f);
-  return p * __uint_as_float(__float_as_uint(t) << 23);
+// Decays per lane (of 4) taken by the FMA-pipe exp2 instead of the SFU (0 or
+// 2): the SFU issues 16 exponentials per SM per clock, the FMA pipe 128
+// lane-operations, so moving a share of the decays balances the two.
+constexpr int kPolyStates = 0;
+
+template <int N, typename T, int NS>
+struct alignas(128) ScanSmem {
+  T x[NS][kTL][kCT];
+  T dt[NS][kTL][kCT];
+  T z[NS][kTL][kCT];
+  T B[NS][kTL][N];
+  T C[NS][kTL][N];
+  float bc[NS][kTL][2][N];  // B, C widened to float32 (and normed)
+  // Per (token, channel) of a stage: (d, d*x) for the recurrence and
+  // (D*x, silu(z)) for the epilogue.  Two buffers by stage parity: a warp
+  // that has finished stage s writes stage s+1's values while another still
+  // reads stage s's (no warp gets further ahead: the next stage's scan waits
+  // for every warp's `conv` arrival).  Rows are padded by 16 bytes so that a
+  // warp's lanes, one row each, fall in distinct banks.
+  float2 ddx[2][kTL][kCT + 2];
+  float2 eg[2][kTL][kCT + 2];
+  T y[kTL][kCT + 16 / sizeof(T)];  // output staging, rows padded by 16 bytes
+  float bias[kCT], skip[kCT];
+  uint64_t full[NS], conv[NS], empty[NS];
+};
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Lane q of a group of G lanes holds partials p[u] of tokens u = 0..G-1; on
@@ -95,291 +106,381 @@ __device__ __forceinline__ float transpose_reduce(float (&p)[G], int q) {
   return p[0];
 }
 
-template <int N, typename T, int CT>
-struct alignas(128) M1Smem {
-  T x[kNS][kTL][CT];
-  T dt[kNS][kTL][CT];
-  T z[kNS][kTL][CT];
-  T B[kNS][kTL][N];
-  T C[kNS][kTL][N];
-  float2 ddx[kTL][CT];      // (d, d*x)
-  float bc[kTL][2][N];      // B, C in float32
-  T y[kTL][CT];
-  uint64_t full[kNS];
-};
+// J consecutive I/O values from shared memory, widened to float32 (bf16 -> f32
+// is exact: the bf16 bits are the top half of the f32 bits).
+template <int J, typename T>
+__device__ __forceinline__ void widen(const T *src, float (&v)[J]) {
+  if constexpr (sizeof(T) == 2) {
+    if constexpr (J == 8) {
+      const uint4 w = *reinterpret_cast<const uint4 *>(src);
+      v[0] = bf16lo(w.x); v[1] = bf16hi(w.x); v[2] = bf16lo(w.y); v[3] = bf16hi(w.y);
+      v[4] = bf16lo(w.z); v[5] = bf16hi(w.z); v[6] = bf16lo(w.w); v[7] = bf16hi(w.w);
+    } else {
+      static_assert(J == 4, "4 or 8 values");
+      const uint2 w = *reinterpret_cast<const uint2 *>(src);
+      v[0] = bf16lo(w.x); v[1] = bf16hi(w.x); v[2] = bf16lo(w.y); v[3] = bf16hi(w.y);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < J; i += 4) {
+      const float4 a = *reinterpret_cast<const float4 *>(src + i);
+      v[i] = a.x; v[i + 1] = a.y; v[i + 2] = a.z; v[i + 3] = a.w;
+    }
+  }
+}
 
-// SPL states per lane (2 or 4), G = N / SPL lanes per channel.  SWX of a
-// lane's SPL decays use the FMA-pipe exp2.  STATES: also store every token's
-// state.
-// PK: packed f32x2 state arithmetic (else scalar); UT: token groups per loop
-// iteration (2 lets one group's shuffle reduction overlap the next group's
-// arithmetic).
-template <int N, typename T, int CT, bool HAS_Z, int SWX, int SPL, bool STATES, bool PK, int UT,
-          bool WR = false>
-__global__ void __launch_bounds__(CT *(N / SPL))
+// NP pairs of float32 (SPL = 2 NP consecutive values) from / to memory.
+template <int NP>
+__device__ __forceinline__ void load_pairs(const float *src, f2 (&v)[NP]) {
+  if constexpr (NP == 2) {
+    const float4 a = *reinterpret_cast<const float4 *>(src);
+    v[0] = mk2(a.x, a.y);
+    v[1] = mk2(a.z, a.w);
+  } else {
+    static_assert(NP == 1, "2 or 4 states per lane");
+    const float2 a = *reinterpret_cast<const float2 *>(src);
+    v[0] = mk2(a.x, a.y);
+  }
+}
+template <int NP>
+__device__ __forceinline__ void store_pairs(float *dst, const f2 (&v)[NP]) {
+  if constexpr (NP == 2)
+    *reinterpret_cast<float4 *>(dst) = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+  else
+    *reinterpret_cast<float2 *>(dst) = make_float2(v[0].x, v[0].y);
+}
+
+// MODE: full scan with readout, or state-only (segments' end states).
+// STATES: also store every token's state.  WR: replace the state at token
+// p.t_write (the state write).
+// SPL: states per lane (4, or 2 for twice the warps on small problems).
+template <int N, int SPL, typename T, int NS, bool HAS_Z, int MODE, bool STATES, bool WR, int PX>
+__global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
     m1_scan_tma_kernel(const __grid_constant__ CUtensorMap mx,
                        const __grid_constant__ CUtensorMap mdt,
                        const __grid_constant__ CUtensorMap mz,
                        const __grid_constant__ CUtensorMap mB,
                        const __grid_constant__ CUtensorMap mC, const M1Params p) {
-  constexpr int G = N / SPL;  // lanes per channel
-  constexpr int NT = CT * G;
-  constexpr int NP = SPL / 2;  // state pairs per lane
+  constexpr int G = N / SPL;        // lanes per channel
+  constexpr int NP = SPL / 2;       // state pairs per lane
+  constexpr int CPW = 32 / G;       // channels per warp
+  constexpr int NW = kCT / CPW;     // warps per CTA
+  constexpr int TPW = kTL / NW;     // B/C rows each warp widens per stage
   constexpr bool kBF16 = sizeof(T) == 2;
-  static_assert(!WR || PK, "the state write is carried by the packed form only");
-  using S = M1Smem<N, T, CT>;
+  constexpr bool kFull = MODE == kModeFull;
+  static_assert(N % 8 == 0 || !kBF16, "bf16 rows of B and C are 16-byte multiples");
+  using S = ScanSmem<N, T, NS>;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   S &s = *reinterpret_cast<S *>(smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u));
 
   const int64_t L = p.L, C = p.C, Gr = p.G;
-  const int b = blockIdx.y;
-  const int64_t c0 = (int64_t)blockIdx.x * CT;
-  const int tid = threadIdx.x;
-  const int cl = tid / G, q = tid % G;
-  const int64_t c = c0 + cl;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int ch = lane / G, q = lane % G;
+  const int cw0 = warp * CPW;  // the warp's first channel within the CTA's 32
+  const int64_t c0 = (int64_t)blockIdx.x * kCT;
+  const int64_t c = c0 + cw0 + ch;
   const bool cvalid = c < C;
+  const int b = blockIdx.y;
+  const int seg = blockIdx.z;
   const int g = (int)(c0 / (C / Gr));
-  const int nst = (int)((L + kTL - 1) / kTL);
+  const int64_t tb = (int64_t)seg * p.seg_len;
+  const int64_t te = tb + p.seg_len < L ? tb + p.seg_len : L;
+  const int nst = (int)((te - tb + kTL - 1) / kTL);
   const bool softplus_on = p.flags & 1u;
   const bool rms_bc = p.flags & 2u;
-  constexpr uint32_t kStageBytes = (3 * kTL * CT + 2 * kTL * N) * sizeof(T);
-  constexpr uint32_t kStageBytesNoZ = (2 * kTL * CT + 2 * kTL * N) * sizeof(T);
+  constexpr uint32_t kStageBytes = ((HAS_Z ? 3 : 2) * kTL * kCT + 2 * kTL * N) * sizeof(T);
 
-  if (tid == 0) {
-    for (int i = 0; i < kNS; ++i) mbar_init(&s.full[i], 1);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.conv[i], NW * 32);  // every lane arrives (release of its own writes)
+      mbar_init(&s.empty[i], NW * 32);
+    }
     fence_mbar_init();
   }
+  if (threadIdx.x < kCT) {
+    const bool v = c0 + threadIdx.x < C;
+    s.bias[threadIdx.x] = (p.dt_bias && v) ? p.dt_bias[c0 + threadIdx.x] : 0.f;
+    s.skip[threadIdx.x] = (p.D && v) ? p.D[c0 + threadIdx.x] : 0.f;
+  }
   __syncthreads();
+
+  const bool issuer = threadIdx.x == 0;
+  int issued = 0;
   auto issue = [&](int stage) {
-    const int buf = stage % kNS, t0 = stage * kTL;
-    mbar_expect_tx(&s.full[buf], HAS_Z ? kStageBytes : kStageBytesNoZ);
+    const int buf = stage % NS;
+    const int t0 = (int)(tb + (int64_t)stage * kTL);
+    mbar_expect_tx(&s.full[buf], kStageBytes);
     tma_load_3d(&s.x[buf][0][0], &mx, &s.full[buf], (int)c0, t0, b);
     tma_load_3d(&s.dt[buf][0][0], &mdt, &s.full[buf], (int)c0, t0, b);
     if (HAS_Z) tma_load_3d(&s.z[buf][0][0], &mz, &s.full[buf], (int)c0, t0, b);
     tma_load_3d(&s.B[buf][0][0], &mB, &s.full[buf], g * N, t0, b);
     tma_load_3d(&s.C[buf][0][0], &mC, &s.full[buf], g * N, t0, b);
   };
-  if (tid == 0)
-    for (int i = 0; i < kNS && i < nst; ++i) issue(i);
+  if (issuer)
+    for (; issued < NS && issued < nst; ++issued) issue(issued);
 
-  float h[SPL], A2[SPL], lim[SPL];
+  // The start state: h0 (or zeros), the carried state of this segment, or
+  // zeros for a segment scanned from its own start.
+  const float *h_in = nullptr;
+  if (MODE == kModeStateOnly) h_in = seg == 0 ? p.h0 : nullptr;
+  else h_in = p.nseg > 1 ? p.seg_ent + (int64_t)seg * p.batch * C * N : p.h0;
+  f2 h[NP], A2[NP];
 #pragma unroll
-  for (int j = 0; j < SPL; ++j) {
-    h[j] = (cvalid && p.h0) ? p.h0[(b * C + c) * N + SPL * q + j] : 0.f;
-    A2[j] = cvalid ? p.A[c * N + SPL * q + j] * kLog2e : 0.f;
-    lim[j] = A2[j] < 0.f ? -127.f / A2[j] : 3.0e38f;
+  for (int j = 0; j < NP; ++j) h[j] = A2[j] = mk2(0.f, 0.f);
+  if (cvalid) {
+    if (h_in) load_pairs<NP>(h_in + (b * C + c) * N + SPL * q, h);
+    load_pairs<NP>(p.A + c * N + SPL * q, A2);
+#pragma unroll
+    for (int j = 0; j < NP; ++j) A2[j] = mk2(A2[j].x * kLog2e, A2[j].y * kLog2e);
   }
   // The FMA-pipe exponential assumes decays (d >= 0, A < 0); a warp where any
-  // of its states could grow uses the SFU for all of them.
-  bool sw_ok = softplus_on;
-#pragma unroll
-  for (int j = SPL - SWX; j < SPL; ++j) sw_ok = sw_ok && (A2[j] < 0.f || !cvalid);
-  sw_ok = __all_sync(0xffffffffu, sw_ok);
-  const float Dc = (cvalid && p.D) ? p.D[c] : 0.f;
-  // Prologue mapping: this thread always handles column pc of the tile.
-  constexpr int TPR = NT / CT;
-  const int pc = tid % CT, pt0 = tid / CT;
-  const bool pvalid = c0 + pc < C;
-  const float bias_pc = (pvalid && p.dt_bias) ? p.dt_bias[c0 + pc] : 0.f;
+  // of its states could grow keeps every decay on the SFU.
+  // (the last pair of a lane's states, when PX == 2)
+  const f2 Al = A2[NP - 1];
+  const f2 liml = mk2(Al.x < 0.f ? -127.f / Al.x : 3.0e38f, Al.y < 0.f ? -127.f / Al.y : 3.0e38f);
+  const bool poly_ok =
+      PX == 2 && __all_sync(0xffffffffu, softplus_on && ((Al.x < 0.f && Al.y < 0.f) || !cvalid));
+  float dsum = 0.f;
+  bool failed = false;
 
   for (int sg = 0; sg < nst; ++sg) {
-    const int buf = sg % kNS;
-    const int64_t t0 = (int64_t)sg * kTL;
-    const int tn = (int)(L - t0 < kTL ? L - t0 : kTL);
-    const bool ok = mbar_wait(&s.full[buf], (sg / kNS) & 1, kWaitLimit);
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0 && p.status) atomicExch(p.status, 1);
-      return;
+    const int buf = sg % NS;
+    const uint32_t ph = (uint32_t)(sg / NS) & 1u;
+    const int64_t t0 = tb + (int64_t)sg * kTL;
+    const int tn = (int)(te - t0 < kTL ? te - t0 : kTL);  // tokens of this segment in the stage
+    if (!__all_sync(0xffffffffu, mbar_wait(&s.full[buf], ph, kWaitLimit))) {
+      failed = true;
+      break;
     }
-    // ---- prologue, once per (token, channel) and per (token, B/C row)
-#pragma unroll 4
-    for (int t = pt0; t < kTL; t += TPR) {
-      float dv = 0.f, xv = 0.f;
-      if (t < tn && pvalid) {
-        xv = ld(&s.x[buf][t][pc]);
-        dv = ld(&s.dt[buf][t][pc]);
-        if (p.rstd) dv *= p.rstd[b * L + t0 + t];
-        dv += bias_pc;
-        if (softplus_on) dv = softplus_sfu(dv);
-      }
-      s.ddx[t][pc] = make_float2(dv, dv * xv);
-    }
-    for (int e = tid; e < kTL * 2; e += NT) {
-      const int t = e >> 1, which = e & 1;
+    // ---- 2. widen this warp's share of the stage's B and C rows
+    for (int e = lane; e < TPW * 2; e += 32) {
+      const int t = warp * TPW + (e >> 1), which = e & 1;
       const T *src = which ? s.C[buf][t] : s.B[buf][t];
+      float *dst = s.bc[buf][t][which];
       float v[N];
-      float ss = 0.f;
-      if constexpr (sizeof(T) == 2) {
+      constexpr int J = N % 8 == 0 ? 8 : 4;
 #pragma unroll
-        for (int n = 0; n < N; n += 8) {
-          const uint4 w = *reinterpret_cast<const uint4 *>(src + n);
-          v[n] = bf16lo(w.x); v[n + 1] = bf16hi(w.x); v[n + 2] = bf16lo(w.y); v[n + 3] = bf16hi(w.y);
-          v[n + 4] = bf16lo(w.z); v[n + 5] = bf16hi(w.z); v[n + 6] = bf16lo(w.w); v[n + 7] = bf16hi(w.w);
-        }
-      } else {
+      for (int n = 0; n < N; n += J) {
+        float w[J];
+        widen<J>(src + n, w);
 #pragma unroll
-        for (int n = 0; n < N; n += 4) {
-          const float4 w = *reinterpret_cast<const float4 *>(src + n);
-          v[n] = w.x; v[n + 1] = w.y; v[n + 2] = w.z; v[n + 3] = w.w;
-        }
+        for (int i = 0; i < J; ++i) v[n + i] = w[i];
       }
+      float r = 1.f;
+      if (rms_bc) {
+        float ss = 0.f;
 #pragma unroll
-      for (int n = 0; n < N; ++n) {
-        if (t >= tn) v[n] = 0.f;
-        ss += v[n] * v[n];
+        for (int n = 0; n < N; ++n) ss += v[n] * v[n];
+        r = rsqrtf(ss / N + p.eps);
       }
-      const float r = rms_bc ? rsqrtf(ss / N + p.eps) : 1.f;
 #pragma unroll
       for (int n = 0; n < N; n += 4)
-        *reinterpret_cast<float4 *>(&s.bc[t][which][n]) =
+        *reinterpret_cast<float4 *>(dst + n) =
             make_float4(v[n] * r, v[n + 1] * r, v[n + 2] * r, v[n + 3] * r);
     }
-    __syncthreads();
 
-    // ---- recurrence, G tokens at a time, UT groups per iteration.  With a
-    // state write, only the group holding the written token takes the form
-    // that lets y read the written state; the others run the plain body.
+    // ---- 3. per (token, channel) of this warp's tokens, all 32 channels:
+    // d = softplus(dt * rstd + bias), d * x, D * x and the gate factor.  Four
+    // lanes share a token, each taking 8 channels (conflict-free 16-byte rows).
+    for (int e = lane; e < TPW * 4; e += 32) {
+      const int t = warp * TPW + (e >> 2), k0 = (e & 3) * 8;
+      const bool tvalid = t < tn;
+      const float rs = (tvalid && p.rstd) ? p.rstd[b * L + t0 + t] : 1.f;
+      float xv[8], dv[8], zv[8];
+      widen<8>(&s.x[buf][t][k0], xv);
+      widen<8>(&s.dt[buf][t][k0], dv);
+      if (HAS_Z) widen<8>(&s.z[buf][t][k0], zv);
+      float2 o[8], og[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float d = fmaf(dv[i], rs, s.bias[k0 + i]);
+        if (softplus_on) d = softplus_sfu(d);
+        o[i] = tvalid ? make_float2(d, d * xv[i]) : make_float2(0.f, 0.f);
+        const float gate = HAS_Z ? (kBF16 ? silu_tanh(zv[i]) : silu(zv[i])) : 1.f;
+        og[i] = make_float2(s.skip[k0 + i] * xv[i], gate);
+      }
+      float4 *dst = reinterpret_cast<float4 *>(&s.ddx[sg & 1][t][k0]);
+      float4 *gst = reinterpret_cast<float4 *>(&s.eg[sg & 1][t][k0]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        dst[i] = make_float4(o[2 * i].x, o[2 * i].y, o[2 * i + 1].x, o[2 * i + 1].y);
+        gst[i] = make_float4(og[2 * i].x, og[2 * i].y, og[2 * i + 1].x, og[2 * i + 1].y);
+      }
+    }
+    mbar_arrive(&s.conv[buf]);
+    if (!__all_sync(0xffffffffu, mbar_wait(&s.conv[buf], ph, kWaitLimit))) {
+      failed = true;
+      break;
+    }
+
+    // ---- 4. the recurrence.  Tokens go in steps of SL; the decays and
+    // write terms of step k+1 (independent of the state) are formed while
+    // step k runs its chain, and the readout of step k-1 is reduced and
+    // stored meanwhile, so that a warp always has independent work at hand.
     const int tw = (WR && p.t_write >= t0 && p.t_write < t0 + tn) ? (int)(p.t_write - t0) : -1;
-#pragma unroll 1
-    for (int tg0 = 0; tg0 < kTL; tg0 += G * UT) {
-      auto group = [&](auto wr) {
+    constexpr int SL = G <= 4 ? 4 : G;  // tokens per step
+    struct Pre {
+      f2 a[SL][NP], w[SL][NP];  // decays and write terms d * x * B
+    };
+    auto pre = [&](int tg, Pre &P) {
 #pragma unroll
-        for (int ug = 0; ug < UT; ++ug) {
-          const int tg = tg0 + ug * G;
-          float part[G];
+      for (int u = 0; u < SL; ++u) {
+        const int t = tg + u;
+        const float2 dd = s.ddx[sg & 1][t][cw0 + ch];
+        f2 bv[NP];
+        load_pairs<NP>(&s.bc[buf][t][0][SPL * q], bv);
+        const f2 d2 = mk2(dd.x, dd.x), dx2 = mk2(dd.y, dd.y);
 #pragma unroll
-          for (int u = 0; u < G; ++u) {
-            const int t = tg + u;
-            const float2 ddx = s.ddx[t][cl];
-            const float d = ddx.x, dx = ddx.y;
-            float bv[SPL], cv[SPL], a[SPL];
-            if constexpr (SPL >= 4) {
-#pragma unroll
-              for (int v = 0; v < SPL / 4; ++v) {
-                const float4 b4 = *reinterpret_cast<const float4 *>(&s.bc[t][0][SPL * q + 4 * v]);
-                const float4 c4 = *reinterpret_cast<const float4 *>(&s.bc[t][1][SPL * q + 4 * v]);
-                bv[4 * v] = b4.x; bv[4 * v + 1] = b4.y; bv[4 * v + 2] = b4.z; bv[4 * v + 3] = b4.w;
-                cv[4 * v] = c4.x; cv[4 * v + 1] = c4.y; cv[4 * v + 2] = c4.z; cv[4 * v + 3] = c4.w;
-              }
-            } else {
-              const float2 b2 = *reinterpret_cast<const float2 *>(&s.bc[t][0][2 * q]);
-              const float2 c2 = *reinterpret_cast<const float2 *>(&s.bc[t][1][2 * q]);
-              bv[0] = b2.x; bv[1] = b2.y;
-              cv[0] = c2.x; cv[1] = c2.y;
-            }
-            if constexpr (PK) {
-#pragma unroll
-              for (int pr = 0; pr < NP; ++pr) {
-                const bool fma_pair = (SWX == 2 && SPL == 4 && pr == 1) && sw_ok;
-                const bool fma_last = (SWX == 1 && pr == NP - 1) && sw_ok;
-                if (fma_pair) {
-                  const f2 e = exp2_fma2(d, mk2(A2[2], A2[3]), mk2(lim[2], lim[3]));
-                  a[2] = e.x; a[3] = e.y;
-                } else {
-                  const f2 xx = mul2(mk2(d, d), mk2(A2[2 * pr], A2[2 * pr + 1]));
-                  a[2 * pr] = ex2(xx.x);
-                  a[2 * pr + 1] =
-                      fma_last ? exp2_fma1(d, A2[2 * pr + 1], lim[2 * pr + 1]) : ex2(xx.y);
-                }
-              }
-              const f2 dx2 = mk2(dx, dx);
-              f2 yacc = mk2(0.f, 0.f);
-              if constexpr (decltype(wr)::value) {
-                // a state written at this token replaces h_t before y_t reads
-                // it ("Mamba", nnterp guide, "The state")
-#pragma unroll
-                for (int pr = 0; pr < NP; ++pr) {
-                  const f2 hn = fma2(mk2(a[2 * pr], a[2 * pr + 1]), mk2(h[2 * pr], h[2 * pr + 1]),
-                                     mul2(dx2, mk2(bv[2 * pr], bv[2 * pr + 1])));
-                  h[2 * pr] = hn.x;
-                  h[2 * pr + 1] = hn.y;
-                }
-                if (t == tw && cvalid) {
-#pragma unroll
-                  for (int j = 0; j < SPL; ++j) h[j] = p.state_write[(b * C + c) * N + SPL * q + j];
-                }
-#pragma unroll
-                for (int pr = 0; pr < NP; ++pr)
-                  yacc = fma2(mk2(cv[2 * pr], cv[2 * pr + 1]), mk2(h[2 * pr], h[2 * pr + 1]), yacc);
-              } else {
-#pragma unroll
-                for (int pr = 0; pr < NP; ++pr) {
-                  const f2 hn = fma2(mk2(a[2 * pr], a[2 * pr + 1]), mk2(h[2 * pr], h[2 * pr + 1]),
-                                     mul2(dx2, mk2(bv[2 * pr], bv[2 * pr + 1])));
-                  h[2 * pr] = hn.x;
-                  h[2 * pr + 1] = hn.y;
-                  yacc = fma2(mk2(cv[2 * pr], cv[2 * pr + 1]), hn, yacc);
-                }
-              }
-              part[u] = yacc.x + yacc.y;
-            } else {
-#pragma unroll
-              for (int j = 0; j < SPL; ++j) {
-                const bool fma_j = (j >= SPL - SWX) && sw_ok;
-                a[j] = fma_j ? exp2_fma1(d, A2[j], lim[j]) : ex2(d * A2[j]);
-              }
-              float acc = 0.f;
-#pragma unroll
-              for (int j = 0; j < SPL; ++j) {
-                h[j] = fmaf(a[j], h[j], dx * bv[j]);
-                acc = fmaf(cv[j], h[j], acc);
-              }
-              part[u] = acc;
-            }
-            if constexpr (STATES) {
-              if (cvalid && t < tn) {
-                float *sp = p.states + ((b * L + t0 + t) * C + c) * N + SPL * q;
-#pragma unroll
-                for (int j = 0; j < SPL; j += 2)
-                  *reinterpret_cast<float2 *>(sp + j) = make_float2(h[j], h[j + 1]);
-              }
-            }
+        for (int j = 0; j < NP; ++j) {
+          if (j == NP - 1 && poly_ok) {
+            P.a[u][j] = exp2_fma2(dd.x, Al, liml);
+          } else {
+            const f2 dA = mul2(d2, A2[j]);
+            P.a[u][j] = mk2(ex2(dA.x), ex2(dA.y));
           }
-          const float yq = transpose_reduce<G>(part, q);
-          const int tt = tg + q;  // this lane's token
-          if (tt < tn && cvalid) {
-            float yv = yq + Dc * ld(&s.x[buf][tt][cl]);
-            if (HAS_Z) {
-              const float zv = ld(&s.z[buf][tt][cl]);
-              yv *= kBF16 ? silu_tanh(zv) : silu(zv);
-            }
-            st(&s.y[tt][cl], yv);
-          }
+          P.w[u][j] = mul2(dx2, bv[j]);
         }
-      };
-      if constexpr (WR) {
-        if (tw >= tg0 && tw < tg0 + G * UT)
-          group(std::true_type{});
-        else
-          group(std::false_type{});
-      } else {
-        group(std::false_type{});
+        if (!kFull) dsum += dd.x;
       }
+    };
+    // y for the tokens of one step from its partials (lane q of each group
+    // of G lanes finishes token tg + G k + q)
+    auto finish = [&](int tg, float (&part)[SL]) {
+#pragma unroll
+      for (int k = 0; k < SL / G; ++k) {
+        float pg[G];
+#pragma unroll
+        for (int u = 0; u < G; ++u) pg[u] = part[G * k + u];
+        const float yq = transpose_reduce<G>(pg, q);
+        const int tt = tg + G * k + q;
+        const float2 eg = s.eg[sg & 1][tt][cw0 + ch];
+        st(&s.y[tt][cw0 + ch], (yq + eg.x) * eg.y);
+      }
+    };
+    Pre cur, nxt;
+    pre(0, cur);
+    float partp[SL];
+#pragma unroll
+    for (int tg = 0; tg < kTL; tg += SL) {
+      if (tg + SL < kTL) pre(tg + SL, nxt);
+      float part[SL];
+#pragma unroll
+      for (int u = 0; u < SL; ++u) {
+        const int t = tg + u;
+#pragma unroll
+        for (int j = 0; j < NP; ++j) h[j] = fma2(cur.a[u][j], h[j], cur.w[u][j]);
+        if (WR && t == tw && cvalid) {
+          // a state written at this token replaces h_t before y_t reads it
+          // ("Mamba", nnterp guide, "The state")
+          load_pairs<NP>(p.state_write + (b * C + c) * N + SPL * q, h);
+        }
+        if (kFull) {
+          f2 cv[NP];
+          load_pairs<NP>(&s.bc[buf][t][1][SPL * q], cv);
+          f2 acc = mul2(cv[0], h[0]);
+#pragma unroll
+          for (int j = 1; j < NP; ++j) acc = fma2(cv[j], h[j], acc);
+          part[u] = acc.x + acc.y;
+        }
+        if (STATES && cvalid && t < tn)
+          store_pairs<NP>(p.states + ((b * L + t0 + t) * C + c) * N + SPL * q, h);
+      }
+      if (kFull && tg >= SL) finish(tg - SL, partp);
+#pragma unroll
+      for (int u = 0; u < SL; ++u) partp[u] = part[u];
+      cur = nxt;
     }
-    __syncthreads();
-    // ---- next loads into this buffer, then the y tile
-    if (tid == 0 && sg + kNS < nst) issue(sg + kNS);
-    {
-      constexpr int kChunk = 16 / sizeof(T);   // elements per 16-byte store
-      constexpr int kPerRow = CT / kChunk;
-      T *y = static_cast<T *>(p.y);
-      for (int e = tid; e < tn * kPerRow; e += NT) {
+    if (kFull) finish(kTL - SL, partp);
+    mbar_arrive(&s.empty[buf]);
+
+    // ---- 5. this warp's y tile to global memory (lanes read rows other
+    // lanes wrote: the warp meets first)
+    if (kFull) {
+      __syncwarp();
+      constexpr int kRowBytes = CPW * (int)sizeof(T);
+      constexpr int kChunk = kRowBytes < 16 ? kRowBytes : 16;
+      constexpr int kPerRow = kRowBytes / kChunk;
+      const bool wvalid = c0 + cw0 < C;
+      char *yg = static_cast<char *>(p.y);
+      for (int e = lane; e < kTL * kPerRow; e += 32) {
         const int t = e / kPerRow, k = e % kPerRow;
-        const int64_t cg = c0 + k * kChunk;
-        T *dst = y + (b * L + t0 + t) * C + cg;
-        if (cg + kChunk <= C) {
-          *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(&s.y[t][k * kChunk]);
-        } else {
-          for (int i = 0; i < kChunk && cg + i < C; ++i) dst[i] = s.y[t][k * kChunk + i];
-        }
+        if (t >= tn || !wvalid) continue;
+        const int64_t off = ((b * L + t0 + t) * C + c0 + cw0) * (int64_t)sizeof(T) + k * kChunk;
+        if (c0 + cw0 + (int64_t)k * kChunk / (int64_t)sizeof(T) >= C) continue;
+        const char *src = reinterpret_cast<const char *>(&s.y[t][cw0]) + k * kChunk;
+        if constexpr (kChunk == 16)
+          *reinterpret_cast<uint4 *>(yg + off) = *reinterpret_cast<const uint4 *>(src);
+        else
+          *reinterpret_cast<uint2 *>(yg + off) = *reinterpret_cast<const uint2 *>(src);
+      }
+      __syncwarp();
+    }
+    // ---- refill the buffer of the previous stage once every warp left it
+    if (issuer && sg >= 1 && issued < nst) {
+      const int prev = sg - 1;
+      if (!mbar_wait(&s.empty[prev % NS], (uint32_t)(prev / NS) & 1u, kWaitLimit)) {
+        failed = true;
+      } else {
+        issue(issued);
+        ++issued;
       }
     }
+    if (__any_sync(0xffffffffu, failed)) break;
   }
-  if (p.h_last && cvalid) {
-    float *hp = p.h_last + (b * C + c) * N + SPL * q;
+
+  if (failed) {
+    if (lane == 0 && p.status) atomicExch(p.status, 1);
+    // let every copy this CTA started land before its shared memory goes
+    if (issuer)
+      for (int st_ = 0; st_ < issued; ++st_)
+        mbar_wait(&s.full[st_ % NS], (uint32_t)(st_ / NS) & 1u, kWaitLimit);
+    return;
+  }
+  if (!cvalid) return;
+  if (MODE == kModeStateOnly) {
+    const int64_t i = ((int64_t)seg * p.batch + b) * C + c;
+    store_pairs<NP>(p.seg_end + i * N + SPL * q, h);
+    if (q == 0) p.seg_dsum[i] = dsum;
+  } else if (p.h_last && seg == p.nseg - 1) {
+    store_pairs<NP>(p.h_last + (b * C + c) * N + SPL * q, h);
+  }
+}
+
+// The carry between segments: for each (batch, channel, state) the states
+// entering segments 1..S-1 from the end states of segments 0..S-2 (segment 0
+// from h0, the others from zeros) and the decay products
+// P_k = exp(A * sum of segment k's steps).  Pairs (P, E) compose as
+// (P_a, E_a) then (P_b, E_b) = (P_a P_b, P_b E_a + E_b); an inclusive
+// shuffle scan over a group of SP lanes (lane k = segment k) gives each
+// segment's entering state.  Also copies h0 (or zeros) as segment 0's
+// entering state, so that the rescan never reads h0 (which h_last may alias).
+template <int SP>
+__global__ void m1_seg_carry_kernel(const M1Params p) {
+  const int64_t items = p.batch * p.C * p.N;
+  const int64_t idx = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / SP;
+  const int k = threadIdx.x % SP;
+  const bool live = idx < items;
+  const int64_t it = live ? idx : 0;
+  const int64_t n = it % p.N, bc = it / p.N, c = bc % p.C;
+  const int nprev = p.nseg - 1;  // segments with an end state
+  float P = 1.f, E = 0.f;
+  if (live && k < nprev) {
+    E = p.seg_end[(int64_t)k * items + it];
+    if (k > 0) P = ex2(p.A[c * p.N + n] * kLog2e * p.seg_dsum[(int64_t)k * p.batch * p.C + bc]);
+  }
 #pragma unroll
-    for (int j = 0; j < SPL; j += 2) *reinterpret_cast<float2 *>(hp + j) = make_float2(h[j], h[j + 1]);
+  for (int o = 1; o < SP; o <<= 1) {
+    const float Pp = __shfl_up_sync(0xffffffffu, P, o, SP);
+    const float Ep = __shfl_up_sync(0xffffffffu, E, o, SP);
+    if (k >= o) {
+      E = fmaf(P, Ep, E);
+      P *= Pp;
+    }
   }
+  if (!live) return;
+  if (k < nprev) p.seg_ent[(int64_t)(k + 1) * items + it] = E;
+  if (k == 0) p.seg_ent[it] = p.h0 ? p.h0[it] : 0.f;
 }
 
 template <typename T>
@@ -387,111 +488,173 @@ CUtensorMapDataType tmap_type() {
   return sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
 }
 
-template <int N, typename T, int CT, bool HZ, int SWX, int SPL, bool ST, bool PK = true,
-          int UT = 1, bool WR = false>
-cudaError_t launch_tma(const M1Params &p, cudaStream_t s) {
-  CUtensorMap mx, mdt, mz, mB, mC;
+struct Maps {
+  CUtensorMap x, dt, z, B, C;
+};
+
+template <int N, typename T>
+bool make_maps(const M1Params &p, Maps &m) {
   const uint64_t es = sizeof(T);
-  {
-    uint64_t dims[3] = {(uint64_t)p.C, (uint64_t)p.L, (uint64_t)p.batch};
-    uint64_t strides[2] = {(uint64_t)p.C * es, (uint64_t)(p.L * p.C) * es};
-    uint32_t box[3] = {(uint32_t)CT, (uint32_t)kTL, 1};
-    if (!encode_tiled(&mx, tmap_type<T>(), 3, p.x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_tiled(&mdt, tmap_type<T>(), 3, p.dt, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return cudaErrorInvalidValue;
-    if (HZ && !encode_tiled(&mz, tmap_type<T>(), 3, p.z, dims, strides, box,
-                            CU_TENSOR_MAP_SWIZZLE_NONE))
-      return cudaErrorInvalidValue;
-    if (!HZ) mz = mx;
+  uint64_t dims[3] = {(uint64_t)p.C, (uint64_t)p.L, (uint64_t)p.batch};
+  uint64_t strides[2] = {(uint64_t)p.C * es, (uint64_t)(p.L * p.C) * es};
+  uint32_t box[3] = {(uint32_t)kCT, (uint32_t)kTL, 1};
+  if (!encode_tiled(&m.x, tmap_type<T>(), 3, p.x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_tiled(&m.dt, tmap_type<T>(), 3, p.dt, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return false;
+  if (p.z) {
+    if (!encode_tiled(&m.z, tmap_type<T>(), 3, p.z, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  } else {
+    m.z = m.x;
   }
-  {
-    const uint64_t GN = (uint64_t)(p.G * p.N);
-    uint64_t dims[3] = {GN, (uint64_t)p.L, (uint64_t)p.batch};
-    uint64_t strides[2] = {GN * es, (uint64_t)p.L * GN * es};
-    uint32_t box[3] = {(uint32_t)N, (uint32_t)kTL, 1};
-    if (!encode_tiled(&mB, tmap_type<T>(), 3, p.B, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_tiled(&mC, tmap_type<T>(), 3, p.Cm, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return cudaErrorInvalidValue;
-  }
-  auto k = m1_scan_tma_kernel<N, T, CT, HZ, SWX, SPL, ST, PK, UT, WR>;
-  const size_t smem = sizeof(M1Smem<N, T, CT>) + 128;
-  if (smem > 48 * 1024)
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  dim3 grid((unsigned)((p.C + CT - 1) / CT), (unsigned)p.batch);
-  k<<<grid, CT * (N / SPL), smem, s>>>(mx, mdt, mz, mB, mC, p);
+  const uint64_t GN = (uint64_t)(p.G * p.N);
+  uint64_t bdims[3] = {GN, (uint64_t)p.L, (uint64_t)p.batch};
+  uint64_t bstrides[2] = {GN * es, (uint64_t)p.L * GN * es};
+  uint32_t bbox[3] = {(uint32_t)N, (uint32_t)kTL, 1};
+  return encode_tiled(&m.B, tmap_type<T>(), 3, p.B, bdims, bstrides, bbox,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) &&
+         encode_tiled(&m.C, tmap_type<T>(), 3, p.Cm, bdims, bstrides, bbox,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <int N, int SPL, typename T, bool HZ, int MODE, bool ST, bool WR>
+cudaError_t launch_spl(const Maps &m, const M1Params &p, int nseg, cudaStream_t s) {
+  constexpr int NS = 3;
+  auto k = m1_scan_tma_kernel<N, SPL, T, NS, HZ, MODE, ST, WR, kPolyStates>;
+  const size_t smem = sizeof(ScanSmem<N, T, NS>) + 128;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((p.C + kCT - 1) / kCT), (unsigned)p.batch, (unsigned)nseg);
+  k<<<grid, kCT * (N / SPL), smem, s>>>(m.x, m.dt, m.z, m.B, m.C, p);
   return cudaGetLastError();
 }
 
-// Variant choice: per-token states (tests only) take one fixed form; the
-// others follow p.variant (states per lane, packed math, unrolling, and 8 =
-// one decay per lane on the FMA-pipe exp2).
+// Four states per lane.  (Two per lane doubles the warps but, measured on
+// the 130m workload, costs 66 % more instructions per state and runs 24 %
+// slower: the transposing reduction spans eight lanes and every B/C load
+// serves half as many states.)
+template <int N, typename T, bool HZ, int MODE, bool ST, bool WR>
+cudaError_t launch_one(const Maps &m, const M1Params &p, int nseg, cudaStream_t s) {
+  return launch_spl<N, 4, T, HZ, MODE, ST, WR>(m, p, nseg, s);
+}
+
 template <int N, typename T, bool HZ>
-cudaError_t launch_v(const M1Params &p, cudaStream_t s) {
-  if (p.states) return launch_tma<N, T, 16, HZ, 0, 4, true>(p, s);
-  // a state written at one token: the default lane split, with the write
-  if (p.state_write) return launch_tma<N, T, 16, HZ, 0, 2, false, true, 1, true>(p, s);
-  // variant = 4 * (packed) + 2 * (two groups per iteration) + (2 states per lane)
-  const bool ok32 = p.G == 1 || (p.C / p.G) % 32 == 0;
-  switch (p.variant) {
-    case 0: return launch_tma<N, T, 16, HZ, 0, 4, false, false, 1>(p, s);
-    case 1: return launch_tma<N, T, 16, HZ, 0, 2, false, false, 1>(p, s);
-    case 2: return launch_tma<N, T, 16, HZ, 0, 4, false, false, 2>(p, s);
-    case 3: return launch_tma<N, T, 16, HZ, 0, 2, false, false, 2>(p, s);
-    case 4: return launch_tma<N, T, 16, HZ, 0, 4, false, true, 1>(p, s);
-    case 5: return launch_tma<N, T, 16, HZ, 0, 2, false, true, 1>(p, s);
-    case 6: return launch_tma<N, T, 16, HZ, 0, 4, false, true, 2>(p, s);
-    case 7: return launch_tma<N, T, 16, HZ, 0, 2, false, true, 2>(p, s);
-    case 8: return launch_tma<N, T, 16, HZ, 1, 4, false, true, 1>(p, s);
-    // 9..12: 32-channel tiles (a tile must not straddle two B/C groups,
-    // else the default form runs)
-    case 9:
-      if (ok32) return launch_tma<N, T, 32, HZ, 0, 4, false, true, 1>(p, s);
-      break;
-    case 10:
-      if (ok32) return launch_tma<N, T, 32, HZ, 0, 8, false, true, 1>(p, s);
-      break;
-    case 11:
-      if (ok32) return launch_tma<N, T, 32, HZ, 0, 2, false, true, 1>(p, s);
-      break;
-    case 12:
-      if (ok32) return launch_tma<N, T, 32, HZ, 1, 4, false, true, 1>(p, s);
-      break;
-    case 13: return launch_tma<N, T, 16, HZ, 1, 2, false, true, 1>(p, s);
-    case 14: return launch_tma<N, T, 16, HZ, 1, 2, false, true, 2>(p, s);
+cudaError_t launch_n(const M1Params &p, cudaStream_t s) {
+  Maps m;
+  if (!make_maps<N, T>(p, m)) return cudaErrorInvalidValue;
+  if (p.states) return launch_one<N, T, HZ, kModeFull, true, false>(m, p, 1, s);
+  if (p.state_write) return launch_one<N, T, HZ, kModeFull, false, true>(m, p, 1, s);
+  if (p.nseg <= 1) return launch_one<N, T, HZ, kModeFull, false, false>(m, p, 1, s);
+  cudaError_t e = launch_one<N, T, HZ, kModeStateOnly, false, false>(m, p, p.nseg - 1, s);
+  if (e != cudaSuccess) return e;
+  const int64_t items = p.batch * p.C * p.N;
+  const int sp = p.nseg - 1 <= 2 ? 2 : p.nseg - 1 <= 4 ? 4 : p.nseg - 1 <= 8 ? 8 : p.nseg - 1 <= 16 ? 16 : 32;
+  const unsigned blocks = (unsigned)((items * sp + 255) / 256);
+  switch (sp) {
+    case 2: m1_seg_carry_kernel<2><<<blocks, 256, 0, s>>>(p); break;
+    case 4: m1_seg_carry_kernel<4><<<blocks, 256, 0, s>>>(p); break;
+    case 8: m1_seg_carry_kernel<8><<<blocks, 256, 0, s>>>(p); break;
+    case 16: m1_seg_carry_kernel<16><<<blocks, 256, 0, s>>>(p); break;
+    default: m1_seg_carry_kernel<32><<<blocks, 256, 0, s>>>(p); break;
   }
-  return launch_tma<N, T, 16, HZ, 0, 2, false, true, 1>(p, s);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_one<N, T, HZ, kModeFull, false, false>(m, p, p.nseg, s);
 }
 
 template <typename T>
-cudaError_t launch_tma_t(const M1Params &p, cudaStream_t s) {
+cudaError_t launch_t(const M1Params &p, cudaStream_t s) {
   const bool hz = p.z != nullptr;
   switch (p.N) {
-    case 8: return hz ? launch_tma<8, T, 16, true, 0, 4, false>(p, s)
-                      : launch_tma<8, T, 16, false, 0, 4, false>(p, s);
-    case 16: return hz ? launch_v<16, T, true>(p, s) : launch_v<16, T, false>(p, s);
-    case 32: return hz ? launch_tma<32, T, 16, true, 0, 4, false>(p, s)
-                       : launch_tma<32, T, 16, false, 0, 4, false>(p, s);
+    case 4:
+      if constexpr (sizeof(T) == 4) return hz ? launch_n<4, T, true>(p, s) : launch_n<4, T, false>(p, s);
+      break;
+    case 8: return hz ? launch_n<8, T, true>(p, s) : launch_n<8, T, false>(p, s);
+    case 16: return hz ? launch_n<16, T, true>(p, s) : launch_n<16, T, false>(p, s);
+    case 32: return hz ? launch_n<32, T, true>(p, s) : launch_n<32, T, false>(p, s);
   }
   return cudaErrorNotSupported;
 }
 
 }  // namespace
 
-// The pipelined kernel needs 16-byte rows for TMA (a 16-channel tile and the
-// B/C rows), a channel tile inside one group, and N in {8, 16, 32}; per-token
-// states only with N = 16.
+// The pipelined kernel needs 16-byte rows for TMA (x/dt/z rows of the tensor
+// and B/C rows of one group), 32-channel tiles inside one B/C group, and
+// N in {8, 16, 32} (N = 4 for float32 I/O).
 bool m1_scan_tma_supported(const M1Params &p) {
-  if (p.states && p.N != 16) return false;
   const int64_t es = p.io == 1 ? 2 : 4;
-  if (p.N != 8 && p.N != 16 && p.N != 32) return false;
+  const bool n_ok = p.N == 8 || p.N == 16 || p.N == 32 || (p.N == 4 && es == 4);
+  if (!n_ok) return false;
   if ((p.N * es) % 16 || (p.C * es) % 16 || (p.G * p.N * es) % 16) return false;
-  if (p.G > 1 && (p.C / p.G) % 16) return false;
+  if (p.G > 1 && (p.C / p.G) % kCT) return false;
   if (p.L >= (1ll << 31) || p.C >= (1ll << 31) || p.batch > 65535) return false;
   return true;
 }
 
+// How many sequence segments a call is cut into.  Cost model, in units of
+// one warp's whole-sequence time when it has its SM sub-partition to itself:
+// a sub-partition runs up to kFull warps at no loss of per-warp speed (the
+// recurrence is latency-bound below that), so k warps take max(1, k / kFull)
+// units per unit of work.  Cutting into S segments costs a state-only pass
+// over the first S - 1 segments (about 0.85 of a full pass per token, no
+// readout), a full pass over S segments of 1/S of the sequence each, and two
+// more launches.  Calls with per-token states or a state write are not cut.
+M1Split m1_scan_split(int64_t batch, int64_t C, int64_t L, int64_t N, int sms) {
+  M1Split r;
+  r.nseg = 1;
+  r.seg_len = L;
+  if (batch <= 0 || L <= 0 || sms <= 0) return r;
+  const double kFull = 3.0, kStateOnly = 0.85;
+  const double slots = 4.0 * sms;  // sub-partitions
+  const double w0 = (double)batch * ((C + kCT - 1) / kCT) * (kCT * (N / 4) / 32);  // warps
+  const double work_ns = (double)L * 50.0;  // one warp alone, per token (measured order)
+  auto cost = [&](double warps, double frac) {
+    const double k = std::ceil(warps / slots);
+    return frac * std::max(1.0, k / kFull);
+  };
+  double best = cost(w0, 1.0);
+  for (int S = 2; S <= 32; S *= 2) {
+    const int64_t len = ((L + S - 1) / S + kTL - 1) / kTL * kTL;
+    if (len < 4 * kTL) break;
+    const int segs = (int)((L + len - 1) / len);
+    if (segs < 2) break;
+    const double t = cost(w0 * (segs - 1), kStateOnly / segs) + cost(w0 * segs, 1.0 / segs) +
+                     2 * 4000.0 / work_ns;  // two more launches of a few microseconds
+    if (t < 0.9 * best) {
+      best = t;
+      r.nseg = segs;
+      r.seg_len = len;
+    }
+  }
+  return r;
+}
+
+size_t m1_scan_split_bytes(const M1Split &r, int64_t batch, int64_t C, int64_t N) {
+  if (r.nseg <= 1) return 0;
+  const size_t bcn = (size_t)(batch * C * N) * sizeof(float);
+  const size_t bc = (size_t)(batch * C) * sizeof(float);
+  const auto a16 = [](size_t v) { return (v + 255) & ~(size_t)255; };
+  return a16(bcn * (r.nseg - 1)) + a16(bc * (r.nseg - 1)) + a16(bcn * r.nseg);
+}
+
+void m1_scan_split_carve(const M1Split &r, int64_t batch, int64_t C, int64_t N, void *ws,
+                         M1Params &p) {
+  p.nseg = r.nseg;
+  p.seg_len = r.seg_len;
+  if (r.nseg <= 1) return;
+  const size_t bcn = (size_t)(batch * C * N) * sizeof(float);
+  const size_t bc = (size_t)(batch * C) * sizeof(float);
+  const auto a16 = [](size_t v) { return (v + 255) & ~(size_t)255; };
+  char *w = static_cast<char *>(ws);
+  p.seg_end = reinterpret_cast<float *>(w);
+  w += a16(bcn * (r.nseg - 1));
+  p.seg_dsum = reinterpret_cast<float *>(w);
+  w += a16(bc * (r.nseg - 1));
+  p.seg_ent = reinterpret_cast<float *>(w);
+}
+
 cudaError_t launch_m1_scan_tma(const M1Params &p, cudaStream_t s) {
-  return p.io == 1 ? launch_tma_t<__nv_bfloat16>(p, s) : launch_tma_t<float>(p, s);
+  return p.io == 1 ? launch_t<__nv_bfloat16>(p, s) : launch_t<float>(p, s);
 }
 
 }  // namespace ssm

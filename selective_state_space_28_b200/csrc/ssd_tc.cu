@@ -86,7 +86,8 @@ struct __align__(1024) SsdSmem {
   uint8_t X[2][kQ * 128];     // [stage]
   uint8_t Xw[kQ * 128];       // w o x of the tile whose Sc is next
   uint8_t Hb[2][kN * 128];    // bf16 copy of the carried state, rows n
-  float cumw[8][kQ];          // per mask-group warp: cumulative log2-decay,
+  float cumw[8][kQ];          // per mask-group warp: cumulative log2-decay
+  float cuml[8][kQ];          //   (a compensated sum: cumw + cuml),
   float ddw[8][kQ];           //   step d_j,
   float vdw[8][kQ];           //   column factor of the off-diagonal mask
   float a[4];                 // exp(cum_last) per tile, ring of four
@@ -130,6 +131,30 @@ struct SsdTcParams {
   float *seg_decay;      // [ntail][nseg]: product of the segment's tile decays
   const float *seg_hin;  // [ntail][nseg][N][P]: the state entering each segment
 };
+
+// Compensated sums.  The mask needs exp(cum_i - cum_j) for tokens i, j of a
+// tile, and the running sum cum of the log-decays d * A can be large (a fast
+// decay over many tokens) beside the step of one token (a near-zero step):
+// the difference of two rounded float sums would lose that step entirely
+// (the "Mamba-2" page's extreme A_h with a tiny step).  Each prefix sum is
+// therefore kept as an unevaluated pair hi + lo (Knuth's TwoSum), and a
+// difference is (hi_i - hi_j) + (lo_i - lo_j): the first term is exact when
+// the two sums are close (Sterbenz), the second restores what rounding cut.
+struct ff {
+  float hi, lo;
+};
+__device__ __forceinline__ ff two_sum(float a, float b) {
+  const float s = a + b;
+  const float bb = s - a;
+  return {s, (a - (s - bb)) + (b - bb)};
+}
+__device__ __forceinline__ ff ff_add(ff a, ff b) {
+  ff r = two_sum(a.hi, b.hi);
+  const float lo = r.lo + (a.lo + b.lo);
+  const float hi = r.hi + lo;  // renormalise (|lo| is below an ulp of r.hi)
+  return {hi, lo - (hi - r.hi)};
+}
+__device__ __forceinline__ float ff_diff(ff a, ff b) { return (a.hi - b.hi) + (a.lo - b.lo); }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -414,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float bias = p.dt_bias ? p.dt_bias[hd] : 0.f;
     const float Dh = p.D ? p.D[hd] : 0.f;
     const bool softplus_on = p.flags & 1u;
-    float *cumw = s.cumw[mg], *ddw = s.ddw[mg], *vdw = s.vdw[mg];
+    float *cumw = s.cumw[mg], *cuml = s.cuml[mg], *ddw = s.ddw[mg], *vdw = s.vdw[mg];
     // lane l handles tokens 4l .. 4l+3 of the tile in the prologue; their dt
     // is fetched a tile ahead and kept as raw bfloat16 bits until used
     const uint16_t *dtb = reinterpret_cast<const uint16_t *>(p.dt);
@@ -433,8 +458,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int valid = (int)(L - t0 < kQ ? L - t0 : kQ);
       // step, log2-decay and inclusive sums over the whole tile (needs only
       // dt, so it runs while the tile's TMA is in flight)
-      float d4[4], p4[4];
-      float run = 0.f;
+      float d4[4];
+      ff p4[4];
+      ff run = {0.f, 0.f};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float d = 0.f;
@@ -443,31 +469,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (softplus_on) d = softplus_sfu(d);
         }
         d4[q] = d;
-        run += d * A2;
+        run = ff_add(run, ff{d * A2, 0.f});
         p4[q] = run;
       }
-      float incl = run;
+      ff incl = run;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
-        const float v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
+        const ff v = {__shfl_up_sync(0xffffffffu, incl.hi, off),
+                      __shfl_up_sync(0xffffffffu, incl.lo, off)};
+        if (lane >= off) incl = ff_add(v, incl);
       }
-      const float total = __shfl_sync(0xffffffffu, incl, 31);
-      const float excl = incl - run;
+      const ff total = {__shfl_sync(0xffffffffu, incl.hi, 31), __shfl_sync(0xffffffffu, incl.lo, 31)};
+      ff excl = {__shfl_up_sync(0xffffffffu, incl.hi, 1), __shfl_up_sync(0xffffffffu, incl.lo, 1)};
+      if (lane == 0) excl = {0.f, 0.f};
       // cum at the last token of each 32-token block (lanes 7, 15, 23, 31)
-      const float blk_end = __shfl_sync(0xffffffffu, incl, (lane & ~7) | 7);
+      const int be = (lane & ~7) | 7;
+      const ff blk_end = {__shfl_sync(0xffffffffu, incl.hi, be), __shfl_sync(0xffffffffu, incl.lo, be)};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float cq = excl + p4[q];
-        cumw[4 * lane + q] = cq;
+        const ff cq = ff_add(excl, p4[q]);
+        cumw[4 * lane + q] = cq.hi;
+        cuml[4 * lane + q] = cq.lo;
         ddw[4 * lane + q] = d4[q];
-        vdw[4 * lane + q] = ex2(blk_end - cq) * d4[q];
+        vdw[4 * lane + q] = ex2(ff_diff(blk_end, cq)) * d4[q];
       }
-      if (mg == 0 && lane == 0) s.a[c & 3] = ex2(total);
+      if (mg == 0 && lane == 0) s.a[c & 3] = ex2(total.hi + total.lo);
       __syncwarp();
-      const float cs = cumw[i];
-      const float e_i = ex2(cs);
-      const float w_i = ex2(total - cs) * ddw[i];
+      const ff cs = {cumw[i], cuml[i]};
+      const float e_i = ex2(cs.hi + cs.lo);
+      const float w_i = ex2(ff_diff(total, cs)) * ddw[i];
       // w o x (this warp's rows, half the columns), the B operand of Sc(c):
       // x of tile c has landed and Sc(c-1) is done with the buffer
       if (!waitw(s, &s.full[k], (c >> 1) & 1, p.status, 8)) break;
@@ -512,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (J < mw) {
           // below the diagonal: S_ij * exp2(cum_i - cum_r) * vd_j, r the
           // block's last token; both factors <= 1
-          const float u = ex2(cs - cumw[32 * J + 31]);
+          const float u = ex2(ff_diff(cs, ff{cumw[32 * J + 31], cuml[32 * J + 31]}));
           const float4 *vd4 = reinterpret_cast<const float4 *>(vdw + j0);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -529,17 +559,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           // diagonal block: S_ij * exp2(cum_i - cum_j) * d_j for j <= i, + D at j = i
           const float4 *c4 = reinterpret_cast<const float4 *>(cumw + j0);
+          const float4 *l4 = reinterpret_cast<const float4 *>(cuml + j0);
           const float4 *d4p = reinterpret_cast<const float4 *>(ddw + j0);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float4 cj = c4[q], dj = d4p[q];
-            const float cjs[4] = {cj.x, cj.y, cj.z, cj.w}, djs[4] = {dj.x, dj.y, dj.z, dj.w};
+            const float4 cj = c4[q], lj = l4[q], dj = d4p[q];
+            const float cjs[4] = {cj.x, cj.y, cj.z, cj.w}, ljs[4] = {lj.x, lj.y, lj.z, lj.w},
+                        djs[4] = {dj.x, dj.y, dj.z, dj.w};
             float f[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int j = j0 + 4 * q + e;
               const float sv = __uint_as_float(r[4 * q + e]);
-              f[e] = (j <= i) ? sv * (ex2(cs - cjs[e]) * djs[e]) + (j == i ? Dh : 0.f) : 0.f;
+              const float dl = ff_diff(cs, ff{cjs[e], ljs[e]});
+              f[e] = (j <= i) ? sv * (ex2(dl) * djs[e]) + (j == i ? Dh : 0.f) : 0.f;
             }
             m[2 * q] = pack_bf16x2(f[0], f[1]);
             m[2 * q + 1] = pack_bf16x2(f[2], f[3]);

@@ -21,29 +21,6 @@ bool all_aligned(Ps... ps) {
   return true;
 }
 
-// Variant of the pipelined Mamba-1 kernel (0..14, see scan_m1_tma.cu);
-// SSM_M1_VARIANT overrides the default for tuning.
-int m1_variant() {
-  static int v = -1;
-  if (v < 0) {
-    const char *e = getenv("SSM_M1_VARIANT");
-    v = e ? atoi(e) : 5;
-    if (v < 0 || v > 14) v = 5;
-  }
-  return v;
-}
-
-// The TMA-pipelined Mamba-1 kernel is used wherever the shape allows;
-// SSM_M1_PIPELINED=0 forces the generic kernel (for comparisons).
-int m1_pipelined() {
-  static int v = -1;
-  if (v < 0) {
-    const char *e = getenv("SSM_M1_PIPELINED");
-    v = (e && e[0] == '0') ? 0 : 1;
-  }
-  return v;
-}
-
 }  // namespace
 
 namespace ssm {
@@ -75,8 +52,39 @@ ssm_status_t pass_state(const float *h0, float *h_last, size_t bytes, cudaStream
   return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
+// The Mamba-1 workspace: a status word (256 bytes), the dt-norm factors
+// (batch * seqlen floats, with SSM_RMSNORM_DT), then the sequence segments'
+// states when the call is cut.  `cut` false keeps the whole sequence in one
+// pass (the allocation-free entry point).
+constexpr size_t kStatusBytes = 256;
+struct M1Layout {
+  size_t rstd_off = 0, seg_off = 0, total = 0;
+  ssm::M1Split split;
+};
+size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
+bool m1_cut_allowed(const ssm_scan_args_t *a) { return !a->states; }
+M1Layout m1_layout(const ssm_scan_args_t *a, int sms, bool cut = true) {
+  M1Layout l;
+  l.rstd_off = kStatusBytes;
+  const size_t rstd = (a->flags & SSM_RMSNORM_DT) ? (size_t)(a->batch * a->seqlen) * sizeof(float) : 0;
+  l.seg_off = l.rstd_off + round256(rstd);
+  ssm::M1Params probe;
+  probe.batch = a->batch;
+  probe.L = a->seqlen;
+  probe.C = a->channels;
+  probe.N = a->state;
+  probe.G = a->groups;
+  probe.io = a->io;
+  if (cut && m1_cut_allowed(a) && a->batch > 0 && a->seqlen > 0 &&
+      ssm::m1_scan_tma_supported(probe))
+    l.split = ssm::m1_scan_split(a->batch, a->channels, a->seqlen, a->state, sms);
+  l.total = l.seg_off + ssm::m1_scan_split_bytes(l.split, a->batch, a->channels, a->state);
+  return l;
+}
+
 // shapes_only: the workspace query validates sizes and flags, not pointers.
-ssm_status_t check_scan(const ssm_scan_args_t *a, size_t *ws, bool shapes_only = false) {
+ssm_status_t check_scan(const ssm_scan_args_t *a, size_t *ws, bool shapes_only = false,
+                        bool size_it = true) {
   if (!a) return SSM_ERR_NULL;
   if (a->io != SSM_F32 && a->io != SSM_BF16) return SSM_ERR_DTYPE;
   if (a->batch < 0 || a->seqlen < 0 || a->channels <= 0 || a->state <= 0 ||
@@ -95,7 +103,7 @@ ssm_status_t check_scan(const ssm_scan_args_t *a, size_t *ws, bool shapes_only =
     return SSM_ERR_ALIGN;
   if (!ssm::m1_scan_supported(a->state, a->channels, a->groups) || a->batch > 65535)
     return SSM_ERR_UNSUPPORTED;
-  *ws = (a->flags & SSM_RMSNORM_DT) ? (size_t)(a->batch * a->seqlen) * sizeof(float) : 0;
+  if (size_it) *ws = m1_layout(a, ssm::device_sm_count()).total;
   return SSM_OK;
 }
 
@@ -154,6 +162,60 @@ ssm_status_t check_ssd(const ssd_scan_args_t *a, size_t *ws, bool shapes_only = 
 
 }  // namespace
 
+namespace ssm {
+
+ssm_status_t scan_validate(const ssm_scan_args_t *a) {
+  size_t ws = 0;
+  return check_scan(a, &ws, false, false);
+}
+
+ssm_status_t scan_run(const ssm_scan_args_t *a, int64_t t_write, const float *state_write,
+                      void *stream, bool allow_cut) {
+  size_t ws = 0;
+  ssm_status_t st = check_scan(a, &ws);
+  if (st != SSM_OK) return st;
+  if (a->batch == 0) return SSM_OK;  // nothing to do, nothing launched
+  const M1Layout lay = m1_layout(a, device_sm_count(), allow_cut && t_write < 0);
+  if (!a->workspace || a->workspace_bytes < lay.total) return SSM_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int *status = static_cast<int *>(a->workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return SSM_ERR_CUDA;
+  if (a->seqlen == 0)
+    return pass_state(a->h0, a->h_last,
+                      (size_t)(a->batch * a->channels * a->state) * sizeof(float), s);
+  M1Params p;
+  p.batch = a->batch;
+  p.L = a->seqlen;
+  p.C = a->channels;
+  p.N = a->state;
+  p.G = a->groups;
+  p.flags = a->flags;
+  p.eps = a->rms_eps;
+  p.io = a->io;
+  p.x = a->x;
+  p.dt = a->dt;
+  p.z = a->z;
+  p.B = a->B;
+  p.Cm = a->C;
+  p.A = a->A;
+  p.D = a->D;
+  p.dt_bias = a->dt_bias;
+  p.h0 = a->h0;
+  p.y = a->y;
+  p.h_last = a->h_last;
+  p.states = a->states;
+  char *w = static_cast<char *>(a->workspace);
+  p.rstd = (a->flags & SSM_RMSNORM_DT) ? reinterpret_cast<float *>(w + lay.rstd_off) : nullptr;
+  p.status = status;
+  p.t_write = t_write;
+  p.state_write = state_write;
+  m1_scan_split_carve(lay.split, a->batch, a->channels, a->state, w + lay.seg_off, p);
+  if (p.nseg <= 1) p.seg_len = a->seqlen;
+  return from_cuda(launch_m1_scan(p, s));
+}
+
+}  // namespace ssm
+
 extern "C" {
 
 int ssm_abi_version(void) { return SSM_ABI_VERSION; }
@@ -182,84 +244,29 @@ ssm_status_t ssm_scan_workspace(const ssm_scan_args_t *a, size_t *bytes) {
 }
 
 ssm_status_t ssm_scan_fwd(const ssm_scan_args_t *a, void *stream) {
-  size_t ws = 0;
-  ssm_status_t st = check_scan(a, &ws);
-  if (st != SSM_OK) return st;
-  if (ws && (!a->workspace || a->workspace_bytes < ws)) return SSM_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (a->batch == 0) return SSM_OK;
-  if (a->seqlen == 0)
-    return pass_state(a->h0, a->h_last,
-                      (size_t)(a->batch * a->channels * a->state) * sizeof(float), s);
-  ssm::M1Params p;
-  p.batch = a->batch;
-  p.L = a->seqlen;
-  p.C = a->channels;
-  p.N = a->state;
-  p.G = a->groups;
-  p.flags = a->flags;
-  p.eps = a->rms_eps;
-  p.io = a->io;
-  p.x = a->x;
-  p.dt = a->dt;
-  p.z = a->z;
-  p.B = a->B;
-  p.Cm = a->C;
-  p.A = a->A;
-  p.D = a->D;
-  p.dt_bias = a->dt_bias;
-  p.h0 = a->h0;
-  p.y = a->y;
-  p.h_last = a->h_last;
-  p.states = a->states;
-  p.rstd = (a->flags & SSM_RMSNORM_DT) ? static_cast<float *>(a->workspace) : nullptr;
-  p.pipelined = m1_pipelined();
-  p.variant = m1_variant();
-  p.status = nullptr;
-  p.t_write = -1;
-  p.state_write = nullptr;
-  return from_cuda(ssm::launch_m1_scan(p, s));
+  return ssm::scan_run(a, -1, nullptr, stream, true);
 }
 
 ssm_status_t ssm_scan_fwd_write(const ssm_scan_args_t *a, int64_t t_write,
                                 const float *state_write, void *stream) {
-  size_t ws = 0;
-  ssm_status_t st = check_scan(a, &ws);
-  if (st != SSM_OK) return st;
-  if (a->batch > 0 && !state_write) return SSM_ERR_NULL;
+  if (a && a->batch > 0 && !state_write) return SSM_ERR_NULL;
   if (!all_aligned(state_write)) return SSM_ERR_ALIGN;
-  if (t_write < 0 || t_write >= a->seqlen) return SSM_ERR_SHAPE;
-  if (ws && (!a->workspace || a->workspace_bytes < ws)) return SSM_ERR_WORKSPACE;
+  if (a && (t_write < 0 || t_write >= a->seqlen)) return SSM_ERR_SHAPE;
+  return ssm::scan_run(a, t_write, state_write, stream, true);
+}
+
+ssm_status_t ssm_workspace_status(const void *workspace, void *stream) {
+  if (!workspace) {
+    void *scratch = nullptr;
+    if (ssm::static_scratch_address(&scratch) != cudaSuccess) return SSM_ERR_CUDA;
+    workspace = scratch;
+  }
+  int word = 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (a->batch == 0) return SSM_OK;
-  ssm::M1Params p;
-  p.batch = a->batch;
-  p.L = a->seqlen;
-  p.C = a->channels;
-  p.N = a->state;
-  p.G = a->groups;
-  p.flags = a->flags;
-  p.eps = a->rms_eps;
-  p.io = a->io;
-  p.x = a->x;
-  p.dt = a->dt;
-  p.z = a->z;
-  p.B = a->B;
-  p.Cm = a->C;
-  p.A = a->A;
-  p.D = a->D;
-  p.dt_bias = a->dt_bias;
-  p.h0 = a->h0;
-  p.y = a->y;
-  p.h_last = a->h_last;
-  p.states = a->states;
-  p.rstd = (a->flags & SSM_RMSNORM_DT) ? static_cast<float *>(a->workspace) : nullptr;
-  p.pipelined = m1_pipelined();  // the pipelined kernel carries it where it can (N = 16)
-  p.variant = m1_variant();
-  p.status = nullptr;
-  p.t_write = t_write;
-  p.state_write = state_write;
-  return from_cuda(ssm::launch_m1_scan(p, s));
+  if (cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return SSM_ERR_CUDA;
+  return word ? SSM_ERR_TIMEOUT : SSM_OK;
 }
 
 ssm_status_t ssd_chunk_scan_workspace(const ssd_scan_args_t *a, size_t *bytes) {
@@ -274,9 +281,9 @@ ssm_status_t ssd_chunk_scan_fwd(const ssd_scan_args_t *a, void *stream) {
   size_t ws = 0;
   ssm_status_t st = check_ssd(a, &ws);
   if (st != SSM_OK) return st;
+  if (a->batch == 0) return SSM_OK;  // nothing to do, nothing launched
   if (ws && (!a->workspace || a->workspace_bytes < ws)) return SSM_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (a->batch == 0) return SSM_OK;
   if (a->seqlen == 0)
     return pass_state(a->h0, a->h_last,
                       (size_t)(a->batch * a->heads * a->state * a->head_dim) * sizeof(float),

@@ -71,14 +71,37 @@ def _io_of(x):
     return _IO[x.dtype]
 
 
+_CHECK_ALL = False
+
+
+def check_every_call(on=True):
+    """Make every scan call synchronise and check its status word (as if
+    check=True were passed), e.g. for a test session."""
+    global _CHECK_ALL
+    _CHECK_ALL = bool(on)
+
+
+def _check_status(ws, stream, where):
+    """Synchronise ``stream`` and raise SsmError(SSM_ERR_TIMEOUT) if the call
+    that used workspace ``ws`` recorded an expired device wait."""
+    L.check(L.lib().ssm_workspace_status(ws.data_ptr(), stream), where)
+
+
+def _workspace(nbytes, workspace, device):
+    if workspace is None or workspace.numel() * workspace.element_size() < nbytes:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return workspace
+
+
 def ssm_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
                  flags=SOFTPLUS, rms_eps=1e-6, want_states=False, y=None, h_last=None,
-                 stream=None, _write=None):
+                 workspace=None, check=False, stream=None, _write=None):
     """Mamba-1 selective scan (include/ssm.h, ssm_scan_fwd).
 
     x, dt, z: [b, L, C]; B, C: [b, L, G, N]; A: [C, N] f32; D, dt_bias: [C] f32;
     h0: [b, C, N] f32.  Returns (y [b, L, C], h_last [b, C, N] f32,
-    states [b, L, C, N] f32 or None)."""
+    states [b, L, C, N] f32 or None).  With check=True (always for host
+    tensors) the stream is synchronised and an expired device wait raises."""
     sg = _Staging([x, dt, A, B, C, D, z, dt_bias, h0])
     x, dt, A, B, C, D, z, dt_bias, h0 = map(sg.dev, (x, dt, A, B, C, D, z, dt_bias, h0))
     if _write is not None:
@@ -98,21 +121,22 @@ def ssm_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
     lib = L.lib()
     nbytes = ctypes.c_size_t(0)
     L.check(lib.ssm_scan_workspace(ctypes.byref(a), ctypes.byref(nbytes)), "ssm_scan_workspace")
-    ws = None
-    if nbytes.value:
-        ws = torch.empty(nbytes.value, dtype=torch.uint8, device=x.device)
-        a.workspace, a.workspace_bytes = ws.data_ptr(), nbytes.value
+    ws = _workspace(nbytes.value, workspace, x.device)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), nbytes.value
+    st = _stream(stream, x.device)
     if _write is None:
-        L.check(lib.ssm_scan_fwd(ctypes.byref(a), _stream(stream, x.device)), "ssm_scan_fwd")
+        L.check(lib.ssm_scan_fwd(ctypes.byref(a), st), "ssm_scan_fwd")
     else:
-        L.check(lib.ssm_scan_fwd_write(ctypes.byref(a), int(_write[0]), _ptr(_write[1]),
-                                       _stream(stream, x.device)), "ssm_scan_fwd_write")
+        L.check(lib.ssm_scan_fwd_write(ctypes.byref(a), int(_write[0]), _ptr(_write[1]), st),
+                "ssm_scan_fwd_write")
+    if check or sg.host or _CHECK_ALL:
+        _check_status(ws, st, "ssm_scan_fwd")
     return sg.back((y, h_last, states))
 
 
 def ssm_scan_fwd_write(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, t, state,
                        flags=SOFTPLUS, rms_eps=1e-6, want_states=False, y=None, h_last=None,
-                       stream=None):
+                       check=False, stream=None):
     """Mamba-1 scan with the state written at token t (include/ssm.h,
     ssm_scan_fwd_write): h_t is replaced by ``state`` [b, C, N] float32, y_t
     reads it and tokens t+1.. continue from it.  Arguments and results as
@@ -120,8 +144,8 @@ def ssm_scan_fwd_write(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
     if state.dtype != torch.float32:
         raise TypeError("state must be float32")
     return ssm_scan_fwd(x, dt, A, B, C, D, z, dt_bias, h0, flags=flags, rms_eps=rms_eps,
-                        want_states=want_states, y=y, h_last=h_last, stream=stream,
-                        _write=(t, state))
+                        want_states=want_states, y=y, h_last=h_last, check=check,
+                        stream=stream, _write=(t, state))
 
 
 def ssd_workspace_bytes(**shape):
@@ -134,11 +158,13 @@ def ssd_workspace_bytes(**shape):
 
 def ssd_chunk_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
                        chunk=256, flags=SOFTPLUS, want_states=False, y=None, h_last=None,
-                       workspace=None, stream=None):
+                       workspace=None, check=False, stream=None):
     """Mamba-2 SSD scan (include/ssm.h, ssd_chunk_scan_fwd).
 
     x, z: [b, L, H, P]; dt: [b, L, H]; B, C: [b, L, G, N]; A, D, dt_bias: [H] f32;
-    h0: [b, H, N, P] f32.  Returns (y, h_last [b, H, N, P], states or None)."""
+    h0: [b, H, N, P] f32.  Returns (y, h_last [b, H, N, P], states or None).
+    With check=True (always for host tensors) the stream is synchronised and
+    an expired device wait raises."""
     sg = _Staging([x, dt, A, B, C, D, z, dt_bias, h0])
     x, dt, A, B, C, D, z, dt_bias, h0 = map(sg.dev, (x, dt, A, B, C, D, z, dt_bias, h0))
     b, Lq, H, P = x.shape
@@ -158,11 +184,12 @@ def ssd_chunk_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
     L.check(lib.ssd_chunk_scan_workspace(ctypes.byref(a), ctypes.byref(nbytes)),
             "ssd_chunk_scan_workspace")
     if nbytes.value:
-        if workspace is None or workspace.numel() * workspace.element_size() < nbytes.value:
-            workspace = torch.empty(nbytes.value, dtype=torch.uint8, device=x.device)
+        workspace = _workspace(nbytes.value, workspace, x.device)
         a.workspace, a.workspace_bytes = workspace.data_ptr(), nbytes.value
-    L.check(lib.ssd_chunk_scan_fwd(ctypes.byref(a), _stream(stream, x.device)),
-            "ssd_chunk_scan_fwd")
+    st = _stream(stream, x.device)
+    L.check(lib.ssd_chunk_scan_fwd(ctypes.byref(a), st), "ssd_chunk_scan_fwd")
+    if nbytes.value and (check or sg.host or _CHECK_ALL):
+        _check_status(workspace, st, "ssd_chunk_scan_fwd")
     return sg.back((y, h_last, states))
 
 

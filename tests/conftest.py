@@ -18,4 +18,7 @@ def cuda_ok():
     import torch
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
+    # every scan call in the GPU tests synchronises and checks its status word
+    from selective_state_space_28_b200 import ops
+    ops.check_every_call(True)
     return True

@@ -26,7 +26,7 @@ def test_exports_every_declared_symbol(lib):
             "ssd_chunk_scan_workspace", "ssm_scan_step", "ssm_status_string",
             "ssm_abi_version", "ssm_conv1d_fwd", "ssm_scan_fwd_static",
             "ssm_gated_rmsnorm_fwd", "ssm_scan_fwd_write", "ssd_attention_fwd",
-            "ssd_attention_workspace"} <= set(names)
+            "ssd_attention_workspace", "ssm_workspace_status"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], check=True,
                          capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
@@ -44,7 +44,7 @@ def test_no_runtime_symbols_leak(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.ssm_abi_version() == 1
+    assert lib.ssm_abi_version() == 2
     for s in range(9):
         assert lib.ssm_status_string(s)
     assert lib.ssm_status_string(99) == b"unknown status"
@@ -83,13 +83,61 @@ def test_scan_null_args(lib):
 
 
 def test_scan_workspace_sizes(lib):
+    """256 bytes of status word, then the dt-norm factors (rounded up to 256
+    bytes) with SSM_RMSNORM_DT; a workspace one byte short is refused before
+    anything is launched."""
     n = ctypes.c_size_t(123)
     assert lib.ssm_scan_workspace(ctypes.byref(_scan()), ctypes.byref(n)) == OK
-    assert n.value == 0
+    assert n.value == 256
     assert lib.ssm_scan_workspace(ctypes.byref(_scan(flags=5)), ctypes.byref(n)) == OK
-    assert n.value == 2 * 8 * 4
-    a = _scan(flags=5, workspace=P, workspace_bytes=63)
-    assert _call_scan(lib, a) == WS
+    assert n.value == 256 + 256  # 2 x 8 factors, rounded up
+    assert _call_scan(lib, _scan(flags=5, workspace=P, workspace_bytes=511)) == WS
+    assert _call_scan(lib, _scan(workspace=None, workspace_bytes=0)) == WS
+
+
+def _scan_ws(lib, **kw):
+    n = ctypes.c_size_t(0)
+    assert lib.ssm_scan_workspace(ctypes.byref(_scan(**kw)), ctypes.byref(n)) == OK
+    return n.value
+
+
+def test_scan_sequence_cut_rule(lib):
+    """The pipelined Mamba-1 kernel cuts the sequence into segments only when
+    batch x channels leaves the SMs short of warps, and then asks for the
+    segments' states in the workspace (sizes for a 148-SM device, which is
+    what the query assumes without one)."""
+    big = dict(channels=1536, state=16, seqlen=2048)
+    assert _scan_ws(lib, batch=8, **big) == 256                  # 1536 warps: whole sequence
+    b1 = _scan_ws(lib, batch=1, **big)                           # 192-384 warps: cut
+    bcn, bc = 1536 * 16 * 4, 1536 * 4
+    # S segments: S - 1 end states, S - 1 step sums, S entering states
+    cuts = [S for S in range(2, 33) if b1 == 256 + (S - 1) * bcn + (S - 1) * bc + S * bcn]
+    assert len(cuts) == 1 and 2048 // cuts[0] >= 128, b1
+    assert _scan_ws(lib, batch=1, channels=1536, state=16, seqlen=64) == 256  # too short
+    # per-token states are never cut
+    assert _scan_ws(lib, batch=1, states=P, **big) == 256
+    # the generic kernel's shapes (state 64) are never cut
+    assert _scan_ws(lib, batch=1, channels=1536, state=64, seqlen=2048) == 256
+
+
+def test_static_entry_checks_before_touching_the_device(lib):
+    """ssm_scan_fwd_static runs every host-side check first: on a host with no
+    GPU a bad call returns its own status, not SSM_ERR_CUDA."""
+    fn = lib.ssm_scan_fwd_static
+    assert fn(None, None) == NULL
+    assert fn(ctypes.byref(_scan(x=None)), None) == NULL
+    assert fn(ctypes.byref(_scan(x=P + 2)), None) == ALIGN
+    assert fn(ctypes.byref(_scan(state=12)), None) == UNSUP
+    assert fn(ctypes.byref(_scan(io=7)), None) == DTYPE
+    # beyond its scratch: batch * seqlen > 262144 with the step norm
+    assert fn(ctypes.byref(_scan(flags=5, batch=2, seqlen=131073)), None) == WS
+    # batch 0: nothing to do
+    assert fn(ctypes.byref(_scan(batch=0, x=None, dt=None, B=None, C=None, A=None,
+                                 y=None)), None) == OK
+
+
+def test_workspace_status_needs_a_stream_copy(lib):
+    assert lib.ssm_workspace_status(None, None) in (OK, 7)  # 7: no device here
 
 
 def test_scan_empty_batch_is_a_no_op(lib):
@@ -142,7 +190,7 @@ def test_workspace_queries_need_no_pointers(lib):
     n = ctypes.c_size_t(7)
     a = _scan(x=None, dt=None, B=None, C=None, A=None, y=None, flags=5)
     assert lib.ssm_scan_workspace(ctypes.byref(a), ctypes.byref(n)) == OK
-    assert n.value == 2 * 8 * 4
+    assert n.value == 256 + 256
     s = _ssd(x=None, dt=None, B=None, C=None, A=None, y=None)
     assert lib.ssd_chunk_scan_workspace(ctypes.byref(s), ctypes.byref(n)) == OK
 
@@ -255,12 +303,11 @@ def test_empty_calls_launch_nothing(lib):
     sequence) returns OK before any device call: these run without a GPU."""
     a = _ssd(batch=0, io=0, x=None, dt=None, B=None, C=None, A=None, y=None)
     assert lib.ssd_chunk_scan_fwd(ctypes.byref(a), None) == OK
-    # the tensor-core shapes still want their (status-word) workspace
+    # the tensor-core shapes too: no workspace is needed when there is no work
     a = _ssd(batch=0, x=None, dt=None, B=None, C=None, A=None, y=None)
-    assert lib.ssd_chunk_scan_fwd(ctypes.byref(a), None) == WS
-    a = _ssd(batch=0, x=None, dt=None, B=None, C=None, A=None, y=None, workspace=P,
-             workspace_bytes=256)
     assert lib.ssd_chunk_scan_fwd(ctypes.byref(a), None) == OK
+    a = _ssd(batch=1, x=P, workspace=None)
+    assert lib.ssd_chunk_scan_fwd(ctypes.byref(a), None) == WS
     s = _scan(batch=0, x=None, dt=None, B=None, C=None, A=None, y=None)
     assert lib.ssm_scan_fwd_write(ctypes.byref(s), 0, ctypes.c_void_p(P), None) == OK
     for kw in (dict(batch=0), dict(seqlen=0)):

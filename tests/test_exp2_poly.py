@@ -8,7 +8,7 @@ import re
 import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SRC = os.path.join(HERE, "..", "selective_state_space_28_b200", "csrc", "scan_m1_tma.cu")
+SRC = os.path.join(HERE, "..", "selective_state_space_28_b200", "csrc", "common.cuh")
 
 
 def _coefficients():
@@ -19,7 +19,8 @@ def _coefficients():
 
 
 def _exp2_fma(d, A2, lim, coef, magic):
-    """float32 emulation of exp2_fma1(d, A2, lim): 2^(d*A2) for d >= 0, A2 < 0."""
+    """float32 emulation of one lane of exp2_fma2(d, A2, lim): 2^(d*A2) for
+    d >= 0, A2 < 0."""
     f32 = np.float32
     d, A2, lim = f32(d), f32(A2), f32(lim)
     dc = np.minimum(d, lim)

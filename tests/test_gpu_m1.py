@@ -191,3 +191,88 @@ def test_host_buffers_round_trip(cuda_ok):
     ref = _oracle(d)
     assert_close_normwise(y, ref[0], REL[torch.bfloat16], "y")
     assert_close_normwise(h, ref[1], REL[torch.bfloat16], "h_last")
+
+
+# ------------------------------------------------------ sequence segments
+# When batch x channels leaves the SMs short of warps the pipelined kernel
+# cuts the sequence into segments: segments from their own start, a carry
+# (an associative scan over (decay product, end state) pairs), and a rescan
+# from the carried states.  The shapes below are cut on a 148-SM B200 (the
+# workspace size says so); the results must match the oracle like the whole
+# sequence does.
+
+def _workspace_bytes(d, flags=I.SOFTPLUS):
+    import ctypes
+    from selective_state_space_28_b200 import _lib as L
+    b, Lq, C = d["x"].shape
+    G, N = d["B"].shape[2], d["B"].shape[3]
+    io = L.SSM_BF16 if d["x"].dtype == torch.bfloat16 else L.SSM_F32
+    a = L.ScanArgs(batch=b, seqlen=Lq, channels=C, state=N, groups=G, io=io, flags=flags,
+                   rms_eps=1e-6)
+    n = ctypes.c_size_t(0)
+    L.check(L.lib().ssm_scan_workspace(ctypes.byref(a), ctypes.byref(n)), "ws")
+    return n.value
+
+
+@pytest.mark.parametrize("b,L,C,N,io,h0", [
+    (1, 2048, 1536, 16, "bf16", True),    # 8 segments of 256 tokens
+    (1, 1000, 1536, 16, "bf16", False),   # ragged last segment, zero start state
+    (2, 4096, 256, 8, "f32", True),       # state 8, float32 I/O
+    (1, 3000, 512, 32, "bf16", True),     # state 32
+])
+def test_sequence_segments_match_the_oracle(cuda_ok, b, L, C, N, io, h0):
+    d = I.m1_inputs(b, L, C, N, io=io, gate=True, seed=200 + L + N, h0=h0)
+    assert _workspace_bytes(d) > 256, "shape not cut into segments"
+    rel = REL[torch.float32 if io == "f32" else torch.bfloat16]
+    _check(d, _run(d), _oracle(d), rel)
+
+
+def test_sequence_segments_with_norms_and_extreme_rates(cuda_ok):
+    """Cut sequence with all three norms, A at the pages' extremes and steps
+    driven to +-25: the decay products the carry multiplies by span 0 to 1."""
+    flags = I.SOFTPLUS | I.RMS_BC | I.RMS_DT
+    d = I.m1_inputs(1, 2048, 512, 16, io="bf16", gate=True, seed=210, h0=True)
+    d["A"][0] = -36316.0
+    d["A"][1] = -4e-4
+    d["A"][2, :8] = -4e-4
+    d["dt"][0, ::97] = 25.0
+    d["dt"][0, 5::13] = -25.0
+    assert _workspace_bytes(d, flags) > 256 + 256 + 2048 * 4
+    _check(d, _run(d, flags=flags), _oracle(d, flags=flags), REL[torch.bfloat16])
+
+
+def test_sequence_segments_zero_steps_on_segment_edges(cuda_ok):
+    """dt_raw = -inf (a zero step) on the first and last tokens of segments
+    and in a run across a segment boundary."""
+    d = I.m1_inputs(1, 2048, 1536, 16, io="bf16", gate=True, seed=212, h0=True)
+    assert _workspace_bytes(d) > 256
+    for t in (0, 255, 256, 257, 511, 512, 1023, 2047):
+        d["dt"][0, t] = -float("inf")
+    d["dt"][0, 700:800, :100] = -float("inf")
+    _check(d, _run(d), _oracle(d), REL[torch.bfloat16])
+
+
+def test_sequence_segments_h_last_may_alias_h0(cuda_ok):
+    """The rescan reads the carried states, never h0, so h_last may be h0
+    itself even when the call runs as three launches."""
+    d = I.m1_inputs(1, 2048, 1536, 16, io="bf16", gate=True, seed=211, h0=True)
+    assert _workspace_bytes(d) > 256
+    ref = _oracle(d)
+    dev = {k: (v.cuda() if v is not None else None) for k, v in d.items()}
+    h_io = dev["h0"].clone()
+    y, h, _ = _ops().ssm_scan_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"],
+                                  D=dev["D"], z=dev["z"], dt_bias=dev["dt_bias"], h0=h_io,
+                                  h_last=h_io)
+    torch.cuda.synchronize()
+    assert_close_normwise(y, ref[0], REL[torch.bfloat16], "y")
+    assert_close_normwise(h_io, ref[1], REL[torch.bfloat16], "h_last aliasing h0")
+
+
+def test_generic_kernel_shapes(cuda_ok):
+    """Shapes the pipelined kernel cannot tile (bf16 rows that are not
+    16-byte multiples, state 64) run the generic kernel and still match."""
+    for b, L, C, N, io in ((2, 50, 36, 16, "bf16"), (1, 70, 64, 64, "f32"),
+                           (2, 40, 24, 4, "bf16")):
+        d = I.m1_inputs(b, L, C, N, io=io, gate=True, seed=220 + C, h0=True)
+        rel = REL[torch.float32 if io == "f32" else torch.bfloat16]
+        _check(d, _run(d), _oracle(d), rel)

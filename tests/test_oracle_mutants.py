@@ -99,15 +99,28 @@ MUTANTS = {
 
 
 def _pin_calls():
+    """Every pin with every combination of its parametrize values (G as 1
+    and 2 where it is a plain default)."""
+    import itertools
     calls = []
     for name, fn in sorted(inspect.getmembers(pins, inspect.isfunction)):
         if not name.startswith("test_"):
             continue
         params = inspect.signature(fn).parameters
-        if "G" in params:
-            calls += [(name, fn, {"G": 1}), (name, fn, {"G": 2})]
-        else:
-            calls.append((name, fn, {}))
+        axes = []
+        for mark in getattr(fn, "pytestmark", []):
+            if mark.name != "parametrize":
+                continue
+            names = [n.strip() for n in mark.args[0].split(",")]
+            vals = [v if len(names) > 1 else (v,) for v in mark.args[1]]
+            axes.append([dict(zip(names, v)) for v in vals])
+        if "G" in params and not any("G" in a[0] for a in axes if a):
+            axes.append([{"G": 1}, {"G": 2}])
+        for combo in itertools.product(*axes) if axes else [()]:
+            kw = {}
+            for d in combo:
+                kw.update(d)
+            calls.append((name, fn, kw))
     return calls
 
 
