@@ -368,6 +368,37 @@ def m1_segments(w):
     return -1
 
 
+def bench_m1_static(w, K, W, dist, device, seed_base):
+    """The same scan through ssm_scan_fwd_static, which never cuts the
+    sequence: the uncut time beside a cut call's."""
+    import ctypes
+    import torch
+    from selective_state_space_28_b200 import _lib as L
+    from selective_state_space_28_b200 import inputs as I
+    nb = m1_bytes(w)
+    sets = []
+    for r in range(n_sets(nb)):
+        d = I.workload_inputs(w, device=device, seed=seed_base + 1000 * r)
+        d["y"] = torch.empty_like(d["x"])
+        d["h_last"] = torch.empty((w.batch, w.channels, w.state), device=device)
+        sets.append(d)
+    st = torch.cuda.current_stream(device).cuda_stream
+
+    def step(i):
+        d = sets[i % len(sets)]
+        a = L.ScanArgs(batch=w.batch, seqlen=w.seqlen, channels=w.channels, state=w.state,
+                       groups=w.groups, io=L.SSM_BF16 if w.io == "bf16" else L.SSM_F32,
+                       flags=w.flags, rms_eps=w.rms_eps, x=d["x"].data_ptr(),
+                       dt=d["dt"].data_ptr(), z=d["z"].data_ptr() if d["z"] is not None else None,
+                       B=d["B"].data_ptr(), C=d["C"].data_ptr(), A=d["A"].data_ptr(),
+                       D=d["D"].data_ptr(), dt_bias=d["dt_bias"].data_ptr(),
+                       y=d["y"].data_ptr(), h_last=d["h_last"].data_ptr())
+        L.check(L.lib().ssm_scan_fwd_static(ctypes.byref(a), st), "ssm_scan_fwd_static")
+    ms = timed(step, K, W, dist, device) / K
+    launch_ms = per_launch_ms(step, max(10, K), device)
+    return {"ms_per_step": ms, "bytes": nb, "launch_ms": launch_ms}
+
+
 def bench_conv(w, K, W, dist, device, pk, seed_base):
     import torch
     from selective_state_space_28_b200 import inputs as I
@@ -521,27 +552,111 @@ def e2e_m1(w, device, n_steps=5):
     return {"ms": ms, "h2d": h2d, "d2h": d2h}
 
 
-def cpu_baseline_m1(w, min_seconds=10.0):
-    """The oracle, as it stands, on a bounded sample of the workload: whole
-    passes over all batch rows, repeated until about `min_seconds` of CPU
-    time, on every host core the process may use."""
-    import oracle
-    from selective_state_space_28_b200 import inputs as I
-    d = I.workload_inputs(w, device="cpu")
-    threads = oracle.default_threads()
+# ------------------------------------------------------------------ CPU baselines
+
+def _time_oracle(fn, threads, min_seconds):
+    """Passes of fn(threads) until about min_seconds; returns (passes, seconds)."""
     passes, sec = 0, 0.0
-    while sec < min_seconds and passes < 50:
+    while sec < min_seconds and passes < 200:
         t0 = time.perf_counter()
-        oracle.m1_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"], z=d["z"],
-                       dt_bias=d["dt_bias"], flags=w.flags, rms_eps=w.rms_eps,
-                       nthreads=threads)
+        fn(threads)
         sec += time.perf_counter() - t0
         passes += 1
-    gbs = m1_bytes(w) * passes / sec / 1e9
-    return {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": "%d full pass(es) of %s (batch %d x %d tokens x %d channels x state %d), "
-                      "float64 C token loop, %.1f s" % (passes, w.name, w.batch, w.seqlen,
-                                                        w.channels, w.state, sec)}
+    return passes, sec
+
+
+def _cpu_entry(unit_per_pass, unit, fn, sample, min_seconds):
+    """The oracle on all the host cores this process may use, and on one."""
+    import oracle
+    threads = oracle.default_threads()
+    fn(threads)  # page in, build
+    n_all, s_all = _time_oracle(fn, threads, min_seconds)
+    n_one, s_one = _time_oracle(fn, 1, min_seconds)
+    try:
+        hw = os.cpu_count()
+    except Exception:  # pragma: no cover
+        hw = None
+    return {"value": unit_per_pass * n_all / s_all, "unit": unit, "cores": threads,
+            "value_1core": unit_per_pass * n_one / s_one, "cores_hw": hw,
+            "affinity_cores": threads, "kind": "oracle",
+            "sample": "%s; %d pass(es) in %.1f s on %d cores, %d in %.1f s on 1 core"
+                      % (sample, n_all, s_all, threads, n_one, s_one)}
+
+
+def cpu_baseline_m1(w, min_seconds=4.0, rows=1, tokens=None):
+    """The float64 oracle, as it stands, on a bounded sample of a Mamba-1
+    workload: `rows` batch rows and the first `tokens` tokens (all channels,
+    so that the step norm over the channels is the workload's)."""
+    import oracle
+    from selective_state_space_28_b200 import inputs as I
+    L = tokens or w.seqlen
+    d = I.m1_inputs(rows, L, w.channels, w.state, w.groups, w.io, w.gate, w.seed)
+    ws = I.Workload(w.name, "m1", batch=rows, seqlen=L, channels=w.channels, state=w.state,
+                    groups=w.groups, io=w.io, gate=w.gate, flags=w.flags)
+    nb = m1_bytes(ws)
+
+    def fn(threads):
+        oracle.m1_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                       dt_bias=d["dt_bias"], flags=w.flags, rms_eps=w.rms_eps,
+                       want_states=w.want_states, nthreads=threads)
+    r = _cpu_entry(nb / 1e9, "GB/s", fn, "%d batch row(s) x %d tokens x %d channels x state %d "
+                   "of %s, float64 C token loop" % (rows, L, w.channels, w.state, w.name),
+                   min_seconds)
+    return r
+
+
+def cpu_baseline_ssd(w, min_seconds=4.0, heads=4):
+    """The oracle's Mamba-2 token loop on one batch row and `heads` of the
+    workload's heads (heads are independent given B and C); tokens/s scaled
+    to the whole head count."""
+    import oracle
+    from selective_state_space_28_b200 import inputs as I
+    d = I.ssd_inputs(1, w.seqlen, heads, w.head_dim, w.state, w.groups, w.io, w.gate, w.seed)
+
+    def fn(threads):
+        oracle.m2_scan(d["x"], d["dt"], d["B"], d["C"], d["A"], d["D"], z=d["z"],
+                       dt_bias=d["dt_bias"], nthreads=threads)
+    return _cpu_entry(w.seqlen * heads / w.heads, "tokens/s", fn,
+                      "1 batch row x %d of %d heads x %d tokens of %s (tokens/s scaled by the "
+                      "head fraction), float64 C token loop" % (heads, w.heads, w.seqlen, w.name),
+                      min_seconds)
+
+
+def cpu_baseline_decode(w, min_seconds=4.0, rows=16):
+    """The oracle's decode step on `rows` batch rows of one Mamba-2 layer and
+    one Mamba-1 layer (the stack runs layer by layer; every layer is the
+    same shape), GB/s of state read-modify-write plus the token."""
+    import oracle
+    from selective_state_space_28_b200 import inputs as I
+    e = I.m2_step_inputs(rows, w.heads, w.head_dim, w.state, w.groups, w.io, seed=w.seed)
+    f = I.m1_step_inputs(rows, w.m1_channels, w.m1_state, 1, w.io, gate=True, seed=w.seed + 1)
+    _, m2b, m1b = decode_bytes(w)
+    nb = (m2b + m1b) * rows / w.batch
+
+    def fn(threads):
+        oracle.m2_step(e["state"], e["x"], e["dt"], e["B"], e["C"], e["A"], e["D"],
+                       dt_bias=e["dt_bias"])
+        oracle.m1_step(f["state"], f["x"], f["dt"], f["B"], f["C"], f["A"], f["D"], z=f["z"],
+                       dt_bias=f["dt_bias"])
+    return _cpu_entry(nb / 1e9, "GB/s", fn, "%d of %d batch rows of one Mamba-2 layer and one "
+                      "Mamba-1 layer of %s, float64 C loop (single-threaded by construction)"
+                      % (rows, w.batch, w.name), min_seconds)
+
+
+def cpu_baselines(min_seconds=3.0):
+    """Oracle timings for every configuration, keyed by workload name."""
+    from selective_state_space_28_b200 import inputs as I
+    W = I.WORKLOADS
+    out = {}
+    out["m1_toy_b1_l64_c32_n4_f32"] = cpu_baseline_m1(W["m1_toy_b1_l64_c32_n4_f32"], min_seconds)
+    out[HEADLINE] = cpu_baseline_m1(W[HEADLINE], min_seconds, rows=1)
+    wf = W["m1_falcon_rms_b4_l8192_c8192_n16_bf16"]
+    out[wf.name] = cpu_baseline_m1(wf, min_seconds, rows=1, tokens=512)
+    ws = W["ssd_2p7b_b4_l4096_h80_p64_n128_bf16"]
+    out[ws.name] = cpu_baseline_ssd(ws, min_seconds)
+    wd = W["decode_2p7b_stack_b256"]
+    out[wd.name] = cpu_baseline_decode(wd, min_seconds)
+    return out
 
 
 def run_only(args):
@@ -602,6 +717,7 @@ def run_ours(args):
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen,
                    "channels": w.channels, "state": w.state, "groups": w.groups,
                    "io_dtype": w.io, "state_dtype": "f32", "gate": w.gate,
+                   "sequence_segments": r["segments"],
                    "l2": "inputs rotated over %d buffer sets (%.0f MB each) > L2"
                          % (r["sets"], r["bytes"] / 1e6),
                    "parallelism": "dp%d (independent batches per GPU)" % dist.world},
@@ -667,6 +783,20 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(ach / hbm, 4), "traffic": traffic_for("conv_2p7b"),
                          "kernel": "conv1d_vec_kernel"}}
+        w1 = I.WORKLOADS["m1_130m_b1_l2048_c1536_n16_bf16"]
+        Kb = max(3, min(K, 20))
+        cut = bench_m1(w1, Kb, max(3, W), dist, device, pk, rank_seed(w1.seed, dist.rank))
+        whole = bench_m1_static(w1, Kb, max(3, W), dist, device, rank_seed(w1.seed, dist.rank))
+        ach = cut["bytes"] / (cut["launch_ms"] * 1e-3) / 1e9
+        wl[w1.name] = {
+            "value": round(job_value(cut["bytes"], dist.world, cut["ms_per_step"]) / 1e9, 2),
+            "unit": "GB/s", "ms_per_step": round(cut["ms_per_step"], 4),
+            "sequence_segments": cut["segments"],
+            "uncut_ms_per_step": round(whole["ms_per_step"], 4),
+            "speedup_from_segments": round(whole["ms_per_step"] / cut["ms_per_step"], 3),
+            "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
+                         "frac": round(ach / hbm, 4), "traffic": None,
+                         "kernel": "m1_scan_tma_kernel (state-only segments, carry, rescan)"}}
         sw = bench_m1(w, max(3, min(K, 10)), 3, dist, device, pk, rank_seed(w.seed, dist.rank),
                       write_at=w.seqlen // 2)
         ach = sw["bytes"] / (sw["launch_ms"] * 1e-3) / 1e9
@@ -674,7 +804,8 @@ def run_ours(args):
             "value": round(job_value(sw["bytes"], dist.world, sw["ms_per_step"]) / 1e9, 2),
             "unit": "GB/s", "ms_per_step": round(sw["ms_per_step"], 4),
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
-                         "frac": round(ach / hbm, 4), "traffic": None,
+                         "frac": round(ach / hbm, 4),
+                         "traffic": traffic_for("m1_scan_tma_130m_write"),
                          "kernel": "m1_scan_tma_kernel (write form)"}}
         wg = I.WORKLOADS["gnorm_2p7b_b4_l4096_w5120_bf16"]
         gn = bench_gnorm(wg, max(3, min(K, 20)), max(3, W), dist, device, pk,
@@ -698,7 +829,10 @@ def run_ours(args):
                          "kernel": "attn_mask_kernel (+ attn_prep_kernel, attn_cb_tc_kernel)"}}
         out["workloads"] = wl
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline_m1(w)
+        cb = cpu_baselines()
+        out["cpu_baseline"] = cb.pop(HEADLINE)
+        for name, entry in cb.items():
+            out.setdefault("workloads", {}).setdefault(name, {})["cpu_baseline"] = entry
     dist.close()
     if dist.rank == 0:
         print(json.dumps(out), flush=True)

@@ -72,6 +72,12 @@ WORKLOADS = {
     "m1_130m_b8_l2048_c1536_n16_bf16": Workload(
         "m1_130m_b8_l2048_c1536_n16_bf16", "m1", batch=8, seqlen=2048,
         channels=1536, state=16, io="bf16", gate=True, seed=1),
+    # The same mixer scan for a single prompt (batch 1): too few (batch,
+    # channel) chains to fill the SMs, so the scan cuts the sequence into
+    # segments joined by the state carry.
+    "m1_130m_b1_l2048_c1536_n16_bf16": Workload(
+        "m1_130m_b1_l2048_c1536_n16_bf16", "m1", batch=1, seqlen=2048,
+        channels=1536, state=16, io="bf16", gate=True, seed=8),
     # Falcon-Mamba-7B width (8192) with the weightless norms, long sequence.
     "m1_falcon_rms_b4_l8192_c8192_n16_bf16": Workload(
         "m1_falcon_rms_b4_l8192_c8192_n16_bf16", "m1", batch=4, seqlen=8192,
