@@ -164,7 +164,9 @@ def test_ssd_status_word_clear(cuda_ok):
     ops = _ops()
     d = I.ssd_inputs(2, 300, 3, 64, 128, io="bf16", seed=9, h0=True)
     dv = {k: (v.cuda() if v is not None else None) for k, v in d.items()}
-    ws = torch.full((256,), 7, dtype=torch.uint8, device="cuda")
+    n = ops.ssd_workspace_bytes(batch=2, seqlen=300, heads=3, head_dim=64, state=128, groups=1,
+                                chunk=256, io=1, flags=1)
+    ws = torch.full((n,), 7, dtype=torch.uint8, device="cuda")
     ops.ssd_chunk_scan_fwd(dv["x"], dv["dt"], dv["A"], dv["B"], dv["C"], D=dv["D"],
                            dt_bias=dv["dt_bias"], h0=dv["h0"], workspace=ws)
     torch.cuda.synchronize()
