@@ -46,8 +46,8 @@ def parse(argv=None):
                     help="measure only the headline workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["m1", "ssd", "decode", "decode_layer", "falcon", "conv",
-                                       "gnorm", "attn"],
+    ap.add_argument("--only", choices=["m1", "m1_write", "m1_b1", "ssd", "decode", "decode_layer",
+                                       "falcon", "falcon_b1", "conv", "gnorm", "attn"],
                     help="run just one workload's timed loop (for profiling); prints its timing")
     return ap.parse_args(argv)
 
@@ -669,14 +669,18 @@ def run_only(args):
     torch.cuda.set_device(dist.local)
     device = torch.device("cuda", dist.local)
     pk = peaks()
-    name = {"m1": HEADLINE, "ssd": "ssd_2p7b_b4_l4096_h80_p64_n128_bf16",
+    name = {"m1": HEADLINE, "m1_write": HEADLINE, "m1_b1": "m1_130m_b1_l2048_c1536_n16_bf16",
+            "falcon_b1": "m1_falcon_rms_b1_l8192_c8192_n16_bf16",
+            "ssd": "ssd_2p7b_b4_l4096_h80_p64_n128_bf16",
             "decode": "decode_2p7b_stack_b256", "decode_layer": "decode_2p7b_layer_b256",
             "falcon": "m1_falcon_rms_b4_l8192_c8192_n16_bf16",
             "conv": "conv_2p7b_b4_l4096_c5376_bf16",
             "gnorm": "gnorm_2p7b_b4_l4096_w5120_bf16",
             "attn": "attn_2p7b_b1_l1024_h80_n128_bf16"}[args.only]
     w = I.WORKLOADS[name]
-    fn = {"m1": bench_m1, "falcon": bench_m1, "ssd": bench_ssd, "decode": bench_decode,
+    fn = {"m1": bench_m1, "m1_b1": bench_m1, "falcon_b1": bench_m1,
+          "m1_write": lambda *a: bench_m1(*a, write_at=w.seqlen // 2),
+          "falcon": bench_m1, "ssd": bench_ssd, "decode": bench_decode,
           "decode_layer": bench_decode, "conv": bench_conv, "gnorm": bench_gnorm,
           "attn": bench_attn}[args.only]
     r = fn(w, args.steps, args.warmup, dist, device, pk, w.seed)

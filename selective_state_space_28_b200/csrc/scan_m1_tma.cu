@@ -17,16 +17,21 @@
 // Per stage, every warp (no CTA-wide barrier anywhere in the loop):
 //   1. waits for the stage's bytes (mbarrier `full`);
 //   2. widens (and, with SSM_RMSNORM_BC, RMS-normalises) its share of the
-//      stage's B and C rows into float32, then arrives on `conv`;
-//   3. computes d and d*x for its own channels, one token per lane;
-//   4. waits on `conv` (every warp's B/C share), then runs the recurrence:
-//      per token each lane updates its four states with packed f32x2
-//      arithmetic and forms its partial C.h; every G tokens the G lanes of a
+//      stage's B and C rows into float32;
+//   3. for its share of the stage's tokens and all 32 channels computes
+//      d = softplus(dt rstd + bias), d x, D x and silu(z), then arrives on
+//      `conv`;
+//   4. waits on `conv` (every warp's share), then runs the recurrence: per
+//      token each lane updates its four states with packed f32x2 arithmetic
+//      and forms its partial C.h, the decays of the next 8 tokens formed
+//      while the current 8 run their chain; every G tokens the G lanes of a
 //      channel trade partials in log2(G) shuffle rounds so that lane q ends
 //      with token q's complete C.h (a transposing reduction), and applies the
 //      skip term, the gate and the rounding for that token;
-//   5. arrives on `empty`; the issuing thread refills a stage's buffer once
-//      every warp has released it.
+//   5. arrives on `empty` (the issuing thread refills a stage's buffer once
+//      every warp has released it) and stores its rows of the previous
+//      stage's y, which every warp has finished by now, in whole 64-byte
+//      rows.
 //
 // Sequence segments (the carry across chunks).  When batch x channels gives
 // too few warps to fill the SMs, the sequence is cut into S segments and run
@@ -46,6 +51,7 @@
 #include "tma.h"
 
 #include <algorithm>
+#include <type_traits>
 #include <cmath>
 
 namespace ssm {
@@ -80,9 +86,14 @@ struct alignas(128) ScanSmem {
   // warp's lanes, one row each, fall in distinct banks.
   float2 ddx[2][kTL][kCT + 2];
   float2 eg[2][kTL][kCT + 2];
-  T y[kTL][kCT + 16 / sizeof(T)];  // output staging, rows padded by 16 bytes
+  // Output staging, two buffers by stage parity: the warps write stage s's y
+  // here, and during stage s+1 (once the `conv` barrier shows every warp has
+  // finished stage s) each warp stores a quarter of its rows to global
+  // memory in full 32-channel rows -- whole 32-byte sectors, so that HBM3e
+  // (no write mask) never has to merge a partly written sector.
+  T y[2][kTL][kCT];
   float bias[kCT], skip[kCT];
-  uint64_t full[NS], conv[NS], empty[NS];
+  uint64_t full[NS], conv[NS], empty[NS], ylast;
 };
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
@@ -196,6 +207,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
       mbar_init(&s.conv[i], NW * 32);  // every lane arrives (release of its own writes)
       mbar_init(&s.empty[i], NW * 32);
     }
+    mbar_init(&s.ylast, NW * 32);
     fence_mbar_init();
   }
   if (threadIdx.x < kCT) {
@@ -207,15 +219,20 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
 
   const bool issuer = threadIdx.x == 0;
   int issued = 0;
+  // x, dt, z are read once (evict-first); the B and C rows of a batch row are
+  // read by every channel block of it (evict-last), so the streams do not push
+  // them out of L2 between the first block that reads them and the last
+  const uint64_t pol_stream = issuer ? createpolicy_evict_first() : 0;
+  const uint64_t pol_shared = issuer ? createpolicy_evict_last() : 0;
   auto issue = [&](int stage) {
     const int buf = stage % NS;
     const int t0 = (int)(tb + (int64_t)stage * kTL);
     mbar_expect_tx(&s.full[buf], kStageBytes);
-    tma_load_3d(&s.x[buf][0][0], &mx, &s.full[buf], (int)c0, t0, b);
-    tma_load_3d(&s.dt[buf][0][0], &mdt, &s.full[buf], (int)c0, t0, b);
-    if (HAS_Z) tma_load_3d(&s.z[buf][0][0], &mz, &s.full[buf], (int)c0, t0, b);
-    tma_load_3d(&s.B[buf][0][0], &mB, &s.full[buf], g * N, t0, b);
-    tma_load_3d(&s.C[buf][0][0], &mC, &s.full[buf], g * N, t0, b);
+    tma_load_3d_hint(&s.x[buf][0][0], &mx, &s.full[buf], (int)c0, t0, b, pol_stream);
+    tma_load_3d_hint(&s.dt[buf][0][0], &mdt, &s.full[buf], (int)c0, t0, b, pol_stream);
+    if (HAS_Z) tma_load_3d_hint(&s.z[buf][0][0], &mz, &s.full[buf], (int)c0, t0, b, pol_stream);
+    tma_load_3d_hint(&s.B[buf][0][0], &mB, &s.full[buf], g * N, t0, b, pol_shared);
+    tma_load_3d_hint(&s.C[buf][0][0], &mC, &s.full[buf], g * N, t0, b, pol_shared);
   };
   if (issuer)
     for (; issued < NS && issued < nst; ++issued) issue(issued);
@@ -243,6 +260,20 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
       PX == 2 && __all_sync(0xffffffffu, softplus_on && ((Al.x < 0.f && Al.y < 0.f) || !cvalid));
   float dsum = 0.f;
   bool failed = false;
+  // Rows [warp * kTL / NW, + kTL / NW) of stage st's y staging (token t0y
+  // onwards, tny of them in the segment) to global memory, 16 bytes a lane.
+  auto store_y = [&](int st, int64_t t0y, int tny) {
+    constexpr int kRows = kTL / NW;
+    constexpr int kChunks = kCT * (int)sizeof(T) / 16;  // per row
+    char *yg = static_cast<char *>(p.y);
+    for (int e = lane; e < kRows * kChunks; e += 32) {
+      const int t = warp * kRows + e / kChunks, k = e % kChunks;
+      const int64_t cg = c0 + (int64_t)k * 16 / (int64_t)sizeof(T);  // chunk's first channel
+      if (t >= tny || cg >= C) continue;  // C is a multiple of 16 bytes' worth
+      *reinterpret_cast<uint4 *>(yg + ((b * L + t0y + t) * C + cg) * (int64_t)sizeof(T)) =
+          *reinterpret_cast<const uint4 *>(reinterpret_cast<const char *>(&s.y[st & 1][t][0]) + 16 * k);
+    }
+  };
 
   for (int sg = 0; sg < nst; ++sg) {
     const int buf = sg % NS;
@@ -319,7 +350,10 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
     // step k runs its chain, and the readout of step k-1 is reduced and
     // stored meanwhile, so that a warp always has independent work at hand.
     const int tw = (WR && p.t_write >= t0 && p.t_write < t0 + tn) ? (int)(p.t_write - t0) : -1;
-    constexpr int SL = G <= 4 ? 4 : G;  // tokens per step
+    // (8 tokens per step: measured 8 % faster than 4 at the Falcon width,
+    // equal on the 130m workload; 16 is slower.  The write form, which
+    // carries two forms of the chain, keeps 4 so that it does not spill.)
+    constexpr int SL = G > 8 ? G : (WR ? 4 : 8);  // tokens per step
     struct Pre {
       f2 a[SL][NP], w[SL][NP];  // decays and write terms d * x * B
     };
@@ -355,7 +389,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
         const float yq = transpose_reduce<G>(pg, q);
         const int tt = tg + G * k + q;
         const float2 eg = s.eg[sg & 1][tt][cw0 + ch];
-        st(&s.y[tt][cw0 + ch], (yq + eg.x) * eg.y);
+        st(&s.y[sg & 1][tt][cw0 + ch], (yq + eg.x) * eg.y);
       }
     };
     Pre cur, nxt;
@@ -365,26 +399,39 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
     for (int tg = 0; tg < kTL; tg += SL) {
       if (tg + SL < kTL) pre(tg + SL, nxt);
       float part[SL];
+      // the chain of one step; only the step holding a written token takes
+      // the form that checks for it (one compare per token costs a fifth of
+      // the loop)
+      auto chain = [&](auto wr) {
 #pragma unroll
-      for (int u = 0; u < SL; ++u) {
-        const int t = tg + u;
+        for (int u = 0; u < SL; ++u) {
+          const int t = tg + u;
 #pragma unroll
-        for (int j = 0; j < NP; ++j) h[j] = fma2(cur.a[u][j], h[j], cur.w[u][j]);
-        if (WR && t == tw && cvalid) {
-          // a state written at this token replaces h_t before y_t reads it
-          // ("Mamba", nnterp guide, "The state")
-          load_pairs<NP>(p.state_write + (b * C + c) * N + SPL * q, h);
+          for (int j = 0; j < NP; ++j) h[j] = fma2(cur.a[u][j], h[j], cur.w[u][j]);
+          if constexpr (decltype(wr)::value) {
+            if (t == tw && cvalid) {
+              // a state written at this token replaces h_t before y_t reads
+              // it ("Mamba", nnterp guide, "The state")
+              load_pairs<NP>(p.state_write + (b * C + c) * N + SPL * q, h);
+            }
+          }
+          if (kFull) {
+            f2 cv[NP];
+            load_pairs<NP>(&s.bc[buf][t][1][SPL * q], cv);
+            f2 acc = mul2(cv[0], h[0]);
+#pragma unroll
+            for (int j = 1; j < NP; ++j) acc = fma2(cv[j], h[j], acc);
+            part[u] = acc.x + acc.y;
+          }
+          if (STATES && cvalid && t < tn)
+            store_pairs<NP>(p.states + ((b * L + t0 + t) * C + c) * N + SPL * q, h);
         }
-        if (kFull) {
-          f2 cv[NP];
-          load_pairs<NP>(&s.bc[buf][t][1][SPL * q], cv);
-          f2 acc = mul2(cv[0], h[0]);
-#pragma unroll
-          for (int j = 1; j < NP; ++j) acc = fma2(cv[j], h[j], acc);
-          part[u] = acc.x + acc.y;
-        }
-        if (STATES && cvalid && t < tn)
-          store_pairs<NP>(p.states + ((b * L + t0 + t) * C + c) * N + SPL * q, h);
+      };
+      if constexpr (WR) {
+        if (tw >= tg && tw < tg + SL) chain(std::true_type{});
+        else chain(std::false_type{});
+      } else {
+        chain(std::false_type{});
       }
       if (kFull && tg >= SL) finish(tg - SL, partp);
 #pragma unroll
@@ -393,29 +440,12 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
     }
     if (kFull) finish(kTL - SL, partp);
     mbar_arrive(&s.empty[buf]);
+    // ---- 5. y of the previous stage: every warp has finished it (they all
+    // arrived on this stage's `conv`), so this warp stores its share of the
+    // rows, after its own recurrence (measured: 2 % faster than storing them
+    // before it, 5 % faster than each warp storing its own 16-byte rows)
+    if (kFull && sg >= 1) store_y(sg - 1, t0 - kTL, kTL);
 
-    // ---- 5. this warp's y tile to global memory (lanes read rows other
-    // lanes wrote: the warp meets first)
-    if (kFull) {
-      __syncwarp();
-      constexpr int kRowBytes = CPW * (int)sizeof(T);
-      constexpr int kChunk = kRowBytes < 16 ? kRowBytes : 16;
-      constexpr int kPerRow = kRowBytes / kChunk;
-      const bool wvalid = c0 + cw0 < C;
-      char *yg = static_cast<char *>(p.y);
-      for (int e = lane; e < kTL * kPerRow; e += 32) {
-        const int t = e / kPerRow, k = e % kPerRow;
-        if (t >= tn || !wvalid) continue;
-        const int64_t off = ((b * L + t0 + t) * C + c0 + cw0) * (int64_t)sizeof(T) + k * kChunk;
-        if (c0 + cw0 + (int64_t)k * kChunk / (int64_t)sizeof(T) >= C) continue;
-        const char *src = reinterpret_cast<const char *>(&s.y[t][cw0]) + k * kChunk;
-        if constexpr (kChunk == 16)
-          *reinterpret_cast<uint4 *>(yg + off) = *reinterpret_cast<const uint4 *>(src);
-        else
-          *reinterpret_cast<uint2 *>(yg + off) = *reinterpret_cast<const uint2 *>(src);
-      }
-      __syncwarp();
-    }
     // ---- refill the buffer of the previous stage once every warp left it
     if (issuer && sg >= 1 && issued < nst) {
       const int prev = sg - 1;
@@ -429,6 +459,16 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
     if (__any_sync(0xffffffffu, failed)) break;
   }
 
+  // y of the last stage, once every warp has written it
+  if (kFull && !failed && nst > 0) {
+    mbar_arrive(&s.ylast);
+    if (__all_sync(0xffffffffu, mbar_wait(&s.ylast, 0, kWaitLimit))) {
+      const int64_t tl = tb + (int64_t)(nst - 1) * kTL;
+      store_y(nst - 1, tl, (int)(te - tl));
+    } else {
+      failed = true;
+    }
+  }
   if (failed) {
     if (lane == 0 && p.status) atomicExch(p.status, 1);
     // let every copy this CTA started land before its shared memory goes

@@ -83,6 +83,12 @@ WORKLOADS = {
         "m1_falcon_rms_b4_l8192_c8192_n16_bf16", "m1", batch=4, seqlen=8192,
         channels=8192, state=16, io="bf16", gate=True,
         flags=SOFTPLUS | RMS_BC | RMS_DT, seed=2),
+    # One prompt at the Falcon width (the profiling case of that kernel: its
+    # inputs exceed L2 while a capture stays a few GB).
+    "m1_falcon_rms_b1_l8192_c8192_n16_bf16": Workload(
+        "m1_falcon_rms_b1_l8192_c8192_n16_bf16", "m1", batch=1, seqlen=8192,
+        channels=8192, state=16, io="bf16", gate=True,
+        flags=SOFTPLUS | RMS_BC | RMS_DT, seed=9),
     # Mamba-2 2.7B-shaped SSD chunk scan (80 heads x 64, state 128, chunk 256).
     "ssd_2p7b_b4_l4096_h80_p64_n128_bf16": Workload(
         "ssd_2p7b_b4_l4096_h80_p64_n128_bf16", "ssd", batch=4, seqlen=4096,
