@@ -25,15 +25,18 @@
 //               issued per tile in the order Sc(c), S(c+1), Y(c).
 //   warps 4-7 and 14-17   mask group, thread = token, two warps per TMEM
 //               lane quarter each taking half of every row's work (each warp
-//               also recomputes the whole tile's cumulative decay, so the
-//               warps run unsynchronised): the tile's step, cumulative decay
-//               and weights, w o x, then the mask applied to S as it is read
-//               from TMEM (D on its diagonal, so Y holds D x), and the row-
-//               scaled C, e_i C_i with e_i = exp(cum_i), both written back as
-//               the bf16 A operand of Y.  The mask exp(cum_i - cum_j) d_j is
-//               elementwise on the four 32 x 32 diagonal blocks; below them it
-//               is a row factor times a column factor, both <= 1 for a
-//               decaying state.
+//               also recomputes the whole tile's decay factors, so the warps
+//               run unsynchronised): the tile's steps d_j and decays
+//               a_j = exp(d_j A), and every factor exp(cum_i - cum_j) as the
+//               product a_{j+1} .. a_i (never as the exponential of a
+//               difference of running sums, which would lose a small step
+//               beside a large sum); w o x; then the mask applied to S as it
+//               is read from TMEM (D on its diagonal, so Y holds D x), and
+//               the row-scaled C, e_i C_i with e_i = a_0 .. a_i, both written
+//               back as the bf16 A operand of Y.  The mask is elementwise on
+//               the four 32 x 32 diagonal blocks (a running product down from
+//               the diagonal); below them it is a row factor times a column
+//               factor, both <= 1 for a decaying state.
 //   warps 0-3   state group: thread n keeps row n of the float32 state in
 //               registers, h = exp(cum_last) h + Sc, and writes its bf16 copy
 //               for Y of the next tile (two buffers).
@@ -86,11 +89,11 @@ struct __align__(1024) SsdSmem {
   uint8_t X[2][kQ * 128];     // [stage]
   uint8_t Xw[kQ * 128];       // w o x of the tile whose Sc is next
   uint8_t Hb[2][kN * 128];    // bf16 copy of the carried state, rows n
-  float cumw[8][kQ];          // per mask-group warp: cumulative log2-decay
-  float cuml[8][kQ];          //   (a compensated sum: cumw + cuml),
+  float adw[8][kQ];           // per mask-group warp: decay a_j of token j,
+  float ppw[8][kQ];           //   a_b ... a_j (b the first token of j's 32-token block),
   float ddw[8][kQ];           //   step d_j,
-  float vdw[8][kQ];           //   column factor of the off-diagonal mask
-  float a[4];                 // exp(cum_last) per tile, ring of four
+  float vdw[8][kQ];           //   a_{j+1} ... a_{b+31} d_j (column factor of the mask)
+  float a[4];                 // exp(cum_last) = a_0 .. a_127 per tile, ring of four
   // Per-tile signals come in pairs indexed by tile parity (xready in fours);
   // the dependencies between roles bound every waiter's lag to less than one
   // lap of its ring, so no waiter can miss a phase.
@@ -131,30 +134,6 @@ struct SsdTcParams {
   float *seg_decay;      // [ntail][nseg]: product of the segment's tile decays
   const float *seg_hin;  // [ntail][nseg][N][P]: the state entering each segment
 };
-
-// Compensated sums.  The mask needs exp(cum_i - cum_j) for tokens i, j of a
-// tile, and the running sum cum of the log-decays d * A can be large (a fast
-// decay over many tokens) beside the step of one token (a near-zero step):
-// the difference of two rounded float sums would lose that step entirely
-// (the "Mamba-2" page's extreme A_h with a tiny step).  Each prefix sum is
-// therefore kept as an unevaluated pair hi + lo (Knuth's TwoSum), and a
-// difference is (hi_i - hi_j) + (lo_i - lo_j): the first term is exact when
-// the two sums are close (Sterbenz), the second restores what rounding cut.
-struct ff {
-  float hi, lo;
-};
-__device__ __forceinline__ ff two_sum(float a, float b) {
-  const float s = a + b;
-  const float bb = s - a;
-  return {s, (a - (s - bb)) + (b - bb)};
-}
-__device__ __forceinline__ ff ff_add(ff a, ff b) {
-  ff r = two_sum(a.hi, b.hi);
-  const float lo = r.lo + (a.lo + b.lo);
-  const float hi = r.hi + lo;  // renormalise (|lo| is below an ulp of r.hi)
-  return {hi, lo - (hi - r.hi)};
-}
-__device__ __forceinline__ float ff_diff(ff a, ff b) { return (a.hi - b.hi) + (a.lo - b.lo); }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -439,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float bias = p.dt_bias ? p.dt_bias[hd] : 0.f;
     const float Dh = p.D ? p.D[hd] : 0.f;
     const bool softplus_on = p.flags & 1u;
-    float *cumw = s.cumw[mg], *cuml = s.cuml[mg], *ddw = s.ddw[mg], *vdw = s.vdw[mg];
+    float *adw = s.adw[mg], *ppw = s.ppw[mg], *ddw = s.ddw[mg], *vdw = s.vdw[mg];
     // lane l handles tokens 4l .. 4l+3 of the tile in the prologue; their dt
     // is fetched a tile ahead and kept as raw bfloat16 bits until used
     const uint16_t *dtb = reinterpret_cast<const uint16_t *>(p.dt);
@@ -456,11 +435,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int k = c & 1;
       const int64_t t0 = (int64_t)(cb + c) * kQ;
       const int valid = (int)(L - t0 < kQ ? L - t0 : kQ);
-      // step, log2-decay and inclusive sums over the whole tile (needs only
-      // dt, so it runs while the tile's TMA is in flight)
-      float d4[4];
-      ff p4[4];
-      ff run = {0.f, 0.f};
+      // The tile's step d_j and decay a_j = exp(d_j A) per token, and every
+      // decay factor of the masked form as a product of the a_j -- never as
+      // the exponential of a difference of running sums, whose rounding
+      // would lose a token's small step beside a large sum (the "Mamba-2"
+      // page's extreme A_h with a tiny step).  Within each 32-token block
+      // (8 lanes): prefix products pp_j = a_b .. a_j and suffix products
+      // a_{j+1} .. a_{b+31}; block totals T_K.  (Needs only dt, so it runs
+      // while the tile's TMA is in flight.)
+      float d4[4], a4[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float d = 0.f;
@@ -469,35 +452,51 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (softplus_on) d = softplus_sfu(d);
         }
         d4[q] = d;
-        run = ff_add(run, ff{d * A2, 0.f});
-        p4[q] = run;
+        a4[q] = ex2(d * A2);
       }
-      ff incl = run;
+      const float lp1 = a4[0] * a4[1], lp2 = lp1 * a4[2], lp3 = lp2 * a4[3];  // in-lane prefixes
+      float incl = lp3;  // products over this lane and the earlier lanes of its block
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const ff v = {__shfl_up_sync(0xffffffffu, incl.hi, off),
-                      __shfl_up_sync(0xffffffffu, incl.lo, off)};
-        if (lane >= off) incl = ff_add(v, incl);
+      for (int off = 1; off < 8; off <<= 1) {
+        const float v = __shfl_up_sync(0xffffffffu, incl, off, 8);
+        if ((lane & 7) >= off) incl *= v;
       }
-      const ff total = {__shfl_sync(0xffffffffu, incl.hi, 31), __shfl_sync(0xffffffffu, incl.lo, 31)};
-      ff excl = {__shfl_up_sync(0xffffffffu, incl.hi, 1), __shfl_up_sync(0xffffffffu, incl.lo, 1)};
-      if (lane == 0) excl = {0.f, 0.f};
-      // cum at the last token of each 32-token block (lanes 7, 15, 23, 31)
-      const int be = (lane & ~7) | 7;
-      const ff blk_end = {__shfl_sync(0xffffffffu, incl.hi, be), __shfl_sync(0xffffffffu, incl.lo, be)};
+      float before = __shfl_up_sync(0xffffffffu, incl, 1, 8);
+      if ((lane & 7) == 0) before = 1.f;
+      float after = lp3;  // products over this lane and the later lanes of its block
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const ff cq = ff_add(excl, p4[q]);
-        cumw[4 * lane + q] = cq.hi;
-        cuml[4 * lane + q] = cq.lo;
-        ddw[4 * lane + q] = d4[q];
-        vdw[4 * lane + q] = ex2(ff_diff(blk_end, cq)) * d4[q];
+      for (int off = 1; off < 8; off <<= 1) {
+        const float v = __shfl_down_sync(0xffffffffu, after, off, 8);
+        if ((lane & 7) + off < 8) after *= v;
       }
-      if (mg == 0 && lane == 0) s.a[c & 3] = ex2(total.hi + total.lo);
+      float later = __shfl_down_sync(0xffffffffu, after, 1, 8);
+      if ((lane & 7) == 7) later = 1.f;
+      const float T0 = __shfl_sync(0xffffffffu, incl, 7), T1 = __shfl_sync(0xffffffffu, incl, 15),
+                  T2 = __shfl_sync(0xffffffffu, incl, 23), T3 = __shfl_sync(0xffffffffu, incl, 31);
+      {
+        const float pp[4] = {before * a4[0], before * lp1, before * lp2, before * lp3};
+        const float sp[4] = {later * a4[3] * a4[2] * a4[1], later * a4[3] * a4[2], later * a4[3], later};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          adw[4 * lane + q] = a4[q];
+          ppw[4 * lane + q] = pp[q];
+          ddw[4 * lane + q] = d4[q];
+          vdw[4 * lane + q] = sp[q] * d4[q];
+        }
+      }
+      if (mg == 0 && lane == 0) s.a[c & 3] = T0 * T1 * T2 * T3;
       __syncwarp();
-      const ff cs = {cumw[i], cuml[i]};
-      const float e_i = ex2(cs.hi + cs.lo);
-      const float w_i = ex2(ff_diff(total, cs)) * ddw[i];
+      // this row's factors: e_i = a_0 .. a_i and w_i = a_{i+1} .. a_127 d_i
+      const float Tb[4] = {T0, T1, T2, T3};
+      float before_blk = 1.f, after_blk = 1.f;
+#pragma unroll
+      for (int K = 0; K < 4; ++K) {
+        if (K < mw) before_blk *= Tb[K];
+        if (K > mw) after_blk *= Tb[K];
+      }
+      const float pp_i = ppw[i];
+      const float e_i = pp_i * before_blk;
+      const float w_i = vdw[i] * after_blk;
       // w o x (this warp's rows, half the columns), the B operand of Sc(c):
       // x of tile c has landed and Sc(c-1) is done with the buffer
       if (!waitw(s, &s.full[k], (c >> 1) & 1, p.status, 8)) break;
@@ -540,9 +539,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q = 0; q < 8; ++q) m[q] = 0u;
         } else if (J < mw) {
-          // below the diagonal: S_ij * exp2(cum_i - cum_r) * vd_j, r the
-          // block's last token; both factors <= 1
-          const float u = ex2(ff_diff(cs, ff{cumw[32 * J + 31], cuml[32 * J + 31]}));
+          // below the diagonal: S_ij * (a_{j+1} .. a_{32J+31}) d_j * u with
+          // u = T_{J+1} .. T_{mw-1} (a_{32 mw} .. a_i); both factors <= 1 for
+          // a decaying state
+          float u = pp_i;
+#pragma unroll
+          for (int K = 1; K < 3; ++K)
+            if (K > J && K < mw) u *= Tb[K];
           const float4 *vd4 = reinterpret_cast<const float4 *>(vdw + j0);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -557,22 +560,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             m[2 * q + 1] = pack_bf16x2(bq.x, bq.y);
           }
         } else {
-          // diagonal block: S_ij * exp2(cum_i - cum_j) * d_j for j <= i, + D at j = i
-          const float4 *c4 = reinterpret_cast<const float4 *>(cumw + j0);
-          const float4 *l4 = reinterpret_cast<const float4 *>(cuml + j0);
+          // diagonal block: S_ij * (a_{j+1} .. a_i) d_j for j <= i, + D at
+          // j = i; the product runs down from j = i (exact, no cancellation)
+          const int il = lane, jl0 = 16 * half;
+          float P = 1.f;  // a_{jtop+1} .. a_i, jtop the last of this warp's columns <= i
+          if (half == 0 && il >= 16) {
+            const float4 *au = reinterpret_cast<const float4 *>(adw + 32 * J + 16);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const float4 a = au[v];
+              if (16 + 4 * v <= il) P *= a.x;
+              if (17 + 4 * v <= il) P *= a.y;
+              if (18 + 4 * v <= il) P *= a.z;
+              if (19 + 4 * v <= il) P *= a.w;
+            }
+          }
+          const float4 *a4p = reinterpret_cast<const float4 *>(adw + j0);
           const float4 *d4p = reinterpret_cast<const float4 *>(ddw + j0);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 cj = c4[q], lj = l4[q], dj = d4p[q];
-            const float cjs[4] = {cj.x, cj.y, cj.z, cj.w}, ljs[4] = {lj.x, lj.y, lj.z, lj.w},
-                        djs[4] = {dj.x, dj.y, dj.z, dj.w};
+          for (int q = 3; q >= 0; --q) {
+            const float4 av = a4p[q], dv = d4p[q];
+            const float as[4] = {av.x, av.y, av.z, av.w}, ds[4] = {dv.x, dv.y, dv.z, dv.w};
             float f[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int j = j0 + 4 * q + e;
+            for (int e = 3; e >= 0; --e) {
+              const int jl = jl0 + 4 * q + e;
               const float sv = __uint_as_float(r[4 * q + e]);
-              const float dl = ff_diff(cs, ff{cjs[e], ljs[e]});
-              f[e] = (j <= i) ? sv * (ex2(dl) * djs[e]) + (j == i ? Dh : 0.f) : 0.f;
+              if (jl <= il) {
+                f[e] = sv * (P * ds[e]) + (jl == il ? Dh : 0.f);
+                P *= as[e];
+              } else {
+                f[e] = 0.f;
+              }
             }
             m[2 * q] = pack_bf16x2(f[0], f[1]);
             m[2 * q + 1] = pack_bf16x2(f[2], f[3]);
