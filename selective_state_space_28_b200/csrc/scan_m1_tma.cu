@@ -219,20 +219,20 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
 
   const bool issuer = threadIdx.x == 0;
   int issued = 0;
-  // x, dt, z are read once (evict-first); the B and C rows of a batch row are
-  // read by every channel block of it (evict-last), so the streams do not push
-  // them out of L2 between the first block that reads them and the last
-  const uint64_t pol_stream = issuer ? createpolicy_evict_first() : 0;
-  const uint64_t pol_shared = issuer ? createpolicy_evict_last() : 0;
+  // No L2 policy on these loads: an evict-first hint on the streamed x, dt, z
+  // boxes (64 B of each 128-B line per CTA) let L2 drop a line after one
+  // channel block had read its half and before its neighbour read the other,
+  // which then came from DRAM again (a quarter more reads at the Falcon
+  // width), and evict-last on B and C gained nothing measurable.
   auto issue = [&](int stage) {
     const int buf = stage % NS;
     const int t0 = (int)(tb + (int64_t)stage * kTL);
     mbar_expect_tx(&s.full[buf], kStageBytes);
-    tma_load_3d_hint(&s.x[buf][0][0], &mx, &s.full[buf], (int)c0, t0, b, pol_stream);
-    tma_load_3d_hint(&s.dt[buf][0][0], &mdt, &s.full[buf], (int)c0, t0, b, pol_stream);
-    if (HAS_Z) tma_load_3d_hint(&s.z[buf][0][0], &mz, &s.full[buf], (int)c0, t0, b, pol_stream);
-    tma_load_3d_hint(&s.B[buf][0][0], &mB, &s.full[buf], g * N, t0, b, pol_shared);
-    tma_load_3d_hint(&s.C[buf][0][0], &mC, &s.full[buf], g * N, t0, b, pol_shared);
+    tma_load_3d(&s.x[buf][0][0], &mx, &s.full[buf], (int)c0, t0, b);
+    tma_load_3d(&s.dt[buf][0][0], &mdt, &s.full[buf], (int)c0, t0, b);
+    if (HAS_Z) tma_load_3d(&s.z[buf][0][0], &mz, &s.full[buf], (int)c0, t0, b);
+    tma_load_3d(&s.B[buf][0][0], &mB, &s.full[buf], g * N, t0, b);
+    tma_load_3d(&s.C[buf][0][0], &mC, &s.full[buf], g * N, t0, b);
   };
   if (issuer)
     for (; issued < NS && issued < nst; ++issued) issue(issued);
