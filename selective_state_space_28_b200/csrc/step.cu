@@ -153,13 +153,19 @@ cudaError_t launch_m2_k(const M2Params &p, int RS, cudaStream_t s) {
   dim3 block((unsigned)(P / 4 * RS));
   if (TT == 1) {
     auto k = m2_recurrent_kernel<T, HZ, K, 1>;
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
     k<<<grid, block, smem, s>>>(p);
   } else {
     auto k = m2_recurrent_kernel<T, HZ, K, 8>;
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
     k<<<grid, block, smem, s>>>(p);
   }
   return cudaGetLastError();

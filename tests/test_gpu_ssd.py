@@ -93,7 +93,7 @@ def test_ssd_split_and_carry(cuda_ok):
 
 def test_2p7b_full_size_sampled(cuda_ok):
     """Mamba-2 2.7B-shaped SSD at full size (b4 L4096 H80 P64 N128 chunk 256,
-    bf16), in the benchmark's launch configuration; the oracle checks three
+    bf16), in the benchmark's launch configuration; the oracle checks four
     heads of two batch rows (heads are independent given B and C)."""
     w = I.WORKLOADS["ssd_2p7b_b4_l4096_h80_p64_n128_bf16"]
     d = I.workload_inputs(w)
