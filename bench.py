@@ -46,7 +46,8 @@ def parse(argv=None):
                     help="measure only the headline workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["m1", "m1_write", "m1_b1", "ssd", "decode", "decode_layer",
+    ap.add_argument("--only", choices=["m1", "m1_write", "m1_b1", "ssd", "ssd_conv", "decode",
+                                       "decode_layer",
                                        "falcon", "falcon_b1", "conv", "gnorm", "attn"],
                     help="run just one workload's timed loop (for profiling); prints its timing")
     return ap.parse_args(argv)
@@ -101,6 +102,25 @@ def ssd_bytes(w):
         n += w.batch * w.seqlen * w.heads * w.head_dim * e
     n += w.batch * w.seqlen * w.heads * e                  # dt
     n += 2 * w.batch * w.seqlen * w.groups * w.state * e   # B, C
+    n += w.batch * w.heads * w.state * w.head_dim * 4      # h_last
+    n += 3 * w.heads * 4
+    return n
+
+
+def ssd_conv_bytes(w):
+    """The fused mixer prologue + SSD: xBC read once (x, B, C before the
+    convolution), dt (and z) read, y written, the float32 conv weights, bias
+    and carried conv state (read and written), h_last, A, D, dt_bias."""
+    e = _esz(w.io)
+    ctot = w.heads * w.head_dim + 2 * w.groups * w.state
+    n = w.batch * w.seqlen * ctot * e                      # xBC
+    n += w.batch * w.seqlen * w.heads * w.head_dim * e     # y
+    if w.gate:
+        n += w.batch * w.seqlen * w.heads * w.head_dim * e
+    n += w.batch * w.seqlen * w.heads * e                  # dt
+    n += 5 * ctot * 4                                      # conv weights, bias
+    if w.extra.get("state", False):
+        n += 2 * w.batch * ctot * 3 * 4
     n += w.batch * w.heads * w.state * w.head_dim * 4      # h_last
     n += 3 * w.heads * 4
     return n
@@ -492,6 +512,46 @@ def bench_ssd(w, K, W, dist, device, pk, seed_base):
             "tokens": w.batch * w.seqlen, "sets": len(sets), "launches_per_step": launches}
 
 
+def bench_ssd_conv(w, K, W, dist, device, pk, seed_base):
+    """The SSD with the mixer's convolution fused in front
+    (ssd_conv_chunk_scan_fwd): xBC before the convolution in, y out."""
+    import torch
+    from selective_state_space_28_b200 import inputs as I
+    from selective_state_space_28_b200 import ops
+    nb = ssd_conv_bytes(w)
+    ctot = w.heads * w.head_dim + 2 * w.groups * w.state
+    sets = []
+    for r in range(n_sets(nb)):
+        d = I.workload_inputs(w, device=device, seed=seed_base + 1000 * r)
+        d["y"] = torch.empty((w.batch, w.seqlen, w.heads, w.head_dim), dtype=d["xBC"].dtype,
+                             device=device)
+        d["h_last"] = torch.empty((w.batch, w.heads, w.state, w.head_dim), device=device)
+        d["cs_out"] = torch.empty((w.batch, ctot, 3), device=device)
+        sets.append(d)
+    ws = ops.ssd_conv_workspace_bytes(batch=w.batch, seqlen=w.seqlen, heads=w.heads,
+                                      head_dim=w.head_dim, state=w.state, groups=w.groups,
+                                      chunk=w.chunk, io=1 if w.io == "bf16" else 0,
+                                      flags=w.flags)
+    wsb = torch.empty(max(ws, 1), dtype=torch.uint8, device=device)
+
+    def step(i):
+        d = sets[i % len(sets)]
+        ops.ssd_conv_chunk_scan_fwd(d["xBC"], d["conv_w"], d["dt"], d["A"], heads=w.heads,
+                                    state=w.state, groups=w.groups, conv_bias=d["conv_bias"],
+                                    conv_state_in=d["conv_state"], D=d["D"], z=d["z"],
+                                    dt_bias=d["dt_bias"], chunk=w.chunk, flags=w.flags,
+                                    y=d["y"], h_last=d["h_last"], conv_state_out=d["cs_out"],
+                                    workspace=wsb)
+    ms = timed(step, K, W, dist, device) / K
+    launch_ms = per_launch_ms(step, max(5, K), device)
+    ops._check_status(wsb, torch.cuda.current_stream(device).cuda_stream, "bench")
+    # the B/C pre-pass, then one SSD launch, or three when the last wave is cut
+    split = ws - 256 - ((w.batch * w.seqlen * 2 * w.groups * w.state * 2 + 255) // 256 * 256)
+    launches = 1 + (3 if split > 0 else 1)
+    return {"ms_per_step": ms, "bytes": nb, "flops": ssd_flops(w), "launch_ms": launch_ms,
+            "tokens": w.batch * w.seqlen, "sets": len(sets), "launches_per_step": launches}
+
+
 def bench_decode(w, K, W, dist, device, pk, seed_base):
     import torch
     from selective_state_space_28_b200 import inputs as I
@@ -672,6 +732,7 @@ def run_only(args):
     name = {"m1": HEADLINE, "m1_write": HEADLINE, "m1_b1": "m1_130m_b1_l2048_c1536_n16_bf16",
             "falcon_b1": "m1_falcon_rms_b1_l8192_c8192_n16_bf16",
             "ssd": "ssd_2p7b_b4_l4096_h80_p64_n128_bf16",
+            "ssd_conv": "ssd_conv_2p7b_b4_l4096_h80_p64_n128_bf16",
             "decode": "decode_2p7b_stack_b256", "decode_layer": "decode_2p7b_layer_b256",
             "falcon": "m1_falcon_rms_b4_l8192_c8192_n16_bf16",
             "conv": "conv_2p7b_b4_l4096_c5376_bf16",
@@ -680,7 +741,8 @@ def run_only(args):
     w = I.WORKLOADS[name]
     fn = {"m1": bench_m1, "m1_b1": bench_m1, "falcon_b1": bench_m1,
           "m1_write": lambda *a: bench_m1(*a, write_at=w.seqlen // 2),
-          "falcon": bench_m1, "ssd": bench_ssd, "decode": bench_decode,
+          "falcon": bench_m1, "ssd": bench_ssd, "ssd_conv": bench_ssd_conv,
+          "decode": bench_decode,
           "decode_layer": bench_decode, "conv": bench_conv, "gnorm": bench_gnorm,
           "attn": bench_attn}[args.only]
     r = fn(w, args.steps, args.warmup, dist, device, pk, w.seed)
@@ -795,6 +857,29 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(ach, 2), "peak": hbm, "unit": "GB/s",
                          "frac": round(ach / hbm, 4), "traffic": traffic_for("conv_2p7b"),
                          "kernel": "conv1d_vec_kernel"}}
+        # The SSD with the convolution fused in front, beside the unfused pair
+        # (the convolution and the SSD lines above, same shapes, this run).
+        wsc = I.WORKLOADS["ssd_conv_2p7b_b4_l4096_h80_p64_n128_bf16"]
+        sc = bench_ssd_conv(wsc, Ke, max(3, W), dist, device, pk, rank_seed(wsc.seed, dist.rank))
+        tf = sc["flops"] / (sc["launch_ms"] * 1e-3) / 1e12
+        unfused = s["ms_per_step"] + cv["ms_per_step"]
+        e = _esz(wsc.io)
+        saved = 2 * wsc.batch * wsc.seqlen * wsc.heads * wsc.head_dim * e
+        wl[wsc.name] = {
+            "value": round(job_value(sc["tokens"], dist.world, sc["ms_per_step"]), 1),
+            "unit": "tokens/s", "ms_per_step": round(sc["ms_per_step"], 4),
+            "gpu_launches": sc["launches_per_step"] * Ke,
+            "unfused_ms_per_step": round(unfused, 4),
+            "speedup_vs_unfused": round(unfused / sc["ms_per_step"], 3),
+            "bytes_saved_per_call": saved,
+            "note": "unfused = the convolution line plus the SSD line; saved = the convolved "
+                    "x written and read back (B and C still make one round trip)",
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2),
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(tf / pk["bf16_tflops"], 4), "traffic": None,
+                         "flops_per_launch": sc["flops"], "bytes_per_launch": sc["bytes"],
+                         "hbm_frac": round(sc["bytes"] / (sc["launch_ms"] * 1e-3) / 1e9 / hbm,
+                                           4)}}
         w1 = I.WORKLOADS["m1_130m_b1_l2048_c1536_n16_bf16"]
         Kb = max(3, min(K, 20))
         cut = bench_m1(w1, Kb, max(3, W), dist, device, pk, rank_seed(w1.seed, dist.rank))

@@ -6,7 +6,9 @@
  *
  *   ssm_scan_fwd        Mamba-1 selective scan over a prompt
  *                       (ssm_scan_fwd_write: with a state written at one token).
- *   ssd_chunk_scan_fwd  Mamba-2 (SSD) scan over a prompt, chunked.
+ *   ssd_chunk_scan_fwd  Mamba-2 (SSD) scan over a prompt, chunked
+ *                       (ssd_conv_chunk_scan_fwd: with the mixer's causal
+ *                       convolution fused in front of it).
  *   ssm_scan_step       one decode token against a cached state.
  *   ssm_conv1d_fwd      the mixers' causal depthwise convolution (+ silu),
  *                       over a prompt or, in place, one decode token.
@@ -44,7 +46,7 @@
 extern "C" {
 #endif
 
-#define SSM_ABI_VERSION 2
+#define SSM_ABI_VERSION 3
 
 typedef enum ssm_status {
   SSM_OK = 0,
@@ -235,6 +237,63 @@ typedef struct ssd_scan_args {
  * SSM_ERR_WORKSPACE. */
 ssm_status_t ssd_chunk_scan_workspace(const ssd_scan_args_t *args, size_t *bytes);
 ssm_status_t ssd_chunk_scan_fwd(const ssd_scan_args_t *args, void *stream);
+
+/* ------------------------------------------------------------------------
+ * ssd_conv_chunk_scan_fwd -- the Mamba-2 mixer's causal convolution and the
+ * SSD scan in one call.
+ *
+ * Defined by: "Mamba-2" (nnterp encyclopedia), the module tree
+ * (Conv1d(channels, channels, kernel_size 4, padding 3, groups = channels),
+ * output cut to the input length) and "The mixer's values" (x, B, C =
+ * silu(conv1d(xBC)) split by channel, then the SSD).  With
+ * channels = heads * head_dim + 2 * groups * state:
+ *
+ *   u[t, c] = silu(conv_bias[c] + sum_{k<4} conv_w[c, k] * xBC[t - 3 + k, c])
+ *   x = u[.., 0 : heads*head_dim] as [.., heads, head_dim],
+ *   B = the next groups*state channels, C = the last groups*state,
+ *   then y and h_last exactly as ssd_chunk_scan_fwd computes them.
+ *
+ *   xBC            : [batch, seqlen, channels] bf16, before the convolution
+ *   conv_w         : [channels, 4] float32; conv_bias: [channels] or NULL (0)
+ *   conv_state_in  : [batch, channels, 3] float32 or NULL (zeros, a sequence
+ *                    start): the inputs of the 3 tokens before t = 0,
+ *                    oldest first
+ *   conv_state_out : [batch, channels, 3] float32 or NULL: the last 3
+ *                    inputs (conv_state_in's entries where seqlen < 3), so a
+ *                    prompt cut in two and run with conv_state_out ->
+ *                    conv_state_in gives the same y; must not overlap
+ *                    conv_state_in (SSM_ERR_SHAPE)
+ *   z, dt, A, D, dt_bias, h0, y, h_last, chunk, flags: as ssd_chunk_scan_fwd
+ *   workspace      : ssd_conv_chunk_scan_workspace() bytes: the status word
+ *                    (word 0, read with ssm_workspace_status()), the
+ *                    convolved B and C (batch * seqlen * 2 * groups * state
+ *                    bf16) and the segment states of a cut last wave (as
+ *                    for ssd_chunk_scan_fwd; device-dependent size)
+ *
+ * The convolved x is never written to memory: each 128-token tile of x is
+ * convolved in shared memory where it lands; B and C, which every head of a
+ * group reads, are convolved once by a pre-pass.  bf16 silu as
+ * ssm_conv1d_fwd.  Only the tensor-core configuration is taken (io
+ * SSM_BF16, state 128, head_dim 64; else SSM_ERR_UNSUPPORTED: run
+ * ssm_conv1d_fwd then ssd_chunk_scan_fwd).
+ * ---------------------------------------------------------------------- */
+typedef struct ssd_conv_scan_args {
+  int64_t batch, seqlen, heads, head_dim, state, groups, chunk;
+  int32_t io;
+  uint32_t flags;
+  const void *xBC;
+  const float *conv_w, *conv_bias, *conv_state_in;
+  float *conv_state_out;
+  const void *z, *dt;
+  const float *A, *D, *dt_bias, *h0;
+  void *y;
+  float *h_last;
+  void *workspace;
+  size_t workspace_bytes;
+} ssd_conv_scan_args_t;
+
+ssm_status_t ssd_conv_chunk_scan_workspace(const ssd_conv_scan_args_t *args, size_t *bytes);
+ssm_status_t ssd_conv_chunk_scan_fwd(const ssd_conv_scan_args_t *args, void *stream);
 
 /* ------------------------------------------------------------------------
  * ssm_scan_step -- one decode token per sequence, state updated in place.

@@ -45,6 +45,17 @@ class SsdArgs(ctypes.Structure):
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class SsdConvArgs(ctypes.Structure):
+    _fields_ = [("batch", _i64), ("seqlen", _i64), ("heads", _i64), ("head_dim", _i64),
+                ("state", _i64), ("groups", _i64), ("chunk", _i64),
+                ("io", ctypes.c_int32), ("flags", ctypes.c_uint32),
+                ("xBC", _vp), ("conv_w", _vp), ("conv_bias", _vp), ("conv_state_in", _vp),
+                ("conv_state_out", _vp), ("z", _vp), ("dt", _vp),
+                ("A", _vp), ("D", _vp), ("dt_bias", _vp), ("h0", _vp),
+                ("y", _vp), ("h_last", _vp),
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
 class StepArgs(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("io", ctypes.c_int32), ("flags", ctypes.c_uint32),
                 ("rms_eps", ctypes.c_float),
@@ -100,6 +111,9 @@ def lib():
         L.ssd_chunk_scan_fwd.argtypes = [ctypes.POINTER(SsdArgs), _vp]
         L.ssd_chunk_scan_workspace.argtypes = [ctypes.POINTER(SsdArgs),
                                                ctypes.POINTER(ctypes.c_size_t)]
+        L.ssd_conv_chunk_scan_fwd.argtypes = [ctypes.POINTER(SsdConvArgs), _vp]
+        L.ssd_conv_chunk_scan_workspace.argtypes = [ctypes.POINTER(SsdConvArgs),
+                                                    ctypes.POINTER(ctypes.c_size_t)]
         L.ssm_scan_step.argtypes = [ctypes.POINTER(StepArgs), _vp]
         L.ssm_conv1d_fwd.argtypes = [ctypes.POINTER(ConvArgs), _vp]
         L.ssm_gated_rmsnorm_fwd.argtypes = [ctypes.POINTER(GatedNormArgs), _vp]
@@ -111,7 +125,8 @@ def lib():
         L.ssm_workspace_status.argtypes = [_vp, _vp]
         for fn in (L.ssm_scan_fwd_static, L.ssm_workspace_status,
                    L.ssm_scan_fwd, L.ssm_scan_workspace, L.ssd_chunk_scan_fwd,
-                   L.ssd_chunk_scan_workspace, L.ssm_scan_step, L.ssm_conv1d_fwd,
+                   L.ssd_chunk_scan_workspace, L.ssd_conv_chunk_scan_fwd,
+                   L.ssd_conv_chunk_scan_workspace, L.ssm_scan_step, L.ssm_conv1d_fwd,
                    L.ssm_gated_rmsnorm_fwd, L.ssm_scan_fwd_write, L.ssd_attention_fwd,
                    L.ssd_attention_workspace):
             fn.restype = ctypes.c_int

@@ -136,8 +136,22 @@ int64_t attention_lower_tiles(int64_t L);
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t s);
 cudaError_t launch_gated_norm(const GatedNormParams &p, cudaStream_t s);
 cudaError_t launch_conv1d(const ConvParams &p, cudaStream_t s);
+// The Mamba-2 mixer's causal convolution fused into the tensor-core SSD:
+// x, B and C come from xBC [batch][L][ctot] (bf16, before the convolution,
+// ctot = H P + 2 G N), convolved with w [ctot][4] and bias, then silu; the
+// three inputs before token 0 from state_in [batch][ctot][3] or zeros;
+// state_out receives the last three inputs.  bc is workspace for the
+// convolved B and C (ssd_conv_bc_bytes).
+struct SsdConv {
+  const void *xbc;
+  int64_t ctot;
+  const float *w, *bias, *state_in;
+  float *state_out;
+  void *bc;
+};
+size_t ssd_conv_bc_bytes(int64_t batch, int64_t L, int64_t G);
 cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split, void *seg_ws,
-                          cudaStream_t s);
+                          cudaStream_t s, const SsdConv *conv = nullptr);
 
 // The Mamba-1 scan behind ssm_scan_fwd, ssm_scan_fwd_write (t_write >= 0)
 // and ssm_scan_fwd_static (allow_cut false: the sequence is never cut into

@@ -41,7 +41,14 @@
 //               registers, h = exp(cum_last) h + Sc, and writes its bf16 copy
 //               for Y of the next tile (two buffers).
 //   warps 8-11  output group, thread = token: y = Y (* silu(z)), with z
-//               fetched one tile ahead.
+//               fetched one tile ahead.  In the fused form (the mixer's
+//               causal convolution in front, "Mamba-2", the module tree and
+//               "The mixer's values": x, B, C = silu(conv1d(xBC))), the
+//               group first convolves each landed x tile in place, a tile
+//               ahead of the mask group: token i from rows i-3..i, the three
+//               rows before the tile kept from the previous tile's raw
+//               inputs; B and C, which every head of a group shares, are
+//               convolved once by ssd_bc_conv_kernel before the scan.
 // With Y, Sc and the bf16 state double-buffered, the only chain carried from
 // tile to tile is the state group's update; every other role has a tile of
 // slack, and the contractions of the next tile run under this tile's
@@ -93,15 +100,24 @@ struct __align__(1024) SsdSmem {
   float ppw[8][kQ];           //   a_b ... a_j (b the first token of j's 32-token block),
   float ddw[8][kQ];           //   step d_j,
   float vdw[8][kQ];           //   a_{j+1} ... a_{b+31} d_j (column factor of the mask)
+  // With the convolution fused: the three inputs before a tile (bf16, 64
+  // channels), two buffers by tile parity.  (Fits in the struct's alignment
+  // padding: the size is unchanged.)
+  __nv_bfloat16 halo[2][3][kP];
   float a[4];                 // exp(cum_last) = a_0 .. a_127 per tile, ring of four
   // Per-tile signals come in pairs indexed by tile parity (xready in fours);
   // the dependencies between roles bound every waiter's lag to less than one
   // lap of its ring, so no waiter can miss a phase.
   uint64_t full[2], empty[2], sdone[2], scdone[2], mready[2], stdone[2], yready[2], yfree[2];
   uint64_t xready[4];
+  uint64_t xconv[2];          // x of a tile convolved in place (fused form)
   uint32_t taddr;
   int abort;
 };
+
+// The CTA's dynamic shared memory (the struct plus 1 KB to align it) must
+// fit the 227 KB a CTA may have.
+static_assert(sizeof(SsdSmem) + 1024 <= 232448, "SsdSmem exceeds the shared memory of a CTA");
 
 // Packed-bf16 TMEM columns (within an S buffer) of Y's A operand.  The mask
 // for tokens 32 J + 16 h .. + 16 (K step 2 J + h of M x), written by the
@@ -133,6 +149,13 @@ struct SsdTcParams {
   float *seg_hend;       // [ntail][nseg][N][P]: end state from the segment's own start state
   float *seg_decay;      // [ntail][nseg]: product of the segment's tile decays
   const float *seg_hin;  // [ntail][nseg][N][P]: the state entering each segment
+  // The fused convolution (CONV): x is read from xBC before the convolution
+  // (row stride ctot), convolved over tokens with the width-4 kernel cw
+  // [ctot][4] and bias cbias, then silu; the inputs before token 0 come from
+  // cs_in [batch][ctot][3] (oldest first) or are zeros.
+  const __nv_bfloat16 *xbc;
+  int64_t ctot;
+  const float *cw, *cbias, *cs_in;
 };
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
@@ -169,6 +192,34 @@ __device__ __forceinline__ void st_cs_u4(void *p, uint4 v) {
                : "memory");
 }
 
+// Named barrier 1 over the output group (warps 8-11, 128 threads), and the
+// same barrier as a vote: every thread of the group gets the OR of `v`.
+__device__ __forceinline__ void out_group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ bool out_group_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+// 16-byte read-only global load.
+__device__ __forceinline__ uint4 ld_nc_u4(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void unpack8(uint4 u, float (&v)[8]) {
+  v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+  v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+}
+
 __device__ __forceinline__ bool aborted(const SsdSmem &s) {
   return *(volatile const int *)&s.abort != 0;
 }
@@ -198,6 +249,7 @@ __device__ __forceinline__ bool waitw(SsdSmem &s, uint64_t *bar, uint32_t parity
   return !fail;
 }
 
+template <bool CONV>
 __global__ void __launch_bounds__(kThreads, 1)
     ssd_tc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mB,
                   const __grid_constant__ CUtensorMap mC, const SsdTcParams p) {
@@ -259,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.yfree[i], 4);   // one arrival per output-group warp
     }
     for (int i = 0; i < 4; ++i) mbar_init(&s.xready[i], 8);
+    for (int i = 0; i < 2; ++i) mbar_init(&s.xconv[i], 4);  // one arrival per output warp
     s.abort = 0;
     fence_mbar_init();
   }
@@ -498,8 +551,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float e_i = pp_i * before_blk;
       const float w_i = vdw[i] * after_blk;
       // w o x (this warp's rows, half the columns), the B operand of Sc(c):
-      // x of tile c has landed and Sc(c-1) is done with the buffer
+      // x of tile c has landed (and, fused, been convolved in place) and
+      // Sc(c-1) is done with the buffer
       if (!waitw(s, &s.full[k], (c >> 1) & 1, p.status, 8)) break;
+      if (CONV && !waitw(s, &s.xconv[k], (c >> 1) & 1, p.status, 15)) break;
       if (c >= 1 && !waitw(s, &s.scdone[k ^ 1], ((c - 1) >> 1) & 1, p.status, 9)) break;
       {
         const uint32_t w2 = pack_bf16x2(w_i, w_i);
@@ -692,11 +747,123 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q = 0; q < 8; ++q) zr[q] = ld_cs_u4(zp + 8 * q);
       }
     };
-    load_z(0);
-    for (int c = 0; c < nch; ++c) {
+    // A wait of this group: voted per warp, or, fused, over the four warps
+    // (they meet in named barriers there, so none may leave the loop alone).
+    auto waito = [&](uint64_t *bar, uint32_t parity, int code) -> bool {
+      if (!CONV) return waitw(s, bar, parity, p.status, code);
+      const bool ok = mbar_wait(bar, parity, kWaitLimit);
+      const bool fail = out_group_any(!ok);
+      if (fail && i == 0) set_abort(s, p.status, code);
+      return !fail;
+    };
+    // Fused form: the causal convolution of x over tokens, then silu, in
+    // place in the landed tile (the three rows before the tile from the
+    // previous tile's raw inputs, kept in `halo`, or for the first tile of
+    // this CTA from xBC or the conv state); one named barrier between the
+    // reads every thread needs from its neighbour's rows and the writes.
+    auto conv_tile = [&](int c) -> bool {
+      const int k = c & 1;
+      const int64_t t0 = (int64_t)(cb + c) * kQ;
+      const int64_t ch0 = hd * kP;
+      // Before this CTA's first tile the three preceding inputs come from
+      // global memory, widened to float32 into the w o x buffer: nobody uses
+      // it before the mask group's first write, which waits for this tile's
+      // xconv.
+      const float *first = reinterpret_cast<const float *>(s.Xw);
+      if (c == 0) {
+        const uint16_t *xr = reinterpret_cast<const uint16_t *>(p.xbc);
+        for (int idx = i; idx < 3 * kP; idx += 128) {
+          const int row = idx / kP, ch = idx % kP;
+          const int64_t tau = t0 - 3 + row;
+          float v = 0.f;
+          if (tau >= 0) v = __uint_as_float((uint32_t)xr[(b * L + tau) * p.ctot + ch0 + ch] << 16);
+          else if (p.cs_in) v = p.cs_in[(b * p.ctot + ch0 + ch) * 3 + (tau + 3)];
+          reinterpret_cast<float *>(s.Xw)[idx] = v;
+        }
+        out_group_sync();
+      }
+      // Thread (cq, tg): channels 4 cq .. + 4 of the head, tokens 16 tg ..
+      // + 16 of the tile, walked in order with the three previous raw inputs
+      // in registers (every row read once).  Its weights and bias first:
+      // their loads overlap the wait for the tile.
+      const int cq = i & 15, tg = i >> 4;
+      const uint32_t qoff = 8u * (uint32_t)(cq & 1);  // the quad within its 16-byte chunk
+      float wq[4][4], bq[4];
+      {
+        const float4 *wv = reinterpret_cast<const float4 *>(p.cw + (ch0 + 4 * cq) * 4);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 w = __ldg(wv + e);
+          wq[e][0] = w.x; wq[e][1] = w.y; wq[e][2] = w.z; wq[e][3] = w.w;
+          bq[e] = p.cbias ? __ldg(p.cbias + ch0 + 4 * cq + e) : 0.f;
+        }
+      }
+      if (!waito(&s.full[k], (c >> 1) & 1, 14)) return false;
+      uint8_t *xs = s.X[k];
+      auto unpack4 = [](uint2 u, float (&v)[4]) {
+        v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+      };
+      // the three raw rows before this thread's first token: the previous
+      // group's rows (read before anyone overwrites them), the previous
+      // tile's last rows (`halo`), or before this CTA's first tile `first`
+      float win[3][4];
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        const int r = 16 * tg - 3 + j;
+        if (r >= 0) {
+          unpack4(*reinterpret_cast<const uint2 *>(xs + sw128(r, cq >> 1) + qoff), win[j]);
+        } else if (c > 0) {
+          unpack4(*reinterpret_cast<const uint2 *>(&s.halo[k][r + 3][4 * cq]), win[j]);
+        } else {
+          const float4 f = *reinterpret_cast<const float4 *>(first + (r + 3) * kP + 4 * cq);
+          win[j][0] = f.x; win[j][1] = f.y; win[j][2] = f.z; win[j][3] = f.w;
+        }
+      }
+      out_group_sync();  // every window is read: rows may be overwritten now
+#pragma unroll 2
+      for (int j = 0; j < 16; ++j) {
+        const int r = 16 * tg + j;
+        uint2 *row = reinterpret_cast<uint2 *>(xs + sw128(r, cq >> 1) + qoff);
+        const uint2 u = *row;
+        // the raw last three rows are the next tile's halo
+        if (tg == 7 && j >= 13) *reinterpret_cast<uint2 *>(&s.halo[k ^ 1][j - 13][4 * cq]) = u;
+        float xv[4];
+        unpack4(u, xv);
+        // u = silu(bias + sum_q w[q] x[t - 3 + q]), the newest input first
+        // (the order of ssm_conv1d_fwd, so both give the same bits)
+        const bool live = t0 + r < L;
+        float o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float acc = fmaf(wq[e][3], xv[e], bq[e]);
+          acc = fmaf(wq[e][2], win[2][e], acc);
+          acc = fmaf(wq[e][1], win[1][e], acc);
+          acc = fmaf(wq[e][0], win[0][e], acc);
+          o[e] = live ? silu_tanh(acc) : 0.f;
+          win[0][e] = win[1][e];
+          win[1][e] = win[2][e];
+          win[2][e] = xv[e];
+        }
+        *row = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.xconv[k]);
+      return true;
+    };
+    bool ok = true;
+    if (CONV) ok = nch > 0 && conv_tile(0);
+    else load_z(0);
+    for (int c = 0; ok && c < nch; ++c) {
       const int k = c & 1;
       const int64_t t = (int64_t)(cb + c) * kQ + i;
-      if (!waitw(s, &s.yready[k], (c >> 1) & 1, p.status, 13)) break;
+      if (CONV) {
+        // the next tile's convolution first: the mask group needs it for
+        // tile c + 1 while this tile's Y is still being formed
+        if (c + 1 < nch && !conv_tile(c + 1)) break;
+        load_z(c);
+      }
+      if (!waito(&s.yready[k], (c >> 1) & 1, 13)) break;
       tc_fence_after();
       __nv_bfloat16 *yp = p.y + ((b * L + t) * H + hd) * kP;
       // two halves of 32 columns; Y[k] is released after the second load
@@ -732,7 +899,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      load_z(c + 1);
+      if (!CONV) load_z(c + 1);
     }
   }
 
@@ -765,6 +932,66 @@ __global__ void __launch_bounds__(kCarrySlice / 4)
       const float d = dc[sg];
       h = make_float4(fmaf(d, h.x, l.x), fmaf(d, h.y, l.y), fmaf(d, h.z, l.z), fmaf(d, h.w, l.w));
     }
+  }
+}
+
+// The fused call's pre-pass.  (1) The B and C channels of xBC (nbc = 2 G N
+// of them from channel c0 on) convolved over tokens, then silu, into
+// bc [batch][L][nbc]: every head of a group reads the same B and C, so they
+// are convolved once here instead of in each head's CTA (x is convolved
+// inside the scan).  A thread takes one token and eight channels.  (2) The
+// conv state out: the last three inputs of every channel, oldest first
+// (from cs_in where the sequence is shorter than three).
+__global__ void __launch_bounds__(256)
+    ssd_bc_conv_kernel(const __nv_bfloat16 *xbc, int64_t batch, int64_t L, int64_t ctot,
+                       int64_t c0, int64_t nbc, const float *cw, const float *cbias,
+                       const float *cs_in, __nv_bfloat16 *bc, float *cs_out) {
+  const int64_t nchunk = nbc / 8, nconv = batch * L * nchunk;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx < nconv) {
+    const int64_t j = idx % nchunk, bt = idx / nchunk, t = bt % L, bb = bt / L;
+    const int64_t ch = c0 + 8 * j;
+    float v[4][8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int64_t tau = t - 3 + q;
+      if (tau >= 0) {
+        unpack8(ld_nc_u4(xbc + (bb * L + tau) * ctot + ch), v[q]);
+      } else if (cs_in) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[q][e] = cs_in[(bb * ctot + ch + e) * 3 + (tau + 3)];
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[q][e] = 0.f;
+      }
+    }
+    float o[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {  // the newest input first, as ssm_conv1d_fwd
+      const float4 w = __ldg(reinterpret_cast<const float4 *>(cw + (ch + e) * 4));
+      float acc = cbias ? __ldg(cbias + ch + e) : 0.f;
+      acc = fmaf(w.w, v[3][e], acc);
+      acc = fmaf(w.z, v[2][e], acc);
+      acc = fmaf(w.y, v[1][e], acc);
+      acc = fmaf(w.x, v[0][e], acc);
+      o[e] = silu_tanh(acc);
+    }
+    *reinterpret_cast<uint4 *>(bc + (bb * L + t) * nbc + 8 * j) =
+        make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                   pack_bf16x2(o[6], o[7]));
+    return;
+  }
+  const int64_t r = idx - nconv;
+  if (!cs_out || r >= batch * ctot) return;
+  const int64_t c = r % ctot, bb = r / ctot;
+  const uint16_t *xr = reinterpret_cast<const uint16_t *>(xbc);
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {
+    const int64_t tau = L - 3 + q;
+    float v = 0.f;
+    if (tau >= 0) v = __uint_as_float((uint32_t)xr[(bb * L + tau) * ctot + c] << 16);
+    else if (cs_in) v = cs_in[(bb * ctot + c) * 3 + (tau + 3)];
+    cs_out[(bb * ctot + c) * 3 + q] = v;
   }
 }
 
@@ -807,23 +1034,34 @@ size_t ssd_tc_split_bytes(const SsdSplit &r) {
 
 size_t ssd_tc_smem_bytes() { return sizeof(SsdSmem) + 1024; }
 
+size_t ssd_conv_bc_bytes(int64_t batch, int64_t L, int64_t G) {
+  return (size_t)(batch * L * 2 * G * kN) * sizeof(__nv_bfloat16);
+}
+
 cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split, void *seg_ws,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, const SsdConv *conv) {
   const int64_t GN = p.G * kN;
+  // x rows are H P channels apart, or, fused, xBC rows (ctot channels); B and
+  // C rows G N apart, or, fused, the pre-pass's [B | C] rows (2 G N).
+  const int64_t xrow = conv ? conv->ctot : p.H * kP;
+  const int64_t bcrow = conv ? 2 * GN : GN;
+  const void *xp = conv ? conv->xbc : p.x;
+  const void *bp = conv ? conv->bc : p.B;
+  const void *cp = conv ? static_cast<const void *>(static_cast<const __nv_bfloat16 *>(conv->bc) + GN)
+                        : p.Cm;
   CUtensorMap mX, mB, mC;
   {
     uint64_t dims[4] = {(uint64_t)kP, (uint64_t)p.H, (uint64_t)p.L, (uint64_t)p.batch};
-    uint64_t strides[3] = {(uint64_t)kP * 2, (uint64_t)(p.H * kP * 2),
-                           (uint64_t)(p.L * p.H * kP * 2)};
+    uint64_t strides[3] = {(uint64_t)kP * 2, (uint64_t)(xrow * 2), (uint64_t)(p.L * xrow * 2)};
     uint32_t box[4] = {64, 1, kQ, 1};
-    if (!encode(&mX, p.x, 4, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!encode(&mX, xp, 4, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
     uint64_t dims[3] = {(uint64_t)GN, (uint64_t)p.L, (uint64_t)p.batch};
-    uint64_t strides[2] = {(uint64_t)GN * 2, (uint64_t)(p.L * GN * 2)};
+    uint64_t strides[2] = {(uint64_t)bcrow * 2, (uint64_t)(p.L * bcrow * 2)};
     uint32_t box[3] = {64, kQ, 1};
-    if (!encode(&mB, p.B, 3, dims, strides, box)) return cudaErrorInvalidValue;
-    if (!encode(&mC, p.Cm, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!encode(&mB, bp, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!encode(&mC, cp, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
   SsdTcParams q;
   q.batch = p.batch;
@@ -848,15 +1086,30 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
   q.seg_hend = nullptr;
   q.seg_decay = nullptr;
   q.seg_hin = nullptr;
+  q.xbc = conv ? static_cast<const __nv_bfloat16 *>(conv->xbc) : nullptr;
+  q.ctot = conv ? conv->ctot : 0;
+  q.cw = conv ? conv->w : nullptr;
+  q.cbias = conv ? conv->bias : nullptr;
+  q.cs_in = conv ? conv->state_in : nullptr;
   const size_t smem = ssd_tc_smem_bytes();
+  auto kern = conv ? ssd_tc_kernel<true> : ssd_tc_kernel<false>;
   // (set on every call: the attribute belongs to the current device)
   {
-    cudaError_t e = cudaFuncSetAttribute(ssd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
+  if (conv) {
+    const int64_t threads = p.batch * p.L * (2 * GN / 8) + p.batch * conv->ctot;
+    ssd_bc_conv_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(conv->xbc), p.batch, p.L, conv->ctot, p.H * kP,
+        2 * GN, conv->w, conv->bias, conv->state_in, static_cast<__nv_bfloat16 *>(conv->bc),
+        conv->state_out);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   if (split.nseg <= 1) {
-    ssd_tc_kernel<<<(unsigned)q.nfull, kThreads, smem, stream>>>(mX, mB, mC, q);
+    kern<<<(unsigned)q.nfull, kThreads, smem, stream>>>(mX, mB, mC, q);
     return cudaGetLastError();
   }
   // Tail cut into segments: (1) every segment of the tail units from its own
@@ -873,7 +1126,7 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
   q.seg_hend = hend;
   q.seg_decay = dec;
   q.seg_hin = hin;
-  ssd_tc_kernel<<<(unsigned)slots, kThreads, smem, stream>>>(mX, mB, mC, q);
+  kern<<<(unsigned)slots, kThreads, smem, stream>>>(mX, mB, mC, q);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ssd_seg_carry_kernel<<<dim3((unsigned)split.ntail, kN * kP / kCarrySlice), kCarrySlice / 4, 0,
@@ -882,7 +1135,7 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
   if (e != cudaSuccess) return e;
   q.nfull = units - split.ntail;
   q.seg_lo = 1;
-  ssd_tc_kernel<<<(unsigned)(q.nfull + split.ntail * (split.nseg - 1)), kThreads, smem, stream>>>(
+  kern<<<(unsigned)(q.nfull + split.ntail * (split.nseg - 1)), kThreads, smem, stream>>>(
       mX, mB, mC, q);
   return cudaGetLastError();
 }

@@ -160,6 +160,50 @@ ssm_status_t check_ssd(const ssd_scan_args_t *a, size_t *ws, bool shapes_only = 
   return SSM_OK;
 }
 
+// The fused convolution + SSD: the tensor-core configuration only.  The
+// workspace holds the status word, the convolved B and C, then the segment
+// states of a cut last wave.
+struct SsdConvLayout {
+  size_t bc_off = 0, seg_off = 0, total = 0;
+};
+
+SsdConvLayout ssd_conv_layout(const ssd_conv_scan_args_t *a, int sms) {
+  const auto r256 = [](size_t v) { return (v + 255) & ~(size_t)255; };
+  SsdConvLayout l;
+  l.bc_off = kSsdStatusBytes;
+  l.seg_off = l.bc_off + r256(ssm::ssd_conv_bc_bytes(a->batch, a->seqlen, a->groups));
+  l.total = l.seg_off + ssm::ssd_tc_split_bytes(ssm::ssd_tc_split(a->batch, a->heads, a->seqlen, sms));
+  return l;
+}
+
+ssm_status_t check_ssd_conv(const ssd_conv_scan_args_t *a, size_t *ws, bool shapes_only) {
+  if (!a) return SSM_ERR_NULL;
+  if (a->io != SSM_F32 && a->io != SSM_BF16) return SSM_ERR_DTYPE;
+  if (a->batch < 0 || a->seqlen < 0 || a->heads <= 0 || a->head_dim <= 0 ||
+      a->state <= 0 || a->groups <= 0 || a->chunk <= 0 || a->heads % a->groups)
+    return SSM_ERR_SHAPE;
+  if (a->flags & ~SSM_DT_SOFTPLUS) return SSM_ERR_UNSUPPORTED;
+  if (a->io != SSM_BF16 || a->state != 128 || a->head_dim != 64 || a->batch > 65535 ||
+      a->heads > 65535 || a->batch * a->heads >= (1ll << 31) || a->seqlen >= (1ll << 31))
+    return SSM_ERR_UNSUPPORTED;
+  const int64_t ctot = a->heads * a->head_dim + 2 * a->groups * a->state;
+  if (!shapes_only && a->batch > 0 && a->seqlen > 0 &&
+      (!a->xBC || !a->conv_w || !a->dt || !a->A || !a->y))
+    return SSM_ERR_NULL;
+  if (!shapes_only &&
+      !all_aligned(a->xBC, a->conv_w, a->conv_bias, a->conv_state_in, a->conv_state_out, a->z,
+                   a->dt, a->A, a->D, a->dt_bias, a->h0, a->y, a->h_last, a->workspace))
+    return SSM_ERR_ALIGN;
+  if (!shapes_only && a->conv_state_in && a->conv_state_out) {
+    const uintptr_t i0 = reinterpret_cast<uintptr_t>(a->conv_state_in);
+    const uintptr_t o0 = reinterpret_cast<uintptr_t>(a->conv_state_out);
+    const uintptr_t n = (uintptr_t)(a->batch * ctot * 3) * sizeof(float);
+    if (n && i0 < o0 + n && o0 < i0 + n) return SSM_ERR_SHAPE;
+  }
+  *ws = ssd_conv_layout(a, ssm::device_sm_count()).total;
+  return SSM_OK;
+}
+
 }  // namespace
 
 namespace ssm {
@@ -298,6 +342,67 @@ ssm_status_t ssd_chunk_scan_fwd(const ssd_scan_args_t *a, void *stream) {
                                         static_cast<char *>(a->workspace) + kSsdStatusBytes, s));
   }
   return from_cuda(ssm::launch_m2_recurrent(p, s));
+}
+
+ssm_status_t ssd_conv_chunk_scan_workspace(const ssd_conv_scan_args_t *a, size_t *bytes) {
+  if (!bytes) return SSM_ERR_NULL;
+  size_t ws = 0;
+  ssm_status_t st = check_ssd_conv(a, &ws, true);
+  if (st == SSM_OK) *bytes = ws;
+  return st;
+}
+
+ssm_status_t ssd_conv_chunk_scan_fwd(const ssd_conv_scan_args_t *a, void *stream) {
+  size_t ws = 0;
+  ssm_status_t st = check_ssd_conv(a, &ws, false);
+  if (st != SSM_OK) return st;
+  if (a->batch == 0) return SSM_OK;  // nothing to do, nothing launched
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t ctot = a->heads * a->head_dim + 2 * a->groups * a->state;
+  if (a->seqlen == 0) {  // both states pass through unchanged
+    st = pass_state(a->h0, a->h_last,
+                    (size_t)(a->batch * a->heads * a->state * a->head_dim) * sizeof(float), s);
+    if (st != SSM_OK) return st;
+    return pass_state(a->conv_state_in, a->conv_state_out,
+                      (size_t)(a->batch * ctot * 3) * sizeof(float), s);
+  }
+  if (!a->workspace || a->workspace_bytes < ws) return SSM_ERR_WORKSPACE;
+  const int sms = ssm::device_sm_count();
+  const SsdConvLayout l = ssd_conv_layout(a, sms);
+  ssm::M2Params p;
+  p.batch = a->batch;
+  p.L = a->seqlen;
+  p.H = a->heads;
+  p.P = a->head_dim;
+  p.N = a->state;
+  p.G = a->groups;
+  p.flags = a->flags;
+  p.io = a->io;
+  p.x = nullptr;
+  p.z = a->z;
+  p.dt = a->dt;
+  p.B = nullptr;
+  p.Cm = nullptr;
+  p.A = a->A;
+  p.D = a->D;
+  p.dt_bias = a->dt_bias;
+  p.h0 = a->h0;
+  p.y = a->y;
+  p.h_last = a->h_last;
+  p.states = nullptr;
+  ssm::SsdConv conv;
+  conv.xbc = a->xBC;
+  conv.ctot = ctot;
+  conv.w = a->conv_w;
+  conv.bias = a->conv_bias;
+  conv.state_in = a->conv_state_in;
+  conv.state_out = a->conv_state_out;
+  char *w = static_cast<char *>(a->workspace);
+  conv.bc = w + l.bc_off;
+  int *status = reinterpret_cast<int *>(w);
+  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return SSM_ERR_CUDA;
+  const ssm::SsdSplit split = ssm::ssd_tc_split(a->batch, a->heads, a->seqlen, sms);
+  return from_cuda(ssm::launch_ssd_tc(p, status, split, w + l.seg_off, s, &conv));
 }
 
 ssm_status_t ssm_scan_step(const ssm_step_args_t *a, void *stream) {

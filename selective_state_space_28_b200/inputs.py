@@ -38,8 +38,9 @@ RMS_DT = 4
 
 @dataclass(frozen=True)
 class Workload:
-    """One named scan workload.  ``kind`` is "m1", "ssd", "decode", "conv", "gnorm"
-    or "attn" (the SSD map's hidden attention; its inputs are the SSD's)."""
+    """One named scan workload.  ``kind`` is "m1", "ssd", "ssd_conv" (the SSD
+    with the mixer's convolution in front), "decode", "conv", "gnorm" or
+    "attn" (the SSD map's hidden attention; its inputs are the SSD's)."""
     name: str
     kind: str
     batch: int
@@ -110,6 +111,13 @@ WORKLOADS = {
     "conv_2p7b_b4_l4096_c5376_bf16": Workload(
         "conv_2p7b_b4_l4096_c5376_bf16", "conv", batch=4, seqlen=4096, channels=5376,
         io="bf16", seed=5, extra={"width": 4, "state": True}),
+    # The SSD workload with the mixer's causal convolution fused in front:
+    # xBC of 5120 + 2 x 128 channels before the convolution, a carried conv
+    # state.
+    "ssd_conv_2p7b_b4_l4096_h80_p64_n128_bf16": Workload(
+        "ssd_conv_2p7b_b4_l4096_h80_p64_n128_bf16", "ssd_conv", batch=4, seqlen=4096,
+        heads=80, head_dim=64, state=128, chunk=256, io="bf16", gate=False, seed=10,
+        extra={"state": True}),
     # The Mamba-2 2.7B mixer's gated norm after the SSD workload: one row of
     # heads x head_dim = 5120 values per token.
     "gnorm_2p7b_b4_l4096_w5120_bf16": Workload(
@@ -237,6 +245,29 @@ def conv_inputs(batch, seqlen, channels, width=4, io="bf16", seed=0, state=False
     return out
 
 
+def ssd_conv_inputs(batch, seqlen, heads, head_dim, state, groups=1, io="bf16", gate=False,
+                    seed=0, h0=False, state_in=False, bias=True, device="cpu"):
+    """Inputs of one Mamba-2 mixer prologue + SSD: the SSD's own inputs (dt,
+    z, A, D, dt_bias, h0, drawn as ssd_inputs draws them) with x, B and C
+    replaced by xBC [b, L, heads*head_dim + 2*groups*state] before the
+    convolution, the width-4 kernel and bias (U(-1/2, 1/2): the Conv1d
+    default bound for 4 taps) and, optionally, a conv state holding earlier
+    inputs (values of the I/O type, as a previous call leaves them)."""
+    out = ssd_inputs(batch, seqlen, heads, head_dim, state, groups, io, gate, seed, h0,
+                     device)
+    for k in ("x", "B", "C"):
+        del out[k]
+    g = _gen(seed + 7, device)
+    ctot = heads * head_dim + 2 * groups * state
+    out["xBC"] = _randn((batch, seqlen, ctot), g, _dtype(io), device)
+    out["conv_w"] = torch.rand((ctot, 4), generator=g, dtype=torch.float32, device=device) - 0.5
+    cb = torch.rand((ctot,), generator=g, dtype=torch.float32, device=device) - 0.5
+    out["conv_bias"] = cb if bias else None
+    out["conv_state"] = (_randn((batch, ctot, 3), g, _dtype(io), device).float()
+                         if state_in else None)
+    return out
+
+
 def gnorm_inputs(batch, seqlen, width, io="bf16", seed=0, gate=True, weight=True,
                  device="cpu"):
     """Inputs of one gated norm: y, z [b, L, width], weight [width]."""
@@ -259,6 +290,10 @@ def workload_inputs(w: Workload, device="cpu", seed: Optional[int] = None):
                           w.io, w.gate, s, device=device)
     if w.kind == "gnorm":
         return gnorm_inputs(w.batch, w.seqlen, w.channels, w.io, s, gate=w.gate, device=device)
+    if w.kind == "ssd_conv":
+        return ssd_conv_inputs(w.batch, w.seqlen, w.heads, w.head_dim, w.state, w.groups,
+                               w.io, w.gate, s, state_in=w.extra.get("state", False),
+                               device=device)
     if w.kind == "conv":
         return conv_inputs(w.batch, w.seqlen, w.channels, w.extra.get("width", 4), w.io, s,
                            state=w.extra.get("state", False), device=device)

@@ -156,6 +156,14 @@ def ssd_workspace_bytes(**shape):
     return n.value
 
 
+def ssd_conv_workspace_bytes(**shape):
+    a = L.SsdConvArgs(**shape)
+    n = ctypes.c_size_t(0)
+    L.check(L.lib().ssd_conv_chunk_scan_workspace(ctypes.byref(a), ctypes.byref(n)),
+            "ssd_conv_chunk_scan_workspace")
+    return n.value
+
+
 def ssd_chunk_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
                        chunk=256, flags=SOFTPLUS, want_states=False, y=None, h_last=None,
                        workspace=None, check=False, stream=None):
@@ -191,6 +199,48 @@ def ssd_chunk_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
     if nbytes.value and (check or sg.host or _CHECK_ALL):
         _check_status(workspace, st, "ssd_chunk_scan_fwd")
     return sg.back((y, h_last, states))
+
+
+def ssd_conv_chunk_scan_fwd(xBC, conv_w, dt, A, *, heads, state, groups=1, conv_bias=None,
+                            conv_state_in=None, want_conv_state=False, D=None, z=None,
+                            dt_bias=None, h0=None, chunk=256, flags=SOFTPLUS, y=None,
+                            h_last=None, conv_state_out=None, workspace=None, check=False,
+                            stream=None):
+    """The Mamba-2 mixer's causal convolution fused in front of the SSD scan
+    (include/ssm.h, ssd_conv_chunk_scan_fwd).
+
+    xBC: [b, L, heads*64 + 2*groups*state] bf16, before the convolution;
+    conv_w: [channels, 4] f32; conv_bias: [channels]; conv_state_in:
+    [b, channels, 3] f32; dt: [b, L, H]; z: [b, L, H, 64]; A, D, dt_bias: [H];
+    h0: [b, H, N, 64].  Returns (y, h_last, conv_state_out or None)."""
+    sg = _Staging([xBC, conv_w, dt, A, conv_bias, conv_state_in, D, z, dt_bias, h0])
+    xBC, conv_w, dt, A, conv_bias, conv_state_in, D, z, dt_bias, h0 = map(
+        sg.dev, (xBC, conv_w, dt, A, conv_bias, conv_state_in, D, z, dt_bias, h0))
+    b, Lq, ctot = xBC.shape
+    P = (ctot - 2 * groups * state) // heads
+    if y is None:
+        y = torch.empty((b, Lq, heads, P), dtype=xBC.dtype, device=xBC.device)
+    if h_last is None:
+        h_last = torch.empty((b, heads, state, P), dtype=torch.float32, device=xBC.device)
+    if conv_state_out is None and want_conv_state:
+        conv_state_out = torch.empty((b, ctot, 3), dtype=torch.float32, device=xBC.device)
+    a = L.SsdConvArgs(batch=b, seqlen=Lq, heads=heads, head_dim=P, state=state, groups=groups,
+                      chunk=chunk, io=_io_of(xBC), flags=flags, xBC=_ptr(xBC),
+                      conv_w=_ptr(conv_w), conv_bias=_ptr(conv_bias),
+                      conv_state_in=_ptr(conv_state_in), conv_state_out=_ptr(conv_state_out),
+                      z=_ptr(z), dt=_ptr(dt), A=_ptr(A), D=_ptr(D), dt_bias=_ptr(dt_bias),
+                      h0=_ptr(h0), y=_ptr(y), h_last=_ptr(h_last))
+    lib = L.lib()
+    nbytes = ctypes.c_size_t(0)
+    L.check(lib.ssd_conv_chunk_scan_workspace(ctypes.byref(a), ctypes.byref(nbytes)),
+            "ssd_conv_chunk_scan_workspace")
+    workspace = _workspace(nbytes.value, workspace, xBC.device)
+    a.workspace, a.workspace_bytes = workspace.data_ptr(), nbytes.value
+    st = _stream(stream, xBC.device)
+    L.check(lib.ssd_conv_chunk_scan_fwd(ctypes.byref(a), st), "ssd_conv_chunk_scan_fwd")
+    if Lq and (check or sg.host or _CHECK_ALL):
+        _check_status(workspace, st, "ssd_conv_chunk_scan_fwd")
+    return sg.back((y, h_last, conv_state_out))
 
 
 def ssm_scan_step(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, *, flags=SOFTPLUS,

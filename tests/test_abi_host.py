@@ -26,7 +26,8 @@ def test_exports_every_declared_symbol(lib):
             "ssd_chunk_scan_workspace", "ssm_scan_step", "ssm_status_string",
             "ssm_abi_version", "ssm_conv1d_fwd", "ssm_scan_fwd_static",
             "ssm_gated_rmsnorm_fwd", "ssm_scan_fwd_write", "ssd_attention_fwd",
-            "ssd_attention_workspace", "ssm_workspace_status"} <= set(names)
+            "ssd_attention_workspace", "ssm_workspace_status", "ssd_conv_chunk_scan_fwd",
+            "ssd_conv_chunk_scan_workspace"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], check=True,
                          capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
@@ -44,7 +45,7 @@ def test_no_runtime_symbols_leak(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.ssm_abi_version() == 2
+    assert lib.ssm_abi_version() == 3
     for s in range(9):
         assert lib.ssm_status_string(s)
     assert lib.ssm_status_string(99) == b"unknown status"
@@ -314,3 +315,31 @@ def test_empty_calls_launch_nothing(lib):
         t = _attn(dt=None, B=None, C=None, A=None, alpha=None, workspace=None,
                   workspace_bytes=0, **kw)
         assert lib.ssd_attention_fwd(ctypes.byref(t), None) == OK
+
+
+def test_fused_conv_ssd_rejects_before_launch(lib):
+    """ssd_conv_chunk_scan_fwd: host checks only (no device is touched)."""
+    ctot = 4 * 64 + 2 * 128
+    a = L.SsdConvArgs(batch=1, seqlen=8, heads=4, head_dim=64, state=128, groups=1, chunk=256,
+                      io=L.SSM_BF16, flags=1, xBC=16, conv_w=16, dt=16, A=16, y=16,
+                      conv_state_in=4096, conv_state_out=4096 + 16)
+    n = ctypes.c_size_t(0)
+    assert lib.ssd_conv_chunk_scan_workspace(ctypes.byref(a), ctypes.byref(n)) == 0
+    # status word, then the convolved B and C (8 tokens x 256 channels bf16)
+    assert n.value == 256 + 4096
+    assert lib.ssd_conv_chunk_scan_fwd(ctypes.byref(a), None) == 2   # the states overlap
+    a.conv_state_out = 4096 + ctot * 3 * 4
+    assert lib.ssd_conv_chunk_scan_fwd(ctypes.byref(a), None) == 6   # no workspace
+    a.xBC = None
+    assert lib.ssd_conv_chunk_scan_fwd(ctypes.byref(a), None) == 1   # NULL xBC
+    a.xBC = 24
+    assert lib.ssd_conv_chunk_scan_fwd(ctypes.byref(a), None) == 4   # misaligned
+    a.xBC = 16
+    for field, value, code in (("state", 64, 5), ("head_dim", 32, 5), ("io", 0, 5),
+                               ("io", 7, 3), ("groups", 3, 2), ("flags", 2, 5)):
+        old = getattr(a, field)
+        setattr(a, field, value)
+        assert lib.ssd_conv_chunk_scan_fwd(ctypes.byref(a), None) == code, field
+        setattr(a, field, old)
+    a.batch = 0
+    assert lib.ssd_conv_chunk_scan_fwd(ctypes.byref(a), None) == 0   # nothing to do
