@@ -22,7 +22,8 @@
 //                 Sc = B^T (w o x)           A = B read MN-major (two buffers)
 //                 Y  = M x + (e o C) h_prev  A = M and e o C from TMEM, both
 //                                            held in S's columns (two buffers)
-//               issued per tile in the order Sc(c), S(c+1), Y(c).
+//               per tile Sc(c) and S(c+1) in whichever order their inputs
+//               arrive, then Y(c).
 //   warps 4-7 and 14-17   mask group, thread = token, two warps per TMEM
 //               lane quarter each taking half of every row's work (each warp
 //               also recomputes the whole tile's decay factors, so the warps
@@ -30,9 +31,10 @@
 //               a_j = exp(d_j A), and every factor exp(cum_i - cum_j) as the
 //               product a_{j+1} .. a_i (never as the exponential of a
 //               difference of running sums, which would lose a small step
-//               beside a large sum); w o x; then the mask applied to S as it
-//               is read from TMEM (D on its diagonal, so Y holds D x), and
-//               the row-scaled C, e_i C_i with e_i = a_0 .. a_i, both written
+//               beside a large sum); it publishes the column factor w_j for
+//               the output group; then the mask applied to S as it is read
+//               from TMEM (D on its diagonal, so Y holds D x), and the
+//               row-scaled C, e_i C_i with e_i = a_0 .. a_i, both written
 //               back as the bf16 A operand of Y.  The mask is elementwise on
 //               the four 32 x 32 diagonal blocks (a running product down from
 //               the diagonal); below them it is a row factor times a column
@@ -40,19 +42,25 @@
 //   warps 0-3   state group: thread n keeps row n of the float32 state in
 //               registers, h = exp(cum_last) h + Sc, and writes its bf16 copy
 //               for Y of the next tile (two buffers).
-//   warps 8-11  output group, thread = token: y = Y (* silu(z)), with z
-//               fetched one tile ahead.  In the fused form (the mixer's
-//               causal convolution in front, "Mamba-2", the module tree and
-//               "The mixer's values": x, B, C = silu(conv1d(xBC))), the
-//               group first convolves each landed x tile in place, a tile
-//               ahead of the mask group: token i from rows i-3..i, the three
-//               rows before the tile kept from the previous tile's raw
-//               inputs; B and C, which every head of a group shares, are
-//               convolved once by ssd_bc_conv_kernel before the scan.
+//   warps 8-11  output group: w o x of the next tile (the B operand of Sc,
+//               from the landed x and the mask group's w_j), then y = Y
+//               (* silu(z)) of this tile, thread = token.  In the fused form
+//               (the mixer's causal convolution in front, "Mamba-2", the
+//               module tree and "The mixer's values": x, B, C =
+//               silu(conv1d(xBC))), the same pass first convolves the landed
+//               x tile in place: thread (4 channels, 16 tokens) walks its
+//               tokens with the three previous raw inputs in registers, the
+//               three rows before the tile kept from the previous tile.  The
+//               mask group never reads x, so the convolution runs beside the
+//               S product and the mask.  B and C, which every head of a
+//               group shares, are convolved once by ssd_bc_conv_kernel
+//               before the scan.
 // With Y, Sc and the bf16 state double-buffered, the only chain carried from
 // tile to tile is the state group's update; every other role has a tile of
 // slack, and the contractions of the next tile run under this tile's
-// elementwise work.
+// elementwise work.  Signals: full/empty (stages), wready (w_j and the tile
+// decay, mask -> output and state groups, four deep), xready (w o x, output
+// -> MMA), sdone/scdone/yready (MMA commits), mready, stdone, yfree.
 //
 // A CTA runs either a whole (batch, head) unit or a segment of its tiles:
 // when the last wave of units is partial, the host cuts those units into
@@ -100,17 +108,20 @@ struct __align__(1024) SsdSmem {
   float ppw[8][kQ];           //   a_b ... a_j (b the first token of j's 32-token block),
   float ddw[8][kQ];           //   step d_j,
   float vdw[8][kQ];           //   a_{j+1} ... a_{b+31} d_j (column factor of the mask)
-  // With the convolution fused: the three inputs before a tile (bf16, 64
-  // channels), two buffers by tile parity.  (Fits in the struct's alignment
-  // padding: the size is unchanged.)
-  __nv_bfloat16 halo[2][3][kP];
+  // The column factor w_j of the tile's tokens (bf16, as the w o x product
+  // uses it), from the mask group to the output group; two buffers by tile
+  // parity.
+  __nv_bfloat16 wt[2][kQ];
+  // With the convolution fused: the three raw inputs before a tile (bf16,
+  // 64 channels).
+  __nv_bfloat16 halo[3][kP];
   float a[4];                 // exp(cum_last) = a_0 .. a_127 per tile, ring of four
-  // Per-tile signals come in pairs indexed by tile parity (xready in fours);
+  // Per-tile signals come in pairs indexed by tile parity (wready in fours);
   // the dependencies between roles bound every waiter's lag to less than one
   // lap of its ring, so no waiter can miss a phase.
   uint64_t full[2], empty[2], sdone[2], scdone[2], mready[2], stdone[2], yready[2], yfree[2];
-  uint64_t xready[4];
-  uint64_t xconv[2];          // x of a tile convolved in place (fused form)
+  uint64_t xready[2];         // w o x written (output group)
+  uint64_t wready[4];         // w_j and the tile decay written (mask group)
   uint32_t taddr;
   int abort;
 };
@@ -310,8 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.yready[i], 1);
       mbar_init(&s.yfree[i], 4);   // one arrival per output-group warp
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&s.xready[i], 8);
-    for (int i = 0; i < 2; ++i) mbar_init(&s.xconv[i], 4);  // one arrival per output warp
+    for (int i = 0; i < 2; ++i) mbar_init(&s.xready[i], 4);  // one arrival per output warp
+    for (int i = 0; i < 4; ++i) mbar_init(&s.wready[i], 4);  // one per half-0 mask warp
     s.abort = 0;
     fence_mbar_init();
   }
@@ -413,22 +424,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; ok && c < nch; ++c) {
       const int k = c & 1;
       const uint32_t ph = (c >> 1) & 1;
-      // Sc(c) = B^T (w o x): needs w o x of tile c
-      if (!waitw(s, &s.xready[c & 3], (c >> 2) & 1, p.status, 3)) break;
-      tc_fence_after();
-      if (leader) {
+      // Sc(c) = B^T (w o x) once w o x of tile c is written, and S(c+1) once
+      // the next tile has landed, in whichever order their inputs arrive
+      // (both only have to follow Y(c-1)): the lanes poll both barriers
+      // (bounded), and a barrier counts as passed when every lane has seen
+      // it, so the warp decides together.
+      bool need_sc = true, need_s = c + 1 < nch;
+      const long long tw = clock64();
+      while (need_sc || need_s) {
+        if (need_sc && __all_sync(0xffffffffu, mbar_try(smem_u32(&s.xready[k]), ph))) {
+          tc_fence_after();
+          if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tb + kColSc + 64 * k, dBm[k] + kk * 128, dXw + kk * 128, id_Sc, kk > 0);
-        mma_commit(&s.scdone[k]);
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tb + kColSc + 64 * k, dBm[k] + kk * 128, dXw + kk * 128, id_Sc, kk > 0);
+            mma_commit(&s.scdone[k]);
+          }
+          __syncwarp();
+          last_bar = &s.scdone[k];
+          last_par = ph;
+          need_sc = false;
+          continue;
+        }
+        if (need_s &&
+            __all_sync(0xffffffffu, mbar_try(smem_u32(&s.full[k ^ 1]), ((c + 1) >> 1) & 1))) {
+          mma_S(c + 1);
+          need_s = false;
+          continue;
+        }
+        if (__any_sync(0xffffffffu, clock64() - tw > kWaitLimit)) break;
       }
-      __syncwarp();
-      last_bar = &s.scdone[k];
-      last_par = ph;
-      // S(c+1), as soon as its tile has landed
-      if (c + 1 < nch) {
-        if (!waitw(s, &s.full[k ^ 1], ((c + 1) >> 1) & 1, p.status, 4)) break;
-        mma_S(c + 1);
+      if (need_sc || need_s) {
+        if (lane == 0) set_abort(s, p.status, need_sc ? 3 : 4);
+        break;
       }
       // Y(c) = M x + (e o C) h_prev: needs the mask group's operands, the
       // state of tile c-1 in Hb, and Y[k] read out by the output group
@@ -459,10 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ mask group
     // Two warps per TMEM lane quarter (warps 4-7 and 14-17): each takes 32
     // rows and, of every row, half the work (16 of each 32-column block of
-    // the mask, one 64-state slab of e o C, half of w o x).  Each warp keeps
-    // its own copy of the tile's per-token factors, so the eight warps never
-    // wait for each other; they meet only in the eight-count xready and
-    // mready barriers.
+    // the mask, one 64-state slab of e o C).  Each warp keeps its own copy
+    // of the tile's per-token factors, so the eight warps never wait for
+    // each other; they meet only in the eight-count mready barrier.  They
+    // do not read x: the output group forms w o x from the w_j published
+    // here, so the convolution of the fused form runs beside S and the mask.
     const int half = warp >= 14 ? 1 : 0;
     const int mw = warp & 3;           // lane quarter = row block
     const int mg = 4 * half + mw;      // this warp's factor copy
@@ -550,28 +579,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float pp_i = ppw[i];
       const float e_i = pp_i * before_blk;
       const float w_i = vdw[i] * after_blk;
-      // w o x (this warp's rows, half the columns), the B operand of Sc(c):
-      // x of tile c has landed (and, fused, been convolved in place) and
-      // Sc(c-1) is done with the buffer
-      if (!waitw(s, &s.full[k], (c >> 1) & 1, p.status, 8)) break;
-      if (CONV && !waitw(s, &s.xconv[k], (c >> 1) & 1, p.status, 15)) break;
-      if (c >= 1 && !waitw(s, &s.scdone[k ^ 1], ((c - 1) >> 1) & 1, p.status, 9)) break;
-      {
-        const uint32_t w2 = pack_bf16x2(w_i, w_i);
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int cc = 4 * half + c4;
-          const uint4 v = *reinterpret_cast<const uint4 *>(s.X[k] + sw128(i, cc));
-          *reinterpret_cast<uint4 *>(s.Xw + sw128(i, cc)) =
-              make_uint4(bmul2(v.x, w2), bmul2(v.y, w2), bmul2(v.z, w2), bmul2(v.w, w2));
-        }
-      }
-      fence_async_smem();
+      // w_i for the output group's w o x (bf16, as the product uses it), and
+      // with it the tile decay above: one arrival per half-0 warp
+      if (half == 0) reinterpret_cast<uint16_t *>(s.wt[k])[i] = (uint16_t)pack_bf16x2(w_i, 0.f);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.xready[c & 3]);
-      // next tile's dt, issued after the proxy fence so the fence never
-      // waits for it; it has the rest of this tile to arrive
+      if (half == 0 && lane == 0) mbar_arrive(&s.wready[c & 3]);
+      // next tile's dt: it has the rest of this tile to arrive
       if (c + 1 < nch) fetch_dt(c + 1);
+      // C of tile c (for e o C) has landed
+      if (!waitw(s, &s.full[k], (c >> 1) & 1, p.status, 8)) break;
       // masked S -> bf16.  Of each 32-column block J this warp takes the 16
       // columns from 32 J + 16 half.  Its packed results go only where this
       // warp itself has already read S (its own halves of blocks 0 and 1),
@@ -696,8 +712,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; c < nch; ++c) {
       const int k = c & 1;
       // h = a h + Sc (thread = row n); a comes from the mask group, whose
-      // xready arrival orders its write before this read
-      if (!waitw(s, &s.xready[c & 3], (c >> 2) & 1, p.status, 11)) break;
+      // wready arrival orders its write before this read
+      if (!waitw(s, &s.wready[c & 3], (c >> 2) & 1, p.status, 11)) break;
       if (!waitw(s, &s.scdone[k], (c >> 1) & 1, p.status, 12)) break;
       tc_fence_after();
       const float a_c = s.a[c & 3];
@@ -745,6 +761,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const __nv_bfloat16 *zp = p.z + ((b * L + t) * H + hd) * kP;
 #pragma unroll
         for (int q = 0; q < 8; ++q) zr[q] = ld_cs_u4(zp + 8 * q);
+      } else if (CONV) {
+        // (assigned on every path, so the previous tile's values are dead
+        // while the next tile's convolution runs)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) zr[q] = make_uint4(0u, 0u, 0u, 0u);
       }
     };
     // A wait of this group: voted per warp, or, fused, over the four warps
@@ -757,18 +778,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       return !fail;
     };
     // Fused form: the causal convolution of x over tokens, then silu, in
-    // place in the landed tile (the three rows before the tile from the
-    // previous tile's raw inputs, kept in `halo`, or for the first tile of
-    // this CTA from xBC or the conv state); one named barrier between the
-    // reads every thread needs from its neighbour's rows and the writes.
-    auto conv_tile = [&](int c) -> bool {
+    // place in the landed tile c, as soon as it lands (the three rows before
+    // the tile from the previous tile's raw inputs, kept in `halo`, or for
+    // the first tile of this CTA from xBC or the conv state).  Thread (cq,
+    // tg): channels 4 cq .. + 4 of the head, tokens 16 tg .. + 16 of the
+    // tile, walked in order with the three previous raw inputs in registers
+    // (every row read once); one barrier between the reads every thread
+    // needs from its neighbour's rows and the in-place writes.
+    auto conv_x = [&](int c) -> bool {
       const int k = c & 1;
       const int64_t t0 = (int64_t)(cb + c) * kQ;
       const int64_t ch0 = hd * kP;
       // Before this CTA's first tile the three preceding inputs come from
-      // global memory, widened to float32 into the w o x buffer: nobody uses
-      // it before the mask group's first write, which waits for this tile's
-      // xconv.
+      // global memory, widened to float32 into the w o x buffer (free until
+      // this group's own first w o x writes).
       const float *first = reinterpret_cast<const float *>(s.Xw);
       if (c == 0) {
         const uint16_t *xr = reinterpret_cast<const uint16_t *>(p.xbc);
@@ -782,87 +805,115 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         out_group_sync();
       }
-      // Thread (cq, tg): channels 4 cq .. + 4 of the head, tokens 16 tg ..
-      // + 16 of the tile, walked in order with the three previous raw inputs
-      // in registers (every row read once).  Its weights and bias first:
-      // their loads overlap the wait for the tile.
       const int cq = i & 15, tg = i >> 4;
       const uint32_t qoff = 8u * (uint32_t)(cq & 1);  // the quad within its 16-byte chunk
-      float wq[4][4], bq[4];
+      // weights and bias of the thread's channels as pairs (0, 1), (2, 3);
+      // their loads overlap the wait for the tile
+      f2 wt3[2], wt2[2], wt1[2], wt0[2], bs[2];
       {
         const float4 *wv = reinterpret_cast<const float4 *>(p.cw + (ch0 + 4 * cq) * 4);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float4 w = __ldg(wv + e);
-          wq[e][0] = w.x; wq[e][1] = w.y; wq[e][2] = w.z; wq[e][3] = w.w;
-          bq[e] = p.cbias ? __ldg(p.cbias + ch0 + 4 * cq + e) : 0.f;
-        }
+        const float4 w0 = __ldg(wv), w1 = __ldg(wv + 1), w2 = __ldg(wv + 2), w3 = __ldg(wv + 3);
+        wt0[0] = mk2(w0.x, w1.x); wt1[0] = mk2(w0.y, w1.y); wt2[0] = mk2(w0.z, w1.z);
+        wt3[0] = mk2(w0.w, w1.w);
+        wt0[1] = mk2(w2.x, w3.x); wt1[1] = mk2(w2.y, w3.y); wt2[1] = mk2(w2.z, w3.z);
+        wt3[1] = mk2(w2.w, w3.w);
+        const float *bp = p.cbias + ch0 + 4 * cq;
+        bs[0] = p.cbias ? mk2(__ldg(bp), __ldg(bp + 1)) : mk2(0.f, 0.f);
+        bs[1] = p.cbias ? mk2(__ldg(bp + 2), __ldg(bp + 3)) : mk2(0.f, 0.f);
       }
       if (!waito(&s.full[k], (c >> 1) & 1, 14)) return false;
       uint8_t *xs = s.X[k];
-      auto unpack4 = [](uint2 u, float (&v)[4]) {
-        v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+      auto unpack2 = [](uint2 u, f2 (&v)[2]) {
+        v[0] = mk2(bf16lo(u.x), bf16hi(u.x));
+        v[1] = mk2(bf16lo(u.y), bf16hi(u.y));
       };
       // the three raw rows before this thread's first token: the previous
       // group's rows (read before anyone overwrites them), the previous
       // tile's last rows (`halo`), or before this CTA's first tile `first`
-      float win[3][4];
+      f2 win[3][2];
 #pragma unroll
       for (int j = 0; j < 3; ++j) {
         const int r = 16 * tg - 3 + j;
         if (r >= 0) {
-          unpack4(*reinterpret_cast<const uint2 *>(xs + sw128(r, cq >> 1) + qoff), win[j]);
+          unpack2(*reinterpret_cast<const uint2 *>(xs + sw128(r, cq >> 1) + qoff), win[j]);
         } else if (c > 0) {
-          unpack4(*reinterpret_cast<const uint2 *>(&s.halo[k][r + 3][4 * cq]), win[j]);
+          unpack2(*reinterpret_cast<const uint2 *>(&s.halo[r + 3][4 * cq]), win[j]);
         } else {
           const float4 f = *reinterpret_cast<const float4 *>(first + (r + 3) * kP + 4 * cq);
-          win[j][0] = f.x; win[j][1] = f.y; win[j][2] = f.z; win[j][3] = f.w;
+          win[j][0] = mk2(f.x, f.y);
+          win[j][1] = mk2(f.z, f.w);
         }
       }
       out_group_sync();  // every window is read: rows may be overwritten now
-#pragma unroll 2
+      const f2 half2 = mk2(0.5f, 0.5f);
+#pragma unroll 4
       for (int j = 0; j < 16; ++j) {
         const int r = 16 * tg + j;
         uint2 *row = reinterpret_cast<uint2 *>(xs + sw128(r, cq >> 1) + qoff);
         const uint2 u = *row;
         // the raw last three rows are the next tile's halo
-        if (tg == 7 && j >= 13) *reinterpret_cast<uint2 *>(&s.halo[k ^ 1][j - 13][4 * cq]) = u;
-        float xv[4];
-        unpack4(u, xv);
-        // u = silu(bias + sum_q w[q] x[t - 3 + q]), the newest input first
-        // (the order of ssm_conv1d_fwd, so both give the same bits)
+        if (tg == 7 && j >= 13) *reinterpret_cast<uint2 *>(&s.halo[j - 13][4 * cq]) = u;
+        f2 xv[2];
+        unpack2(u, xv);
+        // u = silu(bias + sum_q w[q] x[t - 3 + q]), the newest input first,
+        // and silu(z) = z (1 + tanh(z / 2)) / 2: the operations of
+        // ssm_conv1d_fwd lane by lane, so both give the same bits
         const bool live = t0 + r < L;
-        float o[4];
+        uint32_t ov[2];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float acc = fmaf(wq[e][3], xv[e], bq[e]);
-          acc = fmaf(wq[e][2], win[2][e], acc);
-          acc = fmaf(wq[e][1], win[1][e], acc);
-          acc = fmaf(wq[e][0], win[0][e], acc);
-          o[e] = live ? silu_tanh(acc) : 0.f;
-          win[0][e] = win[1][e];
-          win[1][e] = win[2][e];
-          win[2][e] = xv[e];
+        for (int q = 0; q < 2; ++q) {
+          f2 acc = fma2(wt3[q], xv[q], bs[q]);
+          acc = fma2(wt2[q], win[2][q], acc);
+          acc = fma2(wt1[q], win[1][q], acc);
+          acc = fma2(wt0[q], win[0][q], acc);
+          const f2 hz = mul2(half2, acc);
+          float ta, tb2;
+          asm("tanh.approx.f32 %0, %1;" : "=f"(ta) : "f"(hz.x));
+          asm("tanh.approx.f32 %0, %1;" : "=f"(tb2) : "f"(hz.y));
+          const f2 o = mul2(acc, fma2(half2, mk2(ta, tb2), half2));
+          ov[q] = live ? pack_bf16x2(o.x, o.y) : 0u;
+          win[0][q] = win[1][q];
+          win[1][q] = win[2][q];
+          win[2][q] = xv[q];
         }
-        *row = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+        *row = make_uint2(ov[0], ov[1]);
+      }
+      return true;
+    };
+    // w o x of tile c, the B operand of Sc(c) (thread = row), once x has
+    // landed (fused: been convolved), the mask group has published w_j and
+    // Sc(c-1) is done with the buffer.  (Fused, the wready vote is also the
+    // barrier between the convolution's writes and these reads.)
+    auto xprep = [&](int c) -> bool {
+      const int k = c & 1;
+      if (CONV) {
+        if (!conv_x(c)) return false;
+      } else if (!waito(&s.full[k], (c >> 1) & 1, 14)) {
+        return false;
+      }
+      if (!waito(&s.wready[c & 3], (c >> 2) & 1, 15)) return false;
+      if (c >= 1 && !waito(&s.scdone[k ^ 1], ((c - 1) >> 1) & 1, 9)) return false;
+      const uint32_t wb = reinterpret_cast<const uint16_t *>(s.wt[k])[i];
+      const uint32_t w2 = wb | (wb << 16);
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(s.X[k] + sw128(i, cc));
+        *reinterpret_cast<uint4 *>(s.Xw + sw128(i, cc)) =
+            make_uint4(bmul2(v.x, w2), bmul2(v.y, w2), bmul2(v.z, w2), bmul2(v.w, w2));
       }
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.xconv[k]);
+      if (lane == 0) mbar_arrive(&s.xready[k]);
       return true;
     };
-    bool ok = true;
-    if (CONV) ok = nch > 0 && conv_tile(0);
-    else load_z(0);
+    bool ok = nch > 0 && xprep(0);
     for (int c = 0; ok && c < nch; ++c) {
       const int k = c & 1;
       const int64_t t = (int64_t)(cb + c) * kQ + i;
-      if (CONV) {
-        // the next tile's convolution first: the mask group needs it for
-        // tile c + 1 while this tile's Y is still being formed
-        if (c + 1 < nch && !conv_tile(c + 1)) break;
-        load_z(c);
-      }
+      // the next tile's w o x first (and, fused, its convolution): Sc(c+1)
+      // waits for it while this tile's Y is still being formed
+      if (c + 1 < nch && !xprep(c + 1)) break;
+      load_z(c);
       if (!waito(&s.yready[k], (c >> 1) & 1, 13)) break;
       tc_fence_after();
       __nv_bfloat16 *yp = p.y + ((b * L + t) * H + hd) * kP;
@@ -899,7 +950,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!CONV) load_z(c + 1);
     }
   }
 
@@ -935,28 +985,33 @@ __global__ void __launch_bounds__(kCarrySlice / 4)
   }
 }
 
-// The fused call's pre-pass.  (1) The B and C channels of xBC (nbc = 2 G N
-// of them from channel c0 on) convolved over tokens, then silu, into
-// bc [batch][L][nbc]: every head of a group reads the same B and C, so they
-// are convolved once here instead of in each head's CTA (x is convolved
-// inside the scan).  A thread takes one token and eight channels.  (2) The
-// conv state out: the last three inputs of every channel, oldest first
-// (from cs_in where the sequence is shorter than three).
+// The fused call's pre-pass, one batch row per grid row (blockIdx.y).  (1)
+// The B and C channels of xBC (nbc = 2 G N of them from channel c0 on)
+// convolved over tokens, then silu, into bc [batch][L][nbc]: every head of a
+// group reads the same B and C, so they are convolved once here instead of
+// in each head's CTA (x is convolved inside the scan).  A thread takes one
+// token and eight channels.  (2) The blocks after those: the conv state
+// out, the last three inputs of every channel, oldest first (from cs_in
+// where the sequence is shorter than three).  Indices within a row are
+// 32-bit (the host keeps L * nbc / 8 and ctot below 2^31).
 __global__ void __launch_bounds__(256)
-    ssd_bc_conv_kernel(const __nv_bfloat16 *xbc, int64_t batch, int64_t L, int64_t ctot,
-                       int64_t c0, int64_t nbc, const float *cw, const float *cbias,
-                       const float *cs_in, __nv_bfloat16 *bc, float *cs_out) {
-  const int64_t nchunk = nbc / 8, nconv = batch * L * nchunk;
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx < nconv) {
-    const int64_t j = idx % nchunk, bt = idx / nchunk, t = bt % L, bb = bt / L;
-    const int64_t ch = c0 + 8 * j;
+    ssd_bc_conv_kernel(const __nv_bfloat16 *xbc, int64_t L, int64_t ctot, int64_t c0,
+                       int nbc, unsigned conv_blocks, const float *cs_in, const float *cw,
+                       const float *cbias, __nv_bfloat16 *bc, float *cs_out) {
+  const int64_t bb = blockIdx.y;
+  const unsigned nchunk = (unsigned)nbc / 8u;
+  if (blockIdx.x < conv_blocks) {
+    const unsigned idx = blockIdx.x * 256u + threadIdx.x;
+    const unsigned t = idx / nchunk, j = idx - t * nchunk;
+    if (t >= (unsigned)L) return;
+    const int64_t ch = c0 + 8 * (int64_t)j;
+    const __nv_bfloat16 *xrow = xbc + (bb * L + t) * ctot + ch;
     float v[4][8];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int64_t tau = t - 3 + q;
+      const int tau = (int)t - 3 + q;
       if (tau >= 0) {
-        unpack8(ld_nc_u4(xbc + (bb * L + tau) * ctot + ch), v[q]);
+        unpack8(ld_nc_u4(xrow - (int64_t)(3 - q) * ctot), v[q]);
       } else if (cs_in) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[q][e] = cs_in[(bb * ctot + ch + e) * 3 + (tau + 3)];
@@ -981,9 +1036,8 @@ __global__ void __launch_bounds__(256)
                    pack_bf16x2(o[6], o[7]));
     return;
   }
-  const int64_t r = idx - nconv;
-  if (!cs_out || r >= batch * ctot) return;
-  const int64_t c = r % ctot, bb = r / ctot;
+  const unsigned c = (blockIdx.x - conv_blocks) * 256u + threadIdx.x;
+  if (!cs_out || c >= (unsigned)ctot) return;
   const uint16_t *xr = reinterpret_cast<const uint16_t *>(xbc);
 #pragma unroll
   for (int q = 0; q < 3; ++q) {
@@ -1100,10 +1154,11 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
     if (e != cudaSuccess) return e;
   }
   if (conv) {
-    const int64_t threads = p.batch * p.L * (2 * GN / 8) + p.batch * conv->ctot;
-    ssd_bc_conv_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(conv->xbc), p.batch, p.L, conv->ctot, p.H * kP,
-        2 * GN, conv->w, conv->bias, conv->state_in, static_cast<__nv_bfloat16 *>(conv->bc),
+    const unsigned conv_blocks = (unsigned)((p.L * (2 * GN / 8) + 255) / 256);
+    const unsigned state_blocks = conv->state_out ? (unsigned)((conv->ctot + 255) / 256) : 0u;
+    ssd_bc_conv_kernel<<<dim3(conv_blocks + state_blocks, (unsigned)p.batch), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(conv->xbc), p.L, conv->ctot, p.H * kP, (int)(2 * GN),
+        conv_blocks, conv->state_in, conv->w, conv->bias, static_cast<__nv_bfloat16 *>(conv->bc),
         conv->state_out);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -183,8 +183,11 @@ ssm_status_t check_ssd_conv(const ssd_conv_scan_args_t *a, size_t *ws, bool shap
       a->state <= 0 || a->groups <= 0 || a->chunk <= 0 || a->heads % a->groups)
     return SSM_ERR_SHAPE;
   if (a->flags & ~SSM_DT_SOFTPLUS) return SSM_ERR_UNSUPPORTED;
+  // (the convolution pre-pass indexes a batch row's tokens x 8-channel
+  // chunks in 32 bits)
   if (a->io != SSM_BF16 || a->state != 128 || a->head_dim != 64 || a->batch > 65535 ||
-      a->heads > 65535 || a->batch * a->heads >= (1ll << 31) || a->seqlen >= (1ll << 31))
+      a->heads > 65535 || a->batch * a->heads >= (1ll << 31) ||
+      a->seqlen * a->groups * 32 >= (1ll << 31))
     return SSM_ERR_UNSUPPORTED;
   const int64_t ctot = a->heads * a->head_dim + 2 * a->groups * a->state;
   if (!shapes_only && a->batch > 0 && a->seqlen > 0 &&
