@@ -876,7 +876,8 @@ def run_ours(args):
                     "x written and read back (B and C still make one round trip)",
             "roofline": {"bound": "tensor", "achieved": round(tf, 2),
                          "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": round(tf / pk["bf16_tflops"], 4), "traffic": None,
+                         "frac": round(tf / pk["bf16_tflops"], 4),
+                         "traffic": traffic_for("ssd_conv_2p7b"),
                          "flops_per_launch": sc["flops"], "bytes_per_launch": sc["bytes"],
                          "hbm_frac": round(sc["bytes"] / (sc["launch_ms"] * 1e-3) / 1e9 / hbm,
                                            4)}}
