@@ -90,7 +90,9 @@ using namespace sm100;
 constexpr int kQ = 128;   // tokens per tile
 constexpr int kN = 128;   // state size
 constexpr int kP = 64;    // head dim
-constexpr int kThreads = 576;  // 18 warps
+constexpr int kThreads = 576;  // 18 warps; the fused form adds two (640)
+template <bool CONV>
+constexpr int threads_of() { return CONV ? kThreads + 64 : kThreads; }
 constexpr long long kWaitLimit = 2000000000ll;  // cycles (about a second)
 
 // TMEM columns: S[2] (fp32 S; then masked S in the first 64 columns and e o C
@@ -109,9 +111,11 @@ struct __align__(1024) SsdSmem {
   float ddw[8][kQ];           //   step d_j,
   float vdw[8][kQ];           //   a_{j+1} ... a_{b+31} d_j (column factor of the mask)
   // The column factor w_j of the tile's tokens (bf16, as the w o x product
-  // uses it), from the mask group to the output group; two buffers by tile
-  // parity.
-  __nv_bfloat16 wt[2][kQ];
+  // uses it), from the mask group to the output group; four buffers, like
+  // wready: the mask group may publish tile c + 2 before the output group
+  // has read tile c (it need only wait for w o x of tile c - 1), but tile
+  // c + 4 only after w o x of tile c + 1.
+  __nv_bfloat16 wt[4][kQ];
   // With the convolution fused: the three raw inputs before a tile (bf16,
   // 64 channels).
   __nv_bfloat16 halo[3][kP];
@@ -121,6 +125,7 @@ struct __align__(1024) SsdSmem {
   // lap of its ring, so no waiter can miss a phase.
   uint64_t full[2], empty[2], sdone[2], scdone[2], mready[2], stdone[2], yready[2], yfree[2];
   uint64_t xready[2];         // w o x written (output group)
+  uint64_t xconv[2];          // x convolved in place (convolution group, fused form)
   uint64_t wready[4];         // w_j and the tile decay written (mask group)
   uint32_t taddr;
   int abort;
@@ -203,13 +208,15 @@ __device__ __forceinline__ void st_cs_u4(void *p, uint4 v) {
                : "memory");
 }
 
-// Named barrier 1 over the output group (warps 8-11, 128 threads), and the
-// same barrier as a vote: every thread of the group gets the OR of `v`.
-__device__ __forceinline__ void out_group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-__device__ __forceinline__ bool out_group_any(bool v) {
+// Named barrier 1 over the convolution group of the fused form (warps 18
+// and 19, 64 threads), and the same barrier as a vote: every thread of the
+// group gets the OR of `v`.
+constexpr int kConvThreads = 64;
+__device__ __forceinline__ void conv_group_sync() { asm volatile("bar.sync 1, 64;" ::: "memory"); }
+__device__ __forceinline__ bool conv_group_any(bool v) {
   uint32_t r;
   asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 128, p;\n\t"
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 64, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
       : "r"((uint32_t)v)
@@ -261,7 +268,7 @@ __device__ __forceinline__ bool waitw(SsdSmem &s, uint64_t *bar, uint32_t parity
 }
 
 template <bool CONV>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_of<CONV>(), 1)
     ssd_tc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mB,
                   const __grid_constant__ CUtensorMap mC, const SsdTcParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -322,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.yfree[i], 4);   // one arrival per output-group warp
     }
     for (int i = 0; i < 2; ++i) mbar_init(&s.xready[i], 4);  // one arrival per output warp
+    for (int i = 0; i < 2; ++i) mbar_init(&s.xconv[i], 2);   // one per convolution warp
     for (int i = 0; i < 4; ++i) mbar_init(&s.wready[i], 4);  // one per half-0 mask warp
     s.abort = 0;
     fence_mbar_init();
@@ -483,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // barrier of the last commit issued, which tracks every earlier MMA.
     if (lane == 0 && last_bar) mbar_wait(last_bar, last_par, kWaitLimit);
     __syncwarp();
-  } else if ((warp >= 4 && warp < 8) || warp >= 14) {
+  } else if ((warp >= 4 && warp < 8) || (warp >= 14 && warp < 18)) {
     // ------------------------------------------------------------ mask group
     // Two warps per TMEM lane quarter (warps 4-7 and 14-17): each takes 32
     // rows and, of every row, half the work (16 of each 32-column block of
@@ -581,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float w_i = vdw[i] * after_blk;
       // w_i for the output group's w o x (bf16, as the product uses it), and
       // with it the tile decay above: one arrival per half-0 warp
-      if (half == 0) reinterpret_cast<uint16_t *>(s.wt[k])[i] = (uint16_t)pack_bf16x2(w_i, 0.f);
+      if (half == 0) reinterpret_cast<uint16_t *>(s.wt[c & 3])[i] = (uint16_t)pack_bf16x2(w_i, 0.f);
       __syncwarp();
       if (half == 0 && lane == 0) mbar_arrive(&s.wready[c & 3]);
       // next tile's dt: it has the rest of this tile to arrive
@@ -695,6 +703,120 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.mready[k]);
     }
+  } else if (CONV && warp >= 18) {
+    // ------------------------------------------------------------ convolution group
+    // Fused form: the causal convolution of x over tokens, then silu, in
+    // place in each landed tile, with nothing else to do, so it runs beside
+    // the other roles.  Thread (cq, tg): channels 4 cq .. + 4 of the head,
+    // tokens 32 tg .. + 32 of the tile, walked in order with the three
+    // previous raw inputs in registers (every row read once); the three rows
+    // before a tile are the previous tile's raw last rows (`halo`), or
+    // before this CTA's first tile xBC's or the conv state's.  One barrier
+    // between the reads a thread needs from its neighbour's rows and the
+    // in-place writes; every wait is voted over the two warps.
+    const int ci = tid - kThreads;
+    const int cq = ci & 15, tg = ci >> 4;
+    const uint32_t qoff = 8u * (uint32_t)(cq & 1);  // the quad within its 16-byte chunk
+    const int64_t ch0 = hd * kP;
+    auto waitc = [&](uint64_t *bar, uint32_t parity, int code) -> bool {
+      const bool ok = mbar_wait(bar, parity, kWaitLimit);
+      const bool fail = conv_group_any(!ok);
+      if (fail && ci == 0) set_abort(s, p.status, code);
+      return !fail;
+    };
+    // weights and bias of the thread's channels as pairs (0, 1), (2, 3)
+    f2 wt3[2], wt2[2], wt1[2], wt0[2], bs[2];
+    {
+      const float4 *wv = reinterpret_cast<const float4 *>(p.cw + (ch0 + 4 * cq) * 4);
+      const float4 w0 = __ldg(wv), w1 = __ldg(wv + 1), w2 = __ldg(wv + 2), w3 = __ldg(wv + 3);
+      wt0[0] = mk2(w0.x, w1.x); wt1[0] = mk2(w0.y, w1.y); wt2[0] = mk2(w0.z, w1.z);
+      wt3[0] = mk2(w0.w, w1.w);
+      wt0[1] = mk2(w2.x, w3.x); wt1[1] = mk2(w2.y, w3.y); wt2[1] = mk2(w2.z, w3.z);
+      wt3[1] = mk2(w2.w, w3.w);
+      const float *bp = p.cbias + ch0 + 4 * cq;
+      bs[0] = p.cbias ? mk2(__ldg(bp), __ldg(bp + 1)) : mk2(0.f, 0.f);
+      bs[1] = p.cbias ? mk2(__ldg(bp + 2), __ldg(bp + 3)) : mk2(0.f, 0.f);
+    }
+    // Before this CTA's first tile the three preceding inputs come from
+    // global memory, widened to float32 into the w o x buffer: the output
+    // group writes it only after this group's first xconv arrival.
+    const float *first = reinterpret_cast<const float *>(s.Xw);
+    {
+      const uint16_t *xr = reinterpret_cast<const uint16_t *>(p.xbc);
+      const int64_t t0 = (int64_t)cb * kQ;
+      for (int idx = ci; idx < 3 * kP; idx += kConvThreads) {
+        const int row = idx / kP, ch = idx % kP;
+        const int64_t tau = t0 - 3 + row;
+        float v = 0.f;
+        if (tau >= 0) v = __uint_as_float((uint32_t)xr[(b * L + tau) * p.ctot + ch0 + ch] << 16);
+        else if (p.cs_in) v = p.cs_in[(b * p.ctot + ch0 + ch) * 3 + (tau + 3)];
+        reinterpret_cast<float *>(s.Xw)[idx] = v;
+      }
+      conv_group_sync();
+    }
+    auto unpack2 = [](uint2 u, f2 (&v)[2]) {
+      v[0] = mk2(bf16lo(u.x), bf16hi(u.x));
+      v[1] = mk2(bf16lo(u.y), bf16hi(u.y));
+    };
+    const f2 half2 = mk2(0.5f, 0.5f);
+    for (int c = 0; c < nch; ++c) {
+      const int k = c & 1;
+      const int64_t t0 = (int64_t)(cb + c) * kQ;
+      if (!waitc(&s.full[k], (c >> 1) & 1, 16)) break;
+      uint8_t *xs = s.X[k];
+      f2 win[3][2];
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        const int r = 32 * tg - 3 + j;
+        if (r >= 0) {
+          unpack2(*reinterpret_cast<const uint2 *>(xs + sw128(r, cq >> 1) + qoff), win[j]);
+        } else if (c > 0) {
+          unpack2(*reinterpret_cast<const uint2 *>(&s.halo[r + 3][4 * cq]), win[j]);
+        } else {
+          const float4 f = *reinterpret_cast<const float4 *>(first + (r + 3) * kP + 4 * cq);
+          win[j][0] = mk2(f.x, f.y);
+          win[j][1] = mk2(f.z, f.w);
+        }
+      }
+      conv_group_sync();  // every window is read: rows may be overwritten now
+#pragma unroll 4
+      for (int j = 0; j < 32; ++j) {
+        const int r = 32 * tg + j;
+        uint2 *row = reinterpret_cast<uint2 *>(xs + sw128(r, cq >> 1) + qoff);
+        const uint2 u = *row;
+        // the raw last three rows are the next tile's halo
+        if (tg == 3 && j >= 29) *reinterpret_cast<uint2 *>(&s.halo[j - 29][4 * cq]) = u;
+        f2 xv[2];
+        unpack2(u, xv);
+        // u = silu(bias + sum_q w[q] x[t - 3 + q]), the newest input first,
+        // and silu(z) = z (1 + tanh(z / 2)) / 2: the operations of
+        // ssm_conv1d_fwd lane by lane, so both give the same bits
+        const bool live = t0 + r < L;
+        uint32_t ov[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          f2 acc = fma2(wt3[q], xv[q], bs[q]);
+          acc = fma2(wt2[q], win[2][q], acc);
+          acc = fma2(wt1[q], win[1][q], acc);
+          acc = fma2(wt0[q], win[0][q], acc);
+          const f2 hz = mul2(half2, acc);
+          float ta, tb2;
+          asm("tanh.approx.f32 %0, %1;" : "=f"(ta) : "f"(hz.x));
+          asm("tanh.approx.f32 %0, %1;" : "=f"(tb2) : "f"(hz.y));
+          const f2 o = mul2(acc, fma2(half2, mk2(ta, tb2), half2));
+          ov[q] = live ? pack_bf16x2(o.x, o.y) : 0u;
+          win[0][q] = win[1][q];
+          win[1][q] = win[2][q];
+          win[2][q] = xv[q];
+        }
+        *row = make_uint2(ov[0], ov[1]);
+      }
+      // the convolved tile is read by the output group and, as Y's B
+      // operand, by the tensor cores
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.xconv[k]);
+    }
   } else if (warp < 4) {
     // ------------------------------------------------------------ state group
     const int n = tid;
@@ -761,139 +883,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const __nv_bfloat16 *zp = p.z + ((b * L + t) * H + hd) * kP;
 #pragma unroll
         for (int q = 0; q < 8; ++q) zr[q] = ld_cs_u4(zp + 8 * q);
-      } else if (CONV) {
-        // (assigned on every path, so the previous tile's values are dead
-        // while the next tile's convolution runs)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) zr[q] = make_uint4(0u, 0u, 0u, 0u);
       }
-    };
-    // A wait of this group: voted per warp, or, fused, over the four warps
-    // (they meet in named barriers there, so none may leave the loop alone).
-    auto waito = [&](uint64_t *bar, uint32_t parity, int code) -> bool {
-      if (!CONV) return waitw(s, bar, parity, p.status, code);
-      const bool ok = mbar_wait(bar, parity, kWaitLimit);
-      const bool fail = out_group_any(!ok);
-      if (fail && i == 0) set_abort(s, p.status, code);
-      return !fail;
-    };
-    // Fused form: the causal convolution of x over tokens, then silu, in
-    // place in the landed tile c, as soon as it lands (the three rows before
-    // the tile from the previous tile's raw inputs, kept in `halo`, or for
-    // the first tile of this CTA from xBC or the conv state).  Thread (cq,
-    // tg): channels 4 cq .. + 4 of the head, tokens 16 tg .. + 16 of the
-    // tile, walked in order with the three previous raw inputs in registers
-    // (every row read once); one barrier between the reads every thread
-    // needs from its neighbour's rows and the in-place writes.
-    auto conv_x = [&](int c) -> bool {
-      const int k = c & 1;
-      const int64_t t0 = (int64_t)(cb + c) * kQ;
-      const int64_t ch0 = hd * kP;
-      // Before this CTA's first tile the three preceding inputs come from
-      // global memory, widened to float32 into the w o x buffer (free until
-      // this group's own first w o x writes).
-      const float *first = reinterpret_cast<const float *>(s.Xw);
-      if (c == 0) {
-        const uint16_t *xr = reinterpret_cast<const uint16_t *>(p.xbc);
-        for (int idx = i; idx < 3 * kP; idx += 128) {
-          const int row = idx / kP, ch = idx % kP;
-          const int64_t tau = t0 - 3 + row;
-          float v = 0.f;
-          if (tau >= 0) v = __uint_as_float((uint32_t)xr[(b * L + tau) * p.ctot + ch0 + ch] << 16);
-          else if (p.cs_in) v = p.cs_in[(b * p.ctot + ch0 + ch) * 3 + (tau + 3)];
-          reinterpret_cast<float *>(s.Xw)[idx] = v;
-        }
-        out_group_sync();
-      }
-      const int cq = i & 15, tg = i >> 4;
-      const uint32_t qoff = 8u * (uint32_t)(cq & 1);  // the quad within its 16-byte chunk
-      // weights and bias of the thread's channels as pairs (0, 1), (2, 3);
-      // their loads overlap the wait for the tile
-      f2 wt3[2], wt2[2], wt1[2], wt0[2], bs[2];
-      {
-        const float4 *wv = reinterpret_cast<const float4 *>(p.cw + (ch0 + 4 * cq) * 4);
-        const float4 w0 = __ldg(wv), w1 = __ldg(wv + 1), w2 = __ldg(wv + 2), w3 = __ldg(wv + 3);
-        wt0[0] = mk2(w0.x, w1.x); wt1[0] = mk2(w0.y, w1.y); wt2[0] = mk2(w0.z, w1.z);
-        wt3[0] = mk2(w0.w, w1.w);
-        wt0[1] = mk2(w2.x, w3.x); wt1[1] = mk2(w2.y, w3.y); wt2[1] = mk2(w2.z, w3.z);
-        wt3[1] = mk2(w2.w, w3.w);
-        const float *bp = p.cbias + ch0 + 4 * cq;
-        bs[0] = p.cbias ? mk2(__ldg(bp), __ldg(bp + 1)) : mk2(0.f, 0.f);
-        bs[1] = p.cbias ? mk2(__ldg(bp + 2), __ldg(bp + 3)) : mk2(0.f, 0.f);
-      }
-      if (!waito(&s.full[k], (c >> 1) & 1, 14)) return false;
-      uint8_t *xs = s.X[k];
-      auto unpack2 = [](uint2 u, f2 (&v)[2]) {
-        v[0] = mk2(bf16lo(u.x), bf16hi(u.x));
-        v[1] = mk2(bf16lo(u.y), bf16hi(u.y));
-      };
-      // the three raw rows before this thread's first token: the previous
-      // group's rows (read before anyone overwrites them), the previous
-      // tile's last rows (`halo`), or before this CTA's first tile `first`
-      f2 win[3][2];
-#pragma unroll
-      for (int j = 0; j < 3; ++j) {
-        const int r = 16 * tg - 3 + j;
-        if (r >= 0) {
-          unpack2(*reinterpret_cast<const uint2 *>(xs + sw128(r, cq >> 1) + qoff), win[j]);
-        } else if (c > 0) {
-          unpack2(*reinterpret_cast<const uint2 *>(&s.halo[r + 3][4 * cq]), win[j]);
-        } else {
-          const float4 f = *reinterpret_cast<const float4 *>(first + (r + 3) * kP + 4 * cq);
-          win[j][0] = mk2(f.x, f.y);
-          win[j][1] = mk2(f.z, f.w);
-        }
-      }
-      out_group_sync();  // every window is read: rows may be overwritten now
-      const f2 half2 = mk2(0.5f, 0.5f);
-#pragma unroll 4
-      for (int j = 0; j < 16; ++j) {
-        const int r = 16 * tg + j;
-        uint2 *row = reinterpret_cast<uint2 *>(xs + sw128(r, cq >> 1) + qoff);
-        const uint2 u = *row;
-        // the raw last three rows are the next tile's halo
-        if (tg == 7 && j >= 13) *reinterpret_cast<uint2 *>(&s.halo[j - 13][4 * cq]) = u;
-        f2 xv[2];
-        unpack2(u, xv);
-        // u = silu(bias + sum_q w[q] x[t - 3 + q]), the newest input first,
-        // and silu(z) = z (1 + tanh(z / 2)) / 2: the operations of
-        // ssm_conv1d_fwd lane by lane, so both give the same bits
-        const bool live = t0 + r < L;
-        uint32_t ov[2];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          f2 acc = fma2(wt3[q], xv[q], bs[q]);
-          acc = fma2(wt2[q], win[2][q], acc);
-          acc = fma2(wt1[q], win[1][q], acc);
-          acc = fma2(wt0[q], win[0][q], acc);
-          const f2 hz = mul2(half2, acc);
-          float ta, tb2;
-          asm("tanh.approx.f32 %0, %1;" : "=f"(ta) : "f"(hz.x));
-          asm("tanh.approx.f32 %0, %1;" : "=f"(tb2) : "f"(hz.y));
-          const f2 o = mul2(acc, fma2(half2, mk2(ta, tb2), half2));
-          ov[q] = live ? pack_bf16x2(o.x, o.y) : 0u;
-          win[0][q] = win[1][q];
-          win[1][q] = win[2][q];
-          win[2][q] = xv[q];
-        }
-        *row = make_uint2(ov[0], ov[1]);
-      }
-      return true;
     };
     // w o x of tile c, the B operand of Sc(c) (thread = row), once x has
-    // landed (fused: been convolved), the mask group has published w_j and
-    // Sc(c-1) is done with the buffer.  (Fused, the wready vote is also the
-    // barrier between the convolution's writes and these reads.)
+    // landed (fused: been convolved by the convolution group), the mask
+    // group has published w_j and Sc(c-1) is done with the buffer.
     auto xprep = [&](int c) -> bool {
       const int k = c & 1;
-      if (CONV) {
-        if (!conv_x(c)) return false;
-      } else if (!waito(&s.full[k], (c >> 1) & 1, 14)) {
-        return false;
-      }
-      if (!waito(&s.wready[c & 3], (c >> 2) & 1, 15)) return false;
-      if (c >= 1 && !waito(&s.scdone[k ^ 1], ((c - 1) >> 1) & 1, 9)) return false;
-      const uint32_t wb = reinterpret_cast<const uint16_t *>(s.wt[k])[i];
+      if (!waitw(s, CONV ? &s.xconv[k] : &s.full[k], (c >> 1) & 1, p.status, 14)) return false;
+      if (!waitw(s, &s.wready[c & 3], (c >> 2) & 1, p.status, 15)) return false;
+      if (c >= 1 && !waitw(s, &s.scdone[k ^ 1], ((c - 1) >> 1) & 1, p.status, 9)) return false;
+      const uint32_t wb = reinterpret_cast<const uint16_t *>(s.wt[c & 3])[i];
       const uint32_t w2 = wb | (wb << 16);
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc) {
@@ -910,11 +910,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; ok && c < nch; ++c) {
       const int k = c & 1;
       const int64_t t = (int64_t)(cb + c) * kQ + i;
-      // the next tile's w o x first (and, fused, its convolution): Sc(c+1)
-      // waits for it while this tile's Y is still being formed
+      // the next tile's w o x first: Sc(c+1) waits for it while this tile's
+      // Y is still being formed
       if (c + 1 < nch && !xprep(c + 1)) break;
       load_z(c);
-      if (!waito(&s.yready[k], (c >> 1) & 1, 13)) break;
+      if (!waitw(s, &s.yready[k], (c >> 1) & 1, p.status, 13)) break;
       tc_fence_after();
       __nv_bfloat16 *yp = p.y + ((b * L + t) * H + hd) * kP;
       // two halves of 32 columns; Y[k] is released after the second load
@@ -1147,6 +1147,7 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
   q.cs_in = conv ? conv->state_in : nullptr;
   const size_t smem = ssd_tc_smem_bytes();
   auto kern = conv ? ssd_tc_kernel<true> : ssd_tc_kernel<false>;
+  const int nthreads = conv ? threads_of<true>() : threads_of<false>();
   // (set on every call: the attribute belongs to the current device)
   {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1164,7 +1165,7 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
     if (e != cudaSuccess) return e;
   }
   if (split.nseg <= 1) {
-    kern<<<(unsigned)q.nfull, kThreads, smem, stream>>>(mX, mB, mC, q);
+    kern<<<(unsigned)q.nfull, nthreads, smem, stream>>>(mX, mB, mC, q);
     return cudaGetLastError();
   }
   // Tail cut into segments: (1) every segment of the tail units from its own
@@ -1181,7 +1182,7 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
   q.seg_hend = hend;
   q.seg_decay = dec;
   q.seg_hin = hin;
-  kern<<<(unsigned)slots, kThreads, smem, stream>>>(mX, mB, mC, q);
+  kern<<<(unsigned)slots, nthreads, smem, stream>>>(mX, mB, mC, q);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ssd_seg_carry_kernel<<<dim3((unsigned)split.ntail, kN * kP / kCarrySlice), kCarrySlice / 4, 0,
@@ -1190,7 +1191,7 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
   if (e != cudaSuccess) return e;
   q.nfull = units - split.ntail;
   q.seg_lo = 1;
-  kern<<<(unsigned)(q.nfull + split.ntail * (split.nseg - 1)), kThreads, smem, stream>>>(
+  kern<<<(unsigned)(q.nfull + split.ntail * (split.nseg - 1)), nthreads, smem, stream>>>(
       mX, mB, mC, q);
   return cudaGetLastError();
 }

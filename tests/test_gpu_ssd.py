@@ -98,6 +98,9 @@ def test_2p7b_full_size_sampled(cuda_ok):
     w = I.WORKLOADS["ssd_2p7b_b4_l4096_h80_p64_n128_bf16"]
     d = I.workload_inputs(w)
     y, h, _ = _run(d, chunk=w.chunk)
+    for _ in range(2):  # the same bits on every run (the roles' hand-offs leave no race)
+        y2, h2, _ = _run(d, chunk=w.chunk)
+        assert torch.equal(y2, y) and torch.equal(h2, h)
     rows, hs = [0, 3], [0, 40, 60, 79]  # (3, 60) and (3, 79) are in the cut last wave
     sub = dict(d)
     sub["x"] = d["x"][rows][:, :, hs]

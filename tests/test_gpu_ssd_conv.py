@@ -141,6 +141,9 @@ def test_fused_2p7b_full_size_sampled(cuda_ok):
     y, h, so = _fused(d)
     uy, uh, uso = _unfused(d)
     assert torch.equal(y, uy) and torch.equal(h, uh) and torch.equal(so, uso)
+    for _ in range(2):  # the same bits on every run (the roles' hand-offs leave no race)
+        y2, h2, _ = _fused(d)
+        assert torch.equal(y2, y) and torch.equal(h2, h)
     row = dict(d, xbc=d["xbc"][3:], dt=d["dt"][3:], cs=d["cs"][3:], z=None)
     heads = [5, 79]  # (3, 79) is in the cut last wave
     ry, rh, _ = _oracle(row, heads)
