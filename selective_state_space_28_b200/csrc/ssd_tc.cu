@@ -985,12 +985,14 @@ __global__ void __launch_bounds__(kCarrySlice / 4)
   }
 }
 
+constexpr int kBcRun = 8;  // tokens per thread in the B/C convolution pre-pass
+
 // The fused call's pre-pass, one batch row per grid row (blockIdx.y).  (1)
 // The B and C channels of xBC (nbc = 2 G N of them from channel c0 on)
 // convolved over tokens, then silu, into bc [batch][L][nbc]: every head of a
 // group reads the same B and C, so they are convolved once here instead of
-// in each head's CTA (x is convolved inside the scan).  A thread takes one
-// token and eight channels.  (2) The blocks after those: the conv state
+// in each head's CTA (x is convolved inside the scan).  A thread takes
+// eight channels over a run of tokens.  (2) The blocks after those: the conv state
 // out, the last three inputs of every channel, oldest first (from cs_in
 // where the sequence is shorter than three).  Indices within a row are
 // 32-bit (the host keeps L * nbc / 8 and ctot below 2^31).
@@ -1001,39 +1003,56 @@ __global__ void __launch_bounds__(256)
   const int64_t bb = blockIdx.y;
   const unsigned nchunk = (unsigned)nbc / 8u;
   if (blockIdx.x < conv_blocks) {
+    // thread = (8-channel chunk j, run of kBcRun tokens), walked in order
+    // with the three previous inputs in registers
     const unsigned idx = blockIdx.x * 256u + threadIdx.x;
-    const unsigned t = idx / nchunk, j = idx - t * nchunk;
-    if (t >= (unsigned)L) return;
+    const unsigned run = idx / nchunk, j = idx - run * nchunk;
+    const int64_t t0 = (int64_t)run * kBcRun;
+    if (t0 >= L) return;
     const int64_t ch = c0 + 8 * (int64_t)j;
-    const __nv_bfloat16 *xrow = xbc + (bb * L + t) * ctot + ch;
-    float v[4][8];
+    float w[8][4], bias[8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int tau = (int)t - 3 + q;
+    for (int e = 0; e < 8; ++e) {
+      const float4 v = __ldg(reinterpret_cast<const float4 *>(cw + (ch + e) * 4));
+      w[e][0] = v.x; w[e][1] = v.y; w[e][2] = v.z; w[e][3] = v.w;
+      bias[e] = cbias ? __ldg(cbias + ch + e) : 0.f;
+    }
+    float win[3][8];
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const int64_t tau = t0 - 3 + q;
       if (tau >= 0) {
-        unpack8(ld_nc_u4(xrow - (int64_t)(3 - q) * ctot), v[q]);
+        unpack8(ld_nc_u4(xbc + (bb * L + tau) * ctot + ch), win[q]);
       } else if (cs_in) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[q][e] = cs_in[(bb * ctot + ch + e) * 3 + (tau + 3)];
+        for (int e = 0; e < 8; ++e) win[q][e] = cs_in[(bb * ctot + ch + e) * 3 + (tau + 3)];
       } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[q][e] = 0.f;
+        for (int e = 0; e < 8; ++e) win[q][e] = 0.f;
       }
     }
-    float o[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {  // the newest input first, as ssm_conv1d_fwd
-      const float4 w = __ldg(reinterpret_cast<const float4 *>(cw + (ch + e) * 4));
-      float acc = cbias ? __ldg(cbias + ch + e) : 0.f;
-      acc = fmaf(w.w, v[3][e], acc);
-      acc = fmaf(w.z, v[2][e], acc);
-      acc = fmaf(w.y, v[1][e], acc);
-      acc = fmaf(w.x, v[0][e], acc);
-      o[e] = silu_tanh(acc);
+    for (int r = 0; r < kBcRun; ++r) {
+      const int64_t t = t0 + r;
+      if (t >= L) break;
+      float xv[8];
+      unpack8(ld_nc_u4(xbc + (bb * L + t) * ctot + ch), xv);
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {  // the newest input first, as ssm_conv1d_fwd
+        float acc = fmaf(w[e][3], xv[e], bias[e]);
+        acc = fmaf(w[e][2], win[2][e], acc);
+        acc = fmaf(w[e][1], win[1][e], acc);
+        acc = fmaf(w[e][0], win[0][e], acc);
+        o[e] = silu_tanh(acc);
+        win[0][e] = win[1][e];
+        win[1][e] = win[2][e];
+        win[2][e] = xv[e];
+      }
+      *reinterpret_cast<uint4 *>(bc + (bb * L + t) * nbc + 8 * j) =
+          make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                     pack_bf16x2(o[6], o[7]));
     }
-    *reinterpret_cast<uint4 *>(bc + (bb * L + t) * nbc + 8 * j) =
-        make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                   pack_bf16x2(o[6], o[7]));
     return;
   }
   const unsigned c = (blockIdx.x - conv_blocks) * 256u + threadIdx.x;
@@ -1155,7 +1174,8 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
     if (e != cudaSuccess) return e;
   }
   if (conv) {
-    const unsigned conv_blocks = (unsigned)((p.L * (2 * GN / 8) + 255) / 256);
+    const unsigned conv_blocks =
+        (unsigned)(((p.L + kBcRun - 1) / kBcRun * (2 * GN / 8) + 255) / 256);
     const unsigned state_blocks = conv->state_out ? (unsigned)((conv->ctot + 255) / 256) : 0u;
     ssd_bc_conv_kernel<<<dim3(conv_blocks + state_blocks, (unsigned)p.batch), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(conv->xbc), p.L, conv->ctot, p.H * kP, (int)(2 * GN),
