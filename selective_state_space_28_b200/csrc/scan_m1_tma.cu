@@ -153,6 +153,21 @@ __device__ __forceinline__ void load_pairs(const float *src, f2 (&v)[NP]) {
     v[0] = mk2(a.x, a.y);
   }
 }
+// The same from a row of the I/O type: bfloat16 widens exactly to float32,
+// so these are the values the widened copy would hold.
+template <int NP, typename T>
+__device__ __forceinline__ void load_pairs_io(const T *src, f2 (&v)[NP]) {
+  if constexpr (sizeof(T) == 4) {
+    load_pairs<NP>(reinterpret_cast<const float *>(src), v);
+  } else if constexpr (NP == 2) {
+    const uint2 a = *reinterpret_cast<const uint2 *>(src);
+    v[0] = mk2(bf16lo(a.x), bf16hi(a.x));
+    v[1] = mk2(bf16lo(a.y), bf16hi(a.y));
+  } else {
+    const uint32_t a = *reinterpret_cast<const uint32_t *>(src);
+    v[0] = mk2(bf16lo(a), bf16hi(a));
+  }
+}
 template <int NP>
 __device__ __forceinline__ void store_pairs(float *dst, const f2 (&v)[NP]) {
   if constexpr (NP == 2)
@@ -165,7 +180,8 @@ __device__ __forceinline__ void store_pairs(float *dst, const f2 (&v)[NP]) {
 // STATES: also store every token's state.  WR: replace the state at token
 // p.t_write (the state write).
 // SPL: states per lane (4, or 2 for twice the warps on small problems).
-template <int N, int SPL, typename T, int NS, bool HAS_Z, int MODE, bool STATES, bool WR, int PX>
+template <int N, int SPL, typename T, int NS, bool HAS_Z, int MODE, bool STATES, bool WR, int PX,
+          bool RBC>
 __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
     m1_scan_tma_kernel(const __grid_constant__ CUtensorMap mx,
                        const __grid_constant__ CUtensorMap mdt,
@@ -198,7 +214,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
   const int64_t te = tb + p.seg_len < L ? tb + p.seg_len : L;
   const int nst = (int)((te - tb + kTL - 1) / kTL);
   const bool softplus_on = p.flags & 1u;
-  const bool rms_bc = p.flags & 2u;
+  constexpr bool rms_bc = RBC;  // the host picks the instance from SSM_RMSNORM_BC
   constexpr uint32_t kStageBytes = ((HAS_Z ? 3 : 2) * kTL * kCT + 2 * kTL * N) * sizeof(T);
 
   if (threadIdx.x == 0) {
@@ -260,6 +276,14 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
       PX == 2 && __all_sync(0xffffffffu, softplus_on && ((Al.x < 0.f && Al.y < 0.f) || !cvalid));
   float dsum = 0.f;
   bool failed = false;
+  // The prologue's lane always takes the same 8 channels (k0 below): their
+  // step bias and skip weight stay in registers.
+  float biasr[8], skipr[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    biasr[i] = s.bias[(lane & 3) * 8 + i];
+    skipr[i] = s.skip[(lane & 3) * 8 + i];
+  }
   // Rows [warp * kTL / NW, + kTL / NW) of stage st's y staging (token t0y
   // onwards, tny of them in the segment) to global memory, 16 bytes a lane.
   auto store_y = [&](int st, int64_t t0y, int tny) {
@@ -284,7 +308,11 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
       failed = true;
       break;
     }
-    // ---- 2. widen this warp's share of the stage's B and C rows
+    // ---- 2. with RMS norms on B and C, widen and normalise this warp's
+    // share of the stage's B and C rows (without them the recurrence reads
+    // B and C straight from the stage: half the shared-memory wavefronts of
+    // the widened float32 rows)
+    if constexpr (rms_bc)
     for (int e = lane; e < TPW * 2; e += 32) {
       const int t = warp * TPW + (e >> 1), which = e & 1;
       const T *src = which ? s.C[buf][t] : s.B[buf][t];
@@ -325,11 +353,11 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
       float2 o[8], og[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        float d = fmaf(dv[i], rs, s.bias[k0 + i]);
+        float d = fmaf(dv[i], rs, biasr[i]);
         if (softplus_on) d = softplus_sfu(d);
         o[i] = tvalid ? make_float2(d, d * xv[i]) : make_float2(0.f, 0.f);
         const float gate = HAS_Z ? (kBF16 ? silu_tanh(zv[i]) : silu(zv[i])) : 1.f;
-        og[i] = make_float2(s.skip[k0 + i] * xv[i], gate);
+        og[i] = make_float2(skipr[i] * xv[i], gate);
       }
       float4 *dst = reinterpret_cast<float4 *>(&s.ddx[sg & 1][t][k0]);
       float4 *gst = reinterpret_cast<float4 *>(&s.eg[sg & 1][t][k0]);
@@ -363,7 +391,8 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
         const int t = tg + u;
         const float2 dd = s.ddx[sg & 1][t][cw0 + ch];
         f2 bv[NP];
-        load_pairs<NP>(&s.bc[buf][t][0][SPL * q], bv);
+        if constexpr (rms_bc) load_pairs<NP>(&s.bc[buf][t][0][SPL * q], bv);
+        else load_pairs_io<NP>(&s.B[buf][t][SPL * q], bv);
         const f2 d2 = mk2(dd.x, dd.x), dx2 = mk2(dd.y, dd.y);
 #pragma unroll
         for (int j = 0; j < NP; ++j) {
@@ -417,7 +446,8 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
           }
           if (kFull) {
             f2 cv[NP];
-            load_pairs<NP>(&s.bc[buf][t][1][SPL * q], cv);
+            if constexpr (rms_bc) load_pairs<NP>(&s.bc[buf][t][1][SPL * q], cv);
+            else load_pairs_io<NP>(&s.C[buf][t][SPL * q], cv);
             f2 acc = mul2(cv[0], h[0]);
 #pragma unroll
             for (int j = 1; j < NP; ++j) acc = fma2(cv[j], h[j], acc);
@@ -560,7 +590,8 @@ bool make_maps(const M1Params &p, Maps &m) {
 template <int N, int SPL, typename T, bool HZ, int MODE, bool ST, bool WR>
 cudaError_t launch_spl(const Maps &m, const M1Params &p, int nseg, cudaStream_t s) {
   constexpr int NS = 3;
-  auto k = m1_scan_tma_kernel<N, SPL, T, NS, HZ, MODE, ST, WR, kPolyStates>;
+  auto k = (p.flags & 2u) ? m1_scan_tma_kernel<N, SPL, T, NS, HZ, MODE, ST, WR, kPolyStates, true>
+                          : m1_scan_tma_kernel<N, SPL, T, NS, HZ, MODE, ST, WR, kPolyStates, false>;
   const size_t smem = sizeof(ScanSmem<N, T, NS>) + 128;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
