@@ -1,6 +1,7 @@
 // sm100.cuh -- thin inline-PTX wrappers for the sm_100a features the SSD
-// kernel uses: mbarriers (with bounded waits), TMA tile loads (no cluster
-// multicast anywhere), and the 5th-generation tensor core (tcgen05: TMEM
+// kernel uses: mbarriers (with bounded waits), TMA tile loads (every CTA
+// loads its own tiles from this GPU's memory), and the 5th-generation tensor
+// core (tcgen05: TMEM
 // allocation, MMA with shared-memory or TMEM A operand, commit, TMEM
 // load/store).  Descriptor encodings follow the PTX ISA's tcgen05 matrix and
 // instruction descriptor formats.
