@@ -226,9 +226,31 @@ __global__ void __launch_bounds__(128)
 }
 
 template <typename T, int W>
+bool vec_form(const ConvParams &p) {
+  return (p.Cc % Vec<T>::V) == 0;  // rows then hold whole vectors (bases are 16-byte aligned)
+}
+
+// CTAs of the vector form resident per SM (its registers and slots decide),
+// read once per instance from the runtime's occupancy calculator.
+template <typename T, int W>
+int vec_ctas_per_sm() {
+  static const int n = [] {
+    int k = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&k, conv1d_vec_kernel<T, W>, 128, 0) !=
+            cudaSuccess ||
+        k <= 0) {
+      cudaGetLastError();
+      return 0;
+    }
+    return k;
+  }();
+  return n;
+}
+
+template <typename T, int W>
 cudaError_t launch_w(const ConvParams &p, cudaStream_t s) {
   constexpr int V = Vec<T>::V;
-  const bool vec = (p.Cc % V) == 0;  // rows then hold whole vectors (bases are 16-byte aligned)
+  const bool vec = vec_form<T, W>(p);
   const int64_t runs = (p.L + p.run - 1) / p.run;
   const int64_t units = vec ? p.batch * (p.Cc / V) : p.batch * p.Cc;
   dim3 grid((unsigned)((units + 127) / 128), (unsigned)runs);
@@ -245,6 +267,28 @@ cudaError_t launch_w(const ConvParams &p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Tokens per thread of the vector form: whole batches of kTok, at least
+// kRunMin, chosen so that the grid fills whole waves of resident CTAs.  With
+// kRun tokens the bf16 2.7B mixer (b4, 5376 channels: 42 x 32 CTAs at six
+// per SM) would run 1.5 waves, the second half empty; 200-token runs make it
+// one wave of 882 CTAs.
+constexpr int64_t kRunMin = 64;
+template <typename T, int W>
+int64_t fitted_run(const ConvParams &p) {
+  const int64_t bx = (p.batch * (p.Cc / Vec<T>::V) + 127) / 128;
+  const int64_t per_sm = vec_ctas_per_sm<T, W>();
+  if (per_sm <= 0 || bx <= 0) return kRun;
+  const int64_t cap = (int64_t)device_sm_count() * per_sm;
+  const int64_t runs0 = (p.L + kRun - 1) / kRun;
+  int64_t waves = bx * runs0 / cap;  // whole waves the default runs fill
+  if (waves < 1) waves = 1;
+  int64_t runs = cap * waves / bx;  // runs of each column that fit in them
+  if (runs < 1) runs = 1;
+  int64_t run = (p.L + runs - 1) / runs;
+  run = (run + kTok - 1) / kTok * kTok;
+  return run < kRunMin ? kRunMin : run;
+}
+
 template <typename T>
 cudaError_t launch_t(const ConvParams &p, cudaStream_t s) {
   switch (p.W) {
@@ -256,13 +300,25 @@ cudaError_t launch_t(const ConvParams &p, cudaStream_t s) {
   return cudaErrorInvalidValue;
 }
 
+template <typename T>
+int64_t run_t(const ConvParams &p) {
+  switch (p.W) {
+    case 1: return vec_form<T, 1>(p) ? fitted_run<T, 1>(p) : kRun;
+    case 2: return vec_form<T, 2>(p) ? fitted_run<T, 2>(p) : kRun;
+    case 3: return vec_form<T, 3>(p) ? fitted_run<T, 3>(p) : kRun;
+    case 4: return vec_form<T, 4>(p) ? fitted_run<T, 4>(p) : kRun;
+  }
+  return kRun;
+}
+
 }  // namespace
 
-// Tokens per thread: kRun, or the whole sequence when the state is updated
-// in place (the run that reads the incoming state must be the one that
-// writes the new state).
-int64_t conv1d_run_length(int64_t L, bool state_in_place) {
-  return state_in_place ? (L > 0 ? L : 1) : kRun;
+// Tokens per thread: the whole sequence when the state is updated in place
+// (the run that reads the incoming state must be the one that writes the new
+// state), else a run fitted to the device's waves (vector form) or kRun.
+int64_t conv1d_run_length(const ConvParams &p, bool state_in_place) {
+  if (state_in_place) return p.L > 0 ? p.L : 1;
+  return p.io == 1 ? run_t<__nv_bfloat16>(p) : run_t<float>(p);
 }
 
 bool conv1d_supported(const ConvParams &p) {

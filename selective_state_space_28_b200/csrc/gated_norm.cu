@@ -9,12 +9,12 @@
 // needs every head of the token, so it is a pass of its own after the SSD.
 //
 // One CTA per row: the first pass reads y and z with 16-byte streaming loads
-// (for rows up to 8192 bf16 / 4096 float32 values, all of a thread's loads
-// are issued before any is used, so enough bytes are in flight), keeps g in
-// shared memory and accumulates its sum of squares; a block reduction gives
-// the row's scale; the second pass writes out.  Every input is read once and
-// every output written once.  out may be y itself (the whole row is read
-// before any of it is written).
+// and accumulates the sum of squares of g; a block reduction gives the row's
+// scale; the second pass writes out.  Rows up to 8192 bf16 / 4096 float32
+// values keep g in registers (all of a thread's loads issued before any is
+// used, so enough bytes are in flight); wider rows keep it in shared memory.
+// Every input is read once and every output written once.  out may be y
+// itself (the whole row is read before any of it is written).
 #include "common.cuh"
 #include "internal.h"
 
@@ -86,8 +86,71 @@ template <> struct NRaw<float> {
     f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
   }
 };
-constexpr int kMaxVec = 4;  // vectors per thread held in flight at once
+constexpr int kMaxVec = 4;  // vectors per thread the register form holds
 
+// Register form: rows of at most kThreads * V * NV values, whole vectors.
+// Every thread issues all of its (up to NV) y and z loads before using any,
+// keeps its gated values in registers across the block reduction, and writes
+// its outputs from them: each input read once, each output written once, no
+// shared-memory copy of the row.  The launch picks the smallest NV that
+// covers the row (the 2.7B mixer's 5120 bf16 values: NV = 3), so a thread
+// holds no registers for vectors it never loads.
+template <typename T, int NV>
+__global__ void __launch_bounds__(kThreads) gated_norm_reg_kernel(GatedNormParams p) {
+  constexpr int V = NVec<T>::V;
+  __shared__ float red[kThreads / 32];
+  const int64_t W = p.width;
+  const T *y = static_cast<const T *>(p.y) + (int64_t)blockIdx.x * W;
+  const T *z = p.z ? static_cast<const T *>(p.z) + (int64_t)blockIdx.x * W : nullptr;
+  T *o = static_cast<T *>(p.out) + (int64_t)blockIdx.x * W;
+  typename NRaw<T>::R ry[NV], rz[NV];
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int i = (k * kThreads + (int)threadIdx.x) * V;
+    if (i < W) {
+      ry[k] = NRaw<T>::load(y + i);
+      if (z) rz[k] = NRaw<T>::load(z + i);
+    }
+  }
+  float g[NV][V];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int i = (k * kThreads + (int)threadIdx.x) * V;
+    if (i < W) {
+      float yv[V], zv[V];
+      NRaw<T>::widen(ry[k], yv);
+      if (z) NRaw<T>::widen(rz[k], zv);
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        g[k][v] = z ? yv[v] * gate<T>(zv[v]) : yv[v];
+        ss = fmaf(g[k][v], g[k][v], ss);
+      }
+    }
+  }
+  const float inv = rsqrtf(block_sum(ss, red) / (float)W + p.eps);
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int i = (k * kThreads + (int)threadIdx.x) * V;
+    if (i < W) {
+      float ov[V];
+#pragma unroll
+      for (int v = 0; v < V; v += 4) {
+        float4 wq = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (p.weight) wq = *reinterpret_cast<const float4 *>(p.weight + i + v);
+        ov[v] = g[k][v] * inv * wq.x;
+        ov[v + 1] = g[k][v + 1] * inv * wq.y;
+        ov[v + 2] = g[k][v + 2] * inv * wq.z;
+        ov[v + 3] = g[k][v + 3] * inv * wq.w;
+      }
+      NVec<T>::store(o + i, ov);
+    }
+  }
+}
+
+// Shared-memory form, for wider rows (VEC: whole 16-byte vectors) and for
+// rows that are not whole vectors (!VEC): the gated row is kept in shared
+// memory between the two passes.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads) gated_norm_kernel(GatedNormParams p) {
   extern __shared__ float4 g4[];  // [width]: this row's gated values
@@ -100,49 +163,19 @@ __global__ void __launch_bounds__(kThreads) gated_norm_kernel(GatedNormParams p)
   float ss = 0.f;
   if constexpr (VEC) {
     constexpr int V = NVec<T>::V;
-    if (W <= (int64_t)kThreads * V * kMaxVec) {
-      // every load of the thread issued before any is used
-      typename NRaw<T>::R ry[kMaxVec], rz[kMaxVec];
+    for (int64_t i = (int64_t)threadIdx.x * V; i < W; i += (int64_t)kThreads * V) {
+      float yv[V], zv[V];
+      NVec<T>::load(y + i, yv);
+      if (z) NVec<T>::load(z + i, zv);
+      float gv[V];
 #pragma unroll
-      for (int k = 0; k < kMaxVec; ++k) {
-        const int64_t i = ((int64_t)k * kThreads + threadIdx.x) * V;
-        if (i < W) {
-          ry[k] = NRaw<T>::load(y + i);
-          if (z) rz[k] = NRaw<T>::load(z + i);
-        }
+      for (int v = 0; v < V; ++v) {
+        gv[v] = z ? yv[v] * gate<T>(zv[v]) : yv[v];
+        ss = fmaf(gv[v], gv[v], ss);
       }
 #pragma unroll
-      for (int k = 0; k < kMaxVec; ++k) {
-        const int64_t i = ((int64_t)k * kThreads + threadIdx.x) * V;
-        if (i < W) {
-          float yv[V], zv[V], gv[V];
-          NRaw<T>::widen(ry[k], yv);
-          if (z) NRaw<T>::widen(rz[k], zv);
-#pragma unroll
-          for (int v = 0; v < V; ++v) {
-            gv[v] = z ? yv[v] * gate<T>(zv[v]) : yv[v];
-            ss = fmaf(gv[v], gv[v], ss);
-          }
-#pragma unroll
-          for (int v = 0; v < V; v += 4)
-            *reinterpret_cast<float4 *>(&g[i + v]) = make_float4(gv[v], gv[v + 1], gv[v + 2], gv[v + 3]);
-        }
-      }
-    } else {
-      for (int64_t i = (int64_t)threadIdx.x * V; i < W; i += (int64_t)kThreads * V) {
-        float yv[V], zv[V];
-        NVec<T>::load(y + i, yv);
-        if (z) NVec<T>::load(z + i, zv);
-        float gv[V];
-#pragma unroll
-        for (int v = 0; v < V; ++v) {
-          gv[v] = z ? yv[v] * gate<T>(zv[v]) : yv[v];
-          ss = fmaf(gv[v], gv[v], ss);
-        }
-#pragma unroll
-        for (int v = 0; v < V; v += 4)
-          *reinterpret_cast<float4 *>(&g[i + v]) = make_float4(gv[v], gv[v + 1], gv[v + 2], gv[v + 3]);
-      }
+      for (int v = 0; v < V; v += 4)
+        *reinterpret_cast<float4 *>(&g[i + v]) = make_float4(gv[v], gv[v + 1], gv[v + 2], gv[v + 3]);
     }
   } else {
     for (int64_t i = threadIdx.x; i < W; i += kThreads) {
@@ -178,7 +211,19 @@ __global__ void __launch_bounds__(kThreads) gated_norm_kernel(GatedNormParams p)
 
 template <typename T>
 cudaError_t launch_t(const GatedNormParams &p, cudaStream_t s) {
-  const bool vec = (p.width % NVec<T>::V) == 0;  // rows are then whole 16-byte vectors
+  constexpr int V = NVec<T>::V;
+  const bool vec = (p.width % V) == 0;  // rows are then whole 16-byte vectors
+  const int64_t nv = (p.width + (int64_t)kThreads * V - 1) / ((int64_t)kThreads * V);
+  const unsigned grid = (unsigned)p.rows;
+  if (vec && nv <= kMaxVec) {
+    switch (nv) {
+      case 1: gated_norm_reg_kernel<T, 1><<<grid, kThreads, 0, s>>>(p); break;
+      case 2: gated_norm_reg_kernel<T, 2><<<grid, kThreads, 0, s>>>(p); break;
+      case 3: gated_norm_reg_kernel<T, 3><<<grid, kThreads, 0, s>>>(p); break;
+      default: gated_norm_reg_kernel<T, 4><<<grid, kThreads, 0, s>>>(p); break;
+    }
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)p.width * sizeof(float);
   auto kern = vec ? gated_norm_kernel<T, true> : gated_norm_kernel<T, false>;
   if (smem > 48 * 1024) {
@@ -186,7 +231,7 @@ cudaError_t launch_t(const GatedNormParams &p, cudaStream_t s) {
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  kern<<<(unsigned)p.rows, kThreads, smem, s>>>(p);
+  kern<<<grid, kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 

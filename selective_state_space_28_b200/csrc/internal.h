@@ -126,7 +126,7 @@ struct SsdSplit {
 SsdSplit ssd_tc_split(int64_t batch, int64_t H, int64_t L, int sms);
 size_t ssd_tc_split_bytes(const SsdSplit &r);
 int device_sm_count();  // the current device's SMs (148 when it cannot be read)
-int64_t conv1d_run_length(int64_t L, bool state_in_place);
+int64_t conv1d_run_length(const ConvParams &p, bool state_in_place);
 bool conv1d_supported(const ConvParams &p);
 bool gated_norm_supported(const GatedNormParams &p);
 int attn_heads_per_cta(int64_t H, int64_t G);

@@ -506,13 +506,13 @@ ssm_status_t ssm_conv1d_fwd(const ssm_conv_args_t *a, void *stream) {
   p.W = (int)a->width;
   p.io = a->io;
   p.silu = (a->flags & SSM_CONV_SILU) != 0;
-  p.run = ssm::conv1d_run_length(a->seqlen, in_place);
   p.x = a->x;
   p.w = a->w;
   p.bias = a->bias;
   p.state_in = a->state_in;
   p.u = a->u;
   p.state_out = a->width > 1 ? a->state_out : nullptr;
+  p.run = ssm::conv1d_run_length(p, in_place);
   if (!ssm::conv1d_supported(p)) return SSM_ERR_UNSUPPORTED;
   return from_cuda(ssm::launch_conv1d(p, s));
 }

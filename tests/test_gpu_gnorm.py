@@ -15,11 +15,16 @@ def _ops():
     return ops
 
 
-@pytest.mark.parametrize("width", [64, 1536, 5120, 12, 1000])
+@pytest.mark.parametrize("width", [64, 1536, 3072, 4000, 5120, 8192, 8200, 12, 1000, 1002])
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_gnorm_shapes(cuda_ok, width, io):
-    # 16-byte rows take the vector form, others (12 f32 is one; 1000 bf16 is
-    # not) the per-element form
+    # Rows of whole 16-byte vectors (8 bf16 / 4 float32 values) up to 2048
+    # values a vector slot (bf16) or 1024 (f32) per thread, four slots at
+    # most, keep the row in registers: bf16 64..1536 one slot, 3072 and 4000
+    # two, 5120 three (the last one partial), 8192 four; f32 1536 two, 3072
+    # three, 4000 four.  Wider vector rows (bf16 8200, f32 5120..8200) keep
+    # it in shared memory; 1002 and bf16 12 are not whole vectors and take
+    # the per-element form.
     d = I.gnorm_inputs(2, 17, width, io=io, seed=width)
     out = _ops().ssm_gated_rmsnorm_fwd(d["y"].cuda(), d["z"].cuda(), d["weight"].cuda(), 1e-5)
     ref = oracle.gated_rmsnorm(d["y"], d["z"], d["weight"], 1e-5)
