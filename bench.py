@@ -479,7 +479,7 @@ def bench_attn(w, K, W, dist, device, pk, seed_base):
     ms = timed(step, K, W, dist, device) / K
     launch_ms = per_launch_ms(step, max(10, K), device)
     return {"ms_per_step": ms, "bytes": nb, "launch_ms": launch_ms, "sets": len(sets),
-            "launches_per_step": 2}
+            "launches_per_step": 2}  # C . B^T with the pre-pass, the mask pass
 
 
 def bench_ssd(w, K, W, dist, device, pk, seed_base):

@@ -140,8 +140,70 @@ __global__ void __launch_bounds__(256) attn_cb_kernel(AttnParams p) {
       make_float4(acc[0], acc[1], acc[2], acc[3]);
 }
 
+// The pre-pass's running sums for one (batch, head) with 128 threads (the
+// pre-pass blocks of the fused launch below): per 1024-token round each
+// thread loads 8 consecutive tokens and sums them in order; a block-wide scan
+// of the threads' totals (warp shuffles, then the four warps' totals) gives
+// every token's running sum.
+constexpr int kPrepSmall = 128, kPrepRun = 8;
+template <typename T>
+__device__ __forceinline__ void prep_unit_small(const AttnParams &p, int64_t unit) {
+  __shared__ double wsum[kPrepSmall / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t b = unit / p.H, h = unit % p.H;
+  const T *dt = static_cast<const T *>(p.dt);
+  const double A2 = (double)p.A[h] * 1.4426950408889634;
+  const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+  double carry = 0.0;
+  for (int64_t t0 = 0; t0 < p.L; t0 += kPrepSmall * kPrepRun) {
+    const int64_t tb = t0 + (int64_t)tid * kPrepRun;
+    float d[kPrepRun];
+#pragma unroll
+    for (int j = 0; j < kPrepRun; ++j) {
+      d[j] = 0.f;
+      if (tb + j < p.L) {
+        d[j] = ld(dt + (b * p.L + tb + j) * p.H + h) + bias;
+        if (p.flags & 1u) d[j] = softplus(d[j]);
+      }
+    }
+    double run[kPrepRun], v = 0.0;
+#pragma unroll
+    for (int j = 0; j < kPrepRun; ++j) {
+      v += (double)d[j] * A2;
+      run[j] = v;  // within the thread's 8 tokens
+    }
+    double incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const double u = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += u;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    double before = carry, total = carry;
+#pragma unroll
+    for (int w = 0; w < kPrepSmall / 32; ++w) {
+      const double x = wsum[w];
+      if (w < warp) before += x;
+      total += x;
+    }
+    before += incl - v;  // the threads before this one in its warp
+#pragma unroll
+    for (int j = 0; j < kPrepRun; ++j) {
+      if (tb + j < p.L) {
+        p.beta[unit * p.L + tb + j] = d[j];
+        p.cum[unit * p.L + tb + j] = before + run[j];
+      }
+    }
+    carry = total;
+    __syncthreads();  // wsum is rewritten next round
+  }
+}
+
 // The same tile on the tensor cores (bf16 inputs, state 128): one CTA of 128
-// threads per (lower tile, group, batch).  The TMA brings the tile's 128 query
+// threads per (lower tile, group, batch); the launch's blocks past those run
+// the pre-pass (one per (batch, head)), which does not depend on C . B^T, so
+// that both take one launch.  The TMA brings the tile's 128 query
 // rows of C and 128 key rows of B as two 64-state slabs each (128-byte
 // swizzle; rows past the sequence end arrive as zeros); one thread issues the
 // eight K = 16 steps of the 128 x 128 x 128 product into 128 TMEM columns
@@ -161,10 +223,16 @@ __global__ void __launch_bounds__(128)
     attn_cb_tc_kernel(const __grid_constant__ CUtensorMap mB,
                       const __grid_constant__ CUtensorMap mC, AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int64_t ncb = p.ntri * p.G * p.batch;
+  if ((int64_t)blockIdx.x >= ncb) {
+    prep_unit_small<__nv_bfloat16>(p, (int64_t)blockIdx.x - ncb);
+    return;
+  }
   CbSmem &s = *reinterpret_cast<CbSmem *>(smem_raw +
                                           ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t li = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int64_t li = (int64_t)blockIdx.x % p.ntri, g = ((int64_t)blockIdx.x / p.ntri) % p.G,
+                b = (int64_t)blockIdx.x / (p.ntri * p.G);
   int64_t qt = (int64_t)((sqrt(8.0 * (double)li + 1.0) - 1.0) / 2.0);
   while (qt * (qt + 1) / 2 > li) --qt;
   while ((qt + 1) * (qt + 2) / 2 <= li) ++qt;
@@ -234,10 +302,47 @@ __global__ void __launch_bounds__(128)
 }
 
 // The mask pass: one CTA per (query tile, key tile, run of heads of one
-// group), 256 threads with the same element ownership as the C . B^T pass.
-// A tile above the diagonal is zeros; otherwise the thread reads its 64
-// values of C . B^T (from L2) once and, per head, scales them by the decay
-// factors and streams the rows out.
+// group, batch row), 256 threads with the same element ownership as the
+// C . B^T pass.  A tile above the diagonal is zeros; otherwise the thread
+// reads its 64 values of C . B^T (from L2) once and, per head, scales them
+// by the decay factors and streams the rows out.
+//
+// The CTAs cost unequal time (a diagonal tile takes an exponential per
+// element, a tile above it only zeros), and the grid runs several waves, so
+// the linear block index lists them dearest first -- every diagonal tile,
+// then every tile below it, then the zero tiles -- and the block scheduler,
+// which starts blocks in index order, fills the last wave with cheap ones.
+struct MaskItem {
+  int64_t qt, kt, hg, b;
+};
+__device__ __forceinline__ MaskItem mask_item(int64_t r, int64_t ntile, int64_t nhg,
+                                              int64_t batch) {
+  const int64_t hb = nhg * batch;
+  const int64_t nd = ntile * hb, nb = ntile * (ntile - 1) / 2 * hb;
+  int cls = 0;  // 0 diagonal, 1 below, 2 above
+  if (r >= nd) {
+    r -= nd;
+    cls = r >= nb ? 2 : 1;
+    if (cls == 2) r -= nb;
+  }
+  const int64_t k = r / hb, j = r % hb;
+  MaskItem m;
+  m.hg = j % nhg;
+  m.b = j / nhg;
+  if (cls == 0) {
+    m.qt = m.kt = k;
+  } else {
+    // the k-th tile strictly below the diagonal, row by row: qt (qt - 1) / 2 <= k
+    int64_t qt = (int64_t)((1.0 + sqrt(1.0 + 8.0 * (double)k)) / 2.0);
+    while (qt * (qt - 1) / 2 > k) --qt;
+    while ((qt + 1) * qt / 2 <= k) ++qt;
+    const int64_t kt = k - qt * (qt - 1) / 2;
+    m.qt = cls == 1 ? qt : kt;  // the zero tiles are the mirror images
+    m.kt = cls == 1 ? kt : qt;
+  }
+  return m;
+}
+
 __global__ void __launch_bounds__(256) attn_mask_kernel(AttnParams p) {
   __shared__ __align__(16) float colf[kHeadsPerCta][kTile];  // per key: exp2(cum_r - cum_s) beta_s
   __shared__ __align__(16) float betas[kHeadsPerCta][kTile];
@@ -246,10 +351,12 @@ __global__ void __launch_bounds__(256) attn_mask_kernel(AttnParams p) {
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const int64_t L = p.L, H = p.H;
   const int64_t ntile = (L + kTile - 1) / kTile;
-  const int64_t qt = blockIdx.x / ntile, kt = blockIdx.x % ntile;
+  const MaskItem mi =
+      mask_item(blockIdx.x, ntile, (H + p.heads_per_cta - 1) / p.heads_per_cta, p.batch);
+  const int64_t qt = mi.qt, kt = mi.kt;
   const int64_t t0 = qt * kTile, s0 = kt * kTile;
-  const int64_t b = blockIdx.z;
-  const int64_t h0 = (int64_t)blockIdx.y * p.heads_per_cta;
+  const int64_t b = mi.b;
+  const int64_t h0 = mi.hg * p.heads_per_cta;
   const int nh = (int)(H - h0 < p.heads_per_cta ? H - h0 : p.heads_per_cta);
   const int64_t g = h0 / (H / p.G);
 
@@ -393,9 +500,7 @@ __global__ void __launch_bounds__(256) attn_mask_kernel(AttnParams p) {
 template <typename T>
 cudaError_t launch_t(const AttnParams &p, cudaStream_t s) {
   const int64_t units = p.batch * p.H;
-  attn_prep_kernel<T><<<(unsigned)units, kPrep, 0, s>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
   if (std::is_same<T, __nv_bfloat16>::value && p.N == 128) {
     // tensor-core C . B^T: B and C as [batch, L, G * 128] bf16, 64 x 128 boxes
     const uint64_t GN = (uint64_t)(p.G * 128);
@@ -413,18 +518,21 @@ cudaError_t launch_t(const AttnParams &p, cudaStream_t s) {
     const cudaError_t attr = cudaFuncSetAttribute(
         attn_cb_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (attr != cudaSuccess) return attr;
-    attn_cb_tc_kernel<<<dim3((unsigned)p.ntri, (unsigned)p.G, (unsigned)p.batch), 128, smem, s>>>(
-        mB, mC, p);
+    // C . B^T blocks first (the longer ones), then the pre-pass blocks
+    attn_cb_tc_kernel<<<(unsigned)(p.ntri * p.G * p.batch + units), 128, smem, s>>>(mB, mC, p);
   } else {
+    attn_prep_kernel<T><<<(unsigned)units, kPrep, 0, s>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     attn_cb_kernel<T><<<dim3((unsigned)(16 * p.ntri), (unsigned)p.G, (unsigned)p.batch), 256, 0,
                         s>>>(p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t ntile = (p.L + kTile - 1) / kTile;
-  dim3 grid((unsigned)(ntile * ntile), (unsigned)((p.H + p.heads_per_cta - 1) / p.heads_per_cta),
-            (unsigned)p.batch);
-  attn_mask_kernel<<<grid, 256, 0, s>>>(p);
+  const int64_t nblocks =
+      ntile * ntile * ((p.H + p.heads_per_cta - 1) / p.heads_per_cta) * p.batch;
+  attn_mask_kernel<<<(unsigned)nblocks, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -441,7 +549,10 @@ int attn_heads_per_cta(int64_t H, int64_t G) {
 
 bool attention_supported(const AttnParams &p) {
   const int64_t ntile = (p.L + kTile - 1) / kTile;
-  return p.N >= 1 && p.N <= 256 && ntile * ntile < (1ll << 31) &&
+  const int64_t nhg = (p.H + p.heads_per_cta - 1) / p.heads_per_cta;
+  const int64_t ntri = ntile * (ntile + 1) / 2;
+  return p.N >= 1 && p.N <= 256 && ntile * ntile * nhg * p.batch < (1ll << 31) &&
+         ntri * p.G * p.batch + p.batch * p.H < (1ll << 31) &&
          16 * (ntile * (ntile + 1) / 2) < (1ll << 31) && p.batch <= 65535 &&
          p.G <= 65535 && (p.H + p.heads_per_cta - 1) / p.heads_per_cta <= 65535;
 }

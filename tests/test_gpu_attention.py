@@ -55,6 +55,18 @@ def test_attention_tensor_core_tiles(cuda_ok, L, G):
     assert torch.count_nonzero(torch.triu(al, 1)) == 0
 
 
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_attention_long_batched(cuda_ok, io):
+    # more than one 1024-token round of the running sums (the second one
+    # ragged), two batch rows and two groups: bf16 with state 128 runs the
+    # C . B^T tiles and the running sums in one launch, f32 the two passes
+    d = I.ssd_inputs(2, 1100, 4, 16, 128, groups=2, io=io, seed=77)
+    al = _run(d)
+    ref = oracle.m2_attention(d["dt"], d["B"], d["C"], d["A"], d["dt_bias"])
+    assert_close_normwise(al, ref, REL[torch.float32], "alpha")
+    assert torch.count_nonzero(torch.triu(al, 1)) == 0
+
+
 def test_attention_without_softplus(cuda_ok):
     d = I.ssd_inputs(1, 90, 2, 16, 32, io="f32", seed=3)
     d["dt"] = d["dt"].abs() * 0.1   # a positive step without softplus, and no bias
