@@ -585,7 +585,9 @@ def bench_decode(w, K, W, dist, device, pk, seed_base):
 
 def e2e_m1(w, device, n_steps=5):
     """The same metric through the public API with pinned HOST buffers: each
-    step copies its inputs host->device, scans, and reads y and h_last back."""
+    step copies its inputs host->device, scans, and reads y and h_last back
+    (ssm_scan_fwd_host: batch-row chunks, the two directions' copies
+    overlapped with each other and with the scans)."""
     import torch
     from selective_state_space_28_b200 import inputs as I
     from selective_state_space_28_b200 import ops

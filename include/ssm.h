@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define SSM_ABI_VERSION 3
+#define SSM_ABI_VERSION 4
 
 typedef enum ssm_status {
   SSM_OK = 0,
@@ -157,6 +157,38 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_args_t *args, void *stream);
  * streams, or from several threads -- race on it and must be serialised by
  * the caller.  ssm_workspace_status(NULL, stream) reads its status word. */
 ssm_status_t ssm_scan_fwd_static(const ssm_scan_args_t *args, void *stream);
+
+/* ssm_scan_fwd_host -- ssm_scan_fwd for a caller whose tensors live in HOST
+ * memory.
+ *
+ * The pages have no counterpart: this is the end-to-end form of the same
+ * scan.  x, dt, z, B, C, A, D, dt_bias, h0 are host pointers to the inputs,
+ * y, h_last (and states, when not NULL) host pointers that receive the
+ * results, all in ssm_scan_fwd's layouts; args->workspace is DEVICE memory
+ * of ssm_scan_host_workspace() bytes (two chunks' device copies of the
+ * inputs and results, the per-channel constants and the scan's own
+ * workspace; its first word is the status word, as for ssm_scan_fwd).
+ *
+ * The batch rows are taken in up to 8 chunks: while one chunk is scanned on
+ * `stream`, the next chunk's inputs are copied in and the previous chunk's
+ * results copied out on two streams of the library's own (created once per
+ * device, on first use), so that the two directions' copies overlap each
+ * other and the scans; `stream` waits for both copy streams before the call
+ * returns, so a synchronize of `stream` (or work queued on it after the
+ * call) sees every result.  With page-locked (pinned) host buffers the call
+ * only enqueues; pageable buffers work too, but the runtime then copies them
+ * synchronously and nothing overlaps.  The caller must leave the inputs
+ * unchanged and not read the outputs until `stream` has completed the call.
+ * Results are bitwise those of ssm_scan_fwd on the same inputs (every chunk
+ * runs the same kernels on its rows; the sequence is never cut into
+ * segments when there is more than one chunk).  With seqlen 0 the call
+ * synchronises `stream` and fills h_last from h0 (or zeros) on the host.
+ * Calls from several threads are enqueued one at a time (a lock per device);
+ * each needs its own workspace.  Errors: those of ssm_scan_fwd, checked
+ * before anything is enqueued; SSM_ERR_CUDA when a copy or an event cannot
+ * be enqueued (stream then still waits for what was enqueued). */
+ssm_status_t ssm_scan_host_workspace(const ssm_scan_args_t *args, size_t *bytes);
+ssm_status_t ssm_scan_fwd_host(const ssm_scan_args_t *args, void *stream);
 
 /* ssm_scan_fwd_write -- ssm_scan_fwd with the state written at one token.
  *

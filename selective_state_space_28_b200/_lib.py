@@ -123,7 +123,11 @@ def lib():
                                               ctypes.POINTER(ctypes.c_size_t)]
         L.ssm_scan_fwd_static.argtypes = [ctypes.POINTER(ScanArgs), _vp]
         L.ssm_workspace_status.argtypes = [_vp, _vp]
-        for fn in (L.ssm_scan_fwd_static, L.ssm_workspace_status,
+        L.ssm_scan_fwd_host.argtypes = [ctypes.POINTER(ScanArgs), _vp]
+        L.ssm_scan_host_workspace.argtypes = [ctypes.POINTER(ScanArgs),
+                                              ctypes.POINTER(ctypes.c_size_t)]
+        for fn in (L.ssm_scan_fwd_static, L.ssm_workspace_status, L.ssm_scan_fwd_host,
+                   L.ssm_scan_host_workspace,
                    L.ssm_scan_fwd, L.ssm_scan_workspace, L.ssd_chunk_scan_fwd,
                    L.ssd_chunk_scan_workspace, L.ssd_conv_chunk_scan_fwd,
                    L.ssd_conv_chunk_scan_workspace, L.ssm_scan_step, L.ssm_conv1d_fwd,

@@ -156,8 +156,13 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
 // The Mamba-1 scan behind ssm_scan_fwd, ssm_scan_fwd_write (t_write >= 0)
 // and ssm_scan_fwd_static (allow_cut false: the sequence is never cut into
 // segments, so the workspace is the status word and the dt-norm factors).
+// reset_status false leaves the status word as it is (a caller that runs
+// several scans against one status word clears it once).
 ssm_status_t scan_run(const ssm_scan_args_t *a, int64_t t_write, const float *state_write,
-                      void *stream, bool allow_cut);
+                      void *stream, bool allow_cut, bool reset_status = true);
+// The workspace bytes scan_run needs for these shapes and flags (pointers
+// not looked at; allow_cut as in scan_run).
+size_t scan_workspace_bytes(const ssm_scan_args_t *a, bool allow_cut);
 // Every host-side check of ssm_scan_fwd (pointers included), touching no
 // device: SSM_OK or the error status.
 ssm_status_t scan_validate(const ssm_scan_args_t *a);

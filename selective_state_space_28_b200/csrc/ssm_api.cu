@@ -216,8 +216,12 @@ ssm_status_t scan_validate(const ssm_scan_args_t *a) {
   return check_scan(a, &ws, false, false);
 }
 
+size_t scan_workspace_bytes(const ssm_scan_args_t *a, bool allow_cut) {
+  return m1_layout(a, device_sm_count(), allow_cut).total;
+}
+
 ssm_status_t scan_run(const ssm_scan_args_t *a, int64_t t_write, const float *state_write,
-                      void *stream, bool allow_cut) {
+                      void *stream, bool allow_cut, bool reset_status) {
   size_t ws = 0;
   ssm_status_t st = check_scan(a, &ws);
   if (st != SSM_OK) return st;
@@ -226,7 +230,8 @@ ssm_status_t scan_run(const ssm_scan_args_t *a, int64_t t_write, const float *st
   if (!a->workspace || a->workspace_bytes < lay.total) return SSM_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int *status = static_cast<int *>(a->workspace);
-  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return SSM_ERR_CUDA;
+  if (reset_status && cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess)
+    return SSM_ERR_CUDA;
   if (a->seqlen == 0)
     return pass_state(a->h0, a->h_last,
                       (size_t)(a->batch * a->channels * a->state) * sizeof(float), s);

@@ -8,7 +8,9 @@ CUDA kernels; if ``libssm.so`` is missing these functions raise.
 Host tensors are accepted too: they are copied to the GPU on the current
 stream, the call runs there, the outputs are copied back into host tensors
 (pinned when the inputs were pinned) and the stream is synchronised before
-returning.  This is the end-to-end path a caller with host buffers uses.
+returning.  This is the end-to-end path a caller with host buffers uses; for
+ssm_scan_fwd it is the library's own ssm_scan_fwd_host, which overlaps the
+copies in both directions with each other and with the scan.
 """
 import ctypes
 
@@ -103,6 +105,9 @@ def ssm_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
     states [b, L, C, N] f32 or None).  With check=True (always for host
     tensors) the stream is synchronised and an expired device wait raises."""
     sg = _Staging([x, dt, A, B, C, D, z, dt_bias, h0])
+    if sg.host and _write is None:
+        return _scan_host(x, dt, A, B, C, D, z, dt_bias, h0, flags, rms_eps, want_states,
+                          y, h_last, workspace, sg, stream)
     x, dt, A, B, C, D, z, dt_bias, h0 = map(sg.dev, (x, dt, A, B, C, D, z, dt_bias, h0))
     if _write is not None:
         _write = (_write[0], sg.dev(_write[1]))
@@ -132,6 +137,38 @@ def ssm_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *,
     if check or sg.host or _CHECK_ALL:
         _check_status(ws, st, "ssm_scan_fwd")
     return sg.back((y, h_last, states))
+
+
+def _scan_host(x, dt, A, B, C, D, z, dt_bias, h0, flags, rms_eps, want_states, y, h_last,
+               workspace, sg, stream):
+    """ssm_scan_fwd on host tensors through ssm_scan_fwd_host: outputs are host
+    tensors (the given ones, else new ones, pinned when the inputs are), the
+    workspace device memory; the stream is synchronised and the status word
+    checked before returning."""
+    x, dt, A, B, C, D, z, dt_bias, h0 = (None if t is None else t.contiguous()
+                                         for t in (x, dt, A, B, C, D, z, dt_bias, h0))
+    b, Lq, Cn = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if y is None:
+        y = torch.empty(x.shape, dtype=x.dtype, pin_memory=sg.pinned)
+    if h_last is None:
+        h_last = torch.empty((b, Cn, N), dtype=torch.float32, pin_memory=sg.pinned)
+    states = (torch.empty((b, Lq, Cn, N), dtype=torch.float32, pin_memory=sg.pinned)
+              if want_states else None)
+    a = L.ScanArgs(batch=b, seqlen=Lq, channels=Cn, state=N, groups=G, io=_io_of(x),
+                   flags=flags, rms_eps=rms_eps, x=_ptr(x), dt=_ptr(dt), z=_ptr(z),
+                   B=_ptr(B), C=_ptr(C), A=_ptr(A), D=_ptr(D), dt_bias=_ptr(dt_bias),
+                   h0=_ptr(h0), y=_ptr(y), h_last=_ptr(h_last), states=_ptr(states))
+    lib = L.lib()
+    nbytes = ctypes.c_size_t(0)
+    L.check(lib.ssm_scan_host_workspace(ctypes.byref(a), ctypes.byref(nbytes)),
+            "ssm_scan_host_workspace")
+    ws = _workspace(nbytes.value, workspace, sg.device)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), nbytes.value
+    st = _stream(stream, sg.device)
+    L.check(lib.ssm_scan_fwd_host(ctypes.byref(a), st), "ssm_scan_fwd_host")
+    _check_status(ws, st, "ssm_scan_fwd_host")
+    return y, h_last, states
 
 
 def ssm_scan_fwd_write(x, dt, A, B, C, D=None, z=None, dt_bias=None, h0=None, *, t, state,

@@ -45,7 +45,7 @@ def test_no_runtime_symbols_leak(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.ssm_abi_version() == 3
+    assert lib.ssm_abi_version() == 4
     for s in range(9):
         assert lib.ssm_status_string(s)
     assert lib.ssm_status_string(99) == b"unknown status"
@@ -135,6 +135,54 @@ def test_static_entry_checks_before_touching_the_device(lib):
     # batch 0: nothing to do
     assert fn(ctypes.byref(_scan(batch=0, x=None, dt=None, B=None, C=None, A=None,
                                  y=None)), None) == OK
+
+
+def test_host_entry_checks_before_touching_the_device(lib):
+    """ssm_scan_fwd_host runs ssm_scan_fwd's checks, then the workspace
+    check, before anything is enqueued: on a host with no GPU a bad call
+    returns its own status."""
+    fn = lib.ssm_scan_fwd_host
+    assert fn(None, None) == NULL
+    assert fn(ctypes.byref(_scan(x=None)), None) == NULL
+    assert fn(ctypes.byref(_scan(x=P + 2)), None) == ALIGN
+    assert fn(ctypes.byref(_scan(state=12)), None) == UNSUP
+    assert fn(ctypes.byref(_scan(io=7)), None) == DTYPE
+    assert fn(ctypes.byref(_scan(workspace=P, workspace_bytes=255)), None) == WS
+    assert fn(ctypes.byref(_scan(batch=0, x=None, dt=None, B=None, C=None, A=None,
+                                 y=None)), None) == OK
+
+
+def _host_ws(lib, **kw):
+    n = ctypes.c_size_t(0)
+    assert lib.ssm_scan_host_workspace(ctypes.byref(_scan(**kw)), ctypes.byref(n)) == OK
+    return n.value
+
+
+def test_host_workspace_layout(lib):
+    """The host entry's device workspace: the scans' own workspace, the
+    per-channel constants, then one chunk's copies of the inputs and results
+    per slot (two slots when the batch is cut into chunks), each piece
+    rounded up to 256 bytes.  The headline shape (b8 L2048 C1536 N16 bf16,
+    gate and h_last) runs 8 one-row chunks, never cut along the sequence."""
+    big = dict(batch=8, seqlen=2048, channels=1536, state=16, z=P, h_last=P)
+    seq = 2048 * 1536 * 2          # x, dt, z or y of one row
+    bc = 2048 * 16 * 2             # B or C of one row
+    state = 1536 * 16 * 4          # h_last of one row
+    slot = 4 * seq + 2 * bc + state
+    assert _host_ws(lib, **big) == 256 + 1536 * 16 * 4 + 2 * slot
+    # D and dt_bias add one 256-byte-rounded channel vector each
+    assert _host_ws(lib, D=P, dt_bias=P, **big) == 256 + 1536 * 16 * 4 + 2 * 6144 + 2 * slot
+    # 17 rows: 6 chunks of up to 3 rows
+    r17 = dict(big, batch=17)
+    assert _host_ws(lib, **r17) == 256 + 1536 * 16 * 4 + 2 * 3 * slot
+    # one row: one chunk, one slot, and the scan's workspace holds the
+    # segments of the sequence cut (the same size ssm_scan_workspace asks)
+    one = dict(big, batch=1)
+    n = ctypes.c_size_t(0)
+    assert lib.ssm_scan_workspace(ctypes.byref(_scan(**one)), ctypes.byref(n)) == OK
+    cut_ws = (n.value + 255) // 256 * 256
+    assert cut_ws > 256
+    assert _host_ws(lib, **one) == cut_ws + 1536 * 16 * 4 + slot
 
 
 def test_workspace_status_needs_a_stream_copy(lib):
