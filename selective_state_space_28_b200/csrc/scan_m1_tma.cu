@@ -16,19 +16,19 @@
 //
 // Per stage, every warp (no CTA-wide barrier anywhere in the loop):
 //   1. waits for the stage's bytes (mbarrier `full`);
-//   2. widens (and, with SSM_RMSNORM_BC, RMS-normalises) its share of the
-//      stage's B and C rows into float32;
-//   3. for its share of the stage's tokens and all 32 channels computes
-//      d = softplus(dt rstd + bias), d x, D x and silu(z), then arrives on
-//      `conv`;
-//   4. waits on `conv` (every warp's share), then runs the recurrence: per
-//      token each lane updates its four states with packed f32x2 arithmetic
-//      and forms its partial C.h, the decays of the next 8 tokens formed
-//      while the current 8 run their chain; every G tokens the G lanes of a
-//      channel trade partials in log2(G) shuffle rounds so that lane q ends
-//      with token q's complete C.h (a transposing reduction), and applies the
-//      skip term, the gate and the rounding for that token;
-//   5. arrives on `empty` (the issuing thread refills a stage's buffer once
+//   2. for its share of the stage's tokens and all 32 channels computes
+//      d = softplus(dt rstd + bias), d x, D x and silu(z) (with
+//      SSM_RMSNORM_BC also each token's 1/rms of B_t, folded into d x, and
+//      of C_t, kept for the readout), then arrives on `conv`;
+//   3. waits on `conv` (every warp's share), then runs the recurrence, B and
+//      C read as they landed: per token each lane updates its four states
+//      with packed f32x2 arithmetic and forms its partial C.h, the decays of
+//      the next 8 tokens formed while the current 8 run their chain; every G
+//      tokens the G lanes of a channel trade partials in log2(G) shuffle
+//      rounds so that lane q ends with token q's complete C.h (a transposing
+//      reduction), and applies C_t's factor, the skip term, the gate and the
+//      rounding for that token;
+//   4. arrives on `empty` (the issuing thread refills a stage's buffer once
 //      every warp has released it) and stores its rows of the previous
 //      stage's y, which every warp has finished by now, in whole 64-byte
 //      rows.
@@ -77,7 +77,6 @@ struct alignas(128) ScanSmem {
   T z[NS][kTL][kCT];
   T B[NS][kTL][N];
   T C[NS][kTL][N];
-  float bc[NS][kTL][2][N];  // B, C widened to float32 (and normed)
   // Per (token, channel) of a stage: (d, d*x) for the recurrence and
   // (D*x, silu(z)) for the epilogue.  Two buffers by stage parity: a warp
   // that has finished stage s writes stage s+1's values while another still
@@ -86,6 +85,9 @@ struct alignas(128) ScanSmem {
   // warp's lanes, one row each, fall in distinct banks.
   float2 ddx[2][kTL][kCT + 2];
   float2 eg[2][kTL][kCT + 2];
+  // With RMS norms on B and C: each token's factor 1 / rms(C_t), by stage
+  // parity like eg (the factor of B_t is folded into d * x).
+  float rc[2][kTL];
   // Output staging, two buffers by stage parity: the warps write stage s's y
   // here, and during stage s+1 (once the `conv` barrier shows every warp has
   // finished stage s) each warp stores a quarter of its rows to global
@@ -126,17 +128,28 @@ __device__ __forceinline__ void widen(const T *src, float (&v)[J]) {
       const uint4 w = *reinterpret_cast<const uint4 *>(src);
       v[0] = bf16lo(w.x); v[1] = bf16hi(w.x); v[2] = bf16lo(w.y); v[3] = bf16hi(w.y);
       v[4] = bf16lo(w.z); v[5] = bf16hi(w.z); v[6] = bf16lo(w.w); v[7] = bf16hi(w.w);
-    } else {
-      static_assert(J == 4, "4 or 8 values");
+    } else if constexpr (J == 4) {
       const uint2 w = *reinterpret_cast<const uint2 *>(src);
       v[0] = bf16lo(w.x); v[1] = bf16hi(w.x); v[2] = bf16lo(w.y); v[3] = bf16hi(w.y);
+    } else if constexpr (J == 2) {
+      const uint32_t w = *reinterpret_cast<const uint32_t *>(src);
+      v[0] = bf16lo(w); v[1] = bf16hi(w);
+    } else {
+      static_assert(J == 1, "1, 2, 4 or 8 values");
+      v[0] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(src));
     }
-  } else {
+  } else if constexpr (J == 1) {
+    v[0] = *reinterpret_cast<const float *>(src);
+  } else if constexpr (J % 4 == 0) {
 #pragma unroll
     for (int i = 0; i < J; i += 4) {
       const float4 a = *reinterpret_cast<const float4 *>(src + i);
       v[i] = a.x; v[i + 1] = a.y; v[i + 2] = a.z; v[i + 3] = a.w;
     }
+  } else {
+    static_assert(J == 2, "2 or a multiple of 4 values");
+    const float2 a = *reinterpret_cast<const float2 *>(src);
+    v[0] = a.x; v[1] = a.y;
   }
 }
 
@@ -192,7 +205,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
   constexpr int NP = SPL / 2;       // state pairs per lane
   constexpr int CPW = 32 / G;       // channels per warp
   constexpr int NW = kCT / CPW;     // warps per CTA
-  constexpr int TPW = kTL / NW;     // B/C rows each warp widens per stage
+  constexpr int TPW = kTL / NW;     // tokens each warp prepares per stage
   constexpr bool kBF16 = sizeof(T) == 2;
   constexpr bool kFull = MODE == kModeFull;
   static_assert(N % 8 == 0 || !kBF16, "bf16 rows of B and C are 16-byte multiples");
@@ -308,44 +321,40 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
       failed = true;
       break;
     }
-    // ---- 2. with RMS norms on B and C, widen and normalise this warp's
-    // share of the stage's B and C rows (without them the recurrence reads
-    // B and C straight from the stage: half the shared-memory wavefronts of
-    // the widened float32 rows)
-    if constexpr (rms_bc)
-    for (int e = lane; e < TPW * 2; e += 32) {
-      const int t = warp * TPW + (e >> 1), which = e & 1;
-      const T *src = which ? s.C[buf][t] : s.B[buf][t];
-      float *dst = s.bc[buf][t][which];
-      float v[N];
-      constexpr int J = N % 8 == 0 ? 8 : 4;
-#pragma unroll
-      for (int n = 0; n < N; n += J) {
-        float w[J];
-        widen<J>(src + n, w);
-#pragma unroll
-        for (int i = 0; i < J; ++i) v[n + i] = w[i];
-      }
-      float r = 1.f;
-      if (rms_bc) {
-        float ss = 0.f;
-#pragma unroll
-        for (int n = 0; n < N; ++n) ss += v[n] * v[n];
-        r = rsqrtf(ss / N + p.eps);
-      }
-#pragma unroll
-      for (int n = 0; n < N; n += 4)
-        *reinterpret_cast<float4 *>(dst + n) =
-            make_float4(v[n] * r, v[n + 1] * r, v[n + 2] * r, v[n + 3] * r);
-    }
-
-    // ---- 3. per (token, channel) of this warp's tokens, all 32 channels:
+    // ---- 2. per (token, channel) of this warp's tokens, all 32 channels:
     // d = softplus(dt * rstd + bias), d * x, D * x and the gate factor.  Four
     // lanes share a token, each taking 8 channels (conflict-free 16-byte rows).
+    // With RMS norms on B and C the four also form the token's two factors
+    // 1 / rms over the state (a quarter of B_t and C_t each, summed across
+    // the four): B_t's multiplies d * x, so that the recurrence's write term
+    // d x (B_t / rms(B_t)) needs B_t only as it landed; C_t's is kept for the
+    // readout, which scales the reduced C_t . h once.  The recurrence reads
+    // B and C as bfloat16 straight from the stage either way.
     for (int e = lane; e < TPW * 4; e += 32) {
       const int t = warp * TPW + (e >> 2), k0 = (e & 3) * 8;
       const bool tvalid = t < tn;
       const float rs = (tvalid && p.rstd) ? p.rstd[b * L + t0 + t] : 1.f;
+      float rb = 1.f;
+      if constexpr (rms_bc) {
+        constexpr int PN = N / 4;  // values of B_t (and of C_t) per lane of the four
+        // (a token's four lanes are all in the loop or all out of it)
+        const unsigned quad = 0xfu << (lane & 28);
+        float vb[PN], vc[PN];
+        widen<PN>(&s.B[buf][t][(e & 3) * PN], vb);
+        widen<PN>(&s.C[buf][t][(e & 3) * PN], vc);
+        float sb = 0.f, sc = 0.f;
+#pragma unroll
+        for (int i = 0; i < PN; ++i) {
+          sb = fmaf(vb[i], vb[i], sb);
+          sc = fmaf(vc[i], vc[i], sc);
+        }
+        sb += __shfl_xor_sync(quad, sb, 1);
+        sc += __shfl_xor_sync(quad, sc, 1);
+        sb += __shfl_xor_sync(quad, sb, 2);
+        sc += __shfl_xor_sync(quad, sc, 2);
+        rb = rsqrtf(sb / N + p.eps);
+        if ((e & 3) == 0) s.rc[sg & 1][t] = rsqrtf(sc / N + p.eps);
+      }
       float xv[8], dv[8], zv[8];
       widen<8>(&s.x[buf][t][k0], xv);
       widen<8>(&s.dt[buf][t][k0], dv);
@@ -355,7 +364,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
       for (int i = 0; i < 8; ++i) {
         float d = fmaf(dv[i], rs, biasr[i]);
         if (softplus_on) d = softplus_sfu(d);
-        o[i] = tvalid ? make_float2(d, d * xv[i]) : make_float2(0.f, 0.f);
+        o[i] = tvalid ? make_float2(d, d * xv[i] * rb) : make_float2(0.f, 0.f);
         const float gate = HAS_Z ? (kBF16 ? silu_tanh(zv[i]) : silu(zv[i])) : 1.f;
         og[i] = make_float2(skipr[i] * xv[i], gate);
       }
@@ -373,7 +382,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
       break;
     }
 
-    // ---- 4. the recurrence.  Tokens go in steps of SL; the decays and
+    // ---- 3. the recurrence.  Tokens go in steps of SL; the decays and
     // write terms of step k+1 (independent of the state) are formed while
     // step k runs its chain, and the readout of step k-1 is reduced and
     // stored meanwhile, so that a warp always has independent work at hand.
@@ -391,8 +400,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
         const int t = tg + u;
         const float2 dd = s.ddx[sg & 1][t][cw0 + ch];
         f2 bv[NP];
-        if constexpr (rms_bc) load_pairs<NP>(&s.bc[buf][t][0][SPL * q], bv);
-        else load_pairs_io<NP>(&s.B[buf][t][SPL * q], bv);
+        load_pairs_io<NP>(&s.B[buf][t][SPL * q], bv);
         const f2 d2 = mk2(dd.x, dd.x), dx2 = mk2(dd.y, dd.y);
 #pragma unroll
         for (int j = 0; j < NP; ++j) {
@@ -418,7 +426,8 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
         const float yq = transpose_reduce<G>(pg, q);
         const int tt = tg + G * k + q;
         const float2 eg = s.eg[sg & 1][tt][cw0 + ch];
-        st(&s.y[sg & 1][tt][cw0 + ch], (yq + eg.x) * eg.y);
+        const float ch_ = rms_bc ? fmaf(yq, s.rc[sg & 1][tt], eg.x) : yq + eg.x;
+        st(&s.y[sg & 1][tt][cw0 + ch], ch_ * eg.y);
       }
     };
     Pre cur, nxt;
@@ -446,8 +455,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
           }
           if (kFull) {
             f2 cv[NP];
-            if constexpr (rms_bc) load_pairs<NP>(&s.bc[buf][t][1][SPL * q], cv);
-            else load_pairs_io<NP>(&s.C[buf][t][SPL * q], cv);
+            load_pairs_io<NP>(&s.C[buf][t][SPL * q], cv);
             f2 acc = mul2(cv[0], h[0]);
 #pragma unroll
             for (int j = 1; j < NP; ++j) acc = fma2(cv[j], h[j], acc);
@@ -470,7 +478,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
     }
     if (kFull) finish(kTL - SL, partp);
     mbar_arrive(&s.empty[buf]);
-    // ---- 5. y of the previous stage: every warp has finished it (they all
+    // ---- 4. y of the previous stage: every warp has finished it (they all
     // arrived on this stage's `conv`), so this warp stores its share of the
     // rows, after its own recurrence (measured: 2 % faster than storing them
     // before it, 5 % faster than each warp storing its own 16-byte rows)
