@@ -153,8 +153,30 @@ __global__ void __launch_bounds__(kCT *(N / 4))
         make_float4(h[0], h[1], h[2], h[3]);
 }
 
+// Sum of squares of the values in one 16-byte vector of the I/O type.
+__device__ __forceinline__ float sumsq16(const uint4 &w, const __nv_bfloat16 *) {
+  float s = 0.f;
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a = bf16lo(u[i]), b = bf16hi(u[i]);
+    s = fmaf(a, a, s);
+    s = fmaf(b, b, s);
+  }
+  return s;
+}
+__device__ __forceinline__ float sumsq16(const uint4 &w, const float *) {
+  const float a = __uint_as_float(w.x), b = __uint_as_float(w.y), c = __uint_as_float(w.z),
+              d = __uint_as_float(w.w);
+  return fmaf(a, a, fmaf(b, b, fmaf(c, c, d * d)));
+}
+
 // Per (batch, token) RMS factor of the step input over the channels:
-// rstd = 1 / sqrt(mean_c(dt^2) + eps).  One warp per row.
+// rstd = 1 / sqrt(mean_c(dt^2) + eps).  One warp per row.  Rows of whole
+// 16-byte vectors (the base is 16-byte aligned) are read a vector per lane,
+// four vectors in flight per lane, so that the pass streams at the HBM rate
+// rather than at the rate of 2-byte load instructions; other rows value by
+// value.
 template <typename T>
 __global__ void dt_rms_kernel(const T *__restrict__ dt, int64_t rows, int64_t C,
                               float eps, float *__restrict__ rstd) {
@@ -163,9 +185,21 @@ __global__ void dt_rms_kernel(const T *__restrict__ dt, int64_t rows, int64_t C,
   if (row >= rows) return;
   const T *r = dt + row * C;
   float ss = 0.f;
-  for (int64_t c = lane; c < C; c += 32) {
-    const float v = ld(r + c);
-    ss += v * v;
+  constexpr int V = 16 / (int)sizeof(T);  // values per vector
+  if (C % V == 0) {
+    const uint4 *r4 = reinterpret_cast<const uint4 *>(r);
+    const int64_t nv = C / V;
+    int64_t i = lane;
+    for (; i + 96 < nv; i += 128) {
+      const uint4 a = r4[i], b = r4[i + 32], c = r4[i + 64], d = r4[i + 96];
+      ss += (sumsq16(a, r) + sumsq16(b, r)) + (sumsq16(c, r) + sumsq16(d, r));
+    }
+    for (; i < nv; i += 32) ss += sumsq16(r4[i], r);
+  } else {
+    for (int64_t c = lane; c < C; c += 32) {
+      const float v = ld(r + c);
+      ss += v * v;
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);

@@ -88,6 +88,18 @@ def test_rms_norms(cuda_ok, flags):
     _check(d, _run(d, flags=flags), _oracle(d, flags=flags), REL[torch.bfloat16])
 
 
+@pytest.mark.parametrize("io,C", [("bf16", 200), ("bf16", 8200), ("bf16", 100), ("f32", 1032),
+                                  ("f32", 1030)])
+def test_step_norm_widths(cuda_ok, io, C):
+    # the step-norm pre-pass: rows of whole 16-byte vectors (bf16 200: a
+    # partial round of lanes; 8200: four-vector rounds and a remainder; f32
+    # 1032) read by vector, others (bf16 100, f32 1030) value by value
+    d = I.m1_inputs(2, 9, C, 16, io=io, seed=C, h0=True)
+    flags = I.SOFTPLUS | I.RMS_DT
+    _check(d, _run(d, flags=flags), _oracle(d, flags=flags),
+           REL[torch.bfloat16 if io == "bf16" else torch.float32])
+
+
 def test_zero_step_skips_token_bitwise(cuda_ok):
     """dt_raw = -inf -> softplus step exactly 0 -> states[:, 3] == states[:, 2]."""
     d = I.m1_inputs(2, 20, 64, 16, io="f32", seed=11, h0=True)
