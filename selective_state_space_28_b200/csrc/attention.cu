@@ -223,6 +223,9 @@ __global__ void __launch_bounds__(128)
     attn_cb_tc_kernel(const __grid_constant__ CUtensorMap mB,
                       const __grid_constant__ CUtensorMap mC, AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the mask pass may start now: its zero tiles need nothing from this
+  // launch, and its other tiles wait for it to finish (griddepcontrol.wait)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t ncb = p.ntri * p.G * p.batch;
   if ((int64_t)blockIdx.x >= ncb) {
     prep_unit_small<__nv_bfloat16>(p, (int64_t)blockIdx.x - ncb);
@@ -319,11 +322,11 @@ __device__ __forceinline__ MaskItem mask_item(int64_t r, int64_t ntile, int64_t 
                                               int64_t batch) {
   const int64_t hb = nhg * batch;
   const int64_t nd = ntile * hb, nb = ntile * (ntile - 1) / 2 * hb;
-  int cls = 0;  // 0 diagonal, 1 below, 2 above
-  if (r >= nd) {
-    r -= nd;
-    cls = r >= nb ? 2 : 1;
-    if (cls == 2) r -= nb;
+  int cls = 2;  // 2 above (zeros), 0 diagonal, 1 below
+  if (r >= nb) {
+    r -= nb;
+    cls = r >= nd ? 1 : 0;
+    if (cls == 1) r -= nd;
   }
   const int64_t k = r / hb, j = r % hb;
   MaskItem m;
@@ -385,6 +388,8 @@ __global__ void __launch_bounds__(256) attn_mask_kernel(AttnParams p) {
       for (int i = 0; i < 8; ++i) store_row(h0 + hh, i, zero);
     return;
   }
+  // C . B^T and the running sums come from the launch before this one
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // every head's factors first (threads 0..127: one key each; 128..255: one
   // query each), read straight from the running sums -- all of a thread's
   // loads issued before any is used; one barrier
@@ -532,8 +537,19 @@ cudaError_t launch_t(const AttnParams &p, cudaStream_t s) {
   const int64_t ntile = (p.L + kTile - 1) / kTile;
   const int64_t nblocks =
       ntile * ntile * ((p.H + p.heads_per_cta - 1) / p.heads_per_cta) * p.batch;
-  attn_mask_kernel<<<(unsigned)nblocks, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  // launched as a programmatic dependent of the launch before it, so that
+  // its zero tiles are written while that launch still runs
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)nblocks);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_mask_kernel, p);
 }
 
 }  // namespace

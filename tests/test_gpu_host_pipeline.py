@@ -73,6 +73,16 @@ def test_host_options_and_oracle(cuda_ok, io, flags, gate, states):
     assert_close_normwise(h, ref[1], rel, "h_last")
 
 
+@pytest.mark.parametrize("b,L,C,N,G", [(4, 100, 64, 16, 2), (3, 50, 36, 16, 1)])
+def test_host_groups_and_generic_kernel(cuda_ok, b, L, C, N, G):
+    # two groups (B, C rows [b, L, G, N] cut by batch row); 36 bf16 channels
+    # are not whole 16-byte rows, so the chunks run the generic kernel
+    d = I.m1_inputs(b, L, C, N, groups=G, io="bf16", seed=C + G)
+    y, h, _ = _call(d, None, pinned=True)
+    yd, hd, _ = _call(d, None)
+    assert torch.equal(y, yd) and torch.equal(h, hd)
+
+
 def test_host_empty_sequence_passes_the_state(cuda_ok):
     d = I.m1_inputs(3, 0, 64, 16, io="bf16", seed=9)
     h0 = torch.randn(3, 64, 16)
