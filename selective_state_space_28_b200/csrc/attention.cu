@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(128)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the mask pass may start now: its zero tiles need nothing from this
   // launch, and its other tiles wait for it to finish (griddepcontrol.wait)
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_launch_dependents();
   const int64_t ncb = p.ntri * p.G * p.batch;
   if ((int64_t)blockIdx.x >= ncb) {
     prep_unit_small<__nv_bfloat16>(p, (int64_t)blockIdx.x - ncb);
@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(256) attn_mask_kernel(AttnParams p) {
     return;
   }
   // C . B^T and the running sums come from the launch before this one
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  pdl_wait();
   // every head's factors first (threads 0..127: one key each; 128..255: one
   // query each), read straight from the running sums -- all of a thread's
   // loads issued before any is used; one barrier
@@ -537,19 +537,9 @@ cudaError_t launch_t(const AttnParams &p, cudaStream_t s) {
   const int64_t ntile = (p.L + kTile - 1) / kTile;
   const int64_t nblocks =
       ntile * ntile * ((p.H + p.heads_per_cta - 1) / p.heads_per_cta) * p.batch;
-  // launched as a programmatic dependent of the launch before it, so that
-  // its zero tiles are written while that launch still runs
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)nblocks);
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_mask_kernel, p);
+  // a programmatic dependent of the launch before it, so that its zero
+  // tiles are written while that launch still runs
+  return launch_dependent(attn_mask_kernel, dim3((unsigned)nblocks), dim3(256), 0, s, p);
 }
 
 }  // namespace

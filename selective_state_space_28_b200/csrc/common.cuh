@@ -10,6 +10,36 @@ namespace ssm {
 // log2(e): exp(v) = 2^(v * log2(e)).
 constexpr float kLog2e = 1.4426950408889634f;
 
+// ------------------------------------------- programmatic dependent launch
+// A launch made with launch_dependent() may start before the launch ahead of
+// it in the stream has finished: as soon as every CTA of that launch has
+// executed pdl_launch_dependents() (or exited).  Its CTAs that need the
+// earlier launch's results execute pdl_wait() first, which returns once that
+// launch has completed and its memory writes are visible; CTAs that need
+// nothing from it run on.  In a launch made the ordinary way pdl_wait()
+// returns at once.
+
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 // ---------------------------------------------------------------- I/O types
 
 template <typename T> struct IO;

@@ -213,6 +213,10 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
   extern __shared__ __align__(128) uint8_t smem_raw[];
   S &s = *reinterpret_cast<S *>(smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u));
 
+  // The rescan of a cut sequence is a programmatic dependent of the carry,
+  // whose entering states every segment reads: its CTAs are placed while
+  // the carry runs and wait here for it.
+  if (MODE == kModeFull && p.nseg > 1) pdl_wait();
   const int64_t L = p.L, C = p.C, Gr = p.G;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ch = lane / G, q = lane % G;
@@ -535,6 +539,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
 // entering state, so that the rescan never reads h0 (which h_last may alias).
 template <int SP>
 __global__ void m1_seg_carry_kernel(const M1Params p) {
+  pdl_launch_dependents();  // the rescan's CTAs may be placed (they wait for this launch)
   const int64_t items = p.batch * p.C * p.N;
   const int64_t idx = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / SP;
   const int k = threadIdx.x % SP;
@@ -596,7 +601,8 @@ bool make_maps(const M1Params &p, Maps &m) {
 }
 
 template <int N, int SPL, typename T, bool HZ, int MODE, bool ST, bool WR>
-cudaError_t launch_spl(const Maps &m, const M1Params &p, int nseg, cudaStream_t s) {
+cudaError_t launch_spl(const Maps &m, const M1Params &p, int nseg, cudaStream_t s,
+                       bool dependent) {
   constexpr int NS = 3;
   auto k = (p.flags & 2u) ? m1_scan_tma_kernel<N, SPL, T, NS, HZ, MODE, ST, WR, kPolyStates, true>
                           : m1_scan_tma_kernel<N, SPL, T, NS, HZ, MODE, ST, WR, kPolyStates, false>;
@@ -604,6 +610,8 @@ cudaError_t launch_spl(const Maps &m, const M1Params &p, int nseg, cudaStream_t 
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((p.C + kCT - 1) / kCT), (unsigned)p.batch, (unsigned)nseg);
+  if (dependent)
+    return launch_dependent(k, grid, dim3(kCT * (N / SPL)), smem, s, m.x, m.dt, m.z, m.B, m.C, p);
   k<<<grid, kCT * (N / SPL), smem, s>>>(m.x, m.dt, m.z, m.B, m.C, p);
   return cudaGetLastError();
 }
@@ -613,8 +621,9 @@ cudaError_t launch_spl(const Maps &m, const M1Params &p, int nseg, cudaStream_t 
 // slower: the transposing reduction spans eight lanes and every B/C load
 // serves half as many states.)
 template <int N, typename T, bool HZ, int MODE, bool ST, bool WR>
-cudaError_t launch_one(const Maps &m, const M1Params &p, int nseg, cudaStream_t s) {
-  return launch_spl<N, 4, T, HZ, MODE, ST, WR>(m, p, nseg, s);
+cudaError_t launch_one(const Maps &m, const M1Params &p, int nseg, cudaStream_t s,
+                       bool dependent = false) {
+  return launch_spl<N, 4, T, HZ, MODE, ST, WR>(m, p, nseg, s, dependent);
 }
 
 template <int N, typename T, bool HZ>
@@ -638,7 +647,7 @@ cudaError_t launch_n(const M1Params &p, cudaStream_t s) {
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_one<N, T, HZ, kModeFull, false, false>(m, p, p.nseg, s);
+  return launch_one<N, T, HZ, kModeFull, false, false>(m, p, p.nseg, s, true);
 }
 
 template <typename T>

@@ -277,6 +277,10 @@ __global__ void __launch_bounds__(threads_of<CONV>(), 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t L = p.L, H = p.H;
+  // The launch of whole units and carried segments is a programmatic
+  // dependent of the carry: the whole units (first in block order) need
+  // nothing from it and start at once; a carried segment waits for it.
+  if (p.seg_lo > 0 && (int64_t)blockIdx.x >= p.nfull) pdl_wait();
   // This CTA's unit, its tiles [cb, cb + nch), where its start state comes
   // from and where its end state goes.  With seg_lo == 0 (the first pass over
   // the tail) a segment other than the first starts from zeros, writes no y
@@ -968,6 +972,7 @@ constexpr int kCarrySlice = 1024;
 __global__ void __launch_bounds__(kCarrySlice / 4)
     ssd_seg_carry_kernel(const float *hend, const float *decay, float *hin, int nseg) {
   constexpr int kNP = kN * kP;
+  pdl_launch_dependents();  // the whole units of the next launch may start
   const int64_t tu = blockIdx.x;
   const int e = blockIdx.y * kCarrySlice + threadIdx.x * 4;
   const float *he = hend + tu * nseg * kNP + e;
@@ -1211,9 +1216,9 @@ cudaError_t launch_ssd_tc(const M2Params &p, int *status, const SsdSplit &split,
   if (e != cudaSuccess) return e;
   q.nfull = units - split.ntail;
   q.seg_lo = 1;
-  kern<<<(unsigned)(q.nfull + split.ntail * (split.nseg - 1)), nthreads, smem, stream>>>(
-      mX, mB, mC, q);
-  return cudaGetLastError();
+  // (a programmatic dependent of the carry: the whole units run while it does)
+  return launch_dependent(kern, dim3((unsigned)(q.nfull + split.ntail * (split.nseg - 1))),
+                          dim3(nthreads), smem, stream, mX, mB, mC, q);
 }
 
 }  // namespace ssm
