@@ -54,7 +54,7 @@ typedef enum ssm_status {
   SSM_ERR_SHAPE = 2,       /* a size is <= 0, or groups does not divide       */
   SSM_ERR_DTYPE = 3,       /* io is not SSM_F32 / SSM_BF16                    */
   SSM_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned                */
-  SSM_ERR_UNSUPPORTED = 5, /* a valid combination this build has no kernel for */
+  SSM_ERR_UNSUPPORTED = 5, /* a valid combination the library has no kernel for */
   SSM_ERR_WORKSPACE = 6,   /* workspace missing or smaller than required      */
   SSM_ERR_CUDA = 7,        /* a CUDA launch or runtime call failed            */
   SSM_ERR_TIMEOUT = 8      /* a bounded device wait ran out (see

@@ -279,7 +279,7 @@ const char *ssm_status_string(ssm_status_t s) {
     case SSM_ERR_SHAPE: return "invalid size or shape";
     case SSM_ERR_DTYPE: return "unsupported io dtype";
     case SSM_ERR_ALIGN: return "pointer not 16-byte aligned";
-    case SSM_ERR_UNSUPPORTED: return "combination not supported by this build";
+    case SSM_ERR_UNSUPPORTED: return "combination the library has no kernel for";
     case SSM_ERR_WORKSPACE: return "workspace missing or too small";
     case SSM_ERR_CUDA: return "CUDA error";
     case SSM_ERR_TIMEOUT: return "device wait timed out";
