@@ -190,11 +190,10 @@ __device__ __forceinline__ void store_pairs(float *dst, const f2 (&v)[NP]) {
 }
 
 // MODE: full scan with readout, or state-only (segments' end states).
-// STATES: also store every token's state.  WR: replace the state at token
-// p.t_write (the state write).
+// STATES: also store every token's state.  A state written at a token
+// (p.state_write) runs the full scan in three parts (see below).
 // SPL: states per lane (4, or 2 for twice the warps on small problems).
-template <int N, int SPL, typename T, int NS, bool HAS_Z, int MODE, bool STATES, bool WR, int PX,
-          bool RBC>
+template <int N, int SPL, typename T, int NS, bool HAS_Z, int MODE, bool STATES, int PX, bool RBC>
 __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
     m1_scan_tma_kernel(const __grid_constant__ CUtensorMap mx,
                        const __grid_constant__ CUtensorMap mdt,
@@ -227,11 +226,68 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
   const int b = blockIdx.y;
   const int seg = blockIdx.z;
   const int g = (int)(c0 / (C / Gr));
-  const int64_t tb = (int64_t)seg * p.seg_len;
-  const int64_t te = tb + p.seg_len < L ? tb + p.seg_len : L;
+  constexpr bool rms_bc = RBC;  // the host picks the instance from SSM_RMSNORM_BC
+  // A state written at token t (p.state_write): tokens before t do not see
+  // it and tokens after t see only it, so the grid's third dimension takes
+  // three independent parts -- tokens [0, t) from h0, tokens (t, L) from the
+  // written state (which leave h_last), and token t's readout.
+  const bool wsplit = kFull && p.state_write != nullptr;
+  int64_t tb, te;
+  if (wsplit) {
+    tb = seg == 0 ? 0 : p.t_write + 1;
+    te = seg == 0 ? p.t_write : L;
+  } else {
+    tb = (int64_t)seg * p.seg_len;
+    te = tb + p.seg_len < L ? tb + p.seg_len : L;
+  }
+  if (wsplit && seg == 2) {
+    // y_t = C_t . (written state), with the chain's arithmetic: the same
+    // per-lane partials and reduction (its pairing does not depend on the
+    // token's place in a group), C_t's factor formed as the prologue forms
+    // it, the skip term and the gate -- so y_t is the one a scan whose
+    // state at t is the written one gives.  Every lane takes part in the
+    // shuffles; lanes past the last channel store nothing.
+    const int64_t t = p.t_write;
+    const T *Cg = static_cast<const T *>(p.Cm) + ((b * L + t) * Gr + g) * N;
+    f2 hw[NP], cv[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) hw[j] = mk2(0.f, 0.f);
+    if (cvalid) load_pairs<NP>(p.state_write + (b * C + c) * N + SPL * q, hw);
+    load_pairs_io<NP>(Cg + SPL * q, cv);
+    f2 acc = mul2(cv[0], hw[0]);
+#pragma unroll
+    for (int j = 1; j < NP; ++j) acc = fma2(cv[j], hw[j], acc);
+    float pg[G];
+#pragma unroll
+    for (int u = 0; u < G; ++u) pg[u] = acc.x + acc.y;
+    const float yq = transpose_reduce<G>(pg, q);
+    float rc = 1.f;
+    if constexpr (rms_bc) {
+      constexpr int PN = N / 4;
+      float vc[PN];
+      widen<PN>(Cg + (lane & 3) * PN, vc);
+      float sc = 0.f;
+#pragma unroll
+      for (int i = 0; i < PN; ++i) sc = fmaf(vc[i], vc[i], sc);
+      sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+      sc += __shfl_xor_sync(0xffffffffu, sc, 2);
+      rc = rsqrtf(sc / N + p.eps);
+    }
+    if (cvalid && q == 0) {
+      const int64_t i = (b * L + t) * C + c;
+      const float dx = (p.D ? p.D[c] : 0.f) * ld(static_cast<const T *>(p.x) + i);
+      float gate = 1.f;
+      if (HAS_Z) {
+        const float zv = ld(static_cast<const T *>(p.z) + i);
+        gate = kBF16 ? silu_tanh(zv) : silu(zv);
+      }
+      const float v = rms_bc ? fmaf(yq, rc, dx) : yq + dx;
+      st(static_cast<T *>(p.y) + i, v * gate);
+    }
+    return;
+  }
   const int nst = (int)((te - tb + kTL - 1) / kTL);
   const bool softplus_on = p.flags & 1u;
-  constexpr bool rms_bc = RBC;  // the host picks the instance from SSM_RMSNORM_BC
   constexpr uint32_t kStageBytes = ((HAS_Z ? 3 : 2) * kTL * kCT + 2 * kTL * N) * sizeof(T);
 
   if (threadIdx.x == 0) {
@@ -274,6 +330,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
   // zeros for a segment scanned from its own start.
   const float *h_in = nullptr;
   if (MODE == kModeStateOnly) h_in = seg == 0 ? p.h0 : nullptr;
+  else if (wsplit) h_in = seg == 0 ? p.h0 : p.state_write;
   else h_in = p.nseg > 1 ? p.seg_ent + (int64_t)seg * p.batch * C * N : p.h0;
   f2 h[NP], A2[NP];
 #pragma unroll
@@ -390,11 +447,9 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
     // write terms of step k+1 (independent of the state) are formed while
     // step k runs its chain, and the readout of step k-1 is reduced and
     // stored meanwhile, so that a warp always has independent work at hand.
-    const int tw = (WR && p.t_write >= t0 && p.t_write < t0 + tn) ? (int)(p.t_write - t0) : -1;
     // (8 tokens per step: measured 8 % faster than 4 at the Falcon width,
-    // equal on the 130m workload; 16 is slower.  The write form, which
-    // carries two forms of the chain, keeps 4 so that it does not spill.)
-    constexpr int SL = G > 8 ? G : (WR ? 4 : 8);  // tokens per step
+    // equal on the 130m workload; 16 is slower.)
+    constexpr int SL = G > 8 ? G : 8;  // tokens per step
     struct Pre {
       f2 a[SL][NP], w[SL][NP];  // decays and write terms d * x * B
     };
@@ -441,39 +496,22 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
     for (int tg = 0; tg < kTL; tg += SL) {
       if (tg + SL < kTL) pre(tg + SL, nxt);
       float part[SL];
-      // the chain of one step; only the step holding a written token takes
-      // the form that checks for it (one compare per token costs a fifth of
-      // the loop)
-      auto chain = [&](auto wr) {
+      // the chain of one step
 #pragma unroll
-        for (int u = 0; u < SL; ++u) {
-          const int t = tg + u;
+      for (int u = 0; u < SL; ++u) {
+        const int t = tg + u;
 #pragma unroll
-          for (int j = 0; j < NP; ++j) h[j] = fma2(cur.a[u][j], h[j], cur.w[u][j]);
-          if constexpr (decltype(wr)::value) {
-            if (t == tw && cvalid) {
-              // a state written at this token replaces h_t before y_t reads
-              // it ("Mamba", nnterp guide, "The state")
-              load_pairs<NP>(p.state_write + (b * C + c) * N + SPL * q, h);
-            }
-          }
-          if (kFull) {
-            f2 cv[NP];
-            load_pairs_io<NP>(&s.C[buf][t][SPL * q], cv);
-            f2 acc = mul2(cv[0], h[0]);
+        for (int j = 0; j < NP; ++j) h[j] = fma2(cur.a[u][j], h[j], cur.w[u][j]);
+        if (kFull) {
+          f2 cv[NP];
+          load_pairs_io<NP>(&s.C[buf][t][SPL * q], cv);
+          f2 acc = mul2(cv[0], h[0]);
 #pragma unroll
-            for (int j = 1; j < NP; ++j) acc = fma2(cv[j], h[j], acc);
-            part[u] = acc.x + acc.y;
-          }
-          if (STATES && cvalid && t < tn)
-            store_pairs<NP>(p.states + ((b * L + t0 + t) * C + c) * N + SPL * q, h);
+          for (int j = 1; j < NP; ++j) acc = fma2(cv[j], h[j], acc);
+          part[u] = acc.x + acc.y;
         }
-      };
-      if constexpr (WR) {
-        if (tw >= tg && tw < tg + SL) chain(std::true_type{});
-        else chain(std::false_type{});
-      } else {
-        chain(std::false_type{});
+        if (STATES && cvalid && t < tn)
+          store_pairs<NP>(p.states + ((b * L + t0 + t) * C + c) * N + SPL * q, h);
       }
       if (kFull && tg >= SL) finish(tg - SL, partp);
 #pragma unroll
@@ -524,7 +562,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
     const int64_t i = ((int64_t)seg * p.batch + b) * C + c;
     store_pairs<NP>(p.seg_end + i * N + SPL * q, h);
     if (q == 0) p.seg_dsum[i] = dsum;
-  } else if (p.h_last && seg == p.nseg - 1) {
+  } else if (p.h_last && (wsplit ? seg == 1 : seg == p.nseg - 1)) {
     store_pairs<NP>(p.h_last + (b * C + c) * N + SPL * q, h);
   }
 }
@@ -600,12 +638,12 @@ bool make_maps(const M1Params &p, Maps &m) {
                       CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-template <int N, int SPL, typename T, bool HZ, int MODE, bool ST, bool WR>
+template <int N, int SPL, typename T, bool HZ, int MODE, bool ST>
 cudaError_t launch_spl(const Maps &m, const M1Params &p, int nseg, cudaStream_t s,
                        bool dependent) {
   constexpr int NS = 3;
-  auto k = (p.flags & 2u) ? m1_scan_tma_kernel<N, SPL, T, NS, HZ, MODE, ST, WR, kPolyStates, true>
-                          : m1_scan_tma_kernel<N, SPL, T, NS, HZ, MODE, ST, WR, kPolyStates, false>;
+  auto k = (p.flags & 2u) ? m1_scan_tma_kernel<N, SPL, T, NS, HZ, MODE, ST, kPolyStates, true>
+                          : m1_scan_tma_kernel<N, SPL, T, NS, HZ, MODE, ST, kPolyStates, false>;
   const size_t smem = sizeof(ScanSmem<N, T, NS>) + 128;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -620,20 +658,21 @@ cudaError_t launch_spl(const Maps &m, const M1Params &p, int nseg, cudaStream_t 
 // the 130m workload, costs 66 % more instructions per state and runs 24 %
 // slower: the transposing reduction spans eight lanes and every B/C load
 // serves half as many states.)
-template <int N, typename T, bool HZ, int MODE, bool ST, bool WR>
+template <int N, typename T, bool HZ, int MODE, bool ST>
 cudaError_t launch_one(const Maps &m, const M1Params &p, int nseg, cudaStream_t s,
                        bool dependent = false) {
-  return launch_spl<N, 4, T, HZ, MODE, ST, WR>(m, p, nseg, s, dependent);
+  return launch_spl<N, 4, T, HZ, MODE, ST>(m, p, nseg, s, dependent);
 }
 
 template <int N, typename T, bool HZ>
 cudaError_t launch_n(const M1Params &p, cudaStream_t s) {
   Maps m;
   if (!make_maps<N, T>(p, m)) return cudaErrorInvalidValue;
-  if (p.states) return launch_one<N, T, HZ, kModeFull, true, false>(m, p, 1, s);
-  if (p.state_write) return launch_one<N, T, HZ, kModeFull, false, true>(m, p, 1, s);
-  if (p.nseg <= 1) return launch_one<N, T, HZ, kModeFull, false, false>(m, p, 1, s);
-  cudaError_t e = launch_one<N, T, HZ, kModeStateOnly, false, false>(m, p, p.nseg - 1, s);
+  if (p.states) return launch_one<N, T, HZ, kModeFull, true>(m, p, 1, s);
+  // a state write: three independent parts in one launch (see the kernel)
+  if (p.state_write) return launch_one<N, T, HZ, kModeFull, false>(m, p, 3, s);
+  if (p.nseg <= 1) return launch_one<N, T, HZ, kModeFull, false>(m, p, 1, s);
+  cudaError_t e = launch_one<N, T, HZ, kModeStateOnly, false>(m, p, p.nseg - 1, s);
   if (e != cudaSuccess) return e;
   const int64_t items = p.batch * p.C * p.N;
   const int sp = p.nseg - 1 <= 2 ? 2 : p.nseg - 1 <= 4 ? 4 : p.nseg - 1 <= 8 ? 8 : p.nseg - 1 <= 16 ? 16 : 32;
@@ -647,7 +686,7 @@ cudaError_t launch_n(const M1Params &p, cudaStream_t s) {
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_one<N, T, HZ, kModeFull, false, false>(m, p, p.nseg, s, true);
+  return launch_one<N, T, HZ, kModeFull, false>(m, p, p.nseg, s, true);
 }
 
 template <typename T>
