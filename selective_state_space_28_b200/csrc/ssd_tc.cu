@@ -1036,12 +1036,18 @@ __global__ void __launch_bounds__(256)
         for (int e = 0; e < 8; ++e) win[q][e] = 0.f;
       }
     }
+    // every row of the run loaded before any is used (each thread's loads
+    // in flight together, not one latency per token)
+    uint4 raw[kBcRun];
+#pragma unroll
+    for (int r = 0; r < kBcRun; ++r)
+      raw[r] = t0 + r < L ? ld_nc_u4(xbc + (bb * L + t0 + r) * ctot + ch) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
     for (int r = 0; r < kBcRun; ++r) {
       const int64_t t = t0 + r;
       if (t >= L) break;
       float xv[8];
-      unpack8(ld_nc_u4(xbc + (bb * L + t) * ctot + ch), xv);
+      unpack8(raw[r], xv);
       float o[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {  // the newest input first, as ssm_conv1d_fwd
