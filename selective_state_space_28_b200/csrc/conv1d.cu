@@ -123,26 +123,36 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
   for (int s = 0; s < NS - 1; ++s) issue(s);
 
-  float w[V][W], bias[V];
+  // The arithmetic runs on channel pairs (packed f32x2: each lane of a pair
+  // is exactly the scalar fmaf / multiply), half the instructions of
+  // channel by channel; the bits are those of the scalar form and of the
+  // fused scan's convolution.
+  constexpr int VP = V / 2;
+  f2 w[VP][W], bias[VP];
 #pragma unroll
-  for (int v = 0; v < V; ++v) {
+  for (int v = 0; v < VP; ++v) {
 #pragma unroll
-    for (int k = 0; k < W; ++k) w[v][k] = p.w[(c0 + v) * W + k];
-    bias[v] = p.bias ? p.bias[c0 + v] : 0.f;
+    for (int k = 0; k < W; ++k)
+      w[v][k] = mk2(p.w[(c0 + 2 * v) * W + k], p.w[(c0 + 2 * v + 1) * W + k]);
+    bias[v] = p.bias ? mk2(p.bias[c0 + 2 * v], p.bias[c0 + 2 * v + 1]) : mk2(0.f, 0.f);
   }
   // hist[j][v]: input j + 1 tokens before the current one (j < W - 1)
-  float hist[W > 1 ? W - 1 : 1][V];
+  f2 hist[W > 1 ? W - 1 : 1][VP];
 #pragma unroll
   for (int j = 0; j < W - 1; ++j) {
     const int64_t tau = t0 - 1 - j;
+    float hv[V];
     if (tau >= 0) {
-      Vec<T>::widen(Vec<T>::load(x + (b * L + tau) * Cc + c0), hist[j]);
+      Vec<T>::widen(Vec<T>::load(x + (b * L + tau) * Cc + c0), hv);
     } else {
 #pragma unroll
       for (int v = 0; v < V; ++v)
-        hist[j][v] = p.state_in ? p.state_in[((b * Cc) + c0 + v) * (W - 1) + (W - 1) + tau] : 0.f;
+        hv[v] = p.state_in ? p.state_in[((b * Cc) + c0 + v) * (W - 1) + (W - 1) + tau] : 0.f;
     }
+#pragma unroll
+    for (int v = 0; v < VP; ++v) hist[j][v] = mk2(hv[2 * v], hv[2 * v + 1]);
   }
+  const f2 half2 = mk2(0.5f, 0.5f);
   T *pu = u + (b * L + t0) * Cc + c0;
   for (int i = 0; i < nb; ++i) {
     issue((i + NS - 1) % NS);  // the slot batch i - 1 used (an empty group past the end)
@@ -152,24 +162,39 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int a = 0; a < NT; ++a) {
       if (a >= na) break;
-      float xv[V], o[V];
-      Vec<T>::widen(stage[slot][a][tid], xv);
+      float xs[V], o[V];
+      Vec<T>::widen(stage[slot][a][tid], xs);
+      f2 xv[VP];
 #pragma unroll
-      for (int v = 0; v < V; ++v) {
-        float acc = fmaf(w[v][W - 1], xv[v], bias[v]);
+      for (int v = 0; v < VP; ++v) xv[v] = mk2(xs[2 * v], xs[2 * v + 1]);
 #pragma unroll
-        for (int j = 0; j < W - 1; ++j) acc = fmaf(w[v][W - 2 - j], hist[j][v], acc);
-        o[v] = act<T>(acc, p.silu);
+      for (int v = 0; v < VP; ++v) {
+        f2 acc = fma2(w[v][W - 1], xv[v], bias[v]);
+#pragma unroll
+        for (int j = 0; j < W - 1; ++j) acc = fma2(w[v][W - 2 - j], hist[j][v], acc);
+        if (sizeof(T) == 2 && p.silu) {
+          // silu(z) = z (1 + tanh(z / 2)) / 2, as silu_tanh
+          const f2 hz = mul2(half2, acc);
+          float ta, tb;
+          asm("tanh.approx.f32 %0, %1;" : "=f"(ta) : "f"(hz.x));
+          asm("tanh.approx.f32 %0, %1;" : "=f"(tb) : "f"(hz.y));
+          const f2 u = mul2(acc, fma2(half2, mk2(ta, tb), half2));
+          o[2 * v] = u.x;
+          o[2 * v + 1] = u.y;
+        } else {
+          o[2 * v] = act<T>(acc.x, p.silu);
+          o[2 * v + 1] = act<T>(acc.y, p.silu);
+        }
       }
       Vec<T>::store(pu, o);
       pu += Cc;
 #pragma unroll
       for (int j = W - 2; j > 0; --j)
 #pragma unroll
-        for (int v = 0; v < V; ++v) hist[j][v] = hist[j - 1][v];
+        for (int v = 0; v < VP; ++v) hist[j][v] = hist[j - 1][v];
       if (W > 1) {
 #pragma unroll
-        for (int v = 0; v < V; ++v) hist[0][v] = xv[v];
+        for (int v = 0; v < VP; ++v) hist[0][v] = xv[v];
       }
     }
   }
@@ -180,8 +205,10 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int j = 0; j < W - 1; ++j)
 #pragma unroll
-      for (int v = 0; v < V; ++v)
-        p.state_out[((b * Cc) + c0 + v) * (W - 1) + (W - 2 - j)] = hist[j][v];
+      for (int v = 0; v < VP; ++v) {
+        p.state_out[((b * Cc) + c0 + 2 * v) * (W - 1) + (W - 2 - j)] = hist[j][v].x;
+        p.state_out[((b * Cc) + c0 + 2 * v + 1) * (W - 1) + (W - 2 - j)] = hist[j][v].y;
+      }
   }
 }
 
