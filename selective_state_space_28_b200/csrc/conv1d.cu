@@ -11,14 +11,16 @@
 // last W - 1 inputs.  With seqlen 1 and the state updated in place this is the
 // decode form of the same convolution.
 //
-// HBM-streaming layout: a thread owns V = 4 consecutive channels (an 8-byte
-// (bf16) or 16-byte (f32) vector of the tokens-first rows) over a run of kRun
+// HBM-streaming layout: a thread owns V consecutive channels -- 8 bf16 (a
+// 16-byte vector of the tokens-first rows) when the channel count is a
+// multiple of 8, else 4 (8 bytes bf16, 16 bytes float32) -- over a run of
 // tokens, keeps the W - 1 previous inputs in registers, and reads each input
 // once (plus a W - 1 token halo at the start of its run, mostly from L2) and
 // writes each output once; a warp covers 32 consecutive vectors of a row, so
 // every access is coalesced.  The inputs reach the thread through its own
 // shared-memory slots, copied asynchronously several batches ahead, so that
-// enough bytes are in flight per SM without holding them in registers.
+// enough bytes are in flight per SM without holding them in registers.  The
+// arithmetic runs on channel pairs in packed f32x2.
 #include "common.cuh"
 #include "internal.h"
 
@@ -29,8 +31,25 @@ constexpr int kRun = 128;  // tokens per thread (when the state is not updated i
 
 // Streaming (evict-first) vector loads and stores through the compiler's
 // intrinsics (the halo loads and the output stores).
-template <typename T> struct Vec;
-template <> struct Vec<__nv_bfloat16> {
+// V channels a thread: 8 bf16 (16 bytes) where the channel count allows,
+// else 4 (8 bytes); float32 takes 4 (16 bytes).
+template <typename T, int V> struct Vec;
+template <> struct Vec<__nv_bfloat16, 8> {
+  static constexpr int V = 8;
+  using Raw = uint4;
+  static __device__ __forceinline__ Raw load(const __nv_bfloat16 *p) {
+    return __ldcs(reinterpret_cast<const uint4 *>(p));
+  }
+  static __device__ __forceinline__ void widen(const Raw &w, float (&f)[8]) {
+    f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+    f[4] = bf16lo(w.z); f[5] = bf16hi(w.z); f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&f)[8]) {
+    __stcs(reinterpret_cast<uint4 *>(p), make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                     pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
+  }
+};
+template <> struct Vec<__nv_bfloat16, 4> {
   static constexpr int V = 4;
   using Raw = uint2;
   static __device__ __forceinline__ Raw load(const __nv_bfloat16 *p) {
@@ -43,7 +62,7 @@ template <> struct Vec<__nv_bfloat16> {
     __stcs(reinterpret_cast<uint2 *>(p), make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3])));
   }
 };
-template <> struct Vec<float> {
+template <> struct Vec<float, 4> {
   static constexpr int V = 4;
   using Raw = float4;
   static __device__ __forceinline__ Raw load(const float *p) {
@@ -88,11 +107,12 @@ template <int N> __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <typename T, int W>
+template <typename T, int W, int VW>
 __global__ void __launch_bounds__(128)
     conv1d_vec_kernel(ConvParams p) {
-  constexpr int V = Vec<T>::V;
-  using Raw = typename Vec<T>::Raw;
+  using VT = Vec<T, VW>;
+  constexpr int V = VT::V;
+  using Raw = typename VT::Raw;
   constexpr int NS = sizeof(Raw) == 16 ? 3 : kStages;
   constexpr int NT = sizeof(Raw) == 16 ? 8 : kTok;
   __shared__ Raw stage[NS][NT][128];
@@ -143,7 +163,7 @@ __global__ void __launch_bounds__(128)
     const int64_t tau = t0 - 1 - j;
     float hv[V];
     if (tau >= 0) {
-      Vec<T>::widen(Vec<T>::load(x + (b * L + tau) * Cc + c0), hv);
+      VT::widen(VT::load(x + (b * L + tau) * Cc + c0), hv);
     } else {
 #pragma unroll
       for (int v = 0; v < V; ++v)
@@ -163,7 +183,7 @@ __global__ void __launch_bounds__(128)
     for (int a = 0; a < NT; ++a) {
       if (a >= na) break;
       float xs[V], o[V];
-      Vec<T>::widen(stage[slot][a][tid], xs);
+      VT::widen(stage[slot][a][tid], xs);
       f2 xv[VP];
 #pragma unroll
       for (int v = 0; v < VP; ++v) xv[v] = mk2(xs[2 * v], xs[2 * v + 1]);
@@ -186,7 +206,7 @@ __global__ void __launch_bounds__(128)
           o[2 * v + 1] = act<T>(acc.y, p.silu);
         }
       }
-      Vec<T>::store(pu, o);
+      VT::store(pu, o);
       pu += Cc;
 #pragma unroll
       for (int j = W - 2; j > 0; --j)
@@ -252,18 +272,22 @@ __global__ void __launch_bounds__(128)
   }
 }
 
-template <typename T, int W>
-bool vec_form(const ConvParams &p) {
-  return (p.Cc % Vec<T>::V) == 0;  // rows then hold whole vectors (bases are 16-byte aligned)
+// The widest vector whose rows the channel count fills (row bases are then
+// 16-byte aligned): 8 (bf16) or 4 channels a thread, or 0 for the
+// per-channel form.
+template <typename T>
+int vec_width(const ConvParams &p) {
+  if (sizeof(T) == 2 && p.Cc % 8 == 0) return 8;
+  return p.Cc % 4 == 0 ? 4 : 0;
 }
 
-// CTAs of the vector form resident per SM (its registers and slots decide),
+// CTAs of a vector form resident per SM (its registers and slots decide),
 // read once per instance from the runtime's occupancy calculator.
-template <typename T, int W>
+template <typename T, int W, int VW>
 int vec_ctas_per_sm() {
   static const int n = [] {
     int k = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&k, conv1d_vec_kernel<T, W>, 128, 0) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&k, conv1d_vec_kernel<T, W, VW>, 128, 0) !=
             cudaSuccess ||
         k <= 0) {
       cudaGetLastError();
@@ -274,36 +298,44 @@ int vec_ctas_per_sm() {
   return n;
 }
 
-template <typename T, int W>
-cudaError_t launch_w(const ConvParams &p, cudaStream_t s) {
-  constexpr int V = Vec<T>::V;
-  const bool vec = vec_form<T, W>(p);
+template <typename T, int W, int VW>
+cudaError_t launch_vec(const ConvParams &p, cudaStream_t s) {
   const int64_t runs = (p.L + p.run - 1) / p.run;
-  const int64_t units = vec ? p.batch * (p.Cc / V) : p.batch * p.Cc;
+  const int64_t units = p.batch * (p.Cc / VW);
   dim3 grid((unsigned)((units + 127) / 128), (unsigned)runs);
-  if (vec) {
-    // the slots (24-32 KB per CTA) need the shared-memory carve-out for
-    // several CTAs per SM (a preference of the current device: set per call)
-    if (cudaFuncSetAttribute(conv1d_vec_kernel<T, W>,
-                             cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
-      cudaGetLastError();  // a preference only: never fail the call on it
-    conv1d_vec_kernel<T, W><<<grid, 128, 0, s>>>(p);
-  }
-  else
-    conv1d_scalar_kernel<T, W><<<grid, 128, 0, s>>>(p);
+  // the slots (32-48 KB per CTA) need the shared-memory carve-out for
+  // several CTAs per SM (a preference of the current device: set per call)
+  if (cudaFuncSetAttribute(conv1d_vec_kernel<T, W, VW>,
+                           cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+    cudaGetLastError();  // a preference only: never fail the call on it
+  conv1d_vec_kernel<T, W, VW><<<grid, 128, 0, s>>>(p);
   return cudaGetLastError();
 }
 
-// Tokens per thread of the vector form: whole batches of kTok, at least
-// kRunMin, chosen so that the grid fills whole waves of resident CTAs.  With
-// kRun tokens the bf16 2.7B mixer (b4, 5376 channels: 42 x 32 CTAs at six
-// per SM) would run 1.5 waves, the second half empty; 200-token runs make it
-// one wave of 882 CTAs.
-constexpr int64_t kRunMin = 64;
 template <typename T, int W>
+cudaError_t launch_w(const ConvParams &p, cudaStream_t s) {
+  switch (vec_width<T>(p)) {
+    case 8:
+      if constexpr (sizeof(T) == 2) return launch_vec<T, W, 8>(p, s);
+      break;
+    case 4: return launch_vec<T, W, 4>(p, s);
+  }
+  const int64_t runs = (p.L + p.run - 1) / p.run;
+  dim3 grid((unsigned)((p.batch * p.Cc + 127) / 128), (unsigned)runs);
+  conv1d_scalar_kernel<T, W><<<grid, 128, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+// Tokens per thread of a vector form: whole batches of kTok, at least
+// kRunMin, chosen so that the grid fills whole waves of resident CTAs.  With
+// kRun tokens the bf16 2.7B mixer (b4, 5376 channels, 8 a thread: 21 x 32
+// CTAs) would leave the last wave part empty; runs fitted to the resident
+// CTAs fill it.
+constexpr int64_t kRunMin = 64;
+template <typename T, int W, int VW>
 int64_t fitted_run(const ConvParams &p) {
-  const int64_t bx = (p.batch * (p.Cc / Vec<T>::V) + 127) / 128;
-  const int64_t per_sm = vec_ctas_per_sm<T, W>();
+  const int64_t bx = (p.batch * (p.Cc / VW) + 127) / 128;
+  const int64_t per_sm = vec_ctas_per_sm<T, W, VW>();
   if (per_sm <= 0 || bx <= 0) return kRun;
   const int64_t cap = (int64_t)device_sm_count() * per_sm;
   const int64_t runs0 = (p.L + kRun - 1) / kRun;
@@ -314,6 +346,17 @@ int64_t fitted_run(const ConvParams &p) {
   int64_t run = (p.L + runs - 1) / runs;
   run = (run + kTok - 1) / kTok * kTok;
   return run < kRunMin ? kRunMin : run;
+}
+
+template <typename T, int W>
+int64_t run_w(const ConvParams &p) {
+  switch (vec_width<T>(p)) {
+    case 8:
+      if constexpr (sizeof(T) == 2) return fitted_run<T, W, 8>(p);
+      break;
+    case 4: return fitted_run<T, W, 4>(p);
+  }
+  return kRun;
 }
 
 template <typename T>
@@ -330,10 +373,10 @@ cudaError_t launch_t(const ConvParams &p, cudaStream_t s) {
 template <typename T>
 int64_t run_t(const ConvParams &p) {
   switch (p.W) {
-    case 1: return vec_form<T, 1>(p) ? fitted_run<T, 1>(p) : kRun;
-    case 2: return vec_form<T, 2>(p) ? fitted_run<T, 2>(p) : kRun;
-    case 3: return vec_form<T, 3>(p) ? fitted_run<T, 3>(p) : kRun;
-    case 4: return vec_form<T, 4>(p) ? fitted_run<T, 4>(p) : kRun;
+    case 1: return run_w<T, 1>(p);
+    case 2: return run_w<T, 2>(p);
+    case 3: return run_w<T, 3>(p);
+    case 4: return run_w<T, 4>(p);
   }
   return kRun;
 }
