@@ -420,14 +420,35 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
       widen<8>(&s.x[buf][t][k0], xv);
       widen<8>(&s.dt[buf][t][k0], dv);
       if (HAS_Z) widen<8>(&s.z[buf][t][k0], zv);
+      // channel pairs in packed f32x2 where the scalar form is one
+      // operation per channel (each lane exactly that operation)
       float2 o[8], og[8];
+      const f2 rs2 = mk2(rs, rs), rb2 = mk2(rb, rb);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float d = fmaf(dv[i], rs, biasr[i]);
-        if (softplus_on) d = softplus_sfu(d);
-        o[i] = tvalid ? make_float2(d, d * xv[i] * rb) : make_float2(0.f, 0.f);
-        const float gate = HAS_Z ? (kBF16 ? silu_tanh(zv[i]) : silu(zv[i])) : 1.f;
-        og[i] = make_float2(skipr[i] * xv[i], gate);
+      for (int k = 0; k < 4; ++k) {
+        const int i = 2 * k;
+        const f2 x2 = mk2(xv[i], xv[i + 1]);
+        f2 d2 = fma2(mk2(dv[i], dv[i + 1]), rs2, mk2(biasr[i], biasr[i + 1]));
+        if (softplus_on) d2 = mk2(softplus_sfu(d2.x), softplus_sfu(d2.y));
+        const f2 dx2 = mul2(mul2(d2, x2), rb2);
+        const f2 sx2 = mul2(mk2(skipr[i], skipr[i + 1]), x2);
+        f2 g2 = mk2(1.f, 1.f);
+        if (HAS_Z) {
+          if (kBF16) {  // silu(z) = z (1 + tanh(z / 2)) / 2, as silu_tanh
+            const f2 z2 = mk2(zv[i], zv[i + 1]);
+            const f2 hz = mul2(mk2(0.5f, 0.5f), z2);
+            float ta, tb;
+            asm("tanh.approx.f32 %0, %1;" : "=f"(ta) : "f"(hz.x));
+            asm("tanh.approx.f32 %0, %1;" : "=f"(tb) : "f"(hz.y));
+            g2 = mul2(z2, fma2(mk2(0.5f, 0.5f), mk2(ta, tb), mk2(0.5f, 0.5f)));
+          } else {
+            g2 = mk2(silu(zv[i]), silu(zv[i + 1]));
+          }
+        }
+        o[i] = tvalid ? make_float2(d2.x, dx2.x) : make_float2(0.f, 0.f);
+        o[i + 1] = tvalid ? make_float2(d2.y, dx2.y) : make_float2(0.f, 0.f);
+        og[i] = make_float2(sx2.x, g2.x);
+        og[i + 1] = make_float2(sx2.y, g2.y);
       }
       float4 *dst = reinterpret_cast<float4 *>(&s.ddx[sg & 1][t][k0]);
       float4 *gst = reinterpret_cast<float4 *>(&s.eg[sg & 1][t][k0]);
