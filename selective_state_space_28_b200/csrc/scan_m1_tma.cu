@@ -739,35 +739,37 @@ bool m1_scan_tma_supported(const M1Params &p) {
   return true;
 }
 
-// How many sequence segments a call is cut into.  Cost model, in units of
-// one warp's whole-sequence time when it has its SM sub-partition to itself:
-// a sub-partition runs up to kFull warps at no loss of per-warp speed (the
-// recurrence is latency-bound below that), so k warps take max(1, k / kFull)
-// units per unit of work.  Cutting into S segments costs a state-only pass
-// over the first S - 1 segments (about 0.85 of a full pass per token, no
-// readout), a full pass over S segments of 1/S of the sequence each, and two
-// more launches.  Calls with per-token states or a state write are not cut.
+// How many sequence segments a call is cut into.  Cost model (measured on
+// B200 for this kernel, 16 states): a warp's time per token with k warps on
+// its SM sub-partition is flat, ~79 ns, up to about two warps (the chain is
+// latency-bound there), then the sub-partition's issue and SFU throughput is
+// shared, ~33.5 k ns.  A pass of W warps over Ls tokens takes
+// Ls * t(ceil(W / sub-partitions)).  Cutting into S segments costs a
+// state-only pass over the first S - 1 segments (about 0.85 of a full pass
+// per token, no readout), a full pass over S segments of 1/S of the sequence
+// each, and ~14 us of fills, carry and launches.  A cut is taken when it is
+// predicted 10 % faster.  Calls with per-token states or a state write are
+// not cut.
 M1Split m1_scan_split(int64_t batch, int64_t C, int64_t L, int64_t N, int sms) {
   M1Split r;
   r.nseg = 1;
   r.seg_len = L;
   if (batch <= 0 || L <= 0 || sms <= 0) return r;
-  const double kFull = 3.0, kStateOnly = 0.85;
+  const double kStateOnly = 0.85, kCutNs = 14000.0;
   const double slots = 4.0 * sms;  // sub-partitions
   const double w0 = (double)batch * ((C + kCT - 1) / kCT) * (kCT * (N / 4) / 32);  // warps
-  const double work_ns = (double)L * 50.0;  // one warp alone, per token (measured order)
-  auto cost = [&](double warps, double frac) {
+  auto pass_ns = [&](double warps, double tokens) {
     const double k = std::ceil(warps / slots);
-    return frac * std::max(1.0, k / kFull);
+    return tokens * std::max(79.0, 33.5 * k);
   };
-  double best = cost(w0, 1.0);
+  double best = pass_ns(w0, (double)L);
   for (int S = 2; S <= 32; S *= 2) {
     const int64_t len = ((L + S - 1) / S + kTL - 1) / kTL * kTL;
     if (len < 4 * kTL) break;
     const int segs = (int)((L + len - 1) / len);
     if (segs < 2) break;
-    const double t = cost(w0 * (segs - 1), kStateOnly / segs) + cost(w0 * segs, 1.0 / segs) +
-                     2 * 4000.0 / work_ns;  // two more launches of a few microseconds
+    const double t = kStateOnly * pass_ns(w0 * (segs - 1), (double)len) +
+                     pass_ns(w0 * segs, (double)len) + kCutNs;
     if (t < 0.9 * best) {
       best = t;
       r.nseg = segs;
