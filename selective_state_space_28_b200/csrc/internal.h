@@ -21,6 +21,7 @@ struct M1Params {
   float *rstd = nullptr;  // [batch * L] RMS factors of dt rows, or nullptr
   int *status = nullptr;  // device word set non-zero if a bounded wait ran out
   int64_t t_write = -1;                 // token whose state is replaced
+  int part_base = 0;                    // a state write's first part in this launch
   const float *state_write = nullptr;   // [batch, C, N] state written at t_write
   // sequence segments of the pipelined kernel (nseg 1: the whole sequence)
   int nseg = 1;

@@ -228,19 +228,22 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
   const int g = (int)(c0 / (C / Gr));
   constexpr bool rms_bc = RBC;  // the host picks the instance from SSM_RMSNORM_BC
   // A state written at token t (p.state_write): tokens before t do not see
-  // it and tokens after t see only it, so the grid's third dimension takes
-  // three independent parts -- tokens [0, t) from h0, tokens (t, L) from the
-  // written state (which leave h_last), and token t's readout.
+  // it and tokens after t see only it, so the call is three independent
+  // parts -- 0: tokens [0, t) from h0; 1: token t's readout; 2: tokens
+  // (t, L) from the written state, which leave h_last -- taken by the grid's
+  // third dimension from p.part_base on (one launch, or two when h_last
+  // overlaps what parts 0 and 1 read).
   const bool wsplit = kFull && p.state_write != nullptr;
+  const int part = p.part_base + seg;
   int64_t tb, te;
   if (wsplit) {
-    tb = seg == 0 ? 0 : p.t_write + 1;
-    te = seg == 0 ? p.t_write : L;
+    tb = part == 0 ? 0 : p.t_write + 1;
+    te = part == 0 ? p.t_write : L;
   } else {
     tb = (int64_t)seg * p.seg_len;
     te = tb + p.seg_len < L ? tb + p.seg_len : L;
   }
-  if (wsplit && seg == 2) {
+  if (wsplit && part == 1) {
     // y_t = C_t . (written state), with the chain's arithmetic: the same
     // per-lane partials and reduction (its pairing does not depend on the
     // token's place in a group), C_t's factor formed as the prologue forms
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
   // zeros for a segment scanned from its own start.
   const float *h_in = nullptr;
   if (MODE == kModeStateOnly) h_in = seg == 0 ? p.h0 : nullptr;
-  else if (wsplit) h_in = seg == 0 ? p.h0 : p.state_write;
+  else if (wsplit) h_in = part == 0 ? p.h0 : p.state_write;
   else h_in = p.nseg > 1 ? p.seg_ent + (int64_t)seg * p.batch * C * N : p.h0;
   f2 h[NP], A2[NP];
 #pragma unroll
@@ -583,7 +586,7 @@ __global__ void __launch_bounds__(kCT *(N / SPL), N >= 32 ? 2 : 3)
     const int64_t i = ((int64_t)seg * p.batch + b) * C + c;
     store_pairs<NP>(p.seg_end + i * N + SPL * q, h);
     if (q == 0) p.seg_dsum[i] = dsum;
-  } else if (p.h_last && (wsplit ? seg == 1 : seg == p.nseg - 1)) {
+  } else if (p.h_last && (wsplit ? part == 2 : seg == p.nseg - 1)) {
     store_pairs<NP>(p.h_last + (b * C + c) * N + SPL * q, h);
   }
 }
@@ -690,8 +693,24 @@ cudaError_t launch_n(const M1Params &p, cudaStream_t s) {
   Maps m;
   if (!make_maps<N, T>(p, m)) return cudaErrorInvalidValue;
   if (p.states) return launch_one<N, T, HZ, kModeFull, true>(m, p, 1, s);
-  // a state write: three independent parts in one launch (see the kernel)
-  if (p.state_write) return launch_one<N, T, HZ, kModeFull, false>(m, p, 3, s);
+  if (p.state_write) {
+    // three independent parts in one launch (see the kernel), unless h_last
+    // overlaps h0 or the written state: part 2 writes h_last, which parts 0
+    // and 1 read, so it then runs as a launch of its own after theirs
+    const size_t n = (size_t)(p.batch * p.C * p.N) * sizeof(float);
+    auto overlap = [n](const void *a, const void *b) {
+      const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+      return a && b && x < y + n && y < x + n;
+    };
+    if (!overlap(p.h_last, p.h0) && !overlap(p.h_last, p.state_write))
+      return launch_one<N, T, HZ, kModeFull, false>(m, p, 3, s);
+    M1Params q = p;
+    q.part_base = 0;
+    cudaError_t e = launch_one<N, T, HZ, kModeFull, false>(m, q, 2, s);
+    if (e != cudaSuccess) return e;
+    q.part_base = 2;
+    return launch_one<N, T, HZ, kModeFull, false>(m, q, 1, s);
+  }
   if (p.nseg <= 1) return launch_one<N, T, HZ, kModeFull, false>(m, p, 1, s);
   cudaError_t e = launch_one<N, T, HZ, kModeStateOnly, false>(m, p, p.nseg - 1, s);
   if (e != cudaSuccess) return e;

@@ -69,6 +69,25 @@ def test_state_write_of_the_scans_own_state_is_the_scan(cuda_ok):
     assert torch.equal(y2, y) and torch.equal(h2, h)
 
 
+@pytest.mark.parametrize("t", [0, 37, 149])
+def test_state_write_with_h_last_aliasing_h0_or_the_state(cuda_ok, t):
+    # h_last may be h0's buffer (the ABI allows it) or the written state's:
+    # the write then runs the tokens after t as a launch of its own, after
+    # the parts that read h0 and the written state; the results equal the
+    # call with separate buffers, bit for bit
+    d = _dev(I.m1_inputs(3, 150, 96, 16, io="bf16", seed=20 + t, h0=True))
+    ops = _ops()
+    state = torch.randn(3, 96, 16, device="cuda", generator=torch.Generator("cuda").manual_seed(t))
+    y, h, _ = ops.ssm_scan_fwd_write(*_args(d), **_kw(d), t=t, state=state)
+    h0 = d["h0"].clone()
+    y1, h1, _ = ops.ssm_scan_fwd_write(*_args(d), **dict(_kw(d), h0=h0), t=t, state=state,
+                                       h_last=h0)
+    assert torch.equal(y1, y) and torch.equal(h1, h) and torch.equal(h0, h)
+    st = state.clone()
+    y2, h2, _ = ops.ssm_scan_fwd_write(*_args(d), **_kw(d), t=t, state=st, h_last=st)
+    assert torch.equal(y2, y) and torch.equal(h2, h) and torch.equal(st, h)
+
+
 def test_state_write_per_token_kernel_with_states(cuda_ok):
     # with per-token states the per-token kernel carries the write; its
     # states at t are the written state and later ones continue from it
