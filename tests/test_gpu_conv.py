@@ -41,6 +41,19 @@ def test_conv_shapes(cuda_ok, L, io):
 
 
 @pytest.mark.parametrize("W", [1, 2, 3, 4])
+@pytest.mark.parametrize("C", [64, 36])
+def test_conv_bf16_vector_widths(cuda_ok, W, C):
+    # bf16 rows of whole 16-byte vectors take eight channels a thread (64),
+    # rows of 8-byte vectors four (36), for every kernel width; runs cross
+    # the fitted run length (300 tokens)
+    d = I.conv_inputs(2, 300, C, W, io="bf16", seed=7 * W + C, state=True)
+    (u, st), (ur, sr) = _run(d, True, True, True), _ref(d, True, True, True)
+    assert_close_normwise(u, torch.tensor(ur), REL[torch.bfloat16], "u")
+    if W > 1:
+        assert torch.equal(st.double(), torch.tensor(sr))
+
+
+@pytest.mark.parametrize("W", [1, 2, 3, 4])
 @pytest.mark.parametrize("silu,with_bias,with_state", [(True, True, True), (False, False, False),
                                                        (True, False, True), (False, True, False)])
 def test_conv_widths_and_options(cuda_ok, W, silu, with_bias, with_state):

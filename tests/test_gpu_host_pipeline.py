@@ -83,6 +83,18 @@ def test_host_groups_and_generic_kernel(cuda_ok, b, L, C, N, G):
     assert torch.equal(y, yd) and torch.equal(h, hd)
 
 
+def test_host_h_last_into_h0(cuda_ok):
+    # h_last may be h0's (host) buffer: every chunk's h0 rows are uploaded
+    # before its h_last rows come back
+    d = I.m1_inputs(5, 120, 64, 16, io="bf16", seed=31)
+    h0 = torch.randn(5, 64, 16, generator=torch.Generator().manual_seed(31))
+    _, h_ref, _ = _call(d, h0, pinned=True)
+    t = {k: (v.pin_memory() if v is not None else None) for k, v in dict(d, h0=h0.clone()).items()}
+    y, h, _ = _ops().ssm_scan_fwd(t["x"], t["dt"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"],
+                                  dt_bias=t["dt_bias"], h0=t["h0"], h_last=t["h0"])
+    assert torch.equal(h, h_ref) and torch.equal(t["h0"], h_ref)
+
+
 def test_host_empty_sequence_passes_the_state(cuda_ok):
     d = I.m1_inputs(3, 0, 64, 16, io="bf16", seed=9)
     h0 = torch.randn(3, 64, 16)
